@@ -1,0 +1,33 @@
+"""Mutation check of the pins: each copy of the oracle with one planted
+mistake (dropped term, wrong sign, transposed operand, swapped clip bounds,
+greedy instead of random pivots) must fail at least one pin.  The mistakes
+are planted in the oracle's C source at compile time, on the CPU."""
+import os
+
+import pytest
+
+import oracle
+from tests import oracle_pins
+
+MUTANTS = {
+    1: "drops the subtraction of earlier factor columns",
+    2: "adds instead of subtracts in the residual-diagonal update",
+    3: "transposes the factor in the back substitution",
+    4: "swaps the clip bounds",
+    5: "takes the largest residual instead of a random pivot",
+}
+
+
+@pytest.mark.parametrize("k", sorted(MUTANTS), ids=lambda k: f"mutant{k}")
+def test_pins_catch_planted_mistake(tmp_path, k):
+    path = oracle.build(out_path=os.path.join(tmp_path, f"liboracle_m{k}.so"), mutant=k)
+    bad = oracle.Oracle(path)
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        if pin is oracle_pins.pin_philox_matches_library:
+            continue  # slow and unrelated to the planted mistakes
+        try:
+            pin(bad)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught mutant {k} ({MUTANTS[k]})"
