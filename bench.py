@@ -1,0 +1,363 @@
+#!/usr/bin/env python
+"""Benchmark of the WildCat forward (select -> weights -> attend) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, same metric
+
+One step = one wildcat_forward call over the whole workload (all instances)
+with inputs resident in device memory.  Each step is bracketed by its own
+CUDA events on the launching stream; a 256 MiB device write flushes the L2
+cache between steps, outside the events.  With N > 1 (torchrun, one rank per
+GPU) every rank runs its own copy of the workload (weak scaling; instances
+are independent, so there is no collective on the data path) and the
+reported time is the maximum over ranks.
+
+Printed (rank 0): one JSON line with the metric, the device-timed value,
+an end-to-end value through wildcat_forward_host (pinned host buffers,
+copies inside the timed region), a per-stage breakdown, the roofline of the
+dominant kernel (the RPCholesky select), sampled SM clocks, and the oracle
+timed on the host cores as a CPU baseline.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "WildCat fwd calls/s & effective m*n attention entries/s on 1 B200; % roofline"
+LAUNCHES_PER_FORWARD = 9  # select 1 + weights 5 + attend 3
+FLUSH_BYTES = 256 << 20
+EPS = 1e-6
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["wildcat", "reference"], default="wildcat")
+    p.add_argument("--workload", default="c1_vit56")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    return p.parse_args()
+
+
+def workload_config(w, extra=None):
+    cfg = {"workload": f"{w.name}: BH={w.BH} (B={w.B}, H={w.H}), n={w.n}, m={w.m}, d={w.d}, "
+                       f"r={w.r}, {w.dtype} inputs, {w.dist} keys",
+           "BH": w.BH, "n": w.n, "m": w.m, "d": w.d, "r": w.r, "input_dtype": w.dtype,
+           "beta": w.beta, "distribution": w.dist}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def select_bytes(w, ranks):
+    """Algorithmic bytes of one RPCholesky select launch: per step i the key
+    pass (n d b_K), the factor prefix read (4 n i), the new column write (4 n)
+    and the residual read + write (8 n)."""
+    bk = 2 if w.dtype == "bf16" else 4
+    total = 0
+    for rr in ranks:
+        rr = int(rr)
+        total += rr * w.n * (w.d * bk + 12) + 2 * w.n * rr * (rr - 1)
+    return total
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("select.cu", "common.cuh", "philox.cuh"):
+        with open(os.path.join(ROOT, "nystr_coreset_approximate_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per select launch from a committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"rpc_select_{workload_name}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_tr or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_tr.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region (sm clock, reasons)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[4:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for _, _, r in rows for k in range(4) if r[k + 1] == "Active"})
+        return {"sm_mhz": statistics.median(s for s, _, _ in rows),
+                "sm_max_mhz": max(m for _, m, _ in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def cpu_baseline(w, ex, seconds):
+    """The fp64 oracle, as it stands, on the host cores over the whole workload."""
+    import oracle
+
+    orc = oracle.get()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": reps / el, "unit": "calls/s", "cores": orc.num_threads(), "kind": "oracle",
+            "sample": f"{reps} full wildcat_forward calls of the whole workload "
+                      f"({w.BH} instances) in {el:.1f} s, fp64, OpenMP over instances"}
+
+
+def run_reference(args):
+    """Reference arm: the fp64 CPU oracle on the same workload and metric."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    import workloads
+
+    w = workloads.CONFIGS[args.workload]
+    _, ex = workloads.make(w)
+    orc = oracle.get()
+    for _ in range(args.warmup):
+        orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = args.steps / total
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "calls/s",
+           "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": workload_config(w, {"l2": "n/a (host)"}),
+           "entries_per_s": value * w.BH * w.m * w.n,
+           "cpu_baseline": {"value": value, "unit": "calls/s", "cores": orc.num_threads(),
+                            "kind": "oracle",
+                            "sample": f"the whole workload per step ({w.BH} instances), fp64"},
+           "e2e": {"value": value, "unit": "calls/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import nystr_coreset_approximate_b200 as wc
+    import workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    w0 = workloads.CONFIGS[args.workload]
+    w = w0.scaled(seed=w0.seed + 1000 * rank)  # each rank its own batch of instances
+    dev, ex = workloads.make(w)
+    Q, K, V = (dev[k].cuda() for k in ("Q", "K", "V"))
+    plan = wc.ForwardPlan(w.BH, w.m, w.n, w.d, w.r, w.dtype)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- warm-up ----
+    for _ in range(max(args.warmup, 3)):
+        plan.run(Q, K, V, w.beta, w.pivot_seed, EPS)
+    torch.cuda.synchronize()
+    ranks = plan.rank.cpu().tolist()
+
+    # ---- timed forward: K steps, own events per step, L2 flushed in between ----
+    clocks = ClockSampler(local)
+    clocks.start()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    for k in range(args.steps):
+        flush.zero_()
+        starts[k].record()
+        plan.run(Q, K, V, w.beta, w.pivot_seed, EPS)
+        ends[k].record()
+    barrier()
+    clk = clocks.stop()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
+    total_ms = float(total_ms.item())
+
+    # ---- per-stage breakdown through the staged C-ABI calls (same kernels) ----
+    stage_ms = {"select": [], "weights": [], "attend": []}
+    for k in range(args.steps + 2):
+        flush.zero_()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record()
+        S, F, rk, K_S = wc.select(K, w.beta, w.r, w.pivot_seed, EPS)
+        ev[1].record()
+        V_S, wv, vmin, vmax = wc.weights(F, S, rk, V)
+        ev[2].record()
+        wc.attend(Q, K_S, rk, w.beta, V_S, wv, vmin, vmax)
+        ev[3].record()
+        torch.cuda.synchronize()
+        if k >= 2:
+            stage_ms["select"].append(ev[0].elapsed_time(ev[1]))
+            stage_ms["weights"].append(ev[1].elapsed_time(ev[2]))
+            stage_ms["attend"].append(ev[2].elapsed_time(ev[3]))
+    del S, F, rk, K_S, V_S, wv, vmin, vmax
+    sel_ms = statistics.mean(stage_ms["select"])
+
+    # ---- end to end through wildcat_forward_host (host buffers) ----
+    e2e = None
+    if not args.no_e2e:
+        hp = wc.HostForwardPlan(w.BH, w.m, w.n, w.d, w.r, w.dtype)
+        pinned = {k: v.pin_memory() for k, v in dev.items()}
+        O_host = torch.empty((w.BH, w.m, w.d), dtype=torch.float32).pin_memory()
+        S_host = torch.empty((w.BH, w.r), dtype=torch.int32).pin_memory()
+        r_host = torch.empty((w.BH,), dtype=torch.int32).pin_memory()
+        for _ in range(2):
+            hp.run(pinned["Q"], pinned["K"], pinned["V"], O_host, w.beta, w.pivot_seed, EPS,
+                   S_host, r_host)
+        barrier()
+        e_ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            hp.run(pinned["Q"], pinned["K"], pinned["V"], O_host, w.beta, w.pivot_seed, EPS,
+                   S_host, r_host)
+            b.record()
+            b.synchronize()
+            e_ms.append(a.elapsed_time(b))
+        e_tot = torch.tensor([sum(e_ms)], dtype=torch.float64, device="cuda")
+        if world > 1:
+            dist.all_reduce(e_tot, op=dist.ReduceOp.MAX)
+        eb = 2 if w.dtype == "bf16" else 4
+        e2e = {"value": world * args.steps / (float(e_tot.item()) / 1e3), "unit": "calls/s",
+               "h2d_bytes_per_step": eb * w.BH * (w.m + 2 * w.n) * w.d,
+               "d2h_bytes_per_step": 4 * w.BH * w.m * w.d + 4 * w.BH * w.r + 4 * w.BH,
+               "api": "wildcat_forward_host (pinned host buffers)"}
+        del hp
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(w, ex, args.cpu_seconds)
+
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    value = world * args.steps / (total_ms / 1e3)
+    peak, peak_kind = read_peaks()
+    nbytes = select_bytes(w, ranks)
+    achieved = nbytes / (sel_ms / 1e3) / 1e9
+    traffic = recorded_traffic(w0.name)
+    out = {
+        "metric": METRIC, "value": value, "unit": "calls/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": workload_config(w0, {"l2": "flushed between steps (256 MiB device write)",
+                                       "parallelism": f"instances per rank x {world} ranks"}),
+        "entries_per_s": value * w.BH * w.m * w.n,
+        "stages_ms": {k: statistics.mean(v) for k, v in stage_ms.items()},
+        "roofline": {"kernel": "rpc_select_kernel", "bound": "hbm", "achieved": achieved,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": f"{peak_kind} hbm_gbs", "traffic": traffic,
+                     "algorithmic_bytes_per_launch": nbytes, "launch_ms": sel_ms},
+        "gpu_launches": LAUNCHES_PER_FORWARD * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "effective_rank_mean": sum(ranks) / len(ranks),
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,215 @@
+/*
+ * wildcat.h -- C ABI of the B200 (sm_100a) WildCat hot path.
+ *
+ * WildCat approximates softmax attention O = D^-1 A V, A = exp(beta Q K^T),
+ * by attending over a weighted coreset of the keys ("WildCat: Near-Linear
+ * Attention in Theory and Practice", Schroeder & Mackey, Sec. 2):
+ *
+ *   select   randomly pivoted Cholesky (RPCholesky) on the key kernel
+ *            h(K,K) = exp(beta K K^T) picks r pivot keys S and builds the
+ *            partial Cholesky factor F (Sec. 2, "randomly pivoted Cholesky";
+ *            Alg. 1 RPNys)
+ *   weights  Nystrom weights W = h(K_S,K_S)^+ h(K_S,K) applied to (V, 1_n):
+ *            V_S = W V and w = W 1_n, formed as F_S^-T (F^T (V, 1_n))
+ *            (Sec. 2 plug-in estimator; Alg. 2 CompressKV)
+ *   attend   O_hat = diag(U w)^-1 U V_S, U = exp(beta Q K_S^T), each entry
+ *            clipped to the value range [v_min j, v_max j] of V
+ *            (Sec. 2, value-range clip; Alg. 3 WtdAttn)
+ *   forward  the three stages back to back (Alg. 4, the WildCat module)
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - An "instance" is one (batch, head) pair; BH instances are independent
+ *    and are stored one after another (instance b = batch * H + head).
+ *  - All tensors are dense, row-major and contiguous.  Q is [BH, m, d];
+ *    K and V are [BH, n, d]; their dtype is WILDCAT_F32 or WILDCAT_BF16.
+ *    Every other tensor has a fixed type given below.
+ *  - The factor F is float32 [BH, r, n]: F[b, i, l] is entry l of factor
+ *    column i, so each column is contiguous over the n keys.
+ *  - Unless a name ends in _host, every pointer is a DEVICE pointer owned by
+ *    the caller.  The library keeps no pointer after a call returns, and no
+ *    call allocates device memory: scratch space is the caller's
+ *    `workspace` (size from the matching *_workspace_size query, 256-byte
+ *    aligned).
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *    enqueued asynchronously; a call returns once its kernels are launched.
+ *  - Argument checks happen on the host before anything is launched and
+ *    return WILDCAT_ERR_INVALID_ARG / WILDCAT_ERR_UNSUPPORTED with no work
+ *    enqueued.  A failed launch returns WILDCAT_ERR_CUDA.  In every error
+ *    case wildcat_last_error() (per thread) describes the failure.
+ *  - Supported head dims: d in {32, 64, 128}.  Device pointers to Q, K, V,
+ *    K_S must be 16-byte aligned.
+ *  - An instance whose pivots run out before r (total residual mass zero,
+ *    or a pivot residual g_s <= eps, the truncation that stands in for the
+ *    pseudo-inverse) has effective rank r' < r.  That is not an error: the
+ *    rank is reported, S holds -1 past r', and F, K_S, V_S and w hold zeros
+ *    there.
+ *  - Pivot draws: uniform u_i of step i for instance b is Philox4x32-10
+ *    (Salmon et al., SC'11) with key (seed_lo, seed_hi) and counter
+ *    (i, b, 0, 0); u = (x + 1) * 2^-53 where x is the top 53 bits of the
+ *    64-bit word (x1:x0).  The pivot is the first key whose cumulative
+ *    residual diagonal reaches u * T, T the total residual mass.
+ */
+#ifndef WILDCAT_H_
+#define WILDCAT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WILDCAT_OK = 0,
+    WILDCAT_ERR_INVALID_ARG = 1, /* null pointer, bad size, misalignment */
+    WILDCAT_ERR_UNSUPPORTED = 2, /* valid but not implemented (head dim, size limit) */
+    WILDCAT_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+    WILDCAT_ERR_WORKSPACE = 4    /* workspace too small or misaligned */
+} wildcat_status;
+
+typedef enum { WILDCAT_F32 = 0, WILDCAT_BF16 = 1 } wildcat_dtype;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int wildcat_version(void);
+
+/* Message for the last failed call on this thread ("" if none). */
+const char* wildcat_last_error(void);
+
+/* Static name of a status code. */
+const char* wildcat_status_string(int status);
+
+/*
+ * wildcat_select -- RPCholesky coreset selection (Sec. 2, randomly pivoted
+ * Cholesky; Alg. 1 RPNys).  For every instance, r sequential steps: draw the
+ * pivot s from the residual diagonal, form the factor column
+ * F[:, i] = g / sqrt(g_s), g = h(K, k_s) - F[:, :i] F[s, :i]^T, and update the
+ * residual diagonal d <- max(d - F[:, i]^2, 0), d_s = 0.  The kernel is
+ * evaluated as exp(beta (<x, y> - M_K)), M_K = max_l |k_l|^2, a constant
+ * factor that leaves pivots and weights unchanged.
+ *
+ *   K      [BH, n, d] keys, dtype `dtype`
+ *   beta   kernel inverse temperature (> 0, finite)
+ *   r      coreset size, 1 <= r <= n
+ *   seed   64-bit Philox key of the pivot draws
+ *   eps    truncation threshold (relative to max_l h(k_l, k_l)), >= 0
+ *   S      out [BH, r] int32 pivot indices in draw order, -1 past the rank
+ *   F      out [BH, r, n] float32 factor
+ *   rank   out [BH] int32 effective rank r'
+ *   K_S    out [BH, r, d] gathered pivot keys (dtype `dtype`), or NULL
+ */
+wildcat_status wildcat_select(const void* K, int dtype, int64_t BH, int64_t n, int d, float beta,
+                              int r, uint64_t seed, float eps, int32_t* S, float* F,
+                              int32_t* rank, void* K_S, void* stream);
+
+/*
+ * wildcat_select_fixed -- the same factorisation with the pivots given
+ * (test entry point: lets the device path run on the oracle's pivots).
+ * S_fixed [BH, r] int32; a negative or out-of-range entry ends that
+ * instance's factorisation (rank = its position).  S (out, may be NULL)
+ * receives the pivots actually used.  Other arguments as wildcat_select.
+ */
+wildcat_status wildcat_select_fixed(const void* K, int dtype, int64_t BH, int64_t n, int d,
+                                    float beta, int r, float eps, const int32_t* S_fixed,
+                                    int32_t* S, float* F, int32_t* rank, void* K_S, void* stream);
+
+/*
+ * wildcat_weights -- Nystrom weights applied to (V, 1_n) (Sec. 2 plug-in
+ * estimator: W multiplies (V, 1_n) before the queries; Alg. 2 CompressKV).
+ * Y = F^T (V, 1_n) is reduced over the n keys, then F_S^T X = Y is solved by
+ * back substitution with F_S[a, j] = F[b, j, S[a]] (lower triangular in
+ * pivot order; entries above the diagonal are ignored).
+ *
+ *   F, S, rank   from wildcat_select
+ *   V            [BH, n, d] values, dtype `dtype`
+ *   V_S          out [BH, r, d] float32, rows of W V (zero past the rank)
+ *   w            out [BH, r] float32, W 1_n (zero past the rank)
+ *   vmin, vmax   out [BH, d] float32 column-wise range of V
+ *   workspace    >= wildcat_weights_workspace_size(BH, n, d, r) bytes
+ */
+size_t wildcat_weights_workspace_size(int64_t BH, int64_t n, int d, int r);
+wildcat_status wildcat_weights(const float* F, const int32_t* S, const int32_t* rank,
+                               const void* V, int dtype, int64_t BH, int64_t n, int d, int r,
+                               float* V_S, float* w, float* vmin, float* vmax, void* workspace,
+                               size_t ws_bytes, void* stream);
+
+/*
+ * wildcat_attend -- weighted-coreset attention (Alg. 3 WtdAttn):
+ *   u_il = exp(beta <q_i, k_S_l> - beta M_Q),  M_Q = max_i |q_i| * max_l |k_S_l|
+ *   O_hat_ij = fminf(fmaxf(sum_l u_il V_S[l, j] / sum_l u_il w_l, vmin_j), vmax_j)
+ * The shift M_Q (one per instance) keeps every u_il <= 1 and cancels in the
+ * ratio.  A normaliser that is zero or negative (Nystrom weights have mixed
+ * signs) is not special-cased: the ratio is clipped as is, and a NaN ratio
+ * (0/0) becomes vmin_j.
+ *
+ *   Q      [BH, m, d] queries, dtype `dtype`
+ *   K_S    [BH, r, d] pivot keys, dtype `dtype`
+ *   rank   [BH] int32 effective ranks (only the first rank[b] rows are used)
+ *   V_S, w, vmin, vmax   from wildcat_weights
+ *   O      out [BH, m, d] float32
+ *   workspace >= wildcat_attend_workspace_size(BH, m, d, r) bytes
+ */
+size_t wildcat_attend_workspace_size(int64_t BH, int64_t m, int d, int r);
+wildcat_status wildcat_attend(const void* Q, const void* K_S, int dtype, int64_t BH, int64_t m,
+                              int d, int r, const int32_t* rank, float beta, const float* V_S,
+                              const float* w, const float* vmin, const float* vmax, float* O,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * wildcat_forward -- the whole module (Alg. 4): select -> weights -> attend,
+ * all on `stream`, with every intermediate in `workspace`.
+ *
+ *   Q [BH, m, d], K and V [BH, n, d] (dtype `dtype`); O out [BH, m, d] float32
+ *   S_out [BH, r] int32 and rank_out [BH] int32: optional copies (or NULL)
+ *   workspace >= wildcat_forward_workspace_size(BH, m, n, d, r, dtype) bytes
+ */
+size_t wildcat_forward_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int dtype);
+wildcat_status wildcat_forward(const void* Q, const void* K, const void* V, int dtype, int64_t BH,
+                               int64_t m, int64_t n, int d, float beta, int r, uint64_t seed,
+                               float eps, float* O, int32_t* S_out, int32_t* rank_out,
+                               void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * wildcat_forward_host -- wildcat_forward on HOST buffers: copies Q, K, V
+ * from host memory into the device workspace, runs the forward, copies O
+ * (and optionally S, rank) back, and waits for the stream.  Host buffers
+ * should be page-locked for full copy bandwidth.
+ *
+ *   Q_host, K_host, V_host   host input arrays (layouts as wildcat_forward)
+ *   O_host                   host output [BH, m, d] float32
+ *   S_host, rank_host        optional host outputs (or NULL)
+ *   workspace >= wildcat_forward_host_workspace_size(...) bytes (device)
+ */
+size_t wildcat_forward_host_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r,
+                                           int dtype);
+wildcat_status wildcat_forward_host(const void* Q_host, const void* K_host, const void* V_host,
+                                    int dtype, int64_t BH, int64_t m, int64_t n, int d,
+                                    float beta, int r, uint64_t seed, float eps, float* O_host,
+                                    int32_t* S_host, int32_t* rank_host, void* workspace,
+                                    size_t ws_bytes, void* stream);
+
+/*
+ * wildcat_pivot_uniforms -- the pivot uniforms the select kernels draw
+ * (test entry point): u[b, i] for b < BH, i < steps, as float64, written to
+ * the device array u [BH, steps].
+ */
+wildcat_status wildcat_pivot_uniforms(uint64_t seed, int64_t BH, int steps, double* u,
+                                      void* stream);
+
+/*
+ * wildcat_set_select_cluster -- tuning knob for wildcat_select*: number of
+ * CTAs (a thread-block cluster, 1..16, power of two) that share one
+ * instance.  0 restores the automatic choice.  Process-wide; not thread-safe
+ * against concurrent select calls.  Returns WILDCAT_ERR_INVALID_ARG for
+ * other values.
+ */
+wildcat_status wildcat_set_select_cluster(int ctas_per_instance);
+
+/* The cluster size the last select launch on this thread used (0 if none). */
+int wildcat_last_select_cluster(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WILDCAT_H_ */

@@ -1,0 +1,304 @@
+// api.cu -- extern "C" entry points of libwildcat (declared in include/wildcat.h).
+//
+// Host-side argument checks, workspace carving and stage sequencing.  No
+// arithmetic of the method happens here; every stage runs in the kernels of
+// select.cu, weights.cu and attend.cu.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/wildcat.h"
+#include "internal.h"
+
+using wildcat::Carve;
+using wildcat::Status;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+wildcat_status record(const Status& s) {
+    if (s.code == 0) {
+        g_err[0] = '\0';
+        return WILDCAT_OK;
+    }
+    if (s.code == WILDCAT_ERR_CUDA)
+        snprintf(g_err, sizeof(g_err), "%s: %s", s.what, cudaGetErrorString(s.cuda_err));
+    else
+        snprintf(g_err, sizeof(g_err), "%s", s.what);
+    return (wildcat_status)s.code;
+}
+
+wildcat_status bad(int code, const char* fmt, const char* what) {
+    snprintf(g_err, sizeof(g_err), fmt, what);
+    return (wildcat_status)code;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t elem_bytes(int dtype) { return dtype == WILDCAT_BF16 ? 2 : 4; }
+
+wildcat_status check_common(int dtype, int64_t BH, int64_t n, int d, int r, const char* who) {
+    if (dtype != WILDCAT_F32 && dtype != WILDCAT_BF16) return bad(1, "%s: dtype must be WILDCAT_F32 or WILDCAT_BF16", who);
+    if (BH < 0) return bad(1, "%s: BH must be >= 0", who);
+    if (n < 1) return bad(1, "%s: n must be >= 1", who);
+    if (r < 1 || (int64_t)r > n) return bad(1, "%s: r must satisfy 1 <= r <= n", who);
+    if (d != 32 && d != 64 && d != 128) return bad(2, "%s: head dim must be 32, 64 or 128", who);
+    if (r > 8192) return bad(2, "%s: r above 8192 is not supported", who);
+    const double cells = (double)BH * (double)n * (double)(d > r ? d : r);
+    if (cells > 4.0e18) return bad(1, "%s: tensor sizes overflow 64-bit offsets", who);
+    if (BH > 65535) return bad(2, "%s: BH above 65535 is not supported", who);
+    return WILDCAT_OK;
+}
+
+wildcat_status check_scalars(float beta, float eps, const char* who) {
+    if (!std::isfinite(beta) || !(beta > 0.f)) return bad(1, "%s: beta must be finite and > 0", who);
+    if (!std::isfinite(eps) || eps < 0.f) return bad(1, "%s: eps must be finite and >= 0", who);
+    return WILDCAT_OK;
+}
+
+wildcat_status select_impl(const void* K, int dtype, int64_t BH, int64_t n, int d, float beta, int r, uint64_t seed,
+                           float eps, const int32_t* S_fixed, int32_t* S, float* F, int32_t* rank, void* K_S,
+                           void* stream, const char* who) {
+    wildcat_status st = check_common(dtype, BH, n, d, r, who);
+    if (st != WILDCAT_OK) return st;
+    if ((st = check_scalars(beta, eps, who)) != WILDCAT_OK) return st;
+    if (BH == 0) return record(Status::ok());
+    if (!K || !F || !rank) return bad(1, "%s: K, F and rank must be non-null", who);
+    if (!S_fixed && !S) return bad(1, "%s: S must be non-null", who);
+    if (!aligned16(K) || !aligned16(F) || (K_S && !aligned16(K_S)))
+        return bad(1, "%s: K, F and K_S must be 16-byte aligned", who);
+    wildcat::SelectRequest q{K, dtype, BH, n, d, beta, r, seed, eps, S_fixed, S, F, rank, K_S};
+    return record(wildcat::launch_select(q, static_cast<cudaStream_t>(stream)));
+}
+
+struct ForwardLayout {
+    float* F;
+    int32_t* S;
+    int32_t* rank;
+    void* K_S;
+    float* V_S;
+    float* w;
+    float* vmin;
+    float* vmax;
+    void* wws;
+    size_t wws_bytes;
+    void* aws;
+    size_t aws_bytes;
+};
+
+ForwardLayout carve_forward(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, int r, int dtype) {
+    ForwardLayout L{};
+    L.F = static_cast<float*>(cv.take(sizeof(float) * BH * (int64_t)r * n));
+    L.S = static_cast<int32_t*>(cv.take(sizeof(int32_t) * BH * r));
+    L.rank = static_cast<int32_t*>(cv.take(sizeof(int32_t) * BH));
+    L.K_S = cv.take(elem_bytes(dtype) * BH * (int64_t)r * d);
+    L.V_S = static_cast<float*>(cv.take(sizeof(float) * BH * (int64_t)r * d));
+    L.w = static_cast<float*>(cv.take(sizeof(float) * BH * r));
+    L.vmin = static_cast<float*>(cv.take(sizeof(float) * BH * d));
+    L.vmax = static_cast<float*>(cv.take(sizeof(float) * BH * d));
+    L.wws_bytes = wildcat::weights_workspace_bytes(BH, n, d, r);
+    L.wws = cv.take(L.wws_bytes);
+    L.aws_bytes = wildcat::attend_workspace_bytes(BH, m, d, r);
+    L.aws = cv.take(L.aws_bytes);
+    return L;
+}
+
+wildcat_status forward_impl(const void* Q, const void* K, const void* V, int dtype, int64_t BH, int64_t m, int64_t n,
+                            int d, float beta, int r, uint64_t seed, float eps, float* O, int32_t* S_out,
+                            int32_t* rank_out, const ForwardLayout& L, cudaStream_t st) {
+    Status s;
+    wildcat::SelectRequest sq{K, dtype, BH, n, d, beta, r, seed, eps, nullptr, L.S, L.F, L.rank, L.K_S};
+    if ((s = wildcat::launch_select(sq, st)).code) return record(s);
+    wildcat::WeightsRequest wq{L.F, L.S, L.rank, V, dtype, BH, n, d, r, L.V_S, L.w, L.vmin, L.vmax, L.wws,
+                               L.wws_bytes};
+    if ((s = wildcat::launch_weights(wq, st)).code) return record(s);
+    if (m > 0) {
+        wildcat::AttendRequest aq{Q,   L.K_S,  dtype, BH, m, d, r, L.rank, beta, L.V_S, L.w,
+                                  L.vmin, L.vmax, O,   L.aws, L.aws_bytes};
+        if ((s = wildcat::launch_attend(aq, st)).code) return record(s);
+    }
+    cudaError_t e;
+    if (S_out && (e = cudaMemcpyAsync(S_out, L.S, sizeof(int32_t) * BH * r, cudaMemcpyDeviceToDevice, st)))
+        return record(Status::cuda(e, "forward: copy S"));
+    if (rank_out && (e = cudaMemcpyAsync(rank_out, L.rank, sizeof(int32_t) * BH, cudaMemcpyDeviceToDevice, st)))
+        return record(Status::cuda(e, "forward: copy rank"));
+    return record(Status::ok());
+}
+
+}  // namespace
+
+extern "C" {
+
+int wildcat_version(void) { return 100; }
+
+const char* wildcat_last_error(void) { return g_err; }
+
+const char* wildcat_status_string(int status) {
+    switch (status) {
+        case WILDCAT_OK: return "WILDCAT_OK";
+        case WILDCAT_ERR_INVALID_ARG: return "WILDCAT_ERR_INVALID_ARG";
+        case WILDCAT_ERR_UNSUPPORTED: return "WILDCAT_ERR_UNSUPPORTED";
+        case WILDCAT_ERR_CUDA: return "WILDCAT_ERR_CUDA";
+        case WILDCAT_ERR_WORKSPACE: return "WILDCAT_ERR_WORKSPACE";
+    }
+    return "WILDCAT_UNKNOWN_STATUS";
+}
+
+wildcat_status wildcat_select(const void* K, int dtype, int64_t BH, int64_t n, int d, float beta, int r, uint64_t seed,
+                              float eps, int32_t* S, float* F, int32_t* rank, void* K_S, void* stream) {
+    return select_impl(K, dtype, BH, n, d, beta, r, seed, eps, nullptr, S, F, rank, K_S, stream, "wildcat_select");
+}
+
+wildcat_status wildcat_select_fixed(const void* K, int dtype, int64_t BH, int64_t n, int d, float beta, int r,
+                                    float eps, const int32_t* S_fixed, int32_t* S, float* F, int32_t* rank,
+                                    void* K_S, void* stream) {
+    if (!S_fixed && BH > 0) return bad(1, "%s: S_fixed must be non-null", "wildcat_select_fixed");
+    return select_impl(K, dtype, BH, n, d, beta, r, 0, eps, S_fixed, S, F, rank, K_S, stream,
+                       "wildcat_select_fixed");
+}
+
+size_t wildcat_weights_workspace_size(int64_t BH, int64_t n, int d, int r) {
+    if (BH < 0 || n < 1 || r < 1 || d < 1) return 0;
+    return wildcat::weights_workspace_bytes(BH, n, d, r);
+}
+
+wildcat_status wildcat_weights(const float* F, const int32_t* S, const int32_t* rank, const void* V, int dtype,
+                               int64_t BH, int64_t n, int d, int r, float* V_S, float* w, float* vmin, float* vmax,
+                               void* workspace, size_t ws_bytes, void* stream) {
+    const char* who = "wildcat_weights";
+    wildcat_status st = check_common(dtype, BH, n, d, r, who);
+    if (st != WILDCAT_OK) return st;
+    if (BH == 0) return record(Status::ok());
+    if (!F || !S || !rank || !V || !V_S || !w || !vmin || !vmax || !workspace)
+        return bad(1, "%s: null pointer argument", who);
+    if (!aligned16(V) || !aligned16(F)) return bad(1, "%s: F and V must be 16-byte aligned", who);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
+    if (ws_bytes < wildcat::weights_workspace_bytes(BH, n, d, r)) return bad(4, "%s: workspace too small", who);
+    wildcat::WeightsRequest q{F, S, rank, V, dtype, BH, n, d, r, V_S, w, vmin, vmax, workspace, ws_bytes};
+    return record(wildcat::launch_weights(q, static_cast<cudaStream_t>(stream)));
+}
+
+size_t wildcat_attend_workspace_size(int64_t BH, int64_t m, int d, int r) {
+    if (BH < 0 || m < 0) return 0;
+    return wildcat::attend_workspace_bytes(BH, m, d, r);
+}
+
+wildcat_status wildcat_attend(const void* Q, const void* K_S, int dtype, int64_t BH, int64_t m, int d, int r,
+                              const int32_t* rank, float beta, const float* V_S, const float* w, const float* vmin,
+                              const float* vmax, float* O, void* workspace, size_t ws_bytes, void* stream) {
+    const char* who = "wildcat_attend";
+    wildcat_status st = check_common(dtype, BH, r, d, r, who);
+    if (st != WILDCAT_OK) return st;
+    if ((st = check_scalars(beta, 0.f, who)) != WILDCAT_OK) return st;
+    if (m < 0) return bad(1, "%s: m must be >= 0", who);
+    if (BH == 0 || m == 0) return record(Status::ok());
+    if (!Q || !K_S || !rank || !V_S || !w || !vmin || !vmax || !O || !workspace)
+        return bad(1, "%s: null pointer argument", who);
+    if (!aligned16(Q) || !aligned16(K_S)) return bad(1, "%s: Q and K_S must be 16-byte aligned", who);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
+    if (ws_bytes < wildcat::attend_workspace_bytes(BH, m, d, r)) return bad(4, "%s: workspace too small", who);
+    wildcat::AttendRequest q{Q, K_S, dtype, BH, m, d, r, rank, beta, V_S, w, vmin, vmax, O, workspace, ws_bytes};
+    return record(wildcat::launch_attend(q, static_cast<cudaStream_t>(stream)));
+}
+
+size_t wildcat_forward_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int dtype) {
+    if (BH < 0 || m < 0 || n < 1 || r < 1 || d < 1) return 0;
+    Carve cv(nullptr, 0);
+    carve_forward(cv, BH, m, n, d, r, dtype);
+    return cv.used + 256;
+}
+
+wildcat_status wildcat_forward(const void* Q, const void* K, const void* V, int dtype, int64_t BH, int64_t m,
+                               int64_t n, int d, float beta, int r, uint64_t seed, float eps, float* O,
+                               int32_t* S_out, int32_t* rank_out, void* workspace, size_t ws_bytes, void* stream) {
+    const char* who = "wildcat_forward";
+    wildcat_status st = check_common(dtype, BH, n, d, r, who);
+    if (st != WILDCAT_OK) return st;
+    if ((st = check_scalars(beta, eps, who)) != WILDCAT_OK) return st;
+    if (m < 0) return bad(1, "%s: m must be >= 0", who);
+    if (BH == 0) return record(Status::ok());
+    if (!K || !V || !workspace || (m > 0 && (!Q || !O))) return bad(1, "%s: null pointer argument", who);
+    if (!aligned16(K) || !aligned16(V) || (Q && !aligned16(Q)))
+        return bad(1, "%s: Q, K and V must be 16-byte aligned", who);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
+    Carve cv(workspace, ws_bytes);
+    const ForwardLayout L = carve_forward(cv, BH, m, n, d, r, dtype);
+    if (!cv.fits()) return bad(4, "%s: workspace too small", who);
+    return forward_impl(Q, K, V, dtype, BH, m, n, d, beta, r, seed, eps, O, S_out, rank_out, L,
+                        static_cast<cudaStream_t>(stream));
+}
+
+size_t wildcat_forward_host_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int dtype) {
+    if (BH < 0 || m < 0 || n < 1 || r < 1 || d < 1) return 0;
+    Carve cv(nullptr, 0);
+    cv.take(elem_bytes(dtype) * BH * m * d);
+    cv.take(elem_bytes(dtype) * BH * n * d);
+    cv.take(elem_bytes(dtype) * BH * n * d);
+    cv.take(sizeof(float) * BH * m * d);
+    cv.take(sizeof(int32_t) * BH * r);
+    cv.take(sizeof(int32_t) * BH);
+    carve_forward(cv, BH, m, n, d, r, dtype);
+    return cv.used + 256;
+}
+
+wildcat_status wildcat_forward_host(const void* Q_host, const void* K_host, const void* V_host, int dtype, int64_t BH,
+                                    int64_t m, int64_t n, int d, float beta, int r, uint64_t seed, float eps,
+                                    float* O_host, int32_t* S_host, int32_t* rank_host, void* workspace,
+                                    size_t ws_bytes, void* stream) {
+    const char* who = "wildcat_forward_host";
+    wildcat_status st = check_common(dtype, BH, n, d, r, who);
+    if (st != WILDCAT_OK) return st;
+    if ((st = check_scalars(beta, eps, who)) != WILDCAT_OK) return st;
+    if (m < 0) return bad(1, "%s: m must be >= 0", who);
+    if (BH == 0) return record(Status::ok());
+    if (!K_host || !V_host || !workspace || (m > 0 && (!Q_host || !O_host)))
+        return bad(1, "%s: null pointer argument", who);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t eb = elem_bytes(dtype);
+    Carve cv(workspace, ws_bytes);
+    void* Qd = cv.take(eb * BH * m * d);
+    void* Kd = cv.take(eb * BH * n * d);
+    void* Vd = cv.take(eb * BH * n * d);
+    float* Od = static_cast<float*>(cv.take(sizeof(float) * BH * m * d));
+    int32_t* Sd = static_cast<int32_t*>(cv.take(sizeof(int32_t) * BH * r));
+    int32_t* Rd = static_cast<int32_t*>(cv.take(sizeof(int32_t) * BH));
+    const ForwardLayout L = carve_forward(cv, BH, m, n, d, r, dtype);
+    if (!cv.fits()) return bad(4, "%s: workspace too small", who);
+    cudaError_t e;
+    if (m > 0 && (e = cudaMemcpyAsync(Qd, Q_host, eb * BH * m * d, cudaMemcpyHostToDevice, s)))
+        return record(Status::cuda(e, "forward_host: copy Q"));
+    if ((e = cudaMemcpyAsync(Kd, K_host, eb * BH * n * d, cudaMemcpyHostToDevice, s)))
+        return record(Status::cuda(e, "forward_host: copy K"));
+    if ((e = cudaMemcpyAsync(Vd, V_host, eb * BH * n * d, cudaMemcpyHostToDevice, s)))
+        return record(Status::cuda(e, "forward_host: copy V"));
+    st = forward_impl(m > 0 ? Qd : nullptr, Kd, Vd, dtype, BH, m, n, d, beta, r, seed, eps, m > 0 ? Od : nullptr, Sd,
+                      Rd, L, s);
+    if (st != WILDCAT_OK) return st;
+    if (m > 0 && (e = cudaMemcpyAsync(O_host, Od, sizeof(float) * BH * m * d, cudaMemcpyDeviceToHost, s)))
+        return record(Status::cuda(e, "forward_host: copy O"));
+    if (S_host && (e = cudaMemcpyAsync(S_host, Sd, sizeof(int32_t) * BH * r, cudaMemcpyDeviceToHost, s)))
+        return record(Status::cuda(e, "forward_host: copy S"));
+    if (rank_host && (e = cudaMemcpyAsync(rank_host, Rd, sizeof(int32_t) * BH, cudaMemcpyDeviceToHost, s)))
+        return record(Status::cuda(e, "forward_host: copy rank"));
+    if ((e = cudaStreamSynchronize(s))) return record(Status::cuda(e, "forward_host: stream sync"));
+    return record(Status::ok());
+}
+
+wildcat_status wildcat_pivot_uniforms(uint64_t seed, int64_t BH, int steps, double* u, void* stream) {
+    if (BH < 0 || steps < 0) return bad(1, "%s: BH and steps must be >= 0", "wildcat_pivot_uniforms");
+    if (BH * (int64_t)steps > 0 && !u) return bad(1, "%s: u must be non-null", "wildcat_pivot_uniforms");
+    return record(wildcat::launch_pivot_uniforms(seed, BH, steps, u, static_cast<cudaStream_t>(stream)));
+}
+
+wildcat_status wildcat_set_select_cluster(int ctas_per_instance) {
+    const int G = ctas_per_instance;
+    if (G != 0 && G != 1 && G != 2 && G != 4 && G != 8 && G != 16)
+        return bad(1, "%s: cluster size must be 0 (auto) or a power of two <= 16", "wildcat_set_select_cluster");
+    wildcat::select_cluster_override(G);
+    return record(Status::ok());
+}
+
+int wildcat_last_select_cluster(void) { return wildcat::last_select_cluster(); }
+
+}  // extern "C"

@@ -1,0 +1,213 @@
+// attend.cu -- weighted-coreset attention on sm_100a.
+//
+// "WildCat: Near-Linear Attention in Theory and Practice", Sec. 2 plug-in
+// estimator and Alg. 3 WtdAttn: with U = exp(beta Q K_S^T),
+//     O_hat = diag(U w)^-1 U V_S,  each entry clipped to [v_min j, v_max j].
+// A single shift M_Q = max_i |q_i| * max_l |k_S_l| per instance keeps every
+// exponent <= 0 and cancels in the ratio.
+//
+// Kernels:
+//   qnorm_partial / shift_finalize   M_Q per instance
+//   attend_kernel                    per tile of queries: P = exp(beta Q K_S^T
+//                                    - beta M_Q) chunk by chunk, N += P V_S,
+//                                    D += P w, then O = clip(N / D)
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace wildcat {
+
+namespace {
+
+constexpr int kNormThreads = 256;
+
+template <typename E, int D>
+__global__ void __launch_bounds__(kNormThreads) qnorm_partial(const typename E::T* Q, int64_t m,
+                                                              int64_t rows_per_split, float* part) {
+    // part [BH, nsplit]: max |q_i| over a slice of the queries (one warp per row)
+    const int64_t b = blockIdx.y;
+    const int split = blockIdx.x, nsplit = gridDim.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t i0 = split * rows_per_split, i1 = std::min<int64_t>(m, i0 + rows_per_split);
+    float best = 0.f;
+    for (int64_t i = i0 + warp; i < i1; i += kNormThreads / 32) {
+        const typename E::T* q = Q + (b * m + i) * D;
+        float s = 0.f;
+        for (int c = lane; c < D; c += 32) {
+            const float v = E::to_float(q[c]);
+            s = fmaf(v, v, s);
+        }
+        s = warp_sum(s);
+        best = fmaxf(best, sqrtf(s));
+    }
+    __shared__ float wb[kNormThreads / 32];
+    if (lane == 0) wb[warp] = best;
+    __syncthreads();
+    if (warp == 0) {
+        float v = lane < kNormThreads / 32 ? wb[lane] : 0.f;
+        v = warp_max(v);
+        if (lane == 0) part[b * nsplit + split] = v;
+    }
+}
+
+template <typename E, int D>
+__global__ void shift_finalize(const float* part, int nsplit, const typename E::T* K_S, const int32_t* rank, int r,
+                               float* MQ) {
+    const int64_t b = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int rr = rank[b];
+    float kb = 0.f;
+    for (int l = warp; l < rr; l += nw) {
+        const typename E::T* k = K_S + (b * r + l) * D;
+        float s = 0.f;
+        for (int c = lane; c < D; c += 32) {
+            const float v = E::to_float(k[c]);
+            s = fmaf(v, v, s);
+        }
+        kb = fmaxf(kb, sqrtf(warp_sum(s)));
+    }
+    float qb = 0.f;
+    for (int s = lane; s < nsplit; s += 32) qb = fmaxf(qb, part[b * nsplit + s]);
+    qb = warp_max(qb);
+    __shared__ float wk[32];
+    if (lane == 0) wk[warp] = kb;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float k = 0.f;
+        for (int w = 0; w < nw; ++w) k = fmaxf(k, wk[w]);
+        MQ[b] = qb * k;
+    }
+}
+
+constexpr int kAttThreads = 256;
+constexpr int kAttTM = 64;  // queries per CTA
+constexpr int kAttRC = 32;  // coreset rows per chunk
+
+template <int D>
+struct AttSmem {
+    static constexpr int QS = D + 1;  // padded row stride (bank-conflict free)
+    static constexpr size_t q = 0;
+    static constexpr size_t k = q + sizeof(float) * kAttTM * QS;
+    static constexpr size_t v = k + sizeof(float) * kAttRC * D;
+    static constexpr size_t wv = v + sizeof(float) * kAttRC * D;
+    static constexpr size_t p = wv + sizeof(float) * kAttRC;
+    static constexpr size_t total = p + sizeof(float) * kAttTM * (kAttRC + 1);
+};
+
+template <typename E, int D>
+__global__ void __launch_bounds__(kAttThreads) attend_kernel(const typename E::T* Q, const typename E::T* K_S,
+                                                             int64_t m, int r, const int32_t* rank, float beta,
+                                                             const float* V_S, const float* w, const float* vmin,
+                                                             const float* vmax, const float* MQ, float* O) {
+    using L = AttSmem<D>;
+    extern __shared__ __align__(16) unsigned char sm[];
+    float* Qs = reinterpret_cast<float*>(sm + L::q);
+    float* Ks = reinterpret_cast<float*>(sm + L::k);
+    float* Vs = reinterpret_cast<float*>(sm + L::v);
+    float* ws = reinterpret_cast<float*>(sm + L::wv);
+    float* P = reinterpret_cast<float*>(sm + L::p);
+
+    const int64_t b = blockIdx.y;
+    const int64_t i0 = (int64_t)blockIdx.x * kAttTM;
+    const int tid = threadIdx.x;
+    const int rr = rank[b];
+    const float shift = beta * MQ[b];
+
+    for (int e = tid; e < kAttTM * D; e += kAttThreads) {
+        const int ii = e / D, c = e % D;
+        const int64_t i = i0 + ii;
+        Qs[ii * L::QS + c] = i < m ? E::to_float(Q[(b * m + i) * D + c]) : 0.f;
+    }
+    constexpr int CPT = D / 4;  // output columns per thread
+    const int oi = tid / 4, oc = tid % 4;
+    float acc[CPT];
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) acc[k] = 0.f;
+    float den = 0.f;
+
+    for (int l0 = 0; l0 < rr; l0 += kAttRC) {
+        __syncthreads();  // previous chunk fully consumed (and Q tile loaded)
+        for (int e = tid; e < kAttRC * D; e += kAttThreads) {
+            const int ll = e / D, c = e % D;
+            const int l = l0 + ll;
+            const bool ok = l < rr;
+            Ks[ll * D + c] = ok ? E::to_float(K_S[(b * r + l) * D + c]) : 0.f;
+            Vs[ll * D + c] = ok ? V_S[(b * r + l) * (int64_t)D + c] : 0.f;
+        }
+        for (int ll = tid; ll < kAttRC; ll += kAttThreads) ws[ll] = (l0 + ll < rr) ? w[b * r + l0 + ll] : 0.f;
+        __syncthreads();
+        // P[i][l] = exp(beta <q_i, k_l> - beta M_Q), zero past the rank
+        for (int e = tid; e < kAttTM * kAttRC; e += kAttThreads) {
+            const int ii = e % kAttTM, ll = e / kAttTM;
+            float s = 0.f;
+#pragma unroll 8
+            for (int c = 0; c < D; ++c) s = fmaf(Qs[ii * L::QS + c], Ks[ll * D + c], s);
+            P[ii * (kAttRC + 1) + ll] = (l0 + ll < rr) ? expf(beta * s - shift) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int ll = 0; ll < kAttRC; ++ll) {
+            const float p = P[oi * (kAttRC + 1) + ll];
+#pragma unroll
+            for (int k = 0; k < CPT; ++k) acc[k] = fmaf(p, Vs[ll * D + oc + 4 * k], acc[k]);
+            den = fmaf(p, ws[ll], den);
+        }
+    }
+    const int64_t i = i0 + oi;
+    if (i < m) {
+        float* o = O + (b * m + i) * D;
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) {
+            const int c = oc + 4 * k;
+            o[c] = fminf(fmaxf(acc[k] / den, vmin[b * D + c]), vmax[b * D + c]);
+        }
+    }
+}
+
+template <typename E, int D>
+Status run_attend(const AttendRequest& q, cudaStream_t st) {
+    using T = typename E::T;
+    const int nsplit = (int)std::max<int64_t>(1, std::min<int64_t>(64, ceil_div(q.m, 1024)));
+    const int64_t rows_per_split = ceil_div(q.m, nsplit);
+    Carve cv(q.ws, q.ws_bytes);
+    float* part = static_cast<float*>(cv.take(sizeof(float) * q.BH * nsplit));
+    float* MQ = static_cast<float*>(cv.take(sizeof(float) * q.BH));
+    if (!cv.fits()) return Status::fail(4, "attend: workspace too small");
+    const T* Q = static_cast<const T*>(q.Q);
+    const T* KS = static_cast<const T*>(q.K_S);
+    qnorm_partial<E, D><<<dim3(nsplit, (unsigned)q.BH), kNormThreads, 0, st>>>(Q, q.m, rows_per_split, part);
+    shift_finalize<E, D><<<(unsigned)q.BH, 256, 0, st>>>(part, nsplit, KS, q.rank, q.r, MQ);
+    const size_t smem = AttSmem<D>::total;
+    cudaError_t e = cudaFuncSetAttribute(attend_kernel<E, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return Status::cuda(e, "attend: smem attribute");
+    attend_kernel<E, D><<<dim3((unsigned)ceil_div(q.m, kAttTM), (unsigned)q.BH), kAttThreads, smem, st>>>(
+        Q, KS, q.m, q.r, q.rank, q.beta, q.V_S, q.w, q.vmin, q.vmax, MQ, q.O);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return Status::cuda(e, "attend launch");
+    return Status::ok();
+}
+
+}  // namespace
+
+size_t attend_workspace_bytes(int64_t BH, int64_t m, int d, int r) {
+    (void)d;
+    (void)r;
+    const int nsplit = (int)std::max<int64_t>(1, std::min<int64_t>(64, ceil_div(m, 1024)));
+    Carve cv(nullptr, 0);
+    cv.take(sizeof(float) * BH * nsplit);
+    cv.take(sizeof(float) * BH);
+    return cv.used + 256;
+}
+
+Status launch_attend(const AttendRequest& q, cudaStream_t st) {
+    const bool bf = q.dtype == 1;
+    switch (q.d) {
+        case 32: return bf ? run_attend<BF16, 32>(q, st) : run_attend<F32, 32>(q, st);
+        case 64: return bf ? run_attend<BF16, 64>(q, st) : run_attend<F32, 64>(q, st);
+        case 128: return bf ? run_attend<BF16, 128>(q, st) : run_attend<F32, 128>(q, st);
+    }
+    return Status::fail(2, "attend: unsupported head dim");
+}
+
+}  // namespace wildcat

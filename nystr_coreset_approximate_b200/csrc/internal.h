@@ -1,0 +1,93 @@
+// internal.h -- host-side interfaces between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace wildcat {
+
+// Result of a host-side launcher: code follows wildcat_status.
+struct Status {
+    int code;
+    const char* what;      // static text
+    cudaError_t cuda_err;  // for code 3
+    static Status ok() { return {0, "", cudaSuccess}; }
+    static Status fail(int c, const char* w) { return {c, w, cudaSuccess}; }
+    static Status cuda(cudaError_t e, const char* w) { return {3, w, e}; }
+};
+
+struct SelectRequest {
+    const void* K;
+    int dtype;  // 0 f32, 1 bf16
+    int64_t BH, n;
+    int d;
+    float beta;
+    int r;
+    uint64_t seed;
+    float eps;
+    const int32_t* S_fixed;
+    int32_t* S;
+    float* F;
+    int32_t* rank;
+    void* K_S;
+};
+
+Status launch_select(const SelectRequest& q, cudaStream_t stream);
+Status launch_pivot_uniforms(uint64_t seed, int64_t BH, int steps, double* u, cudaStream_t stream);
+int select_cluster_override(int G);  // G < 0: query only
+int last_select_cluster();
+
+// ---- weights: Y = F^T (V, 1), then F_S^T X = Y ----
+struct WeightsRequest {
+    const float* F;
+    const int32_t* S;
+    const int32_t* rank;
+    const void* V;
+    int dtype;
+    int64_t BH, n;
+    int d, r;
+    float* V_S;
+    float* w;
+    float* vmin;
+    float* vmax;
+    void* ws;
+    size_t ws_bytes;
+};
+size_t weights_workspace_bytes(int64_t BH, int64_t n, int d, int r);
+Status launch_weights(const WeightsRequest& q, cudaStream_t stream);
+
+// ---- attend ----
+struct AttendRequest {
+    const void* Q;
+    const void* K_S;
+    int dtype;
+    int64_t BH, m;
+    int d, r;
+    const int32_t* rank;
+    float beta;
+    const float* V_S;
+    const float* w;
+    const float* vmin;
+    const float* vmax;
+    float* O;
+    void* ws;
+    size_t ws_bytes;
+};
+size_t attend_workspace_bytes(int64_t BH, int64_t m, int d, int r);
+Status launch_attend(const AttendRequest& q, cudaStream_t stream);
+
+// 256-byte aligned bump allocator over a caller-provided workspace.
+struct Carve {
+    char* base;
+    size_t cap, used;
+    explicit Carve(void* p, size_t c) : base(static_cast<char*>(p)), cap(c), used(0) {}
+    void* take(size_t bytes) {
+        const size_t at = (used + 255) & ~size_t(255);
+        used = at + bytes;
+        return base ? base + at : nullptr;
+    }
+    bool fits() const { return used <= cap; }
+};
+
+}  // namespace wildcat

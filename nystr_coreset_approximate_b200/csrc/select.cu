@@ -1,0 +1,603 @@
+// select.cu -- RPCholesky coreset selection on sm_100a.
+//
+// "WildCat: Near-Linear Attention in Theory and Practice", Sec. 2
+// (randomly pivoted Cholesky; Alg. 1 RPNys).  For each instance, r
+// sequential steps:
+//   draw s with probability proportional to the residual diagonal d,
+//   g = h(K, k_s) - F[:, :i] F[s, :i]^T,   h(x, y) = exp(beta (<x,y> - M_K)),
+//   F[:, i] = g / sqrt(g_s),   d <- max(d - F[:, i]^2, 0),   d_s = 0,
+// stopping early when the total mass or the pivot residual g_s vanishes.
+//
+// Mapping: one thread-block cluster of G CTAs per instance.  CTA c owns the
+// key rows [c R, c R + R).  It keeps the residual diagonal of its rows in
+// shared memory (double-buffered across steps) together with fp64 chunk sums
+// of it; the pivot search reads the other CTAs' chunk sums and the chosen
+// chunk through distributed shared memory, so the cluster needs one
+// hardware cluster barrier per step.  Every CTA runs the search on the same
+// data with the same arithmetic, so all CTAs agree on s without a second
+// barrier.  The column pass streams the CTA's slice of F[:, :i] (float4,
+// L2-only loads: the slice is touched once per step) and of K, spread over
+// JG thread groups that split the factor columns and the head dimension.
+#include <cooperative_groups.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+#include "philox.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace wildcat {
+
+namespace {
+
+constexpr int kSelectThreads = 512;
+constexpr int kMaxPL = 16;  // R <= 16384 rows per CTA -> at most 16 values per lane
+
+struct SelectArgs {
+    const void* K;
+    int64_t BH, n;
+    float beta;
+    int r;
+    uint64_t seed;
+    float eps;
+    const int32_t* S_fixed;  // nullptr: draw pivots
+    int32_t* S;              // may be nullptr in fixed mode
+    float* F;
+    int32_t* rank;
+    void* K_S;  // may be nullptr
+    int G;      // CTAs per instance (cluster size)
+    int R;      // rows per CTA, multiple of 4
+    int JG;     // thread groups splitting factor columns / head dim
+    int PL;     // residual values per lane in one search chunk (multiple of 4)
+};
+
+struct SmemLayout {
+    size_t ctot, csum, dbuf, ks, fs, red, misc, total;
+    __host__ __device__ SmemLayout(int R, int r, int D, int JG, int NT, int VEC) {
+        size_t o = 0;
+        ctot = o;  o += 2 * sizeof(double);
+        csum = o;  o += 2 * 32 * sizeof(double);
+        dbuf = o;  o += 2 * (size_t)R * sizeof(float);
+        ks = o;    o += (size_t)D * sizeof(float);
+        fs = o;    o += (size_t)round_up(r, 4) * sizeof(float);
+        o = round_up(o, 16);
+        red = o;   o += (size_t)(JG > 1 ? JG - 1 : 0) * (NT / JG) * 2 * VEC * sizeof(float);
+        misc = o;  o += 16 * sizeof(float);
+        total = round_up(o, 16);
+    }
+};
+
+// Inclusive fp64 warp scan (Hillis-Steele); identical on every CTA.
+__device__ __forceinline__ double warp_scan_incl(double v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    return v;
+}
+
+// Sum of one search chunk (PL values per lane, lane-sequential then scan).
+__device__ __forceinline__ double chunk_total(const float* chunk, int PL, int lane) {
+    double s = 0.0;
+    for (int k = 0; k < PL; ++k) s += (double)chunk[lane * PL + k];
+    return __shfl_sync(0xffffffffu, warp_scan_incl(s, lane), 31);
+}
+
+template <typename E, int D, int VEC>
+__global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const SelectArgs a) {
+    // Launched with a cluster dimension of a.G (one cluster per instance).
+    using T = typename E::T;
+    constexpr int NT = kSelectThreads;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int crank = (int)cluster.block_rank();
+    const int64_t b = blockIdx.x / a.G;
+    if (b >= a.BH) return;  // whole clusters only: G divides gridDim.x
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int R = a.R, r = a.r, JG = a.JG, TPG = NT / JG;
+    const int64_t n = a.n;
+    const int64_t row0 = (int64_t)crank * R;
+    const int64_t row_end = (row0 + R < n) ? row0 + R : n;
+    const int nrows = row_end > row0 ? (int)(row_end - row0) : 0;
+    const int CH = 32 * a.PL;
+    const int nch = (int)ceil_div(R, CH);
+    const int Rpad = nch * CH;  // residual buffers cover whole search chunks
+
+    extern __shared__ __align__(16) unsigned char smem[];
+    const SmemLayout L(Rpad, r, D, JG, NT, VEC);
+    double* ctot = reinterpret_cast<double*>(smem + L.ctot);
+    double* csum = reinterpret_cast<double*>(smem + L.csum);
+    float* dbuf = reinterpret_cast<float*>(smem + L.dbuf);
+    float* ks = reinterpret_cast<float*>(smem + L.ks);
+    float* fs = reinterpret_cast<float*>(smem + L.fs);
+    float* red = reinterpret_cast<float*>(smem + L.red);
+    float* misc = reinterpret_cast<float*>(smem + L.misc);
+    int* imisc = reinterpret_cast<int*>(misc);
+    // misc[0] local max |k|^2, misc[1] M_K, misc[2] g_s, imisc[3] s, imisc[4] stop
+
+    const T* Kb = reinterpret_cast<const T*>(a.K) + b * n * D;
+    float* Fb = a.F + b * (int64_t)r * n;
+
+    // ---------------- prologue: M_K and the initial residual diagonal ----------------
+    float lmax = -INFINITY;
+    for (int row = tid; row < Rpad; row += NT) {
+        float sq = 0.f;
+        if (row < nrows) {
+            const T* kr = Kb + (row0 + row) * D;
+#pragma unroll
+            for (int c = 0; c < D; c += 8) {
+                float v[8];
+                load8(kr + c, v);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) sq = fmaf(v[k], v[k], sq);
+            }
+            lmax = fmaxf(lmax, sq);
+        }
+        dbuf[row] = sq;  // temporarily |k|^2
+    }
+    lmax = warp_max(lmax);
+    __shared__ float wmax[NT / 32];
+    if (lane == 0) wmax[warp] = lmax;
+    __syncthreads();
+    if (warp == 0) {
+        float v = lane < NT / 32 ? wmax[lane] : -INFINITY;
+        v = warp_max(v);
+        if (lane == 0) misc[0] = v;
+    }
+    cluster.sync();
+    if (warp == 0) {
+        float v = -INFINITY;
+        if (lane < a.G) v = *cluster.map_shared_rank(&misc[0], lane);
+        v = warp_max(v);
+        if (lane == 0) misc[1] = v;
+    }
+    __syncthreads();
+    const float MK = misc[1];
+    const float beta = a.beta;
+    for (int row = tid; row < Rpad; row += NT)
+        dbuf[row] = row < nrows ? expf(beta * (dbuf[row] - MK)) : 0.f;
+    __syncthreads();
+    for (int k = warp; k < nch; k += NT / 32) {
+        const double t = chunk_total(dbuf + (size_t)k * CH, a.PL, lane);
+        if (lane == 0) csum[k] = t;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        double v = lane < nch ? csum[lane] : 0.0;
+        double tot = 0.0;
+        for (int k = 0; k < nch; ++k) tot += __shfl_sync(0xffffffffu, v, k);
+        if (lane == 0) ctot[0] = tot;
+    }
+    cluster.sync();
+
+    // ---------------- r sequential steps ----------------
+    int i = 0;
+    for (; i < r; ++i) {
+        const int cur = i & 1, nxt = cur ^ 1;
+        float* dcur = dbuf + (size_t)cur * Rpad;
+        float* dnxt = dbuf + (size_t)nxt * Rpad;
+
+        // -- pivot search (warp 0 of every CTA, identical arithmetic) --
+        if (warp == 0) {
+            int s = -1;
+            if (a.S_fixed) {
+                const int sf = a.S_fixed[b * r + i];
+                s = (sf >= 0 && (int64_t)sf < n) ? sf : -1;
+            } else {
+                const double tc = lane < a.G ? *cluster.map_shared_rank(&ctot[cur], lane) : 0.0;
+                double T = 0.0;
+                for (int c = 0; c < a.G; ++c) T += __shfl_sync(0xffffffffu, tc, c);
+                if (T > 0.0) {
+                    const double t = pivot_uniform(a.seed, (uint32_t)i, (uint32_t)b) * T;
+                    // owner CTA: first whose cumulative total reaches t
+                    double cum = 0.0;
+                    int owner = -1, lastpos = -1;
+                    for (int c = 0; c < a.G; ++c) {
+                        const double v = __shfl_sync(0xffffffffu, tc, c);
+                        if (v > 0.0) lastpos = c;
+                        if (owner < 0) {
+                            if (cum + v >= t) owner = c;
+                            else cum += v;
+                        }
+                    }
+                    if (owner < 0) {  // rounding pushed t past the total
+                        owner = lastpos;
+                        cum = 0.0;
+                        for (int c = 0; c < owner; ++c) cum += __shfl_sync(0xffffffffu, tc, c);
+                    }
+                    // chunk inside the owner
+                    const double* rcs = cluster.map_shared_rank(csum + cur * 32, owner);
+                    const double cv = lane < nch ? rcs[lane] : 0.0;
+                    int chunk = -1, lastc = -1;
+                    double cum2 = cum;
+                    for (int k = 0; k < nch; ++k) {
+                        const double v = __shfl_sync(0xffffffffu, cv, k);
+                        if (v > 0.0) lastc = k;
+                        if (chunk < 0) {
+                            if (cum2 + v >= t) chunk = k;
+                            else cum2 += v;
+                        }
+                    }
+                    if (chunk < 0) {
+                        chunk = lastc;
+                        cum2 = cum;
+                        for (int k = 0; k < chunk; ++k) cum2 += __shfl_sync(0xffffffffu, cv, k);
+                    }
+                    // row inside the chunk
+                    const float* rd =
+                        cluster.map_shared_rank(dbuf + (size_t)cur * Rpad, owner) + (size_t)chunk * CH;
+                    float vals[kMaxPL];
+#pragma unroll
+                    for (int k = 0; k < kMaxPL; ++k) vals[k] = k < a.PL ? rd[lane * a.PL + k] : 0.f;
+                    double part = 0.0;
+#pragma unroll
+                    for (int k = 0; k < kMaxPL; ++k)
+                        if (k < a.PL) part += (double)vals[k];
+                    const double incl = warp_scan_incl(part, lane);
+                    double c = cum2 + (incl - part);
+                    int hit = -1, lastnz = -1;
+#pragma unroll
+                    for (int k = 0; k < kMaxPL; ++k) {
+                        if (k >= a.PL) break;
+                        const float v = vals[k];
+                        if (v > 0.f) lastnz = k;
+                        c += (double)v;
+                        if (hit < 0 && v > 0.f && c >= t) hit = k;
+                    }
+                    const unsigned hm = __ballot_sync(0xffffffffu, hit >= 0);
+                    int local;
+                    if (hm) {
+                        const int src = __ffs(hm) - 1;
+                        local = src * a.PL + __shfl_sync(0xffffffffu, hit, src);
+                    } else {
+                        const unsigned nm = __ballot_sync(0xffffffffu, lastnz >= 0);
+                        const int src = 31 - __clz(nm);
+                        local = src * a.PL + __shfl_sync(0xffffffffu, lastnz, src);
+                    }
+                    s = (int)((int64_t)owner * R + (int64_t)chunk * CH + local);
+                }
+            }
+            if (lane == 0) {
+                imisc[3] = s;
+                imisc[4] = (s < 0);
+            }
+        }
+        __syncthreads();
+        if (imisc[4]) break;
+        const int s = imisc[3];
+
+        // -- pivot key and the pivot's row of the factor --
+        const T* kp = Kb + (int64_t)s * D;
+        for (int c = tid; c < D; c += NT) ks[c] = E::to_float(kp[c]);
+        for (int j = tid; j < i; j += NT) fs[j] = ld_cg1(Fb + (int64_t)j * n + s);
+        __syncthreads();
+        // -- pivot residual g_s, the same on every CTA --
+        if (warp == 0) {
+            float dot = 0.f, acc = 0.f;
+            for (int c = lane; c < D; c += 32) dot = fmaf(ks[c], ks[c], dot);
+            for (int j = lane; j < i; j += 32) acc = fmaf(fs[j], fs[j], acc);
+            dot = warp_sum(dot);
+            acc = warp_sum(acc);
+            if (lane == 0) {
+                const float gs = expf(beta * (dot - MK)) - acc;
+                misc[2] = gs;
+                imisc[4] = !(gs > a.eps);  // max_l h(k_l, k_l) is exp(0) = 1
+            }
+        }
+        __syncthreads();
+        if (imisc[4]) break;
+        const float gs = misc[2];
+        const float piv = sqrtf(gs);
+        if (crank == 0) {
+            if (tid == 0 && a.S) a.S[b * r + i] = s;
+            if (a.K_S) {
+                T* dst = reinterpret_cast<T*>(a.K_S) + (b * r + i) * D;
+                for (int c = tid; c < D; c += NT) dst[c] = kp[c];
+            }
+        }
+
+        // -- column pass over the CTA's rows --
+        const int g = tid / TPG, tt = tid % TPG;
+        const int jl = (i + JG - 1) / JG, j0 = min(i, g * jl), j1 = min(i, j0 + jl);
+        constexpr int DC = D;  // head-dim split must keep 8-element loads whole
+        const int dl = DC / JG, c0 = g * dl, c1 = c0 + dl;
+        for (int base = 0; base < nrows; base += TPG * VEC) {
+            const int row = base + tt * VEC;
+            const bool valid = row < nrows;
+            float acc[VEC], dp[VEC];
+#pragma unroll
+            for (int k = 0; k < VEC; ++k) acc[k] = dp[k] = 0.f;
+            if (valid) {
+                const float* fcol = Fb + row0 + row;
+                int j = j0;
+                if constexpr (VEC == 4) {
+                    for (; j + 4 <= j1; j += 4) {
+                        float4 v[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) v[u] = ld_cg4(fcol + (int64_t)(j + u) * n);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const float f = fs[j + u];
+                            acc[0] = fmaf(v[u].x, f, acc[0]);
+                            acc[1] = fmaf(v[u].y, f, acc[1]);
+                            acc[2] = fmaf(v[u].z, f, acc[2]);
+                            acc[3] = fmaf(v[u].w, f, acc[3]);
+                        }
+                    }
+                    for (; j < j1; ++j) {
+                        const float4 v = ld_cg4(fcol + (int64_t)j * n);
+                        const float f = fs[j];
+                        acc[0] = fmaf(v.x, f, acc[0]);
+                        acc[1] = fmaf(v.y, f, acc[1]);
+                        acc[2] = fmaf(v.z, f, acc[2]);
+                        acc[3] = fmaf(v.w, f, acc[3]);
+                    }
+                } else {
+                    for (; j < j1; ++j) acc[0] = fmaf(ld_cg1(fcol + (int64_t)j * n), fs[j], acc[0]);
+                }
+#pragma unroll
+                for (int k = 0; k < VEC; ++k) {
+                    const T* kr = Kb + (row0 + row + k) * D;
+                    for (int c = c0; c < c1; c += 8) {
+                        float v[8];
+                        load8(kr + c, v);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) dp[k] = fmaf(v[e], ks[c + e], dp[k]);
+                    }
+                }
+            }
+            if (JG > 1) {
+                if (g > 0) {
+                    float* dst = red + ((size_t)(g - 1) * TPG + tt) * 2 * VEC;
+#pragma unroll
+                    for (int k = 0; k < VEC; ++k) {
+                        dst[k] = acc[k];
+                        dst[VEC + k] = dp[k];
+                    }
+                }
+                __syncthreads();
+                if (g == 0) {
+                    for (int h = 0; h < JG - 1; ++h) {
+                        const float* src = red + ((size_t)h * TPG + tt) * 2 * VEC;
+#pragma unroll
+                        for (int k = 0; k < VEC; ++k) {
+                            acc[k] += src[k];
+                            dp[k] += src[VEC + k];
+                        }
+                    }
+                }
+            }
+            if (g == 0 && valid) {
+                float out[VEC];
+#pragma unroll
+                for (int k = 0; k < VEC; ++k) {
+                    const int64_t l = row0 + row + k;
+                    float gl = expf(beta * (dp[k] - MK)) - acc[k];
+                    if (l == s) gl = gs;
+                    const float f = gl / piv;
+                    out[k] = f;
+                    float dn = fmaxf(dcur[row + k] - f * f, 0.f);
+                    if (l == s) dn = 0.f;
+                    dnxt[row + k] = dn;
+                }
+                float* dstF = Fb + (int64_t)i * n + row0 + row;
+                if constexpr (VEC == 4) {
+                    *reinterpret_cast<float4*>(dstF) = make_float4(out[0], out[1], out[2], out[3]);
+                } else {
+                    dstF[0] = out[0];
+                }
+            }
+            if (JG > 1) __syncthreads();
+        }
+        // rows of the slice past n keep zero mass
+        for (int row = nrows + tid; row < Rpad; row += NT) dnxt[row] = 0.f;
+        __syncthreads();
+        // -- chunk sums of the new residual diagonal --
+        for (int k = warp; k < nch; k += NT / 32) {
+            const double t = chunk_total(dnxt + (size_t)k * CH, a.PL, lane);
+            if (lane == 0) csum[nxt * 32 + k] = t;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            const double v = lane < nch ? csum[nxt * 32 + lane] : 0.0;
+            double tot = 0.0;
+            for (int k = 0; k < nch; ++k) tot += __shfl_sync(0xffffffffu, v, k);
+            if (lane == 0) ctot[nxt] = tot;
+        }
+        cluster.sync();
+    }
+
+    // ---------------- effective rank, padding past it ----------------
+    const int rr = i;
+    for (int j = rr; j < r; ++j) {
+        float* dst = Fb + (int64_t)j * n + row0;
+        for (int row = tid; row < nrows; row += NT) dst[row] = 0.f;
+    }
+    if (crank == 0) {
+        if (tid == 0) a.rank[b] = rr;
+        for (int j = rr + tid; j < r; j += NT)
+            if (a.S) a.S[b * r + j] = -1;
+        if (a.K_S) {
+            T* dst = reinterpret_cast<T*>(a.K_S) + b * r * D;
+            for (int64_t e = (int64_t)rr * D + tid; e < (int64_t)r * D; e += NT) dst[e] = T(0.f);
+        }
+    }
+    // keep this CTA's shared memory alive until every peer is done reading it
+    cluster.sync();
+}
+
+__global__ void pivot_uniform_kernel(uint64_t seed, int64_t BH, int steps, double* u) {
+    const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (t >= BH * steps) return;
+    const int64_t b = t / steps;
+    const int i = (int)(t % steps);
+    u[t] = pivot_uniform(seed, (uint32_t)i, (uint32_t)b);
+}
+
+template <typename E, int D, int VEC>
+cudaError_t launch_select_t(const SelectArgs& a, size_t smem, cudaStream_t stream) {
+    auto kern = rpc_select_kernel<E, D, VEC>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (a.G > 8) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.BH * a.G));
+    cfg.blockDim = dim3(kSelectThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = a.G;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+template <typename E, int D, int VEC>
+int max_clusters_t(int G, size_t smem) {
+    auto kern = rpc_select_kernel<E, D, VEC>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return 0;
+    if (G > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+        return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)G);
+    cfg.blockDim = dim3(kSelectThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = G;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nc = 0;
+    if (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return nc;
+}
+
+template <typename E, int VEC>
+int dispatch_d(int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int G_query, cudaError_t* err) {
+    switch (d) {
+        case 32:
+            if (a) { *err = launch_select_t<E, 32, VEC>(*a, smem, stream); return 0; }
+            return max_clusters_t<E, 32, VEC>(G_query, smem);
+        case 64:
+            if (a) { *err = launch_select_t<E, 64, VEC>(*a, smem, stream); return 0; }
+            return max_clusters_t<E, 64, VEC>(G_query, smem);
+        case 128:
+            if (a) { *err = launch_select_t<E, 128, VEC>(*a, smem, stream); return 0; }
+            return max_clusters_t<E, 128, VEC>(G_query, smem);
+    }
+    if (err) *err = cudaErrorInvalidValue;
+    return 0;
+}
+
+int dispatch(int dtype, int vec, int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int G_query,
+             cudaError_t* err) {
+    if (dtype == 1) {
+        return vec == 4 ? dispatch_d<BF16, 4>(d, a, smem, stream, G_query, err)
+                        : dispatch_d<BF16, 1>(d, a, smem, stream, G_query, err);
+    }
+    return vec == 4 ? dispatch_d<F32, 4>(d, a, smem, stream, G_query, err)
+                    : dispatch_d<F32, 1>(d, a, smem, stream, G_query, err);
+}
+
+int g_cluster_override = 0;
+thread_local int g_last_cluster = 0;
+
+}  // namespace
+
+constexpr int kMaxRowsPerCta = 16384;
+
+int select_cluster_override(int G) {
+    if (G < 0) return g_cluster_override;
+    g_cluster_override = G;
+    return G;
+}
+int last_select_cluster() { return g_last_cluster; }
+
+static void plan(int64_t n, int d, int r, int G, int vec, SelectArgs* a, size_t* smem) {
+    const int R = (int)round_up(ceil_div(n, G), 4);
+    int JG = 1;
+    const int maxJG = min(8, d / 8);
+    while (JG * 2 <= maxJG && (int64_t)(kSelectThreads / (JG * 2)) * vec >= R) JG *= 2;
+    const int PL = (int)std::max<int64_t>(4, round_up(ceil_div(ceil_div(R, 32), 32), 4));
+    const int Rpad = (int)round_up(R, 32 * PL);
+    a->G = G;
+    a->R = R;
+    a->JG = JG;
+    a->PL = PL;
+    *smem = SmemLayout(Rpad, r, d, JG, kSelectThreads, vec).total;
+}
+
+Status launch_select(const SelectRequest& q, cudaStream_t stream) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int vec = (q.n % 4 == 0) ? 4 : 1;
+    SelectArgs a{};
+    a.K = q.K;
+    a.BH = q.BH;
+    a.n = q.n;
+    a.beta = q.beta;
+    a.r = q.r;
+    a.seed = q.seed;
+    a.eps = q.eps;
+    a.S_fixed = q.S_fixed;
+    a.S = q.S;
+    a.F = q.F;
+    a.rank = q.rank;
+    a.K_S = q.K_S;
+
+    int G;
+    if (g_cluster_override > 0) {
+        G = g_cluster_override;
+    } else {
+        G = 1;
+        while (G * 2 <= 16 && (int64_t)(G * 2) * q.BH <= sms && q.n / (G * 2) >= 512) G *= 2;
+    }
+    while (G < 16 && ceil_div(q.n, G) > kMaxRowsPerCta) G *= 2;
+    if (ceil_div(q.n, G) > kMaxRowsPerCta)
+        return Status::fail(2, "select: n / 16 exceeds the per-CTA row limit (16384)");
+    if (g_cluster_override <= 0) {
+        // shrink until the cluster shape is schedulable
+        for (;;) {
+            size_t smem;
+            plan(q.n, q.d, q.r, G, vec, &a, &smem);
+            if (smem > 227 * 1024) return Status::fail(2, "select: shared memory plan exceeds 227 KB");
+            if (dispatch(q.dtype, vec, q.d, nullptr, smem, stream, G, nullptr) > 0 || G == 1) break;
+            G /= 2;
+        }
+    }
+    size_t smem;
+    plan(q.n, q.d, q.r, G, vec, &a, &smem);
+    if (smem > 227 * 1024) return Status::fail(2, "select: shared memory plan exceeds 227 KB");
+    cudaError_t err = cudaSuccess;
+    dispatch(q.dtype, vec, q.d, &a, smem, stream, G, &err);
+    if (err == cudaSuccess) err = cudaGetLastError();
+    if (err != cudaSuccess) return Status::cuda(err, "select launch");
+    g_last_cluster = G;
+    return Status::ok();
+}
+
+Status launch_pivot_uniforms(uint64_t seed, int64_t BH, int steps, double* u, cudaStream_t stream) {
+    const int64_t total = BH * steps;
+    if (total == 0) return Status::ok();
+    pivot_uniform_kernel<<<(unsigned)ceil_div(total, 256), 256, 0, stream>>>(seed, BH, steps, u);
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return Status::cuda(err, "pivot uniforms launch");
+    return Status::ok();
+}
+
+}  // namespace wildcat

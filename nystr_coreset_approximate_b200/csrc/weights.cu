@@ -1,0 +1,256 @@
+// weights.cu -- Nystrom weights applied to (V, 1_n) on sm_100a.
+//
+// "WildCat: Near-Linear Attention in Theory and Practice", Sec. 2: the
+// plug-in estimator multiplies W with (V, 1_n) before the queries touch it;
+// Alg. 2 CompressKV keeps V_S = W V and w = W 1_n.  With the partial
+// Cholesky factor F (n x r') of the key kernel and its pivot block
+// F_S = F[S, :] (lower triangular in pivot order),
+//     W = h(K_S,K_S)^-1 h(K_S,K) = F_S^-T F^T,
+// so (V_S, w) = F_S^-T Y with Y = F^T (V, 1_n).
+//
+// Kernels:
+//   colrange_*   column-wise [v_min, v_max] of V (value-range clip bounds)
+//   fty_kernel   Y partials: F^T (V, 1) over a slice of the keys (split-K)
+//   gather_fs    F_S[a, j] = F[j, S_a] for j <= a (pivot rows of the factor)
+//   trsm_kernel  sums the split-K partials and back-substitutes F_S^T X = Y
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace wildcat {
+
+namespace {
+
+constexpr int kRangeThreads = 256;
+
+template <typename E, int D>
+__global__ void __launch_bounds__(kRangeThreads) colrange_partial(const typename E::T* V, int64_t n,
+                                                                  int64_t rows_per_split, float* part) {
+    // part [BH, nsplit, 2, D]
+    const int64_t b = blockIdx.y;
+    const int split = blockIdx.x, nsplit = gridDim.x;
+    constexpr int RS = kRangeThreads / D;  // row slots
+    const int c = threadIdx.x % D, rs = threadIdx.x / D;
+    const int64_t l0 = split * rows_per_split, l1 = min(n, l0 + rows_per_split);
+    float lo = INFINITY, hi = -INFINITY;
+    const typename E::T* Vb = V + b * n * D;
+    for (int64_t l = l0 + rs; l < l1; l += RS) {
+        const float v = E::to_float(Vb[l * D + c]);
+        lo = fminf(lo, v);
+        hi = fmaxf(hi, v);
+    }
+    __shared__ float slo[kRangeThreads], shi[kRangeThreads];
+    slo[threadIdx.x] = lo;
+    shi[threadIdx.x] = hi;
+    __syncthreads();
+    if (rs == 0) {
+        for (int k = 1; k < RS; ++k) {
+            lo = fminf(lo, slo[k * D + c]);
+            hi = fmaxf(hi, shi[k * D + c]);
+        }
+        float* p = part + ((b * nsplit + split) * 2) * D;
+        p[c] = lo;
+        p[D + c] = hi;
+    }
+}
+
+__global__ void colrange_finalize(const float* part, int nsplit, int D, int64_t BH, float* vmin, float* vmax) {
+    const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (t >= BH * D) return;
+    const int64_t b = t / D;
+    const int c = (int)(t % D);
+    float lo = INFINITY, hi = -INFINITY;
+    for (int s = 0; s < nsplit; ++s) {
+        const float* p = part + ((b * nsplit + s) * 2) * D;
+        lo = fminf(lo, p[c]);
+        hi = fmaxf(hi, p[D + c]);
+    }
+    vmin[t] = lo;
+    vmax[t] = hi;
+}
+
+// ---- Y partials = F^T (V, 1) over one key slice: SIMT fp32 ----
+constexpr int kFtyThreads = 256;
+constexpr int kFtyTJ = 32;  // factor columns per CTA
+constexpr int kFtyNK = 32;  // keys per smem stage
+
+template <typename E, int D>
+__global__ void __launch_bounds__(kFtyThreads) fty_kernel(const float* F, const typename E::T* V, int64_t n,
+                                                          int r, int64_t keys_per_split, float* Ypart,
+                                                          int64_t BH) {
+    // Ypart [nsplit, BH, r, D + 1]
+    const int jt = blockIdx.x, split = blockIdx.y;
+    const int64_t b = blockIdx.z;
+    const int nsplit = gridDim.y;
+    const int j0 = jt * kFtyTJ;
+    const int64_t l0 = split * keys_per_split, l1 = min(n, l0 + keys_per_split);
+    constexpr int TPR = kFtyThreads / kFtyTJ;  // threads per factor column
+    constexpr int CPT = D / TPR;               // value columns per thread
+    const int jj = threadIdx.x / TPR, tx = threadIdx.x % TPR;
+
+    __shared__ float Fs[kFtyTJ][kFtyNK + 1];
+    __shared__ __align__(16) float Vs[kFtyNK][D];
+    float acc[CPT];
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) acc[k] = 0.f;
+    float one = 0.f;
+    const float* Fb = F + b * (int64_t)r * n;
+    const typename E::T* Vb = V + b * n * D;
+    for (int64_t lb = l0; lb < l1; lb += kFtyNK) {
+        for (int e = threadIdx.x; e < kFtyTJ * kFtyNK; e += kFtyThreads) {
+            const int rj = e / kFtyNK, kk = e % kFtyNK;
+            const int64_t l = lb + kk;
+            const int j = j0 + rj;
+            Fs[rj][kk] = (j < r && l < l1) ? __ldcg(Fb + (int64_t)j * n + l) : 0.f;
+        }
+        for (int e = threadIdx.x; e < kFtyNK * D; e += kFtyThreads) {
+            const int kk = e / D, c = e % D;
+            const int64_t l = lb + kk;
+            Vs[kk][c] = l < l1 ? E::to_float(Vb[l * D + c]) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < kFtyNK; ++kk) {
+            const float f = Fs[jj][kk];
+#pragma unroll
+            for (int k = 0; k < CPT; ++k) acc[k] = fmaf(f, Vs[kk][tx + TPR * k], acc[k]);
+            one += f;
+        }
+        __syncthreads();
+    }
+    const int j = j0 + jj;
+    if (j < r) {
+        float* y = Ypart + (((int64_t)split * BH + b) * r + j) * (D + 1);
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) y[tx + TPR * k] = acc[k];
+        if (tx == 0) y[D] = one;
+    }
+}
+
+// F_S[b, a, j] = F[b, j, S[b, a]] for j <= a < rank; zero elsewhere.
+__global__ void gather_fs(const float* F, const int32_t* S, const int32_t* rank, int64_t n, int r, float* FS) {
+    const int64_t b = blockIdx.y;
+    const int a = blockIdx.x;
+    const int rr = rank[b];
+    float* dst = FS + (b * r + a) * (int64_t)r;
+    const int s = a < rr ? S[b * r + a] : -1;
+    for (int j = threadIdx.x; j < r; j += blockDim.x)
+        dst[j] = (s >= 0 && j <= a) ? __ldcg(F + (b * r + j) * n + s) : 0.f;
+}
+
+// Back substitution F_S^T X = Y for one instance and one block of CB right-hand columns.
+constexpr int kTrsmThreads = 256;
+constexpr int kTrsmCB = 16;
+
+__global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* Ypart, int nsplit, const float* FS,
+                                                            const int32_t* rank, int64_t BH, int r, int D,
+                                                            float* V_S, float* w) {
+    extern __shared__ float X[];  // [r][CB]
+    const int64_t b = blockIdx.y;
+    const int cb0 = blockIdx.x * kTrsmCB;
+    const int DP = D + 1;
+    const int rr = rank[b];
+    const int c = threadIdx.x % kTrsmCB, rs = threadIdx.x / kTrsmCB;
+    constexpr int RS = kTrsmThreads / kTrsmCB;
+    const int col = cb0 + c;
+    for (int a = rs; a < r; a += RS) {
+        float y = 0.f;
+        if (a < rr && col < DP)
+            for (int s = 0; s < nsplit; ++s) y += Ypart[(((int64_t)s * BH + b) * r + a) * DP + col];
+        X[a * kTrsmCB + c] = y;
+    }
+    __syncthreads();
+    const float* Lb = FS + b * (int64_t)r * r;
+    for (int ap = rr - 1; ap >= 0; --ap) {
+        const float* Lrow = Lb + (int64_t)ap * r;
+        const float xa = X[ap * kTrsmCB + c] / Lrow[ap];
+        for (int a = rs; a < ap; a += RS) X[a * kTrsmCB + c] = fmaf(-Lrow[a], xa, X[a * kTrsmCB + c]);
+        __syncthreads();
+        if (rs == 0) X[ap * kTrsmCB + c] = xa;
+    }
+    __syncthreads();
+    if (col < DP) {
+        for (int a = rs; a < r; a += RS) {
+            const float v = a < rr ? X[a * kTrsmCB + c] : 0.f;
+            if (col < D)
+                V_S[(b * r + a) * (int64_t)D + col] = v;
+            else
+                w[b * r + a] = v;
+        }
+    }
+}
+
+struct WeightsPlan {
+    int nsplit_range;
+    int64_t rows_per_range;
+    int nsplit_k;
+    int64_t keys_per_split;
+};
+
+WeightsPlan make_plan(int64_t BH, int64_t n, int r) {
+    WeightsPlan p{};
+    p.nsplit_range = (int)std::max<int64_t>(1, std::min<int64_t>(64, ceil_div(296, std::max<int64_t>(1, BH))));
+    p.nsplit_range = (int)std::min<int64_t>(p.nsplit_range, std::max<int64_t>(1, n / 64));
+    p.rows_per_range = ceil_div(n, p.nsplit_range);
+    const int64_t tiles = ceil_div(r, kFtyTJ) * BH;
+    int64_t sk = ceil_div(2 * 148, tiles);
+    sk = std::max<int64_t>(1, std::min<int64_t>(sk, std::max<int64_t>(1, n / 256)));
+    sk = std::min<int64_t>(sk, 64);
+    p.keys_per_split = round_up(ceil_div(n, sk), kFtyNK);
+    p.nsplit_k = (int)ceil_div(n, p.keys_per_split);
+    return p;
+}
+
+template <typename E, int D>
+Status run_weights(const WeightsRequest& q, cudaStream_t st) {
+    const WeightsPlan p = make_plan(q.BH, q.n, q.r);
+    Carve cv(q.ws, q.ws_bytes);
+    float* part = static_cast<float*>(cv.take(sizeof(float) * q.BH * p.nsplit_range * 2 * D));
+    float* Ypart = static_cast<float*>(cv.take(sizeof(float) * p.nsplit_k * q.BH * (int64_t)q.r * (D + 1)));
+    float* FS = static_cast<float*>(cv.take(sizeof(float) * q.BH * (int64_t)q.r * q.r));
+    if (!cv.fits()) return Status::fail(4, "weights: workspace too small");
+    using T = typename E::T;
+    const T* V = static_cast<const T*>(q.V);
+
+    colrange_partial<E, D><<<dim3(p.nsplit_range, (unsigned)q.BH), kRangeThreads, 0, st>>>(V, q.n, p.rows_per_range,
+                                                                                           part);
+    colrange_finalize<<<(unsigned)ceil_div(q.BH * D, 256), 256, 0, st>>>(part, p.nsplit_range, D, q.BH, q.vmin,
+                                                                          q.vmax);
+    fty_kernel<E, D><<<dim3((unsigned)ceil_div(q.r, kFtyTJ), p.nsplit_k, (unsigned)q.BH), kFtyThreads, 0, st>>>(
+        q.F, V, q.n, q.r, p.keys_per_split, Ypart, q.BH);
+    gather_fs<<<dim3(q.r, (unsigned)q.BH), 128, 0, st>>>(q.F, q.S, q.rank, q.n, q.r, FS);
+    const size_t smem = sizeof(float) * (size_t)q.r * kTrsmCB;
+    cudaError_t e = cudaFuncSetAttribute(trsm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return Status::cuda(e, "weights: trsm smem attribute");
+    trsm_kernel<<<dim3((unsigned)ceil_div(D + 1, kTrsmCB), (unsigned)q.BH), kTrsmThreads, smem, st>>>(
+        Ypart, p.nsplit_k, FS, q.rank, q.BH, q.r, D, q.V_S, q.w);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return Status::cuda(e, "weights launch");
+    return Status::ok();
+}
+
+}  // namespace
+
+size_t weights_workspace_bytes(int64_t BH, int64_t n, int d, int r) {
+    const WeightsPlan p = make_plan(BH, n, r);
+    Carve cv(nullptr, 0);
+    cv.take(sizeof(float) * BH * p.nsplit_range * 2 * d);
+    cv.take(sizeof(float) * p.nsplit_k * BH * (int64_t)r * (d + 1));
+    cv.take(sizeof(float) * BH * (int64_t)r * r);
+    return cv.used + 256;
+}
+
+Status launch_weights(const WeightsRequest& q, cudaStream_t st) {
+    if ((size_t)q.r * kTrsmCB * sizeof(float) > 227 * 1024)
+        return Status::fail(2, "weights: r too large for the on-chip triangular solve");
+    const bool bf = q.dtype == 1;
+    switch (q.d) {
+        case 32: return bf ? run_weights<BF16, 32>(q, st) : run_weights<F32, 32>(q, st);
+        case 64: return bf ? run_weights<BF16, 64>(q, st) : run_weights<F32, 64>(q, st);
+        case 128: return bf ? run_weights<BF16, 128>(q, st) : run_weights<F32, 128>(q, st);
+    }
+    return Status::fail(2, "weights: unsupported head dim");
+}
+
+}  // namespace wildcat

@@ -49,6 +49,8 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_philox4x32_10.restype = None
     lib.oracle_pivot_uniform.argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int64]
     lib.oracle_pivot_uniform.restype = ctypes.c_double
+    lib.oracle_pivot_uniforms.argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int64, _f64p]
+    lib.oracle_pivot_uniforms.restype = None
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_exact_attention.argtypes = [_f64p, _f64p, _f64p, ctypes.c_int64, ctypes.c_int64,
@@ -123,6 +125,12 @@ class Oracle:
     def pivot_uniform(self, seed: int, step: int, inst: int) -> float:
         """Uniform in (0, 1] that draws pivot `step` of instance `inst`."""
         return float(self.lib.oracle_pivot_uniform(int(seed), int(step), int(inst)))
+
+    def pivot_uniforms(self, seed: int, BH: int, steps: int) -> np.ndarray:
+        """u[b, i] for every instance b < BH and step i < steps."""
+        u = np.zeros((BH, steps))
+        self.lib.oracle_pivot_uniforms(int(seed), int(BH), int(steps), u.ctypes.data_as(_f64p))
+        return u
 
     # -- exact attention ---------------------------------------------------------
     def exact_attention(self, Q, K, V, beta, rows=None):

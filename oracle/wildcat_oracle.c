@@ -96,6 +96,12 @@ double oracle_pivot_uniform(uint64_t seed, int64_t step, int64_t inst) {
     return ((double)bits + 1.0) * 0x1.0p-53;
 }
 
+/* u[b * steps + i] for b < BH, i < steps. */
+void oracle_pivot_uniforms(uint64_t seed, int64_t BH, int64_t steps, double* u) {
+    for (int64_t b = 0; b < BH; ++b)
+        for (int64_t i = 0; i < steps; ++i) u[b * steps + i] = oracle_pivot_uniform(seed, i, b);
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -1,0 +1,64 @@
+"""Helpers shared by the GPU parity tests (device path vs the fp64 oracle)."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+import workloads
+
+# Fixed-pivot parity bound on max_ij |O_gpu - O_oracle| / (v_max j - v_min j)
+# (the benchmark spec's tolerance: 1e-4 for float32 inputs, 2e-2 for bfloat16).
+TOL_R12 = {"f32": 1e-4, "bf16": 2e-2}
+# A pivot draw whose u*T lands within this fraction of T from a bucket edge
+# is a near-tie: fp32 (device) and fp64 (oracle) residuals may pick
+# neighbouring buckets there, and every later pivot may differ.
+TIE_MARGIN = 1e-4
+
+
+def case(name, dist, BH, n, m, d, r, dtype, seed=7, pivot_seed=11, beta=None):
+    return workloads.Workload(name=name, B=BH, H=1, n=n, m=m, d=d, r=r, dtype=dtype, dist=dist,
+                              beta=beta if beta is not None else 1.0 / math.sqrt(d), seed=seed,
+                              pivot_seed=pivot_seed)
+
+
+def cuda_inputs(dev):
+    return {k: v.cuda() for k, v in dev.items()}
+
+
+def r12(O_a, O_b, vmin, vmax):
+    """max over instances, rows, columns of |O_a - O_b| / (v_max j - v_min j)."""
+    span = np.maximum(vmax - vmin, 1e-30)[:, None, :]
+    return float(np.max(np.abs(np.asarray(O_a, np.float64) - O_b) / span))
+
+
+def pivots_agree_until_tie(S_gpu, S_orc, margin, rank_gpu, rank_orc):
+    """Pivot sequences must agree step by step until the oracle records a
+    near-tie draw; returns the number of steps compared for each instance."""
+    compared = []
+    for b in range(S_gpu.shape[0]):
+        k = 0
+        upto = min(rank_gpu[b], rank_orc[b])
+        while k < upto:
+            if S_gpu[b, k] != S_orc[b, k]:
+                assert margin[b, k] < TIE_MARGIN, (
+                    f"instance {b}: pivots differ at step {k} ({S_gpu[b, k]} vs {S_orc[b, k]}) "
+                    f"with oracle margin {margin[b, k]:.3e} (not a near-tie)")
+                break
+            k += 1
+        if k == upto and rank_gpu[b] != rank_orc[b]:
+            raise AssertionError(f"instance {b}: ranks differ ({rank_gpu[b]} vs {rank_orc[b]}) "
+                                 "with identical pivots")
+        compared.append(k)
+    return compared
+
+
+def column_rel_err(F_gpu, F_orc, rank):
+    """max over factor columns i < rank of max_l |dF| / max_l |F_orc|."""
+    worst = 0.0
+    for b in range(F_gpu.shape[0]):
+        for i in range(int(rank[b])):
+            ref = F_orc[b, i]
+            scale = max(np.abs(ref).max(), 1e-30)
+            worst = max(worst, float(np.abs(F_gpu[b, i] - ref).max() / scale))
+    return worst
