@@ -238,15 +238,18 @@ static int rpc_one(const double* Kb, int64_t n, int d, double beta, int r, uint6
                 margin[i] = (lo < hi ? lo : hi) / T;
             }
         }
-        /* 3e: column of the residual kernel at the pivot */
+        /* 3e: column of the residual kernel at the pivot,
+         *     g_l = kappa(k_l, k_s) - F_l0 F_s0 - F_l1 F_s1 - ... (in that order;
+         *     the loop over l is innermost only to walk F contiguously) */
         const double* ks = Kb + s * d;
-        for (int64_t l = 0; l < n; ++l) {
-            double v = exp(beta * (dot(Kb + l * d, ks, d) - MK));
+        for (int64_t l = 0; l < n; ++l) g[l] = exp(beta * (dot(Kb + l * d, ks, d) - MK));
 #if ORACLE_MUTANT != 1 /* planted (1): drop the subtraction of earlier columns */
-            for (int j = 0; j < i; ++j) v -= F[(int64_t)j * n + l] * F[(int64_t)j * n + s];
-#endif
-            g[l] = v;
+        for (int j = 0; j < i; ++j) {
+            const double* Fj = F + (int64_t)j * n;
+            const double fs = Fj[s];
+            for (int64_t l = 0; l < n; ++l) g[l] -= Fj[l] * fs;
         }
+#endif
         /* 3f: truncation stands in for the pseudo-inverse */
         if (!(g[s] > eps * dmax)) break;
         /* 3g: new factor column */

@@ -32,9 +32,15 @@ def r12(O_a, O_b, vmin, vmax):
     return float(np.max(np.abs(np.asarray(O_a, np.float64) - O_b) / span))
 
 
-def pivots_agree_until_tie(S_gpu, S_orc, margin, rank_gpu, rank_orc):
+def pivots_agree_until_tie(S_gpu, S_orc, margin, rank_gpu, rank_orc, F_gpu=None, F_orc=None,
+                           eps=1e-6):
     """Pivot sequences must agree step by step until the oracle records a
-    near-tie draw; returns the number of steps compared for each instance."""
+    near-tie draw; returns the number of steps compared for each instance.
+
+    With identical pivots the two sides may still stop at different steps
+    when the pivot residual g_s sits at the truncation threshold eps (float32
+    on the device, float64 in the oracle).  That is accepted only as a
+    near-tie: the side that went on must have had g_s = F[i, s]^2 < 2 eps."""
     compared = []
     for b in range(S_gpu.shape[0]):
         k = 0
@@ -47,8 +53,17 @@ def pivots_agree_until_tie(S_gpu, S_orc, margin, rank_gpu, rank_orc):
                 break
             k += 1
         if k == upto and rank_gpu[b] != rank_orc[b]:
-            raise AssertionError(f"instance {b}: ranks differ ({rank_gpu[b]} vs {rank_orc[b]}) "
-                                 "with identical pivots")
+            if rank_gpu[b] > rank_orc[b]:
+                S, F = S_gpu, F_gpu
+            else:
+                S, F = S_orc, F_orc
+            ok = False
+            if F is not None:
+                s = int(S[b, upto])
+                gs = float(F[b, upto, s]) ** 2
+                ok = gs < 2 * eps
+            assert ok, (f"instance {b}: ranks differ ({rank_gpu[b]} vs {rank_orc[b]}) with "
+                        "identical pivots and no truncation near-tie")
         compared.append(k)
     return compared
 
