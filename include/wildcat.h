@@ -156,6 +156,36 @@ wildcat_status wildcat_attend(const void* Q, const void* K_S, int dtype, int64_t
                               void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * wildcat_attend_noalloc -- wildcat_attend for callers that cannot allocate
+ * device memory.  The paper has no counterpart; this is a deployment
+ * convenience.  Such callers only hold pointers handed to them by another
+ * component that owns the GPU's memory (for example a serving engine that
+ * reserves nearly all of it for its KV cache), or run in a loop where a
+ * cudaMalloc, which can synchronise the device, is not acceptable, so they
+ * cannot supply the `workspace` that wildcat_attend needs.
+ *
+ * Same arguments and result as wildcat_attend, without workspace.  The
+ * caller still provides every input and the output O.  The call allocates
+ * nothing: its scratch is a static device array of
+ * WILDCAT_NOALLOC_SCRATCH_BYTES (1 MiB) that every GPU loading this library
+ * holds until the process exits.  Sizes needing more than that, about
+ * 4 * BH * (min(64, ceil(m / 1024)) + 1) bytes, return
+ * WILDCAT_ERR_UNSUPPORTED before anything is launched.
+ *
+ * The first call on each device looks up the array's device address (a
+ * host-side runtime query, no allocation); make that first call before any
+ * stream capture.  All calls share the one array, so calls whose work
+ * overlaps on the GPU (e.g. on two streams) race and must be serialised by
+ * the caller.  Each call writes every scratch word before reading it, so
+ * the contents left by an earlier call do not matter.
+ */
+#define WILDCAT_NOALLOC_SCRATCH_BYTES (1u << 20)
+wildcat_status wildcat_attend_noalloc(const void* Q, const void* K_S, int dtype, int64_t BH,
+                                      int64_t m, int d, int r, const int32_t* rank, float beta,
+                                      const float* V_S, const float* w, const float* vmin,
+                                      const float* vmax, float* O, void* stream);
+
+/*
  * wildcat_forward -- the whole module (Alg. 4): select -> weights -> attend,
  * all on `stream`, with every intermediate in `workspace`.
  *

@@ -24,7 +24,7 @@ from typing import Optional
 
 __all__ = [
     "WildcatError", "library_path", "lib", "declared_symbols", "select", "select_fixed",
-    "weights", "attend", "forward", "forward_host", "ForwardPlan", "pivot_uniforms",
+    "weights", "attend", "attend_noalloc", "forward", "forward_host", "ForwardPlan", "pivot_uniforms",
     "set_select_cluster", "last_select_cluster", "DTYPES",
 ]
 
@@ -54,6 +54,8 @@ _SIGS = {
     "wildcat_attend_workspace_size": ([_i64, _i64, _int, _int], _sz),
     "wildcat_attend": ([_vp, _vp, _int, _i64, _i64, _int, _int, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp,
                         _sz, _vp], _int),
+    "wildcat_attend_noalloc": ([_vp, _vp, _int, _i64, _i64, _int, _int, _vp, _f32, _vp, _vp, _vp, _vp,
+                                _vp, _vp], _int),
     "wildcat_forward_workspace_size": ([_i64, _i64, _i64, _int, _int, _int], _sz),
     "wildcat_forward": ([_vp, _vp, _vp, _int, _i64, _i64, _i64, _int, _f32, _int, _u64, _f32, _vp, _vp,
                          _vp, _vp, _sz, _vp], _int),
@@ -224,6 +226,27 @@ def attend(Q, K_S, rank, beta: float, V_S, w, vmin, vmax, *, stream=None):
                             _dev(V_S, "V_S", torch.float32), _dev(w, "w", torch.float32),
                             _dev(vmin, "vmin", torch.float32), _dev(vmax, "vmax", torch.float32),
                             _dev(O, "O"), _dev(ws, "workspace"), nbytes, _stream(stream)))
+    return O
+
+
+def attend_noalloc(Q, K_S, rank, beta: float, V_S, w, vmin, vmax, *, out=None, stream=None):
+    """wildcat_attend_noalloc: the same result as ``attend`` from a library
+    call that allocates nothing (its scratch is a static 1 MiB device array;
+    for callers that cannot allocate device memory).  ``out`` (optional) is
+    the caller's O [BH, m, d] float32; without it torch allocates O here,
+    outside the library call."""
+    torch = _torch()
+    BH, m, d = _shape3(Q, "Q")
+    r = K_S.shape[1]
+    if K_S.dtype != Q.dtype:
+        raise TypeError("Q and K_S must share a dtype")
+    O = out if out is not None else torch.empty((BH, m, d), dtype=torch.float32, device=Q.device)
+    _check(lib().wildcat_attend_noalloc(_dev(Q, "Q"), _dev(K_S, "K_S"), _dtype_code(Q), BH, m, d, r,
+                                        _dev(rank, "rank", torch.int32), float(beta),
+                                        _dev(V_S, "V_S", torch.float32), _dev(w, "w", torch.float32),
+                                        _dev(vmin, "vmin", torch.float32),
+                                        _dev(vmax, "vmax", torch.float32),
+                                        _dev(O, "O", torch.float32), _stream(stream)))
     return O
 
 

@@ -201,6 +201,21 @@ wildcat_status wildcat_attend(const void* Q, const void* K_S, int dtype, int64_t
     return record(wildcat::launch_attend(q, static_cast<cudaStream_t>(stream)));
 }
 
+wildcat_status wildcat_attend_noalloc(const void* Q, const void* K_S, int dtype, int64_t BH, int64_t m, int d, int r,
+                                      const int32_t* rank, float beta, const float* V_S, const float* w,
+                                      const float* vmin, const float* vmax, float* O, void* stream) {
+    const char* who = "wildcat_attend_noalloc";
+    wildcat_status st = check_common(dtype, BH, r, d, r, who);
+    if (st != WILDCAT_OK) return st;
+    if ((st = check_scalars(beta, 0.f, who)) != WILDCAT_OK) return st;
+    if (m < 0) return bad(1, "%s: m must be >= 0", who);
+    if (BH == 0 || m == 0) return record(Status::ok());
+    if (!Q || !K_S || !rank || !V_S || !w || !vmin || !vmax || !O) return bad(1, "%s: null pointer argument", who);
+    if (!aligned16(Q) || !aligned16(K_S)) return bad(1, "%s: Q and K_S must be 16-byte aligned", who);
+    wildcat::AttendRequest q{Q, K_S, dtype, BH, m, d, r, rank, beta, V_S, w, vmin, vmax, O, nullptr, 0};
+    return record(wildcat::launch_attend_noalloc(q, static_cast<cudaStream_t>(stream)));
+}
+
 size_t wildcat_forward_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int dtype) {
     if (BH < 0 || m < 0 || n < 1 || r < 1 || d < 1) return 0;
     Carve cv(nullptr, 0);

@@ -12,6 +12,7 @@
 //                                    - beta M_Q) chunk by chunk, N += P V_S,
 //                                    D += P w, then O = clip(N / D)
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -208,6 +209,73 @@ Status launch_attend(const AttendRequest& q, cudaStream_t st) {
         case 128: return bf ? run_attend<BF16, 128>(q, st) : run_attend<F32, 128>(q, st);
     }
     return Status::fail(2, "attend: unsupported head dim");
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free attend (wildcat_attend_noalloc).
+//
+// Some callers cannot hand the library a workspace: they only hold pointers
+// that another component gave them, inside a process whose device memory is
+// owned by that component (for example a serving engine that reserves almost
+// all of the GPU for its KV cache and routes every allocation through its own
+// pool), or they run in a latency-critical loop where a cudaMalloc, which can
+// synchronise the device, is not acceptable.  For them the attend's small
+// scratch (per-instance query-norm partials and the shift M_Q) lives in the
+// fixed device array below instead of a caller workspace.
+//
+// The array is kNoAllocScratchBytes (1 MiB) and exists on every GPU on which
+// this library's kernels are loaded, until the process exits.  Host code may
+// not pass the array's name to a kernel (on the host it is only a stand-in
+// symbol), so the device address is looked up with cudaGetSymbolAddress once
+// per device, with that device current, on the first no-alloc call made
+// there; make that first call before any stream capture.  All calls share
+// the array: calls whose kernels overlap on the GPU (for example on two
+// streams at once) race on it and must be serialised by the caller.  Every
+// scratch word a call reads is written earlier in the same call, so nothing
+// needs clearing between calls.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;
+constexpr int kNoAllocMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_attend_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kNoAllocMaxDevices] = {};
+
+Status attend_scratch_address(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return Status::cuda(e, "attend_noalloc: cudaGetDevice");
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return Status::fail(2, "attend_noalloc: device ordinal above 63");
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_attend_scratch);
+        if (e != cudaSuccess || p == nullptr)
+            return Status::cuda(e != cudaSuccess ? e : cudaErrorInvalidSymbol,
+                                "attend_noalloc: cudaGetSymbolAddress of the static scratch");
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return Status::ok();
+}
+}  // namespace
+
+size_t attend_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+Status launch_attend_noalloc(const AttendRequest& q_in, cudaStream_t st) {
+    if (attend_workspace_bytes(q_in.BH, q_in.m, q_in.d, q_in.r) > kNoAllocScratchBytes)
+        return Status::fail(2,
+                            "wildcat_attend_noalloc: BH and m need more scratch than the 1 MiB static array "
+                            "(about 4 * BH * (min(64, ceil(m / 1024)) + 1) bytes); use wildcat_attend with a workspace");
+    void* scratch = nullptr;
+    const Status s = attend_scratch_address(&scratch);
+    if (s.code) return s;
+    AttendRequest q = q_in;
+    q.ws = scratch;
+    q.ws_bytes = kNoAllocScratchBytes;
+    return launch_attend(q, st);
 }
 
 }  // namespace wildcat

@@ -76,6 +76,9 @@ struct AttendRequest {
 };
 size_t attend_workspace_bytes(int64_t BH, int64_t m, int d, int r);
 Status launch_attend(const AttendRequest& q, cudaStream_t stream);
+// attend with its scratch in a static device array (no workspace argument)
+size_t attend_noalloc_scratch_bytes();
+Status launch_attend_noalloc(const AttendRequest& q, cudaStream_t stream);
 
 // 256-byte aligned bump allocator over a caller-provided workspace.
 struct Carve {
