@@ -36,9 +36,17 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "WildCat fwd calls/s & effective m*n attention entries/s on 1 B200; % roofline"
-LAUNCHES_PER_FORWARD = 9  # select 1 + weights 5 + attend 3
 FLUSH_BYTES = 256 << 20
 EPS = 1e-6
+
+
+def launches_per_forward(w):
+    """Kernels one wildcat_forward launches: select 1, weights 5 (range partial
+    and finalize, F^T(V,1), pivot-block gather, solve), attend 3 on CUDA
+    cores (norm partials, shift, attend) or 4 on the tensor-core path (plus
+    the hi/lo split of [V_S|w])."""
+    tc = w.dtype == "bf16" and w.d in (64, 128)
+    return 1 + 5 + (4 if tc else 3)
 
 
 def parse():
@@ -221,6 +229,7 @@ def main():
 
     import nystr_coreset_approximate_b200 as wc
     import workloads
+    from nystr_coreset_approximate_b200 import sharding
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -264,10 +273,7 @@ def main():
     barrier()
     clk = clocks.stop()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(total_ms, op=dist.ReduceOp.MAX)
-    total_ms = float(total_ms.item())
+    total_ms = sharding.max_over_ranks(sum(step_ms), device="cuda")
 
     # ---- per-stage breakdown through the staged C-ABI calls (same kernels) ----
     stage_ms = {"select": [], "weights": [], "attend": []}
@@ -311,11 +317,9 @@ def main():
             b.record()
             b.synchronize()
             e_ms.append(a.elapsed_time(b))
-        e_tot = torch.tensor([sum(e_ms)], dtype=torch.float64, device="cuda")
-        if world > 1:
-            dist.all_reduce(e_tot, op=dist.ReduceOp.MAX)
+        e_tot = sharding.max_over_ranks(sum(e_ms), device="cuda")
         eb = 2 if w.dtype == "bf16" else 4
-        e2e = {"value": world * args.steps / (float(e_tot.item()) / 1e3), "unit": "calls/s",
+        e2e = {"value": world * args.steps / (e_tot / 1e3), "unit": "calls/s",
                "h2d_bytes_per_step": eb * w.BH * (w.m + 2 * w.n) * w.d,
                "d2h_bytes_per_step": 4 * w.BH * w.m * w.d + 4 * w.BH * w.r + 4 * w.BH,
                "api": "wildcat_forward_host (pinned host buffers)"}
@@ -349,7 +353,7 @@ def main():
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} hbm_gbs", "traffic": traffic,
                      "algorithmic_bytes_per_launch": nbytes, "launch_ms": sel_ms},
-        "gpu_launches": LAUNCHES_PER_FORWARD * args.steps,
+        "gpu_launches": launches_per_forward(w) * args.steps,
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cpu,

@@ -14,7 +14,11 @@
  *            (Sec. 2 plug-in estimator; Alg. 2 CompressKV)
  *   attend   O_hat = diag(U w)^-1 U V_S, U = exp(beta Q K_S^T), each entry
  *            clipped to the value range [v_min j, v_max j] of V
- *            (Sec. 2, value-range clip; Alg. 3 WtdAttn)
+ *            (Sec. 2, value-range clip; Alg. 3 WtdAttn); bf16 inputs with
+ *            d in {64, 128} run on the tensor cores (tcgen05, fp32
+ *            accumulation in tensor memory, P rounded to bf16 once and used
+ *            for both numerator and denominator, [V_S | w] split into bf16
+ *            hi + lo parts); other inputs on CUDA cores in fp32
  *   forward  the three stages back to back (Alg. 4, the WildCat module)
  *
  * Conventions shared by every call
@@ -46,9 +50,12 @@
  *    there.
  *  - Pivot draws: uniform u_i of step i for instance b is Philox4x32-10
  *    (Salmon et al., SC'11) with key (seed_lo, seed_hi) and counter
- *    (i, b, 0, 0); u = (x + 1) * 2^-53 where x is the top 53 bits of the
- *    64-bit word (x1:x0).  The pivot is the first key whose cumulative
- *    residual diagonal reaches u * T, T the total residual mass.
+ *    (i, inst0 + b, 0, 0); u = (x + 1) * 2^-53 where x is the top 53 bits of
+ *    the 64-bit word (x1:x0).  The pivot is the first key whose cumulative
+ *    residual diagonal reaches u * T, T the total residual mass.  inst0 is
+ *    the global index of the call's first instance: a batch split into
+ *    shards (e.g. one per GPU) draws exactly the pivots of the whole batch
+ *    when each shard passes its offset.
  */
 #ifndef WILDCAT_H_
 #define WILDCAT_H_
@@ -65,7 +72,8 @@ typedef enum {
     WILDCAT_ERR_INVALID_ARG = 1, /* null pointer, bad size, misalignment */
     WILDCAT_ERR_UNSUPPORTED = 2, /* valid but not implemented (head dim, size limit) */
     WILDCAT_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
-    WILDCAT_ERR_WORKSPACE = 4    /* workspace too small or misaligned */
+    WILDCAT_ERR_WORKSPACE = 4,   /* workspace too small or misaligned */
+    WILDCAT_ERR_TIMEOUT = 5      /* a kernel's bounded wait expired (see wildcat_get_device_status) */
 } wildcat_status;
 
 typedef enum { WILDCAT_F32 = 0, WILDCAT_BF16 = 1 } wildcat_dtype;
@@ -92,6 +100,7 @@ const char* wildcat_status_string(int status);
  *   beta   kernel inverse temperature (> 0, finite)
  *   r      coreset size, 1 <= r <= n
  *   seed   64-bit Philox key of the pivot draws
+ *   inst0  global index of instance 0 of this call (0 unless sharded), >= 0
  *   eps    truncation threshold (relative to max_l h(k_l, k_l)), >= 0
  *   S      out [BH, r] int32 pivot indices in draw order, -1 past the rank
  *   F      out [BH, r, n] float32 factor
@@ -99,7 +108,7 @@ const char* wildcat_status_string(int status);
  *   K_S    out [BH, r, d] gathered pivot keys (dtype `dtype`), or NULL
  */
 wildcat_status wildcat_select(const void* K, int dtype, int64_t BH, int64_t n, int d, float beta,
-                              int r, uint64_t seed, float eps, int32_t* S, float* F,
+                              int r, uint64_t seed, int64_t inst0, float eps, int32_t* S, float* F,
                               int32_t* rank, void* K_S, void* stream);
 
 /*
@@ -187,7 +196,8 @@ wildcat_status wildcat_attend_noalloc(const void* Q, const void* K_S, int dtype,
 
 /*
  * wildcat_forward -- the whole module (Alg. 4): select -> weights -> attend,
- * all on `stream`, with every intermediate in `workspace`.
+ * all on `stream`, with every intermediate in `workspace`.  seed, inst0 and
+ * eps as in wildcat_select.
  *
  *   Q [BH, m, d], K and V [BH, n, d] (dtype `dtype`); O out [BH, m, d] float32
  *   S_out [BH, r] int32 and rank_out [BH] int32: optional copies (or NULL)
@@ -196,8 +206,8 @@ wildcat_status wildcat_attend_noalloc(const void* Q, const void* K_S, int dtype,
 size_t wildcat_forward_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int dtype);
 wildcat_status wildcat_forward(const void* Q, const void* K, const void* V, int dtype, int64_t BH,
                                int64_t m, int64_t n, int d, float beta, int r, uint64_t seed,
-                               float eps, float* O, int32_t* S_out, int32_t* rank_out,
-                               void* workspace, size_t ws_bytes, void* stream);
+                               int64_t inst0, float eps, float* O, int32_t* S_out,
+                               int32_t* rank_out, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * wildcat_forward_host -- wildcat_forward on HOST buffers: copies Q, K, V
@@ -214,17 +224,38 @@ size_t wildcat_forward_host_workspace_size(int64_t BH, int64_t m, int64_t n, int
                                            int dtype);
 wildcat_status wildcat_forward_host(const void* Q_host, const void* K_host, const void* V_host,
                                     int dtype, int64_t BH, int64_t m, int64_t n, int d,
-                                    float beta, int r, uint64_t seed, float eps, float* O_host,
-                                    int32_t* S_host, int32_t* rank_host, void* workspace,
-                                    size_t ws_bytes, void* stream);
+                                    float beta, int r, uint64_t seed, int64_t inst0, float eps,
+                                    float* O_host, int32_t* S_host, int32_t* rank_host,
+                                    void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * wildcat_pivot_uniforms -- the pivot uniforms the select kernels draw
- * (test entry point): u[b, i] for b < BH, i < steps, as float64, written to
- * the device array u [BH, steps].
+ * (test entry point): u[b, i] for b < BH, i < steps (instance offset 0), as
+ * float64, written to the device array u [BH, steps].
  */
 wildcat_status wildcat_pivot_uniforms(uint64_t seed, int64_t BH, int steps, double* u,
                                       void* stream);
+
+/*
+ * wildcat_get_device_status -- waits for `stream`, then reports and clears
+ * the device status word of the current device.  Kernels that wait on the
+ * tensor cores (mbarrier waits) bound every wait by a time limit; when one
+ * expires the kernel records WILDCAT_ERR_TIMEOUT there, stops issuing work,
+ * releases its tensor memory and returns, leaving its output incomplete.
+ * Returns WILDCAT_OK, WILDCAT_ERR_TIMEOUT, or WILDCAT_ERR_CUDA if the stream
+ * or the status word could not be read.
+ */
+wildcat_status wildcat_get_device_status(void* stream);
+
+/*
+ * wildcat_test_force_wait_timeout -- test hook for the bounded waits.  With
+ * nanoseconds > 0 every later tensor-core attend launch first waits that long
+ * on a barrier phase that nothing completes, records WILDCAT_ERR_TIMEOUT in
+ * the device status word, releases its tensor memory and returns without
+ * writing O.  0 turns the hook off.  Process-wide; for tests only.
+ * Returns WILDCAT_ERR_INVALID_ARG outside [0, 1e9].
+ */
+wildcat_status wildcat_test_force_wait_timeout(int64_t nanoseconds);
 
 /*
  * wildcat_set_select_cluster -- tuning knob for wildcat_select*: number of

@@ -25,7 +25,7 @@ from typing import Optional
 __all__ = [
     "WildcatError", "library_path", "lib", "declared_symbols", "select", "select_fixed",
     "weights", "attend", "attend_noalloc", "forward", "forward_host", "ForwardPlan", "pivot_uniforms",
-    "set_select_cluster", "last_select_cluster", "DTYPES",
+    "set_select_cluster", "last_select_cluster", "device_status", "DTYPES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -44,8 +44,8 @@ _SIGS = {
     "wildcat_version": ([], _int),
     "wildcat_last_error": ([], ctypes.c_char_p),
     "wildcat_status_string": ([_int], ctypes.c_char_p),
-    "wildcat_select": ([_vp, _int, _i64, _i64, _int, _f32, _int, _u64, _f32, _vp, _vp, _vp, _vp, _vp],
-                       _int),
+    "wildcat_select": ([_vp, _int, _i64, _i64, _int, _f32, _int, _u64, _i64, _f32, _vp, _vp, _vp, _vp,
+                        _vp], _int),
     "wildcat_select_fixed": ([_vp, _int, _i64, _i64, _int, _f32, _int, _f32, _vp, _vp, _vp, _vp, _vp,
                               _vp], _int),
     "wildcat_weights_workspace_size": ([_i64, _i64, _int, _int], _sz),
@@ -57,12 +57,14 @@ _SIGS = {
     "wildcat_attend_noalloc": ([_vp, _vp, _int, _i64, _i64, _int, _int, _vp, _f32, _vp, _vp, _vp, _vp,
                                 _vp, _vp], _int),
     "wildcat_forward_workspace_size": ([_i64, _i64, _i64, _int, _int, _int], _sz),
-    "wildcat_forward": ([_vp, _vp, _vp, _int, _i64, _i64, _i64, _int, _f32, _int, _u64, _f32, _vp, _vp,
-                         _vp, _vp, _sz, _vp], _int),
+    "wildcat_forward": ([_vp, _vp, _vp, _int, _i64, _i64, _i64, _int, _f32, _int, _u64, _i64, _f32, _vp,
+                         _vp, _vp, _vp, _sz, _vp], _int),
     "wildcat_forward_host_workspace_size": ([_i64, _i64, _i64, _int, _int, _int], _sz),
-    "wildcat_forward_host": ([_vp, _vp, _vp, _int, _i64, _i64, _i64, _int, _f32, _int, _u64, _f32, _vp,
-                              _vp, _vp, _vp, _sz, _vp], _int),
+    "wildcat_forward_host": ([_vp, _vp, _vp, _int, _i64, _i64, _i64, _int, _f32, _int, _u64, _i64, _f32,
+                              _vp, _vp, _vp, _vp, _sz, _vp], _int),
     "wildcat_pivot_uniforms": ([_u64, _i64, _int, _vp, _vp], _int),
+    "wildcat_get_device_status": ([_vp], _int),
+    "wildcat_test_force_wait_timeout": ([_i64], _int),
     "wildcat_set_select_cluster": ([_int], _int),
     "wildcat_last_select_cluster": ([], _int),
 }
@@ -154,10 +156,12 @@ def _shape3(t, name):
 
 
 # --------------------------------------------------------------------------- calls
-def select(K, beta: float, r: int, seed: int = 0, eps: float = 1e-6, *, out=None, stream=None):
+def select(K, beta: float, r: int, seed: int = 0, eps: float = 1e-6, *, inst0: int = 0, out=None,
+           stream=None):
     """RPCholesky coreset selection (Alg. 1 RPNys).  K [BH, n, d] (float32 or
-    bfloat16, CUDA).  Returns (S [BH,r] int32, F [BH,r,n] float32, rank [BH]
-    int32, K_S [BH,r,d])."""
+    bfloat16, CUDA).  inst0 is the global index of K's first instance (for a
+    shard of a larger batch).  Returns (S [BH,r] int32, F [BH,r,n] float32,
+    rank [BH] int32, K_S [BH,r,d])."""
     torch = _torch()
     BH, n, d = _shape3(K, "K")
     S, F, rank, K_S = out if out is not None else (
@@ -166,7 +170,8 @@ def select(K, beta: float, r: int, seed: int = 0, eps: float = 1e-6, *, out=None
         torch.empty((BH,), dtype=torch.int32, device=K.device),
         torch.empty((BH, r, d), dtype=K.dtype, device=K.device))
     _check(lib().wildcat_select(_dev(K, "K"), _dtype_code(K), BH, n, d, float(beta), int(r),
-                                int(seed) & (2**64 - 1), float(eps), _dev(S, "S", torch.int32),
+                                int(seed) & (2**64 - 1), int(inst0), float(eps),
+                                _dev(S, "S", torch.int32),
                                 _dev(F, "F", torch.float32), _dev(rank, "rank", torch.int32),
                                 _opt(K_S, "K_S", K.dtype), _stream(stream)))
     return S, F, rank, K_S
@@ -265,24 +270,27 @@ class ForwardPlan:
         self.S = torch.empty((BH, r), dtype=torch.int32, device=device)
         self.rank = torch.empty((BH,), dtype=torch.int32, device=device)
 
-    def run(self, Q, K, V, beta, seed, eps=1e-6, stream=None):
+    def run(self, Q, K, V, beta, seed, eps=1e-6, stream=None, inst0=0):
         _check(lib().wildcat_forward(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), self.code, self.BH,
                                      self.m, self.n, self.d, float(beta), self.r,
-                                     int(seed) & (2**64 - 1), float(eps), _dev(self.O, "O"),
+                                     int(seed) & (2**64 - 1), int(inst0), float(eps),
+                                     _dev(self.O, "O"),
                                      _dev(self.S, "S"), _dev(self.rank, "rank"),
                                      _dev(self.ws, "workspace"), self.ws_bytes, _stream(stream)))
         return self.O, self.S, self.rank
 
 
-def forward(Q, K, V, beta: float, r: int, seed: int = 0, eps: float = 1e-6, *, stream=None):
-    """The whole WildCat module (Alg. 4).  Returns (O_hat, S, rank)."""
+def forward(Q, K, V, beta: float, r: int, seed: int = 0, eps: float = 1e-6, *, inst0: int = 0,
+            stream=None):
+    """The whole WildCat module (Alg. 4).  Returns (O_hat, S, rank).  inst0:
+    global index of the first instance (for a shard of a larger batch)."""
     BH, m, d = _shape3(Q, "Q")
     n = K.shape[1]
     code = _dtype_code(K)
     if Q.dtype != K.dtype or V.dtype != K.dtype:
         raise TypeError("Q, K, V must share a dtype")
     plan = ForwardPlan(BH, m, n, d, r, "bf16" if code else "f32", device=K.device)
-    O, S, rank = plan.run(Q, K, V, beta, seed, eps, stream)
+    O, S, rank = plan.run(Q, K, V, beta, seed, eps, stream, inst0)
     return O.clone(), S.clone(), rank.clone()
 
 
@@ -298,14 +306,14 @@ class HostForwardPlan:
         self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
 
     def run(self, Q_host, K_host, V_host, O_host, beta, seed, eps=1e-6, S_host=None,
-            rank_host=None, stream=None):
+            rank_host=None, stream=None, inst0=0):
         for t, nm in ((Q_host, "Q"), (K_host, "K"), (V_host, "V"), (O_host, "O")):
             if t.is_cuda or not t.is_contiguous():
                 raise ValueError(f"{nm} must be a contiguous host tensor")
         _check(lib().wildcat_forward_host(
             _vp(Q_host.data_ptr()), _vp(K_host.data_ptr()), _vp(V_host.data_ptr()), self.code,
             self.BH, self.m, self.n, self.d, float(beta), self.r, int(seed) & (2**64 - 1),
-            float(eps), _vp(O_host.data_ptr()),
+            int(inst0), float(eps), _vp(O_host.data_ptr()),
             None if S_host is None else _vp(S_host.data_ptr()),
             None if rank_host is None else _vp(rank_host.data_ptr()),
             _dev(self.ws, "workspace"), self.ws_bytes, _stream(stream)))
@@ -332,6 +340,12 @@ def pivot_uniforms(seed: int, BH: int, steps: int, device="cuda"):
     _check(lib().wildcat_pivot_uniforms(int(seed) & (2**64 - 1), BH, steps, _dev(u, "u"),
                                         _stream()))
     return u
+
+
+def device_status(stream=None) -> int:
+    """Wait for the stream, then return and clear the device status word
+    (0 = fine, 5 = a kernel's bounded wait expired)."""
+    return int(lib().wildcat_get_device_status(_stream(stream)))
 
 
 def set_select_cluster(G: int):

@@ -57,17 +57,18 @@ wildcat_status check_scalars(float beta, float eps, const char* who) {
 }
 
 wildcat_status select_impl(const void* K, int dtype, int64_t BH, int64_t n, int d, float beta, int r, uint64_t seed,
-                           float eps, const int32_t* S_fixed, int32_t* S, float* F, int32_t* rank, void* K_S,
-                           void* stream, const char* who) {
+                           int64_t inst0, float eps, const int32_t* S_fixed, int32_t* S, float* F, int32_t* rank,
+                           void* K_S, void* stream, const char* who) {
     wildcat_status st = check_common(dtype, BH, n, d, r, who);
     if (st != WILDCAT_OK) return st;
     if ((st = check_scalars(beta, eps, who)) != WILDCAT_OK) return st;
+    if (inst0 < 0 || inst0 + BH > 4294967296LL) return bad(1, "%s: inst0 must satisfy 0 <= inst0, inst0 + BH <= 2^32", who);
     if (BH == 0) return record(Status::ok());
     if (!K || !F || !rank) return bad(1, "%s: K, F and rank must be non-null", who);
     if (!S_fixed && !S) return bad(1, "%s: S must be non-null", who);
     if (!aligned16(K) || !aligned16(F) || (K_S && !aligned16(K_S)))
         return bad(1, "%s: K, F and K_S must be 16-byte aligned", who);
-    wildcat::SelectRequest q{K, dtype, BH, n, d, beta, r, seed, eps, S_fixed, S, F, rank, K_S};
+    wildcat::SelectRequest q{K, dtype, BH, n, d, beta, r, seed, inst0, eps, S_fixed, S, F, rank, K_S};
     return record(wildcat::launch_select(q, static_cast<cudaStream_t>(stream)));
 }
 
@@ -104,10 +105,10 @@ ForwardLayout carve_forward(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, 
 }
 
 wildcat_status forward_impl(const void* Q, const void* K, const void* V, int dtype, int64_t BH, int64_t m, int64_t n,
-                            int d, float beta, int r, uint64_t seed, float eps, float* O, int32_t* S_out,
-                            int32_t* rank_out, const ForwardLayout& L, cudaStream_t st) {
+                            int d, float beta, int r, uint64_t seed, int64_t inst0, float eps, float* O,
+                            int32_t* S_out, int32_t* rank_out, const ForwardLayout& L, cudaStream_t st) {
     Status s;
-    wildcat::SelectRequest sq{K, dtype, BH, n, d, beta, r, seed, eps, nullptr, L.S, L.F, L.rank, L.K_S};
+    wildcat::SelectRequest sq{K, dtype, BH, n, d, beta, r, seed, inst0, eps, nullptr, L.S, L.F, L.rank, L.K_S};
     if ((s = wildcat::launch_select(sq, st)).code) return record(s);
     wildcat::WeightsRequest wq{L.F, L.S, L.rank, V, dtype, BH, n, d, r, L.V_S, L.w, L.vmin, L.vmax, L.wws,
                                L.wws_bytes};
@@ -140,20 +141,23 @@ const char* wildcat_status_string(int status) {
         case WILDCAT_ERR_UNSUPPORTED: return "WILDCAT_ERR_UNSUPPORTED";
         case WILDCAT_ERR_CUDA: return "WILDCAT_ERR_CUDA";
         case WILDCAT_ERR_WORKSPACE: return "WILDCAT_ERR_WORKSPACE";
+        case WILDCAT_ERR_TIMEOUT: return "WILDCAT_ERR_TIMEOUT";
     }
     return "WILDCAT_UNKNOWN_STATUS";
 }
 
 wildcat_status wildcat_select(const void* K, int dtype, int64_t BH, int64_t n, int d, float beta, int r, uint64_t seed,
-                              float eps, int32_t* S, float* F, int32_t* rank, void* K_S, void* stream) {
-    return select_impl(K, dtype, BH, n, d, beta, r, seed, eps, nullptr, S, F, rank, K_S, stream, "wildcat_select");
+                              int64_t inst0, float eps, int32_t* S, float* F, int32_t* rank, void* K_S,
+                              void* stream) {
+    return select_impl(K, dtype, BH, n, d, beta, r, seed, inst0, eps, nullptr, S, F, rank, K_S, stream,
+                       "wildcat_select");
 }
 
 wildcat_status wildcat_select_fixed(const void* K, int dtype, int64_t BH, int64_t n, int d, float beta, int r,
                                     float eps, const int32_t* S_fixed, int32_t* S, float* F, int32_t* rank,
                                     void* K_S, void* stream) {
     if (!S_fixed && BH > 0) return bad(1, "%s: S_fixed must be non-null", "wildcat_select_fixed");
-    return select_impl(K, dtype, BH, n, d, beta, r, 0, eps, S_fixed, S, F, rank, K_S, stream,
+    return select_impl(K, dtype, BH, n, d, beta, r, 0, 0, eps, S_fixed, S, F, rank, K_S, stream,
                        "wildcat_select_fixed");
 }
 
@@ -224,7 +228,7 @@ size_t wildcat_forward_workspace_size(int64_t BH, int64_t m, int64_t n, int d, i
 }
 
 wildcat_status wildcat_forward(const void* Q, const void* K, const void* V, int dtype, int64_t BH, int64_t m,
-                               int64_t n, int d, float beta, int r, uint64_t seed, float eps, float* O,
+                               int64_t n, int d, float beta, int r, uint64_t seed, int64_t inst0, float eps, float* O,
                                int32_t* S_out, int32_t* rank_out, void* workspace, size_t ws_bytes, void* stream) {
     const char* who = "wildcat_forward";
     wildcat_status st = check_common(dtype, BH, n, d, r, who);
@@ -239,7 +243,8 @@ wildcat_status wildcat_forward(const void* Q, const void* K, const void* V, int 
     Carve cv(workspace, ws_bytes);
     const ForwardLayout L = carve_forward(cv, BH, m, n, d, r, dtype);
     if (!cv.fits()) return bad(4, "%s: workspace too small", who);
-    return forward_impl(Q, K, V, dtype, BH, m, n, d, beta, r, seed, eps, O, S_out, rank_out, L,
+    if (inst0 < 0 || inst0 + BH > 4294967296LL) return bad(1, "%s: inst0 must satisfy 0 <= inst0, inst0 + BH <= 2^32", who);
+    return forward_impl(Q, K, V, dtype, BH, m, n, d, beta, r, seed, inst0, eps, O, S_out, rank_out, L,
                         static_cast<cudaStream_t>(stream));
 }
 
@@ -257,8 +262,8 @@ size_t wildcat_forward_host_workspace_size(int64_t BH, int64_t m, int64_t n, int
 }
 
 wildcat_status wildcat_forward_host(const void* Q_host, const void* K_host, const void* V_host, int dtype, int64_t BH,
-                                    int64_t m, int64_t n, int d, float beta, int r, uint64_t seed, float eps,
-                                    float* O_host, int32_t* S_host, int32_t* rank_host, void* workspace,
+                                    int64_t m, int64_t n, int d, float beta, int r, uint64_t seed, int64_t inst0,
+                                    float eps, float* O_host, int32_t* S_host, int32_t* rank_host, void* workspace,
                                     size_t ws_bytes, void* stream) {
     const char* who = "wildcat_forward_host";
     wildcat_status st = check_common(dtype, BH, n, d, r, who);
@@ -268,6 +273,7 @@ wildcat_status wildcat_forward_host(const void* Q_host, const void* K_host, cons
     if (BH == 0) return record(Status::ok());
     if (!K_host || !V_host || !workspace || (m > 0 && (!Q_host || !O_host)))
         return bad(1, "%s: null pointer argument", who);
+    if (inst0 < 0 || inst0 + BH > 4294967296LL) return bad(1, "%s: inst0 must satisfy 0 <= inst0, inst0 + BH <= 2^32", who);
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t eb = elem_bytes(dtype);
@@ -287,8 +293,8 @@ wildcat_status wildcat_forward_host(const void* Q_host, const void* K_host, cons
         return record(Status::cuda(e, "forward_host: copy K"));
     if ((e = cudaMemcpyAsync(Vd, V_host, eb * BH * n * d, cudaMemcpyHostToDevice, s)))
         return record(Status::cuda(e, "forward_host: copy V"));
-    st = forward_impl(m > 0 ? Qd : nullptr, Kd, Vd, dtype, BH, m, n, d, beta, r, seed, eps, m > 0 ? Od : nullptr, Sd,
-                      Rd, L, s);
+    st = forward_impl(m > 0 ? Qd : nullptr, Kd, Vd, dtype, BH, m, n, d, beta, r, seed, inst0, eps,
+                      m > 0 ? Od : nullptr, Sd, Rd, L, s);
     if (st != WILDCAT_OK) return st;
     if (m > 0 && (e = cudaMemcpyAsync(O_host, Od, sizeof(float) * BH * m * d, cudaMemcpyDeviceToHost, s)))
         return record(Status::cuda(e, "forward_host: copy O"));
@@ -304,6 +310,22 @@ wildcat_status wildcat_pivot_uniforms(uint64_t seed, int64_t BH, int steps, doub
     if (BH < 0 || steps < 0) return bad(1, "%s: BH and steps must be >= 0", "wildcat_pivot_uniforms");
     if (BH * (int64_t)steps > 0 && !u) return bad(1, "%s: u must be non-null", "wildcat_pivot_uniforms");
     return record(wildcat::launch_pivot_uniforms(seed, BH, steps, u, static_cast<cudaStream_t>(stream)));
+}
+
+wildcat_status wildcat_get_device_status(void* stream) {
+    const cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return record(Status::cuda(e, "wildcat_get_device_status: stream sync"));
+    const int v = wildcat::read_device_status(true);
+    if (v < 0) return record(Status::fail(3, "wildcat_get_device_status: cannot read the status word"));
+    if (v == WILDCAT_ERR_TIMEOUT) return record(Status::fail(5, "a kernel's bounded wait expired"));
+    return record(Status::ok());
+}
+
+wildcat_status wildcat_test_force_wait_timeout(int64_t nanoseconds) {
+    if (nanoseconds < 0 || nanoseconds > 1000000000LL)
+        return bad(1, "%s: nanoseconds must be in [0, 1e9]", "wildcat_test_force_wait_timeout");
+    wildcat::set_attend_force_timeout((unsigned long long)nanoseconds);
+    return record(Status::ok());
 }
 
 wildcat_status wildcat_set_select_cluster(int ctas_per_instance) {

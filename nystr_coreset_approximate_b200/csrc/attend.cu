@@ -191,9 +191,8 @@ Status run_attend(const AttendRequest& q, cudaStream_t st) {
 
 }  // namespace
 
-size_t attend_workspace_bytes(int64_t BH, int64_t m, int d, int r) {
-    (void)d;
-    (void)r;
+// Scratch of the CUDA-core attend: query-norm partials and M_Q.
+size_t attend_simt_workspace_bytes(int64_t BH, int64_t m) {
     const int nsplit = (int)std::max<int64_t>(1, std::min<int64_t>(64, ceil_div(m, 1024)));
     Carve cv(nullptr, 0);
     cv.take(sizeof(float) * BH * nsplit);
@@ -201,7 +200,15 @@ size_t attend_workspace_bytes(int64_t BH, int64_t m, int d, int r) {
     return cv.used + 256;
 }
 
-Status launch_attend(const AttendRequest& q, cudaStream_t st) {
+// Scratch of wildcat_attend: the CUDA-core scratch, then (head dims served by
+// the tensor-core kernel) the bf16 hi/lo copies of [V_S | w]^T.
+size_t attend_workspace_bytes(int64_t BH, int64_t m, int d, int r) {
+    size_t bytes = attend_simt_workspace_bytes(BH, m);
+    if (attend_tc_supported(1, d)) bytes += attend_tc_scratch_bytes(BH, d, r) + 256;
+    return bytes;
+}
+
+Status launch_attend_simt(const AttendRequest& q, cudaStream_t st) {
     const bool bf = q.dtype == 1;
     switch (q.d) {
         case 32: return bf ? run_attend<BF16, 32>(q, st) : run_attend<F32, 32>(q, st);
@@ -209,6 +216,32 @@ Status launch_attend(const AttendRequest& q, cudaStream_t st) {
         case 128: return bf ? run_attend<BF16, 128>(q, st) : run_attend<F32, 128>(q, st);
     }
     return Status::fail(2, "attend: unsupported head dim");
+}
+
+// bf16 inputs with d in {64, 128} run on the tensor cores (attend_tc.cu);
+// everything else on the CUDA-core kernel above.
+Status launch_attend(const AttendRequest& q, cudaStream_t st) {
+    if (!attend_tc_supported(q.dtype, q.d)) return launch_attend_simt(q, st);
+    const int nsplit = (int)std::max<int64_t>(1, std::min<int64_t>(64, ceil_div(q.m, 1024)));
+    const int64_t rows_per_split = ceil_div(q.m, nsplit);
+    Carve cv(q.ws, q.ws_bytes);
+    float* part = static_cast<float*>(cv.take(sizeof(float) * q.BH * nsplit));
+    float* MQ = static_cast<float*>(cv.take(sizeof(float) * q.BH));
+    cv.used = attend_simt_workspace_bytes(q.BH, q.m);
+    void* b2 = cv.take(attend_tc_scratch_bytes(q.BH, q.d, q.r));
+    if (!cv.fits()) return Status::fail(4, "attend: workspace too small");
+    const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(q.Q);
+    const __nv_bfloat16* KS = static_cast<const __nv_bfloat16*>(q.K_S);
+    if (q.d == 64) {
+        qnorm_partial<BF16, 64><<<dim3(nsplit, (unsigned)q.BH), kNormThreads, 0, st>>>(Q, q.m, rows_per_split, part);
+        shift_finalize<BF16, 64><<<(unsigned)q.BH, 256, 0, st>>>(part, nsplit, KS, q.rank, q.r, MQ);
+    } else {
+        qnorm_partial<BF16, 128><<<dim3(nsplit, (unsigned)q.BH), kNormThreads, 0, st>>>(Q, q.m, rows_per_split, part);
+        shift_finalize<BF16, 128><<<(unsigned)q.BH, 256, 0, st>>>(part, nsplit, KS, q.rank, q.r, MQ);
+    }
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return Status::cuda(e, "attend: shift launch");
+    return launch_attend_tc(q, MQ, b2, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -221,7 +254,8 @@ Status launch_attend(const AttendRequest& q, cudaStream_t st) {
 // pool), or they run in a latency-critical loop where a cudaMalloc, which can
 // synchronise the device, is not acceptable.  For them the attend's small
 // scratch (per-instance query-norm partials and the shift M_Q) lives in the
-// fixed device array below instead of a caller workspace.
+// fixed device array below instead of a caller workspace.  It runs the
+// CUDA-core attend kernel, whose scratch is small enough for a fixed array.
 //
 // The array is kNoAllocScratchBytes (1 MiB) and exists on every GPU on which
 // this library's kernels are loaded, until the process exits.  Host code may
@@ -265,7 +299,7 @@ Status attend_scratch_address(void** out) {
 size_t attend_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
 Status launch_attend_noalloc(const AttendRequest& q_in, cudaStream_t st) {
-    if (attend_workspace_bytes(q_in.BH, q_in.m, q_in.d, q_in.r) > kNoAllocScratchBytes)
+    if (attend_simt_workspace_bytes(q_in.BH, q_in.m) > kNoAllocScratchBytes)
         return Status::fail(2,
                             "wildcat_attend_noalloc: BH and m need more scratch than the 1 MiB static array "
                             "(about 4 * BH * (min(64, ceil(m / 1024)) + 1) bytes); use wildcat_attend with a workspace");
@@ -275,7 +309,7 @@ Status launch_attend_noalloc(const AttendRequest& q_in, cudaStream_t st) {
     AttendRequest q = q_in;
     q.ws = scratch;
     q.ws_bytes = kNoAllocScratchBytes;
-    return launch_attend(q, st);
+    return launch_attend_simt(q, st);
 }
 
 }  // namespace wildcat

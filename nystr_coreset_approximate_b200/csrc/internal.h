@@ -25,6 +25,7 @@ struct SelectRequest {
     float beta;
     int r;
     uint64_t seed;
+    int64_t inst0;
     float eps;
     const int32_t* S_fixed;
     int32_t* S;
@@ -56,6 +57,10 @@ struct WeightsRequest {
 };
 size_t weights_workspace_bytes(int64_t BH, int64_t n, int d, int r);
 Status launch_weights(const WeightsRequest& q, cudaStream_t stream);
+// tensor-core F^T (V, 1) partials (weights_tc.cu)
+bool weights_tc_supported(int dtype, int d, int64_t n);
+Status launch_weights_tc(const float* F, const void* V, const int32_t* rank, int64_t BH, int64_t n, int d, int r,
+                         int nsplit, int64_t keys_per_split, float* Ypart, cudaStream_t stream);
 
 // ---- attend ----
 struct AttendRequest {
@@ -75,7 +80,18 @@ struct AttendRequest {
     size_t ws_bytes;
 };
 size_t attend_workspace_bytes(int64_t BH, int64_t m, int d, int r);
+size_t attend_simt_workspace_bytes(int64_t BH, int64_t m);
 Status launch_attend(const AttendRequest& q, cudaStream_t stream);
+Status launch_attend_simt(const AttendRequest& q, cudaStream_t stream);
+// tensor-core attend (attend_tc.cu)
+bool attend_tc_supported(int dtype, int d);
+size_t attend_tc_scratch_bytes(int64_t BH, int d, int r);
+Status launch_attend_tc(const AttendRequest& q, const float* MQ, void* b2_scratch, cudaStream_t stream);
+// device status word set by bounded waits that expired (0 = none); -1 if unreadable
+int read_device_status(bool clear);
+// test hook: the tensor-core attend first waits `ns` nanoseconds on a barrier
+// that nothing completes, then reports a timeout (0 = off)
+void set_attend_force_timeout(unsigned long long ns);
 // attend with its scratch in a static device array (no workspace argument)
 size_t attend_noalloc_scratch_bytes();
 Status launch_attend_noalloc(const AttendRequest& q, cudaStream_t stream);

@@ -34,6 +34,7 @@ namespace {
 
 constexpr int kSelectThreads = 512;
 constexpr int kMaxPL = 16;  // R <= 16384 rows per CTA -> at most 16 values per lane
+constexpr size_t kSmemCap = 227 * 1024;
 
 struct SelectArgs {
     const void* K;
@@ -41,6 +42,7 @@ struct SelectArgs {
     float beta;
     int r;
     uint64_t seed;
+    int64_t inst0;           // global index of instance 0 (Philox counter word 1 = inst0 + b)
     float eps;
     const int32_t* S_fixed;  // nullptr: draw pivots
     int32_t* S;              // may be nullptr in fixed mode
@@ -54,16 +56,20 @@ struct SelectArgs {
 };
 
 struct SmemLayout {
-    size_t ctot, csum, dbuf, ks, fs, red, misc, total;
-    __host__ __device__ SmemLayout(int R, int r, int D, int JG, int NT, int VEC) {
+    size_t ring, kres, inbox, csl, dbuf, dotb, ks, fs, red, misc, total;
+    __host__ __device__ SmemLayout(int Rpad, int r, int D, int JG, int NT, int VEC, int G, int depth,
+                                   size_t kres_bytes) {
         size_t o = 0;
-        ctot = o;  o += 2 * sizeof(double);
-        csum = o;  o += 2 * 32 * sizeof(double);
-        dbuf = o;  o += 2 * (size_t)R * sizeof(float);
+        ring = o;  o += (size_t)depth * NT * 16;               // per-thread cp.async ring, [slot][thread] x 16 B
+        kres = o;  o += round_up(kres_bytes, 16);              // the CTA's key rows, when resident
+        inbox = o; o += 2 * (size_t)G * 33 * sizeof(double);  // [parity][source CTA][32 chunk sums + total]
+        csl = o;   o += 32 * sizeof(double);                   // own chunk sums
+        dbuf = o;  o += 2 * (size_t)Rpad * sizeof(float);      // residual diagonal, double-buffered
+        dotb = o;  o += (size_t)Rpad * sizeof(float);          // <k_l, k_s> of the step
         ks = o;    o += (size_t)D * sizeof(float);
         fs = o;    o += (size_t)round_up(r, 4) * sizeof(float);
         o = round_up(o, 16);
-        red = o;   o += (size_t)(JG > 1 ? JG - 1 : 0) * (NT / JG) * 2 * VEC * sizeof(float);
+        red = o;   o += (size_t)(JG > 1 ? JG - 1 : 0) * (NT / JG) * VEC * sizeof(float);
         misc = o;  o += 16 * sizeof(float);
         total = round_up(o, 16);
     }
@@ -86,31 +92,53 @@ __device__ __forceinline__ double chunk_total(const float* chunk, int PL, int la
     return __shfl_sync(0xffffffffu, warp_scan_incl(s, lane), 31);
 }
 
-template <typename E, int D, int VEC>
+// cp.async helpers (16-byte copies global -> shared, L2 only)
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+template <typename E, int D, int VEC, int DEPTH, bool KRES>
 __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const SelectArgs a) {
     // Launched with a cluster dimension of a.G (one cluster per instance).
     using T = typename E::T;
-    constexpr int NT = kSelectThreads;
+    constexpr int NT = kSelectThreads, NW = NT / 32;
+    constexpr int EPL = 16 / (int)sizeof(T);  // key elements per 16-byte load
+    constexpr int LPR = D / EPL;              // lanes per key row
+    constexpr int RPW = 32 / LPR;             // key rows per warp-wide load
+    constexpr int UF = 8;                     // factor loads in flight per thread (scalar path)
     cg::cluster_group cluster = cg::this_cluster();
     const int crank = (int)cluster.block_rank();
     const int64_t b = blockIdx.x / a.G;
     if (b >= a.BH) return;  // whole clusters only: G divides gridDim.x
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int R = a.R, r = a.r, JG = a.JG, TPG = NT / JG;
+    const int R = a.R, r = a.r, JG = a.JG, TPG = NT / JG, G = a.G;
     const int64_t n = a.n;
     const int64_t row0 = (int64_t)crank * R;
     const int64_t row_end = (row0 + R < n) ? row0 + R : n;
     const int nrows = row_end > row0 ? (int)(row_end - row0) : 0;
-    const int CH = 32 * a.PL;
+    const int PL = a.PL, CH = 32 * PL;
     const int nch = (int)ceil_div(R, CH);
     const int Rpad = nch * CH;  // residual buffers cover whole search chunks
 
     extern __shared__ __align__(16) unsigned char smem[];
-    const SmemLayout L(Rpad, r, D, JG, NT, VEC);
-    double* ctot = reinterpret_cast<double*>(smem + L.ctot);
-    double* csum = reinterpret_cast<double*>(smem + L.csum);
+    const SmemLayout L(Rpad, r, D, JG, NT, VEC, G, DEPTH, KRES ? (size_t)R * D * sizeof(T) : 0);
+    // Each thread streams through its own DEPTH slots of 16 bytes
+    // (slot q of thread t at ring4[q * NT + t]); it only ever reads slots it
+    // filled itself, so the pipeline needs no barrier.  A slot is refilled
+    // two iterations after it was read, keeping DEPTH - 2 copies in flight.
+    float4* ring4 = reinterpret_cast<float4*>(smem + L.ring) + tid;
+    constexpr int INFL = DEPTH - 2;
+    double* inbox = reinterpret_cast<double*>(smem + L.inbox);
+    double* csl = reinterpret_cast<double*>(smem + L.csl);
     float* dbuf = reinterpret_cast<float*>(smem + L.dbuf);
+    float* dotb = reinterpret_cast<float*>(smem + L.dotb);
     float* ks = reinterpret_cast<float*>(smem + L.ks);
     float* fs = reinterpret_cast<float*>(smem + L.fs);
     float* red = reinterpret_cast<float*>(smem + L.red);
@@ -120,58 +148,142 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
 
     const T* Kb = reinterpret_cast<const T*>(a.K) + b * n * D;
     float* Fb = a.F + b * (int64_t)r * n;
+    const int kl_row = lane / LPR, kl_part = lane % LPR;
+
+    // Warp-cooperative pass over the CTA's key rows: out[row] = <k_row, x>
+    // (x = ks) or |k_row|^2 (x = nullptr).  LPR lanes share one row, each
+    // copying 16 contiguous bytes, so a warp reads RPW whole rows per item;
+    // items stream through the thread's cp.async ring.
+    const T* kres = reinterpret_cast<const T*>(smem + L.kres);
+    auto key_pass = [&](const float* x, float* out) {
+        float xr[EPL];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) xr[e] = x ? x[kl_part * EPL + e] : 0.f;
+        if constexpr (KRES) {
+            // key rows resident in shared memory: no global traffic
+            for (int base = warp * RPW; base < nrows; base += NW * RPW) {
+                const int row = base + kl_row;
+                float part = 0.f;
+                if (row < nrows) {
+                    const float4 raw = *reinterpret_cast<const float4*>(kres + (size_t)row * D + kl_part * EPL);
+                    float v[EPL];
+                    if constexpr (sizeof(T) == 2) {
+                        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float2 f = __bfloat1622float2(h[k]);
+                            v[2 * k] = f.x;
+                            v[2 * k + 1] = f.y;
+                        }
+                    } else {
+                        v[0] = raw.x; v[1] = raw.y; v[2] = raw.z; v[3] = raw.w;
+                    }
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) part = fmaf(v[e], x ? xr[e] : v[e], part);
+                }
+#pragma unroll
+                for (int o = LPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+                if (kl_part == 0 && row < nrows) out[row] = part;
+            }
+            return;
+        }
+        const int first = warp * RPW + kl_row;                    // row of item 0 for this lane
+        const int items = nrows > warp * RPW ? (int)ceil_div(nrows - warp * RPW, NW * RPW) : 0;  // warp-uniform
+        const T* src0 = Kb + (row0 + first) * D + kl_part * EPL;
+        const int64_t step = (int64_t)NW * RPW * D;
+#pragma unroll
+        for (int q = 0; q < INFL; ++q) {
+            if (q < items && first + q * NW * RPW < nrows) cp_async16(ring4 + q * NT, src0 + q * step);
+            cp_async_commit();
+        }
+        for (int q = 0; q < items; ++q) {
+            const int qn = q + INFL;
+            if (qn < items && first + qn * NW * RPW < nrows) cp_async16(ring4 + (qn % DEPTH) * NT, src0 + qn * step);
+            cp_async_commit();
+            cp_async_wait<INFL>();
+            const int row = first + q * NW * RPW;
+            float part = 0.f;
+            if (row < nrows) {
+                const float4 raw = ring4[(q % DEPTH) * NT];
+                float v[EPL];
+                if constexpr (sizeof(T) == 2) {
+                    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 f = __bfloat1622float2(h[k]);
+                        v[2 * k] = f.x;
+                        v[2 * k + 1] = f.y;
+                    }
+                } else {
+                    v[0] = raw.x; v[1] = raw.y; v[2] = raw.z; v[3] = raw.w;
+                }
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) part = fmaf(v[e], x ? xr[e] : v[e], part);
+            }
+#pragma unroll
+            for (int o = LPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+            if (kl_part == 0 && row < nrows) out[row] = part;
+        }
+        cp_async_wait<0>();
+    };
+
+    // Chunk sums of a freshly written residual buffer, pushed with the CTA
+    // total into every peer's inbox[par][crank], then the cluster barrier.
+    auto publish = [&](const float* dnew, int par) {
+        for (int k = warp; k < nch; k += NW) {
+            const double t = chunk_total(dnew + (size_t)k * CH, PL, lane);
+            if (lane == 0) csl[k] = t;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            const double v = lane < nch ? csl[lane] : 0.0;
+            double tot = 0.0;
+            for (int k = 0; k < nch; ++k) tot += __shfl_sync(0xffffffffu, v, k);
+            for (int c = 0; c < G; ++c) {
+                double* dst = cluster.map_shared_rank(inbox + ((size_t)par * G + crank) * 33, c);
+                if (lane < nch) dst[lane] = v;
+                if (lane == 0) dst[32] = tot;
+            }
+        }
+        cluster.sync();
+    };
 
     // ---------------- prologue: M_K and the initial residual diagonal ----------------
-    float lmax = -INFINITY;
-    for (int row = tid; row < Rpad; row += NT) {
-        float sq = 0.f;
-        if (row < nrows) {
-            const T* kr = Kb + (row0 + row) * D;
-#pragma unroll
-            for (int c = 0; c < D; c += 8) {
-                float v[8];
-                load8(kr + c, v);
-#pragma unroll
-                for (int k = 0; k < 8; ++k) sq = fmaf(v[k], v[k], sq);
-            }
-            lmax = fmaxf(lmax, sq);
-        }
-        dbuf[row] = sq;  // temporarily |k|^2
+    if constexpr (KRES) {
+        const char* src = reinterpret_cast<const char*>(Kb + row0 * D);
+        char* dst = reinterpret_cast<char*>(smem + L.kres);
+        const int chunks = nrows * D * (int)sizeof(T) / 16;
+        for (int c = tid; c < chunks; c += NT) cp_async16(dst + (size_t)c * 16, src + (size_t)c * 16);
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
     }
+    key_pass(nullptr, dotb);  // |k_l|^2
+    __syncthreads();
+    float lmax = -INFINITY;
+    for (int row = tid; row < nrows; row += NT) lmax = fmaxf(lmax, dotb[row]);
     lmax = warp_max(lmax);
-    __shared__ float wmax[NT / 32];
+    __shared__ float wmax[NW];
     if (lane == 0) wmax[warp] = lmax;
     __syncthreads();
     if (warp == 0) {
-        float v = lane < NT / 32 ? wmax[lane] : -INFINITY;
+        float v = lane < NW ? wmax[lane] : -INFINITY;
         v = warp_max(v);
         if (lane == 0) misc[0] = v;
     }
     cluster.sync();
     if (warp == 0) {
         float v = -INFINITY;
-        if (lane < a.G) v = *cluster.map_shared_rank(&misc[0], lane);
+        if (lane < G) v = *cluster.map_shared_rank(&misc[0], lane);
         v = warp_max(v);
         if (lane == 0) misc[1] = v;
     }
     __syncthreads();
     const float MK = misc[1];
     const float beta = a.beta;
-    for (int row = tid; row < Rpad; row += NT)
-        dbuf[row] = row < nrows ? expf(beta * (dbuf[row] - MK)) : 0.f;
+    for (int row = tid; row < Rpad; row += NT) dbuf[row] = row < nrows ? expf(beta * (dotb[row] - MK)) : 0.f;
     __syncthreads();
-    for (int k = warp; k < nch; k += NT / 32) {
-        const double t = chunk_total(dbuf + (size_t)k * CH, a.PL, lane);
-        if (lane == 0) csum[k] = t;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        double v = lane < nch ? csum[lane] : 0.0;
-        double tot = 0.0;
-        for (int k = 0; k < nch; ++k) tot += __shfl_sync(0xffffffffu, v, k);
-        if (lane == 0) ctot[0] = tot;
-    }
-    cluster.sync();
+    publish(dbuf, 0);
 
     // ---------------- r sequential steps ----------------
     int i = 0;
@@ -179,6 +291,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
         const int cur = i & 1, nxt = cur ^ 1;
         float* dcur = dbuf + (size_t)cur * Rpad;
         float* dnxt = dbuf + (size_t)nxt * Rpad;
+        const double* ib = inbox + (size_t)cur * G * 33;
 
         // -- pivot search (warp 0 of every CTA, identical arithmetic) --
         if (warp == 0) {
@@ -187,15 +300,15 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                 const int sf = a.S_fixed[b * r + i];
                 s = (sf >= 0 && (int64_t)sf < n) ? sf : -1;
             } else {
-                const double tc = lane < a.G ? *cluster.map_shared_rank(&ctot[cur], lane) : 0.0;
+                const double tc = lane < G ? ib[lane * 33 + 32] : 0.0;
                 double T = 0.0;
-                for (int c = 0; c < a.G; ++c) T += __shfl_sync(0xffffffffu, tc, c);
+                for (int c = 0; c < G; ++c) T += __shfl_sync(0xffffffffu, tc, c);
                 if (T > 0.0) {
-                    const double t = pivot_uniform(a.seed, (uint32_t)i, (uint32_t)b) * T;
+                    const double t = pivot_uniform(a.seed, (uint32_t)i, (uint32_t)(a.inst0 + b)) * T;
                     // owner CTA: first whose cumulative total reaches t
                     double cum = 0.0;
                     int owner = -1, lastpos = -1;
-                    for (int c = 0; c < a.G; ++c) {
+                    for (int c = 0; c < G; ++c) {
                         const double v = __shfl_sync(0xffffffffu, tc, c);
                         if (v > 0.0) lastpos = c;
                         if (owner < 0) {
@@ -208,9 +321,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                         cum = 0.0;
                         for (int c = 0; c < owner; ++c) cum += __shfl_sync(0xffffffffu, tc, c);
                     }
-                    // chunk inside the owner
-                    const double* rcs = cluster.map_shared_rank(csum + cur * 32, owner);
-                    const double cv = lane < nch ? rcs[lane] : 0.0;
+                    // owner's chunk reached by t (its chunk sums are in the local inbox)
+                    const double cv = lane < nch ? ib[owner * 33 + lane] : 0.0;
                     int chunk = -1, lastc = -1;
                     double cum2 = cum;
                     for (int k = 0; k < nch; ++k) {
@@ -226,22 +338,22 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                         cum2 = cum;
                         for (int k = 0; k < chunk; ++k) cum2 += __shfl_sync(0xffffffffu, cv, k);
                     }
-                    // row inside the chunk
+                    // row inside the chunk: one read of the owner's residuals
                     const float* rd =
                         cluster.map_shared_rank(dbuf + (size_t)cur * Rpad, owner) + (size_t)chunk * CH;
                     float vals[kMaxPL];
 #pragma unroll
-                    for (int k = 0; k < kMaxPL; ++k) vals[k] = k < a.PL ? rd[lane * a.PL + k] : 0.f;
+                    for (int k = 0; k < kMaxPL; ++k) vals[k] = k < PL ? rd[lane * PL + k] : 0.f;
                     double part = 0.0;
 #pragma unroll
                     for (int k = 0; k < kMaxPL; ++k)
-                        if (k < a.PL) part += (double)vals[k];
+                        if (k < PL) part += (double)vals[k];
                     const double incl = warp_scan_incl(part, lane);
                     double c = cum2 + (incl - part);
                     int hit = -1, lastnz = -1;
 #pragma unroll
                     for (int k = 0; k < kMaxPL; ++k) {
-                        if (k >= a.PL) break;
+                        if (k >= PL) break;
                         const float v = vals[k];
                         if (v > 0.f) lastnz = k;
                         c += (double)v;
@@ -251,11 +363,11 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                     int local;
                     if (hm) {
                         const int src = __ffs(hm) - 1;
-                        local = src * a.PL + __shfl_sync(0xffffffffu, hit, src);
+                        local = src * PL + __shfl_sync(0xffffffffu, hit, src);
                     } else {
                         const unsigned nm = __ballot_sync(0xffffffffu, lastnz >= 0);
                         const int src = 31 - __clz(nm);
-                        local = src * a.PL + __shfl_sync(0xffffffffu, lastnz, src);
+                        local = src * PL + __shfl_sync(0xffffffffu, lastnz, src);
                     }
                     s = (int)((int64_t)owner * R + (int64_t)chunk * CH + local);
                 }
@@ -269,12 +381,12 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
         if (imisc[4]) break;
         const int s = imisc[3];
 
-        // -- pivot key and the pivot's row of the factor --
+        // -- pivot key and the pivot's row of the factor (loads issued together) --
         const T* kp = Kb + (int64_t)s * D;
         for (int c = tid; c < D; c += NT) ks[c] = E::to_float(kp[c]);
         for (int j = tid; j < i; j += NT) fs[j] = ld_cg1(Fb + (int64_t)j * n + s);
         __syncthreads();
-        // -- pivot residual g_s, the same on every CTA --
+        // -- pivot residual g_s (warp 0, the same on every CTA) and <k_l, k_s> --
         if (warp == 0) {
             float dot = 0.f, acc = 0.f;
             for (int c = lane; c < D; c += 32) dot = fmaf(ks[c], ks[c], dot);
@@ -287,6 +399,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                 imisc[4] = !(gs > a.eps);  // max_l h(k_l, k_l) is exp(0) = 1
             }
         }
+        key_pass(ks, dotb);
         __syncthreads();
         if (imisc[4]) break;
         const float gs = misc[2];
@@ -299,74 +412,61 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
             }
         }
 
-        // -- column pass over the CTA's rows --
+        // -- factor pass over the CTA's rows: acc_l = sum_j F[j, l] F[j, s] --
         const int g = tid / TPG, tt = tid % TPG;
         const int jl = (i + JG - 1) / JG, j0 = min(i, g * jl), j1 = min(i, j0 + jl);
-        constexpr int DC = D;  // head-dim split must keep 8-element loads whole
-        const int dl = DC / JG, c0 = g * dl, c1 = c0 + dl;
         for (int base = 0; base < nrows; base += TPG * VEC) {
             const int row = base + tt * VEC;
             const bool valid = row < nrows;
-            float acc[VEC], dp[VEC];
+            float acc[VEC];
 #pragma unroll
-            for (int k = 0; k < VEC; ++k) acc[k] = dp[k] = 0.f;
+            for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
             if (valid) {
                 const float* fcol = Fb + row0 + row;
                 int j = j0;
                 if constexpr (VEC == 4) {
-                    for (; j + 4 <= j1; j += 4) {
-                        float4 v[4];
+                    const int cnt = j1 - j0;
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) v[u] = ld_cg4(fcol + (int64_t)(j + u) * n);
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const float f = fs[j + u];
-                            acc[0] = fmaf(v[u].x, f, acc[0]);
-                            acc[1] = fmaf(v[u].y, f, acc[1]);
-                            acc[2] = fmaf(v[u].z, f, acc[2]);
-                            acc[3] = fmaf(v[u].w, f, acc[3]);
-                        }
+                    for (int q = 0; q < INFL; ++q) {
+                        if (q < cnt) cp_async16(ring4 + q * NT, fcol + (int64_t)(j0 + q) * n);
+                        cp_async_commit();
                     }
-                    for (; j < j1; ++j) {
-                        const float4 v = ld_cg4(fcol + (int64_t)j * n);
-                        const float f = fs[j];
+                    for (int q = 0; q < cnt; ++q) {
+                        const int qn = q + INFL;
+                        if (qn < cnt) cp_async16(ring4 + (qn % DEPTH) * NT, fcol + (int64_t)(j0 + qn) * n);
+                        cp_async_commit();
+                        cp_async_wait<INFL>();
+                        const float4 v = ring4[(q % DEPTH) * NT];
+                        const float f = fs[j0 + q];
                         acc[0] = fmaf(v.x, f, acc[0]);
                         acc[1] = fmaf(v.y, f, acc[1]);
                         acc[2] = fmaf(v.z, f, acc[2]);
                         acc[3] = fmaf(v.w, f, acc[3]);
                     }
+                    cp_async_wait<0>();
                 } else {
-                    for (; j < j1; ++j) acc[0] = fmaf(ld_cg1(fcol + (int64_t)j * n), fs[j], acc[0]);
-                }
+                    for (; j + UF <= j1; j += UF) {
+                        float v[UF];
 #pragma unroll
-                for (int k = 0; k < VEC; ++k) {
-                    const T* kr = Kb + (row0 + row + k) * D;
-                    for (int c = c0; c < c1; c += 8) {
-                        float v[8];
-                        load8(kr + c, v);
+                        for (int u = 0; u < UF; ++u) v[u] = ld_cg1(fcol + (int64_t)(j + u) * n);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) dp[k] = fmaf(v[e], ks[c + e], dp[k]);
+                        for (int u = 0; u < UF; ++u) acc[0] = fmaf(v[u], fs[j + u], acc[0]);
                     }
+                    for (; j < j1; ++j) acc[0] = fmaf(ld_cg1(fcol + (int64_t)j * n), fs[j], acc[0]);
                 }
             }
             if (JG > 1) {
                 if (g > 0) {
-                    float* dst = red + ((size_t)(g - 1) * TPG + tt) * 2 * VEC;
+                    float* dst = red + ((size_t)(g - 1) * TPG + tt) * VEC;
 #pragma unroll
-                    for (int k = 0; k < VEC; ++k) {
-                        dst[k] = acc[k];
-                        dst[VEC + k] = dp[k];
-                    }
+                    for (int k = 0; k < VEC; ++k) dst[k] = acc[k];
                 }
                 __syncthreads();
                 if (g == 0) {
                     for (int h = 0; h < JG - 1; ++h) {
-                        const float* src = red + ((size_t)h * TPG + tt) * 2 * VEC;
+                        const float* src = red + ((size_t)h * TPG + tt) * VEC;
 #pragma unroll
-                        for (int k = 0; k < VEC; ++k) {
-                            acc[k] += src[k];
-                            dp[k] += src[VEC + k];
-                        }
+                        for (int k = 0; k < VEC; ++k) acc[k] += src[k];
                     }
                 }
             }
@@ -375,7 +475,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
 #pragma unroll
                 for (int k = 0; k < VEC; ++k) {
                     const int64_t l = row0 + row + k;
-                    float gl = expf(beta * (dp[k] - MK)) - acc[k];
+                    float gl = expf(beta * (dotb[row + k] - MK)) - acc[k];
                     if (l == s) gl = gs;
                     const float f = gl / piv;
                     out[k] = f;
@@ -395,19 +495,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
         // rows of the slice past n keep zero mass
         for (int row = nrows + tid; row < Rpad; row += NT) dnxt[row] = 0.f;
         __syncthreads();
-        // -- chunk sums of the new residual diagonal --
-        for (int k = warp; k < nch; k += NT / 32) {
-            const double t = chunk_total(dnxt + (size_t)k * CH, a.PL, lane);
-            if (lane == 0) csum[nxt * 32 + k] = t;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            const double v = lane < nch ? csum[nxt * 32 + lane] : 0.0;
-            double tot = 0.0;
-            for (int k = 0; k < nch; ++k) tot += __shfl_sync(0xffffffffu, v, k);
-            if (lane == 0) ctot[nxt] = tot;
-        }
-        cluster.sync();
+        publish(dnxt, nxt);
     }
 
     // ---------------- effective rank, padding past it ----------------
@@ -437,9 +525,9 @@ __global__ void pivot_uniform_kernel(uint64_t seed, int64_t BH, int steps, doubl
     u[t] = pivot_uniform(seed, (uint32_t)i, (uint32_t)b);
 }
 
-template <typename E, int D, int VEC>
+template <typename E, int D, int VEC, int DEPTH, bool KRES>
 cudaError_t launch_select_t(const SelectArgs& a, size_t smem, cudaStream_t stream) {
-    auto kern = rpc_select_kernel<E, D, VEC>;
+    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KRES>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (a.G > 8) {
@@ -461,9 +549,9 @@ cudaError_t launch_select_t(const SelectArgs& a, size_t smem, cudaStream_t strea
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <typename E, int D, int VEC>
+template <typename E, int D, int VEC, int DEPTH, bool KRES>
 int max_clusters_t(int G, size_t smem) {
-    auto kern = rpc_select_kernel<E, D, VEC>;
+    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KRES>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return 0;
     if (G > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
@@ -487,31 +575,47 @@ int max_clusters_t(int G, size_t smem) {
     return nc;
 }
 
-template <typename E, int VEC>
+template <typename E, int VEC, int DEPTH, bool KRES>
 int dispatch_d(int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int G_query, cudaError_t* err) {
     switch (d) {
         case 32:
-            if (a) { *err = launch_select_t<E, 32, VEC>(*a, smem, stream); return 0; }
-            return max_clusters_t<E, 32, VEC>(G_query, smem);
+            if (a) { *err = launch_select_t<E, 32, VEC, DEPTH, KRES>(*a, smem, stream); return 0; }
+            return max_clusters_t<E, 32, VEC, DEPTH, KRES>(G_query, smem);
         case 64:
-            if (a) { *err = launch_select_t<E, 64, VEC>(*a, smem, stream); return 0; }
-            return max_clusters_t<E, 64, VEC>(G_query, smem);
+            if (a) { *err = launch_select_t<E, 64, VEC, DEPTH, KRES>(*a, smem, stream); return 0; }
+            return max_clusters_t<E, 64, VEC, DEPTH, KRES>(G_query, smem);
         case 128:
-            if (a) { *err = launch_select_t<E, 128, VEC>(*a, smem, stream); return 0; }
-            return max_clusters_t<E, 128, VEC>(G_query, smem);
+            if (a) { *err = launch_select_t<E, 128, VEC, DEPTH, KRES>(*a, smem, stream); return 0; }
+            return max_clusters_t<E, 128, VEC, DEPTH, KRES>(G_query, smem);
     }
     if (err) *err = cudaErrorInvalidValue;
     return 0;
 }
 
-int dispatch(int dtype, int vec, int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int G_query,
-             cudaError_t* err) {
-    if (dtype == 1) {
-        return vec == 4 ? dispatch_d<BF16, 4>(d, a, smem, stream, G_query, err)
-                        : dispatch_d<BF16, 1>(d, a, smem, stream, G_query, err);
+// Kernel variants: the vectorised path with ring depth 24/16/12/6 (12 also
+// with resident keys); the scalar path (n not a multiple of 4) with depth 6.
+struct Variant {
+    int depth;
+    bool kres;
+};
+
+template <typename E>
+int dispatch_e(const Variant& v, int vec, int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int G_query,
+               cudaError_t* err) {
+    if (vec != 4) return dispatch_d<E, 1, 6, false>(d, a, smem, stream, G_query, err);
+    if (v.kres) return dispatch_d<E, 4, 12, true>(d, a, smem, stream, G_query, err);
+    switch (v.depth) {
+        case 24: return dispatch_d<E, 4, 24, false>(d, a, smem, stream, G_query, err);
+        case 16: return dispatch_d<E, 4, 16, false>(d, a, smem, stream, G_query, err);
+        case 12: return dispatch_d<E, 4, 12, false>(d, a, smem, stream, G_query, err);
     }
-    return vec == 4 ? dispatch_d<F32, 4>(d, a, smem, stream, G_query, err)
-                    : dispatch_d<F32, 1>(d, a, smem, stream, G_query, err);
+    return dispatch_d<E, 4, 6, false>(d, a, smem, stream, G_query, err);
+}
+
+int dispatch(const Variant& v, int dtype, int vec, int d, const SelectArgs* a, size_t smem, cudaStream_t stream,
+             int G_query, cudaError_t* err) {
+    return dtype == 1 ? dispatch_e<BF16>(v, vec, d, a, smem, stream, G_query, err)
+                      : dispatch_e<F32>(v, vec, d, a, smem, stream, G_query, err);
 }
 
 int g_cluster_override = 0;
@@ -528,18 +632,33 @@ int select_cluster_override(int G) {
 }
 int last_select_cluster() { return g_last_cluster; }
 
-static void plan(int64_t n, int d, int r, int G, int vec, SelectArgs* a, size_t* smem) {
+static void plan(int64_t n, int r, int d, int dtype, int G, int vec, SelectArgs* a, size_t* smem, Variant* v) {
     const int R = (int)round_up(ceil_div(n, G), 4);
     int JG = 1;
-    const int maxJG = min(8, d / 8);
-    while (JG * 2 <= maxJG && (int64_t)(kSelectThreads / (JG * 2)) * vec >= R) JG *= 2;
+    while (JG * 2 <= 8 && (int64_t)(kSelectThreads / (JG * 2)) * vec >= R) JG *= 2;
     const int PL = (int)std::max<int64_t>(4, round_up(ceil_div(ceil_div(R, 32), 32), 4));
     const int Rpad = (int)round_up(R, 32 * PL);
     a->G = G;
     a->R = R;
     a->JG = JG;
     a->PL = PL;
-    *smem = SmemLayout(Rpad, r, d, JG, kSelectThreads, vec).total;
+    auto bytes = [&](int depth, bool kres) {
+        const size_t kb = kres ? (size_t)R * d * (dtype == 1 ? 2 : 4) : 0;
+        return SmemLayout(Rpad, r, d, JG, kSelectThreads, vec, G, depth, kb).total;
+    };
+    if (vec != 4) {
+        *v = {6, false};
+    } else if (bytes(12, true) <= kSmemCap) {
+        *v = {12, true};  // keys stay in shared memory: the per-step key pass reads no global memory
+    } else {
+        *v = {6, false};
+        for (int depth : {24, 16, 12})
+            if (bytes(depth, false) <= kSmemCap) {
+                *v = {depth, false};
+                break;
+            }
+    }
+    *smem = bytes(v->depth, v->kres);
 }
 
 Status launch_select(const SelectRequest& q, cudaStream_t stream) {
@@ -553,6 +672,7 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     a.beta = q.beta;
     a.r = q.r;
     a.seed = q.seed;
+    a.inst0 = q.inst0;
     a.eps = q.eps;
     a.S_fixed = q.S_fixed;
     a.S = q.S;
@@ -570,21 +690,21 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     while (G < 16 && ceil_div(q.n, G) > kMaxRowsPerCta) G *= 2;
     if (ceil_div(q.n, G) > kMaxRowsPerCta)
         return Status::fail(2, "select: n / 16 exceeds the per-CTA row limit (16384)");
+    size_t smem = 0;
+    Variant var{};
     if (g_cluster_override <= 0) {
         // shrink until the cluster shape is schedulable
         for (;;) {
-            size_t smem;
-            plan(q.n, q.d, q.r, G, vec, &a, &smem);
-            if (smem > 227 * 1024) return Status::fail(2, "select: shared memory plan exceeds 227 KB");
-            if (dispatch(q.dtype, vec, q.d, nullptr, smem, stream, G, nullptr) > 0 || G == 1) break;
+            plan(q.n, q.r, q.d, q.dtype, G, vec, &a, &smem, &var);
+            if (smem > kSmemCap) return Status::fail(2, "select: shared memory plan exceeds 227 KB");
+            if (dispatch(var, q.dtype, vec, q.d, nullptr, smem, stream, G, nullptr) > 0 || G == 1) break;
             G /= 2;
         }
     }
-    size_t smem;
-    plan(q.n, q.d, q.r, G, vec, &a, &smem);
-    if (smem > 227 * 1024) return Status::fail(2, "select: shared memory plan exceeds 227 KB");
+    plan(q.n, q.r, q.d, q.dtype, G, vec, &a, &smem, &var);
+    if (smem > kSmemCap) return Status::fail(2, "select: shared memory plan exceeds 227 KB");
     cudaError_t err = cudaSuccess;
-    dispatch(q.dtype, vec, q.d, &a, smem, stream, G, &err);
+    dispatch(var, q.dtype, vec, q.d, &a, smem, stream, G, &err);
     if (err == cudaSuccess) err = cudaGetLastError();
     if (err != cudaSuccess) return Status::cuda(err, "select launch");
     g_last_cluster = G;

@@ -1,0 +1,134 @@
+// tc_common.cuh -- tcgen05 / TMEM / mbarrier / cp.async helpers (sm_100a).
+//
+// Shared-memory operands use the UMMA K-major (or MN-major) layout with
+// 128-byte swizzling: rows of 128 bytes grouped in 8-row atoms of 1024
+// bytes, 16-byte chunk c of row r stored at chunk c ^ (r % 8).
+#pragma once
+
+#include <stdint.h>
+
+namespace wildcat {
+namespace tc {
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per bounded wait
+
+__device__ __forceinline__ unsigned smem_u32(const void* p) { return (unsigned)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Byte offset of 16-byte chunk c8 (0..7) of row `row` inside a K-major,
+// 128-byte-swizzled block whose rows are 128 bytes (64 bf16) long.
+__device__ __forceinline__ unsigned swz(int row, int c8) {
+    return (unsigned)((row >> 3) * 1024 + (row & 7) * 128 + ((c8 ^ (row & 7)) << 4));
+}
+
+// UMMA shared-memory descriptor: K-major, SWIZZLE_128B, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t umma_desc(unsigned saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);        // start address
+    d |= (uint64_t)1u << 16;                         // leading byte offset (unused with swizzle)
+    d |= (uint64_t)(1024u >> 4) << 32;               // stride byte offset: next 8-row group
+    d |= (uint64_t)1u << 46;                         // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                         // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4)                    // D format fp32
+           | (1u << 7)                  // A format bf16
+           | (1u << 10)                 // B format bf16
+           | ((uint32_t)(N >> 3) << 17)  // N / 8
+           | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+__device__ __forceinline__ void mma_bf16(unsigned tmem_d, uint64_t a, uint64_t b, uint32_t idesc, int accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(void* mbar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(mbar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_init(void* mbar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(mbar)), "r"(count) : "memory");
+}
+
+// Bounded wait for the phase with the given parity; returns false on timeout.
+__device__ __forceinline__ bool mbar_wait(void* mbar, unsigned parity,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
+    const unsigned a = smem_u32(mbar);
+    const unsigned long long t0 = globaltimer();
+    for (;;) {
+        unsigned done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+        if (globaltimer() - t0 > limit_ns) return false;
+    }
+}
+
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld16(unsigned taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
+}
+
+__device__ __forceinline__ void cp_async16_zfill(unsigned dst, const void* src, bool ok) {
+    const int n = ok ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+
+}  // namespace tc
+}  // namespace wildcat
+
+namespace wildcat {
+namespace tc {
+
+// UMMA shared-memory descriptor for an MN-major, SWIZZLE_128B operand: each
+// row of 128 bytes holds 64 consecutive MN elements of one K index; 8-row K
+// groups are 1024 bytes apart and 64-element MN blocks `mn_block_bytes` apart.
+__device__ __forceinline__ uint64_t umma_desc_mn(unsigned saddr, unsigned mn_block_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);             // start address
+    d |= (uint64_t)((mn_block_bytes >> 4) & 0x3FFFu) << 16;  // leading byte offset: next MN block
+    d |= (uint64_t)(1024u >> 4) << 32;                    // stride byte offset: next 8-row K group
+    d |= (uint64_t)1u << 46;                              // descriptor version (sm_100)
+    d |= (uint64_t)2u << 61;                              // SWIZZLE_128B
+    return d;
+}
+
+// bf16 x bf16 -> fp32 with A K-major and B MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_bmn(int M, int N) { return idesc_bf16(M, N) | (1u << 16); }
+
+}  // namespace tc
+}  // namespace wildcat

@@ -10,7 +10,9 @@
 //
 // Kernels:
 //   colrange_*   column-wise [v_min, v_max] of V (value-range clip bounds)
-//   fty_kernel   Y partials: F^T (V, 1) over a slice of the keys (split-K)
+//   fty_kernel   Y partials: F^T (V, 1) over a slice of the keys (split-K),
+//                CUDA cores (float32 values, or n % 4 != 0); bf16 values use the
+//                tensor-core kernel of weights_tc.cu
 //   gather_fs    F_S[a, j] = F[j, S_a] for j <= a (pivot rows of the factor)
 //   trsm_kernel  sums the split-K partials and back-substitutes F_S^T X = Y
 #include <algorithm>
@@ -78,12 +80,13 @@ constexpr int kFtyNK = 32;  // keys per smem stage
 template <typename E, int D>
 __global__ void __launch_bounds__(kFtyThreads) fty_kernel(const float* F, const typename E::T* V, int64_t n,
                                                           int r, int64_t keys_per_split, float* Ypart,
-                                                          int64_t BH) {
-    // Ypart [nsplit, BH, r, D + 1]
+                                                          int64_t BH, const int32_t* rank) {
+    // Ypart [nsplit, BH, r, D + 1]; rows at or past the instance's rank are
+    // never read by the solve, so tiles that start there do no work.
     const int jt = blockIdx.x, split = blockIdx.y;
     const int64_t b = blockIdx.z;
-    const int nsplit = gridDim.y;
     const int j0 = jt * kFtyTJ;
+    if (j0 >= rank[b]) return;
     const int64_t l0 = split * keys_per_split, l1 = min(n, l0 + keys_per_split);
     constexpr int TPR = kFtyThreads / kFtyTJ;  // threads per factor column
     constexpr int CPT = D / TPR;               // value columns per thread
@@ -128,15 +131,15 @@ __global__ void __launch_bounds__(kFtyThreads) fty_kernel(const float* F, const 
     }
 }
 
-// F_S[b, a, j] = F[b, j, S[b, a]] for j <= a < rank; zero elsewhere.
+// F_S[b, a, j] = F[b, j, S[b, a]] for j <= a < rank (the solve reads nothing else).
 __global__ void gather_fs(const float* F, const int32_t* S, const int32_t* rank, int64_t n, int r, float* FS) {
     const int64_t b = blockIdx.y;
     const int a = blockIdx.x;
     const int rr = rank[b];
+    if (a >= rr) return;  // the solve reads rows below the rank only
     float* dst = FS + (b * r + a) * (int64_t)r;
-    const int s = a < rr ? S[b * r + a] : -1;
-    for (int j = threadIdx.x; j < r; j += blockDim.x)
-        dst[j] = (s >= 0 && j <= a) ? __ldcg(F + (b * r + j) * n + s) : 0.f;
+    const int s = S[b * r + a];
+    for (int j = threadIdx.x; j <= a; j += blockDim.x) dst[j] = __ldcg(F + (b * r + j) * n + s);
 }
 
 // Back substitution F_S^T X = Y for one instance and one block of CB right-hand columns.
@@ -184,8 +187,11 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* Ypart, 
 struct WeightsPlan {
     int nsplit_range;
     int64_t rows_per_range;
-    int nsplit_k;
+    int nsplit_k;            // split-K of the CUDA-core F^T (V, 1)
     int64_t keys_per_split;
+    int nsplit_tc;           // split-K of the tensor-core F^T (V, 1)
+    int64_t keys_per_split_tc;
+    int max_split() const { return nsplit_k > nsplit_tc ? nsplit_k : nsplit_tc; }
 };
 
 WeightsPlan make_plan(int64_t BH, int64_t n, int r) {
@@ -199,6 +205,13 @@ WeightsPlan make_plan(int64_t BH, int64_t n, int r) {
     sk = std::min<int64_t>(sk, 64);
     p.keys_per_split = round_up(ceil_div(n, sk), kFtyNK);
     p.nsplit_k = (int)ceil_div(n, p.keys_per_split);
+    // tensor-core tiles cover 128 factor columns; aim at ~4 CTAs per SM
+    const int64_t tiles_tc = ceil_div(r, 128) * BH;
+    int64_t st = ceil_div(4 * 148, tiles_tc);
+    st = std::max<int64_t>(1, std::min<int64_t>(st, std::max<int64_t>(1, n / 512)));
+    st = std::min<int64_t>(st, 128);
+    p.keys_per_split_tc = round_up(ceil_div(n, st), 64);
+    p.nsplit_tc = (int)ceil_div(n, p.keys_per_split_tc);
     return p;
 }
 
@@ -207,7 +220,7 @@ Status run_weights(const WeightsRequest& q, cudaStream_t st) {
     const WeightsPlan p = make_plan(q.BH, q.n, q.r);
     Carve cv(q.ws, q.ws_bytes);
     float* part = static_cast<float*>(cv.take(sizeof(float) * q.BH * p.nsplit_range * 2 * D));
-    float* Ypart = static_cast<float*>(cv.take(sizeof(float) * p.nsplit_k * q.BH * (int64_t)q.r * (D + 1)));
+    float* Ypart = static_cast<float*>(cv.take(sizeof(float) * p.max_split() * q.BH * (int64_t)q.r * (D + 1)));
     float* FS = static_cast<float*>(cv.take(sizeof(float) * q.BH * (int64_t)q.r * q.r));
     if (!cv.fits()) return Status::fail(4, "weights: workspace too small");
     using T = typename E::T;
@@ -217,14 +230,22 @@ Status run_weights(const WeightsRequest& q, cudaStream_t st) {
                                                                                            part);
     colrange_finalize<<<(unsigned)ceil_div(q.BH * D, 256), 256, 0, st>>>(part, p.nsplit_range, D, q.BH, q.vmin,
                                                                           q.vmax);
-    fty_kernel<E, D><<<dim3((unsigned)ceil_div(q.r, kFtyTJ), p.nsplit_k, (unsigned)q.BH), kFtyThreads, 0, st>>>(
-        q.F, V, q.n, q.r, p.keys_per_split, Ypart, q.BH);
+    int nsplit = p.nsplit_k;
+    if (weights_tc_supported(q.dtype, D, q.n)) {
+        nsplit = p.nsplit_tc;
+        const Status s = launch_weights_tc(q.F, q.V, q.rank, q.BH, q.n, D, q.r, p.nsplit_tc, p.keys_per_split_tc, Ypart,
+                                           st);
+        if (s.code) return s;
+    } else {
+        fty_kernel<E, D><<<dim3((unsigned)ceil_div(q.r, kFtyTJ), p.nsplit_k, (unsigned)q.BH), kFtyThreads, 0, st>>>(
+            q.F, V, q.n, q.r, p.keys_per_split, Ypart, q.BH, q.rank);
+    }
     gather_fs<<<dim3(q.r, (unsigned)q.BH), 128, 0, st>>>(q.F, q.S, q.rank, q.n, q.r, FS);
     const size_t smem = sizeof(float) * (size_t)q.r * kTrsmCB;
     cudaError_t e = cudaFuncSetAttribute(trsm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return Status::cuda(e, "weights: trsm smem attribute");
     trsm_kernel<<<dim3((unsigned)ceil_div(D + 1, kTrsmCB), (unsigned)q.BH), kTrsmThreads, smem, st>>>(
-        Ypart, p.nsplit_k, FS, q.rank, q.BH, q.r, D, q.V_S, q.w);
+        Ypart, nsplit, FS, q.rank, q.BH, q.r, D, q.V_S, q.w);
     e = cudaGetLastError();
     if (e != cudaSuccess) return Status::cuda(e, "weights launch");
     return Status::ok();
@@ -236,7 +257,7 @@ size_t weights_workspace_bytes(int64_t BH, int64_t n, int d, int r) {
     const WeightsPlan p = make_plan(BH, n, r);
     Carve cv(nullptr, 0);
     cv.take(sizeof(float) * BH * p.nsplit_range * 2 * d);
-    cv.take(sizeof(float) * p.nsplit_k * BH * (int64_t)r * (d + 1));
+    cv.take(sizeof(float) * p.max_split() * BH * (int64_t)r * (d + 1));
     cv.take(sizeof(float) * BH * (int64_t)r * r);
     return cv.used + 256;
 }

@@ -31,11 +31,11 @@ def test_status_strings_and_version(L):
 
 
 def _select(L, **kw):
-    a = dict(K=FAKE, dtype=1, BH=2, n=100, d=64, beta=0.125, r=10, seed=0, eps=1e-6, S=FAKE, F=FAKE,
-             rank=FAKE, K_S=None, stream=None)
+    a = dict(K=FAKE, dtype=1, BH=2, n=100, d=64, beta=0.125, r=10, seed=0, inst0=0, eps=1e-6, S=FAKE,
+             F=FAKE, rank=FAKE, K_S=None, stream=None)
     a.update(kw)
     return L.wildcat_select(a["K"], a["dtype"], a["BH"], a["n"], a["d"], a["beta"], a["r"], a["seed"],
-                            a["eps"], a["S"], a["F"], a["rank"], a["K_S"], a["stream"])
+                            a["inst0"], a["eps"], a["S"], a["F"], a["rank"], a["K_S"], a["stream"])
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -54,6 +54,8 @@ def _select(L, **kw):
     (dict(S=None), 1),
     (dict(K=ctypes.c_void_p((1 << 20) + 4)), 1),  # misaligned
     (dict(r=9000, n=10000), 2),
+    (dict(inst0=-1), 1),
+    (dict(inst0=2**32 - 1), 1),
 ])
 def test_select_rejects_on_host(L, kw, code):
     assert _select(L, **kw) == code
@@ -86,7 +88,7 @@ def test_forward_workspace_accounts_for_the_factor(L):
     assert ws < 4 * BH * r * n * 2
     wh = int(L.wildcat_forward_host_workspace_size(BH, m, n, d, r, 1))
     assert wh >= ws + 2 * BH * (m + 2 * n) * d + 4 * BH * m * d
-    assert L.wildcat_forward(FAKE, FAKE, FAKE, 1, BH, m, n, d, 0.125, r, 0, 1e-6, FAKE, None,
+    assert L.wildcat_forward(FAKE, FAKE, FAKE, 1, BH, m, n, d, 0.125, r, 0, 0, 1e-6, FAKE, None,
                              None, ctypes.c_void_p(1 << 20), ws - 4096, None) == 4
 
 

@@ -44,7 +44,10 @@ def test_noalloc_matches_attend_on_two_calls():
         vmin, vmax = args[6].cpu().numpy(), args[7].cpu().numpy()
         span = np.maximum(vmax - vmin, 1e-30)[:, None, :]
         err = np.max(np.abs(O_na.cpu().numpy() - O_ref.cpu().numpy()) / span)
-        assert err <= 1e-4, (w.dtype, err)
+        # the parity tolerance of the tests: 1e-4 of the value range for float32
+        # inputs, 2e-2 for bfloat16 (wildcat_attend runs bf16 on the tensor
+        # cores; the no-alloc variant runs the CUDA-core kernel)
+        assert err <= (1e-4 if w.dtype == "f32" else 2e-2), (w.dtype, err)
 
 
 def test_noalloc_rejects_sizes_beyond_the_static_scratch():
