@@ -59,6 +59,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--nbins", type=int, default=1,
+                   help="divide-and-conquer bins (1 = the unbinned method)")
     return p.parse_args()
 
 
@@ -245,7 +247,11 @@ def main():
     w = w0.scaled(seed=w0.seed + 1000 * rank)  # each rank its own batch of instances
     dev, ex = workloads.make(w)
     Q, K, V = (dev[k].cuda() for k in ("Q", "K", "V"))
-    plan = wc.ForwardPlan(w.BH, w.m, w.n, w.d, w.r, w.dtype)
+    nb = max(1, args.nbins)
+    if nb > 1:
+        plan = wc.BinnedForwardPlan(w.BH, w.m, w.n, w.d, w.r, nb, w.dtype)
+    else:
+        plan = wc.ForwardPlan(w.BH, w.m, w.n, w.d, w.r, w.dtype)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
     def barrier():
@@ -257,7 +263,7 @@ def main():
     for _ in range(max(args.warmup, 3)):
         plan.run(Q, K, V, w.beta, w.pivot_seed, EPS)
     torch.cuda.synchronize()
-    ranks = plan.rank.cpu().tolist()
+    ranks = plan.rank.reshape(-1).cpu().tolist()  # per instance (per bin when binned)
 
     # ---- timed forward: K steps, own events per step, L2 flushed in between ----
     clocks = ClockSampler(local)
@@ -275,29 +281,37 @@ def main():
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = sharding.max_over_ranks(sum(step_ms), device="cuda")
 
-    # ---- per-stage breakdown through the staged C-ABI calls (same kernels) ----
+    # ---- per-stage breakdown through the staged C-ABI calls (same kernels;
+    #      binned: the same calls on the [BH * nbins, n / nbins] view) ----
+    Kv = K.view(w.BH * nb, w.n // nb, w.d)
+    Vv = V.view(w.BH * nb, w.n // nb, w.d)
+    rv = w.r // nb
     stage_ms = {"select": [], "weights": [], "attend": []}
     for k in range(args.steps + 2):
         flush.zero_()
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         ev[0].record()
-        S, F, rk, K_S = wc.select(K, w.beta, w.r, w.pivot_seed, EPS)
+        S, F, rk, K_S = wc.select(Kv, w.beta, rv, w.pivot_seed, EPS)
         ev[1].record()
-        V_S, wv, vmin, vmax = wc.weights(F, S, rk, V)
+        V_S, wv, vmin, vmax = wc.weights(F, S, rk, Vv)
         ev[2].record()
-        wc.attend(Q, K_S, rk, w.beta, V_S, wv, vmin, vmax)
+        if nb == 1:
+            wc.attend(Q, K_S, rk, w.beta, V_S, wv, vmin, vmax)
         ev[3].record()
         torch.cuda.synchronize()
         if k >= 2:
             stage_ms["select"].append(ev[0].elapsed_time(ev[1]))
             stage_ms["weights"].append(ev[1].elapsed_time(ev[2]))
-            stage_ms["attend"].append(ev[2].elapsed_time(ev[3]))
+            if nb == 1:
+                stage_ms["attend"].append(ev[2].elapsed_time(ev[3]))
     del S, F, rk, K_S, V_S, wv, vmin, vmax
+    if not stage_ms["attend"]:
+        del stage_ms["attend"]
     sel_ms = statistics.mean(stage_ms["select"])
 
     # ---- end to end through wildcat_forward_host (host buffers) ----
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and nb == 1:
         hp = wc.HostForwardPlan(w.BH, w.m, w.n, w.d, w.r, w.dtype)
         pinned = {k: v.pin_memory() for k, v in dev.items()}
         O_host = torch.empty((w.BH, w.m, w.d), dtype=torch.float32).pin_memory()
@@ -337,23 +351,24 @@ def main():
 
     value = world * args.steps / (total_ms / 1e3)
     peak, peak_kind = read_peaks()
-    nbytes = select_bytes(w, ranks)
+    nbytes = select_bytes(w.scaled(n=w.n // nb), ranks)
     achieved = nbytes / (sel_ms / 1e3) / 1e9
-    traffic = recorded_traffic(w0.name)
+    traffic = recorded_traffic(w0.name if nb == 1 else f"{w0.name}_bins{nb}")
     out = {
         "metric": METRIC, "value": value, "unit": "calls/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
         "config": workload_config(w0, {"l2": "flushed between steps (256 MiB device write)",
-                                       "parallelism": f"instances per rank x {world} ranks"}),
+                                       "parallelism": f"instances per rank x {world} ranks",
+                                       "nbins": nb}),
         "entries_per_s": value * w.BH * w.m * w.n,
         "stages_ms": {k: statistics.mean(v) for k, v in stage_ms.items()},
         "roofline": {"kernel": "rpc_select_kernel", "bound": "hbm", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} hbm_gbs", "traffic": traffic,
                      "algorithmic_bytes_per_launch": nbytes, "launch_ms": sel_ms},
-        "gpu_launches": launches_per_forward(w) * args.steps,
+        "gpu_launches": (launches_per_forward(w) + (1 if nb > 1 else 0)) * args.steps,
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cpu,

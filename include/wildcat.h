@@ -165,6 +165,28 @@ wildcat_status wildcat_attend(const void* Q, const void* K_S, int dtype, int64_t
                               void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * wildcat_decode_attend -- KV-cache decode with new tokens (Sec. 2: after
+ * CompressKV, m new tokens cost O(rmd + m^2 d)).  New query i attends over
+ * the compressed cache (K_S, V_S, w from select/weights) and, exactly, over
+ * the new tokens j <= i (causal):
+ *   N_i = sum_l u_il V_S[l] + sum_{j<=i} e_ij V_new[j],  D_i = sum_l u_il w_l + sum_{j<=i} e_ij,
+ *   u_il = exp(beta <q_i, k_S_l> - beta M), e_ij = exp(beta <q_i, k_new_j> - beta M),
+ *   M = max_i |q_i| * max(max_l |k_S_l|, max_j |k_new_j|) per instance,
+ *   O_i = clip(N_i / D_i) to the range of the cache (vmin, vmax) and V_new.
+ *
+ *   Q_new, K_new, V_new  [BH, m, d] new tokens, dtype `dtype`
+ *   K_S, rank, V_S, w, vmin, vmax   the compressed cache
+ *   O      out [BH, m, d] float32
+ *   workspace >= wildcat_decode_attend_workspace_size(BH, d) bytes
+ */
+size_t wildcat_decode_attend_workspace_size(int64_t BH, int d);
+wildcat_status wildcat_decode_attend(const void* Q_new, const void* K_new, const void* V_new,
+                                     const void* K_S, int dtype, int64_t BH, int64_t m, int d, int r,
+                                     const int32_t* rank, float beta, const float* V_S,
+                                     const float* w, const float* vmin, const float* vmax,
+                                     float* O, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * wildcat_attend_noalloc -- wildcat_attend for callers that cannot allocate
  * device memory.  The paper has no counterpart; this is a deployment
  * convenience.  Such callers only hold pointers handed to them by another
@@ -208,6 +230,29 @@ wildcat_status wildcat_forward(const void* Q, const void* K, const void* V, int 
                                int64_t m, int64_t n, int d, float beta, int r, uint64_t seed,
                                int64_t inst0, float eps, float* O, int32_t* S_out,
                                int32_t* rank_out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * wildcat_forward_binned -- the module with divide-and-conquer binning
+ * (Sec. 2: B bins, r / B pivots each, selected in parallel).  The n keys of
+ * every instance are cut into nbins contiguous bins of n / nbins keys; bin q
+ * gets its own RPCholesky coreset of r / nbins pivots (pivot draws use the
+ * instance index (inst0 + b) * nbins + q) and its own Nystrom weights over
+ * its own keys (block-diagonal W).  The output attends over the union of the
+ * bins' coresets; the value range is over all n keys.  n and r must be
+ * multiples of nbins; nbins = 1 is wildcat_forward.
+ *
+ *   S_out    [BH, r] int32 global key index of every union row, -1 past a
+ *            bin's rank (or NULL); row q * (r / nbins) + a is bin q's a-th pivot
+ *   rank_out [BH, nbins] int32 effective rank of every bin (or NULL)
+ *   workspace >= wildcat_forward_binned_workspace_size(...) bytes
+ */
+size_t wildcat_forward_binned_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r,
+                                             int nbins, int dtype);
+wildcat_status wildcat_forward_binned(const void* Q, const void* K, const void* V, int dtype,
+                                      int64_t BH, int64_t m, int64_t n, int d, float beta, int r,
+                                      int nbins, uint64_t seed, int64_t inst0, float eps, float* O,
+                                      int32_t* S_out, int32_t* rank_out, void* workspace,
+                                      size_t ws_bytes, void* stream);
 
 /*
  * wildcat_forward_host -- wildcat_forward on HOST buffers: copies Q, K, V

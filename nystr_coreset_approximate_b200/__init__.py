@@ -24,7 +24,7 @@ from typing import Optional
 
 __all__ = [
     "WildcatError", "library_path", "lib", "declared_symbols", "select", "select_fixed",
-    "weights", "attend", "attend_noalloc", "forward", "forward_host", "ForwardPlan", "pivot_uniforms",
+    "weights", "attend", "attend_noalloc", "decode_attend", "forward", "forward_binned", "BinnedForwardPlan", "forward_host", "ForwardPlan", "pivot_uniforms",
     "set_select_cluster", "last_select_cluster", "device_status", "DTYPES",
 ]
 
@@ -56,9 +56,15 @@ _SIGS = {
                         _sz, _vp], _int),
     "wildcat_attend_noalloc": ([_vp, _vp, _int, _i64, _i64, _int, _int, _vp, _f32, _vp, _vp, _vp, _vp,
                                 _vp, _vp], _int),
+    "wildcat_decode_attend_workspace_size": ([_i64, _int], _sz),
+    "wildcat_decode_attend": ([_vp, _vp, _vp, _vp, _int, _i64, _i64, _int, _int, _vp, _f32, _vp, _vp, _vp,
+                               _vp, _vp, _vp, _sz, _vp], _int),
     "wildcat_forward_workspace_size": ([_i64, _i64, _i64, _int, _int, _int], _sz),
     "wildcat_forward": ([_vp, _vp, _vp, _int, _i64, _i64, _i64, _int, _f32, _int, _u64, _i64, _f32, _vp,
                          _vp, _vp, _vp, _sz, _vp], _int),
+    "wildcat_forward_binned_workspace_size": ([_i64, _i64, _i64, _int, _int, _int, _int], _sz),
+    "wildcat_forward_binned": ([_vp, _vp, _vp, _int, _i64, _i64, _i64, _int, _f32, _int, _int, _u64, _i64,
+                                _f32, _vp, _vp, _vp, _vp, _sz, _vp], _int),
     "wildcat_forward_host_workspace_size": ([_i64, _i64, _i64, _int, _int, _int], _sz),
     "wildcat_forward_host": ([_vp, _vp, _vp, _int, _i64, _i64, _i64, _int, _f32, _int, _u64, _i64, _f32,
                               _vp, _vp, _vp, _vp, _sz, _vp], _int),
@@ -255,6 +261,29 @@ def attend_noalloc(Q, K_S, rank, beta: float, V_S, w, vmin, vmax, *, out=None, s
     return O
 
 
+def decode_attend(Q_new, K_new, V_new, K_S, rank, beta: float, V_S, w, vmin, vmax, *, stream=None):
+    """KV-cache decode with new tokens: Q_new/K_new/V_new [BH, m, d] attend
+    over the compressed cache (K_S, V_S, w, rank, vmin, vmax) and causally
+    over the new tokens.  Returns O [BH, m, d] float32."""
+    torch = _torch()
+    BH, m, d = _shape3(Q_new, "Q_new")
+    r = K_S.shape[1]
+    for t, nm in ((K_new, "K_new"), (V_new, "V_new"), (K_S, "K_S")):
+        if t.dtype != Q_new.dtype:
+            raise TypeError(f"{nm} must share Q_new's dtype")
+    O = torch.empty((BH, m, d), dtype=torch.float32, device=Q_new.device)
+    L = lib()
+    nbytes = int(L.wildcat_decode_attend_workspace_size(BH, d))
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=Q_new.device)
+    _check(L.wildcat_decode_attend(_dev(Q_new, "Q_new"), _dev(K_new, "K_new"), _dev(V_new, "V_new"),
+                                   _dev(K_S, "K_S"), _dtype_code(Q_new), BH, m, d, r,
+                                   _dev(rank, "rank", torch.int32), float(beta),
+                                   _dev(V_S, "V_S", torch.float32), _dev(w, "w", torch.float32),
+                                   _dev(vmin, "vmin", torch.float32), _dev(vmax, "vmax", torch.float32),
+                                   _dev(O, "O"), _dev(ws, "workspace"), nbytes, _stream(stream)))
+    return O
+
+
 class ForwardPlan:
     """Preallocated workspace and outputs for repeated wildcat_forward calls
     on one shape (what a serving loop or the benchmark holds on to)."""
@@ -290,6 +319,44 @@ def forward(Q, K, V, beta: float, r: int, seed: int = 0, eps: float = 1e-6, *, i
     if Q.dtype != K.dtype or V.dtype != K.dtype:
         raise TypeError("Q, K, V must share a dtype")
     plan = ForwardPlan(BH, m, n, d, r, "bf16" if code else "f32", device=K.device)
+    O, S, rank = plan.run(Q, K, V, beta, seed, eps, stream, inst0)
+    return O.clone(), S.clone(), rank.clone()
+
+
+class BinnedForwardPlan:
+    """Preallocated workspace and outputs for wildcat_forward_binned."""
+
+    def __init__(self, BH, m, n, d, r, nbins, dtype: str, device="cuda"):
+        torch = _torch()
+        self.BH, self.m, self.n, self.d, self.r, self.nbins = BH, m, n, d, r, nbins
+        self.code = DTYPES[dtype]
+        L = lib()
+        self.ws_bytes = int(L.wildcat_forward_binned_workspace_size(BH, m, n, d, r, nbins, self.code))
+        if self.ws_bytes == 0:
+            raise ValueError("n and r must be multiples of nbins")
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
+        self.O = torch.empty((BH, m, d), dtype=torch.float32, device=device)
+        self.S = torch.empty((BH, r), dtype=torch.int32, device=device)
+        self.rank = torch.empty((BH, nbins), dtype=torch.int32, device=device)
+
+    def run(self, Q, K, V, beta, seed, eps=1e-6, stream=None, inst0=0):
+        _check(lib().wildcat_forward_binned(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), self.code, self.BH,
+                                            self.m, self.n, self.d, float(beta), self.r, self.nbins,
+                                            int(seed) & (2**64 - 1), int(inst0), float(eps),
+                                            _dev(self.O, "O"), _dev(self.S, "S"), _dev(self.rank, "rank"),
+                                            _dev(self.ws, "workspace"), self.ws_bytes, _stream(stream)))
+        return self.O, self.S, self.rank
+
+
+def forward_binned(Q, K, V, beta: float, r: int, nbins: int, seed: int = 0, eps: float = 1e-6, *,
+                   inst0: int = 0, stream=None):
+    """WildCat with divide-and-conquer binning (Sec. 2): nbins contiguous key
+    bins with r / nbins pivots each.  Returns (O_hat, S [BH, r] global key
+    indices, rank [BH, nbins])."""
+    BH, m, d = _shape3(Q, "Q")
+    n = K.shape[1]
+    code = _dtype_code(K)
+    plan = BinnedForwardPlan(BH, m, n, d, r, nbins, "bf16" if code else "f32", device=K.device)
     O, S, rank = plan.run(Q, K, V, beta, seed, eps, stream, inst0)
     return O.clone(), S.clone(), rank.clone()
 

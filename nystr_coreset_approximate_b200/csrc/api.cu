@@ -126,6 +126,54 @@ wildcat_status forward_impl(const void* Q, const void* K, const void* V, int dty
     return record(Status::ok());
 }
 
+struct BinnedLayout {
+    float* F;
+    int32_t* S;
+    int32_t* rank_b;
+    void* K_S;
+    float* V_S;
+    float* w;
+    float* vmin_b;
+    float* vmax_b;
+    float* vmin;
+    float* vmax;
+    int32_t* rank_att;
+    void* wws;
+    size_t wws_bytes;
+    void* aws;
+    size_t aws_bytes;
+};
+
+BinnedLayout carve_binned(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, int r, int nbins, int dtype) {
+    const int64_t nb = n / nbins;
+    const int rb = r / nbins;
+    const int64_t BB = BH * nbins;
+    BinnedLayout L{};
+    L.F = static_cast<float*>(cv.take(sizeof(float) * BB * (int64_t)rb * nb));
+    L.S = static_cast<int32_t*>(cv.take(sizeof(int32_t) * BH * r));
+    L.rank_b = static_cast<int32_t*>(cv.take(sizeof(int32_t) * BB));
+    L.K_S = cv.take(elem_bytes(dtype) * BH * (int64_t)r * d);
+    L.V_S = static_cast<float*>(cv.take(sizeof(float) * BH * (int64_t)r * d));
+    L.w = static_cast<float*>(cv.take(sizeof(float) * BH * r));
+    L.vmin_b = static_cast<float*>(cv.take(sizeof(float) * BB * d));
+    L.vmax_b = static_cast<float*>(cv.take(sizeof(float) * BB * d));
+    L.vmin = static_cast<float*>(cv.take(sizeof(float) * BH * d));
+    L.vmax = static_cast<float*>(cv.take(sizeof(float) * BH * d));
+    L.rank_att = static_cast<int32_t*>(cv.take(sizeof(int32_t) * BH));
+    L.wws_bytes = wildcat::weights_workspace_bytes(BB, nb, d, rb);
+    L.wws = cv.take(L.wws_bytes);
+    L.aws_bytes = wildcat::attend_workspace_bytes(BH, m, d, r);
+    L.aws = cv.take(L.aws_bytes);
+    return L;
+}
+
+wildcat_status check_bins(int64_t BH, int64_t n, int r, int nbins, const char* who) {
+    if (nbins < 1) return bad(1, "%s: nbins must be >= 1", who);
+    if (n % nbins || r % nbins) return bad(1, "%s: n and r must be multiples of nbins", who);
+    if (BH * nbins > 65535) return bad(2, "%s: BH * nbins above 65535 is not supported", who);
+    return WILDCAT_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -220,6 +268,30 @@ wildcat_status wildcat_attend_noalloc(const void* Q, const void* K_S, int dtype,
     return record(wildcat::launch_attend_noalloc(q, static_cast<cudaStream_t>(stream)));
 }
 
+size_t wildcat_decode_attend_workspace_size(int64_t BH, int d) {
+    if (BH < 0 || d < 1) return 0;
+    return wildcat::decode_workspace_bytes(BH, d);
+}
+
+wildcat_status wildcat_decode_attend(const void* Q_new, const void* K_new, const void* V_new, const void* K_S,
+                                     int dtype, int64_t BH, int64_t m, int d, int r, const int32_t* rank, float beta,
+                                     const float* V_S, const float* w, const float* vmin, const float* vmax, float* O,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+    const char* who = "wildcat_decode_attend";
+    wildcat_status st = check_common(dtype, BH, r, d, r, who);
+    if (st != WILDCAT_OK) return st;
+    if ((st = check_scalars(beta, 0.f, who)) != WILDCAT_OK) return st;
+    if (m < 0) return bad(1, "%s: m must be >= 0", who);
+    if (BH == 0 || m == 0) return record(Status::ok());
+    if (!Q_new || !K_new || !V_new || !K_S || !rank || !V_S || !w || !vmin || !vmax || !O || !workspace)
+        return bad(1, "%s: null pointer argument", who);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
+    if (ws_bytes < wildcat::decode_workspace_bytes(BH, d)) return bad(4, "%s: workspace too small", who);
+    wildcat::DecodeRequest q{Q_new, K_new, V_new, K_S, dtype, BH, m, d, r, rank, beta, V_S, w, vmin, vmax, O,
+                             workspace, ws_bytes};
+    return record(wildcat::launch_decode(q, static_cast<cudaStream_t>(stream)));
+}
+
 size_t wildcat_forward_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int dtype) {
     if (BH < 0 || m < 0 || n < 1 || r < 1 || d < 1) return 0;
     Carve cv(nullptr, 0);
@@ -246,6 +318,54 @@ wildcat_status wildcat_forward(const void* Q, const void* K, const void* V, int 
     if (inst0 < 0 || inst0 + BH > 4294967296LL) return bad(1, "%s: inst0 must satisfy 0 <= inst0, inst0 + BH <= 2^32", who);
     return forward_impl(Q, K, V, dtype, BH, m, n, d, beta, r, seed, inst0, eps, O, S_out, rank_out, L,
                         static_cast<cudaStream_t>(stream));
+}
+
+size_t wildcat_forward_binned_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int nbins, int dtype) {
+    if (BH < 0 || m < 0 || n < 1 || r < 1 || d < 1 || nbins < 1 || n % nbins || r % nbins) return 0;
+    Carve cv(nullptr, 0);
+    carve_binned(cv, BH, m, n, d, r, nbins, dtype);
+    return cv.used + 256;
+}
+
+wildcat_status wildcat_forward_binned(const void* Q, const void* K, const void* V, int dtype, int64_t BH, int64_t m,
+                                      int64_t n, int d, float beta, int r, int nbins, uint64_t seed, int64_t inst0,
+                                      float eps, float* O, int32_t* S_out, int32_t* rank_out, void* workspace,
+                                      size_t ws_bytes, void* stream) {
+    const char* who = "wildcat_forward_binned";
+    wildcat_status st = check_common(dtype, BH, n, d, r, who);
+    if (st != WILDCAT_OK) return st;
+    if ((st = check_scalars(beta, eps, who)) != WILDCAT_OK) return st;
+    if ((st = check_bins(BH, n, r, nbins, who)) != WILDCAT_OK) return st;
+    if (m < 0) return bad(1, "%s: m must be >= 0", who);
+    if (inst0 < 0 || (inst0 + BH) * nbins > 4294967296LL)
+        return bad(1, "%s: inst0 must satisfy 0 <= inst0, (inst0 + BH) * nbins <= 2^32", who);
+    if (BH == 0) return record(Status::ok());
+    if (!K || !V || !workspace || (m > 0 && (!Q || !O))) return bad(1, "%s: null pointer argument", who);
+    if (!aligned16(K) || !aligned16(V) || (Q && !aligned16(Q)))
+        return bad(1, "%s: Q, K and V must be 16-byte aligned", who);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
+    Carve cv(workspace, ws_bytes);
+    const BinnedLayout L = carve_binned(cv, BH, m, n, d, r, nbins, dtype);
+    if (!cv.fits()) return bad(4, "%s: workspace too small", who);
+    const int64_t nb = n / nbins, BB = BH * nbins;
+    const int rb = r / nbins;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Status z;
+    wildcat::SelectRequest sq{K, dtype, BB, nb, d, beta, rb, seed, inst0 * nbins, eps, nullptr, L.S, L.F, L.rank_b,
+                              L.K_S};
+    if ((z = wildcat::launch_select(sq, s)).code) return record(z);
+    wildcat::WeightsRequest wq{L.F, L.S, L.rank_b, V, dtype, BB, nb, d, rb, L.V_S, L.w, L.vmin_b, L.vmax_b, L.wws,
+                               L.wws_bytes};
+    if ((z = wildcat::launch_weights(wq, s)).code) return record(z);
+    if ((z = wildcat::launch_binning_finish(L.vmin_b, L.vmax_b, L.S, L.rank_b, BH, nbins, nb, rb, d, L.vmin, L.vmax,
+                                            L.rank_att, S_out, rank_out, s)).code)
+        return record(z);
+    if (m > 0) {
+        wildcat::AttendRequest aq{Q,      L.K_S,  dtype, BH, m, d, r, L.rank_att, beta, L.V_S, L.w,
+                                  L.vmin, L.vmax, O,     L.aws, L.aws_bytes};
+        if ((z = wildcat::launch_attend(aq, s)).code) return record(z);
+    }
+    return record(Status::ok());
 }
 
 size_t wildcat_forward_host_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int dtype) {

@@ -96,6 +96,33 @@ void set_attend_force_timeout(unsigned long long ns);
 size_t attend_noalloc_scratch_bytes();
 Status launch_attend_noalloc(const AttendRequest& q, cudaStream_t stream);
 
+// KV-cache decode with new tokens (decode.cu)
+struct DecodeRequest {
+    const void* Qn;
+    const void* Kn;
+    const void* Vn;
+    const void* K_S;
+    int dtype;
+    int64_t BH, m;
+    int d, r;
+    const int32_t* rank;
+    float beta;
+    const float* V_S;
+    const float* w;
+    const float* vmin;
+    const float* vmax;
+    float* O;
+    void* ws;
+    size_t ws_bytes;
+};
+size_t decode_workspace_bytes(int64_t BH, int d);
+Status launch_decode(const DecodeRequest& q, cudaStream_t stream);
+
+// binned forward glue (binning.cu)
+Status launch_binning_finish(const float* vmin_b, const float* vmax_b, const int32_t* S_b, const int32_t* rank_b,
+                             int64_t BH, int nbins, int64_t nb, int rb, int d, float* vmin, float* vmax,
+                             int32_t* rank_att, int32_t* S_out, int32_t* rank_out, cudaStream_t st);
+
 // 256-byte aligned bump allocator over a caller-provided workspace.
 struct Carve {
     char* base;

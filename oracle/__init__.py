@@ -80,6 +80,16 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
                                            ctypes.c_int, ctypes.c_uint64, ctypes.c_double,
                                            _i32p, _i64p, ctypes.c_int64, _f64p, _i32p, _i32p]
     lib.oracle_wildcat_forward.restype = ctypes.c_int
+    lib.oracle_wildcat_forward_binned.argtypes = [_f64p, _f64p, _f64p, ctypes.c_int64,
+                                                  ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                                  ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_uint64, ctypes.c_double, _i32p, _i64p,
+                                                  ctypes.c_int64, _f64p, _i32p, _i32p]
+    lib.oracle_wildcat_forward_binned.restype = ctypes.c_int
+    lib.oracle_decode_attend.argtypes = [_f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _i32p, _f64p,
+                                         _f64p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_double, _f64p]
+    lib.oracle_decode_attend.restype = ctypes.c_int
     return lib
 
 
@@ -253,6 +263,54 @@ class Oracle:
         if err:
             raise MemoryError("oracle_wildcat_forward")
         return O, S, rank
+
+
+    def wildcat_forward_binned(self, Q, K, V, beta, r, nbins, seed=0, eps=1e-6, rows=None,
+                               S_fixed=None):
+        """WildCat with divide-and-conquer binning (Sec. 2): nbins contiguous
+        bins, r / nbins pivots each, block-diagonal weights, attend over the
+        union.  Returns (O_hat, S [BH, r] global key indices, rank [BH, nbins])."""
+        Q, qp = self._f64(Q)
+        K, kp = self._f64(K)
+        V, vp = self._f64(V)
+        BH, m, d = Q.shape
+        n = K.shape[1]
+        rows_a, rp, nr = self._rows(rows)
+        O = np.zeros((BH, nr if rows is not None else m, d))
+        S = np.full((BH, r), -1, dtype=np.int32)
+        rank = np.zeros((BH, nbins), dtype=np.int32)
+        Sf, sfp = self._i32(S_fixed)
+        err = self.lib.oracle_wildcat_forward_binned(
+            qp, kp, vp, BH, m, n, d, float(beta), int(r), int(nbins), int(seed), float(eps), sfp,
+            rp, nr,
+            O.ctypes.data_as(_f64p), S.ctypes.data_as(_i32p), rank.ctypes.data_as(_i32p))
+        if err == 2:
+            raise ValueError("n and r must be multiples of nbins")
+        if err:
+            raise MemoryError("oracle_wildcat_forward_binned")
+        return O, S, rank
+
+
+    def decode_attend(self, Qn, Kn, Vn, KS, VS, w, rank, vmin, vmax, beta):
+        """New tokens over the compressed cache plus causal exact attention
+        among themselves (Sec. 2, KV-cache decode).  Returns O [BH, m, d]."""
+        Qn, qp = self._f64(Qn)
+        Kn, kp = self._f64(Kn)
+        Vn, vp = self._f64(Vn)
+        KS, ksp = self._f64(KS)
+        VS, vsp = self._f64(VS)
+        w, wp = self._f64(w)
+        rank, rkp = self._i32(rank)
+        vmin, lop = self._f64(vmin)
+        vmax, hip = self._f64(vmax)
+        BH, m, d = Qn.shape
+        r = KS.shape[1]
+        O = np.zeros((BH, m, d))
+        err = self.lib.oracle_decode_attend(qp, kp, vp, ksp, vsp, wp, rkp, lop, hip, BH, m, d, r,
+                                            float(beta), O.ctypes.data_as(_f64p))
+        if err:
+            raise MemoryError("oracle_decode_attend")
+        return O
 
 
 _default: Optional[Oracle] = None

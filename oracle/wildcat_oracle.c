@@ -500,3 +500,157 @@ int oracle_wildcat_forward(const double* Q, const double* K, const double* V, in
     }
     return err;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Divide and conquer (Sec. 2, binning): the n keys of an instance are cut   */
+/* into nbins contiguous bins of n / nbins keys; each bin gets its own      */
+/* RPNys coreset of r / nbins pivots and its own Nystrom weights over its    */
+/* own keys (the pivot draws of bin q of instance b use instance index      */
+/* b * nbins + q); the coreset is the union and the weights are block       */
+/* diagonal.  The plug-in output then attends over the union exactly as     */
+/* without bins (rows past a bin's rank are zero and contribute nothing).   */
+/*   S_fixed  [BH, r]  global key indices to use instead of draws (or NULL); */
+/*            row q * (r / nbins) + a must lie in bin q, -1 ends the bin    */
+/*   S_out    [BH, r]  global key index of every union row (-1 past a bin's */
+/*            rank)                                                         */
+/*   rank_out [BH, nbins] effective rank of every bin                       */
+/* ------------------------------------------------------------------------ */
+int oracle_wildcat_forward_binned(const double* Q, const double* K, const double* V, int64_t BH,
+                                  int64_t m, int64_t n, int d, double beta, int r, int nbins,
+                                  uint64_t seed, double eps, const int32_t* S_fixed,
+                                  const int64_t* rows, int64_t nrows, double* O, int32_t* S_out,
+                                  int32_t* rank_out) {
+    if (nbins < 1 || n % nbins || r % nbins) return 2;
+    const int64_t nb = n / nbins;
+    const int rb = r / nbins;
+    const int64_t nr = rows ? nrows : m;
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t b = 0; b < BH; ++b) {
+        double* F = (double*)malloc(sizeof(double) * (size_t)rb * (size_t)nb);
+        double* dg = (double*)malloc(sizeof(double) * (size_t)nb);
+        double* g = (double*)malloc(sizeof(double) * (size_t)nb);
+        double* Y = (double*)malloc(sizeof(double) * (size_t)rb * (size_t)(d + 1));
+        double* VS = (double*)malloc(sizeof(double) * (size_t)r * (size_t)d);
+        double* w = (double*)malloc(sizeof(double) * (size_t)r);
+        double* KS = (double*)malloc(sizeof(double) * (size_t)r * (size_t)d);
+        double* vmin = (double*)malloc(sizeof(double) * (size_t)d);
+        double* vmax = (double*)malloc(sizeof(double) * (size_t)d);
+        double* N = (double*)malloc(sizeof(double) * (size_t)d);
+        int32_t* Sb = (int32_t*)malloc(sizeof(int32_t) * (size_t)rb);
+        int32_t* Sf = (int32_t*)malloc(sizeof(int32_t) * (size_t)rb);
+        if (!F || !dg || !g || !Y || !VS || !w || !KS || !vmin || !vmax || !N || !Sb || !Sf) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+            const double* Kb = K + b * n * d;
+            const double* Vb = V + b * n * d;
+            for (int q = 0; q < nbins; ++q) {
+                const double* Kq = Kb + (int64_t)q * nb * d;
+                const double* Vq = Vb + (int64_t)q * nb * d;
+                if (S_fixed)
+                    for (int a = 0; a < rb; ++a) {
+                        const int32_t sg = S_fixed[b * r + q * rb + a];
+                        Sf[a] = (sg >= q * nb && sg < (q + 1) * nb) ? (int32_t)(sg - q * nb) : -1;
+                    }
+                const int rr = rpc_one(Kq, nb, d, beta, rb, seed, b * nbins + q, eps, 1,
+                                       S_fixed ? Sf : NULL, Sb, F, NULL, NULL, dg, g);
+                if (rank_out) rank_out[b * nbins + q] = rr;
+                weights_one(F, Sb, rr, Vq, nb, d, rb, VS + (int64_t)q * rb * d, w + q * rb, Y);
+                for (int a = 0; a < rb; ++a) {
+                    const int row = q * rb + a;
+                    if (S_out) S_out[b * r + row] = a < rr ? (int32_t)(q * nb + Sb[a]) : -1;
+                    for (int c = 0; c < d; ++c)
+                        KS[(int64_t)row * d + c] = a < rr ? Kq[(int64_t)Sb[a] * d + c] : 0.0;
+                }
+            }
+            oracle_value_range(Vb, 1, n, d, vmin, vmax);
+            const double MQ = query_shift(Q + b * m * d, m, KS, r, d);
+            for (int64_t ii = 0; ii < nr; ++ii) {
+                const int64_t i = rows ? rows[ii] : ii;
+                attend_row(Q + (b * m + i) * d, KS, VS, w, r, vmin, vmax, d, beta, MQ,
+                           O + (b * nr + ii) * d, N);
+            }
+        }
+        free(F); free(dg); free(g); free(Y); free(VS); free(w); free(KS);
+        free(vmin); free(vmax); free(N); free(Sb); free(Sf);
+    }
+    return err;
+}
+
+/* ------------------------------------------------------------------------ */
+/* KV-cache decode with new tokens (Sec. 2: after CompressKV, m new tokens  */
+/* cost O(rmd + m^2 d) instead of O(nmd + m^2 d)).  New query i attends over */
+/* the weighted coreset of the compressed cache and, exactly, over the new  */
+/* tokens j <= i (causal):                                                  */
+/*   N_i = sum_l u_il V_S,l + sum_{j<=i} e_ij v_j                           */
+/*   D_i = sum_l u_il w_l   + sum_{j<=i} e_ij                               */
+/*   u_il = exp(beta <q_i, k_S_l> - beta M), e_ij = exp(beta <q_i, k_j> - beta M) */
+/* with one shift M = max_i |q_i| * max(max_l |k_S_l|, max_j |k_j|), and    */
+/* O_i = clip(N_i / D_i) to the range of the old values (vmin, vmax of the  */
+/* cache) and the new values together.                                      */
+/*   Qn, Kn, Vn [BH, m, d] new tokens; KS, VS [BH, r, d], w [BH, r], rank   */
+/*   [BH], vmin/vmax [BH, d] from the compressed cache; O [BH, m, d]        */
+/* ------------------------------------------------------------------------ */
+int oracle_decode_attend(const double* Qn, const double* Kn, const double* Vn, const double* KS,
+                         const double* VS, const double* w, const int32_t* rank,
+                         const double* vmin, const double* vmax, int64_t BH, int64_t m, int d,
+                         int r, double beta, double* O) {
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t b = 0; b < BH; ++b) {
+        double* N = (double*)malloc(sizeof(double) * (size_t)d);
+        double* lo = (double*)malloc(sizeof(double) * (size_t)d);
+        double* hi = (double*)malloc(sizeof(double) * (size_t)d);
+        if (!N || !lo || !hi) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+            const double* Qb = Qn + b * m * d;
+            const double* Kb = Kn + b * m * d;
+            const double* Vb = Vn + b * m * d;
+            const double* KSb = KS + b * (int64_t)r * d;
+            const double* VSb = VS + b * (int64_t)r * d;
+            const int rr = rank[b];
+            double qn = 0.0, kn = 0.0;
+            for (int64_t i = 0; i < m; ++i) {
+                const double v = sqrt(dot(Qb + i * d, Qb + i * d, d));
+                if (v > qn) qn = v;
+                const double u = sqrt(dot(Kb + i * d, Kb + i * d, d));
+                if (u > kn) kn = u;
+            }
+            for (int l = 0; l < rr; ++l) {
+                const double v = sqrt(dot(KSb + (int64_t)l * d, KSb + (int64_t)l * d, d));
+                if (v > kn) kn = v;
+            }
+            const double M = qn * kn;
+            for (int c = 0; c < d; ++c) {
+                lo[c] = vmin[b * d + c];
+                hi[c] = vmax[b * d + c];
+                for (int64_t j = 0; j < m; ++j) {
+                    const double v = Vb[j * d + c];
+                    if (v < lo[c]) lo[c] = v;
+                    if (v > hi[c]) hi[c] = v;
+                }
+            }
+            for (int64_t i = 0; i < m; ++i) {
+                const double* q = Qb + i * d;
+                double D = 0.0;
+                for (int c = 0; c < d; ++c) N[c] = 0.0;
+                for (int l = 0; l < rr; ++l) {
+                    const double u = exp(beta * dot(q, KSb + (int64_t)l * d, d) - beta * M);
+                    for (int c = 0; c < d; ++c) N[c] += u * VSb[(int64_t)l * d + c];
+                    D += u * w[b * r + l];
+                }
+                for (int64_t j = 0; j <= i; ++j) {
+                    const double e = exp(beta * dot(q, Kb + j * d, d) - beta * M);
+                    for (int c = 0; c < d; ++c) N[c] += e * Vb[j * d + c];
+                    D += e;
+                }
+                for (int c = 0; c < d; ++c) O[(b * m + i) * d + c] = fmin(fmax(N[c] / D, lo[c]), hi[c]);
+            }
+        }
+        free(N); free(lo); free(hi);
+    }
+    return err;
+}

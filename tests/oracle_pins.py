@@ -334,6 +334,59 @@ def pin_hand_examples(o):
                                        np.array(c["O_exact"], float), rtol=0, atol=1e-12)
 
 
+# --------------------------------------------------------------------------- binning
+def pin_binning_closed_forms(o):
+    """Divide-and-conquer binning (Sec. 2): one bin is the unbinned method
+    bit for bit; r = n (every key a pivot of its bin) makes every bin's
+    weights a permutation, so the union estimate is exact attention; pivots
+    of bin q lie inside bin q and are distinct."""
+    Q, K, V = _rand(131, 2, 20, 48, 6)
+    a = o.wildcat_forward(Q, K, V, 0.4, 12, seed=3)
+    b1 = o.wildcat_forward_binned(Q, K, V, 0.4, 12, 1, seed=3)
+    np.testing.assert_array_equal(a[0], b1[0])
+    np.testing.assert_array_equal(a[1], b1[1])
+    O, S, rank = o.wildcat_forward_binned(Q, K, V, 0.4, 48, 4, seed=3, eps=1e-14)
+    assert np.all(rank == 12)
+    np.testing.assert_allclose(O, o.exact_attention(Q, K, V, 0.4), rtol=0, atol=1e-12)
+    O, S, rank = o.wildcat_forward_binned(Q, K, V, 0.4, 16, 4, seed=5)
+    for b in range(2):
+        for q in range(4):
+            rows = S[b, 4 * q:4 * q + rank[b, q]]
+            assert np.all((rows >= 12 * q) & (rows < 12 * q + 12))
+        valid = S[b][S[b] >= 0]
+        assert len(set(valid.tolist())) == len(valid)
+
+
+# --------------------------------------------------------------------------- decode
+def pin_decode_closed_form(o):
+    """KV-cache decode: with the cache compressed at full rank (r = n, W a
+    permutation), new token i attends exactly over all n cached keys and
+    the new keys j <= i (causal softmax by numpy); with no cache rows
+    (rank 0) it is plain causal attention among the new tokens."""
+    rng = np.random.default_rng(141)
+    BH, n, m, d, beta = 2, 24, 7, 5, 0.45
+    K, V = rng.standard_normal((BH, n, d)), rng.standard_normal((BH, n, d))
+    Qn, Kn, Vn = (rng.standard_normal((BH, m, d)) for _ in range(3))
+    res = o.rpcholesky(K, beta, n, seed=2, eps=1e-14)
+    assert np.all(res["rank"] == n)
+    VS, w = o.weights(res["F"], res["S"], res["rank"], V)
+    KS = o.gather(K, res["S"], res["rank"])
+    lo, hi = o.value_range(V)
+    O = o.decode_attend(Qn, Kn, Vn, KS, VS, w, res["rank"], lo, hi, beta)
+    for b in range(BH):
+        for i in range(m):
+            keys = np.concatenate([K[b], Kn[b, :i + 1]])
+            vals = np.concatenate([V[b], Vn[b, :i + 1]])
+            p = special.softmax(beta * keys @ Qn[b, i])
+            np.testing.assert_allclose(O[b, i], p @ vals, rtol=0, atol=1e-9)
+    zero = np.zeros(BH, np.int32)
+    O0 = o.decode_attend(Qn, Kn, Vn, KS, VS, w, zero, lo, hi, beta)
+    for b in range(BH):
+        for i in range(m):
+            p = special.softmax(beta * Kn[b, :i + 1] @ Qn[b, i])
+            np.testing.assert_allclose(O0[b, i], p @ Vn[b, :i + 1], rtol=0, atol=1e-12)
+
+
 ALL_PINS = [
     pin_exact_bruteforce,
     pin_full_rank_is_exact,
@@ -349,4 +402,6 @@ ALL_PINS = [
     pin_error_falls_with_rank,
     pin_single_pivot_closed_form,
     pin_hand_examples,
+    pin_binning_closed_forms,
+    pin_decode_closed_form,
 ]

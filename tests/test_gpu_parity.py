@@ -25,7 +25,7 @@ CASES = [
     gc.case("bf16_walk_d128", "walk", 2, 4100, 64, 128, 200, "bf16"),
     gc.case("bf16_iid_d128", "iid", 1, 5000, 300, 128, 128, "bf16"),
     gc.case("bf16_many_small", "iid", 300, 96, 40, 64, 8, "bf16"),
-    gc.case("bf16_rank_chunks", "mixture16", 2, 1600, 700, 64, 300, "bf16"),
+    gc.case("bf16_rank_chunks", "mixture16", 2, 1600, 1600, 64, 300, "bf16"),
 ]
 
 
@@ -255,7 +255,7 @@ def test_bounded_wait_reports_timeout_and_recovers():
     """A tensor-core wait that runs out (the test hook makes the attend wait
     on a barrier phase nothing completes, for 1 ms) is reported through the
     device status word; the context stays usable and the next call is clean."""
-    w = gc.case("timeout", "mixture16", 2, 784, 300, 64, 64, "bf16")
+    w = gc.case("timeout", "mixture16", 2, 784, 784, 64, 64, "bf16")
     dev, _ = workloads.make(w)
     d = gc.cuda_inputs(dev)
     S, F, rank, K_S = wc.select(d["K"], w.beta, w.r, 3)
