@@ -232,6 +232,42 @@ wildcat_status wildcat_forward(const void* Q, const void* K, const void* V, int 
                                int32_t* rank_out, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Options of wildcat_forward_ex (Sec. 2: divide-and-conquer bins, recentring
+ * of the keys and temperature rescaling).
+ *   nbins     >= 1: keys cut into nbins contiguous bins (see
+ *             wildcat_forward_binned); 1 = no binning
+ *   recenter  0 or 1: select and weight the coreset on the recentred keys
+ *             k_l - kbar, kbar the instance's mean key (softmax attention is
+ *             unchanged by the shift)
+ *   tau       > 0: temperature; the coreset is selected and weighted with
+ *             the key kernel exp(beta <x, y> / tau^2), i.e. on keys K / tau,
+ *             while queries become tau Q, leaving attention unchanged.  The
+ *             pages' closed form for tau (their eq. 12) did not survive, so
+ *             tau is the caller's; 1 = no rescaling.
+ * The attend step needs neither: with the original pivot keys and beta, the
+ * recentring shift and 1 / tau cancel in N / D.
+ */
+typedef struct {
+    int nbins;
+    int recenter;
+    float tau;
+} wildcat_options;
+
+/*
+ * wildcat_forward_ex -- wildcat_forward with wildcat_options (NULL: the
+ * defaults {1, 0, 1}, identical to wildcat_forward).  S_out [BH, r] global
+ * key indices and rank_out [BH, nbins] as in wildcat_forward_binned.
+ *   workspace >= wildcat_forward_ex_workspace_size(...) bytes
+ */
+size_t wildcat_forward_ex_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int dtype,
+                                         const wildcat_options* opts);
+wildcat_status wildcat_forward_ex(const void* Q, const void* K, const void* V, int dtype, int64_t BH,
+                                  int64_t m, int64_t n, int d, float beta, int r, uint64_t seed,
+                                  int64_t inst0, float eps, const wildcat_options* opts, float* O,
+                                  int32_t* S_out, int32_t* rank_out, void* workspace,
+                                  size_t ws_bytes, void* stream);
+
+/*
  * wildcat_forward_binned -- the module with divide-and-conquer binning
  * (Sec. 2: B bins, r / B pivots each, selected in parallel).  The n keys of
  * every instance are cut into nbins contiguous bins of n / nbins keys; bin q
@@ -239,7 +275,8 @@ wildcat_status wildcat_forward(const void* Q, const void* K, const void* V, int 
  * instance index (inst0 + b) * nbins + q) and its own Nystrom weights over
  * its own keys (block-diagonal W).  The output attends over the union of the
  * bins' coresets; the value range is over all n keys.  n and r must be
- * multiples of nbins; nbins = 1 is wildcat_forward.
+ * multiples of nbins; nbins = 1 is wildcat_forward.  Same as
+ * wildcat_forward_ex with options {nbins, 0, 1}.
  *
  *   S_out    [BH, r] int32 global key index of every union row, -1 past a
  *            bin's rank (or NULL); row q * (r / nbins) + a is bin q's a-th pivot

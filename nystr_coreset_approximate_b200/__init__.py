@@ -24,7 +24,7 @@ from typing import Optional
 
 __all__ = [
     "WildcatError", "library_path", "lib", "declared_symbols", "select", "select_fixed",
-    "weights", "attend", "attend_noalloc", "decode_attend", "forward", "forward_binned", "BinnedForwardPlan", "forward_host", "ForwardPlan", "pivot_uniforms",
+    "weights", "attend", "attend_noalloc", "decode_attend", "forward", "forward_ex", "Options", "forward_binned", "BinnedForwardPlan", "forward_host", "ForwardPlan", "pivot_uniforms",
     "set_select_cluster", "last_select_cluster", "device_status", "DTYPES",
 ]
 
@@ -62,6 +62,9 @@ _SIGS = {
     "wildcat_forward_workspace_size": ([_i64, _i64, _i64, _int, _int, _int], _sz),
     "wildcat_forward": ([_vp, _vp, _vp, _int, _i64, _i64, _i64, _int, _f32, _int, _u64, _i64, _f32, _vp,
                          _vp, _vp, _vp, _sz, _vp], _int),
+    "wildcat_forward_ex_workspace_size": ([_i64, _i64, _i64, _int, _int, _int, _vp], _sz),
+    "wildcat_forward_ex": ([_vp, _vp, _vp, _int, _i64, _i64, _i64, _int, _f32, _int, _u64, _i64, _f32, _vp,
+                            _vp, _vp, _vp, _vp, _sz, _vp], _int),
     "wildcat_forward_binned_workspace_size": ([_i64, _i64, _i64, _int, _int, _int, _int], _sz),
     "wildcat_forward_binned": ([_vp, _vp, _vp, _int, _i64, _i64, _i64, _int, _f32, _int, _int, _u64, _i64,
                                 _f32, _vp, _vp, _vp, _vp, _sz, _vp], _int),
@@ -359,6 +362,35 @@ def forward_binned(Q, K, V, beta: float, r: int, nbins: int, seed: int = 0, eps:
     plan = BinnedForwardPlan(BH, m, n, d, r, nbins, "bf16" if code else "f32", device=K.device)
     O, S, rank = plan.run(Q, K, V, beta, seed, eps, stream, inst0)
     return O.clone(), S.clone(), rank.clone()
+
+
+class Options(ctypes.Structure):
+    """wildcat_options: divide-and-conquer bins, key recentring, temperature."""
+    _fields_ = [("nbins", ctypes.c_int), ("recenter", ctypes.c_int), ("tau", ctypes.c_float)]
+
+
+def forward_ex(Q, K, V, beta: float, r: int, seed: int = 0, eps: float = 1e-6, *, nbins: int = 1,
+               recenter: bool = False, tau: float = 1.0, inst0: int = 0, stream=None):
+    """WildCat with the options of Sec. 2 (bins, recentring, temperature).
+    Returns (O_hat, S [BH, r] global key indices, rank [BH, nbins])."""
+    torch = _torch()
+    BH, m, d = _shape3(Q, "Q")
+    n = K.shape[1]
+    code = _dtype_code(K)
+    opts = Options(int(nbins), int(bool(recenter)), float(tau))
+    L = lib()
+    nbytes = int(L.wildcat_forward_ex_workspace_size(BH, m, n, d, r, code, ctypes.byref(opts)))
+    if nbytes == 0:
+        raise ValueError("n and r must be multiples of nbins")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=K.device)
+    O = torch.empty((BH, m, d), dtype=torch.float32, device=K.device)
+    S = torch.empty((BH, r), dtype=torch.int32, device=K.device)
+    rank = torch.empty((BH, nbins), dtype=torch.int32, device=K.device)
+    _check(L.wildcat_forward_ex(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), code, BH, m, n, d, float(beta), int(r),
+                                int(seed) & (2**64 - 1), int(inst0), float(eps), ctypes.byref(opts),
+                                _dev(O, "O"), _dev(S, "S"), _dev(rank, "rank"), _dev(ws, "workspace"), nbytes,
+                                _stream(stream)))
+    return O, S, rank
 
 
 class HostForwardPlan:

@@ -142,9 +142,12 @@ struct BinnedLayout {
     size_t wws_bytes;
     void* aws;
     size_t aws_bytes;
+    float* kbar;   // recentring only
+    void* mws;
 };
 
-BinnedLayout carve_binned(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, int r, int nbins, int dtype) {
+BinnedLayout carve_binned(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, int r, int nbins, int dtype,
+                          bool recenter) {
     const int64_t nb = n / nbins;
     const int rb = r / nbins;
     const int64_t BB = BH * nbins;
@@ -164,6 +167,8 @@ BinnedLayout carve_binned(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, in
     L.wws = cv.take(L.wws_bytes);
     L.aws_bytes = wildcat::attend_workspace_bytes(BH, m, d, r);
     L.aws = cv.take(L.aws_bytes);
+    L.kbar = recenter ? static_cast<float*>(cv.take(sizeof(float) * BH * d)) : nullptr;
+    L.mws = recenter ? cv.take(wildcat::key_mean_workspace_bytes(BH, n, d)) : nullptr;
     return L;
 }
 
@@ -320,22 +325,31 @@ wildcat_status wildcat_forward(const void* Q, const void* K, const void* V, int 
                         static_cast<cudaStream_t>(stream));
 }
 
-size_t wildcat_forward_binned_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int nbins, int dtype) {
+size_t wildcat_forward_ex_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int dtype,
+                                         const wildcat_options* opts) {
+    const int nbins = opts ? opts->nbins : 1;
     if (BH < 0 || m < 0 || n < 1 || r < 1 || d < 1 || nbins < 1 || n % nbins || r % nbins) return 0;
     Carve cv(nullptr, 0);
-    carve_binned(cv, BH, m, n, d, r, nbins, dtype);
+    carve_binned(cv, BH, m, n, d, r, nbins, dtype, opts && opts->recenter);
     return cv.used + 256;
 }
 
-wildcat_status wildcat_forward_binned(const void* Q, const void* K, const void* V, int dtype, int64_t BH, int64_t m,
-                                      int64_t n, int d, float beta, int r, int nbins, uint64_t seed, int64_t inst0,
-                                      float eps, float* O, int32_t* S_out, int32_t* rank_out, void* workspace,
-                                      size_t ws_bytes, void* stream) {
-    const char* who = "wildcat_forward_binned";
+wildcat_status wildcat_forward_ex(const void* Q, const void* K, const void* V, int dtype, int64_t BH, int64_t m,
+                                  int64_t n, int d, float beta, int r, uint64_t seed, int64_t inst0, float eps,
+                                  const wildcat_options* opts, float* O, int32_t* S_out, int32_t* rank_out,
+                                  void* workspace, size_t ws_bytes, void* stream) {
+    const char* who = "wildcat_forward_ex";
+    const int nbins = opts ? opts->nbins : 1;
+    const bool recenter = opts && opts->recenter;
+    const float tau = opts ? opts->tau : 1.f;
     wildcat_status st = check_common(dtype, BH, n, d, r, who);
     if (st != WILDCAT_OK) return st;
     if ((st = check_scalars(beta, eps, who)) != WILDCAT_OK) return st;
     if ((st = check_bins(BH, n, r, nbins, who)) != WILDCAT_OK) return st;
+    if (opts && opts->recenter != 0 && opts->recenter != 1) return bad(1, "%s: recenter must be 0 or 1", who);
+    if (!std::isfinite(tau) || !(tau > 0.f)) return bad(1, "%s: tau must be finite and > 0", who);
+    const float beta_key = beta / (tau * tau);
+    if (!std::isfinite(beta_key) || !(beta_key > 0.f)) return bad(1, "%s: beta / tau^2 must be finite and > 0", who);
     if (m < 0) return bad(1, "%s: m must be >= 0", who);
     if (inst0 < 0 || (inst0 + BH) * nbins > 4294967296LL)
         return bad(1, "%s: inst0 must satisfy 0 <= inst0, (inst0 + BH) * nbins <= 2^32", who);
@@ -345,14 +359,15 @@ wildcat_status wildcat_forward_binned(const void* Q, const void* K, const void* 
         return bad(1, "%s: Q, K and V must be 16-byte aligned", who);
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
     Carve cv(workspace, ws_bytes);
-    const BinnedLayout L = carve_binned(cv, BH, m, n, d, r, nbins, dtype);
+    const BinnedLayout L = carve_binned(cv, BH, m, n, d, r, nbins, dtype, recenter);
     if (!cv.fits()) return bad(4, "%s: workspace too small", who);
     const int64_t nb = n / nbins, BB = BH * nbins;
     const int rb = r / nbins;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Status z;
-    wildcat::SelectRequest sq{K, dtype, BB, nb, d, beta, rb, seed, inst0 * nbins, eps, nullptr, L.S, L.F, L.rank_b,
-                              L.K_S};
+    if (recenter && (z = wildcat::launch_key_mean(K, dtype, BH, n, d, L.mws, L.kbar, s)).code) return record(z);
+    wildcat::SelectRequest sq{K, dtype, BB, nb, d, beta_key, rb, seed, inst0 * nbins, eps, nullptr, L.S, L.F, L.rank_b,
+                              L.K_S, L.kbar, nbins};
     if ((z = wildcat::launch_select(sq, s)).code) return record(z);
     wildcat::WeightsRequest wq{L.F, L.S, L.rank_b, V, dtype, BB, nb, d, rb, L.V_S, L.w, L.vmin_b, L.vmax_b, L.wws,
                                L.wws_bytes};
@@ -361,11 +376,27 @@ wildcat_status wildcat_forward_binned(const void* Q, const void* K, const void* 
                                             L.rank_att, S_out, rank_out, s)).code)
         return record(z);
     if (m > 0) {
+        // the attend is unchanged by recentring and temperature: it uses the
+        // original pivot keys and beta (the shift and 1/tau cancel in N / D)
         wildcat::AttendRequest aq{Q,      L.K_S,  dtype, BH, m, d, r, L.rank_att, beta, L.V_S, L.w,
                                   L.vmin, L.vmax, O,     L.aws, L.aws_bytes};
         if ((z = wildcat::launch_attend(aq, s)).code) return record(z);
     }
     return record(Status::ok());
+}
+
+size_t wildcat_forward_binned_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int nbins, int dtype) {
+    const wildcat_options o{nbins, 0, 1.f};
+    return wildcat_forward_ex_workspace_size(BH, m, n, d, r, dtype, &o);
+}
+
+wildcat_status wildcat_forward_binned(const void* Q, const void* K, const void* V, int dtype, int64_t BH, int64_t m,
+                                      int64_t n, int d, float beta, int r, int nbins, uint64_t seed, int64_t inst0,
+                                      float eps, float* O, int32_t* S_out, int32_t* rank_out, void* workspace,
+                                      size_t ws_bytes, void* stream) {
+    const wildcat_options o{nbins, 0, 1.f};
+    return wildcat_forward_ex(Q, K, V, dtype, BH, m, n, d, beta, r, seed, inst0, eps, &o, O, S_out, rank_out,
+                              workspace, ws_bytes, stream);
 }
 
 size_t wildcat_forward_host_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int dtype) {

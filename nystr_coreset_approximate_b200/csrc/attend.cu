@@ -26,22 +26,26 @@ constexpr int kNormThreads = 256;
 template <typename E, int D>
 __global__ void __launch_bounds__(kNormThreads) qnorm_partial(const typename E::T* Q, int64_t m,
                                                               int64_t rows_per_split, float* part) {
-    // part [BH, nsplit]: max |q_i| over a slice of the queries (one warp per row)
+    // part [BH, nsplit]: max |q_i| over a slice of the queries; one thread
+    // per row with independent 16-byte loads (no per-row reduction chain)
     const int64_t b = blockIdx.y;
     const int split = blockIdx.x, nsplit = gridDim.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t i0 = split * rows_per_split, i1 = std::min<int64_t>(m, i0 + rows_per_split);
     float best = 0.f;
-    for (int64_t i = i0 + warp; i < i1; i += kNormThreads / 32) {
+    for (int64_t i = i0 + threadIdx.x; i < i1; i += kNormThreads) {
         const typename E::T* q = Q + (b * m + i) * D;
         float s = 0.f;
-        for (int c = lane; c < D; c += 32) {
-            const float v = E::to_float(q[c]);
-            s = fmaf(v, v, s);
+#pragma unroll
+        for (int c = 0; c < D; c += 8) {
+            float v[8];
+            load8(q + c, v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s = fmaf(v[e], v[e], s);
         }
-        s = warp_sum(s);
         best = fmaxf(best, sqrtf(s));
     }
+    best = warp_max(best);
     __shared__ float wb[kNormThreads / 32];
     if (lane == 0) wb[warp] = best;
     __syncthreads();

@@ -4,18 +4,28 @@
 // estimator and Alg. 3 WtdAttn, for bfloat16 inputs:
 //     P = exp(beta Q K_S^T - beta M_Q),   N = P [V_S | w],   O = clip(N_v / N_w).
 //
-// One CTA (128 threads) per tile of 128 queries of one instance.  Per chunk
-// of 128 coreset rows:
+// One CTA (256 threads; two per query row, splitting its columns) per tile
+// of 128 queries of one instance.  Per chunk
+// of 64 coreset rows:
 //   GEMM1  S = Q K_S^T     tcgen05.mma kind::f16 (bf16 x bf16 -> fp32 in TMEM),
-//                          M = 128, N = 128, K = d
-//   exp    thread i (= TMEM lane i = query row i) loads its row of S with
-//          tcgen05.ld, forms P = exp(beta s - beta M_Q) and writes it as
+//                          M = 128, N = 64, K = d
+//   exp    the two threads of query row i (TMEM lane i) load their halves
+//          of row i of S with tcgen05.ld, form P = exp(beta s - beta M_Q)
+//          (one exp2f of an fma; P is rounded to bf16 anyway) and write it as
 //          bf16 into shared memory in the UMMA K-major 128-byte-swizzled
 //          layout
 //   GEMM2  N += P [V_S | w]  with [V_S | w] split as hi + lo bf16 parts (two
-//          MMAs), M = 128, N = d + 16, K = 128, accumulated in TMEM across
+//          MMAs), M = 128, N = d + 16, K = 64, accumulated in TMEM across
 //          chunks.  The numerator and the denominator use the same rounded P.
 // Epilogue: thread i reads its row of N and writes O_i = clip(N_i / N_iw).
+//
+// Pipeline: the K_S / [V_S|w] chunks go through three shared-memory stages
+// (copies two chunks ahead), S has two tensor-memory buffers and P two
+// shared-memory buffers, so GEMM1 of chunk c + 1 runs while chunk c is
+// exponentiated and the copies of chunk c + 2 land while GEMM2 of chunk c
+// runs.  Barrier k of each pair completes once per two chunks; every wait
+// names the phase of the chunk it needs, which is always the barrier's most
+// recent or next phase.
 //
 // Operands are staged with cp.async into the swizzled layout (16-byte
 // chunk c of row r of an 8-row, 128-byte-wide atom sits at chunk c ^ (r % 8)).
@@ -34,23 +44,25 @@ __device__ int g_device_status = 0;  // WILDCAT_ERR_TIMEOUT when a bounded wait 
 namespace {
 
 using namespace tc;
-constexpr int kTcThreads = 128;
+constexpr int kTcThreads = 256;  // two threads per query row: each takes half of the columns
 unsigned long long g_force_timeout_ns = 0;  // test hook, 0 = off
-constexpr int kTcRC = 128;  // coreset rows per chunk
+constexpr int kTcRC = 64;  // coreset rows per chunk
 
 template <int D>
 struct TcSmem {
-    static constexpr int NE = D + 16;                         // value columns + w + zero padding
-    static constexpr int KB1 = D / 64;                        // 128-byte K blocks of Q / K_S rows
-    static constexpr int KB2 = kTcRC / 64;                    // 128-byte K blocks of P / [V_S|w]^T rows
-    static constexpr size_t a1 = 0;                           // Q tile    128 x D
-    static constexpr size_t b1 = a1 + (size_t)KB1 * 128 * 128;  // K_S chunk 128 x D
-    static constexpr size_t a2 = b1 + (size_t)KB1 * 128 * 128;  // P         128 x 128
-    static constexpr size_t b2h = a2 + (size_t)KB2 * 128 * 128; // [V_S|w]^T hi  NE x 128
-    static constexpr size_t b2l = b2h + (size_t)KB2 * NE * 128;
-    static constexpr size_t bar = b2l + (size_t)KB2 * NE * 128;  // 2 mbarriers + TMEM base
-    static constexpr size_t total = bar + 64 + 1024;            // + slack for 1024-byte alignment
-    static constexpr unsigned tmem_cols = (128 + NE) <= 256 ? 256u : 512u;
+    static constexpr int NE = D + 16;                           // value columns + w + zero padding
+    static constexpr int KB1 = D / 64;                          // 128-byte K blocks of Q / K_S rows
+    static constexpr int NSTAGE = 3;                            // K_S / [V_S|w] chunk stages
+    static constexpr size_t a1 = 0;                             // Q tile 128 x D
+    static constexpr size_t b1_bytes = (size_t)KB1 * kTcRC * 128;  // K_S chunk  RC x D
+    static constexpr size_t b2_bytes = (size_t)NE * 128;           // [V_S|w]^T  NE x RC (one 128-byte K block)
+    static constexpr size_t stage_bytes = b1_bytes + 2 * b2_bytes;
+    static constexpr size_t stages = a1 + (size_t)KB1 * 128 * 128;
+    static constexpr size_t a2 = stages + NSTAGE * stage_bytes;   // P, two buffers of 128 x RC
+    static constexpr size_t a2_bytes = 128 * 128;
+    static constexpr size_t bar = a2 + 2 * a2_bytes;              // 4 mbarriers + TMEM base
+    static constexpr size_t total = bar + 64 + 1024;              // + slack for 1024-byte alignment
+    static constexpr unsigned tmem_cols = (2 * kTcRC + NE) <= 256 ? 256u : 512u;
 };
 
 template <int D>
@@ -64,20 +76,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr int NE = L::NE;
     extern __shared__ unsigned char sm_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
-    const unsigned sA1 = smem_u32(sm + L::a1), sB1 = smem_u32(sm + L::b1), sA2 = smem_u32(sm + L::a2);
-    const unsigned sB2h = smem_u32(sm + L::b2h), sB2l = smem_u32(sm + L::b2l);
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + L::bar);
-    unsigned* tmem_base_slot = reinterpret_cast<unsigned*>(sm + L::bar + 16);
+    const unsigned sbase = smem_u32(sm);
+    const unsigned sA1 = sbase + L::a1;
+    uint64_t* mbS = reinterpret_cast<uint64_t*>(sm + L::bar);       // GEMM1 done, per S buffer
+    uint64_t* mbG = mbS + 2;                                        // GEMM2 done, per P buffer
+    unsigned* tmem_base_slot = reinterpret_cast<unsigned*>(sm + L::bar + 32);
 
     const int tid = threadIdx.x, warp = tid >> 5;
+    const int row = tid & 127, half = tid >> 7;  // query row (= TMEM lane) and column half
     const int64_t b = blockIdx.y;
     const int64_t i0 = (int64_t)blockIdx.x * 128;
     const int rr = rank[b];
-    const float shift = beta * MQ[b];
+    const int nch = (rr + kTcRC - 1) / kTcRC;
+    // P = exp(beta s - beta M_Q) = 2^(s * beta log2 e - beta M_Q log2 e); P is
+    // rounded to bf16 (8 significant bits), so exp2f's accuracy is ample
+    const float bl2e = beta * 1.4426950408889634f;
+    const float sl2e = beta * MQ[b] * 1.4426950408889634f;
 
     if (tid == 0) {
-        mbar_init(&mbar[0], 1);
-        mbar_init(&mbar[1], 1);
+        for (int k = 0; k < 4; ++k) mbar_init(&mbS[k], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -86,111 +103,149 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    // Q tile: row tid, D/8 chunks of 16 bytes
+    auto stage_addr = [&](int st) { return sbase + (unsigned)(L::stages + (size_t)st * L::stage_bytes); };
+    // copies of chunk c (rows l0 .. l0 + RC of K_S and of [V_S|w]^T hi / lo) into stage c % 3
+    auto load_chunk = [&](int c) {
+        const unsigned sb = stage_addr(c % L::NSTAGE);
+        const int l0 = c * kTcRC;
+        for (int e = tid; e < kTcRC * (D / 8); e += kTcThreads) {
+            const int row = e / (D / 8), cc = e % (D / 8);
+            const int l = l0 + row;
+            const bool ok = l < rr;
+            const __nv_bfloat16* src = K_S + ((b * r + (ok ? l : 0)) * (int64_t)D) + cc * 8;
+            cp_async16_zfill(sb + (cc >> 3) * (kTcRC * 128) + swz(row, cc & 7), src, ok);
+        }
+        for (int e = tid; e < NE * (kTcRC / 8); e += kTcThreads) {
+            const int row = e / (kTcRC / 8), cc = e % (kTcRC / 8);
+            const int64_t off = ((b * NE + row) * (int64_t)rpad) + l0 + cc * 8;
+            const unsigned dst = swz(row, cc);
+            cp_async16_zfill(sb + L::b1_bytes + dst, B2h + off, true);
+            cp_async16_zfill(sb + L::b1_bytes + L::b2_bytes + dst, B2l + off, true);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    // Q tile: row `row`, this thread's half of its 16-byte chunks
     {
-        const int64_t i = i0 + tid;
+        const int64_t i = i0 + row;
         const bool ok = i < m;
         const __nv_bfloat16* src = Q + ((b * m + (ok ? i : 0)) * D);
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c)
-            cp_async16_zfill(sA1 + (c >> 3) * (128 * 128) + swz(tid, c & 7), src + c * 8, ok);
+        for (int c = half * (D / 16); c < (half + 1) * (D / 16); ++c)
+            cp_async16_zfill(sA1 + (c >> 3) * (128 * 128) + swz(row, c & 7), src + c * 8, ok);
     }
+    if (nch > 0) load_chunk(0);  // committed together with the Q tile
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+    if (nch > 1) load_chunk(1);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const unsigned tmem = *tmem_base_slot;
-    const unsigned tmem_S = tmem, tmem_N = tmem + 128;
-    const unsigned lane_off = (unsigned)(warp * 32) << 16;
+    const unsigned tmem_N = tmem + 2 * kTcRC;
+    const unsigned lane_off = (unsigned)((warp & 3) * 32) << 16;  // warps w and w + 4 share lanes
     constexpr uint32_t id1 = idesc_bf16(128, kTcRC), id2 = idesc_bf16(128, NE);
 
-    bool ok = true;
-    int chunk = 0;
-    if (force_timeout_ns) {
-        // test hook: wait for a barrier phase that nothing will complete
-        const bool w = mbar_wait(&mbar[1], 0, force_timeout_ns);
-        if (__syncthreads_or(!w)) ok = false;
-    }
-    for (int l0 = 0; ok && l0 < rr; l0 += kTcRC, ++chunk) {
-        // -- stage K_S chunk (row tid) and the hi/lo [V_S|w]^T chunk --
-        {
-            const int l = l0 + tid;
-            const bool okr = l < rr;
-            const __nv_bfloat16* src = K_S + ((b * r + (okr ? l : 0)) * (int64_t)D);
-#pragma unroll
-            for (int c = 0; c < D / 8; ++c)
-                cp_async16_zfill(sB1 + (c >> 3) * (128 * 128) + swz(tid, c & 7), src + c * 8, okr);
-            for (int e = tid; e < NE * (kTcRC / 8); e += kTcThreads) {
-                const int row = e / (kTcRC / 8), c = e % (kTcRC / 8);
-                const int64_t off = ((b * NE + row) * (int64_t)rpad) + l0 + c * 8;
-                const unsigned dst = (c >> 3) * (NE * 128) + swz(row, c & 7);
-                cp_async16_zfill(sB2h + dst, B2h + off, true);
-                cp_async16_zfill(sB2l + dst, B2l + off, true);
-            }
-            cp_async_wait_all();
-            fence_async_smem();
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // -- GEMM1: S = Q K_S^T --
-        if (tid == 0) {
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const unsigned off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-                mma_bf16(tmem_S, umma_desc(sA1 + off), umma_desc(sB1 + off), id1, kk > 0);
-            }
-            mma_commit(&mbar[0]);
-        }
-        const bool w1 = mbar_wait(&mbar[0], chunk & 1);
-        if (__syncthreads_or(!w1)) { ok = false; break; }
-        tc_fence_after();
-        // -- P = exp(beta s - beta M_Q) in bf16, written as the K-major A operand of GEMM2 --
-#pragma unroll 1
-        for (int c0 = 0; c0 < kTcRC; c0 += 16) {
-            float v[16];
-            tmem_ld16(tmem_S + lane_off + c0, v);
-            uint32_t pk[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int l = l0 + c0 + 2 * k;
-                const float p0 = l < rr ? expf(beta * v[2 * k] - shift) : 0.f;
-                const float p1 = l + 1 < rr ? expf(beta * v[2 * k + 1] - shift) : 0.f;
-                const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                pk[k] = *reinterpret_cast<const uint32_t*>(&h);
-            }
-            const int cc = c0 >> 3;  // 16-byte chunk index along the 128 coreset columns
-            unsigned char* base = sm + L::a2 + (cc >> 3) * (128 * 128);
-            *reinterpret_cast<uint4*>(base + swz(tid, cc & 7)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            *reinterpret_cast<uint4*>(base + swz(tid, (cc + 1) & 7)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-        }
+    // make the copies of chunk c visible to the tensor cores (all threads)
+    auto publish_copies = [&](bool one_more_pending) {
+        if (one_more_pending) asm volatile("cp.async.wait_group 1;" ::: "memory");
+        else asm volatile("cp.async.wait_group 0;" ::: "memory");
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // -- GEMM2: N += P [V_S|w] (hi and lo parts) --
+    };
+    auto issue_gemm1 = [&](int c) {
         if (tid == 0) {
+            const unsigned sb = stage_addr(c % L::NSTAGE);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const unsigned oa = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+                const unsigned ob = (kk >> 2) * (kTcRC * 128) + (kk & 3) * 32;
+                mma_bf16(tmem + (c & 1) * kTcRC, umma_desc(sA1 + oa), umma_desc(sb + ob), id1, kk > 0);
+            }
+            mma_commit(&mbS[c & 1]);
+        }
+    };
+
+    bool ok = true;
+    if (force_timeout_ns) {
+        // test hook: wait for a barrier phase that nothing will complete
+        const bool w = mbar_wait(&mbG[0], 0, force_timeout_ns);
+        if (__syncthreads_or(!w)) ok = false;
+    }
+    if (ok && nch > 0) {
+        publish_copies(nch > 1);
+        issue_gemm1(0);
+    }
+    int c = 0;
+    for (; ok && c < nch; ++c) {
+        // (1) copies of chunk c + 2 into the stage chunk c - 1 used, once GEMM2(c - 1) has read it
+        if (c + 2 < nch) {
+            if (c >= 1) {
+                const bool w = mbar_wait(&mbG[(c - 1) & 1], ((c - 1) >> 1) & 1);
+                if (__syncthreads_or(!w)) { ok = false; break; }
+            }
+            load_chunk(c + 2);
+        }
+        // (2) GEMM1 of chunk c + 1 runs on the tensor cores while this chunk is exponentiated
+        if (c + 1 < nch) {
+            publish_copies(c + 2 < nch);
+            issue_gemm1(c + 1);
+        }
+        // (3) P = exp(beta s - beta M_Q) of chunk c, rounded once to bf16
+        const bool w1 = mbar_wait(&mbS[c & 1], (c >> 1) & 1);
+        if (__syncthreads_or(!w1)) { ok = false; break; }
+        tc_fence_after();
+        constexpr int HC = kTcRC / 2;  // columns per thread
+        uint32_t pk[HC / 2];
+#pragma unroll
+        for (int c0 = 0; c0 < HC; c0 += 16) {
+            float v[16];
+            tmem_ld16(tmem + (c & 1) * kTcRC + lane_off + half * HC + c0, v);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int l = c * kTcRC + half * HC + c0 + 2 * k;
+                const float p0 = l < rr ? exp2f(fmaf(v[2 * k], bl2e, -sl2e)) : 0.f;
+                const float p1 = l + 1 < rr ? exp2f(fmaf(v[2 * k + 1], bl2e, -sl2e)) : 0.f;
+                const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                pk[c0 / 2 + k] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+        }
+        if (c >= 2) {  // GEMM2(c - 2) has finished reading this P buffer
+            const bool w = mbar_wait(&mbG[c & 1], ((c - 2) >> 1) & 1);
+            if (__syncthreads_or(!w)) { ok = false; break; }
+        }
+        unsigned char* pa = sm + L::a2 + (c & 1) * L::a2_bytes;
+#pragma unroll
+        for (int cc = 0; cc < HC / 8; ++cc)
+            *reinterpret_cast<uint4*>(pa + swz(row, half * (HC / 8) + cc)) =
+                make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        // (4) GEMM2: N += P [V_S|w] (hi and lo parts)
+        if (tid == 0) {
+            const unsigned sA2 = sbase + (unsigned)(L::a2 + (c & 1) * L::a2_bytes);
+            const unsigned sb = stage_addr(c % L::NSTAGE) + (unsigned)L::b1_bytes;
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
-                const unsigned sb = part ? sB2l : sB2h;
 #pragma unroll
-                for (int kk = 0; kk < kTcRC / 16; ++kk) {
-                    const unsigned offa = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-                    const unsigned offb = (kk >> 2) * (NE * 128) + (kk & 3) * 32;
-                    mma_bf16(tmem_N, umma_desc(sA2 + offa), umma_desc(sb + offb), id2,
-                             (chunk > 0 || part > 0 || kk > 0) ? 1 : 0);
-                }
+                for (int kk = 0; kk < kTcRC / 16; ++kk)
+                    mma_bf16(tmem_N, umma_desc(sA2 + kk * 32), umma_desc(sb + part * L::b2_bytes + kk * 32), id2,
+                             (c > 0 || part > 0 || kk > 0) ? 1 : 0);
             }
-            mma_commit(&mbar[1]);
+            mma_commit(&mbG[c & 1]);
         }
-        const bool w2 = mbar_wait(&mbar[1], chunk & 1);
-        if (__syncthreads_or(!w2)) { ok = false; break; }
+    }
+    if (ok && nch > 0) {  // the last GEMM2 before reading N
+        const bool w = mbar_wait(&mbG[(nch - 1) & 1], ((nch - 1) >> 1) & 1);
+        if (__syncthreads_or(!w)) ok = false;
         tc_fence_after();
     }
-
-    cp_async_wait_all();  // the Q tile when the loop did not run
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     // -- epilogue: O = clip(N_v / N_w).  tcgen05.ld is warp-collective, so
     //    every lane loads; only the stores depend on the row being < m. --
-    const int64_t i = i0 + tid;
+    const int64_t i = i0 + row;
     const bool row_ok = i < m;
     if (ok) {
         float* o = O + (b * m + (row_ok ? i : 0)) * D;
@@ -198,13 +253,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const float* hi = vmax + b * D;
         if (rr == 0) {
             if (row_ok)
-                for (int c = 0; c < D; ++c) o[c] = lo[c];  // 0 / 0 clipped to v_min
+                for (int c2 = half * (D / 2); c2 < (half + 1) * (D / 2); ++c2) o[c2] = lo[c2];  // 0/0 -> v_min
         } else {
             float wv[16];
             tmem_ld16(tmem_N + lane_off + D, wv);
             const float den = wv[0];
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 16) {
+            for (int c0 = half * (D / 2); c0 < (half + 1) * (D / 2); c0 += 16) {
                 float v[16];
                 tmem_ld16(tmem_N + lane_off + c0, v);
                 if (row_ok) {
@@ -220,13 +275,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
             }
         }
-    } else if (tid == 0) {
-        atomicExch(&g_device_status, 5);
-    }
-    if (!ok && chunk > 0) {
-        // give outstanding tensor-core work one more bounded chance to retire
-        mbar_wait(&mbar[0], chunk & 1);
-        mbar_wait(&mbar[1], chunk & 1);
+    } else {
+        if (tid == 0) atomicExch(&g_device_status, 5);
+        // give issued tensor-core work one more bounded chance to retire
+        if (nch > 0 && !force_timeout_ns) {
+            mbar_wait(&mbS[0], 0, 100000000ull);
+            mbar_wait(&mbG[0], 0, 100000000ull);
+        }
     }
     tc_fence_before();
     __syncthreads();

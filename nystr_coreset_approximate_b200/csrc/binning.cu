@@ -9,7 +9,9 @@
 // the remaining glue: the value range over all n keys (the minimum and
 // maximum of the per-bin ranges), the attend's row count (all r union rows;
 // rows past a bin's rank are zero in K_S, V_S and w and contribute nothing),
-// and the optional global pivot indices and per-bin ranks.
+// and the optional global pivot indices and per-bin ranks.  It also holds the
+// per-instance key mean used for recentring (Sec. 2: softmax attention is
+// invariant under a global shift of the keys).
 #include "common.cuh"
 #include "internal.h"
 
@@ -43,7 +45,68 @@ __global__ void binning_finish_kernel(const float* vmin_b, const float* vmax_b, 
         for (int q = threadIdx.x; q < nbins; q += blockDim.x) rank_out[b * nbins + q] = rank_b[b * nbins + q];
 }
 
+constexpr int kMeanThreads = 256;
+
+template <typename E>
+__global__ void __launch_bounds__(kMeanThreads) key_mean_partial(const typename E::T* K, int64_t n, int d,
+                                                                 int64_t rows_per_split, double* part) {
+    // part [BH, nsplit, d]: fp64 column sums of a slice of the keys
+    const int64_t b = blockIdx.y;
+    const int split = blockIdx.x, nsplit = gridDim.x;
+    const int slots = kMeanThreads / d;
+    const int c = threadIdx.x % d, slot = threadIdx.x / d;
+    const int64_t l0 = split * rows_per_split, l1 = min(n, l0 + rows_per_split);
+    double acc = 0.0;
+    if (slot < slots)
+        for (int64_t l = l0 + slot; l < l1; l += slots) acc += (double)E::to_float(K[(b * n + l) * d + c]);
+    __shared__ double red[kMeanThreads];
+    red[threadIdx.x] = acc;
+    __syncthreads();
+    if (slot == 0) {
+        for (int k = 1; k < slots; ++k) acc += red[k * d + c];
+        part[(b * nsplit + split) * d + c] = acc;
+    }
+}
+
+__global__ void key_mean_finalize(const double* part, int nsplit, int64_t BH, int64_t n, int d, float* kbar) {
+    const int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (t >= BH * d) return;
+    const int64_t b = t / d;
+    const int c = (int)(t % d);
+    double s = 0.0;
+    for (int k = 0; k < nsplit; ++k) s += part[(b * nsplit + k) * d + c];
+    kbar[t] = (float)(s / (double)n);
+}
+
+int mean_splits(int64_t BH, int64_t n) {
+    int64_t s = ceil_div(296, BH > 0 ? BH : 1);
+    s = s < 1 ? 1 : (s > 64 ? 64 : s);
+    const int64_t cap = n / 256 > 0 ? n / 256 : 1;
+    return (int)(s < cap ? s : cap);
+}
+
 }  // namespace
+
+size_t key_mean_workspace_bytes(int64_t BH, int64_t n, int d) {
+    return sizeof(double) * (size_t)BH * mean_splits(BH, n) * d + 256;
+}
+
+Status launch_key_mean(const void* K, int dtype, int64_t BH, int64_t n, int d, void* ws, float* kbar,
+                       cudaStream_t st) {
+    const int nsplit = mean_splits(BH, n);
+    const int64_t rows = ceil_div(n, nsplit);
+    double* part = static_cast<double*>(ws);
+    if (dtype == 1)
+        key_mean_partial<BF16><<<dim3(nsplit, (unsigned)BH), kMeanThreads, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(K), n, d, rows, part);
+    else
+        key_mean_partial<F32><<<dim3(nsplit, (unsigned)BH), kMeanThreads, 0, st>>>(static_cast<const float*>(K), n,
+                                                                                   d, rows, part);
+    key_mean_finalize<<<(unsigned)ceil_div(BH * d, 256), 256, 0, st>>>(part, nsplit, BH, n, d, kbar);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return Status::cuda(e, "key mean launch");
+    return Status::ok();
+}
 
 Status launch_binning_finish(const float* vmin_b, const float* vmax_b, const int32_t* S_b, const int32_t* rank_b,
                              int64_t BH, int nbins, int64_t nb, int rb, int d, float* vmin, float* vmax,

@@ -32,6 +32,8 @@ struct SelectRequest {
     float* F;
     int32_t* rank;
     void* K_S;
+    const float* kbar = nullptr;  // recentring: per-instance key mean (or nullptr)
+    int kbar_div = 1;             // instance b uses kbar row b / kbar_div
 };
 
 Status launch_select(const SelectRequest& q, cudaStream_t stream);
@@ -117,6 +119,11 @@ struct DecodeRequest {
 };
 size_t decode_workspace_bytes(int64_t BH, int d);
 Status launch_decode(const DecodeRequest& q, cudaStream_t stream);
+
+// per-instance key mean (binning.cu), fp64 partial sums then fp32 mean
+size_t key_mean_workspace_bytes(int64_t BH, int64_t n, int d);
+Status launch_key_mean(const void* K, int dtype, int64_t BH, int64_t n, int d, void* ws, float* kbar,
+                       cudaStream_t st);
 
 // binned forward glue (binning.cu)
 Status launch_binning_finish(const float* vmin_b, const float* vmax_b, const int32_t* S_b, const int32_t* rank_b,

@@ -43,6 +43,8 @@ struct SelectArgs {
     int r;
     uint64_t seed;
     int64_t inst0;           // global index of instance 0 (Philox counter word 1 = inst0 + b)
+    const float* kbar;       // per-instance key mean subtracted from every key (or nullptr)
+    int kbar_div;            // instance b uses kbar row b / kbar_div (bins of one instance share it)
     float eps;
     const int32_t* S_fixed;  // nullptr: draw pivots
     int32_t* S;              // may be nullptr in fixed mode
@@ -155,6 +157,12 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     // copying 16 contiguous bytes, so a warp reads RPW whole rows per item;
     // items stream through the thread's cp.async ring.
     const T* kres = reinterpret_cast<const T*>(smem + L.kres);
+    // Recentring: every key enters as k - kbar (kbar = 0 without recentring,
+    // which leaves the arithmetic bit-identical).
+    float kbr[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e)
+        kbr[e] = a.kbar ? a.kbar[(b / a.kbar_div) * D + kl_part * EPL + e] : 0.f;
     auto key_pass = [&](const float* x, float* out) {
         float xr[EPL];
 #pragma unroll
@@ -179,6 +187,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                         v[0] = raw.x; v[1] = raw.y; v[2] = raw.z; v[3] = raw.w;
                     }
 #pragma unroll
+                    for (int e = 0; e < EPL; ++e) v[e] -= kbr[e];
+#pragma unroll
                     for (int e = 0; e < EPL; ++e) part = fmaf(v[e], x ? xr[e] : v[e], part);
                 }
 #pragma unroll
@@ -196,15 +206,22 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
             if (q < items && first + q * NW * RPW < nrows) cp_async16(ring4 + q * NT, src0 + q * step);
             cp_async_commit();
         }
+        // slot and source advance incrementally (no division or 64-bit multiply per item)
+        int slot_rd = 0, slot_wr = INFL;
+        const T* src_wr = src0 + INFL * step;
+        int row_wr = first + INFL * NW * RPW;
         for (int q = 0; q < items; ++q) {
-            const int qn = q + INFL;
-            if (qn < items && first + qn * NW * RPW < nrows) cp_async16(ring4 + (qn % DEPTH) * NT, src0 + qn * step);
+            if (q + INFL < items && row_wr < nrows) cp_async16(ring4 + slot_wr * NT, src_wr);
             cp_async_commit();
+            src_wr += step;
+            row_wr += NW * RPW;
+            slot_wr = slot_wr + 1 == DEPTH ? 0 : slot_wr + 1;
             cp_async_wait<INFL>();
             const int row = first + q * NW * RPW;
             float part = 0.f;
+            const float4 raw = ring4[slot_rd * NT];
+            slot_rd = slot_rd + 1 == DEPTH ? 0 : slot_rd + 1;
             if (row < nrows) {
-                const float4 raw = ring4[(q % DEPTH) * NT];
                 float v[EPL];
                 if constexpr (sizeof(T) == 2) {
                     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
@@ -217,6 +234,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                 } else {
                     v[0] = raw.x; v[1] = raw.y; v[2] = raw.z; v[3] = raw.w;
                 }
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) v[e] -= kbr[e];
 #pragma unroll
                 for (int e = 0; e < EPL; ++e) part = fmaf(v[e], x ? xr[e] : v[e], part);
             }
@@ -383,7 +402,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
 
         // -- pivot key and the pivot's row of the factor (loads issued together) --
         const T* kp = Kb + (int64_t)s * D;
-        for (int c = tid; c < D; c += NT) ks[c] = E::to_float(kp[c]);
+        for (int c = tid; c < D; c += NT)
+            ks[c] = E::to_float(kp[c]) - (a.kbar ? a.kbar[(b / a.kbar_div) * D + c] : 0.f);
         for (int j = tid; j < i; j += NT) fs[j] = ld_cg1(Fb + (int64_t)j * n + s);
         __syncthreads();
         // -- pivot residual g_s (warp 0, the same on every CTA) and <k_l, k_s> --
@@ -431,12 +451,16 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                         if (q < cnt) cp_async16(ring4 + q * NT, fcol + (int64_t)(j0 + q) * n);
                         cp_async_commit();
                     }
+                    int slot_rd = 0, slot_wr = INFL;
+                    const float* src_wr = fcol + (int64_t)(j0 + INFL) * n;
                     for (int q = 0; q < cnt; ++q) {
-                        const int qn = q + INFL;
-                        if (qn < cnt) cp_async16(ring4 + (qn % DEPTH) * NT, fcol + (int64_t)(j0 + qn) * n);
+                        if (q + INFL < cnt) cp_async16(ring4 + slot_wr * NT, src_wr);
                         cp_async_commit();
+                        src_wr += n;
+                        slot_wr = slot_wr + 1 == DEPTH ? 0 : slot_wr + 1;
                         cp_async_wait<INFL>();
-                        const float4 v = ring4[(q % DEPTH) * NT];
+                        const float4 v = ring4[slot_rd * NT];
+                        slot_rd = slot_rd + 1 == DEPTH ? 0 : slot_rd + 1;
                         const float f = fs[j0 + q];
                         acc[0] = fmaf(v.x, f, acc[0]);
                         acc[1] = fmaf(v.y, f, acc[1]);
@@ -673,6 +697,8 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     a.r = q.r;
     a.seed = q.seed;
     a.inst0 = q.inst0;
+    a.kbar = q.kbar;
+    a.kbar_div = q.kbar_div > 0 ? q.kbar_div : 1;
     a.eps = q.eps;
     a.S_fixed = q.S_fixed;
     a.S = q.S;

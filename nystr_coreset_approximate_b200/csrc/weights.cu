@@ -15,6 +15,7 @@
 //                tensor-core kernel of weights_tc.cu
 //   gather_fs    F_S[a, j] = F[j, S_a] for j <= a (pivot rows of the factor)
 //   trsm_kernel  sums the split-K partials and back-substitutes F_S^T X = Y
+//                (blocked by 32 pivots)
 #include <algorithm>
 
 #include "common.cuh"
@@ -142,14 +143,20 @@ __global__ void gather_fs(const float* F, const int32_t* S, const int32_t* rank,
     for (int j = threadIdx.x; j <= a; j += blockDim.x) dst[j] = __ldcg(F + (b * r + j) * n + s);
 }
 
-// Back substitution F_S^T X = Y for one instance and one block of CB right-hand columns.
+// Back substitution F_S^T X = Y for one instance and one block of CB
+// right-hand columns, blocked by 32 pivots: for each block of rows (bottom
+// up) all threads first subtract the contribution of the rows already
+// solved, then one warp solves the 32 x 32 diagonal block from shared
+// memory, one lane per column.  Two block barriers per 32 pivots.
 constexpr int kTrsmThreads = 256;
 constexpr int kTrsmCB = 16;
+constexpr int kTrsmBlk = 32;
 
 __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* Ypart, int nsplit, const float* FS,
                                                             const int32_t* rank, int64_t BH, int r, int D,
                                                             float* V_S, float* w) {
-    extern __shared__ float X[];  // [r][CB]
+    extern __shared__ float X[];  // [r][CB], then the diagonal block [32][33]
+    float* Ld = X + (size_t)r * kTrsmCB;
     const int64_t b = blockIdx.y;
     const int cb0 = blockIdx.x * kTrsmCB;
     const int DP = D + 1;
@@ -164,15 +171,32 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* Ypart, 
         X[a * kTrsmCB + c] = y;
     }
     __syncthreads();
-    const float* Lb = FS + b * (int64_t)r * r;
-    for (int ap = rr - 1; ap >= 0; --ap) {
-        const float* Lrow = Lb + (int64_t)ap * r;
-        const float xa = X[ap * kTrsmCB + c] / Lrow[ap];
-        for (int a = rs; a < ap; a += RS) X[a * kTrsmCB + c] = fmaf(-Lrow[a], xa, X[a * kTrsmCB + c]);
+    const float* Lb = FS + b * (int64_t)r * r;  // Lb[a' * r + a] = F_S[a', a], a <= a'
+    const int nblk = (rr + kTrsmBlk - 1) / kTrsmBlk;
+    for (int blk = nblk - 1; blk >= 0; --blk) {
+        const int a0 = blk * kTrsmBlk, a1 = min(rr, a0 + kTrsmBlk);
+        // (1) X[a] -= sum_{a' >= a1} F_S[a', a] X[a'] for the block's rows; stage the diagonal block
+        for (int a = a0 + rs; a < a1; a += RS) {
+            float acc = X[a * kTrsmCB + c];
+            for (int ap = a1; ap < rr; ++ap) acc = fmaf(-Lb[(int64_t)ap * r + a], X[ap * kTrsmCB + c], acc);
+            X[a * kTrsmCB + c] = acc;
+        }
+        for (int e = threadIdx.x; e < kTrsmBlk * kTrsmBlk; e += kTrsmThreads) {
+            const int i = e / kTrsmBlk, j = e % kTrsmBlk;  // Ld[i][j] = F_S[a0 + i, a0 + j]
+            Ld[i * (kTrsmBlk + 1) + j] = (a0 + i < a1 && j <= i) ? Lb[(int64_t)(a0 + i) * r + a0 + j] : 0.f;
+        }
         __syncthreads();
-        if (rs == 0) X[ap * kTrsmCB + c] = xa;
+        // (2) the diagonal block, bottom up, one lane per right-hand column
+        if (threadIdx.x < kTrsmCB) {
+            for (int i = a1 - a0 - 1; i >= 0; --i) {
+                const float xa = X[(a0 + i) * kTrsmCB + c] / Ld[i * (kTrsmBlk + 1) + i];
+                X[(a0 + i) * kTrsmCB + c] = xa;
+                for (int j = 0; j < i; ++j)
+                    X[(a0 + j) * kTrsmCB + c] = fmaf(-Ld[i * (kTrsmBlk + 1) + j], xa, X[(a0 + j) * kTrsmCB + c]);
+            }
+        }
+        __syncthreads();
     }
-    __syncthreads();
     if (col < DP) {
         for (int a = rs; a < r; a += RS) {
             const float v = a < rr ? X[a * kTrsmCB + c] : 0.f;
@@ -241,7 +265,7 @@ Status run_weights(const WeightsRequest& q, cudaStream_t st) {
             q.F, V, q.n, q.r, p.keys_per_split, Ypart, q.BH, q.rank);
     }
     gather_fs<<<dim3(q.r, (unsigned)q.BH), 128, 0, st>>>(q.F, q.S, q.rank, q.n, q.r, FS);
-    const size_t smem = sizeof(float) * (size_t)q.r * kTrsmCB;
+    const size_t smem = sizeof(float) * ((size_t)q.r * kTrsmCB + kTrsmBlk * (kTrsmBlk + 1));
     cudaError_t e = cudaFuncSetAttribute(trsm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return Status::cuda(e, "weights: trsm smem attribute");
     trsm_kernel<<<dim3((unsigned)ceil_div(D + 1, kTrsmCB), (unsigned)q.BH), kTrsmThreads, smem, st>>>(
@@ -263,7 +287,7 @@ size_t weights_workspace_bytes(int64_t BH, int64_t n, int d, int r) {
 }
 
 Status launch_weights(const WeightsRequest& q, cudaStream_t st) {
-    if ((size_t)q.r * kTrsmCB * sizeof(float) > 227 * 1024)
+    if (((size_t)q.r * kTrsmCB + kTrsmBlk * (kTrsmBlk + 1)) * sizeof(float) > 227 * 1024)
         return Status::fail(2, "weights: r too large for the on-chip triangular solve");
     const bool bf = q.dtype == 1;
     switch (q.d) {

@@ -83,6 +83,7 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_wildcat_forward_binned.argtypes = [_f64p, _f64p, _f64p, ctypes.c_int64,
                                                   ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                                                   ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.c_int, ctypes.c_double,
                                                   ctypes.c_uint64, ctypes.c_double, _i32p, _i64p,
                                                   ctypes.c_int64, _f64p, _i32p, _i32p]
     lib.oracle_wildcat_forward_binned.restype = ctypes.c_int
@@ -266,10 +267,12 @@ class Oracle:
 
 
     def wildcat_forward_binned(self, Q, K, V, beta, r, nbins, seed=0, eps=1e-6, rows=None,
-                               S_fixed=None):
+                               S_fixed=None, recenter=False, tau=1.0):
         """WildCat with divide-and-conquer binning (Sec. 2): nbins contiguous
         bins, r / nbins pivots each, block-diagonal weights, attend over the
-        union.  Returns (O_hat, S [BH, r] global key indices, rank [BH, nbins])."""
+        union; optionally on recentred keys and with temperature tau (key
+        kernel exp(beta <x,y> / tau^2)).  Returns (O_hat, S [BH, r] global
+        key indices, rank [BH, nbins])."""
         Q, qp = self._f64(Q)
         K, kp = self._f64(K)
         V, vp = self._f64(V)
@@ -281,8 +284,8 @@ class Oracle:
         rank = np.zeros((BH, nbins), dtype=np.int32)
         Sf, sfp = self._i32(S_fixed)
         err = self.lib.oracle_wildcat_forward_binned(
-            qp, kp, vp, BH, m, n, d, float(beta), int(r), int(nbins), int(seed), float(eps), sfp,
-            rp, nr,
+            qp, kp, vp, BH, m, n, d, float(beta), int(r), int(nbins), int(bool(recenter)),
+            float(tau), int(seed), float(eps), sfp, rp, nr,
             O.ctypes.data_as(_f64p), S.ctypes.data_as(_i32p), rank.ctypes.data_as(_i32p))
         if err == 2:
             raise ValueError("n and r must be multiples of nbins")

@@ -502,7 +502,8 @@ int oracle_wildcat_forward(const double* Q, const double* K, const double* V, in
 }
 
 /* ------------------------------------------------------------------------ */
-/* Divide and conquer (Sec. 2, binning): the n keys of an instance are cut   */
+/* Divide and conquer (Sec. 2, binning), with the optional recentring and   */
+/* temperature of Sec. 2: the n keys of an instance are cut                 */
 /* into nbins contiguous bins of n / nbins keys; each bin gets its own      */
 /* RPNys coreset of r / nbins pivots and its own Nystrom weights over its    */
 /* own keys (the pivot draws of bin q of instance b use instance index      */
@@ -517,10 +518,15 @@ int oracle_wildcat_forward(const double* Q, const double* K, const double* V, in
 /* ------------------------------------------------------------------------ */
 int oracle_wildcat_forward_binned(const double* Q, const double* K, const double* V, int64_t BH,
                                   int64_t m, int64_t n, int d, double beta, int r, int nbins,
-                                  uint64_t seed, double eps, const int32_t* S_fixed,
-                                  const int64_t* rows, int64_t nrows, double* O, int32_t* S_out,
-                                  int32_t* rank_out) {
-    if (nbins < 1 || n % nbins || r % nbins) return 2;
+                                  int recenter, double tau, uint64_t seed, double eps,
+                                  const int32_t* S_fixed, const int64_t* rows, int64_t nrows,
+                                  double* O, int32_t* S_out, int32_t* rank_out) {
+    if (nbins < 1 || n % nbins || r % nbins || !(tau > 0.0)) return 2;
+    /* Sec. 2: selection and weights use the recentred keys k_l - kbar and the
+     * key kernel exp(beta <x, y> / tau^2) (keys K / tau, queries tau Q); the
+     * output step uses the original keys and beta, which differs only by a
+     * per-query factor that cancels in N / D. */
+    const double beta_key = beta / (tau * tau);
     const int64_t nb = n / nbins;
     const int rb = r / nbins;
     const int64_t nr = rows ? nrows : m;
@@ -539,21 +545,31 @@ int oracle_wildcat_forward_binned(const double* Q, const double* K, const double
         double* N = (double*)malloc(sizeof(double) * (size_t)d);
         int32_t* Sb = (int32_t*)malloc(sizeof(int32_t) * (size_t)rb);
         int32_t* Sf = (int32_t*)malloc(sizeof(int32_t) * (size_t)rb);
-        if (!F || !dg || !g || !Y || !VS || !w || !KS || !vmin || !vmax || !N || !Sb || !Sf) {
+        double* Kc = (double*)malloc(sizeof(double) * (size_t)n * (size_t)d);
+        if (!F || !dg || !g || !Y || !VS || !w || !KS || !vmin || !vmax || !N || !Sb || !Sf || !Kc) {
 #pragma omp atomic write
             err = 1;
         } else {
             const double* Kb = K + b * n * d;
             const double* Vb = V + b * n * d;
+            for (int c = 0; c < d; ++c) {
+                double mean = 0.0;
+                if (recenter) {
+                    for (int64_t l = 0; l < n; ++l) mean += Kb[l * d + c];
+                    mean /= (double)n;
+                }
+                for (int64_t l = 0; l < n; ++l) Kc[l * d + c] = Kb[l * d + c] - mean;
+            }
             for (int q = 0; q < nbins; ++q) {
                 const double* Kq = Kb + (int64_t)q * nb * d;
+                const double* Kcq = Kc + (int64_t)q * nb * d;
                 const double* Vq = Vb + (int64_t)q * nb * d;
                 if (S_fixed)
                     for (int a = 0; a < rb; ++a) {
                         const int32_t sg = S_fixed[b * r + q * rb + a];
                         Sf[a] = (sg >= q * nb && sg < (q + 1) * nb) ? (int32_t)(sg - q * nb) : -1;
                     }
-                const int rr = rpc_one(Kq, nb, d, beta, rb, seed, b * nbins + q, eps, 1,
+                const int rr = rpc_one(Kcq, nb, d, beta_key, rb, seed, b * nbins + q, eps, 1,
                                        S_fixed ? Sf : NULL, Sb, F, NULL, NULL, dg, g);
                 if (rank_out) rank_out[b * nbins + q] = rr;
                 weights_one(F, Sb, rr, Vq, nb, d, rb, VS + (int64_t)q * rb * d, w + q * rb, Y);
@@ -573,7 +589,7 @@ int oracle_wildcat_forward_binned(const double* Q, const double* K, const double
             }
         }
         free(F); free(dg); free(g); free(Y); free(VS); free(w); free(KS);
-        free(vmin); free(vmax); free(N); free(Sb); free(Sf);
+        free(vmin); free(vmax); free(N); free(Sb); free(Sf); free(Kc);
     }
     return err;
 }

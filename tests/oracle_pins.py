@@ -387,6 +387,32 @@ def pin_decode_closed_form(o):
             np.testing.assert_allclose(O0[b, i], p @ Vn[b, :i + 1], rtol=0, atol=1e-12)
 
 
+# --------------------------------------------------------------------------- recentring / temperature
+def pin_recentring_and_temperature(o):
+    """Recentring and temperature (Sec. 2): with recenter off and tau = 1 the
+    options change nothing; the pivots with temperature tau are those of the
+    plain method on keys K / tau (key kernel exp(beta<x,y>/tau^2)); the
+    pivots with recentring are those of the plain method on K - mean(K)
+    (numpy); full-rank bins stay exact attention with both options on."""
+    Q, K, V = _rand(151, 2, 20, 48, 6, scale=1.2)
+    beta = 0.4
+    a = o.wildcat_forward_binned(Q, K, V, beta, 16, 2, seed=3)
+    b = o.wildcat_forward_binned(Q, K, V, beta, 16, 2, seed=3, recenter=False, tau=1.0)
+    np.testing.assert_array_equal(a[0], b[0])
+    tau = 1.7
+    _, S_t, _ = o.wildcat_forward_binned(Q, K, V, beta, 16, 1, seed=4, tau=tau)
+    _, S_k, _ = o.wildcat_forward(Q, K / tau, V, beta, 16, seed=4)
+    np.testing.assert_array_equal(S_t, S_k)
+    Kc = K - K.mean(axis=1, keepdims=True)
+    _, S_r, _ = o.wildcat_forward_binned(Q, K, V, beta, 16, 1, seed=5, recenter=True)
+    _, S_c, _ = o.wildcat_forward(Q, Kc, V, beta, 16, seed=5)
+    np.testing.assert_array_equal(S_r, S_c)
+    O, _, rank = o.wildcat_forward_binned(Q, K, V, beta, 48, 4, seed=6, eps=1e-14, recenter=True,
+                                          tau=1.3)
+    assert np.all(rank == 12)
+    np.testing.assert_allclose(O, o.exact_attention(Q, K, V, beta), rtol=0, atol=1e-11)
+
+
 ALL_PINS = [
     pin_exact_bruteforce,
     pin_full_rank_is_exact,
@@ -404,4 +430,5 @@ ALL_PINS = [
     pin_hand_examples,
     pin_binning_closed_forms,
     pin_decode_closed_form,
+    pin_recentring_and_temperature,
 ]
