@@ -61,6 +61,8 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--nbins", type=int, default=1,
                    help="divide-and-conquer bins (1 = the unbinned method)")
+    p.add_argument("--select-kernel", type=int, choices=[0, 1, 2], default=0,
+                   help="0 = automatic (the cp.async kernel), 1 = cp.async, 2 = bulk-copy where it applies")
     return p.parse_args()
 
 
@@ -96,24 +98,32 @@ def read_peaks():
         return 6650.0, "fallback"
 
 
-def kernel_source_hash():
+SELECT_KERNELS = {
+    # last_select_kernel() code -> (kernel name, profile prefix, source files)
+    1: ("rpc_select_kernel", "rpc_select", ("select.cu", "common.cuh", "philox.cuh")),
+    2: ("rpc_select_bulk_kernel", "rpc_select_bulk",
+        ("select_bulk.cu", "common.cuh", "philox.cuh", "tc_common.cuh")),
+}
+
+
+def kernel_source_hash(kind=1):
     h = hashlib.sha256()
-    for name in ("select.cu", "common.cuh", "philox.cuh"):
+    for name in SELECT_KERNELS[kind][2]:
         with open(os.path.join(ROOT, "nystr_coreset_approximate_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload_name):
+def recorded_traffic(workload_name, kind=1):
     """DRAM bytes per select launch from a committed ncu summary, if it was
     taken on the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", f"rpc_select_{workload_name}.md")
+    path = os.path.join(ROOT, "profiles", f"{SELECT_KERNELS[kind][1]}_{workload_name}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
     m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_hash or not m_tr or m_hash.group(1) != kernel_source_hash():
+    if not m_hash or not m_tr or m_hash.group(1) != kernel_source_hash(kind):
         return None
     return float(m_tr.group(1))
 
@@ -237,6 +247,7 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
+    wc.set_select_kernel(args.select_kernel)
     if world > 1:
         from datetime import timedelta
 
@@ -264,6 +275,8 @@ def main():
         plan.run(Q, K, V, w.beta, w.pivot_seed, EPS)
     torch.cuda.synchronize()
     ranks = plan.rank.reshape(-1).cpu().tolist()  # per instance (per bin when binned)
+    sel_kind = wc.last_select_kernel()
+    sel_cluster = wc.last_select_cluster()
 
     # ---- timed forward: K steps, own events per step, L2 flushed in between ----
     clocks = ClockSampler(local)
@@ -353,7 +366,7 @@ def main():
     peak, peak_kind = read_peaks()
     nbytes = select_bytes(w.scaled(n=w.n // nb), ranks)
     achieved = nbytes / (sel_ms / 1e3) / 1e9
-    traffic = recorded_traffic(w0.name if nb == 1 else f"{w0.name}_bins{nb}")
+    traffic = recorded_traffic(w0.name if nb == 1 else f"{w0.name}_bins{nb}", sel_kind)
     out = {
         "metric": METRIC, "value": value, "unit": "calls/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": total_ms / args.steps,
@@ -361,10 +374,12 @@ def main():
         "data": "synthetic",
         "config": workload_config(w0, {"l2": "flushed between steps (256 MiB device write)",
                                        "parallelism": f"instances per rank x {world} ranks",
-                                       "nbins": nb}),
+                                       "nbins": nb,
+                                       "select_kernel": SELECT_KERNELS[sel_kind][0],
+                                       "select_cluster_ctas": sel_cluster}),
         "entries_per_s": value * w.BH * w.m * w.n,
         "stages_ms": {k: statistics.mean(v) for k, v in stage_ms.items()},
-        "roofline": {"kernel": "rpc_select_kernel", "bound": "hbm", "achieved": achieved,
+        "roofline": {"kernel": SELECT_KERNELS[sel_kind][0], "bound": "hbm", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} hbm_gbs", "traffic": traffic,
                      "algorithmic_bytes_per_launch": nbytes, "launch_ms": sel_ms},

@@ -143,6 +143,32 @@ wildcat_status wildcat_weights(const float* F, const int32_t* S, const int32_t* 
                                size_t ws_bytes, void* stream);
 
 /*
+ * wildcat_weights_inverse -- the same outputs as wildcat_weights, through the
+ * inverse that RPNys maintains (Sec. 2): h(K_S, K_S)^-1 is grown pivot by
+ * pivot with the rank-one update (y = H_S^-1 b, sc = h(k_s, k_s) - b.y,
+ * H_S'^-1 = [[H_S^-1, 0], [0, 0]] + g g^T, g = (y, -1) / sqrt(sc)), then
+ * W (V, 1_n) = H_S^-1 h(K_S, K) (V, 1_n).  Equal to the factor route in exact
+ * arithmetic; provided to compare the two numerically.  fp64 arithmetic
+ * throughout from the inputs widened exactly; V_S and w are rounded to
+ * float32 at the end.  h carries the shift M = max_l |k_l|^2, which cancels.
+ *
+ *   K, V   [BH, n, d] keys and values, dtype `dtype`
+ *   S      [BH, r] int32 pivots in selection order; S[b, a] in [0, n) for
+ *          a < rank[b] (as written by wildcat_select; not checked on the device)
+ *   rank   [BH] int32 effective ranks, 0 <= rank[b] <= r
+ *   beta   the kernel's beta (> 0)
+ *   V_S, w, vmin, vmax   outputs as wildcat_weights (rows >= rank[b] zero)
+ *   workspace >= wildcat_weights_inverse_workspace_size(BH, n, d, r) bytes,
+ *          256-byte aligned; about 16 BH r^2 bytes (two r x r fp64 arrays)
+ * Returns WILDCAT_ERR_UNSUPPORTED for r > 2048 (the size query returns 0).
+ */
+size_t wildcat_weights_inverse_workspace_size(int64_t BH, int64_t n, int d, int r);
+wildcat_status wildcat_weights_inverse(const void* K, const void* V, int dtype, const int32_t* S,
+                                       const int32_t* rank, int64_t BH, int64_t n, int d, int r,
+                                       float beta, float* V_S, float* w, float* vmin, float* vmax,
+                                       void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * wildcat_attend -- weighted-coreset attention (Alg. 3 WtdAttn):
  *   u_il = exp(beta <q_i, k_S_l> - beta M_Q),  M_Q = max_i |q_i| * max_l |k_S_l|
  *   O_hat_ij = fminf(fmaxf(sum_l u_il V_S[l, j] / sum_l u_il w_l, vmin_j), vmax_j)
@@ -320,10 +346,13 @@ wildcat_status wildcat_pivot_uniforms(uint64_t seed, int64_t BH, int steps, doub
 
 /*
  * wildcat_get_device_status -- waits for `stream`, then reports and clears
- * the device status word of the current device.  Kernels that wait on the
- * tensor cores (mbarrier waits) bound every wait by a time limit; when one
- * expires the kernel records WILDCAT_ERR_TIMEOUT there, stops issuing work,
- * releases its tensor memory and returns, leaving its output incomplete.
+ * the device status words of the current device.  Kernels that wait on
+ * mbarriers (the tensor-core weights and attend, the bulk-copy select) bound
+ * every wait by a time limit; when one expires the kernel records
+ * WILDCAT_ERR_TIMEOUT there, stops issuing work, waits (bounded) for its
+ * copies in flight, releases its tensor memory and returns, leaving its
+ * output incomplete (the select stops every CTA of the instance at the same
+ * step and reports the steps taken as the rank).
  * Returns WILDCAT_OK, WILDCAT_ERR_TIMEOUT, or WILDCAT_ERR_CUDA if the stream
  * or the status word could not be read.
  */
@@ -340,9 +369,38 @@ wildcat_status wildcat_get_device_status(void* stream);
 wildcat_status wildcat_test_force_wait_timeout(int64_t nanoseconds);
 
 /*
+ * wildcat_test_force_select_timeout -- test hook for the bounded waits of
+ * the bulk-copy select kernel.  With nanoseconds > 0 every later launch of
+ * that kernel waits that long, after step 1, on a barrier phase that nothing
+ * completes; the expiry is handled like any other (WILDCAT_ERR_TIMEOUT in
+ * the device status word, every instance stops after two steps).  0 turns
+ * the hook off.  Process-wide; for tests only.  Returns
+ * WILDCAT_ERR_INVALID_ARG outside [0, 1e9].
+ */
+wildcat_status wildcat_test_force_select_timeout(int64_t nanoseconds);
+
+/*
+ * wildcat_set_select_kernel -- which select kernel wildcat_select* launch:
+ * 0 (default) and 1 the cp.async kernel (per-thread asynchronous copies);
+ * 2 the bulk-copy kernel (copy-engine stages on mbarriers) wherever it
+ * applies (n % 4 == 0, n / cluster size <= 8192, 16-byte aligned K and F,
+ * d in {32, 64, 128}), else the cp.async kernel.  Both compute the same
+ * factorisation (results agree to float32 rounding).  Process-wide; not
+ * thread-safe against concurrent select calls.  Returns
+ * WILDCAT_ERR_INVALID_ARG for other values.
+ */
+wildcat_status wildcat_set_select_kernel(int kernel);
+
+/* The select kernel the last select launch on this thread used: 1 the
+ * cp.async kernel, 2 the bulk-copy kernel, 0 if none. */
+int wildcat_last_select_kernel(void);
+
+/*
  * wildcat_set_select_cluster -- tuning knob for wildcat_select*: number of
  * CTAs (a thread-block cluster, 1..16, power of two) that share one
- * instance.  0 restores the automatic choice.  Process-wide; not thread-safe
+ * instance.  0 restores the automatic choice: the G with the least
+ * ceil(BH / clusters that fit at once) * ceil(n / G), from the occupancy
+ * API (a 16-CTA cluster needs 16 SMs of one GPC, so few of them fit).  Process-wide; not thread-safe
  * against concurrent select calls.  Returns WILDCAT_ERR_INVALID_ARG for
  * other values.
  */

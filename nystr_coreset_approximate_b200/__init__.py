@@ -24,8 +24,9 @@ from typing import Optional
 
 __all__ = [
     "WildcatError", "library_path", "lib", "declared_symbols", "select", "select_fixed",
-    "weights", "attend", "attend_noalloc", "decode_attend", "forward", "forward_ex", "Options", "forward_binned", "BinnedForwardPlan", "forward_host", "ForwardPlan", "pivot_uniforms",
-    "set_select_cluster", "last_select_cluster", "device_status", "DTYPES",
+    "weights", "weights_inverse", "attend", "attend_noalloc", "decode_attend", "forward", "forward_ex", "Options", "forward_binned", "BinnedForwardPlan", "forward_host", "ForwardPlan", "pivot_uniforms",
+    "set_select_cluster", "last_select_cluster", "set_select_kernel", "last_select_kernel",
+    "force_select_timeout", "device_status", "DTYPES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -51,6 +52,9 @@ _SIGS = {
     "wildcat_weights_workspace_size": ([_i64, _i64, _int, _int], _sz),
     "wildcat_weights": ([_vp, _vp, _vp, _vp, _int, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _sz,
                          _vp], _int),
+    "wildcat_weights_inverse_workspace_size": ([_i64, _i64, _int, _int], _sz),
+    "wildcat_weights_inverse": ([_vp, _vp, _int, _vp, _vp, _i64, _i64, _int, _int, _f32, _vp, _vp, _vp,
+                                 _vp, _vp, _sz, _vp], _int),
     "wildcat_attend_workspace_size": ([_i64, _i64, _int, _int], _sz),
     "wildcat_attend": ([_vp, _vp, _int, _i64, _i64, _int, _int, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp,
                         _sz, _vp], _int),
@@ -76,6 +80,9 @@ _SIGS = {
     "wildcat_test_force_wait_timeout": ([_i64], _int),
     "wildcat_set_select_cluster": ([_int], _int),
     "wildcat_last_select_cluster": ([], _int),
+    "wildcat_test_force_select_timeout": ([_i64], _int),
+    "wildcat_set_select_kernel": ([_int], _int),
+    "wildcat_last_select_kernel": ([], _int),
 }
 
 
@@ -220,6 +227,30 @@ def weights(F, S, rank, V, *, stream=None):
                              _dev(rank, "rank", torch.int32), _dev(V, "V"), _dtype_code(V), BH, n, d,
                              r, _dev(V_S, "V_S"), _dev(w, "w"), _dev(vmin, "vmin"),
                              _dev(vmax, "vmax"), _dev(ws, "workspace"), nbytes, _stream(stream)))
+    return V_S, w, vmin, vmax
+
+
+def weights_inverse(K, S, rank, V, beta: float, *, stream=None):
+    """The Nystrom weights through the maintained inverse of h(K_S, K_S) (Sec. 2,
+    RPNys rank-one update), fp64 inside.  Same outputs as weights():
+    (V_S [BH,r,d], w [BH,r], vmin [BH,d], vmax [BH,d]), float32."""
+    torch = _torch()
+    BH, n, d = _shape3(V, "V")
+    r = S.shape[1]
+    dev = V.device
+    V_S = torch.empty((BH, r, d), dtype=torch.float32, device=dev)
+    w = torch.empty((BH, r), dtype=torch.float32, device=dev)
+    vmin = torch.empty((BH, d), dtype=torch.float32, device=dev)
+    vmax = torch.empty((BH, d), dtype=torch.float32, device=dev)
+    L = lib()
+    nbytes = int(L.wildcat_weights_inverse_workspace_size(BH, n, d, r))
+    if nbytes == 0:
+        raise ValueError("weights_inverse supports 1 <= r <= 2048")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    _check(L.wildcat_weights_inverse(_dev(K, "K"), _dev(V, "V"), _dtype_code(V), _dev(S, "S", torch.int32),
+                                     _dev(rank, "rank", torch.int32), BH, n, d, r, float(beta),
+                                     _dev(V_S, "V_S"), _dev(w, "w"), _dev(vmin, "vmin"), _dev(vmax, "vmax"),
+                                     _dev(ws, "workspace"), nbytes, _stream(stream)))
     return V_S, w, vmin, vmax
 
 
@@ -454,3 +485,20 @@ def set_select_cluster(G: int):
 
 def last_select_cluster() -> int:
     return int(lib().wildcat_last_select_cluster())
+
+
+def set_select_kernel(kernel: int):
+    """0 = automatic (the cp.async kernel), 1 = the cp.async kernel, 2 = the
+    bulk-copy kernel where it applies."""
+    _check(lib().wildcat_set_select_kernel(int(kernel)))
+
+
+def last_select_kernel() -> int:
+    """1 = the cp.async kernel, 2 = the bulk-copy kernel (last select launch)."""
+    return int(lib().wildcat_last_select_kernel())
+
+
+def force_select_timeout(nanoseconds: int):
+    """Test hook: the bulk-copy select kernel waits this long on a barrier
+    nothing completes (0 = off)."""
+    _check(lib().wildcat_test_force_select_timeout(int(nanoseconds)))

@@ -181,6 +181,17 @@ wildcat_status check_bins(int64_t BH, int64_t n, int r, int nbins, const char* w
 
 }  // namespace
 
+namespace wildcat {
+int read_device_status(bool clear) {
+    const int parts[3] = {read_attend_status(clear), read_weights_status(clear), read_select_status(clear)};
+    for (const int v : parts)
+        if (v < 0) return -1;
+    for (const int v : parts)
+        if (v) return v;
+    return 0;
+}
+}  // namespace wildcat
+
 extern "C" {
 
 int wildcat_version(void) { return 100; }
@@ -233,6 +244,30 @@ wildcat_status wildcat_weights(const float* F, const int32_t* S, const int32_t* 
     if (ws_bytes < wildcat::weights_workspace_bytes(BH, n, d, r)) return bad(4, "%s: workspace too small", who);
     wildcat::WeightsRequest q{F, S, rank, V, dtype, BH, n, d, r, V_S, w, vmin, vmax, workspace, ws_bytes};
     return record(wildcat::launch_weights(q, static_cast<cudaStream_t>(stream)));
+}
+
+size_t wildcat_weights_inverse_workspace_size(int64_t BH, int64_t n, int d, int r) {
+    if (BH < 0 || n < 1 || r < 1 || d < 1 || r > wildcat::kInverseMaxRank) return 0;
+    return wildcat::weights_inverse_workspace_bytes(BH, n, d, r);
+}
+
+wildcat_status wildcat_weights_inverse(const void* K, const void* V, int dtype, const int32_t* S,
+                                       const int32_t* rank, int64_t BH, int64_t n, int d, int r, float beta,
+                                       float* V_S, float* w, float* vmin, float* vmax, void* workspace,
+                                       size_t ws_bytes, void* stream) {
+    const char* who = "wildcat_weights_inverse";
+    wildcat_status st = check_common(dtype, BH, n, d, r, who);
+    if (st != WILDCAT_OK) return st;
+    if ((st = check_scalars(beta, 0.f, who)) != WILDCAT_OK) return st;
+    if (r > wildcat::kInverseMaxRank) return bad(2, "%s: r above 2048 is not supported", who);
+    if (BH == 0) return record(Status::ok());
+    if (!K || !V || !S || !rank || !V_S || !w || !vmin || !vmax || !workspace)
+        return bad(1, "%s: null pointer argument", who);
+    if (!aligned16(K) || !aligned16(V)) return bad(1, "%s: K and V must be 16-byte aligned", who);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
+    if (ws_bytes < wildcat::weights_inverse_workspace_bytes(BH, n, d, r)) return bad(4, "%s: workspace too small", who);
+    wildcat::WeightsInverseRequest q{K, V, dtype, S, rank, BH, n, d, r, beta, V_S, w, vmin, vmax, workspace, ws_bytes};
+    return record(wildcat::launch_weights_inverse(q, static_cast<cudaStream_t>(stream)));
 }
 
 size_t wildcat_attend_workspace_size(int64_t BH, int64_t m, int d, int r) {
@@ -478,6 +513,22 @@ wildcat_status wildcat_test_force_wait_timeout(int64_t nanoseconds) {
     wildcat::set_attend_force_timeout((unsigned long long)nanoseconds);
     return record(Status::ok());
 }
+
+wildcat_status wildcat_test_force_select_timeout(int64_t nanoseconds) {
+    if (nanoseconds < 0 || nanoseconds > 1000000000LL)
+        return bad(1, "%s: nanoseconds must be in [0, 1e9]", "wildcat_test_force_select_timeout");
+    wildcat::set_select_force_timeout((unsigned long long)nanoseconds);
+    return record(Status::ok());
+}
+
+wildcat_status wildcat_set_select_kernel(int kernel) {
+    if (kernel < 0 || kernel > 2)
+        return bad(1, "%s: kernel must be 0 (automatic), 1 (cp.async) or 2 (bulk-copy)", "wildcat_set_select_kernel");
+    wildcat::select_kernel_override(kernel);
+    return record(Status::ok());
+}
+
+int wildcat_last_select_kernel(void) { return wildcat::last_select_kernel(); }
 
 wildcat_status wildcat_set_select_cluster(int ctas_per_instance) {
     const int G = ctas_per_instance;

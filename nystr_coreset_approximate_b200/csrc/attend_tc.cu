@@ -347,7 +347,7 @@ Status launch_attend_tc(const AttendRequest& q, const float* MQ, void* b2ws, cud
 
 void set_attend_force_timeout(unsigned long long ns) { g_force_timeout_ns = ns; }
 
-int read_device_status(bool clear) {
+int read_attend_status(bool clear) {
     int v = 0;
     if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return -1;
     if (clear && v) {

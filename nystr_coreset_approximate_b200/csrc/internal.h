@@ -40,6 +40,22 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream);
 Status launch_pivot_uniforms(uint64_t seed, int64_t BH, int steps, double* u, cudaStream_t stream);
 int select_cluster_override(int G);  // G < 0: query only
 int last_select_cluster();
+int select_kernel_override(int k);  // k < 0: query only; 0 automatic, 1 the cp.async kernel, 2 the bulk-copy kernel
+int last_select_kernel();           // 1 cp.async kernel, 2 bulk-copy kernel
+// cluster-size choice shared by both select kernels (select.cu)
+struct ClusterKey {
+    int dev, kernel;
+    int64_t n, BH;
+    int r, d, dtype;
+    bool operator<(const ClusterKey& o) const;
+};
+int cached_cluster_lookup(const ClusterKey& key);   // 0 if absent
+void cached_cluster_store(const ClusterKey& key, int G);
+int choose_cluster_rows(int64_t n, int64_t BH, int (*fit)(int G, void* ctx), void* ctx);
+// bulk-copy select kernel (select_bulk.cu); *used = false when the shape is not one it handles.
+// G_override > 0 fixes the cluster size.
+Status launch_select_bulk(const SelectRequest& q, int G_override, cudaStream_t stream, bool* used, int* G_used);
+void set_select_force_timeout(unsigned long long ns);
 
 // ---- weights: Y = F^T (V, 1), then F_S^T X = Y ----
 struct WeightsRequest {
@@ -59,6 +75,30 @@ struct WeightsRequest {
 };
 size_t weights_workspace_bytes(int64_t BH, int64_t n, int d, int r);
 Status launch_weights(const WeightsRequest& q, cudaStream_t stream);
+// column-wise value range of V alone (the same kernels as launch_weights)
+size_t value_range_workspace_bytes(int64_t BH, int64_t n, int d);
+Status launch_value_range(const void* V, int dtype, int64_t BH, int64_t n, int d, float* vmin, float* vmax,
+                          void* ws, size_t ws_bytes, cudaStream_t stream);
+// weights through the maintained inverse of h(K_S, K_S) (weights_inverse.cu)
+struct WeightsInverseRequest {
+    const void* K;
+    const void* V;
+    int dtype;
+    const int32_t* S;
+    const int32_t* rank;
+    int64_t BH, n;
+    int d, r;
+    float beta;
+    float* V_S;
+    float* w;
+    float* vmin;
+    float* vmax;
+    void* ws;
+    size_t ws_bytes;
+};
+size_t weights_inverse_workspace_bytes(int64_t BH, int64_t n, int d, int r);
+Status launch_weights_inverse(const WeightsInverseRequest& q, cudaStream_t stream);
+constexpr int kInverseMaxRank = 2048;
 // tensor-core F^T (V, 1) partials (weights_tc.cu)
 bool weights_tc_supported(int dtype, int d, int64_t n);
 Status launch_weights_tc(const float* F, const void* V, const int32_t* rank, int64_t BH, int64_t n, int d, int r,
@@ -90,7 +130,10 @@ bool attend_tc_supported(int dtype, int d);
 size_t attend_tc_scratch_bytes(int64_t BH, int d, int r);
 Status launch_attend_tc(const AttendRequest& q, const float* MQ, void* b2_scratch, cudaStream_t stream);
 // device status word set by bounded waits that expired (0 = none); -1 if unreadable
-int read_device_status(bool clear);
+int read_device_status(bool clear);  // first non-zero of the per-file status words below
+int read_attend_status(bool clear);
+int read_weights_status(bool clear);
+int read_select_status(bool clear);
 // test hook: the tensor-core attend first waits `ns` nanoseconds on a barrier
 // that nothing completes, then reports a timeout (0 = off)
 void set_attend_force_timeout(unsigned long long ns);

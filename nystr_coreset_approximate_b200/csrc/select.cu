@@ -21,6 +21,9 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 #include "common.cuh"
 #include "internal.h"
@@ -643,11 +646,57 @@ int dispatch(const Variant& v, int dtype, int vec, int d, const SelectArgs* a, s
 }
 
 int g_cluster_override = 0;
+int g_kernel_override = 0;
 thread_local int g_last_cluster = 0;
+thread_local int g_last_kernel = 0;
 
 }  // namespace
 
 constexpr int kMaxRowsPerCta = 16384;
+
+// Memo of the automatic cluster size per device and shape (the occupancy
+// queries cost host time on every launch otherwise).
+bool ClusterKey::operator<(const ClusterKey& o) const {
+    return std::tie(dev, kernel, n, BH, r, d, dtype) < std::tie(o.dev, o.kernel, o.n, o.BH, o.r, o.d, o.dtype);
+}
+
+static std::mutex g_cluster_mu;
+static std::map<ClusterKey, int> g_cluster_memo;
+
+int cached_cluster_lookup(const ClusterKey& key) {
+    std::lock_guard<std::mutex> lock(g_cluster_mu);
+    const auto it = g_cluster_memo.find(key);
+    return it == g_cluster_memo.end() ? 0 : it->second;
+}
+
+void cached_cluster_store(const ClusterKey& key, int G) {
+    std::lock_guard<std::mutex> lock(g_cluster_mu);
+    g_cluster_memo[key] = G;
+}
+
+// Cluster size for one select launch.  Candidates are G in {1, 2, 4, 8, 16}
+// with at most kMaxRowsPerCta rows per CTA and at least 512 (unless G = 1);
+// fit(G) is the number of clusters of G CTAs that fit on the GPU at once
+// (0 = not schedulable).  The cost of G is the rows one CTA streams times
+// the waves of clusters, ceil(BH / fit) * ceil(n / G): a 16-CTA cluster must
+// sit inside one GPC, so fewer of them fit than the SM count suggests.
+int choose_cluster_rows(int64_t n, int64_t BH, int (*fit)(int G, void* ctx), void* ctx) {
+    int best = 0;
+    double best_cost = 0.0;
+    for (int g = 1; g <= 16; g *= 2) {
+        const int64_t rows = ceil_div(n, g);
+        if (rows > kMaxRowsPerCta) continue;
+        if (g > 1 && n / g < 512) break;
+        const int f = fit(g, ctx);
+        if (f <= 0) continue;
+        const double cost = (double)ceil_div(BH, f) * (double)rows;
+        if (best == 0 || cost < best_cost * 0.999) {
+            best = g;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
 
 int select_cluster_override(int G) {
     if (G < 0) return g_cluster_override;
@@ -655,6 +704,12 @@ int select_cluster_override(int G) {
     return G;
 }
 int last_select_cluster() { return g_last_cluster; }
+int select_kernel_override(int k) {
+    if (k < 0) return g_kernel_override;
+    g_kernel_override = k;
+    return k;
+}
+int last_select_kernel() { return g_last_kernel; }
 
 static void plan(int64_t n, int r, int d, int dtype, int G, int vec, SelectArgs* a, size_t* smem, Variant* v) {
     const int R = (int)round_up(ceil_div(n, G), 4);
@@ -686,8 +741,6 @@ static void plan(int64_t n, int r, int d, int dtype, int G, int vec, SelectArgs*
 }
 
 Status launch_select(const SelectRequest& q, cudaStream_t stream) {
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int vec = (q.n % 4 == 0) ? 4 : 1;
     SelectArgs a{};
     a.K = q.K;
@@ -706,26 +759,49 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     a.rank = q.rank;
     a.K_S = q.K_S;
 
-    int G;
-    if (g_cluster_override > 0) {
-        G = g_cluster_override;
-    } else {
-        G = 1;
-        while (G * 2 <= 16 && (int64_t)(G * 2) * q.BH <= sms && q.n / (G * 2) >= 512) G *= 2;
+    if (g_kernel_override == 2) {
+        // the bulk-copy kernel (select_bulk.cu) where its shape rules allow
+        bool used = false;
+        int G_used = 0;
+        const Status st = launch_select_bulk(q, g_cluster_override, stream, &used, &G_used);
+        if (used) {
+            if (st.code == 0) {
+                g_last_cluster = G_used;
+                g_last_kernel = 2;
+            }
+            return st;
+        }
     }
-    while (G < 16 && ceil_div(q.n, G) > kMaxRowsPerCta) G *= 2;
-    if (ceil_div(q.n, G) > kMaxRowsPerCta)
-        return Status::fail(2, "select: n / 16 exceeds the per-CTA row limit (16384)");
     size_t smem = 0;
     Variant var{};
-    if (g_cluster_override <= 0) {
-        // shrink until the cluster shape is schedulable
-        for (;;) {
-            plan(q.n, q.r, q.d, q.dtype, G, vec, &a, &smem, &var);
-            if (smem > kSmemCap) return Status::fail(2, "select: shared memory plan exceeds 227 KB");
-            if (dispatch(var, q.dtype, vec, q.d, nullptr, smem, stream, G, nullptr) > 0 || G == 1) break;
-            G /= 2;
+    int G = g_cluster_override;
+    if (G <= 0) {
+        // the cluster size with the least work per CTA times waves of clusters
+        int dev = 0;
+        cudaGetDevice(&dev);
+        const ClusterKey key{dev, 1, q.n, q.BH, q.r, q.d, q.dtype};
+        G = cached_cluster_lookup(key);
+        if (G <= 0) {
+            struct Ctx {
+                const SelectRequest* q;
+                const SelectArgs* a;
+                int vec;
+                cudaStream_t stream;
+            } ctx{&q, &a, vec, stream};
+            G = choose_cluster_rows(q.n, q.BH, [](int g, void* p) -> int {
+                const Ctx& c = *static_cast<const Ctx*>(p);
+                SelectArgs t = *c.a;
+                Variant v{};
+                size_t sm = 0;
+                plan(c.q->n, c.q->r, c.q->d, c.q->dtype, g, c.vec, &t, &sm, &v);
+                if (sm > kSmemCap) return 0;
+                return dispatch(v, c.q->dtype, c.vec, c.q->d, nullptr, sm, c.stream, g, nullptr);
+            }, &ctx);
+            if (G > 0) cached_cluster_store(key, G);
         }
+        if (G <= 0) return Status::fail(2, "select: no schedulable cluster shape (n / 16 above 16384 rows?)");
+    } else if (ceil_div(q.n, G) > kMaxRowsPerCta) {
+        return Status::fail(2, "select: n / G exceeds the per-CTA row limit (16384)");
     }
     plan(q.n, q.r, q.d, q.dtype, G, vec, &a, &smem, &var);
     if (smem > kSmemCap) return Status::fail(2, "select: shared memory plan exceeds 227 KB");
@@ -734,6 +810,7 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     if (err == cudaSuccess) err = cudaGetLastError();
     if (err != cudaSuccess) return Status::cuda(err, "select launch");
     g_last_cluster = G;
+    g_last_kernel = 1;
     return Status::ok();
 }
 

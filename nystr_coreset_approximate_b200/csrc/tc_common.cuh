@@ -64,21 +64,27 @@ __device__ __forceinline__ void mbar_init(void* mbar, unsigned count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(mbar)), "r"(count) : "memory");
 }
 
+__device__ __forceinline__ bool mbar_try(unsigned a, unsigned parity) {
+    unsigned done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // Bounded wait for the phase with the given parity; returns false on timeout.
+// The clock is read only once the phase is found incomplete.
 __device__ __forceinline__ bool mbar_wait(void* mbar, unsigned parity,
                                           unsigned long long limit_ns = kWaitLimitNs) {
     const unsigned a = smem_u32(mbar);
+    if (mbar_try(a, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (;;) {
-        unsigned done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(done)
-            : "r"(a), "r"(parity)
-            : "memory");
-        if (done) return true;
+        if (mbar_try(a, parity)) return true;
         if (globaltimer() - t0 > limit_ns) return false;
     }
 }

@@ -144,10 +144,11 @@ __global__ void gather_fs(const float* F, const int32_t* S, const int32_t* rank,
 }
 
 // Back substitution F_S^T X = Y for one instance and one block of CB
-// right-hand columns, blocked by 32 pivots: for each block of rows (bottom
-// up) all threads first subtract the contribution of the rows already
-// solved, then one warp solves the 32 x 32 diagonal block from shared
-// memory, one lane per column.  Two block barriers per 32 pivots.
+// right-hand columns, blocked by 32 pivots, right-looking: blocks are solved
+// bottom up; one half-warp solves a 32 x 32 diagonal block from shared
+// memory (one lane per column), then all threads subtract the solved rows
+// from every row above the block, reading rows of F_S contiguously.  Two
+// block barriers per 32 pivots.
 constexpr int kTrsmThreads = 256;
 constexpr int kTrsmCB = 16;
 constexpr int kTrsmBlk = 32;
@@ -157,6 +158,7 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* Ypart, 
                                                             float* V_S, float* w) {
     extern __shared__ float X[];  // [r][CB], then the diagonal block [32][33]
     float* Ld = X + (size_t)r * kTrsmCB;
+    constexpr int LDS = kTrsmBlk + 1;
     const int64_t b = blockIdx.y;
     const int cb0 = blockIdx.x * kTrsmCB;
     const int DP = D + 1;
@@ -164,37 +166,46 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* Ypart, 
     const int c = threadIdx.x % kTrsmCB, rs = threadIdx.x / kTrsmCB;
     constexpr int RS = kTrsmThreads / kTrsmCB;
     const int col = cb0 + c;
+    const float* Lb = FS + b * (int64_t)r * r;  // Lb[a' * r + a] = F_S[a', a], a <= a'
+    // diagonal block of pivots [a0, a0 + nb): Ld[i][j] = F_S[a0 + i, a0 + j], j <= i
+    auto stage_diag = [&](int a0, int nb) {
+        for (int e = threadIdx.x; e < kTrsmBlk * kTrsmBlk; e += kTrsmThreads) {
+            const int i = e / kTrsmBlk, j = e % kTrsmBlk;
+            Ld[i * LDS + j] = (i < nb && j <= i) ? Lb[(int64_t)(a0 + i) * r + a0 + j] : 0.f;
+        }
+    };
     for (int a = rs; a < r; a += RS) {
         float y = 0.f;
         if (a < rr && col < DP)
             for (int s = 0; s < nsplit; ++s) y += Ypart[(((int64_t)s * BH + b) * r + a) * DP + col];
         X[a * kTrsmCB + c] = y;
     }
-    __syncthreads();
-    const float* Lb = FS + b * (int64_t)r * r;  // Lb[a' * r + a] = F_S[a', a], a <= a'
     const int nblk = (rr + kTrsmBlk - 1) / kTrsmBlk;
+    if (nblk > 0) {
+        const int a0 = (nblk - 1) * kTrsmBlk;
+        stage_diag(a0, rr - a0);
+    }
+    __syncthreads();
     for (int blk = nblk - 1; blk >= 0; --blk) {
-        const int a0 = blk * kTrsmBlk, a1 = min(rr, a0 + kTrsmBlk);
-        // (1) X[a] -= sum_{a' >= a1} F_S[a', a] X[a'] for the block's rows; stage the diagonal block
-        for (int a = a0 + rs; a < a1; a += RS) {
-            float acc = X[a * kTrsmCB + c];
-            for (int ap = a1; ap < rr; ++ap) acc = fmaf(-Lb[(int64_t)ap * r + a], X[ap * kTrsmCB + c], acc);
-            X[a * kTrsmCB + c] = acc;
-        }
-        for (int e = threadIdx.x; e < kTrsmBlk * kTrsmBlk; e += kTrsmThreads) {
-            const int i = e / kTrsmBlk, j = e % kTrsmBlk;  // Ld[i][j] = F_S[a0 + i, a0 + j]
-            Ld[i * (kTrsmBlk + 1) + j] = (a0 + i < a1 && j <= i) ? Lb[(int64_t)(a0 + i) * r + a0 + j] : 0.f;
-        }
-        __syncthreads();
-        // (2) the diagonal block, bottom up, one lane per right-hand column
+        const int a0 = blk * kTrsmBlk, nb = min(rr, a0 + kTrsmBlk) - a0;
+        // (1) the diagonal block, bottom up, one lane per right-hand column
         if (threadIdx.x < kTrsmCB) {
-            for (int i = a1 - a0 - 1; i >= 0; --i) {
-                const float xa = X[(a0 + i) * kTrsmCB + c] / Ld[i * (kTrsmBlk + 1) + i];
+            for (int i = nb - 1; i >= 0; --i) {
+                const float xa = X[(a0 + i) * kTrsmCB + c] / Ld[i * LDS + i];
                 X[(a0 + i) * kTrsmCB + c] = xa;
                 for (int j = 0; j < i; ++j)
-                    X[(a0 + j) * kTrsmCB + c] = fmaf(-Ld[i * (kTrsmBlk + 1) + j], xa, X[(a0 + j) * kTrsmCB + c]);
+                    X[(a0 + j) * kTrsmCB + c] = fmaf(-Ld[i * LDS + j], xa, X[(a0 + j) * kTrsmCB + c]);
             }
         }
+        __syncthreads();
+        // (2) rows above the block: X[a] -= sum_i F_S[a0 + i, a] X[a0 + i]; stage the next diagonal block
+        for (int a = rs; a < a0; a += RS) {
+            float acc = X[a * kTrsmCB + c];
+            const float* Lcol = Lb + (int64_t)a0 * r + a;
+            for (int i = 0; i < nb; ++i) acc = fmaf(-Lcol[(int64_t)i * r], X[(a0 + i) * kTrsmCB + c], acc);
+            X[a * kTrsmCB + c] = acc;
+        }
+        if (blk > 0) stage_diag(a0 - kTrsmBlk, kTrsmBlk);
         __syncthreads();
     }
     if (col < DP) {
@@ -284,6 +295,40 @@ size_t weights_workspace_bytes(int64_t BH, int64_t n, int d, int r) {
     cv.take(sizeof(float) * p.max_split() * BH * (int64_t)r * (d + 1));
     cv.take(sizeof(float) * BH * (int64_t)r * r);
     return cv.used + 256;
+}
+
+size_t value_range_workspace_bytes(int64_t BH, int64_t n, int d) {
+    const WeightsPlan p = make_plan(BH, n, 1);
+    return sizeof(float) * BH * p.nsplit_range * 2 * d + 256;
+}
+
+Status launch_value_range(const void* V, int dtype, int64_t BH, int64_t n, int d, float* vmin, float* vmax,
+                          void* ws, size_t ws_bytes, cudaStream_t st) {
+    const WeightsPlan p = make_plan(BH, n, 1);
+    Carve cv(ws, ws_bytes);
+    float* part = static_cast<float*>(cv.take(sizeof(float) * BH * p.nsplit_range * 2 * d));
+    if (!cv.fits()) return Status::fail(4, "value range: workspace too small");
+    const dim3 grid(p.nsplit_range, (unsigned)BH);
+    const bool bf = dtype == 1;
+    switch (d) {
+        case 32:
+            if (bf) colrange_partial<BF16, 32><<<grid, kRangeThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(V), n, p.rows_per_range, part);
+            else colrange_partial<F32, 32><<<grid, kRangeThreads, 0, st>>>(static_cast<const float*>(V), n, p.rows_per_range, part);
+            break;
+        case 64:
+            if (bf) colrange_partial<BF16, 64><<<grid, kRangeThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(V), n, p.rows_per_range, part);
+            else colrange_partial<F32, 64><<<grid, kRangeThreads, 0, st>>>(static_cast<const float*>(V), n, p.rows_per_range, part);
+            break;
+        case 128:
+            if (bf) colrange_partial<BF16, 128><<<grid, kRangeThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(V), n, p.rows_per_range, part);
+            else colrange_partial<F32, 128><<<grid, kRangeThreads, 0, st>>>(static_cast<const float*>(V), n, p.rows_per_range, part);
+            break;
+        default: return Status::fail(2, "value range: unsupported head dim");
+    }
+    colrange_finalize<<<(unsigned)ceil_div(BH * d, 256), 256, 0, st>>>(part, p.nsplit_range, d, BH, vmin, vmax);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return Status::cuda(e, "value range launch");
+    return Status::ok();
 }
 
 Status launch_weights(const WeightsRequest& q, cudaStream_t st) {

@@ -23,7 +23,7 @@
 
 namespace wildcat {
 
-extern __device__ int g_device_status;
+__device__ int g_weights_status = 0;  // WILDCAT_ERR_TIMEOUT when a bounded wait expired
 
 namespace {
 
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(kWtThreads)
         }
     }
     if (!ok) {
-        if (tid == 0) atomicExch(&g_device_status, 5);
+        if (tid == 0) atomicExch(&g_weights_status, 5);
         mbar_wait(&mbar[0], chunk & 1);
     }
     tc_fence_before();
@@ -217,6 +217,16 @@ Status launch_weights_tc(const float* F, const void* V, const int32_t* rank, int
         case 128: return run_wt<128>(F, V, rank, BH, n, r, nsplit, keys_per_split, Ypart, st);
     }
     return Status::fail(2, "weights_tc: unsupported head dim");
+}
+
+int read_weights_status(bool clear) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_weights_status, sizeof(int)) != cudaSuccess) return -1;
+    if (clear && v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(g_weights_status, &z, sizeof(int));
+    }
+    return v;
 }
 
 }  // namespace wildcat

@@ -65,6 +65,10 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_weights.argtypes = [_f64p, _i32p, _i32p, _f64p, ctypes.c_int64, ctypes.c_int64,
                                    ctypes.c_int, ctypes.c_int, _f64p, _f64p]
     lib.oracle_weights.restype = ctypes.c_int
+    lib.oracle_weights_inverse.argtypes = [_f64p, _i32p, _i32p, _f64p, ctypes.c_int64,
+                                           ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                           ctypes.c_double, _f64p, _f64p]
+    lib.oracle_weights_inverse.restype = ctypes.c_int
     lib.oracle_value_range.argtypes = [_f64p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                                        _f64p, _f64p]
     lib.oracle_value_range.restype = None
@@ -200,6 +204,23 @@ class Oracle:
                                       w.ctypes.data_as(_f64p))
         if err:
             raise MemoryError("oracle_weights")
+        return VS, w
+
+    def weights_inverse(self, K, S, rank, V, beta):
+        """The same W (V, 1_n) through h(K_S, K_S)^-1 maintained by the rank-one
+        update of RPNys (Sec. 2): returns (V_S [BH,r,d], w [BH,r])."""
+        K, kp = self._f64(K)
+        S, sp = self._i32(S)
+        rank, rkp = self._i32(rank)
+        V, vp = self._f64(V)
+        BH, n, d = K.shape
+        r = S.shape[1]
+        VS = np.zeros((BH, r, d))
+        w = np.zeros((BH, r))
+        err = self.lib.oracle_weights_inverse(kp, sp, rkp, vp, BH, n, d, r, float(beta),
+                                              VS.ctypes.data_as(_f64p), w.ctypes.data_as(_f64p))
+        if err:
+            raise MemoryError("oracle_weights_inverse")
         return VS, w
 
     def value_range(self, V):

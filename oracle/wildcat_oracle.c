@@ -19,6 +19,8 @@
  *                      CompressKV: V_S = W V, w = W 1_n)
  *   plug-in output     O_hat = diag(U W 1)^-1 U W V, U = h(Q, K_S), each entry
  *                      clipped to [v_min j, v_max j] (Sec. 2; Alg. 3 WtdAttn)
+ *   inverse route      the same W through h(K_S,K_S)^-1 grown by the rank-one
+ *                      update of RPNys as each pivot joins (Sec. 2)
  *
  * Readings where the pages are silent (the text of Alg. 1 and of the update
  * formulas was lost in extraction):
@@ -351,6 +353,93 @@ int oracle_weights(const double* F, const int32_t* S, const int32_t* rank, const
                         VS + b * (int64_t)r * d, w + b * r, Y);
         }
         free(Y);
+    }
+    return err;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Nystrom weights through the maintained inverse (Sec. 2, the rank-one     */
+/* update of RPNys): as pivot s_a joins S, with b = h(K_S, k_s) and         */
+/* c = h(k_s, k_s), y = H_S^-1 b and the residual sc = c - b.y,             */
+/*   H_S'^-1 = [[H_S^-1, 0], [0, 0]] + g g^T,  g = (y, -1) / sqrt(sc).      */
+/* Then W (V, 1_n) = H_S^-1 h(K_S, K) (V, 1_n).  h carries the shift M_K of */
+/* the factor route, which cancels in W.  Rows >= r' are zero.              */
+/* ------------------------------------------------------------------------ */
+static void weights_inverse_one(const double* Kb, const int32_t* S, int rr, const double* Vb,
+                                int64_t n, int d, int r, double beta, double* VS, double* w,
+                                double* inv, double* y, double* Z) {
+    double MK = -INFINITY;
+    for (int64_t l = 0; l < n; ++l) {
+        const double q = dot(Kb + l * d, Kb + l * d, d);
+        if (q > MK) MK = q;
+    }
+    /* the inverse, grown one pivot at a time (inv is rr x rr, row-major) */
+    for (int a = 0; a < rr; ++a) {
+        const double* ks = Kb + (int64_t)S[a] * d;
+        for (int j = 0; j < a; ++j) {
+            double acc = 0.0;
+            for (int k = 0; k < a; ++k)
+                acc += inv[j * rr + k] * exp(beta * (dot(Kb + (int64_t)S[k] * d, ks, d) - MK));
+            y[j] = acc;
+        }
+        double sc = exp(beta * (dot(ks, ks, d) - MK));
+        for (int j = 0; j < a; ++j) sc -= exp(beta * (dot(Kb + (int64_t)S[j] * d, ks, d) - MK)) * y[j];
+        for (int j = 0; j < a; ++j)
+            for (int k = 0; k < a; ++k)
+#if ORACLE_MUTANT == 6 /* planted: wrong sign in the rank-one update */
+                inv[j * rr + k] -= y[j] * y[k] / sc;
+#else
+                inv[j * rr + k] += y[j] * y[k] / sc;
+#endif
+        for (int j = 0; j < a; ++j) {
+            inv[j * rr + a] = -y[j] / sc;
+            inv[a * rr + j] = -y[j] / sc;
+        }
+        inv[a * rr + a] = 1.0 / sc;
+    }
+    /* Z = h(K_S, K) (V, 1_n), sequential over l */
+    const int dp = d + 1;
+    for (int a = 0; a < rr; ++a) {
+        const double* ks = Kb + (int64_t)S[a] * d;
+        for (int c = 0; c < dp; ++c) Z[a * dp + c] = 0.0;
+        for (int64_t l = 0; l < n; ++l) {
+            const double h = exp(beta * (dot(ks, Kb + l * d, d) - MK));
+            for (int c = 0; c < d; ++c) Z[a * dp + c] += h * Vb[l * d + c];
+            Z[a * dp + d] += h;
+        }
+    }
+    for (int a = 0; a < r; ++a) {
+        for (int c = 0; c < dp; ++c) {
+            double acc = 0.0;
+            if (a < rr)
+                for (int k = 0; k < rr; ++k) acc += inv[a * rr + k] * Z[k * dp + c];
+            if (c < d)
+                VS[(int64_t)a * d + c] = acc;
+            else
+                w[a] = acc;
+        }
+    }
+}
+
+int oracle_weights_inverse(const double* K, const int32_t* S, const int32_t* rank, const double* V,
+                           int64_t BH, int64_t n, int d, int r, double beta, double* VS, double* w) {
+    int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t b = 0; b < BH; ++b) {
+        const int rr = rank[b];
+        double* inv = (double*)calloc((size_t)rr * (size_t)rr + 1, sizeof(double));
+        double* y = (double*)malloc(sizeof(double) * ((size_t)rr + 1));
+        double* Z = (double*)malloc(sizeof(double) * ((size_t)rr + 1) * (size_t)(d + 1));
+        if (!inv || !y || !Z) {
+#pragma omp atomic write
+            err = 1;
+        } else {
+            weights_inverse_one(K + b * n * d, S + b * r, rr, V + b * n * d, n, d, r, beta,
+                                VS + b * (int64_t)r * d, w + b * r, inv, y, Z);
+        }
+        free(inv);
+        free(y);
+        free(Z);
     }
     return err;
 }

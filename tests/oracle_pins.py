@@ -413,11 +413,46 @@ def pin_recentring_and_temperature(o):
     np.testing.assert_allclose(O, o.exact_attention(Q, K, V, beta), rtol=0, atol=1e-11)
 
 
+# --------------------------------------------------------------------------- inverse route
+def pin_inverse_route_weights(o):
+    """The inverse-maintenance weights route equals a dense LU solve of
+    h(K_S,K_S) X = h(K_S,K) (V,1) (numpy.linalg.solve) and the factor route on
+    the same pivots; it interpolates (W[:, S] = I, checked through V = e_S
+    columns); one pivot gives the closed form W = h(k_s, K) / h(k_s, k_s)."""
+    n, d, r, beta = 44, 6, 10, 0.35
+    _, K, V = _rand(161, 2, 1, n, d)
+    res = o.rpcholesky(K, beta, r, seed=9, eps=1e-13)
+    VS_f, w_f = o.weights(res["F"], res["S"], res["rank"], V)
+    VS_i, w_i = o.weights_inverse(K, res["S"], res["rank"], V, beta)
+    for b in range(2):
+        rr = res["rank"][b]
+        s = res["S"][b][:rr]
+        H = _H(K[b], beta)
+        ref = np.linalg.solve(H[np.ix_(s, s)], H[s, :]) @ np.concatenate([V[b], np.ones((n, 1))], 1)
+        got = np.concatenate([VS_i[b][:rr], w_i[b][:rr, None]], 1)
+        np.testing.assert_allclose(got, ref, rtol=0, atol=1e-9 * np.abs(ref).max())
+        np.testing.assert_allclose(VS_i[b], VS_f[b], rtol=0, atol=1e-9 * np.abs(VS_f[b]).max())
+        np.testing.assert_allclose(w_i[b], w_f[b], rtol=0, atol=1e-9 * np.abs(w_f[b]).max())
+        # interpolation: value column a = e_{S_a} (a < d) gives row a' weight delta_{a a'}
+        E = np.zeros((1, n, d))
+        E[0, s[:d], np.arange(d)] = 1.0
+        VS_e, _ = o.weights_inverse(K[b:b + 1], res["S"][b:b + 1], res["rank"][b:b + 1], E, beta)
+        np.testing.assert_allclose(VS_e[0][:rr], np.eye(rr, d), rtol=0, atol=1e-9)
+    S1 = np.array([[7], [30]], np.int32)
+    VS1, w1 = o.weights_inverse(K, S1, np.array([1, 1], np.int32), V, beta)
+    for b in range(2):
+        hk = np.exp(beta * (K[b] @ K[b][S1[b, 0]]))
+        hkk = np.exp(beta * K[b][S1[b, 0]] @ K[b][S1[b, 0]])
+        np.testing.assert_allclose(VS1[b, 0], hk @ V[b] / hkk, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(w1[b, 0], hk.sum() / hkk, rtol=1e-12)
+
+
 ALL_PINS = [
     pin_exact_bruteforce,
     pin_full_rank_is_exact,
     pin_weights_textbook_solve,
     pin_inverse_update_route,
+    pin_inverse_route_weights,
     pin_partial_cholesky_interpolates,
     pin_residual_invariants,
     pin_philox_matches_library,

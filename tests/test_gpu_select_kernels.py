@@ -1,0 +1,135 @@
+"""The two select kernels -- the per-thread cp.async kernel (the default) and
+the bulk-copy kernel (where its shape rules allow) -- against the fp64 oracle
+and against each other, and the bulk kernel's bounded-wait path.
+
+- Pivots drawn by either kernel agree with the oracle's own draws step by
+  step until a near-tie; on the device's pivots (fixed-pivot mode, the oracle
+  following the device's stopping step) every factor column is within 2e-4
+  of the oracle's, relative to the column's largest entry.
+- On the same fixed pivots the two kernels' factors agree to 2e-4 and stop at
+  the same step.
+- A bounded wait that runs out (the test hook) is reported through the
+  device status word, every instance stops at the same step, and the next
+  call is clean.
+"""
+import numpy as np
+import pytest
+import torch
+
+import nystr_coreset_approximate_b200 as wc
+import workloads
+from tests import gpu_common as gc
+
+pytestmark = pytest.mark.gpu
+
+EPS = 1e-6
+
+# (case, cluster size or 0 = automatic); the comment names the code path
+SHAPES = [
+    (gc.case("kres_g4", "mixture16", 4, 3136, 3136, 64, 128, "bf16"), 0),    # resident keys, 4 CTAs
+    (gc.case("stream_g1", "iid", 3, 4096, 64, 64, 200, "bf16"), 0),          # streamed keys, 1 CTA, contiguous stages
+    (gc.case("stream_g16", "iid", 2, 16384, 64, 128, 96, "bf16"), 0),        # 16-CTA clusters
+    (gc.case("rows8192", "iid", 2, 32768, 64, 128, 40, "bf16"), 4),          # 8192 rows per CTA, 4 quads per thread
+    (gc.case("f32_d32", "iid", 3, 1000, 64, 32, 50, "f32"), 0),              # float32, two column groups
+    (gc.case("tiny_full", "iid", 2, 12, 12, 32, 12, "f32"), 0),              # 12 rows, 16 column groups, full rank
+    (gc.case("ragged_g8", "iid", 2, 5000, 64, 64, 64, "bf16"), 8),           # last CTA shorter than the rest
+    (gc.case("walk_trunc", "walk", 2, 8192, 64, 128, 400, "bf16"), 0),       # early truncation
+]
+
+
+@pytest.fixture(autouse=True)
+def _restore_knobs():
+    yield
+    wc.set_select_kernel(0)
+    wc.set_select_cluster(0)
+    wc.force_select_timeout(0)
+
+
+def _run(K, w, kernel, S_fixed=None):
+    wc.set_select_kernel(kernel)
+    if S_fixed is None:
+        S, F, rank, K_S = wc.select(K, w.beta, w.r, w.pivot_seed, EPS)
+    else:
+        S, F, rank, K_S = wc.select_fixed(K, w.beta, S_fixed, EPS)
+    torch.cuda.synchronize()
+    used = wc.last_select_kernel()
+    return S.cpu().numpy(), F.cpu().numpy(), rank.cpu().numpy(), K_S, used
+
+
+@pytest.mark.parametrize("w,G", SHAPES, ids=[w.name for w, _ in SHAPES])
+def test_both_kernels_match_the_oracle(orc, w, G):
+    dev, ex = workloads.make(w)
+    K = dev["K"].cuda()
+    wc.set_select_cluster(G)
+    own = orc.rpcholesky(ex["K"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
+    for kernel, expect in ((2, 2), (1, 1), (0, 1)):
+        S, F, rank, K_S, used = _run(K, w, kernel)
+        assert used == expect
+        gc.pivots_agree_until_tie(S, own["S"], own["margin"], rank, own["rank"], F, own["F"], EPS)
+        for b in range(w.BH):
+            rr = rank[b]
+            assert rr >= 1 and len(set(S[b, :rr].tolist())) == rr and np.all(S[b, rr:] == -1)
+            assert np.all(F[b, rr:] == 0)
+        fx = orc.rpcholesky(ex["K"], w.beta, w.r, eps=0.0, S_fixed=S)
+        assert np.array_equal(fx["rank"], rank)
+        assert gc.column_rel_err(F, fx["F"], rank) < 2e-4
+        KS_ref = orc.gather(ex["K"], S, rank)
+        assert np.array_equal(K_S.float().cpu().numpy().astype(np.float64), KS_ref)
+    assert wc.device_status() == 0
+
+
+@pytest.mark.parametrize("w,G", SHAPES[:5], ids=[w.name for w, _ in SHAPES[:5]])
+def test_kernels_agree_on_fixed_pivots(orc, w, G):
+    dev, ex = workloads.make(w)
+    K = dev["K"].cuda()
+    wc.set_select_cluster(G)
+    own = orc.rpcholesky(ex["K"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
+    S_fixed = torch.from_numpy(own["S"]).cuda()
+    _, F_a, rank_a, _, used_a = _run(K, w, 2, S_fixed)
+    _, F_b, rank_b, _, used_b = _run(K, w, 1, S_fixed)
+    assert (used_a, used_b) == (2, 1)
+    assert np.array_equal(rank_a, rank_b)
+    assert gc.column_rel_err(F_a, F_b.astype(np.float64), rank_a) < 2e-4
+
+
+def test_recentred_keys_bulk_kernel(orc):
+    """The bulk kernel's recentring hook: a forward with recenter on draws
+    the pivots the oracle draws on K - mean(K)."""
+    w = gc.case("recentre", "iid", 2, 2048, 64, 64, 48, "bf16")
+    dev, ex = workloads.make(w)
+    d = gc.cuda_inputs(dev)
+    wc.set_select_kernel(2)
+    O, S, rank = wc.forward_ex(d["Q"], d["K"], d["V"], w.beta, w.r, w.pivot_seed, EPS, recenter=True)
+    assert wc.last_select_kernel() == 2
+    S, rank = S.cpu().numpy(), rank.cpu().numpy().reshape(w.BH)
+    _, S_o, rank_o = orc.wildcat_forward_binned(ex["Q"], ex["K"], ex["V"], w.beta, w.r, 1,
+                                                seed=w.pivot_seed, eps=EPS, recenter=True)
+    res = orc.rpcholesky(ex["K"] - ex["K"].mean(axis=1, keepdims=True), w.beta, w.r,
+                         seed=w.pivot_seed, eps=EPS)
+    assert np.array_equal(S_o, res["S"])
+    gc.pivots_agree_until_tie(S, res["S"], res["margin"], rank, res["rank"])
+
+
+def test_bulk_select_bounded_wait_reports_timeout_and_recovers():
+    """The test hook makes every CTA's warp 0 wait 1 ms, after step 1, on a
+    barrier phase nothing completes.  The expiry is recorded in the device
+    status word, the abort reaches every CTA of the cluster with the chunk
+    sums, all stop after two steps, and the next call is clean."""
+    w = gc.case("sel_timeout", "iid", 3, 4096, 64, 64, 32, "bf16")
+    dev, _ = workloads.make(w)
+    K = dev["K"].cuda()
+    wc.set_select_cluster(4)
+    wc.set_select_kernel(2)
+    assert wc.device_status() == 0
+    wc.force_select_timeout(1_000_000)
+    try:
+        S, F, rank, _ = wc.select(K, w.beta, w.r, w.pivot_seed, EPS)
+        assert wc.last_select_kernel() == 2
+        assert wc.device_status() == 5
+        assert torch.all(rank == 2)
+        assert torch.all(S[:, 2:] == -1)
+    finally:
+        wc.force_select_timeout(0)
+    S, F, rank, _ = wc.select(K, w.beta, w.r, w.pivot_seed, EPS)
+    assert wc.device_status() == 0
+    assert torch.all(rank == w.r)

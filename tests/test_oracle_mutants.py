@@ -1,6 +1,6 @@
 """Mutation check of the pins: each copy of the oracle with one planted
 mistake (dropped term, wrong sign, transposed operand, swapped clip bounds,
-greedy instead of random pivots) must fail at least one pin.  The mistakes
+greedy instead of random pivots, a wrong sign in the inverse update) must fail at least one pin.  The mistakes
 are planted in the oracle's C source at compile time, on the CPU."""
 import os
 
@@ -15,6 +15,7 @@ MUTANTS = {
     3: "transposes the factor in the back substitution",
     4: "swaps the clip bounds",
     5: "takes the largest residual instead of a random pivot",
+    6: "flips the sign of the rank-one inverse update",
 }
 
 
