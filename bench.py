@@ -61,6 +61,8 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--nbins", type=int, default=1,
                    help="divide-and-conquer bins (1 = the unbinned method)")
+    p.add_argument("--weights-inverse", action="store_true",
+                   help="also time the inverse-maintenance weights route on the selected pivots")
     p.add_argument("--select-kernel", type=int, choices=[0, 1, 2], default=0,
                    help="0 = automatic (the cp.async kernel), 1 = cp.async, 2 = bulk-copy where it applies")
     return p.parse_args()
@@ -317,6 +319,28 @@ def main():
             stage_ms["weights"].append(ev[1].elapsed_time(ev[2]))
             if nb == 1:
                 stage_ms["attend"].append(ev[2].elapsed_time(ev[3]))
+    inv = None
+    if args.weights_inverse and nb == 1:
+        # the inverse route (fp64) on the same pivots; ALU-bound by its Z contraction
+        inv_ms = []
+        for k in range(args.steps + 2):
+            flush.zero_()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record()
+            wc.weights_inverse(K, S, rk, V, w.beta)
+            a1.record()
+            torch.cuda.synchronize()
+            if k >= 2:
+                inv_ms.append(a0.elapsed_time(a1))
+        rks = rk.cpu().tolist()
+        zflops = sum(4.0 * rr * w.n * (w.d + 1) for rr in rks)       # dot products + accumulation, fp64
+        invflops = sum(4.0 * rr ** 3 / 3.0 + 2.0 * rr * rr * (w.d + 1) for rr in rks)
+        ms_inv = statistics.mean(inv_ms)
+        peak64 = 148 * 64 * 2 * 1.965e9 / 1e12
+        ach = (zflops + invflops) / (ms_inv / 1e3) / 1e12
+        inv = {"ms": ms_inv, "fp64_flops_per_call": zflops + invflops, "achieved_tflops": ach,
+               "peak_tflops": peak64, "frac": ach / peak64, "bound": "alu",
+               "peak_source": "fp64 unit count: 148 SMs x 64 FMA/clk x 2 x 1.965 GHz"}
     del S, F, rk, K_S, V_S, wv, vmin, vmax
     if not stage_ms["attend"]:
         del stage_ms["attend"]
@@ -389,6 +413,8 @@ def main():
         "cpu_baseline": cpu,
         "effective_rank_mean": sum(ranks) / len(ranks),
     }
+    if inv is not None:
+        out["weights_inverse"] = inv
     print(json.dumps(out), flush=True)
     return 0
 

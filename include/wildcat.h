@@ -320,8 +320,11 @@ wildcat_status wildcat_forward_binned(const void* Q, const void* K, const void* 
 /*
  * wildcat_forward_host -- wildcat_forward on HOST buffers: copies Q, K, V
  * from host memory into the device workspace, runs the forward, copies O
- * (and optionally S, rank) back, and waits for the stream.  Host buffers
- * should be page-locked for full copy bandwidth.
+ * (and optionally S, rank) back, and waits for the stream.  K is copied
+ * first on a library-owned copy stream; V and Q follow while the select
+ * runs on `stream`, and the weights and attend stages wait for them.  Calls
+ * on one device are serialized (a per-device lock guards the copy stream).
+ * Host buffers should be page-locked for full copy bandwidth.
  *
  *   Q_host, K_host, V_host   host input arrays (layouts as wildcat_forward)
  *   O_host                   host output [BH, m, d] float32

@@ -6,6 +6,8 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <map>
+#include <mutex>
 
 #include "../../include/wildcat.h"
 #include "internal.h"
@@ -104,15 +106,21 @@ ForwardLayout carve_forward(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, 
     return L;
 }
 
+// wait_v / wait_q (optional): events the weights / attend stage waits for
+// (the host-buffer forward copies V and Q while the select runs).
 wildcat_status forward_impl(const void* Q, const void* K, const void* V, int dtype, int64_t BH, int64_t m, int64_t n,
                             int d, float beta, int r, uint64_t seed, int64_t inst0, float eps, float* O,
-                            int32_t* S_out, int32_t* rank_out, const ForwardLayout& L, cudaStream_t st) {
+                            int32_t* S_out, int32_t* rank_out, const ForwardLayout& L, cudaStream_t st,
+                            cudaEvent_t wait_v = nullptr, cudaEvent_t wait_q = nullptr) {
     Status s;
+    cudaError_t ew;
     wildcat::SelectRequest sq{K, dtype, BH, n, d, beta, r, seed, inst0, eps, nullptr, L.S, L.F, L.rank, L.K_S};
     if ((s = wildcat::launch_select(sq, st)).code) return record(s);
+    if (wait_v && (ew = cudaStreamWaitEvent(st, wait_v, 0))) return record(Status::cuda(ew, "forward: wait for V"));
     wildcat::WeightsRequest wq{L.F, L.S, L.rank, V, dtype, BH, n, d, r, L.V_S, L.w, L.vmin, L.vmax, L.wws,
                                L.wws_bytes};
     if ((s = wildcat::launch_weights(wq, st)).code) return record(s);
+    if (wait_q && (ew = cudaStreamWaitEvent(st, wait_q, 0))) return record(Status::cuda(ew, "forward: wait for Q"));
     if (m > 0) {
         wildcat::AttendRequest aq{Q,   L.K_S,  dtype, BH, m, d, r, L.rank, beta, L.V_S, L.w,
                                   L.vmin, L.vmax, O,   L.aws, L.aws_bytes};
@@ -180,6 +188,33 @@ wildcat_status check_bins(int64_t BH, int64_t n, int r, int nbins, const char* w
 }
 
 }  // namespace
+
+// One copy stream and four events per device for the host-buffer forward,
+// created on first use; a call holds the device's mutex while it runs.
+struct HostPipe {
+    std::mutex mu;
+    cudaStream_t cs = nullptr;
+    cudaEvent_t ready = nullptr, k_in = nullptr, v_in = nullptr, q_in = nullptr;
+};
+
+HostPipe* host_pipe(int dev) {
+    static std::mutex pool_mu;
+    static std::map<int, HostPipe*> pool;
+    std::lock_guard<std::mutex> lock(pool_mu);
+    auto it = pool.find(dev);
+    if (it != pool.end()) return it->second;
+    HostPipe* hp = new HostPipe();
+    bool ok = cudaStreamCreateWithFlags(&hp->cs, cudaStreamNonBlocking) == cudaSuccess;
+    for (cudaEvent_t* ev : {&hp->ready, &hp->k_in, &hp->v_in, &hp->q_in})
+        ok = ok && cudaEventCreateWithFlags(ev, cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        delete hp;  // the handles that were created are left to the context's teardown
+        return nullptr;
+    }
+    pool[dev] = hp;
+    return hp;
+}
 
 namespace wildcat {
 int read_device_status(bool clear) {
@@ -468,25 +503,41 @@ wildcat_status wildcat_forward_host(const void* Q_host, const void* K_host, cons
     void* Kd = cv.take(eb * BH * n * d);
     void* Vd = cv.take(eb * BH * n * d);
     float* Od = static_cast<float*>(cv.take(sizeof(float) * BH * m * d));
-    int32_t* Sd = static_cast<int32_t*>(cv.take(sizeof(int32_t) * BH * r));
-    int32_t* Rd = static_cast<int32_t*>(cv.take(sizeof(int32_t) * BH));
+    cv.take(sizeof(int32_t) * BH * r);
+    cv.take(sizeof(int32_t) * BH);
     const ForwardLayout L = carve_forward(cv, BH, m, n, d, r, dtype);
     if (!cv.fits()) return bad(4, "%s: workspace too small", who);
-    cudaError_t e;
-    if (m > 0 && (e = cudaMemcpyAsync(Qd, Q_host, eb * BH * m * d, cudaMemcpyHostToDevice, s)))
-        return record(Status::cuda(e, "forward_host: copy Q"));
-    if ((e = cudaMemcpyAsync(Kd, K_host, eb * BH * n * d, cudaMemcpyHostToDevice, s)))
+    // K first on a copy stream: the select needs only K, so V and Q cross
+    // the bus while it runs; the weights and attend stages wait for them.
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e) return record(Status::cuda(e, "forward_host: current device"));
+    HostPipe* hp = host_pipe(dev);
+    if (!hp) return record(Status::cuda(cudaErrorMemoryAllocation, "forward_host: copy stream"));
+    std::lock_guard<std::mutex> lock(hp->mu);
+    if ((e = cudaEventRecord(hp->ready, s))) return record(Status::cuda(e, "forward_host: record"));
+    if ((e = cudaStreamWaitEvent(hp->cs, hp->ready, 0))) return record(Status::cuda(e, "forward_host: wait"));
+    if ((e = cudaMemcpyAsync(Kd, K_host, eb * BH * n * d, cudaMemcpyHostToDevice, hp->cs)))
         return record(Status::cuda(e, "forward_host: copy K"));
-    if ((e = cudaMemcpyAsync(Vd, V_host, eb * BH * n * d, cudaMemcpyHostToDevice, s)))
+    if ((e = cudaEventRecord(hp->k_in, hp->cs))) return record(Status::cuda(e, "forward_host: record"));
+    if ((e = cudaMemcpyAsync(Vd, V_host, eb * BH * n * d, cudaMemcpyHostToDevice, hp->cs)))
         return record(Status::cuda(e, "forward_host: copy V"));
+    if ((e = cudaEventRecord(hp->v_in, hp->cs))) return record(Status::cuda(e, "forward_host: record"));
+    if (m > 0 && (e = cudaMemcpyAsync(Qd, Q_host, eb * BH * m * d, cudaMemcpyHostToDevice, hp->cs)))
+        return record(Status::cuda(e, "forward_host: copy Q"));
+    if ((e = cudaEventRecord(hp->q_in, hp->cs))) return record(Status::cuda(e, "forward_host: record"));
+    if ((e = cudaStreamWaitEvent(s, hp->k_in, 0))) return record(Status::cuda(e, "forward_host: wait for K"));
     st = forward_impl(m > 0 ? Qd : nullptr, Kd, Vd, dtype, BH, m, n, d, beta, r, seed, inst0, eps,
-                      m > 0 ? Od : nullptr, Sd, Rd, L, s);
-    if (st != WILDCAT_OK) return st;
+                      m > 0 ? Od : nullptr, nullptr, nullptr, L, s, hp->v_in, hp->q_in);
+    if (st != WILDCAT_OK) {
+        cudaStreamSynchronize(hp->cs);
+        return st;
+    }
     if (m > 0 && (e = cudaMemcpyAsync(O_host, Od, sizeof(float) * BH * m * d, cudaMemcpyDeviceToHost, s)))
         return record(Status::cuda(e, "forward_host: copy O"));
-    if (S_host && (e = cudaMemcpyAsync(S_host, Sd, sizeof(int32_t) * BH * r, cudaMemcpyDeviceToHost, s)))
+    if (S_host && (e = cudaMemcpyAsync(S_host, L.S, sizeof(int32_t) * BH * r, cudaMemcpyDeviceToHost, s)))
         return record(Status::cuda(e, "forward_host: copy S"));
-    if (rank_host && (e = cudaMemcpyAsync(rank_host, Rd, sizeof(int32_t) * BH, cudaMemcpyDeviceToHost, s)))
+    if (rank_host && (e = cudaMemcpyAsync(rank_host, L.rank, sizeof(int32_t) * BH, cudaMemcpyDeviceToHost, s)))
         return record(Status::cuda(e, "forward_host: copy rank"));
     if ((e = cudaStreamSynchronize(s))) return record(Status::cuda(e, "forward_host: stream sync"));
     return record(Status::ok());

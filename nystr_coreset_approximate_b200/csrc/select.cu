@@ -102,6 +102,10 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
     const unsigned d = (unsigned)__cvta_generic_to_shared(smem_dst);
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(gmem_src) : "memory");
 }
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d), "l"(gmem_src) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
@@ -144,7 +148,6 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     double* csl = reinterpret_cast<double*>(smem + L.csl);
     float* dbuf = reinterpret_cast<float*>(smem + L.dbuf);
     float* dotb = reinterpret_cast<float*>(smem + L.dotb);
-    float* ks = reinterpret_cast<float*>(smem + L.ks);
     float* fs = reinterpret_cast<float*>(smem + L.fs);
     float* red = reinterpret_cast<float*>(smem + L.red);
     float* misc = reinterpret_cast<float*>(smem + L.misc);
@@ -166,61 +169,76 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
 #pragma unroll
     for (int e = 0; e < EPL; ++e)
         kbr[e] = a.kbar ? a.kbar[(b / a.kbar_div) * D + kl_part * EPL + e] : 0.f;
-    auto key_pass = [&](const float* x, float* out) {
-        float xr[EPL];
+    // The first INFL items of the streamed key pass; they do not depend on
+    // the pivot, so a step can issue them before the previous one ends.
+    const int kfirst = warp * RPW + kl_row;  // row of item 0 for this lane
+    const int kitems = nrows > warp * RPW ? (int)ceil_div(nrows - warp * RPW, NW * RPW) : 0;  // warp-uniform
+    const T* ksrc0 = Kb + (row0 + kfirst) * D + kl_part * EPL;
+    const int64_t kstep = (int64_t)NW * RPW * D;
+    auto key_prime = [&]() {
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) xr[e] = x ? x[kl_part * EPL + e] : 0.f;
+        for (int q = 0; q < INFL; ++q) {
+            if (q < kitems && kfirst + q * NW * RPW < nrows) cp_async16(ring4 + q * NT, ksrc0 + q * kstep);
+            cp_async_commit();
+        }
+    };
+    // out[row] = <k_row - kbar, x> (or |k_row - kbar|^2 when self)
+    auto key_pass = [&](const float (&x)[EPL], bool self, float* out, bool primed) {
         if constexpr (KRES) {
-            // key rows resident in shared memory: no global traffic
-            for (int base = warp * RPW; base < nrows; base += NW * RPW) {
-                const int row = base + kl_row;
-                float part = 0.f;
-                if (row < nrows) {
-                    const float4 raw = *reinterpret_cast<const float4*>(kres + (size_t)row * D + kl_part * EPL);
-                    float v[EPL];
-                    if constexpr (sizeof(T) == 2) {
-                        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+            // key rows resident in shared memory: no global traffic; four rows per lane in flight
+            for (int base = warp * RPW; base < nrows; base += 4 * NW * RPW) {
+                float part[4];
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const float2 f = __bfloat1622float2(h[k]);
-                            v[2 * k] = f.x;
-                            v[2 * k + 1] = f.y;
+                for (int u = 0; u < 4; ++u) {
+                    const int row = base + u * NW * RPW + kl_row;
+                    part[u] = 0.f;
+                    if (row < nrows) {
+                        const float4 raw = *reinterpret_cast<const float4*>(kres + (size_t)row * D + kl_part * EPL);
+                        float v[EPL];
+                        if constexpr (sizeof(T) == 2) {
+                            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const float2 f = __bfloat1622float2(h[k]);
+                                v[2 * k] = f.x;
+                                v[2 * k + 1] = f.y;
+                            }
+                        } else {
+                            v[0] = raw.x; v[1] = raw.y; v[2] = raw.z; v[3] = raw.w;
                         }
-                    } else {
-                        v[0] = raw.x; v[1] = raw.y; v[2] = raw.z; v[3] = raw.w;
+#pragma unroll
+                        for (int e = 0; e < EPL; ++e) v[e] -= kbr[e];
+#pragma unroll
+                        for (int e = 0; e < EPL; ++e) part[u] = fmaf(v[e], self ? v[e] : x[e], part[u]);
                     }
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) v[e] -= kbr[e];
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) part = fmaf(v[e], x ? xr[e] : v[e], part);
                 }
 #pragma unroll
-                for (int o = LPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-                if (kl_part == 0 && row < nrows) out[row] = part;
+                for (int o = LPR / 2; o > 0; o >>= 1)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) part[u] += __shfl_xor_sync(0xffffffffu, part[u], o);
+                if (kl_part == 0) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int row = base + u * NW * RPW + kl_row;
+                        if (row < nrows) out[row] = part[u];
+                    }
+                }
             }
             return;
         }
-        const int first = warp * RPW + kl_row;                    // row of item 0 for this lane
-        const int items = nrows > warp * RPW ? (int)ceil_div(nrows - warp * RPW, NW * RPW) : 0;  // warp-uniform
-        const T* src0 = Kb + (row0 + first) * D + kl_part * EPL;
-        const int64_t step = (int64_t)NW * RPW * D;
-#pragma unroll
-        for (int q = 0; q < INFL; ++q) {
-            if (q < items && first + q * NW * RPW < nrows) cp_async16(ring4 + q * NT, src0 + q * step);
-            cp_async_commit();
-        }
+        if (!primed) key_prime();
         // slot and source advance incrementally (no division or 64-bit multiply per item)
         int slot_rd = 0, slot_wr = INFL;
-        const T* src_wr = src0 + INFL * step;
-        int row_wr = first + INFL * NW * RPW;
-        for (int q = 0; q < items; ++q) {
-            if (q + INFL < items && row_wr < nrows) cp_async16(ring4 + slot_wr * NT, src_wr);
+        const T* src_wr = ksrc0 + INFL * kstep;
+        int row_wr = kfirst + INFL * NW * RPW;
+        for (int q = 0; q < kitems; ++q) {
+            if (q + INFL < kitems && row_wr < nrows) cp_async16(ring4 + slot_wr * NT, src_wr);
             cp_async_commit();
-            src_wr += step;
+            src_wr += kstep;
             row_wr += NW * RPW;
             slot_wr = slot_wr + 1 == DEPTH ? 0 : slot_wr + 1;
             cp_async_wait<INFL>();
-            const int row = first + q * NW * RPW;
+            const int row = kfirst + q * NW * RPW;
             float part = 0.f;
             const float4 raw = ring4[slot_rd * NT];
             slot_rd = slot_rd + 1 == DEPTH ? 0 : slot_rd + 1;
@@ -240,7 +258,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
 #pragma unroll
                 for (int e = 0; e < EPL; ++e) v[e] -= kbr[e];
 #pragma unroll
-                for (int e = 0; e < EPL; ++e) part = fmaf(v[e], x ? xr[e] : v[e], part);
+                for (int e = 0; e < EPL; ++e) part = fmaf(v[e], self ? v[e] : x[e], part);
             }
 #pragma unroll
             for (int o = LPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
@@ -249,25 +267,31 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
         cp_async_wait<0>();
     };
 
-    // Chunk sums of a freshly written residual buffer, pushed with the CTA
-    // total into every peer's inbox[par][crank], then the cluster barrier.
-    auto publish = [&](const float* dnew, int par) {
-        for (int k = warp; k < nch; k += NW) {
-            const double t = chunk_total(dnew + (size_t)k * CH, PL, lane);
-            if (lane == 0) csl[k] = t;
+    // Chunk sums of a freshly written residual buffer (unless the epilogue
+    // formed them), pushed with the CTA total into every peer's
+    // inbox[par][crank]; the cluster barrier is split so that warp 0 draws
+    // the next step's uniform while the cluster arrives.
+    double u_next = 0.0;  // warp 0: the uniform of the next step
+    auto publish = [&](const float* dnew, int par, bool have_csl, int next_step) {
+        if (!have_csl) {
+            for (int k = warp; k < nch; k += NW) {
+                const double t = chunk_total(dnew + (size_t)k * CH, PL, lane);
+                if (lane == 0) csl[k] = t;
+            }
+            __syncthreads();
         }
-        __syncthreads();
         if (warp == 0) {
             const double v = lane < nch ? csl[lane] : 0.0;
-            double tot = 0.0;
-            for (int k = 0; k < nch; ++k) tot += __shfl_sync(0xffffffffu, v, k);
+            const double tot = __shfl_sync(0xffffffffu, warp_scan_incl(v, lane), 31);
             for (int c = 0; c < G; ++c) {
                 double* dst = cluster.map_shared_rank(inbox + ((size_t)par * G + crank) * 33, c);
                 if (lane < nch) dst[lane] = v;
                 if (lane == 0) dst[32] = tot;
             }
         }
-        cluster.sync();
+        cluster.barrier_arrive();
+        if (warp == 0) u_next = pivot_uniform(a.seed, (uint32_t)next_step, (uint32_t)(a.inst0 + b));
+        cluster.barrier_wait();
     };
 
     // ---------------- prologue: M_K and the initial residual diagonal ----------------
@@ -280,7 +304,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
         cp_async_wait<0>();
         __syncthreads();
     }
-    key_pass(nullptr, dotb);  // |k_l|^2
+    {
+        const float none[EPL] = {};
+        key_pass(none, true, dotb, false);  // |k_l - kbar|^2
+    }
     __syncthreads();
     float lmax = -INFINITY;
     for (int row = tid; row < nrows; row += NT) lmax = fmaxf(lmax, dotb[row]);
@@ -305,9 +332,29 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     const float beta = a.beta;
     for (int row = tid; row < Rpad; row += NT) dbuf[row] = row < nrows ? expf(beta * (dotb[row] - MK)) : 0.f;
     __syncthreads();
-    publish(dbuf, 0);
+    publish(dbuf, 0, false, 0);
 
     // ---------------- r sequential steps ----------------
+    // The epilogue forms the search's chunk sums itself when a chunk is
+    // exactly one warp's rows (4 per lane): then group-0 warp w of a row
+    // block covers chunk (base + 128 w) / 128 with the search's lane layout.
+    const bool fused_csl = (VEC == 4 && PL == 4);
+    const int g = tid / TPG, tt = tid % TPG;
+    // The first INFL factor items of row block 0 for step `st` (resident keys
+    // only: the ring is idle during the key pass then); they do not depend on
+    // the pivot either.
+    auto fpass_prime = [&](int st) {
+        const int jl = (st + JG - 1) / JG, j0 = min(st, g * jl), j1 = min(st, j0 + jl);
+        const int row = tt * VEC;
+        const int cnt = row < nrows ? j1 - j0 : 0;
+        const float* fcol = Fb + row0 + row;
+#pragma unroll
+        for (int q = 0; q < INFL; ++q) {
+            if (q < cnt) cp_async16(ring4 + q * NT, fcol + (int64_t)(j0 + q) * n);
+            cp_async_commit();
+        }
+    };
+    bool primed = false;  // the next step's first ring items are in flight
     int i = 0;
     for (; i < r; ++i) {
         const int cur = i & 1, nxt = cur ^ 1;
@@ -323,75 +370,57 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                 s = (sf >= 0 && (int64_t)sf < n) ? sf : -1;
             } else {
                 const double tc = lane < G ? ib[lane * 33 + 32] : 0.0;
-                double T = 0.0;
-                for (int c = 0; c < G; ++c) T += __shfl_sync(0xffffffffu, tc, c);
-                if (T > 0.0) {
-                    const double t = pivot_uniform(a.seed, (uint32_t)i, (uint32_t)(a.inst0 + b)) * T;
-                    // owner CTA: first whose cumulative total reaches t
-                    double cum = 0.0;
-                    int owner = -1, lastpos = -1;
-                    for (int c = 0; c < G; ++c) {
-                        const double v = __shfl_sync(0xffffffffu, tc, c);
-                        if (v > 0.0) lastpos = c;
-                        if (owner < 0) {
-                            if (cum + v >= t) owner = c;
-                            else cum += v;
-                        }
-                    }
-                    if (owner < 0) {  // rounding pushed t past the total
-                        owner = lastpos;
-                        cum = 0.0;
-                        for (int c = 0; c < owner; ++c) cum += __shfl_sync(0xffffffffu, tc, c);
-                    }
-                    // owner's chunk reached by t (its chunk sums are in the local inbox)
+                const double incl = warp_scan_incl(tc, lane);
+                const double T = __shfl_sync(0xffffffffu, incl, 31);
+                const unsigned pos_cta = __ballot_sync(0xffffffffu, tc > 0.0);
+                if (T > 0.0 && pos_cta) {
+                    const double t = u_next * T;
+                    // owner CTA: first with positive mass whose running total reaches t
+                    unsigned m = __ballot_sync(0xffffffffu, tc > 0.0 && incl >= t);
+                    const int owner = m ? __ffs(m) - 1 : 31 - __clz(pos_cta);
+                    const double t1 = t - __shfl_sync(0xffffffffu, incl - tc, owner);
+                    // owner's chunk (its chunk sums are in the local inbox)
                     const double cv = lane < nch ? ib[owner * 33 + lane] : 0.0;
-                    int chunk = -1, lastc = -1;
-                    double cum2 = cum;
-                    for (int k = 0; k < nch; ++k) {
-                        const double v = __shfl_sync(0xffffffffu, cv, k);
-                        if (v > 0.0) lastc = k;
-                        if (chunk < 0) {
-                            if (cum2 + v >= t) chunk = k;
-                            else cum2 += v;
+                    const double ci = warp_scan_incl(cv, lane);
+                    const unsigned pos_ch = __ballot_sync(0xffffffffu, cv > 0.0);
+                    if (pos_ch) {  // warp-uniform; a positive total implies a positive chunk
+                        m = __ballot_sync(0xffffffffu, cv > 0.0 && ci >= t1);
+                        const int chunk = m ? __ffs(m) - 1 : 31 - __clz(pos_ch);
+                        const double t2 = t1 - __shfl_sync(0xffffffffu, ci - cv, chunk);
+                        // row inside the chunk: one read of the owner's residuals
+                        const float* rd =
+                            cluster.map_shared_rank(dbuf + (size_t)cur * Rpad, owner) + (size_t)chunk * CH;
+                        float vals[kMaxPL];
+#pragma unroll
+                        for (int k = 0; k < kMaxPL; ++k) vals[k] = k < PL ? rd[lane * PL + k] : 0.f;
+                        double part = 0.0;
+#pragma unroll
+                        for (int k = 0; k < kMaxPL; ++k)
+                            if (k < PL) part += (double)vals[k];
+                        double c = warp_scan_incl(part, lane) - part;
+                        int hit = -1, lastnz = -1;
+#pragma unroll
+                        for (int k = 0; k < kMaxPL; ++k) {
+                            if (k >= PL) break;
+                            const float v = vals[k];
+                            if (v > 0.f) lastnz = k;
+                            c += (double)v;
+                            if (hit < 0 && v > 0.f && c >= t2) hit = k;
                         }
+                        const unsigned hm = __ballot_sync(0xffffffffu, hit >= 0);
+                        int local = -1;
+                        if (hm) {
+                            const int src = __ffs(hm) - 1;
+                            local = src * PL + __shfl_sync(0xffffffffu, hit, src);
+                        } else {
+                            const unsigned nm = __ballot_sync(0xffffffffu, lastnz >= 0);
+                            if (nm) {
+                                const int src = 31 - __clz(nm);
+                                local = src * PL + __shfl_sync(0xffffffffu, lastnz, src);
+                            }
+                        }
+                        if (local >= 0) s = (int)((int64_t)owner * R + (int64_t)chunk * CH + local);
                     }
-                    if (chunk < 0) {
-                        chunk = lastc;
-                        cum2 = cum;
-                        for (int k = 0; k < chunk; ++k) cum2 += __shfl_sync(0xffffffffu, cv, k);
-                    }
-                    // row inside the chunk: one read of the owner's residuals
-                    const float* rd =
-                        cluster.map_shared_rank(dbuf + (size_t)cur * Rpad, owner) + (size_t)chunk * CH;
-                    float vals[kMaxPL];
-#pragma unroll
-                    for (int k = 0; k < kMaxPL; ++k) vals[k] = k < PL ? rd[lane * PL + k] : 0.f;
-                    double part = 0.0;
-#pragma unroll
-                    for (int k = 0; k < kMaxPL; ++k)
-                        if (k < PL) part += (double)vals[k];
-                    const double incl = warp_scan_incl(part, lane);
-                    double c = cum2 + (incl - part);
-                    int hit = -1, lastnz = -1;
-#pragma unroll
-                    for (int k = 0; k < kMaxPL; ++k) {
-                        if (k >= PL) break;
-                        const float v = vals[k];
-                        if (v > 0.f) lastnz = k;
-                        c += (double)v;
-                        if (hit < 0 && v > 0.f && c >= t) hit = k;
-                    }
-                    const unsigned hm = __ballot_sync(0xffffffffu, hit >= 0);
-                    int local;
-                    if (hm) {
-                        const int src = __ffs(hm) - 1;
-                        local = src * PL + __shfl_sync(0xffffffffu, hit, src);
-                    } else {
-                        const unsigned nm = __ballot_sync(0xffffffffu, lastnz >= 0);
-                        const int src = 31 - __clz(nm);
-                        local = src * PL + __shfl_sync(0xffffffffu, lastnz, src);
-                    }
-                    s = (int)((int64_t)owner * R + (int64_t)chunk * CH + local);
                 }
             }
             if (lane == 0) {
@@ -403,30 +432,35 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
         if (imisc[4]) break;
         const int s = imisc[3];
 
-        // -- pivot key and the pivot's row of the factor (loads issued together) --
-        const T* kp = Kb + (int64_t)s * D;
-        for (int c = tid; c < D; c += NT)
-            ks[c] = E::to_float(kp[c]) - (a.kbar ? a.kbar[(b / a.kbar_div) * D + c] : 0.f);
-        for (int j = tid; j < i; j += NT) fs[j] = ld_cg1(Fb + (int64_t)j * n + s);
-        __syncthreads();
-        // -- pivot residual g_s (warp 0, the same on every CTA) and <k_l, k_s> --
-        if (warp == 0) {
-            float dot = 0.f, acc = 0.f;
-            for (int c = lane; c < D; c += 32) dot = fmaf(ks[c], ks[c], dot);
-            for (int j = lane; j < i; j += 32) acc = fmaf(fs[j], fs[j], acc);
-            dot = warp_sum(dot);
-            acc = warp_sum(acc);
-            if (lane == 0) {
-                const float gs = expf(beta * (dot - MK)) - acc;
-                misc[2] = gs;
-                imisc[4] = !(gs > a.eps);  // max_l h(k_l, k_l) is exp(0) = 1
+        // -- the pivot's factor row (asynchronous; first needed by the factor
+        //    pass) and the pivot key (registers of every lane) --
+        for (int j = tid; j < i; j += NT) cp_async4(fs + j, Fb + (int64_t)j * n + s);
+        cp_async_commit();
+        float xr[EPL];
+        {
+            float4 raw;
+            if constexpr (KRES) {
+                const int owner = (int)(s / R), lrow = (int)(s - (int64_t)owner * R);
+                raw = *cluster.map_shared_rank(
+                    reinterpret_cast<const float4*>(kres + (size_t)lrow * D + kl_part * EPL), owner);
+            } else {
+                raw = __ldg(reinterpret_cast<const float4*>(Kb + (int64_t)s * D + kl_part * EPL));
             }
+            if constexpr (sizeof(T) == 2) {
+                const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float2 f = __bfloat1622float2(h[k]);
+                    xr[2 * k] = f.x;
+                    xr[2 * k + 1] = f.y;
+                }
+            } else {
+                xr[0] = raw.x; xr[1] = raw.y; xr[2] = raw.z; xr[3] = raw.w;
+            }
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) xr[e] -= kbr[e];
         }
-        key_pass(ks, dotb);
-        __syncthreads();
-        if (imisc[4]) break;
-        const float gs = misc[2];
-        const float piv = sqrtf(gs);
+        const T* kp = Kb + (int64_t)s * D;
         if (crank == 0) {
             if (tid == 0 && a.S) a.S[b * r + i] = s;
             if (a.K_S) {
@@ -434,10 +468,30 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                 for (int c = tid; c < D; c += NT) dst[c] = kp[c];
             }
         }
+        // -- <k_l - kbar, k_s - kbar> for the CTA's rows --
+        key_pass(xr, false, dotb, primed && !KRES);
+        cp_async_wait<0>();
+        __syncthreads();
+        // -- pivot residual g_s (warp 0, the same on every CTA), read after the next barrier --
+        if (warp == 0) {
+            float dot = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) dot = fmaf(xr[e], xr[e], dot);
+#pragma unroll
+            for (int o = LPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+            float acc = 0.f;
+            for (int j = lane; j < i; j += 32) acc = fmaf(fs[j], fs[j], acc);
+            acc = warp_sum(acc);
+            if (lane == 0) {
+                const float gs = expf(beta * (dot - MK)) - acc;
+                misc[2] = gs;
+                imisc[4] = !(gs > a.eps);  // max_l h(k_l, k_l) is exp(0) = 1
+            }
+        }
 
         // -- factor pass over the CTA's rows: acc_l = sum_j F[j, l] F[j, s] --
-        const int g = tid / TPG, tt = tid % TPG;
         const int jl = (i + JG - 1) / JG, j0 = min(i, g * jl), j1 = min(i, j0 + jl);
+        bool stop = false;
         for (int base = 0; base < nrows; base += TPG * VEC) {
             const int row = base + tt * VEC;
             const bool valid = row < nrows;
@@ -449,10 +503,12 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                 int j = j0;
                 if constexpr (VEC == 4) {
                     const int cnt = j1 - j0;
+                    if (!(KRES && primed && base == 0)) {
 #pragma unroll
-                    for (int q = 0; q < INFL; ++q) {
-                        if (q < cnt) cp_async16(ring4 + q * NT, fcol + (int64_t)(j0 + q) * n);
-                        cp_async_commit();
+                        for (int q = 0; q < INFL; ++q) {
+                            if (q < cnt) cp_async16(ring4 + q * NT, fcol + (int64_t)(j0 + q) * n);
+                            cp_async_commit();
+                        }
                     }
                     int slot_rd = 0, slot_wr = INFL;
                     const float* src_wr = fcol + (int64_t)(j0 + INFL) * n;
@@ -481,6 +537,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                     }
                     for (; j < j1; ++j) acc[0] = fmaf(ld_cg1(fcol + (int64_t)j * n), fs[j], acc[0]);
                 }
+            } else if (VEC == 4 && KRES && primed && base == 0) {
+                cp_async_wait<0>();  // the primed (empty) groups of a thread without rows
             }
             if (JG > 1) {
                 if (g > 0) {
@@ -496,34 +554,70 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                         for (int k = 0; k < VEC; ++k) acc[k] += src[k];
                     }
                 }
+            } else if (base == 0) {
+                __syncthreads();  // g_s of warp 0
             }
-            if (g == 0 && valid) {
-                float out[VEC];
+            if (base == 0 && imisc[4]) {  // uniform: read after a barrier
+                stop = true;
+                break;
+            }
+            const float gs = misc[2];
+            const float piv = sqrtf(gs);
+            if (g == 0) {
+                double p = 0.0;
+                if (valid) {
+                    float out[VEC];
 #pragma unroll
-                for (int k = 0; k < VEC; ++k) {
-                    const int64_t l = row0 + row + k;
-                    float gl = expf(beta * (dotb[row + k] - MK)) - acc[k];
-                    if (l == s) gl = gs;
-                    const float f = gl / piv;
-                    out[k] = f;
-                    float dn = fmaxf(dcur[row + k] - f * f, 0.f);
-                    if (l == s) dn = 0.f;
-                    dnxt[row + k] = dn;
+                    for (int k = 0; k < VEC; ++k) {
+                        const int64_t l = row0 + row + k;
+                        float gl = expf(beta * (dotb[row + k] - MK)) - acc[k];
+                        if (l == s) gl = gs;
+                        const float f = gl / piv;
+                        out[k] = f;
+                        float dn = fmaxf(dcur[row + k] - f * f, 0.f);
+                        if (l == s) dn = 0.f;
+                        dnxt[row + k] = dn;
+                        p += (double)dn;
+                    }
+                    float* dstF = Fb + (int64_t)i * n + row0 + row;
+                    if constexpr (VEC == 4) {
+                        *reinterpret_cast<float4*>(dstF) = make_float4(out[0], out[1], out[2], out[3]);
+                    } else {
+                        dstF[0] = out[0];
+                    }
                 }
-                float* dstF = Fb + (int64_t)i * n + row0 + row;
-                if constexpr (VEC == 4) {
-                    *reinterpret_cast<float4*>(dstF) = make_float4(out[0], out[1], out[2], out[3]);
-                } else {
-                    dstF[0] = out[0];
+                if (fused_csl) {  // the search's chunk arithmetic: four in order per lane, then the warp scan
+                    const double incl = warp_scan_incl(p, lane);
+                    const int ch = (base >> 7) + (tt >> 5);
+                    if (lane == 31 && ch < nch) csl[ch] = incl;
                 }
             }
             if (JG > 1) __syncthreads();
         }
-        // rows of the slice past n keep zero mass
+        if (nrows == 0) {  // a CTA without rows takes the same barrier and stop test as the others
+            __syncthreads();
+            stop = imisc[4] != 0;
+        }
+        if (stop) break;
+        // rows of the slice past n keep zero mass; chunks no row block reached sum to zero
         for (int row = nrows + tid; row < Rpad; row += NT) dnxt[row] = 0.f;
+        if (fused_csl) {
+            const int covered = (int)(ceil_div(nrows, TPG * VEC) * (TPG * VEC / 128));
+            for (int k = covered + tid; k < nch; k += NT) csl[k] = 0.0;
+        }
         __syncthreads();
-        publish(dnxt, nxt);
+        // the next step's first ring items, in flight across the cluster barrier and the search
+        primed = i + 1 < r;
+        if (primed) {
+            if constexpr (KRES) {
+                if (VEC == 4) fpass_prime(i + 1);
+            } else {
+                key_prime();
+            }
+        }
+        publish(dnxt, nxt, fused_csl, i + 1);
     }
+    cp_async_wait<0>();  // a primed step that never ran
 
     // ---------------- effective rank, padding past it ----------------
     const int rr = i;
