@@ -105,6 +105,7 @@ SELECT_KERNELS = {
     1: ("rpc_select_kernel", "rpc_select", ("select.cu", "common.cuh", "philox.cuh")),
     2: ("rpc_select_bulk_kernel", "rpc_select_bulk",
         ("select_bulk.cu", "common.cuh", "philox.cuh", "tc_common.cuh")),
+    3: ("rpc_select_kernel (global sync)", "rpc_select_gs", ("select.cu", "common.cuh", "philox.cuh")),
 }
 
 

@@ -112,6 +112,25 @@ wildcat_status wildcat_select(const void* K, int dtype, int64_t BH, int64_t n, i
                               int32_t* rank, void* K_S, void* stream);
 
 /*
+ * wildcat_select_ws -- wildcat_select with a workspace (>= wildcat_select_
+ * workspace_size(BH, n) bytes, 256-byte aligned, owned by the caller).  With
+ * it the library may run the global-sync form of the select kernel: when
+ * there are few instances (BH well below the SM count) each instance gets
+ * up to 32 CTAs that meet at a counter barrier in the workspace instead of
+ * a thread-block cluster (clusters of 16 CTAs must share one GPC, so few fit
+ * at once).  The grid is launched cooperatively (all CTAs co-resident); every
+ * barrier wait is bounded (2 s, WILDCAT_ERR_TIMEOUT in the device status
+ * word on expiry).  Results equal wildcat_select's to float32 rounding.
+ * workspace may be NULL (then exactly wildcat_select).  wildcat_forward*
+ * carve this workspace from theirs.
+ */
+size_t wildcat_select_workspace_size(int64_t BH, int64_t n);
+wildcat_status wildcat_select_ws(const void* K, int dtype, int64_t BH, int64_t n, int d, float beta,
+                                 int r, uint64_t seed, int64_t inst0, float eps, int32_t* S,
+                                 float* F, int32_t* rank, void* K_S, void* workspace,
+                                 size_t ws_bytes, void* stream);
+
+/*
  * wildcat_select_fixed -- the same factorisation with the pivots given
  * (test entry point: lets the device path run on the oracle's pivots).
  * S_fixed [BH, r] int32; a negative or out-of-range entry ends that
@@ -384,10 +403,13 @@ wildcat_status wildcat_test_force_select_timeout(int64_t nanoseconds);
 
 /*
  * wildcat_set_select_kernel -- which select kernel wildcat_select* launch:
- * 0 (default) and 1 the cp.async kernel (per-thread asynchronous copies);
- * 2 the bulk-copy kernel (copy-engine stages on mbarriers) wherever it
- * applies (n % 4 == 0, n / cluster size <= 8192, 16-byte aligned K and F,
- * d in {32, 64, 128}), else the cp.async kernel.  Both compute the same
+ * 0 (default) the cp.async kernel (per-thread asynchronous copies), in its
+ * global-sync form when a workspace is given and that form has less work per
+ * CTA; 1 the cp.async kernel on clusters only; 2 the bulk-copy kernel
+ * (copy-engine stages on mbarriers) wherever it applies (n % 4 == 0,
+ * n / cluster size <= 8192, 16-byte aligned K and F, d in {32, 64, 128}),
+ * else the cp.async kernel; 3 the global-sync form wherever a workspace is
+ * given and all CTAs fit at once.  Both compute the same
  * factorisation (results agree to float32 rounding).  Process-wide; not
  * thread-safe against concurrent select calls.  Returns
  * WILDCAT_ERR_INVALID_ARG for other values.
@@ -395,7 +417,8 @@ wildcat_status wildcat_test_force_select_timeout(int64_t nanoseconds);
 wildcat_status wildcat_set_select_kernel(int kernel);
 
 /* The select kernel the last select launch on this thread used: 1 the
- * cp.async kernel, 2 the bulk-copy kernel, 0 if none. */
+ * cp.async kernel on clusters, 2 the bulk-copy kernel, 3 the cp.async
+ * kernel in global-sync form, 0 if none. */
 int wildcat_last_select_kernel(void);
 
 /*

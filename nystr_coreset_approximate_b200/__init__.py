@@ -52,6 +52,9 @@ _SIGS = {
     "wildcat_weights_workspace_size": ([_i64, _i64, _int, _int], _sz),
     "wildcat_weights": ([_vp, _vp, _vp, _vp, _int, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _sz,
                          _vp], _int),
+    "wildcat_select_workspace_size": ([_i64, _i64], _sz),
+    "wildcat_select_ws": ([_vp, _int, _i64, _i64, _int, _f32, _int, _u64, _i64, _f32, _vp, _vp, _vp, _vp, _vp,
+                           _sz, _vp], _int),
     "wildcat_weights_inverse_workspace_size": ([_i64, _i64, _int, _int], _sz),
     "wildcat_weights_inverse": ([_vp, _vp, _int, _vp, _vp, _i64, _i64, _int, _int, _f32, _vp, _vp, _vp,
                                  _vp, _vp, _sz, _vp], _int),
@@ -185,11 +188,14 @@ def select(K, beta: float, r: int, seed: int = 0, eps: float = 1e-6, *, inst0: i
         torch.empty((BH, r, n), dtype=torch.float32, device=K.device),
         torch.empty((BH,), dtype=torch.int32, device=K.device),
         torch.empty((BH, r, d), dtype=K.dtype, device=K.device))
-    _check(lib().wildcat_select(_dev(K, "K"), _dtype_code(K), BH, n, d, float(beta), int(r),
-                                int(seed) & (2**64 - 1), int(inst0), float(eps),
-                                _dev(S, "S", torch.int32),
-                                _dev(F, "F", torch.float32), _dev(rank, "rank", torch.int32),
-                                _opt(K_S, "K_S", K.dtype), _stream(stream)))
+    L = lib()
+    nbytes = int(L.wildcat_select_workspace_size(BH, n))
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=K.device)
+    _check(L.wildcat_select_ws(_dev(K, "K"), _dtype_code(K), BH, n, d, float(beta), int(r),
+                               int(seed) & (2**64 - 1), int(inst0), float(eps),
+                               _dev(S, "S", torch.int32),
+                               _dev(F, "F", torch.float32), _dev(rank, "rank", torch.int32),
+                               _opt(K_S, "K_S", K.dtype), _dev(ws, "workspace"), nbytes, _stream(stream)))
     return S, F, rank, K_S
 
 
@@ -488,8 +494,9 @@ def last_select_cluster() -> int:
 
 
 def set_select_kernel(kernel: int):
-    """0 = automatic (the cp.async kernel), 1 = the cp.async kernel, 2 = the
-    bulk-copy kernel where it applies."""
+    """0 = automatic, 1 = the cp.async kernel on clusters, 2 = the bulk-copy
+    kernel where it applies, 3 = the cp.async kernel in global-sync form where
+    it applies."""
     _check(lib().wildcat_set_select_kernel(int(kernel)))
 
 

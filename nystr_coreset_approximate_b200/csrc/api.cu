@@ -60,7 +60,7 @@ wildcat_status check_scalars(float beta, float eps, const char* who) {
 
 wildcat_status select_impl(const void* K, int dtype, int64_t BH, int64_t n, int d, float beta, int r, uint64_t seed,
                            int64_t inst0, float eps, const int32_t* S_fixed, int32_t* S, float* F, int32_t* rank,
-                           void* K_S, void* stream, const char* who) {
+                           void* K_S, void* stream, const char* who, void* ws = nullptr, size_t ws_bytes = 0) {
     wildcat_status st = check_common(dtype, BH, n, d, r, who);
     if (st != WILDCAT_OK) return st;
     if ((st = check_scalars(beta, eps, who)) != WILDCAT_OK) return st;
@@ -70,7 +70,10 @@ wildcat_status select_impl(const void* K, int dtype, int64_t BH, int64_t n, int 
     if (!S_fixed && !S) return bad(1, "%s: S must be non-null", who);
     if (!aligned16(K) || !aligned16(F) || (K_S && !aligned16(K_S)))
         return bad(1, "%s: K, F and K_S must be 16-byte aligned", who);
+    if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
     wildcat::SelectRequest q{K, dtype, BH, n, d, beta, r, seed, inst0, eps, S_fixed, S, F, rank, K_S};
+    q.ws = ws;
+    q.ws_bytes = ws_bytes;
     return record(wildcat::launch_select(q, static_cast<cudaStream_t>(stream)));
 }
 
@@ -87,6 +90,8 @@ struct ForwardLayout {
     size_t wws_bytes;
     void* aws;
     size_t aws_bytes;
+    void* sws;  // select workspace (global-sync mode)
+    size_t sws_bytes;
 };
 
 ForwardLayout carve_forward(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, int r, int dtype) {
@@ -103,6 +108,8 @@ ForwardLayout carve_forward(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, 
     L.wws = cv.take(L.wws_bytes);
     L.aws_bytes = wildcat::attend_workspace_bytes(BH, m, d, r);
     L.aws = cv.take(L.aws_bytes);
+    L.sws_bytes = wildcat::select_workspace_bytes(BH, n);
+    L.sws = cv.take(L.sws_bytes);
     return L;
 }
 
@@ -115,6 +122,8 @@ wildcat_status forward_impl(const void* Q, const void* K, const void* V, int dty
     Status s;
     cudaError_t ew;
     wildcat::SelectRequest sq{K, dtype, BH, n, d, beta, r, seed, inst0, eps, nullptr, L.S, L.F, L.rank, L.K_S};
+    sq.ws = L.sws;
+    sq.ws_bytes = L.sws_bytes;
     if ((s = wildcat::launch_select(sq, st)).code) return record(s);
     if (wait_v && (ew = cudaStreamWaitEvent(st, wait_v, 0))) return record(Status::cuda(ew, "forward: wait for V"));
     wildcat::WeightsRequest wq{L.F, L.S, L.rank, V, dtype, BH, n, d, r, L.V_S, L.w, L.vmin, L.vmax, L.wws,
@@ -152,6 +161,8 @@ struct BinnedLayout {
     size_t aws_bytes;
     float* kbar;   // recentring only
     void* mws;
+    void* sws;     // select workspace (global-sync mode)
+    size_t sws_bytes;
 };
 
 BinnedLayout carve_binned(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, int r, int nbins, int dtype,
@@ -177,6 +188,8 @@ BinnedLayout carve_binned(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, in
     L.aws = cv.take(L.aws_bytes);
     L.kbar = recenter ? static_cast<float*>(cv.take(sizeof(float) * BH * d)) : nullptr;
     L.mws = recenter ? cv.take(wildcat::key_mean_workspace_bytes(BH, n, d)) : nullptr;
+    L.sws_bytes = wildcat::select_workspace_bytes(BB, nb);
+    L.sws = cv.take(L.sws_bytes);
     return L;
 }
 
@@ -218,7 +231,8 @@ HostPipe* host_pipe(int dev) {
 
 namespace wildcat {
 int read_device_status(bool clear) {
-    const int parts[3] = {read_attend_status(clear), read_weights_status(clear), read_select_status(clear)};
+    const int parts[4] = {read_attend_status(clear), read_weights_status(clear), read_select_status(clear),
+                          read_select_gs_status(clear)};
     for (const int v : parts)
         if (v < 0) return -1;
     for (const int v : parts)
@@ -250,6 +264,18 @@ wildcat_status wildcat_select(const void* K, int dtype, int64_t BH, int64_t n, i
                               void* stream) {
     return select_impl(K, dtype, BH, n, d, beta, r, seed, inst0, eps, nullptr, S, F, rank, K_S, stream,
                        "wildcat_select");
+}
+
+size_t wildcat_select_workspace_size(int64_t BH, int64_t n) {
+    if (BH < 0 || n < 1) return 0;
+    return wildcat::select_workspace_bytes(BH, n);
+}
+
+wildcat_status wildcat_select_ws(const void* K, int dtype, int64_t BH, int64_t n, int d, float beta, int r,
+                                 uint64_t seed, int64_t inst0, float eps, int32_t* S, float* F, int32_t* rank,
+                                 void* K_S, void* workspace, size_t ws_bytes, void* stream) {
+    return select_impl(K, dtype, BH, n, d, beta, r, seed, inst0, eps, nullptr, S, F, rank, K_S, stream,
+                       "wildcat_select_ws", workspace, ws_bytes);
 }
 
 wildcat_status wildcat_select_fixed(const void* K, int dtype, int64_t BH, int64_t n, int d, float beta, int r,
@@ -438,6 +464,8 @@ wildcat_status wildcat_forward_ex(const void* Q, const void* K, const void* V, i
     if (recenter && (z = wildcat::launch_key_mean(K, dtype, BH, n, d, L.mws, L.kbar, s)).code) return record(z);
     wildcat::SelectRequest sq{K, dtype, BB, nb, d, beta_key, rb, seed, inst0 * nbins, eps, nullptr, L.S, L.F, L.rank_b,
                               L.K_S, L.kbar, nbins};
+    sq.ws = L.sws;
+    sq.ws_bytes = L.sws_bytes;
     if ((z = wildcat::launch_select(sq, s)).code) return record(z);
     wildcat::WeightsRequest wq{L.F, L.S, L.rank_b, V, dtype, BB, nb, d, rb, L.V_S, L.w, L.vmin_b, L.vmax_b, L.wws,
                                L.wws_bytes};
@@ -573,8 +601,9 @@ wildcat_status wildcat_test_force_select_timeout(int64_t nanoseconds) {
 }
 
 wildcat_status wildcat_set_select_kernel(int kernel) {
-    if (kernel < 0 || kernel > 2)
-        return bad(1, "%s: kernel must be 0 (automatic), 1 (cp.async) or 2 (bulk-copy)", "wildcat_set_select_kernel");
+    if (kernel < 0 || kernel > 3)
+        return bad(1, "%s: kernel must be 0 (automatic), 1 (cp.async), 2 (bulk-copy) or 3 (global sync)",
+                   "wildcat_set_select_kernel");
     wildcat::select_kernel_override(kernel);
     return record(Status::ok());
 }

@@ -34,14 +34,17 @@ struct SelectRequest {
     void* K_S;
     const float* kbar = nullptr;  // recentring: per-instance key mean (or nullptr)
     int kbar_div = 1;             // instance b uses kbar row b / kbar_div
+    void* ws = nullptr;           // optional workspace (global-sync mode), 256-byte aligned
+    size_t ws_bytes = 0;
 };
 
 Status launch_select(const SelectRequest& q, cudaStream_t stream);
 Status launch_pivot_uniforms(uint64_t seed, int64_t BH, int steps, double* u, cudaStream_t stream);
 int select_cluster_override(int G);  // G < 0: query only
 int last_select_cluster();
-int select_kernel_override(int k);  // k < 0: query only; 0 automatic, 1 the cp.async kernel, 2 the bulk-copy kernel
-int last_select_kernel();           // 1 cp.async kernel, 2 bulk-copy kernel
+int select_kernel_override(int k);  // k < 0: query only; 0 automatic, 1 cp.async (clusters), 2 bulk-copy,
+                                    // 3 cp.async with global sync where a workspace allows
+int last_select_kernel();           // 1 cp.async (clusters), 2 bulk-copy, 3 cp.async (global sync)
 // cluster-size choice shared by both select kernels (select.cu)
 struct ClusterKey {
     int dev, kernel;
@@ -51,7 +54,9 @@ struct ClusterKey {
 };
 int cached_cluster_lookup(const ClusterKey& key);   // 0 if absent
 void cached_cluster_store(const ClusterKey& key, int G);
-int choose_cluster_rows(int64_t n, int64_t BH, int (*fit)(int G, void* ctx), void* ctx);
+int choose_cluster_rows(int64_t n, int64_t BH, int (*fit)(int G, void* ctx), void* ctx, double* cost_out);
+size_t select_workspace_bytes(int64_t BH, int64_t n);  // global-sync exchange buffers
+int read_select_gs_status(bool clear);
 // bulk-copy select kernel (select_bulk.cu); *used = false when the shape is not one it handles.
 // G_override > 0 fixes the cluster size.
 Status launch_select_bulk(const SelectRequest& q, int G_override, cudaStream_t stream, bool* used, int* G_used);

@@ -58,16 +58,22 @@ struct SelectArgs {
     int R;      // rows per CTA, multiple of 4
     int JG;     // thread groups splitting factor columns / head dim
     int PL;     // residual values per lane in one search chunk (multiple of 4)
+    // global-sync mode (the CTAs of an instance are not a cluster): exchange buffers
+    double* gs_inbox;  // [BH][2][G][33] chunk sums + total per CTA
+    float* gs_resid;   // [BH][2][G][Rpad] residual diagonal copies
+    unsigned* gs_bar;  // [BH] barrier counters, zero at launch
+    float* gs_mk;      // [BH][G] per-CTA max |k|^2
+    int gs;            // 1: the launch is the global-sync one
 };
 
 struct SmemLayout {
     size_t ring, kres, inbox, csl, dbuf, dotb, ks, fs, red, misc, total;
     __host__ __device__ SmemLayout(int Rpad, int r, int D, int JG, int NT, int VEC, int G, int depth,
-                                   size_t kres_bytes) {
+                                   size_t kres_bytes, bool gs = false) {
         size_t o = 0;
         ring = o;  o += (size_t)depth * NT * 16;               // per-thread cp.async ring, [slot][thread] x 16 B
         kres = o;  o += round_up(kres_bytes, 16);              // the CTA's key rows, when resident
-        inbox = o; o += 2 * (size_t)G * 33 * sizeof(double);  // [parity][source CTA][32 chunk sums + total]
+        inbox = o; o += gs ? 0 : 2 * (size_t)G * 33 * sizeof(double);  // [parity][source CTA][32 chunk sums + total]
         csl = o;   o += 32 * sizeof(double);                   // own chunk sums
         dbuf = o;  o += 2 * (size_t)Rpad * sizeof(float);      // residual diagonal, double-buffered
         dotb = o;  o += (size_t)Rpad * sizeof(float);          // <k_l, k_s> of the step
@@ -97,6 +103,21 @@ __device__ __forceinline__ double chunk_total(const float* chunk, int PL, int la
     return __shfl_sync(0xffffffffu, warp_scan_incl(s, lane), 31);
 }
 
+// Global-sync mode helpers: acquire load of a barrier counter, the clock for
+// the bounded wait, and the status word a timed-out wait records.
+constexpr unsigned long long kGsWaitNs = 2000000000ull;
+__device__ int g_select_gs_status = 0;
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ unsigned long long gs_clock() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 // cp.async helpers (16-byte copies global -> shared, L2 only)
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
     const unsigned d = (unsigned)__cvta_generic_to_shared(smem_dst);
@@ -112,9 +133,12 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-template <typename E, int D, int VEC, int DEPTH, bool KRES>
+template <typename E, int D, int VEC, int DEPTH, bool KRES, bool GS>
 __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const SelectArgs a) {
-    // Launched with a cluster dimension of a.G (one cluster per instance).
+    // Launched with a cluster dimension of a.G (one cluster per instance), or,
+    // with GS, as one cooperative grid whose a.G CTAs per instance exchange
+    // chunk sums and residuals through global memory and meet at a counter
+    // barrier (all CTAs are co-resident by the cooperative launch).
     using T = typename E::T;
     constexpr int NT = kSelectThreads, NW = NT / 32;
     constexpr int EPL = 16 / (int)sizeof(T);  // key elements per 16-byte load
@@ -122,7 +146,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     constexpr int RPW = 32 / LPR;             // key rows per warp-wide load
     constexpr int UF = 8;                     // factor loads in flight per thread (scalar path)
     cg::cluster_group cluster = cg::this_cluster();
-    const int crank = (int)cluster.block_rank();
+    const int crank = GS ? (int)(blockIdx.x % a.G) : (int)cluster.block_rank();
     const int64_t b = blockIdx.x / a.G;
     if (b >= a.BH) return;  // whole clusters only: G divides gridDim.x
 
@@ -137,7 +161,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     const int Rpad = nch * CH;  // residual buffers cover whole search chunks
 
     extern __shared__ __align__(16) unsigned char smem[];
-    const SmemLayout L(Rpad, r, D, JG, NT, VEC, G, DEPTH, KRES ? (size_t)R * D * sizeof(T) : 0);
+    const SmemLayout L(Rpad, r, D, JG, NT, VEC, G, DEPTH, KRES ? (size_t)R * D * sizeof(T) : 0, GS);
     // Each thread streams through its own DEPTH slots of 16 bytes
     // (slot q of thread t at ring4[q * NT + t]); it only ever reads slots it
     // filled itself, so the pipeline needs no barrier.  A slot is refilled
@@ -152,7 +176,37 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     float* red = reinterpret_cast<float*>(smem + L.red);
     float* misc = reinterpret_cast<float*>(smem + L.misc);
     int* imisc = reinterpret_cast<int*>(misc);
-    // misc[0] local max |k|^2, misc[1] M_K, misc[2] g_s, imisc[3] s, imisc[4] stop
+    // misc[0] local max |k|^2, misc[1] M_K, misc[2] g_s, imisc[3] s, imisc[4] stop, imisc[5] abort (GS)
+
+    // Global-sync mode: the instance's barrier is a counter in global memory;
+    // barrier k completes when all G CTAs have added one for it.  The wait is
+    // bounded (2 s): on expiry the CTA records WILDCAT_ERR_TIMEOUT and stops
+    // (its peers then run out at their next barrier).  Peer data is read with
+    // L2-only loads after the barrier.
+    int gs_k = 0;
+    auto gsync = [&]() -> bool {
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            atomicAdd(a.gs_bar + b, 1u);
+            const unsigned target = (unsigned)G * (unsigned)(gs_k + 1);
+            const unsigned long long t0 = gs_clock();
+            while (ld_acquire_u32(a.gs_bar + b) < target) {
+                if (gs_clock() - t0 > kGsWaitNs) {
+                    imisc[5] = 1;
+                    atomicExch(&g_select_gs_status, 5);
+                    break;
+                }
+            }
+            __threadfence();
+        }
+        ++gs_k;
+        __syncthreads();
+        return imisc[5] == 0;
+    };
+    if (GS && tid == 0) imisc[5] = 0;
+    auto ginbox = [&](int par, int c) -> double* { return a.gs_inbox + (((size_t)b * 2 + par) * G + c) * 33; };
+    auto gres = [&](int par) -> float* { return a.gs_resid + (((size_t)b * 2 + par) * G + crank) * (size_t)Rpad; };
 
     const T* Kb = reinterpret_cast<const T*>(a.K) + b * n * D;
     float* Fb = a.F + b * (int64_t)r * n;
@@ -280,18 +334,30 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
             }
             __syncthreads();
         }
-        if (warp == 0) {
-            const double v = lane < nch ? csl[lane] : 0.0;
-            const double tot = __shfl_sync(0xffffffffu, warp_scan_incl(v, lane), 31);
-            for (int c = 0; c < G; ++c) {
-                double* dst = cluster.map_shared_rank(inbox + ((size_t)par * G + crank) * 33, c);
+        if constexpr (GS) {
+            if (warp == 0) {
+                const double v = lane < nch ? csl[lane] : 0.0;
+                const double tot = __shfl_sync(0xffffffffu, warp_scan_incl(v, lane), 31);
+                double* dst = ginbox(par, crank);
                 if (lane < nch) dst[lane] = v;
                 if (lane == 0) dst[32] = tot;
+                u_next = pivot_uniform(a.seed, (uint32_t)next_step, (uint32_t)(a.inst0 + b));
             }
+            gsync();
+        } else {
+            if (warp == 0) {
+                const double v = lane < nch ? csl[lane] : 0.0;
+                const double tot = __shfl_sync(0xffffffffu, warp_scan_incl(v, lane), 31);
+                for (int c = 0; c < G; ++c) {
+                    double* dst = cluster.map_shared_rank(inbox + ((size_t)par * G + crank) * 33, c);
+                    if (lane < nch) dst[lane] = v;
+                    if (lane == 0) dst[32] = tot;
+                }
+            }
+            cluster.barrier_arrive();
+            if (warp == 0) u_next = pivot_uniform(a.seed, (uint32_t)next_step, (uint32_t)(a.inst0 + b));
+            cluster.barrier_wait();
         }
-        cluster.barrier_arrive();
-        if (warp == 0) u_next = pivot_uniform(a.seed, (uint32_t)next_step, (uint32_t)(a.inst0 + b));
-        cluster.barrier_wait();
     };
 
     // ---------------- prologue: M_K and the initial residual diagonal ----------------
@@ -320,19 +386,35 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
         v = warp_max(v);
         if (lane == 0) misc[0] = v;
     }
-    cluster.sync();
-    if (warp == 0) {
-        float v = -INFINITY;
-        if (lane < G) v = *cluster.map_shared_rank(&misc[0], lane);
-        v = warp_max(v);
-        if (lane == 0) misc[1] = v;
+    if constexpr (GS) {
+        if (tid == 0) a.gs_mk[b * G + crank] = misc[0];
+        gsync();
+        if (warp == 0) {
+            float v = -INFINITY;
+            if (lane < G) v = __ldcg(a.gs_mk + b * G + lane);
+            v = warp_max(v);
+            if (lane == 0) misc[1] = v;
+        }
+    } else {
+        cluster.sync();
+        if (warp == 0) {
+            float v = -INFINITY;
+            if (lane < G) v = *cluster.map_shared_rank(&misc[0], lane);
+            v = warp_max(v);
+            if (lane == 0) misc[1] = v;
+        }
     }
     __syncthreads();
     const float MK = misc[1];
     const float beta = a.beta;
-    for (int row = tid; row < Rpad; row += NT) dbuf[row] = row < nrows ? expf(beta * (dotb[row] - MK)) : 0.f;
+    for (int row = tid; row < Rpad; row += NT) {
+        const float v = row < nrows ? expf(beta * (dotb[row] - MK)) : 0.f;
+        dbuf[row] = v;
+        if constexpr (GS) gres(0)[row] = v;
+    }
     __syncthreads();
     publish(dbuf, 0, false, 0);
+    const bool gs_ok = !(GS && imisc[5]);
 
     // ---------------- r sequential steps ----------------
     // The epilogue forms the search's chunk sums itself when a chunk is
@@ -356,7 +438,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     };
     bool primed = false;  // the next step's first ring items are in flight
     int i = 0;
-    for (; i < r; ++i) {
+    for (; gs_ok && i < r; ++i) {
         const int cur = i & 1, nxt = cur ^ 1;
         float* dcur = dbuf + (size_t)cur * Rpad;
         float* dnxt = dbuf + (size_t)nxt * Rpad;
@@ -369,7 +451,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                 const int sf = a.S_fixed[b * r + i];
                 s = (sf >= 0 && (int64_t)sf < n) ? sf : -1;
             } else {
-                const double tc = lane < G ? ib[lane * 33 + 32] : 0.0;
+                const double tc = lane < G ? (GS ? __ldcg(ginbox(cur, lane) + 32) : ib[lane * 33 + 32]) : 0.0;
                 const double incl = warp_scan_incl(tc, lane);
                 const double T = __shfl_sync(0xffffffffu, incl, 31);
                 const unsigned pos_cta = __ballot_sync(0xffffffffu, tc > 0.0);
@@ -380,7 +462,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                     const int owner = m ? __ffs(m) - 1 : 31 - __clz(pos_cta);
                     const double t1 = t - __shfl_sync(0xffffffffu, incl - tc, owner);
                     // owner's chunk (its chunk sums are in the local inbox)
-                    const double cv = lane < nch ? ib[owner * 33 + lane] : 0.0;
+                    const double cv =
+                        lane < nch ? (GS ? __ldcg(ginbox(cur, owner) + lane) : ib[owner * 33 + lane]) : 0.0;
                     const double ci = warp_scan_incl(cv, lane);
                     const unsigned pos_ch = __ballot_sync(0xffffffffu, cv > 0.0);
                     if (pos_ch) {  // warp-uniform; a positive total implies a positive chunk
@@ -388,11 +471,18 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                         const int chunk = m ? __ffs(m) - 1 : 31 - __clz(pos_ch);
                         const double t2 = t1 - __shfl_sync(0xffffffffu, ci - cv, chunk);
                         // row inside the chunk: one read of the owner's residuals
-                        const float* rd =
-                            cluster.map_shared_rank(dbuf + (size_t)cur * Rpad, owner) + (size_t)chunk * CH;
                         float vals[kMaxPL];
+                        if constexpr (GS) {
+                            const float* rd = a.gs_resid + (((size_t)b * 2 + cur) * G + owner) * (size_t)Rpad +
+                                              (size_t)chunk * CH;
 #pragma unroll
-                        for (int k = 0; k < kMaxPL; ++k) vals[k] = k < PL ? rd[lane * PL + k] : 0.f;
+                            for (int k = 0; k < kMaxPL; ++k) vals[k] = k < PL ? __ldcg(rd + lane * PL + k) : 0.f;
+                        } else {
+                            const float* rd =
+                                cluster.map_shared_rank(dbuf + (size_t)cur * Rpad, owner) + (size_t)chunk * CH;
+#pragma unroll
+                            for (int k = 0; k < kMaxPL; ++k) vals[k] = k < PL ? rd[lane * PL + k] : 0.f;
+                        }
                         double part = 0.0;
 #pragma unroll
                         for (int k = 0; k < kMaxPL; ++k)
@@ -577,6 +667,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                         float dn = fmaxf(dcur[row + k] - f * f, 0.f);
                         if (l == s) dn = 0.f;
                         dnxt[row + k] = dn;
+                        if constexpr (GS) gres(nxt)[row + k] = dn;
                         p += (double)dn;
                     }
                     float* dstF = Fb + (int64_t)i * n + row0 + row;
@@ -600,7 +691,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
         }
         if (stop) break;
         // rows of the slice past n keep zero mass; chunks no row block reached sum to zero
-        for (int row = nrows + tid; row < Rpad; row += NT) dnxt[row] = 0.f;
+        for (int row = nrows + tid; row < Rpad; row += NT) {
+            dnxt[row] = 0.f;
+            if constexpr (GS) gres(nxt)[row] = 0.f;
+        }
         if (fused_csl) {
             const int covered = (int)(ceil_div(nrows, TPG * VEC) * (TPG * VEC / 128));
             for (int k = covered + tid; k < nch; k += NT) csl[k] = 0.0;
@@ -616,6 +710,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
             }
         }
         publish(dnxt, nxt, fused_csl, i + 1);
+        if (GS && imisc[5]) break;  // a barrier ran out (uniform: read after the barrier's block sync)
     }
     cp_async_wait<0>();  // a primed step that never ran
 
@@ -635,7 +730,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
         }
     }
     // keep this CTA's shared memory alive until every peer is done reading it
-    cluster.sync();
+    if constexpr (!GS) cluster.sync();
 }
 
 __global__ void pivot_uniform_kernel(uint64_t seed, int64_t BH, int steps, double* u) {
@@ -646,12 +741,12 @@ __global__ void pivot_uniform_kernel(uint64_t seed, int64_t BH, int steps, doubl
     u[t] = pivot_uniform(seed, (uint32_t)i, (uint32_t)b);
 }
 
-template <typename E, int D, int VEC, int DEPTH, bool KRES>
+template <typename E, int D, int VEC, int DEPTH, bool KRES, bool GS>
 cudaError_t launch_select_t(const SelectArgs& a, size_t smem, cudaStream_t stream) {
-    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KRES>;
+    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KRES, GS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    if (a.G > 8) {
+    if (!GS && a.G > 8) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
     }
@@ -661,22 +756,44 @@ cudaError_t launch_select_t(const SelectArgs& a, size_t smem, cudaStream_t strea
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = a.G;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    if (GS) {
+        // every CTA of the grid is co-resident, or the launch fails
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    } else {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = a.G;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+    }
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <typename E, int D, int VEC, int DEPTH, bool KRES>
-int max_clusters_t(int G, size_t smem) {
-    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KRES>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+// Clusters of G CTAs that fit at once (cluster mode) or CTAs that fit at
+// once on the whole GPU (global-sync mode).
+template <typename E, int D, int VEC, int DEPTH, bool KRES, bool GS>
+int fit_t(int G, size_t smem) {
+    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KRES, GS>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+        cudaGetLastError();
         return 0;
-    if (G > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+    }
+    if (GS) {
+        int per_sm = 0, dev = 0, sms = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSelectThreads, smem) != cudaSuccess ||
+            cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        return per_sm * sms;
+    }
+    if (G > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+        cudaGetLastError();
         return 0;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)G);
     cfg.blockDim = dim3(kSelectThreads);
@@ -696,18 +813,18 @@ int max_clusters_t(int G, size_t smem) {
     return nc;
 }
 
-template <typename E, int VEC, int DEPTH, bool KRES>
+template <typename E, int VEC, int DEPTH, bool KRES, bool GS>
 int dispatch_d(int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int G_query, cudaError_t* err) {
     switch (d) {
         case 32:
-            if (a) { *err = launch_select_t<E, 32, VEC, DEPTH, KRES>(*a, smem, stream); return 0; }
-            return max_clusters_t<E, 32, VEC, DEPTH, KRES>(G_query, smem);
+            if (a) { *err = launch_select_t<E, 32, VEC, DEPTH, KRES, GS>(*a, smem, stream); return 0; }
+            return fit_t<E, 32, VEC, DEPTH, KRES, GS>(G_query, smem);
         case 64:
-            if (a) { *err = launch_select_t<E, 64, VEC, DEPTH, KRES>(*a, smem, stream); return 0; }
-            return max_clusters_t<E, 64, VEC, DEPTH, KRES>(G_query, smem);
+            if (a) { *err = launch_select_t<E, 64, VEC, DEPTH, KRES, GS>(*a, smem, stream); return 0; }
+            return fit_t<E, 64, VEC, DEPTH, KRES, GS>(G_query, smem);
         case 128:
-            if (a) { *err = launch_select_t<E, 128, VEC, DEPTH, KRES>(*a, smem, stream); return 0; }
-            return max_clusters_t<E, 128, VEC, DEPTH, KRES>(G_query, smem);
+            if (a) { *err = launch_select_t<E, 128, VEC, DEPTH, KRES, GS>(*a, smem, stream); return 0; }
+            return fit_t<E, 128, VEC, DEPTH, KRES, GS>(G_query, smem);
     }
     if (err) *err = cudaErrorInvalidValue;
     return 0;
@@ -715,28 +832,41 @@ int dispatch_d(int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int
 
 // Kernel variants: the vectorised path with ring depth 24/16/12/6 (12 also
 // with resident keys); the scalar path (n not a multiple of 4) with depth 6.
+// The global-sync mode exists for the vectorised streamed-key variants.
 struct Variant {
     int depth;
     bool kres;
 };
 
 template <typename E>
-int dispatch_e(const Variant& v, int vec, int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int G_query,
-               cudaError_t* err) {
-    if (vec != 4) return dispatch_d<E, 1, 6, false>(d, a, smem, stream, G_query, err);
-    if (v.kres) return dispatch_d<E, 4, 12, true>(d, a, smem, stream, G_query, err);
-    switch (v.depth) {
-        case 24: return dispatch_d<E, 4, 24, false>(d, a, smem, stream, G_query, err);
-        case 16: return dispatch_d<E, 4, 16, false>(d, a, smem, stream, G_query, err);
-        case 12: return dispatch_d<E, 4, 12, false>(d, a, smem, stream, G_query, err);
+int dispatch_e(const Variant& v, int vec, int d, bool gs, const SelectArgs* a, size_t smem, cudaStream_t stream,
+               int G_query, cudaError_t* err) {
+    if (gs) {
+        if (vec != 4 || v.kres) {
+            if (err) *err = cudaErrorInvalidValue;
+            return 0;
+        }
+        switch (v.depth) {
+            case 24: return dispatch_d<E, 4, 24, false, true>(d, a, smem, stream, G_query, err);
+            case 16: return dispatch_d<E, 4, 16, false, true>(d, a, smem, stream, G_query, err);
+            case 12: return dispatch_d<E, 4, 12, false, true>(d, a, smem, stream, G_query, err);
+        }
+        return dispatch_d<E, 4, 6, false, true>(d, a, smem, stream, G_query, err);
     }
-    return dispatch_d<E, 4, 6, false>(d, a, smem, stream, G_query, err);
+    if (vec != 4) return dispatch_d<E, 1, 6, false, false>(d, a, smem, stream, G_query, err);
+    if (v.kres) return dispatch_d<E, 4, 12, true, false>(d, a, smem, stream, G_query, err);
+    switch (v.depth) {
+        case 24: return dispatch_d<E, 4, 24, false, false>(d, a, smem, stream, G_query, err);
+        case 16: return dispatch_d<E, 4, 16, false, false>(d, a, smem, stream, G_query, err);
+        case 12: return dispatch_d<E, 4, 12, false, false>(d, a, smem, stream, G_query, err);
+    }
+    return dispatch_d<E, 4, 6, false, false>(d, a, smem, stream, G_query, err);
 }
 
-int dispatch(const Variant& v, int dtype, int vec, int d, const SelectArgs* a, size_t smem, cudaStream_t stream,
-             int G_query, cudaError_t* err) {
-    return dtype == 1 ? dispatch_e<BF16>(v, vec, d, a, smem, stream, G_query, err)
-                      : dispatch_e<F32>(v, vec, d, a, smem, stream, G_query, err);
+int dispatch(const Variant& v, int dtype, int vec, int d, bool gs, const SelectArgs* a, size_t smem,
+             cudaStream_t stream, int G_query, cudaError_t* err) {
+    return dtype == 1 ? dispatch_e<BF16>(v, vec, d, gs, a, smem, stream, G_query, err)
+                      : dispatch_e<F32>(v, vec, d, gs, a, smem, stream, G_query, err);
 }
 
 int g_cluster_override = 0;
@@ -774,7 +904,7 @@ void cached_cluster_store(const ClusterKey& key, int G) {
 // (0 = not schedulable).  The cost of G is the rows one CTA streams times
 // the waves of clusters, ceil(BH / fit) * ceil(n / G): a 16-CTA cluster must
 // sit inside one GPC, so fewer of them fit than the SM count suggests.
-int choose_cluster_rows(int64_t n, int64_t BH, int (*fit)(int G, void* ctx), void* ctx) {
+int choose_cluster_rows(int64_t n, int64_t BH, int (*fit)(int G, void* ctx), void* ctx, double* cost_out) {
     int best = 0;
     double best_cost = 0.0;
     for (int g = 1; g <= 16; g *= 2) {
@@ -789,7 +919,29 @@ int choose_cluster_rows(int64_t n, int64_t BH, int (*fit)(int G, void* ctx), voi
             best_cost = cost;
         }
     }
+    if (cost_out) *cost_out = best_cost;
     return best;
+}
+
+// Exchange buffers of the global-sync mode (G <= kGsMaxG CTAs per instance).
+constexpr int kGsMaxG = 32;
+size_t select_workspace_bytes(int64_t BH, int64_t n) {
+    Carve cv(nullptr, 0);
+    cv.take(sizeof(double) * BH * 2 * kGsMaxG * 33);
+    cv.take(sizeof(float) * BH * 2 * (n + (int64_t)kGsMaxG * 520));  // G Rpad <= n + G (4 + 511)
+    cv.take(sizeof(unsigned) * BH);
+    cv.take(sizeof(float) * BH * kGsMaxG);
+    return cv.used + 256;
+}
+
+int read_select_gs_status(bool clear) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_select_gs_status, sizeof(int)) != cudaSuccess) return -1;
+    if (clear && v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(g_select_gs_status, &z, sizeof(int));
+    }
+    return v;
 }
 
 int select_cluster_override(int G) {
@@ -805,7 +957,8 @@ int select_kernel_override(int k) {
 }
 int last_select_kernel() { return g_last_kernel; }
 
-static void plan(int64_t n, int r, int d, int dtype, int G, int vec, SelectArgs* a, size_t* smem, Variant* v) {
+static void plan(int64_t n, int r, int d, int dtype, int G, int vec, bool gs, SelectArgs* a, size_t* smem,
+                 Variant* v) {
     const int R = (int)round_up(ceil_div(n, G), 4);
     int JG = 1;
     while (JG * 2 <= 8 && (int64_t)(kSelectThreads / (JG * 2)) * vec >= R) JG *= 2;
@@ -817,9 +970,16 @@ static void plan(int64_t n, int r, int d, int dtype, int G, int vec, SelectArgs*
     a->PL = PL;
     auto bytes = [&](int depth, bool kres) {
         const size_t kb = kres ? (size_t)R * d * (dtype == 1 ? 2 : 4) : 0;
-        return SmemLayout(Rpad, r, d, JG, kSelectThreads, vec, G, depth, kb).total;
+        return SmemLayout(Rpad, r, d, JG, kSelectThreads, vec, G, depth, kb, gs).total;
     };
-    if (vec != 4) {
+    if (gs) {
+        *v = {6, false};  // streamed keys only
+        for (int depth : {24, 16, 12})
+            if (bytes(depth, false) <= kSmemCap) {
+                *v = {depth, false};
+                break;
+            }
+    } else if (vec != 4) {
         *v = {6, false};
     } else if (bytes(12, true) <= kSmemCap) {
         *v = {12, true};  // keys stay in shared memory: the per-step key pass reads no global memory
@@ -832,6 +992,24 @@ static void plan(int64_t n, int r, int d, int dtype, int G, int vec, SelectArgs*
             }
     }
     *smem = bytes(v->depth, v->kres);
+}
+
+struct ClusterCtx {
+    const SelectRequest* q;
+    const SelectArgs* a;
+    int vec;
+    cudaStream_t stream;
+};
+
+// Clusters of g CTAs that fit at once for this request's kernel variant.
+static int cluster_fit(int g, void* p) {
+    const ClusterCtx& c = *static_cast<const ClusterCtx*>(p);
+    SelectArgs t = *c.a;
+    Variant v{};
+    size_t sm = 0;
+    plan(c.q->n, c.q->r, c.q->d, c.q->dtype, g, c.vec, false, &t, &sm, &v);
+    if (sm > kSmemCap) return 0;
+    return dispatch(v, c.q->dtype, c.vec, c.q->d, false, nullptr, sm, c.stream, g, nullptr);
 }
 
 Status launch_select(const SelectRequest& q, cudaStream_t stream) {
@@ -868,39 +1046,75 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     }
     size_t smem = 0;
     Variant var{};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    ClusterCtx ctx{&q, &a, vec, stream};
+
+    // Global-sync mode: given a workspace and few instances, more CTAs per
+    // instance than clusters allow (all co-resident by a cooperative launch).
+    const bool ws_ok = q.ws && q.ws_bytes >= select_workspace_bytes(q.BH, q.n) && vec == 4 &&
+                       (reinterpret_cast<uintptr_t>(q.ws) & 255u) == 0;
+    if (ws_ok && g_kernel_override != 1 && g_cluster_override <= 0) {
+        const ClusterKey gkey{dev, g_kernel_override == 3 ? 4 : 3, q.n, q.BH, q.r, q.d, q.dtype};
+        int Gg = cached_cluster_lookup(gkey);
+        if (Gg == 0) {
+            Gg = -1;
+            int sms = 0;
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            const int cand = (int)std::min<int64_t>(kGsMaxG, sms / std::max<int64_t>(1, q.BH));
+            if (cand >= 2 && q.n / cand >= 512 && ceil_div(q.n, cand) <= kMaxRowsPerCta) {
+                SelectArgs t = a;
+                Variant v{};
+                size_t sm = 0;
+                plan(q.n, q.r, q.d, q.dtype, cand, vec, true, &t, &sm, &v);
+                const int fit = sm <= kSmemCap ? dispatch(v, q.dtype, vec, q.d, true, nullptr, sm, stream, cand, nullptr)
+                                               : 0;
+                if (fit >= q.BH * cand) {
+                    double cc = 0.0;
+                    const int Gc = choose_cluster_rows(q.n, q.BH, cluster_fit, &ctx, &cc);
+                    // the global barrier and L2 round trips cost more per step than a cluster's
+                    const double cg = 1.15 * (double)ceil_div(q.n, cand);
+                    if (g_kernel_override == 3 || Gc <= 0 || cg < cc) Gg = cand;
+                }
+            }
+            cached_cluster_store(gkey, Gg);
+        }
+        if (Gg > 0) {
+            plan(q.n, q.r, q.d, q.dtype, Gg, vec, true, &a, &smem, &var);
+            Carve cv(q.ws, q.ws_bytes);
+            a.gs_inbox = static_cast<double*>(cv.take(sizeof(double) * q.BH * 2 * kGsMaxG * 33));
+            a.gs_resid = static_cast<float*>(cv.take(sizeof(float) * q.BH * 2 * (q.n + (int64_t)kGsMaxG * 520)));
+            a.gs_bar = static_cast<unsigned*>(cv.take(sizeof(unsigned) * q.BH));
+            a.gs_mk = static_cast<float*>(cv.take(sizeof(float) * q.BH * kGsMaxG));
+            if (!cv.fits()) return Status::fail(4, "select: workspace too small");
+            a.gs = 1;
+            cudaError_t err = cudaMemsetAsync(a.gs_bar, 0, sizeof(unsigned) * q.BH, stream);
+            if (err == cudaSuccess) dispatch(var, q.dtype, vec, q.d, true, &a, smem, stream, Gg, &err);
+            if (err == cudaSuccess) err = cudaGetLastError();
+            if (err != cudaSuccess) return Status::cuda(err, "select (global sync) launch");
+            g_last_cluster = Gg;
+            g_last_kernel = 3;
+            return Status::ok();
+        }
+    }
+
     int G = g_cluster_override;
     if (G <= 0) {
         // the cluster size with the least work per CTA times waves of clusters
-        int dev = 0;
-        cudaGetDevice(&dev);
         const ClusterKey key{dev, 1, q.n, q.BH, q.r, q.d, q.dtype};
         G = cached_cluster_lookup(key);
         if (G <= 0) {
-            struct Ctx {
-                const SelectRequest* q;
-                const SelectArgs* a;
-                int vec;
-                cudaStream_t stream;
-            } ctx{&q, &a, vec, stream};
-            G = choose_cluster_rows(q.n, q.BH, [](int g, void* p) -> int {
-                const Ctx& c = *static_cast<const Ctx*>(p);
-                SelectArgs t = *c.a;
-                Variant v{};
-                size_t sm = 0;
-                plan(c.q->n, c.q->r, c.q->d, c.q->dtype, g, c.vec, &t, &sm, &v);
-                if (sm > kSmemCap) return 0;
-                return dispatch(v, c.q->dtype, c.vec, c.q->d, nullptr, sm, c.stream, g, nullptr);
-            }, &ctx);
+            G = choose_cluster_rows(q.n, q.BH, cluster_fit, &ctx, nullptr);
             if (G > 0) cached_cluster_store(key, G);
         }
         if (G <= 0) return Status::fail(2, "select: no schedulable cluster shape (n / 16 above 16384 rows?)");
     } else if (ceil_div(q.n, G) > kMaxRowsPerCta) {
         return Status::fail(2, "select: n / G exceeds the per-CTA row limit (16384)");
     }
-    plan(q.n, q.r, q.d, q.dtype, G, vec, &a, &smem, &var);
+    plan(q.n, q.r, q.d, q.dtype, G, vec, false, &a, &smem, &var);
     if (smem > kSmemCap) return Status::fail(2, "select: shared memory plan exceeds 227 KB");
     cudaError_t err = cudaSuccess;
-    dispatch(var, q.dtype, vec, q.d, &a, smem, stream, G, &err);
+    dispatch(var, q.dtype, vec, q.d, false, &a, smem, stream, G, &err);
     if (err == cudaSuccess) err = cudaGetLastError();
     if (err != cudaSuccess) return Status::cuda(err, "select launch");
     g_last_cluster = G;

@@ -878,7 +878,7 @@ Status launch_select_bulk(const SelectRequest& q, int G_override, cudaStream_t s
                 int mc = 0;
                 if (dispatch(c.q->dtype, c.q->d, kr, c.q->kbar != nullptr, t, sm, c.stream, &mc) != cudaSuccess) return 0;
                 return mc;
-            }, &ctx);
+            }, &ctx, nullptr);
             if (G <= 0) return Status::ok();
             cached_cluster_store(key, G);
         }

@@ -14,8 +14,9 @@
 //                CUDA cores (float32 values, or n % 4 != 0); bf16 values use the
 //                tensor-core kernel of weights_tc.cu
 //   gather_fs    F_S[a, j] = F[j, S_a] for j <= a (pivot rows of the factor)
-//   trsm_kernel  sums the split-K partials and back-substitutes F_S^T X = Y
-//                (blocked by 32 pivots)
+//   trsm_warp_kernel / trsm_kernel  sum the split-K partials and
+//                back-substitute F_S^T X = Y (one warp per column for
+//                r <= 1024, else blocked by 32 pivots)
 #include <algorithm>
 
 #include "common.cuh"
@@ -219,6 +220,49 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* Ypart, 
     }
 }
 
+// Back substitution with one warp per right-hand column (r <= kTrsmWarpMaxR):
+// the column lives in shared memory; pivot a (bottom up) gives
+// x_a = y_a / F_S[a, a], then the lanes subtract F_S[a, j] x_a from every
+// y_j, j < a, reading row a of the pivot block contiguously.  Warps are
+// independent: no block barrier.
+constexpr int kTrsmWarps = 16;
+constexpr int kTrsmWarpMaxR = 1024;
+
+__global__ void __launch_bounds__(kTrsmWarps * 32) trsm_warp_kernel(const float* Ypart, int nsplit, const float* FS,
+                                                                    const int32_t* rank, int64_t BH, int r, int D,
+                                                                    float* V_S, float* w) {
+    extern __shared__ float ysm[];  // [kTrsmWarps][r]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t b = blockIdx.y;
+    const int col = blockIdx.x * kTrsmWarps + warp;
+    const int DP = D + 1;
+    if (col >= DP) return;  // no block-wide synchronisation below
+    const int rr = rank[b];
+    float* y = ysm + (size_t)warp * r;
+    for (int j = lane; j < rr; j += 32) {
+        float s = 0.f;
+        for (int sp = 0; sp < nsplit; ++sp) s += Ypart[(((int64_t)sp * BH + b) * r + j) * DP + col];
+        y[j] = s;
+    }
+    __syncwarp();
+    const float* Lb = FS + b * (int64_t)r * r;  // Lb[a * r + j] = F_S[a, j], j <= a
+    for (int a = rr - 1; a >= 0; --a) {
+        const float* La = Lb + (int64_t)a * r;
+        const float xa = y[a] / La[a];
+        __syncwarp();
+        if (lane == 0) y[a] = xa;
+        for (int j = lane; j < a; j += 32) y[j] = fmaf(-La[j], xa, y[j]);
+        __syncwarp();
+    }
+    for (int j = lane; j < r; j += 32) {
+        const float v = j < rr ? y[j] : 0.f;
+        if (col < D)
+            V_S[(b * r + j) * (int64_t)D + col] = v;
+        else
+            w[b * r + j] = v;
+    }
+}
+
 struct WeightsPlan {
     int nsplit_range;
     int64_t rows_per_range;
@@ -276,11 +320,20 @@ Status run_weights(const WeightsRequest& q, cudaStream_t st) {
             q.F, V, q.n, q.r, p.keys_per_split, Ypart, q.BH, q.rank);
     }
     gather_fs<<<dim3(q.r, (unsigned)q.BH), 128, 0, st>>>(q.F, q.S, q.rank, q.n, q.r, FS);
-    const size_t smem = sizeof(float) * ((size_t)q.r * kTrsmCB + kTrsmBlk * (kTrsmBlk + 1));
-    cudaError_t e = cudaFuncSetAttribute(trsm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return Status::cuda(e, "weights: trsm smem attribute");
-    trsm_kernel<<<dim3((unsigned)ceil_div(D + 1, kTrsmCB), (unsigned)q.BH), kTrsmThreads, smem, st>>>(
-        Ypart, nsplit, FS, q.rank, q.BH, q.r, D, q.V_S, q.w);
+    cudaError_t e;
+    if (q.r <= kTrsmWarpMaxR) {
+        const size_t smem = sizeof(float) * (size_t)kTrsmWarps * q.r;
+        e = cudaFuncSetAttribute(trsm_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return Status::cuda(e, "weights: trsm smem attribute");
+        trsm_warp_kernel<<<dim3((unsigned)ceil_div(D + 1, kTrsmWarps), (unsigned)q.BH), kTrsmWarps * 32, smem, st>>>(
+            Ypart, nsplit, FS, q.rank, q.BH, q.r, D, q.V_S, q.w);
+    } else {
+        const size_t smem = sizeof(float) * ((size_t)q.r * kTrsmCB + kTrsmBlk * (kTrsmBlk + 1));
+        e = cudaFuncSetAttribute(trsm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return Status::cuda(e, "weights: trsm smem attribute");
+        trsm_kernel<<<dim3((unsigned)ceil_div(D + 1, kTrsmCB), (unsigned)q.BH), kTrsmThreads, smem, st>>>(
+            Ypart, nsplit, FS, q.rank, q.BH, q.r, D, q.V_S, q.w);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return Status::cuda(e, "weights launch");
     return Status::ok();
