@@ -118,6 +118,53 @@ __device__ __forceinline__ unsigned long long gs_clock() {
     return t;
 }
 
+// One lane's share of a key-row dot product: 16 bytes of the row (EPL
+// elements) against x.  Without recentring the pairs go through the packed
+// fp32x2 FMA (two partial sums); with it every element is shifted first.
+__device__ __forceinline__ void ffma2(float2& acc, float2 a, float2 b) {
+    unsigned long long A = *reinterpret_cast<unsigned long long*>(&a);
+    unsigned long long B = *reinterpret_cast<unsigned long long*>(&b);
+    unsigned long long C = *reinterpret_cast<unsigned long long*>(&acc);
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(C) : "l"(A), "l"(B));
+    acc = *reinterpret_cast<float2*>(&C);
+}
+
+template <typename T, int EPL, bool KB>
+__device__ __forceinline__ float lane_dot(const float4& raw, const float (&x)[EPL], const float (&kbr)[EPL]) {
+    if constexpr (!KB) {
+        float2 acc = make_float2(0.f, 0.f);
+        if constexpr (sizeof(T) == 2) {
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(&raw);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 v = make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u));
+                ffma2(acc, v, make_float2(x[2 * k], x[2 * k + 1]));
+            }
+        } else {
+            ffma2(acc, make_float2(raw.x, raw.y), make_float2(x[0], x[1]));
+            ffma2(acc, make_float2(raw.z, raw.w), make_float2(x[2], x[3]));
+        }
+        return acc.x + acc.y;
+    } else {
+        float v[EPL];
+        if constexpr (sizeof(T) == 2) {
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 f = __bfloat1622float2(h[k]);
+                v[2 * k] = f.x;
+                v[2 * k + 1] = f.y;
+            }
+        } else {
+            v[0] = raw.x; v[1] = raw.y; v[2] = raw.z; v[3] = raw.w;
+        }
+        float part = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) part = fmaf(v[e] - kbr[e], x[e], part);
+        return part;
+    }
+}
+
 // cp.async helpers (16-byte copies global -> shared, L2 only)
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
     const unsigned d = (unsigned)__cvta_generic_to_shared(smem_dst);
@@ -223,6 +270,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
 #pragma unroll
     for (int e = 0; e < EPL; ++e)
         kbr[e] = a.kbar ? a.kbar[(b / a.kbar_div) * D + kl_part * EPL + e] : 0.f;
+    const bool has_kbar = a.kbar != nullptr;
     // The first INFL items of the streamed key pass; they do not depend on
     // the pivot, so a step can issue them before the previous one ends.
     const int kfirst = warp * RPW + kl_row;  // row of item 0 for this lane
@@ -248,22 +296,26 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                     part[u] = 0.f;
                     if (row < nrows) {
                         const float4 raw = *reinterpret_cast<const float4*>(kres + (size_t)row * D + kl_part * EPL);
-                        float v[EPL];
-                        if constexpr (sizeof(T) == 2) {
-                            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+                        if (self) {
+                            float v[EPL];
+                            if constexpr (sizeof(T) == 2) {
+                                const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const float2 f = __bfloat1622float2(h[k]);
-                                v[2 * k] = f.x;
-                                v[2 * k + 1] = f.y;
+                                for (int k = 0; k < 4; ++k) {
+                                    const float2 f = __bfloat1622float2(h[k]);
+                                    v[2 * k] = f.x;
+                                    v[2 * k + 1] = f.y;
+                                }
+                            } else {
+                                v[0] = raw.x; v[1] = raw.y; v[2] = raw.z; v[3] = raw.w;
                             }
+#pragma unroll
+                            for (int e = 0; e < EPL; ++e) v[e] -= kbr[e];
+#pragma unroll
+                            for (int e = 0; e < EPL; ++e) part[u] = fmaf(v[e], v[e], part[u]);
                         } else {
-                            v[0] = raw.x; v[1] = raw.y; v[2] = raw.z; v[3] = raw.w;
+                            part[u] = has_kbar ? lane_dot<T, EPL, true>(raw, x, kbr) : lane_dot<T, EPL, false>(raw, x, kbr);
                         }
-#pragma unroll
-                        for (int e = 0; e < EPL; ++e) v[e] -= kbr[e];
-#pragma unroll
-                        for (int e = 0; e < EPL; ++e) part[u] = fmaf(v[e], self ? v[e] : x[e], part[u]);
                     }
                 }
 #pragma unroll
@@ -297,22 +349,26 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
             const float4 raw = ring4[slot_rd * NT];
             slot_rd = slot_rd + 1 == DEPTH ? 0 : slot_rd + 1;
             if (row < nrows) {
-                float v[EPL];
-                if constexpr (sizeof(T) == 2) {
-                    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+                if (self) {
+                    float v[EPL];
+                    if constexpr (sizeof(T) == 2) {
+                        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float2 f = __bfloat1622float2(h[k]);
-                        v[2 * k] = f.x;
-                        v[2 * k + 1] = f.y;
+                        for (int k = 0; k < 4; ++k) {
+                            const float2 f = __bfloat1622float2(h[k]);
+                            v[2 * k] = f.x;
+                            v[2 * k + 1] = f.y;
+                        }
+                    } else {
+                        v[0] = raw.x; v[1] = raw.y; v[2] = raw.z; v[3] = raw.w;
                     }
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) v[e] -= kbr[e];
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) part = fmaf(v[e], v[e], part);
                 } else {
-                    v[0] = raw.x; v[1] = raw.y; v[2] = raw.z; v[3] = raw.w;
+                    part = has_kbar ? lane_dot<T, EPL, true>(raw, x, kbr) : lane_dot<T, EPL, false>(raw, x, kbr);
                 }
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) v[e] -= kbr[e];
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) part = fmaf(v[e], self ? v[e] : x[e], part);
             }
 #pragma unroll
             for (int o = LPR / 2; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
@@ -480,8 +536,15 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                         } else {
                             const float* rd =
                                 cluster.map_shared_rank(dbuf + (size_t)cur * Rpad, owner) + (size_t)chunk * CH;
+                            if (PL == 4) {  // one 16-byte read per lane
+                                const float4 q4 = *reinterpret_cast<const float4*>(rd + lane * 4);
 #pragma unroll
-                            for (int k = 0; k < kMaxPL; ++k) vals[k] = k < PL ? rd[lane * PL + k] : 0.f;
+                                for (int k = 0; k < kMaxPL; ++k) vals[k] = 0.f;
+                                vals[0] = q4.x; vals[1] = q4.y; vals[2] = q4.z; vals[3] = q4.w;
+                            } else {
+#pragma unroll
+                                for (int k = 0; k < kMaxPL; ++k) vals[k] = k < PL ? rd[lane * PL + k] : 0.f;
+                            }
                         }
                         double part = 0.0;
 #pragma unroll
