@@ -63,7 +63,7 @@ def parse():
                    help="divide-and-conquer bins (1 = the unbinned method)")
     p.add_argument("--weights-inverse", action="store_true",
                    help="also time the inverse-maintenance weights route on the selected pivots")
-    p.add_argument("--select-kernel", type=int, choices=[0, 1, 2], default=0,
+    p.add_argument("--select-kernel", type=int, choices=[0, 1, 2, 3, 4], default=0,
                    help="0 = automatic (the cp.async kernel), 1 = cp.async, 2 = bulk-copy where it applies")
     return p.parse_args()
 
@@ -106,6 +106,8 @@ SELECT_KERNELS = {
     2: ("rpc_select_bulk_kernel", "rpc_select_bulk",
         ("select_bulk.cu", "common.cuh", "philox.cuh", "tc_common.cuh")),
     3: ("rpc_select_kernel (global sync)", "rpc_select_gs", ("select.cu", "common.cuh", "philox.cuh")),
+    4: ("rpc_select_kernel (tensor-core key pass)", "rpc_select",
+        ("select.cu", "common.cuh", "philox.cuh", "tc_common.cuh")),
 }
 
 

@@ -403,13 +403,16 @@ wildcat_status wildcat_test_force_select_timeout(int64_t nanoseconds);
 
 /*
  * wildcat_set_select_kernel -- which select kernel wildcat_select* launch:
- * 0 (default) the cp.async kernel (per-thread asynchronous copies), in its
+ * 0 (default) the cp.async kernel (per-thread asynchronous copies): in its
  * global-sync form when a workspace is given and that form has less work per
- * CTA; 1 the cp.async kernel on clusters only; 2 the bulk-copy kernel
- * (copy-engine stages on mbarriers) wherever it applies (n % 4 == 0,
- * n / cluster size <= 8192, 16-byte aligned K and F, d in {32, 64, 128}),
- * else the cp.async kernel; 3 the global-sync form wherever a workspace is
- * given and all CTAs fit at once.  Both compute the same
+ * CTA, else on clusters; 1 the cp.async kernel on clusters only;
+ * 2 the bulk-copy kernel (copy-engine stages on mbarriers) wherever it
+ * applies (n % 4 == 0, n / cluster size <= 8192, 16-byte aligned K and F,
+ * d in {32, 64, 128}), else the cp.async kernel; 3 the global-sync form
+ * wherever a workspace is given and all CTAs fit at once; 4 the cp.async
+ * kernel on clusters with the key pass on the tensor cores where the keys
+ * stay resident in shared memory and are bfloat16 with d in {64, 128}
+ * (measured slower than the CUDA-core key pass; kept for comparison).  Both compute the same
  * factorisation (results agree to float32 rounding).  Process-wide; not
  * thread-safe against concurrent select calls.  Returns
  * WILDCAT_ERR_INVALID_ARG for other values.
@@ -417,8 +420,9 @@ wildcat_status wildcat_test_force_select_timeout(int64_t nanoseconds);
 wildcat_status wildcat_set_select_kernel(int kernel);
 
 /* The select kernel the last select launch on this thread used: 1 the
- * cp.async kernel on clusters, 2 the bulk-copy kernel, 3 the cp.async
- * kernel in global-sync form, 0 if none. */
+ * cp.async kernel on clusters (CUDA-core key pass), 2 the bulk-copy kernel,
+ * 3 the cp.async kernel in global-sync form, 4 the cp.async kernel on
+ * clusters with the tensor-core key pass, 0 if none. */
 int wildcat_last_select_kernel(void);
 
 /*

@@ -494,9 +494,10 @@ def last_select_cluster() -> int:
 
 
 def set_select_kernel(kernel: int):
-    """0 = automatic, 1 = the cp.async kernel on clusters, 2 = the bulk-copy
-    kernel where it applies, 3 = the cp.async kernel in global-sync form where
-    it applies."""
+    """0 = automatic, 1 = the cp.async kernel on clusters (CUDA-core key pass),
+    2 = the bulk-copy kernel where it applies, 3 = the cp.async kernel in
+    global-sync form where it applies, 4 = the cp.async kernel on clusters with
+    the tensor-core key pass where it applies."""
     _check(lib().wildcat_set_select_kernel(int(kernel)))
 
 

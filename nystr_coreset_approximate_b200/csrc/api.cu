@@ -601,9 +601,9 @@ wildcat_status wildcat_test_force_select_timeout(int64_t nanoseconds) {
 }
 
 wildcat_status wildcat_set_select_kernel(int kernel) {
-    if (kernel < 0 || kernel > 3)
-        return bad(1, "%s: kernel must be 0 (automatic), 1 (cp.async), 2 (bulk-copy) or 3 (global sync)",
-                   "wildcat_set_select_kernel");
+    if (kernel < 0 || kernel > 4)
+        return bad(1, "%s: kernel must be 0 (automatic), 1 (cp.async), 2 (bulk-copy), 3 (global sync) or 4 "
+                   "(cp.async with the tensor-core key pass)", "wildcat_set_select_kernel");
     wildcat::select_kernel_override(kernel);
     return record(Status::ok());
 }

@@ -42,9 +42,10 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream);
 Status launch_pivot_uniforms(uint64_t seed, int64_t BH, int steps, double* u, cudaStream_t stream);
 int select_cluster_override(int G);  // G < 0: query only
 int last_select_cluster();
-int select_kernel_override(int k);  // k < 0: query only; 0 automatic, 1 cp.async (clusters), 2 bulk-copy,
-                                    // 3 cp.async with global sync where a workspace allows
-int last_select_kernel();           // 1 cp.async (clusters), 2 bulk-copy, 3 cp.async (global sync)
+int select_kernel_override(int k);  // k < 0: query only; 0 automatic, 1 cp.async (clusters, CUDA-core key
+                                    // pass), 2 bulk-copy, 3 cp.async with global sync where a workspace
+                                    // allows, 4 cp.async (clusters) with the tensor-core key pass where it applies
+int last_select_kernel();           // 1, 2, 3 as above; 4 clusters with the tensor-core key pass
 // cluster-size choice shared by both select kernels (select.cu)
 struct ClusterKey {
     int dev, kernel;

@@ -28,6 +28,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "philox.cuh"
+#include "tc_common.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -36,6 +37,8 @@ namespace wildcat {
 namespace {
 
 constexpr int kSelectThreads = 512;
+constexpr int kFsByWarp0 = 512;  // factor rows up to this length are gathered by warp 0 alone
+constexpr unsigned kTckCols = 128;  // tensor memory columns of the key pass: 8 tiles x 16
 constexpr int kMaxPL = 16;  // R <= 16384 rows per CTA -> at most 16 values per lane
 constexpr size_t kSmemCap = 227 * 1024;
 
@@ -67,12 +70,19 @@ struct SelectArgs {
 };
 
 struct SmemLayout {
-    size_t ring, kres, inbox, csl, dbuf, dotb, ks, fs, red, misc, total;
+    size_t ring, kres, inbox, csl, dbuf, dotb, ks, fs, red, misc, btile, mbar, total;
     __host__ __device__ SmemLayout(int Rpad, int r, int D, int JG, int NT, int VEC, int G, int depth,
-                                   size_t kres_bytes, bool gs = false) {
+                                   size_t kres_bytes, bool gs = false, bool tck = false) {
         size_t o = 0;
-        ring = o;  o += (size_t)depth * NT * 16;               // per-thread cp.async ring, [slot][thread] x 16 B
-        kres = o;  o += round_up(kres_bytes, 16);              // the CTA's key rows, when resident
+        if (tck) {
+            // key rows first, 1024-byte aligned tiles for the tensor cores; the
+            // last 128-row tile may read past them into the ring (rows ignored)
+            kres = o;  o += round_up(kres_bytes, 1024);
+            ring = o;  o += (size_t)depth * NT * 16;
+        } else {
+            ring = o;  o += (size_t)depth * NT * 16;               // per-thread cp.async ring, [slot][thread] x 16 B
+            kres = o;  o += round_up(kres_bytes, 16);              // the CTA's key rows, when resident
+        }
         inbox = o; o += gs ? 0 : 2 * (size_t)G * 33 * sizeof(double);  // [parity][source CTA][32 chunk sums + total]
         csl = o;   o += 32 * sizeof(double);                   // own chunk sums
         dbuf = o;  o += 2 * (size_t)Rpad * sizeof(float);      // residual diagonal, double-buffered
@@ -82,6 +92,14 @@ struct SmemLayout {
         o = round_up(o, 16);
         red = o;   o += (size_t)(JG > 1 ? JG - 1 : 0) * (NT / JG) * VEC * sizeof(float);
         misc = o;  o += 16 * sizeof(float);
+        if (tck) {
+            o = round_up(o, 1024);
+            btile = o; o += (size_t)(D / 64) * 16 * 128;  // B: 16 columns x d, K-major, 128-byte swizzle
+            mbar = o;  o += 16;                           // MMA completion barrier, TMEM base address
+            o += 1024;                                    // slack: the base is rounded up to 1024 bytes
+        } else {
+            btile = mbar = 0;
+        }
         total = round_up(o, 16);
     }
 };
@@ -180,8 +198,12 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-template <typename E, int D, int VEC, int DEPTH, bool KRES, bool GS>
+template <typename E, int D, int VEC, int DEPTH, int KM, bool GS>
 __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const SelectArgs a) {
+    // KM: 0 keys streamed each step, 1 keys resident in shared memory,
+    // 2 resident and multiplied by the tensor cores (bf16, d in {64, 128}).
+    constexpr bool KRES = KM >= 1;
+    constexpr bool TCK = KM == 2;
     // Launched with a cluster dimension of a.G (one cluster per instance), or,
     // with GS, as one cooperative grid whose a.G CTAs per instance exchange
     // chunk sums and residuals through global memory and meet at a counter
@@ -207,8 +229,13 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     const int nch = (int)ceil_div(R, CH);
     const int Rpad = nch * CH;  // residual buffers cover whole search chunks
 
-    extern __shared__ __align__(16) unsigned char smem[];
-    const SmemLayout L(Rpad, r, D, JG, NT, VEC, G, DEPTH, KRES ? (size_t)R * D * sizeof(T) : 0, GS);
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    // the tensor-core key pass needs 1024-byte aligned tiles (the same offset in every CTA)
+    unsigned char* smem = TCK ? reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                                  ~uintptr_t(1023))
+                              : smem_raw;
+    const int Rk = (int)round_up(R, 8);  // resident key rows (whole 8-row swizzle atoms)
+    const SmemLayout L(Rpad, r, D, JG, NT, VEC, G, DEPTH, KRES ? (size_t)Rk * D * sizeof(T) : 0, GS, TCK);
     // Each thread streams through its own DEPTH slots of 16 bytes
     // (slot q of thread t at ring4[q * NT + t]); it only ever reads slots it
     // filled itself, so the pipeline needs no barrier.  A slot is refilled
@@ -220,6 +247,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     float* dbuf = reinterpret_cast<float*>(smem + L.dbuf);
     float* dotb = reinterpret_cast<float*>(smem + L.dotb);
     float* fs = reinterpret_cast<float*>(smem + L.fs);
+    T* ksm = reinterpret_cast<T*>(smem + L.ks);  // the pivot's key row (D elements)
     float* red = reinterpret_cast<float*>(smem + L.red);
     float* misc = reinterpret_cast<float*>(smem + L.misc);
     int* imisc = reinterpret_cast<int*>(misc);
@@ -263,7 +291,16 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     // (x = ks) or |k_row|^2 (x = nullptr).  LPR lanes share one row, each
     // copying 16 contiguous bytes, so a warp reads RPW whole rows per item;
     // items stream through the thread's cp.async ring.
-    const T* kres = reinterpret_cast<const T*>(smem + L.kres);
+    // 16-byte piece pc of resident key row `row`: row-major, or (tensor-core
+    // key pass) 64-element K blocks of 128-byte rows in 8-row atoms with the
+    // 128-byte swizzle (piece c of row r at c ^ (r % 8)), the UMMA K-major layout
+    auto kres_off = [&](int row, int pc) -> size_t {
+        if constexpr (TCK)
+            return (size_t)(pc >> 3) * Rk * 128 + (size_t)(row >> 3) * 1024 + (row & 7) * 128 +
+                   (((pc & 7) ^ (row & 7)) << 4);
+        else
+            return ((size_t)row * D + pc * EPL) * sizeof(T);
+    };
     // Recentring: every key enters as k - kbar (kbar = 0 without recentring,
     // which leaves the arithmetic bit-identical).
     float kbr[EPL];
@@ -295,7 +332,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                     const int row = base + u * NW * RPW + kl_row;
                     part[u] = 0.f;
                     if (row < nrows) {
-                        const float4 raw = *reinterpret_cast<const float4*>(kres + (size_t)row * D + kl_part * EPL);
+                        const float4 raw = *reinterpret_cast<const float4*>(smem + L.kres + kres_off(row, kl_part));
                         if (self) {
                             float v[EPL];
                             if constexpr (sizeof(T) == 2) {
@@ -418,13 +455,38 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
 
     // ---------------- prologue: M_K and the initial residual diagonal ----------------
     if constexpr (KRES) {
-        const char* src = reinterpret_cast<const char*>(Kb + row0 * D);
-        char* dst = reinterpret_cast<char*>(smem + L.kres);
-        const int chunks = nrows * D * (int)sizeof(T) / 16;
-        for (int c = tid; c < chunks; c += NT) cp_async16(dst + (size_t)c * 16, src + (size_t)c * 16);
+        const int pieces = nrows * LPR;
+        for (int c = tid; c < pieces; c += NT) {
+            const int row = c / LPR, pc = c % LPR;
+            cp_async16(smem + L.kres + kres_off(row, pc), Kb + (row0 + row) * D + pc * EPL);
+        }
         cp_async_commit();
         cp_async_wait<0>();
         __syncthreads();
+    }
+    // tensor-core key pass: B operand (zero outside its first three columns),
+    // the MMA completion barrier and the accumulator columns in tensor memory
+    unsigned tmem = 0;
+    uint64_t* tc_bar = reinterpret_cast<uint64_t*>(smem + L.mbar);
+    unsigned tc_phase = 0;
+    if constexpr (TCK) {
+        for (int e = tid; e < (D / 64) * 16 * 128 / 16; e += NT)
+            reinterpret_cast<float4*>(smem + L.btile)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (tid == 0) {
+            tc::mbar_init(tc_bar, 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+        if (warp == 0) {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             tc::smem_u32(smem + L.mbar + 8)),
+                         "r"(kTckCols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+        tmem = *reinterpret_cast<volatile unsigned*>(smem + L.mbar + 8);
     }
     {
         const float none[EPL] = {};
@@ -576,6 +638,24 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                     }
                 }
             }
+            if (s >= 0) {
+                // warp 0 fetches the pivot's key into shared memory and starts the
+                // factor row while the other warps wait at the barrier
+                if (lane < LPR) {
+                    float4 piece;
+                    if constexpr (KRES) {
+                        const int owner = (int)(s / R), lrow = (int)(s - (int64_t)owner * R);
+                        piece = *cluster.map_shared_rank(
+                            reinterpret_cast<const float4*>(smem + L.kres + kres_off(lrow, lane)), owner);
+                    } else {
+                        piece = __ldg(reinterpret_cast<const float4*>(Kb + (int64_t)s * D + lane * EPL));
+                    }
+                    reinterpret_cast<float4*>(ksm)[lane] = piece;
+                }
+                if (i <= kFsByWarp0)
+                    for (int j = lane; j < i; j += 32) cp_async4(fs + j, Fb + (int64_t)j * n + s);
+                cp_async_commit();
+            }
             if (lane == 0) {
                 imisc[3] = s;
                 imisc[4] = (s < 0);
@@ -586,19 +666,15 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
         const int s = imisc[3];
 
         // -- the pivot's factor row (asynchronous; first needed by the factor
-        //    pass) and the pivot key (registers of every lane) --
-        for (int j = tid; j < i; j += NT) cp_async4(fs + j, Fb + (int64_t)j * n + s);
-        cp_async_commit();
+        //    pass; warp 0 issued it for short rows) and the pivot key
+        //    (registers of every lane) --
+        if (i > kFsByWarp0) {
+            for (int j = tid; j < i; j += NT) cp_async4(fs + j, Fb + (int64_t)j * n + s);
+            cp_async_commit();
+        }
         float xr[EPL];
         {
-            float4 raw;
-            if constexpr (KRES) {
-                const int owner = (int)(s / R), lrow = (int)(s - (int64_t)owner * R);
-                raw = *cluster.map_shared_rank(
-                    reinterpret_cast<const float4*>(kres + (size_t)lrow * D + kl_part * EPL), owner);
-            } else {
-                raw = __ldg(reinterpret_cast<const float4*>(Kb + (int64_t)s * D + kl_part * EPL));
-            }
+            const float4 raw = reinterpret_cast<const float4*>(ksm)[kl_part];
             if constexpr (sizeof(T) == 2) {
                 const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
@@ -613,16 +689,61 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
 #pragma unroll
             for (int e = 0; e < EPL; ++e) xr[e] -= kbr[e];
         }
-        const T* kp = Kb + (int64_t)s * D;
         if (crank == 0) {
             if (tid == 0 && a.S) a.S[b * r + i] = s;
             if (a.K_S) {
                 T* dst = reinterpret_cast<T*>(a.K_S) + (b * r + i) * D;
-                for (int c = tid; c < D; c += NT) dst[c] = kp[c];
+                for (int c = tid; c < D; c += NT) dst[c] = ksm[c];
             }
         }
         // -- <k_l - kbar, k_s - kbar> for the CTA's rows --
-        key_pass(xr, false, dotb, primed && !KRES);
+        if constexpr (TCK) {
+            // B rows 0..2: x = k_s - kbar split into bf16 hi + mid + lo (x to ~2^-24)
+            for (int e = tid; e < D; e += NT) {
+                const float x = E::to_float(ksm[e]) - (has_kbar ? a.kbar[(b / a.kbar_div) * D + e] : 0.f);
+                const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+                const float r1 = x - __bfloat162float(hi);
+                const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+                const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+                const int kb = e >> 6, c8 = (e & 63) >> 3, w = e & 7;
+                __nv_bfloat16* bt = reinterpret_cast<__nv_bfloat16*>(smem + L.btile + kb * 2048);
+                bt[(0 * 128 + ((c8 ^ 0) << 4)) / 2 + w] = hi;
+                bt[(1 * 128 + ((c8 ^ 1) << 4)) / 2 + w] = mid;
+                bt[(2 * 128 + ((c8 ^ 2) << 4)) / 2 + w] = lo;
+            }
+            tc::fence_async_smem();
+            tc::tc_fence_before();
+            __syncthreads();
+            tc::tc_fence_after();
+            const int ntiles = (nrows + 127) / 128;
+            if (tid == 0 && ntiles > 0) {
+                const unsigned ka = tc::smem_u32(smem + L.kres), kbt = tc::smem_u32(smem + L.btile);
+                constexpr uint32_t idesc = tc::idesc_bf16(128, 16);
+                for (int t = 0; t < ntiles; ++t) {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const unsigned oa = (unsigned)((kk >> 2) * Rk * 128 + t * 16384 + (kk & 3) * 32);
+                        const unsigned ob = (unsigned)((kk >> 2) * 2048 + (kk & 3) * 32);
+                        tc::mma_bf16(tmem + t * 16, tc::umma_desc(ka + oa), tc::umma_desc(kbt + ob), idesc, kk > 0);
+                    }
+                }
+                tc::mma_commit(tc_bar);
+            }
+            if (ntiles > 0) {
+                if (!tc::mbar_wait(tc_bar, tc_phase & 1u)) atomicExch(&g_select_gs_status, 5);
+                ++tc_phase;
+                tc::tc_fence_after();
+                for (int t = warp >> 2; t < ntiles; t += NW / 4) {
+                    float v[16];
+                    tc::tmem_ld16(tmem + ((unsigned)(32 * (warp & 3)) << 16) + t * 16, v);
+                    const int row = t * 128 + 32 * (warp & 3) + lane;
+                    if (row < nrows) dotb[row] = (v[0] + v[1]) + v[2];
+                }
+                tc::tc_fence_before();
+            }
+        } else {
+            key_pass(xr, false, dotb, primed && !KRES);
+        }
         cp_async_wait<0>();
         __syncthreads();
         // -- pivot residual g_s (warp 0, the same on every CTA), read after the next barrier --
@@ -792,6 +913,13 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
             for (int64_t e = (int64_t)rr * D + tid; e < (int64_t)r * D; e += NT) dst[e] = T(0.f);
         }
     }
+    if constexpr (TCK) {
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+        if (warp == 0)
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTckCols) : "memory");
+    }
     // keep this CTA's shared memory alive until every peer is done reading it
     if constexpr (!GS) cluster.sync();
 }
@@ -804,9 +932,9 @@ __global__ void pivot_uniform_kernel(uint64_t seed, int64_t BH, int steps, doubl
     u[t] = pivot_uniform(seed, (uint32_t)i, (uint32_t)b);
 }
 
-template <typename E, int D, int VEC, int DEPTH, bool KRES, bool GS>
+template <typename E, int D, int VEC, int DEPTH, int KM, bool GS>
 cudaError_t launch_select_t(const SelectArgs& a, size_t smem, cudaStream_t stream) {
-    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KRES, GS>;
+    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KM, GS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (!GS && a.G > 8) {
@@ -836,9 +964,9 @@ cudaError_t launch_select_t(const SelectArgs& a, size_t smem, cudaStream_t strea
 
 // Clusters of G CTAs that fit at once (cluster mode) or CTAs that fit at
 // once on the whole GPU (global-sync mode).
-template <typename E, int D, int VEC, int DEPTH, bool KRES, bool GS>
+template <typename E, int D, int VEC, int DEPTH, int KM, bool GS>
 int fit_t(int G, size_t smem) {
-    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KRES, GS>;
+    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KM, GS>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
         cudaGetLastError();
         return 0;
@@ -876,18 +1004,21 @@ int fit_t(int G, size_t smem) {
     return nc;
 }
 
-template <typename E, int VEC, int DEPTH, bool KRES, bool GS>
+template <typename E, int VEC, int DEPTH, int KM, bool GS>
 int dispatch_d(int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int G_query, cudaError_t* err) {
     switch (d) {
         case 32:
-            if (a) { *err = launch_select_t<E, 32, VEC, DEPTH, KRES, GS>(*a, smem, stream); return 0; }
-            return fit_t<E, 32, VEC, DEPTH, KRES, GS>(G_query, smem);
+            if constexpr (KM != 2) {
+                if (a) { *err = launch_select_t<E, 32, VEC, DEPTH, KM, GS>(*a, smem, stream); return 0; }
+                return fit_t<E, 32, VEC, DEPTH, KM, GS>(G_query, smem);
+            }
+            break;
         case 64:
-            if (a) { *err = launch_select_t<E, 64, VEC, DEPTH, KRES, GS>(*a, smem, stream); return 0; }
-            return fit_t<E, 64, VEC, DEPTH, KRES, GS>(G_query, smem);
+            if (a) { *err = launch_select_t<E, 64, VEC, DEPTH, KM, GS>(*a, smem, stream); return 0; }
+            return fit_t<E, 64, VEC, DEPTH, KM, GS>(G_query, smem);
         case 128:
-            if (a) { *err = launch_select_t<E, 128, VEC, DEPTH, KRES, GS>(*a, smem, stream); return 0; }
-            return fit_t<E, 128, VEC, DEPTH, KRES, GS>(G_query, smem);
+            if (a) { *err = launch_select_t<E, 128, VEC, DEPTH, KM, GS>(*a, smem, stream); return 0; }
+            return fit_t<E, 128, VEC, DEPTH, KM, GS>(G_query, smem);
     }
     if (err) *err = cudaErrorInvalidValue;
     return 0;
@@ -898,32 +1029,37 @@ int dispatch_d(int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int
 // The global-sync mode exists for the vectorised streamed-key variants.
 struct Variant {
     int depth;
-    bool kres;
+    int km;  // key mode: 0 streamed, 1 resident, 2 resident with the tensor-core key pass
 };
 
 template <typename E>
 int dispatch_e(const Variant& v, int vec, int d, bool gs, const SelectArgs* a, size_t smem, cudaStream_t stream,
                int G_query, cudaError_t* err) {
     if (gs) {
-        if (vec != 4 || v.kres) {
+        if (vec != 4 || v.km) {
             if (err) *err = cudaErrorInvalidValue;
             return 0;
         }
         switch (v.depth) {
-            case 24: return dispatch_d<E, 4, 24, false, true>(d, a, smem, stream, G_query, err);
-            case 16: return dispatch_d<E, 4, 16, false, true>(d, a, smem, stream, G_query, err);
-            case 12: return dispatch_d<E, 4, 12, false, true>(d, a, smem, stream, G_query, err);
+            case 24: return dispatch_d<E, 4, 24, 0, true>(d, a, smem, stream, G_query, err);
+            case 16: return dispatch_d<E, 4, 16, 0, true>(d, a, smem, stream, G_query, err);
+            case 12: return dispatch_d<E, 4, 12, 0, true>(d, a, smem, stream, G_query, err);
         }
-        return dispatch_d<E, 4, 6, false, true>(d, a, smem, stream, G_query, err);
+        return dispatch_d<E, 4, 6, 0, true>(d, a, smem, stream, G_query, err);
     }
-    if (vec != 4) return dispatch_d<E, 1, 6, false, false>(d, a, smem, stream, G_query, err);
-    if (v.kres) return dispatch_d<E, 4, 12, true, false>(d, a, smem, stream, G_query, err);
+    if (vec != 4) return dispatch_d<E, 1, 6, 0, false>(d, a, smem, stream, G_query, err);
+    if (v.km == 2) {
+        if constexpr (sizeof(typename E::T) == 2) return dispatch_d<E, 4, 12, 2, false>(d, a, smem, stream, G_query, err);
+        if (err) *err = cudaErrorInvalidValue;
+        return 0;
+    }
+    if (v.km == 1) return dispatch_d<E, 4, 12, 1, false>(d, a, smem, stream, G_query, err);
     switch (v.depth) {
-        case 24: return dispatch_d<E, 4, 24, false, false>(d, a, smem, stream, G_query, err);
-        case 16: return dispatch_d<E, 4, 16, false, false>(d, a, smem, stream, G_query, err);
-        case 12: return dispatch_d<E, 4, 12, false, false>(d, a, smem, stream, G_query, err);
+        case 24: return dispatch_d<E, 4, 24, 0, false>(d, a, smem, stream, G_query, err);
+        case 16: return dispatch_d<E, 4, 16, 0, false>(d, a, smem, stream, G_query, err);
+        case 12: return dispatch_d<E, 4, 12, 0, false>(d, a, smem, stream, G_query, err);
     }
-    return dispatch_d<E, 4, 6, false, false>(d, a, smem, stream, G_query, err);
+    return dispatch_d<E, 4, 6, 0, false>(d, a, smem, stream, G_query, err);
 }
 
 int dispatch(const Variant& v, int dtype, int vec, int d, bool gs, const SelectArgs* a, size_t smem,
@@ -1031,30 +1167,35 @@ static void plan(int64_t n, int r, int d, int dtype, int G, int vec, bool gs, Se
     a->R = R;
     a->JG = JG;
     a->PL = PL;
-    auto bytes = [&](int depth, bool kres) {
-        const size_t kb = kres ? (size_t)R * d * (dtype == 1 ? 2 : 4) : 0;
-        return SmemLayout(Rpad, r, d, JG, kSelectThreads, vec, G, depth, kb, gs).total;
+    auto bytes = [&](int depth, int km) {
+        const size_t kb = km ? (size_t)round_up(R, 8) * d * (dtype == 1 ? 2 : 4) : 0;
+        return SmemLayout(Rpad, r, d, JG, kSelectThreads, vec, G, depth, kb, gs, km == 2).total;
     };
+    // tensor-core key pass for resident bf16 keys: on request only (it measured
+    // slower than the CUDA-core pass on 784 resident rows: 1.33 vs 1.26 ms)
+    const bool tc_ok = g_kernel_override == 4 && dtype == 1 && (d == 64 || d == 128) && R <= 1024;
     if (gs) {
-        *v = {6, false};  // streamed keys only
+        *v = {6, 0};  // streamed keys only
         for (int depth : {24, 16, 12})
-            if (bytes(depth, false) <= kSmemCap) {
-                *v = {depth, false};
+            if (bytes(depth, 0) <= kSmemCap) {
+                *v = {depth, 0};
                 break;
             }
     } else if (vec != 4) {
-        *v = {6, false};
-    } else if (bytes(12, true) <= kSmemCap) {
-        *v = {12, true};  // keys stay in shared memory: the per-step key pass reads no global memory
+        *v = {6, 0};
+    } else if (tc_ok && bytes(12, 2) <= kSmemCap) {
+        *v = {12, 2};  // resident keys, key pass on the tensor cores
+    } else if (bytes(12, 1) <= kSmemCap) {
+        *v = {12, 1};  // keys stay in shared memory: the per-step key pass reads no global memory
     } else {
-        *v = {6, false};
+        *v = {6, 0};
         for (int depth : {24, 16, 12})
-            if (bytes(depth, false) <= kSmemCap) {
-                *v = {depth, false};
+            if (bytes(depth, 0) <= kSmemCap) {
+                *v = {depth, 0};
                 break;
             }
     }
-    *smem = bytes(v->depth, v->kres);
+    *smem = bytes(v->depth, v->km);
 }
 
 struct ClusterCtx {
@@ -1117,7 +1258,7 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     // instance than clusters allow (all co-resident by a cooperative launch).
     const bool ws_ok = q.ws && q.ws_bytes >= select_workspace_bytes(q.BH, q.n) && vec == 4 &&
                        (reinterpret_cast<uintptr_t>(q.ws) & 255u) == 0;
-    if (ws_ok && g_kernel_override != 1 && g_cluster_override <= 0) {
+    if (ws_ok && g_kernel_override != 1 && g_kernel_override != 4 && g_cluster_override <= 0) {
         const ClusterKey gkey{dev, g_kernel_override == 3 ? 4 : 3, q.n, q.BH, q.r, q.d, q.dtype};
         int Gg = cached_cluster_lookup(gkey);
         if (Gg == 0) {
@@ -1164,7 +1305,7 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     int G = g_cluster_override;
     if (G <= 0) {
         // the cluster size with the least work per CTA times waves of clusters
-        const ClusterKey key{dev, 1, q.n, q.BH, q.r, q.d, q.dtype};
+        const ClusterKey key{dev, g_kernel_override == 4 ? 5 : 1, q.n, q.BH, q.r, q.d, q.dtype};
         G = cached_cluster_lookup(key);
         if (G <= 0) {
             G = choose_cluster_rows(q.n, q.BH, cluster_fit, &ctx, nullptr);
@@ -1181,7 +1322,7 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     if (err == cudaSuccess) err = cudaGetLastError();
     if (err != cudaSuccess) return Status::cuda(err, "select launch");
     g_last_cluster = G;
-    g_last_kernel = 1;
+    g_last_kernel = var.km == 2 ? 4 : 1;
     return Status::ok();
 }
 

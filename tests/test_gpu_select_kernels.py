@@ -62,9 +62,11 @@ def test_both_kernels_match_the_oracle(orc, w, G):
     K = dev["K"].cuda()
     wc.set_select_cluster(G)
     own = orc.rpcholesky(ex["K"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
-    for kernel, expect in ((2, (2,)), (1, (1,)), (0, (1, 3))):
+    for kernel, expect in ((2, (2,)), (1, (1,)), (0, (1, 3, 4)), (4, (1, 4))):
         S, F, rank, K_S, used = _run(K, w, kernel)
         assert used in expect
+        if w.name == "kres_g4" and kernel == 4:
+            assert used == 4  # resident bf16 keys, d = 64: tensor-core key pass
         gc.pivots_agree_until_tie(S, own["S"], own["margin"], rank, own["rank"], F, own["F"], EPS)
         for b in range(w.BH):
             rr = rank[b]
@@ -78,6 +80,26 @@ def test_both_kernels_match_the_oracle(orc, w, G):
     assert wc.device_status() == 0
 
 
+def test_tensor_core_key_pass_recentred(orc):
+    """Resident bf16 keys with recentring: the tensor-core key pass splits
+    k_s - kbar into three bf16 parts; pivots follow the oracle's draws on
+    K - mean(K) and the factor matches the oracle on the device's pivots."""
+    w = gc.case("tck_recentre", "walk", 4, 3136, 64, 64, 96, "bf16")
+    dev, ex = workloads.make(w)
+    d = gc.cuda_inputs(dev)
+    wc.set_select_kernel(4)
+    O, S, rank = wc.forward_ex(d["Q"], d["K"], d["V"], w.beta, w.r, w.pivot_seed, EPS, recenter=True)
+    assert wc.last_select_kernel() == 4
+    S, rank = S.cpu().numpy(), rank.cpu().numpy().reshape(w.BH)
+    Kc = ex["K"] - ex["K"].mean(axis=1, keepdims=True)
+    res = orc.rpcholesky(Kc, w.beta, w.r, seed=w.pivot_seed, eps=EPS)
+    gc.pivots_agree_until_tie(S, res["S"], res["margin"], rank, res["rank"])
+    fx = orc.wildcat_forward_binned(ex["Q"], ex["K"], ex["V"], w.beta, w.r, 1, eps=0.0, S_fixed=S,
+                                    recenter=True)
+    lo, hi = orc.value_range(ex["V"])
+    assert gc.r12(O.cpu().numpy(), fx[0], lo, hi) <= gc.TOL_R12["bf16"]
+
+
 @pytest.mark.parametrize("w,G", SHAPES[:5], ids=[w.name for w, _ in SHAPES[:5]])
 def test_kernels_agree_on_fixed_pivots(orc, w, G):
     dev, ex = workloads.make(w)
@@ -87,9 +109,11 @@ def test_kernels_agree_on_fixed_pivots(orc, w, G):
     S_fixed = torch.from_numpy(own["S"]).cuda()
     _, F_a, rank_a, _, used_a = _run(K, w, 2, S_fixed)
     _, F_b, rank_b, _, used_b = _run(K, w, 1, S_fixed)
-    assert (used_a, used_b) == (2, 1)
-    assert np.array_equal(rank_a, rank_b)
+    _, F_c, rank_c, _, used_c = _run(K, w, 4, S_fixed)
+    assert (used_a, used_b) == (2, 1) and used_c in (1, 4)
+    assert np.array_equal(rank_a, rank_b) and np.array_equal(rank_c, rank_b)
     assert gc.column_rel_err(F_a, F_b.astype(np.float64), rank_a) < 2e-4
+    assert gc.column_rel_err(F_c, F_b.astype(np.float64), rank_c) < 2e-4
 
 
 def test_recentred_keys_bulk_kernel(orc):
