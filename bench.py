@@ -61,6 +61,8 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--nbins", type=int, default=1,
                    help="divide-and-conquer bins (1 = the unbinned method)")
+    p.add_argument("--select-cluster", type=int, default=0,
+                   help="CTAs per instance in the select (0 = automatic; a fixed size keeps 512-thread CTAs)")
     p.add_argument("--weights-inverse", action="store_true",
                    help="also time the inverse-maintenance weights route on the selected pivots")
     p.add_argument("--select-kernel", type=int, choices=[0, 1, 2, 3, 4], default=0,
@@ -253,6 +255,7 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     wc.set_select_kernel(args.select_kernel)
+    wc.set_select_cluster(args.select_cluster)
     if world > 1:
         from datetime import timedelta
 
@@ -282,6 +285,7 @@ def main():
     ranks = plan.rank.reshape(-1).cpu().tolist()  # per instance (per bin when binned)
     sel_kind = wc.last_select_kernel()
     sel_cluster = wc.last_select_cluster()
+    sel_threads = wc.last_select_threads()
 
     # ---- timed forward: K steps, own events per step, L2 flushed in between ----
     clocks = ClockSampler(local)
@@ -403,7 +407,8 @@ def main():
                                        "parallelism": f"instances per rank x {world} ranks",
                                        "nbins": nb,
                                        "select_kernel": SELECT_KERNELS[sel_kind][0],
-                                       "select_cluster_ctas": sel_cluster}),
+                                       "select_cluster_ctas": sel_cluster,
+                                       "select_cta_threads": sel_threads}),
         "entries_per_s": value * w.BH * w.m * w.n,
         "stages_ms": {k: statistics.mean(v) for k, v in stage_ms.items()},
         "roofline": {"kernel": SELECT_KERNELS[sel_kind][0], "bound": "hbm", "achieved": achieved,

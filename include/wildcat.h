@@ -392,12 +392,15 @@ wildcat_status wildcat_test_force_wait_timeout(int64_t nanoseconds);
 
 /*
  * wildcat_test_force_select_timeout -- test hook for the bounded waits of
- * the bulk-copy select kernel.  With nanoseconds > 0 every later launch of
- * that kernel waits that long, after step 1, on a barrier phase that nothing
- * completes; the expiry is handled like any other (WILDCAT_ERR_TIMEOUT in
- * the device status word, every instance stops after two steps).  0 turns
- * the hook off.  Process-wide; for tests only.  Returns
- * WILDCAT_ERR_INVALID_ARG outside [0, 1e9].
+ * the select kernels that have them.  With nanoseconds > 0, every later
+ * launch of the bulk-copy kernel waits that long, after step 1, on a barrier
+ * phase that nothing completes (every instance then stops after two steps);
+ * in the global-sync form, CTA 0 of every instance never arrives at the
+ * third counter barrier and every wait there ends after `nanoseconds`
+ * (every instance stops after one step).  Either expiry is handled like any
+ * other: WILDCAT_ERR_TIMEOUT in the device status word.  0 turns the hook
+ * off.  Process-wide; for tests only.  Returns WILDCAT_ERR_INVALID_ARG
+ * outside [0, 1e9].
  */
 wildcat_status wildcat_test_force_select_timeout(int64_t nanoseconds);
 
@@ -424,6 +427,11 @@ wildcat_status wildcat_set_select_kernel(int kernel);
  * 3 the cp.async kernel in global-sync form, 4 the cp.async kernel on
  * clusters with the tensor-core key pass, 0 if none. */
 int wildcat_last_select_kernel(void);
+
+/* Threads per CTA of the last select launch on this thread: 512, or 256 when
+ * the automatic choice put two CTAs on each SM (twice the cluster size, half
+ * the rows per CTA; resident keys only).  0 if none. */
+int wildcat_last_select_threads(void);
 
 /*
  * wildcat_set_select_cluster -- tuning knob for wildcat_select*: number of

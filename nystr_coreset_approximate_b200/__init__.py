@@ -26,7 +26,7 @@ __all__ = [
     "WildcatError", "library_path", "lib", "declared_symbols", "select", "select_fixed",
     "weights", "weights_inverse", "attend", "attend_noalloc", "decode_attend", "forward", "forward_ex", "Options", "forward_binned", "BinnedForwardPlan", "forward_host", "ForwardPlan", "pivot_uniforms",
     "set_select_cluster", "last_select_cluster", "set_select_kernel", "last_select_kernel",
-    "force_select_timeout", "device_status", "DTYPES",
+    "force_select_timeout", "last_select_threads", "device_status", "DTYPES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +86,7 @@ _SIGS = {
     "wildcat_test_force_select_timeout": ([_i64], _int),
     "wildcat_set_select_kernel": ([_int], _int),
     "wildcat_last_select_kernel": ([], _int),
+    "wildcat_last_select_threads": ([], _int),
 }
 
 
@@ -504,6 +505,11 @@ def set_select_kernel(kernel: int):
 def last_select_kernel() -> int:
     """1 = the cp.async kernel, 2 = the bulk-copy kernel (last select launch)."""
     return int(lib().wildcat_last_select_kernel())
+
+
+def last_select_threads() -> int:
+    """Threads per CTA of the last select launch (256 or 512)."""
+    return int(lib().wildcat_last_select_threads())
 
 
 def force_select_timeout(nanoseconds: int):

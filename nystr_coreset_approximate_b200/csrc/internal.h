@@ -46,6 +46,7 @@ int select_kernel_override(int k);  // k < 0: query only; 0 automatic, 1 cp.asyn
                                     // pass), 2 bulk-copy, 3 cp.async with global sync where a workspace
                                     // allows, 4 cp.async (clusters) with the tensor-core key pass where it applies
 int last_select_kernel();           // 1, 2, 3 as above; 4 clusters with the tensor-core key pass
+int last_select_threads();          // threads per CTA of the last select launch (256 or 512)
 // cluster-size choice shared by both select kernels (select.cu)
 struct ClusterKey {
     int dev, kernel;
@@ -55,13 +56,15 @@ struct ClusterKey {
 };
 int cached_cluster_lookup(const ClusterKey& key);   // 0 if absent
 void cached_cluster_store(const ClusterKey& key, int G);
-int choose_cluster_rows(int64_t n, int64_t BH, int (*fit)(int G, void* ctx), void* ctx, double* cost_out);
+int choose_cluster_rows(int64_t n, int64_t BH, int (*fit)(int G, void* ctx), void* ctx, double* cost_out,
+                        int min_rows = 512);
 size_t select_workspace_bytes(int64_t BH, int64_t n);  // global-sync exchange buffers
 int read_select_gs_status(bool clear);
 // bulk-copy select kernel (select_bulk.cu); *used = false when the shape is not one it handles.
 // G_override > 0 fixes the cluster size.
 Status launch_select_bulk(const SelectRequest& q, int G_override, cudaStream_t stream, bool* used, int* G_used);
 void set_select_force_timeout(unsigned long long ns);
+unsigned long long select_force_timeout_ns();
 
 // ---- weights: Y = F^T (V, 1), then F_S^T X = Y ----
 struct WeightsRequest {

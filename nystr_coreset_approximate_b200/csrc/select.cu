@@ -36,7 +36,6 @@ namespace wildcat {
 
 namespace {
 
-constexpr int kSelectThreads = 512;
 constexpr int kFsByWarp0 = 512;  // factor rows up to this length are gathered by warp 0 alone
 constexpr unsigned kTckCols = 128;  // tensor memory columns of the key pass: 8 tiles x 16
 constexpr int kMaxPL = 16;  // R <= 16384 rows per CTA -> at most 16 values per lane
@@ -67,6 +66,7 @@ struct SelectArgs {
     unsigned* gs_bar;  // [BH] barrier counters, zero at launch
     float* gs_mk;      // [BH][G] per-CTA max |k|^2
     int gs;            // 1: the launch is the global-sync one
+    unsigned long long gs_force_ns;  // test hook: CTA 0 of each instance skips barrier 2; waits end after this
 };
 
 struct SmemLayout {
@@ -198,8 +198,10 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-template <typename E, int D, int VEC, int DEPTH, int KM, bool GS>
-__global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const SelectArgs a) {
+template <typename E, int D, int VEC, int DEPTH, int KM, bool GS, int NTH>
+__global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const SelectArgs a) {
+    // NTH threads per CTA: 512 (one CTA per SM), or 256 with twice the CTAs
+    // per instance and two CTAs per SM, whose barriers and searches overlap.
     // KM: 0 keys streamed each step, 1 keys resident in shared memory,
     // 2 resident and multiplied by the tensor cores (bf16, d in {64, 128}).
     constexpr bool KRES = KM >= 1;
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     // chunk sums and residuals through global memory and meet at a counter
     // barrier (all CTAs are co-resident by the cooperative launch).
     using T = typename E::T;
-    constexpr int NT = kSelectThreads, NW = NT / 32;
+    constexpr int NT = NTH, NW = NT / 32;
     constexpr int EPL = 16 / (int)sizeof(T);  // key elements per 16-byte load
     constexpr int LPR = D / EPL;              // lanes per key row
     constexpr int RPW = 32 / LPR;             // key rows per warp-wide load
@@ -263,11 +265,13 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
         __syncthreads();
         if (tid == 0) {
             __threadfence();
-            atomicAdd(a.gs_bar + b, 1u);
+            const bool skip = a.gs_force_ns && gs_k == 2 && crank == 0;  // test hook: never arrive
+            if (!skip) atomicAdd(a.gs_bar + b, 1u);
             const unsigned target = (unsigned)G * (unsigned)(gs_k + 1);
+            const unsigned long long limit = a.gs_force_ns ? a.gs_force_ns : kGsWaitNs;
             const unsigned long long t0 = gs_clock();
             while (ld_acquire_u32(a.gs_bar + b) < target) {
-                if (gs_clock() - t0 > kGsWaitNs) {
+                if (gs_clock() - t0 > limit) {
                     imisc[5] = 1;
                     atomicExch(&g_select_gs_status, 5);
                     break;
@@ -308,8 +312,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     for (int e = 0; e < EPL; ++e)
         kbr[e] = a.kbar ? a.kbar[(b / a.kbar_div) * D + kl_part * EPL + e] : 0.f;
     const bool has_kbar = a.kbar != nullptr;
-    // The first INFL items of the streamed key pass; they do not depend on
-    // the pivot, so a step can issue them before the previous one ends.
+    // The first INFL items of the streamed key pass.
     const int kfirst = warp * RPW + kl_row;  // row of item 0 for this lane
     const int kitems = nrows > warp * RPW ? (int)ceil_div(nrows - warp * RPW, NW * RPW) : 0;  // warp-uniform
     const T* ksrc0 = Kb + (row0 + kfirst) * D + kl_part * EPL;
@@ -322,7 +325,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
         }
     };
     // out[row] = <k_row - kbar, x> (or |k_row - kbar|^2 when self)
-    auto key_pass = [&](const float (&x)[EPL], bool self, float* out, bool primed) {
+    auto key_pass = [&](const float (&x)[EPL], bool self, float* out) {
         if constexpr (KRES) {
             // key rows resident in shared memory: no global traffic; four rows per lane in flight
             for (int base = warp * RPW; base < nrows; base += 4 * NW * RPW) {
@@ -369,7 +372,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
             }
             return;
         }
-        if (!primed) key_prime();
+        key_prime();
         // slot and source advance incrementally (no division or 64-bit multiply per item)
         int slot_rd = 0, slot_wr = INFL;
         const T* src_wr = ksrc0 + INFL * kstep;
@@ -490,7 +493,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     }
     {
         const float none[EPL] = {};
-        key_pass(none, true, dotb, false);  // |k_l - kbar|^2
+        key_pass(none, true, dotb);  // |k_l - kbar|^2
     }
     __syncthreads();
     float lmax = -INFINITY;
@@ -540,23 +543,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
     // block covers chunk (base + 128 w) / 128 with the search's lane layout.
     const bool fused_csl = (VEC == 4 && PL == 4);
     const int g = tid / TPG, tt = tid % TPG;
-    // The first INFL factor items of row block 0 for step `st` (resident keys
-    // only: the ring is idle during the key pass then); they do not depend on
-    // the pivot either.
-    auto fpass_prime = [&](int st) {
-        const int jl = (st + JG - 1) / JG, j0 = min(st, g * jl), j1 = min(st, j0 + jl);
-        const int row = tt * VEC;
-        const int cnt = row < nrows ? j1 - j0 : 0;
-        const float* fcol = Fb + row0 + row;
-#pragma unroll
-        for (int q = 0; q < INFL; ++q) {
-            if (q < cnt) cp_async16(ring4 + q * NT, fcol + (int64_t)(j0 + q) * n);
-            cp_async_commit();
-        }
-    };
-    bool primed = false;  // the next step's first ring items are in flight
     int i = 0;
     for (; gs_ok && i < r; ++i) {
+        // a barrier ran out: the steps before it are complete (uniform: read after the barrier's block sync)
+        if (GS && imisc[5]) break;
         const int cur = i & 1, nxt = cur ^ 1;
         float* dcur = dbuf + (size_t)cur * Rpad;
         float* dnxt = dbuf + (size_t)nxt * Rpad;
@@ -742,7 +732,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                 tc::tc_fence_before();
             }
         } else {
-            key_pass(xr, false, dotb, primed && !KRES);
+            key_pass(xr, false, dotb);
         }
         cp_async_wait<0>();
         __syncthreads();
@@ -777,12 +767,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                 int j = j0;
                 if constexpr (VEC == 4) {
                     const int cnt = j1 - j0;
-                    if (!(KRES && primed && base == 0)) {
 #pragma unroll
-                        for (int q = 0; q < INFL; ++q) {
-                            if (q < cnt) cp_async16(ring4 + q * NT, fcol + (int64_t)(j0 + q) * n);
-                            cp_async_commit();
-                        }
+                    for (int q = 0; q < INFL; ++q) {
+                        if (q < cnt) cp_async16(ring4 + q * NT, fcol + (int64_t)(j0 + q) * n);
+                        cp_async_commit();
                     }
                     int slot_rd = 0, slot_wr = INFL;
                     const float* src_wr = fcol + (int64_t)(j0 + INFL) * n;
@@ -811,8 +799,6 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
                     }
                     for (; j < j1; ++j) acc[0] = fmaf(ld_cg1(fcol + (int64_t)j * n), fs[j], acc[0]);
                 }
-            } else if (VEC == 4 && KRES && primed && base == 0) {
-                cp_async_wait<0>();  // the primed (empty) groups of a thread without rows
             }
             if (JG > 1) {
                 if (g > 0) {
@@ -884,19 +870,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) rpc_select_kernel(const Sel
             for (int k = covered + tid; k < nch; k += NT) csl[k] = 0.0;
         }
         __syncthreads();
-        // the next step's first ring items, in flight across the cluster barrier and the search
-        primed = i + 1 < r;
-        if (primed) {
-            if constexpr (KRES) {
-                if (VEC == 4) fpass_prime(i + 1);
-            } else {
-                key_prime();
-            }
-        }
         publish(dnxt, nxt, fused_csl, i + 1);
-        if (GS && imisc[5]) break;  // a barrier ran out (uniform: read after the barrier's block sync)
     }
-    cp_async_wait<0>();  // a primed step that never ran
 
     // ---------------- effective rank, padding past it ----------------
     const int rr = i;
@@ -932,9 +907,9 @@ __global__ void pivot_uniform_kernel(uint64_t seed, int64_t BH, int steps, doubl
     u[t] = pivot_uniform(seed, (uint32_t)i, (uint32_t)b);
 }
 
-template <typename E, int D, int VEC, int DEPTH, int KM, bool GS>
+template <typename E, int D, int VEC, int DEPTH, int KM, bool GS, int NTH>
 cudaError_t launch_select_t(const SelectArgs& a, size_t smem, cudaStream_t stream) {
-    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KM, GS>;
+    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KM, GS, NTH>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (!GS && a.G > 8) {
@@ -943,7 +918,7 @@ cudaError_t launch_select_t(const SelectArgs& a, size_t smem, cudaStream_t strea
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.BH * a.G));
-    cfg.blockDim = dim3(kSelectThreads);
+    cfg.blockDim = dim3(NTH);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -964,16 +939,16 @@ cudaError_t launch_select_t(const SelectArgs& a, size_t smem, cudaStream_t strea
 
 // Clusters of G CTAs that fit at once (cluster mode) or CTAs that fit at
 // once on the whole GPU (global-sync mode).
-template <typename E, int D, int VEC, int DEPTH, int KM, bool GS>
+template <typename E, int D, int VEC, int DEPTH, int KM, bool GS, int NTH>
 int fit_t(int G, size_t smem) {
-    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KM, GS>;
+    auto kern = rpc_select_kernel<E, D, VEC, DEPTH, KM, GS, NTH>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
         cudaGetLastError();
         return 0;
     }
     if (GS) {
         int per_sm = 0, dev = 0, sms = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSelectThreads, smem) != cudaSuccess ||
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NTH, smem) != cudaSuccess ||
             cudaGetDevice(&dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
             cudaGetLastError();
@@ -987,7 +962,7 @@ int fit_t(int G, size_t smem) {
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)G);
-    cfg.blockDim = dim3(kSelectThreads);
+    cfg.blockDim = dim3(NTH);
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1004,21 +979,21 @@ int fit_t(int G, size_t smem) {
     return nc;
 }
 
-template <typename E, int VEC, int DEPTH, int KM, bool GS>
+template <typename E, int VEC, int DEPTH, int KM, bool GS, int NTH = 512>
 int dispatch_d(int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int G_query, cudaError_t* err) {
     switch (d) {
         case 32:
             if constexpr (KM != 2) {
-                if (a) { *err = launch_select_t<E, 32, VEC, DEPTH, KM, GS>(*a, smem, stream); return 0; }
-                return fit_t<E, 32, VEC, DEPTH, KM, GS>(G_query, smem);
+                if (a) { *err = launch_select_t<E, 32, VEC, DEPTH, KM, GS, NTH>(*a, smem, stream); return 0; }
+                return fit_t<E, 32, VEC, DEPTH, KM, GS, NTH>(G_query, smem);
             }
             break;
         case 64:
-            if (a) { *err = launch_select_t<E, 64, VEC, DEPTH, KM, GS>(*a, smem, stream); return 0; }
-            return fit_t<E, 64, VEC, DEPTH, KM, GS>(G_query, smem);
+            if (a) { *err = launch_select_t<E, 64, VEC, DEPTH, KM, GS, NTH>(*a, smem, stream); return 0; }
+            return fit_t<E, 64, VEC, DEPTH, KM, GS, NTH>(G_query, smem);
         case 128:
-            if (a) { *err = launch_select_t<E, 128, VEC, DEPTH, KM, GS>(*a, smem, stream); return 0; }
-            return fit_t<E, 128, VEC, DEPTH, KM, GS>(G_query, smem);
+            if (a) { *err = launch_select_t<E, 128, VEC, DEPTH, KM, GS, NTH>(*a, smem, stream); return 0; }
+            return fit_t<E, 128, VEC, DEPTH, KM, GS, NTH>(G_query, smem);
     }
     if (err) *err = cudaErrorInvalidValue;
     return 0;
@@ -1029,7 +1004,8 @@ int dispatch_d(int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int
 // The global-sync mode exists for the vectorised streamed-key variants.
 struct Variant {
     int depth;
-    int km;  // key mode: 0 streamed, 1 resident, 2 resident with the tensor-core key pass
+    int km;        // key mode: 0 streamed, 1 resident, 2 resident with the tensor-core key pass
+    int nt = 512;  // threads per CTA (256 only for resident keys on CUDA cores)
 };
 
 template <typename E>
@@ -1053,7 +1029,10 @@ int dispatch_e(const Variant& v, int vec, int d, bool gs, const SelectArgs* a, s
         if (err) *err = cudaErrorInvalidValue;
         return 0;
     }
-    if (v.km == 1) return dispatch_d<E, 4, 12, 1, false>(d, a, smem, stream, G_query, err);
+    if (v.km == 1) {
+        if (v.nt == 256) return dispatch_d<E, 4, 12, 1, false, 256>(d, a, smem, stream, G_query, err);
+        return dispatch_d<E, 4, 12, 1, false>(d, a, smem, stream, G_query, err);
+    }
     switch (v.depth) {
         case 24: return dispatch_d<E, 4, 24, 0, false>(d, a, smem, stream, G_query, err);
         case 16: return dispatch_d<E, 4, 16, 0, false>(d, a, smem, stream, G_query, err);
@@ -1072,6 +1051,7 @@ int g_cluster_override = 0;
 int g_kernel_override = 0;
 thread_local int g_last_cluster = 0;
 thread_local int g_last_kernel = 0;
+thread_local int g_last_threads = 0;
 
 }  // namespace
 
@@ -1098,18 +1078,19 @@ void cached_cluster_store(const ClusterKey& key, int G) {
 }
 
 // Cluster size for one select launch.  Candidates are G in {1, 2, 4, 8, 16}
-// with at most kMaxRowsPerCta rows per CTA and at least 512 (unless G = 1);
+// with at most kMaxRowsPerCta rows per CTA and at least min_rows (unless G = 1);
 // fit(G) is the number of clusters of G CTAs that fit on the GPU at once
 // (0 = not schedulable).  The cost of G is the rows one CTA streams times
 // the waves of clusters, ceil(BH / fit) * ceil(n / G): a 16-CTA cluster must
 // sit inside one GPC, so fewer of them fit than the SM count suggests.
-int choose_cluster_rows(int64_t n, int64_t BH, int (*fit)(int G, void* ctx), void* ctx, double* cost_out) {
+int choose_cluster_rows(int64_t n, int64_t BH, int (*fit)(int G, void* ctx), void* ctx, double* cost_out,
+                        int min_rows) {
     int best = 0;
     double best_cost = 0.0;
     for (int g = 1; g <= 16; g *= 2) {
         const int64_t rows = ceil_div(n, g);
         if (rows > kMaxRowsPerCta) continue;
-        if (g > 1 && n / g < 512) break;
+        if (g > 1 && n / g < min_rows) break;
         const int f = fit(g, ctx);
         if (f <= 0) continue;
         const double cost = (double)ceil_div(BH, f) * (double)rows;
@@ -1155,12 +1136,13 @@ int select_kernel_override(int k) {
     return k;
 }
 int last_select_kernel() { return g_last_kernel; }
+int last_select_threads() { return g_last_threads; }
 
 static void plan(int64_t n, int r, int d, int dtype, int G, int vec, bool gs, SelectArgs* a, size_t* smem,
-                 Variant* v) {
+                 Variant* v, int nt = 512) {
     const int R = (int)round_up(ceil_div(n, G), 4);
     int JG = 1;
-    while (JG * 2 <= 8 && (int64_t)(kSelectThreads / (JG * 2)) * vec >= R) JG *= 2;
+    while (JG * 2 <= 8 && (int64_t)(nt / (JG * 2)) * vec >= R) JG *= 2;
     const int PL = (int)std::max<int64_t>(4, round_up(ceil_div(ceil_div(R, 32), 32), 4));
     const int Rpad = (int)round_up(R, 32 * PL);
     a->G = G;
@@ -1169,7 +1151,7 @@ static void plan(int64_t n, int r, int d, int dtype, int G, int vec, bool gs, Se
     a->PL = PL;
     auto bytes = [&](int depth, int km) {
         const size_t kb = km ? (size_t)round_up(R, 8) * d * (dtype == 1 ? 2 : 4) : 0;
-        return SmemLayout(Rpad, r, d, JG, kSelectThreads, vec, G, depth, kb, gs, km == 2).total;
+        return SmemLayout(Rpad, r, d, JG, nt, vec, G, depth, kb, gs, km == 2).total;
     };
     // tensor-core key pass for resident bf16 keys: on request only (it measured
     // slower than the CUDA-core pass on 784 resident rows: 1.33 vs 1.26 ms)
@@ -1195,6 +1177,12 @@ static void plan(int64_t n, int r, int d, int dtype, int G, int vec, bool gs, Se
                 break;
             }
     }
+    if (nt != 512) {
+        // the 256-thread form exists for resident keys on CUDA cores only
+        *v = (!gs && vec == 4 && bytes(12, 1) <= kSmemCap) ? Variant{12, 1, nt} : Variant{0, -1, nt};
+        *smem = v->km < 0 ? kSmemCap + 1 : bytes(12, 1);
+        return;
+    }
     *smem = bytes(v->depth, v->km);
 }
 
@@ -1203,6 +1191,7 @@ struct ClusterCtx {
     const SelectArgs* a;
     int vec;
     cudaStream_t stream;
+    int nt = 512;
 };
 
 // Clusters of g CTAs that fit at once for this request's kernel variant.
@@ -1211,10 +1200,14 @@ static int cluster_fit(int g, void* p) {
     SelectArgs t = *c.a;
     Variant v{};
     size_t sm = 0;
-    plan(c.q->n, c.q->r, c.q->d, c.q->dtype, g, c.vec, false, &t, &sm, &v);
+    plan(c.q->n, c.q->r, c.q->d, c.q->dtype, g, c.vec, false, &t, &sm, &v, c.nt);
     if (sm > kSmemCap) return 0;
     return dispatch(v, c.q->dtype, c.vec, c.q->d, false, nullptr, sm, c.stream, g, nullptr);
 }
+
+// Two 256-thread CTAs per SM overlap each other's barriers and searches but
+// share the SM's issue slots and bandwidth: their rows per CTA count 1.3x.
+constexpr double kHalfCtaCost = 1.3;
 
 Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     const int vec = (q.n % 4 == 0) ? 4 : 1;
@@ -1244,6 +1237,7 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
             if (st.code == 0) {
                 g_last_cluster = G_used;
                 g_last_kernel = 2;
+                g_last_threads = 512;
             }
             return st;
         }
@@ -1275,7 +1269,7 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
                                                : 0;
                 if (fit >= q.BH * cand) {
                     double cc = 0.0;
-                    const int Gc = choose_cluster_rows(q.n, q.BH, cluster_fit, &ctx, &cc);
+                    const int Gc = choose_cluster_rows(q.n, q.BH, cluster_fit, &ctx, &cc, 512);
                     // the global barrier and L2 round trips cost more per step than a cluster's
                     const double cg = 1.15 * (double)ceil_div(q.n, cand);
                     if (g_kernel_override == 3 || Gc <= 0 || cg < cc) Gg = cand;
@@ -1292,30 +1286,49 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
             a.gs_mk = static_cast<float*>(cv.take(sizeof(float) * q.BH * kGsMaxG));
             if (!cv.fits()) return Status::fail(4, "select: workspace too small");
             a.gs = 1;
+            a.gs_force_ns = select_force_timeout_ns();
             cudaError_t err = cudaMemsetAsync(a.gs_bar, 0, sizeof(unsigned) * q.BH, stream);
             if (err == cudaSuccess) dispatch(var, q.dtype, vec, q.d, true, &a, smem, stream, Gg, &err);
             if (err == cudaSuccess) err = cudaGetLastError();
             if (err != cudaSuccess) return Status::cuda(err, "select (global sync) launch");
             g_last_cluster = Gg;
             g_last_kernel = 3;
+            g_last_threads = 512;
             return Status::ok();
         }
     }
 
     int G = g_cluster_override;
+    int nt = 512;
     if (G <= 0) {
-        // the cluster size with the least work per CTA times waves of clusters
+        // the cluster size (and CTA width) with the least work per CTA times waves of clusters
         const ClusterKey key{dev, g_kernel_override == 4 ? 5 : 1, q.n, q.BH, q.r, q.d, q.dtype};
-        G = cached_cluster_lookup(key);
-        if (G <= 0) {
-            G = choose_cluster_rows(q.n, q.BH, cluster_fit, &ctx, nullptr);
-            if (G > 0) cached_cluster_store(key, G);
+        const int memo = cached_cluster_lookup(key);
+        if (memo > 0) {
+            G = memo & 0xff;
+            nt = (memo & 0x100) ? 256 : 512;
+        } else {
+            double c512 = 0.0, c256 = 0.0;
+            G = choose_cluster_rows(q.n, q.BH, cluster_fit, &ctx, &c512, 512);
+            if (g_kernel_override != 4) {
+                ClusterCtx ctx256 = ctx;
+                ctx256.nt = 256;
+                const int G256 = choose_cluster_rows(q.n, q.BH, cluster_fit, &ctx256, &c256, 256);
+                // only in one wave: with waves of clusters the rows-per-CTA model
+                // misjudged it (128 instances of 4096 keys ran 1.7x slower)
+                const bool one_wave = G256 > 0 && cluster_fit(G256, &ctx256) >= q.BH;
+                if (one_wave && (G <= 0 || kHalfCtaCost * c256 < c512)) {
+                    G = G256;
+                    nt = 256;
+                }
+            }
+            if (G > 0) cached_cluster_store(key, G | (nt == 256 ? 0x100 : 0));
         }
         if (G <= 0) return Status::fail(2, "select: no schedulable cluster shape (n / 16 above 16384 rows?)");
     } else if (ceil_div(q.n, G) > kMaxRowsPerCta) {
         return Status::fail(2, "select: n / G exceeds the per-CTA row limit (16384)");
     }
-    plan(q.n, q.r, q.d, q.dtype, G, vec, false, &a, &smem, &var);
+    plan(q.n, q.r, q.d, q.dtype, G, vec, false, &a, &smem, &var, nt);
     if (smem > kSmemCap) return Status::fail(2, "select: shared memory plan exceeds 227 KB");
     cudaError_t err = cudaSuccess;
     dispatch(var, q.dtype, vec, q.d, false, &a, smem, stream, G, &err);
@@ -1323,6 +1336,7 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     if (err != cudaSuccess) return Status::cuda(err, "select launch");
     g_last_cluster = G;
     g_last_kernel = var.km == 2 ? 4 : 1;
+    g_last_threads = nt;
     return Status::ok();
 }
 

@@ -821,6 +821,7 @@ bool plan_bulk(int64_t n, int r, int d, int dtype, int G, BulkArgs* a, size_t* s
 }  // namespace
 
 void set_select_force_timeout(unsigned long long ns) { g_force_select_timeout_ns = ns; }
+unsigned long long select_force_timeout_ns() { return g_force_select_timeout_ns; }
 
 int read_select_status(bool clear) {
     int v = 0;

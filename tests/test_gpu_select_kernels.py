@@ -67,6 +67,9 @@ def test_both_kernels_match_the_oracle(orc, w, G):
         assert used in expect
         if w.name == "kres_g4" and kernel == 4:
             assert used == 4  # resident bf16 keys, d = 64: tensor-core key pass
+        if w.name == "kres_g4" and kernel == 0 and G == 0:
+            # automatic: two 256-thread CTAs per SM, 8 per instance
+            assert wc.last_select_threads() == 256 and wc.last_select_cluster() == 8
         gc.pivots_agree_until_tie(S, own["S"], own["margin"], rank, own["rank"], F, own["F"], EPS)
         for b in range(w.BH):
             rr = rank[b]
@@ -207,3 +210,26 @@ def test_global_sync_forward_matches_staged_calls(orc):
     O = wc.attend(d["Q"], K_S, rank, w.beta, V_S, wv, vmin, vmax)
     assert torch.equal(S_f, S) and torch.equal(rank_f, rank) and torch.equal(O_f, O)
     assert wc.device_status() == 0
+
+
+def test_global_sync_barrier_timeout_reports_and_recovers():
+    """The test hook keeps CTA 0 of every instance from arriving at the third
+    counter barrier; every CTA's bounded wait ends (1 ms), the timeout is
+    recorded, all stop after one step, and the next call is clean."""
+    w = gc.case("gs_timeout", "iid", 2, 16384, 64, 128, 32, "bf16")
+    dev, _ = workloads.make(w)
+    K = dev["K"].cuda()
+    wc.set_select_kernel(3)
+    assert wc.device_status() == 0
+    wc.force_select_timeout(1_000_000)
+    try:
+        S, F, rank, _ = wc.select(K, w.beta, w.r, w.pivot_seed, EPS)
+        assert wc.last_select_kernel() == 3
+        assert wc.device_status() == 5
+        assert torch.all(rank == 1)
+    finally:
+        wc.force_select_timeout(0)
+    S, F, rank, _ = wc.select(K, w.beta, w.r, w.pivot_seed, EPS)
+    assert wc.last_select_kernel() == 3
+    assert wc.device_status() == 0
+    assert torch.all(rank == w.r)
