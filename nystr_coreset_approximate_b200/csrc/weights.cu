@@ -220,32 +220,62 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* Ypart, 
     }
 }
 
-// Back substitution with one warp per right-hand column (r <= kTrsmWarpMaxR):
-// the column lives in shared memory; pivot a (bottom up) gives
-// x_a = y_a / F_S[a, a], then the lanes subtract F_S[a, j] x_a from every
-// y_j, j < a, reading row a of the pivot block contiguously.  Warps are
-// independent: no block barrier.
+// Back substitution with one warp per right-hand column (r <= kTrsmWarpMaxR).
+// When the pivot block fits in shared memory (r <= ~220) the CTA first sums
+// the split-K partials of its 16 columns (coalesced over the columns) and
+// copies F_S there, so the per-pivot row reads stay on chip; otherwise each
+// warp sums its own column and reads the rows from global memory.  Then
+// pivot a (bottom up) gives x_a = y_a / F_S[a, a], and the lanes subtract
+// F_S[a, j] x_a from every y_j, j < a, reading row a contiguously.
 constexpr int kTrsmWarps = 16;
 constexpr int kTrsmWarpMaxR = 1024;
+constexpr size_t kTrsmSmemCap = 200 * 1024;
 
-__global__ void __launch_bounds__(kTrsmWarps * 32) trsm_warp_kernel(const float* Ypart, int nsplit, const float* FS,
+inline bool trsm_fs_in_smem(int r) {
+    return sizeof(float) * ((size_t)kTrsmWarps * r + (size_t)r * r) <= kTrsmSmemCap;
+}
+
+template <bool FS_SMEM>
+__global__ void __launch_bounds__(kTrsmWarps * 32) trsm_warp_kernel(const float* __restrict__ Ypart, int nsplit,
+                                                                    const float* __restrict__ FS,
                                                                     const int32_t* rank, int64_t BH, int r, int D,
                                                                     float* V_S, float* w) {
-    extern __shared__ float ysm[];  // [kTrsmWarps][r]
+    extern __shared__ float ysm[];  // [kTrsmWarps][r], then (FS_SMEM) F_S [r][r]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t b = blockIdx.y;
-    const int col = blockIdx.x * kTrsmWarps + warp;
+    const int cb0 = blockIdx.x * kTrsmWarps;
     const int DP = D + 1;
-    if (col >= DP) return;  // no block-wide synchronisation below
     const int rr = rank[b];
+    const int col = cb0 + warp;
+    const float* __restrict__ Lg = FS + b * (int64_t)r * r;  // Lg[a * r + j] = F_S[a, j], j <= a
     float* y = ysm + (size_t)warp * r;
-    for (int j = lane; j < rr; j += 32) {
-        float s = 0.f;
-        for (int sp = 0; sp < nsplit; ++sp) s += Ypart[(((int64_t)sp * BH + b) * r + j) * DP + col];
-        y[j] = s;
+    const float* Lb = Lg;
+    if constexpr (FS_SMEM) {
+        // the CTA sums its 16 columns' partials (coalesced over columns) and stages F_S
+        float* Ls = ysm + (size_t)kTrsmWarps * r;
+        for (int e = threadIdx.x; e < rr * kTrsmWarps; e += kTrsmWarps * 32) {
+            const int j = e / kTrsmWarps, c = e % kTrsmWarps;
+            float s = 0.f;
+            if (cb0 + c < DP)
+                for (int sp = 0; sp < nsplit; ++sp) s += Ypart[(((int64_t)sp * BH + b) * r + j) * DP + cb0 + c];
+            ysm[(size_t)c * r + j] = s;
+        }
+        for (int e = threadIdx.x; e < rr * r; e += kTrsmWarps * 32) {
+            const int a = e / r, j = e % r;
+            Ls[e] = j <= a ? Lg[e] : 0.f;
+        }
+        __syncthreads();
+        Lb = Ls;
+        if (col >= DP) return;  // no block-wide synchronisation below
+    } else {
+        if (col >= DP) return;  // warps are independent from here on
+        for (int j = lane; j < rr; j += 32) {
+            float s = 0.f;
+            for (int sp = 0; sp < nsplit; ++sp) s += Ypart[(((int64_t)sp * BH + b) * r + j) * DP + col];
+            y[j] = s;
+        }
+        __syncwarp();
     }
-    __syncwarp();
-    const float* Lb = FS + b * (int64_t)r * r;  // Lb[a * r + j] = F_S[a, j], j <= a
     for (int a = rr - 1; a >= 0; --a) {
         const float* La = Lb + (int64_t)a * r;
         const float xa = y[a] / La[a];
@@ -322,10 +352,12 @@ Status run_weights(const WeightsRequest& q, cudaStream_t st) {
     gather_fs<<<dim3(q.r, (unsigned)q.BH), 128, 0, st>>>(q.F, q.S, q.rank, q.n, q.r, FS);
     cudaError_t e;
     if (q.r <= kTrsmWarpMaxR) {
-        const size_t smem = sizeof(float) * (size_t)kTrsmWarps * q.r;
-        e = cudaFuncSetAttribute(trsm_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        const bool fs_sm = trsm_fs_in_smem(q.r);
+        const size_t smem = sizeof(float) * ((size_t)kTrsmWarps * q.r + (fs_sm ? (size_t)q.r * q.r : 0));
+        auto kern = fs_sm ? trsm_warp_kernel<true> : trsm_warp_kernel<false>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return Status::cuda(e, "weights: trsm smem attribute");
-        trsm_warp_kernel<<<dim3((unsigned)ceil_div(D + 1, kTrsmWarps), (unsigned)q.BH), kTrsmWarps * 32, smem, st>>>(
+        kern<<<dim3((unsigned)ceil_div(D + 1, kTrsmWarps), (unsigned)q.BH), kTrsmWarps * 32, smem, st>>>(
             Ypart, nsplit, FS, q.rank, q.BH, q.r, D, q.V_S, q.w);
     } else {
         const size_t smem = sizeof(float) * ((size_t)q.r * kTrsmCB + kTrsmBlk * (kTrsmBlk + 1));
