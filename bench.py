@@ -40,13 +40,13 @@ FLUSH_BYTES = 256 << 20
 EPS = 1e-6
 
 
-def launches_per_forward(w):
-    """Kernels one wildcat_forward launches: select 1, weights 5 (range partial
-    and finalize, F^T(V,1), pivot-block gather, solve), attend 3 on CUDA
-    cores (norm partials, shift, attend) or 4 on the tensor-core path (plus
-    the hi/lo split of [V_S|w])."""
+def launches_per_forward(w, select_launches=1):
+    """Kernels one wildcat_forward launches: select 1 (or one per phase of a
+    long coreset), weights 5 (range partial and finalize, F^T(V,1),
+    pivot-block gather, solve), attend 3 on CUDA cores (norm partials, shift,
+    attend) or 4 on the tensor-core path (plus the hi/lo split of [V_S|w])."""
     tc = w.dtype == "bf16" and w.d in (64, 128)
-    return 1 + 5 + (4 if tc else 3)
+    return select_launches + 5 + (4 if tc else 3)
 
 
 def parse():
@@ -65,6 +65,8 @@ def parse():
                    help="CTAs per instance in the select (0 = automatic; a fixed size keeps 512-thread CTAs)")
     p.add_argument("--weights-inverse", action="store_true",
                    help="also time the inverse-maintenance weights route on the selected pivots")
+    p.add_argument("--select-phase-steps", type=int, default=0,
+                   help="select steps per launch (0 = automatic: r / 8 for r >= 512; < 0 = one launch)")
     p.add_argument("--select-kernel", type=int, choices=[0, 1, 2, 3, 4], default=0,
                    help="0 = automatic (the cp.async kernel), 1 = cp.async, 2 = bulk-copy where it applies")
     return p.parse_args()
@@ -256,6 +258,7 @@ def main():
     torch.cuda.set_device(local)
     wc.set_select_kernel(args.select_kernel)
     wc.set_select_cluster(args.select_cluster)
+    wc.set_select_phase_steps(args.select_phase_steps)
     if world > 1:
         from datetime import timedelta
 
@@ -286,6 +289,7 @@ def main():
     sel_kind = wc.last_select_kernel()
     sel_cluster = wc.last_select_cluster()
     sel_threads = wc.last_select_threads()
+    sel_launches = wc.last_select_phases()
 
     # ---- timed forward: K steps, own events per step, L2 flushed in between ----
     clocks = ClockSampler(local)
@@ -408,14 +412,15 @@ def main():
                                        "nbins": nb,
                                        "select_kernel": SELECT_KERNELS[sel_kind][0],
                                        "select_cluster_ctas": sel_cluster,
-                                       "select_cta_threads": sel_threads}),
+                                       "select_cta_threads": sel_threads,
+                                       "select_launches": sel_launches}),
         "entries_per_s": value * w.BH * w.m * w.n,
         "stages_ms": {k: statistics.mean(v) for k, v in stage_ms.items()},
         "roofline": {"kernel": SELECT_KERNELS[sel_kind][0], "bound": "hbm", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} hbm_gbs", "traffic": traffic,
                      "algorithmic_bytes_per_launch": nbytes, "launch_ms": sel_ms},
-        "gpu_launches": (launches_per_forward(w) + (1 if nb > 1 else 0)) * args.steps,
+        "gpu_launches": (launches_per_forward(w, sel_launches) + (1 if nb > 1 else 0)) * args.steps,
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cpu,

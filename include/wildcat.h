@@ -121,8 +121,14 @@ wildcat_status wildcat_select(const void* K, int dtype, int64_t BH, int64_t n, i
  * at once).  The grid is launched cooperatively (all CTAs co-resident); every
  * barrier wait is bounded (2 s, WILDCAT_ERR_TIMEOUT in the device status
  * word on expiry).  Results equal wildcat_select's to float32 rounding.
- * workspace may be NULL (then exactly wildcat_select).  wildcat_forward*
- * carve this workspace from theirs.
+ * The workspace also enables phases for long coresets (r >= 512, BH at most
+ * the SM count): the steps run as launches of about r / 8 steps; between
+ * them each instance still going keeps its residual diagonal in the
+ * workspace, and the next launch (global sync over the whole GPU) gives each
+ * such instance about SMs / (instances still going) CTAs, up to 32.  The
+ * instances whose factor truncated early no longer leave the longest ones on
+ * the few CTAs of the first launch.  workspace may be NULL (then exactly
+ * wildcat_select).  wildcat_forward* carve this workspace from theirs.
  */
 size_t wildcat_select_workspace_size(int64_t BH, int64_t n);
 wildcat_status wildcat_select_ws(const void* K, int dtype, int64_t BH, int64_t n, int d, float beta,
@@ -432,6 +438,21 @@ int wildcat_last_select_kernel(void);
  * the automatic choice put two CTAs on each SM (twice the cluster size, half
  * the rows per CTA; resident keys only).  0 if none. */
 int wildcat_last_select_threads(void);
+
+/*
+ * wildcat_set_select_phase_steps -- steps per launch of a select call that
+ * has a workspace (wildcat_select_ws and the forward calls): 0 (default)
+ * automatic, ceil(r / 8) when r >= 512 and a single launch otherwise; > 0
+ * that many steps per launch for any r (the phases apply where the
+ * workspace, BH <= SM count and n % 4 == 0 allow them); < 0 always one
+ * launch.  Results do not depend on it beyond float32 rounding of the
+ * search sums.  Process-wide; not thread-safe against concurrent select
+ * calls.  Always returns WILDCAT_OK.
+ */
+wildcat_status wildcat_set_select_phase_steps(int steps);
+
+/* Launches of the last select call on this thread (1 = no phases), 0 if none. */
+int wildcat_last_select_phases(void);
 
 /*
  * wildcat_set_select_cluster -- tuning knob for wildcat_select*: number of

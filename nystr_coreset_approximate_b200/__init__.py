@@ -26,7 +26,8 @@ __all__ = [
     "WildcatError", "library_path", "lib", "declared_symbols", "select", "select_fixed",
     "weights", "weights_inverse", "attend", "attend_noalloc", "decode_attend", "forward", "forward_ex", "Options", "forward_binned", "BinnedForwardPlan", "forward_host", "ForwardPlan", "pivot_uniforms",
     "set_select_cluster", "last_select_cluster", "set_select_kernel", "last_select_kernel",
-    "force_select_timeout", "last_select_threads", "device_status", "DTYPES",
+    "force_select_timeout", "last_select_threads", "set_select_phase_steps", "last_select_phases",
+    "device_status", "DTYPES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -87,6 +88,8 @@ _SIGS = {
     "wildcat_set_select_kernel": ([_int], _int),
     "wildcat_last_select_kernel": ([], _int),
     "wildcat_last_select_threads": ([], _int),
+    "wildcat_set_select_phase_steps": ([_int], _int),
+    "wildcat_last_select_phases": ([], _int),
 }
 
 
@@ -510,6 +513,17 @@ def last_select_kernel() -> int:
 def last_select_threads() -> int:
     """Threads per CTA of the last select launch (256 or 512)."""
     return int(lib().wildcat_last_select_threads())
+
+
+def set_select_phase_steps(steps: int):
+    """Steps per select launch when a workspace is given: 0 = automatic
+    (r / 8 for r >= 512), > 0 = that many, < 0 = one launch."""
+    _check(lib().wildcat_set_select_phase_steps(int(steps)))
+
+
+def last_select_phases() -> int:
+    """Launches of the last select call (1 = no phases)."""
+    return int(lib().wildcat_last_select_phases())
 
 
 def force_select_timeout(nanoseconds: int):

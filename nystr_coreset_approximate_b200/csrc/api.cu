@@ -612,6 +612,13 @@ int wildcat_last_select_kernel(void) { return wildcat::last_select_kernel(); }
 
 int wildcat_last_select_threads(void) { return wildcat::last_select_threads(); }
 
+wildcat_status wildcat_set_select_phase_steps(int steps) {
+    wildcat::select_phase_steps_override(steps, true);
+    return record(Status::ok());
+}
+
+int wildcat_last_select_phases(void) { return wildcat::last_select_phases(); }
+
 wildcat_status wildcat_set_select_cluster(int ctas_per_instance) {
     const int G = ctas_per_instance;
     if (G != 0 && G != 1 && G != 2 && G != 4 && G != 8 && G != 16)

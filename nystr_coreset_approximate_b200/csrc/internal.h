@@ -47,6 +47,8 @@ int select_kernel_override(int k);  // k < 0: query only; 0 automatic, 1 cp.asyn
                                     // allows, 4 cp.async (clusters) with the tensor-core key pass where it applies
 int last_select_kernel();           // 1, 2, 3 as above; 4 clusters with the tensor-core key pass
 int last_select_threads();          // threads per CTA of the last select launch (256 or 512)
+int select_phase_steps_override(int k, bool set);  // steps per launch: 0 automatic, < 0 one launch
+int last_select_phases();           // launches of the last select call (1 = no phases)
 // cluster-size choice shared by both select kernels (select.cu)
 struct ClusterKey {
     int dev, kernel;

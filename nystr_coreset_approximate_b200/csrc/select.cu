@@ -40,6 +40,7 @@ constexpr int kFsByWarp0 = 512;  // factor rows up to this length are gathered b
 constexpr unsigned kTckCols = 128;  // tensor memory columns of the key pass: 8 tiles x 16
 constexpr int kMaxPL = 16;  // R <= 16384 rows per CTA -> at most 16 values per lane
 constexpr size_t kSmemCap = 227 * 1024;
+constexpr int kGsMaxCtas = 32;  // global-sync CTAs per instance: one search lane each
 
 struct SelectArgs {
     const void* K;
@@ -67,6 +68,30 @@ struct SelectArgs {
     float* gs_mk;      // [BH][G] per-CTA max |k|^2
     int gs;            // 1: the launch is the global-sync one
     unsigned long long gs_force_ns;  // test hook: CTA 0 of each instance skips barrier 2; waits end after this
+    // phases: the launch runs steps [step0, step_end); an instance still going at
+    // step_end saves its residual diagonal and joins the list of the next phase
+    int step0, step_end;
+    float* ph_resid;       // [BH][n] residual diagonal of paused instances
+    float* ph_mk;          // [BH] M_K (written by the first phase)
+    const int* act_in;     // resumed launch (global sync): instances to continue, count at act_n_in
+    const int* act_n_in;
+    int* act_out;          // instances paused at step_end (order of arrival), count at act_n_out
+    int* act_n_out;
+    int grid_ctas;         // resumed launch: CTAs of the grid (else BH G)
+};
+
+// Rows per CTA, thread groups and search-chunk width for G CTAs per instance
+// (host plan and the resumed launch's per-phase choice use the same rule).
+struct SelectShape {
+    int R, JG, PL, Rpad;
+    __host__ __device__ SelectShape(int64_t n, int G, int nt, int vec) {
+        R = (int)round_up(ceil_div(n, G), 4);
+        JG = 1;
+        while (JG * 2 <= 8 && (int64_t)(nt / (JG * 2)) * vec >= R) JG *= 2;
+        const int64_t pl = round_up(ceil_div(ceil_div(R, 32), 32), 4);
+        PL = (int)(pl > 4 ? pl : 4);
+        Rpad = (int)round_up(R, 32 * PL);
+    }
 };
 
 struct SmemLayout {
@@ -217,17 +242,41 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
     constexpr int RPW = 32 / LPR;             // key rows per warp-wide load
     constexpr int UF = 8;                     // factor loads in flight per thread (scalar path)
     cg::cluster_group cluster = cg::this_cluster();
-    const int crank = GS ? (int)(blockIdx.x % a.G) : (int)cluster.block_rank();
-    const int64_t b = blockIdx.x / a.G;
-    if (b >= a.BH) return;  // whole clusters only: G divides gridDim.x
+    int G = a.G, R = a.R, JG = a.JG, PL = a.PL;
+    int64_t b;
+    int crank;
+    const bool resume = GS && a.act_in != nullptr;
+    if (resume) {
+        // a resumed phase: the A instances still going share the grid, each
+        // with as many CTAs as fit (a.G is the least the host planned for)
+        const int A = *a.act_n_in;
+        if (A <= 0) return;
+        int g = (int)(gridDim.x / (unsigned)A);
+        g = g < kGsMaxCtas ? g : kGsMaxCtas;
+        const int64_t by_rows = a.n / 512;
+        g = (int64_t)g < by_rows ? g : (int)(by_rows > 1 ? by_rows : 1);
+        G = g > a.G ? g : a.G;
+        const SelectShape sh(a.n, G, NTH, VEC);
+        R = sh.R;
+        JG = sh.JG;
+        PL = sh.PL;
+        const int slot = (int)(blockIdx.x / (unsigned)G);
+        if (slot >= A) return;  // whole groups only
+        b = a.act_in[slot];
+        crank = (int)(blockIdx.x % (unsigned)G);
+    } else {
+        crank = GS ? (int)(blockIdx.x % a.G) : (int)cluster.block_rank();
+        b = blockIdx.x / a.G;
+        if (b >= a.BH) return;  // whole clusters only: G divides gridDim.x
+    }
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int R = a.R, r = a.r, JG = a.JG, TPG = NT / JG, G = a.G;
+    const int r = a.r, TPG = NT / JG;
     const int64_t n = a.n;
     const int64_t row0 = (int64_t)crank * R;
     const int64_t row_end = (row0 + R < n) ? row0 + R : n;
     const int nrows = row_end > row0 ? (int)(row_end - row0) : 0;
-    const int PL = a.PL, CH = 32 * PL;
+    const int CH = 32 * PL;
     const int nch = (int)ceil_div(R, CH);
     const int Rpad = nch * CH;  // residual buffers cover whole search chunks
 
@@ -457,6 +506,27 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
     };
 
     // ---------------- prologue: M_K and the initial residual diagonal ----------------
+    // (a resumed phase reads both back instead)
+    const int step0 = a.step0;
+    float MK;
+    // tensor-core key pass: B operand (zero outside its first three columns),
+    // the MMA completion barrier and the accumulator columns in tensor memory
+    unsigned tmem = 0;
+    uint64_t* tc_bar = reinterpret_cast<uint64_t*>(smem + L.mbar);
+    unsigned tc_phase = 0;
+    if (resume) {
+        if (tid == 0) misc[1] = a.ph_mk[b];
+        const float* src = a.ph_resid + b * n + row0;
+        float* d0 = dbuf + (size_t)(step0 & 1) * Rpad;
+        for (int row = tid; row < Rpad; row += NT) {
+            const float v = row < nrows ? __ldcg(src + row) : 0.f;
+            d0[row] = v;
+            gres(step0 & 1)[row] = v;
+        }
+        __syncthreads();
+        MK = misc[1];
+        publish(d0, step0 & 1, false, step0);
+    } else {
     if constexpr (KRES) {
         const int pieces = nrows * LPR;
         for (int c = tid; c < pieces; c += NT) {
@@ -467,11 +537,6 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
         cp_async_wait<0>();
         __syncthreads();
     }
-    // tensor-core key pass: B operand (zero outside its first three columns),
-    // the MMA completion barrier and the accumulator columns in tensor memory
-    unsigned tmem = 0;
-    uint64_t* tc_bar = reinterpret_cast<uint64_t*>(smem + L.mbar);
-    unsigned tc_phase = 0;
     if constexpr (TCK) {
         for (int e = tid; e < (D / 64) * 16 * 128 / 16; e += NT)
             reinterpret_cast<float4*>(smem + L.btile)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -526,15 +591,17 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
         }
     }
     __syncthreads();
-    const float MK = misc[1];
-    const float beta = a.beta;
+    MK = misc[1];
+    if (a.ph_mk && crank == 0 && tid == 0) a.ph_mk[b] = MK;
     for (int row = tid; row < Rpad; row += NT) {
-        const float v = row < nrows ? expf(beta * (dotb[row] - MK)) : 0.f;
+        const float v = row < nrows ? expf(a.beta * (dotb[row] - MK)) : 0.f;
         dbuf[row] = v;
         if constexpr (GS) gres(0)[row] = v;
     }
     __syncthreads();
     publish(dbuf, 0, false, 0);
+    }
+    const float beta = a.beta;
     const bool gs_ok = !(GS && imisc[5]);
 
     // ---------------- r sequential steps ----------------
@@ -543,8 +610,9 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
     // block covers chunk (base + 128 w) / 128 with the search's lane layout.
     const bool fused_csl = (VEC == 4 && PL == 4);
     const int g = tid / TPG, tt = tid % TPG;
-    int i = 0;
-    for (; gs_ok && i < r; ++i) {
+    const int step_end = a.step_end;
+    int i = step0;
+    for (; gs_ok && i < step_end; ++i) {
         // a barrier ran out: the steps before it are complete (uniform: read after the barrier's block sync)
         if (GS && imisc[5]) break;
         const int cur = i & 1, nxt = cur ^ 1;
@@ -873,19 +941,27 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
         publish(dnxt, nxt, fused_csl, i + 1);
     }
 
-    // ---------------- effective rank, padding past it ----------------
-    const int rr = i;
-    for (int j = rr; j < r; ++j) {
-        float* dst = Fb + (int64_t)j * n + row0;
-        for (int row = tid; row < nrows; row += NT) dst[row] = 0.f;
-    }
-    if (crank == 0) {
-        if (tid == 0) a.rank[b] = rr;
-        for (int j = rr + tid; j < r; j += NT)
-            if (a.S) a.S[b * r + j] = -1;
-        if (a.K_S) {
-            T* dst = reinterpret_cast<T*>(a.K_S) + b * r * D;
-            for (int64_t e = (int64_t)rr * D + tid; e < (int64_t)r * D; e += NT) dst[e] = T(0.f);
+    // ---------------- pause at the phase end, or the effective rank and padding past it ----------------
+    if (i == step_end && step_end < r && !(GS && imisc[5])) {
+        // still going: keep the residual diagonal (the buffer of step i) for the next phase
+        const float* dcur = dbuf + (size_t)(i & 1) * Rpad;
+        float* dst = a.ph_resid + b * n + row0;
+        for (int row = tid; row < nrows; row += NT) dst[row] = dcur[row];
+        if (crank == 0 && tid == 0) a.act_out[atomicAdd(a.act_n_out, 1)] = (int)b;
+    } else {
+        const int rr = i;
+        for (int j = rr; j < r; ++j) {
+            float* dst = Fb + (int64_t)j * n + row0;
+            for (int row = tid; row < nrows; row += NT) dst[row] = 0.f;
+        }
+        if (crank == 0) {
+            if (tid == 0) a.rank[b] = rr;
+            for (int j = rr + tid; j < r; j += NT)
+                if (a.S) a.S[b * r + j] = -1;
+            if (a.K_S) {
+                T* dst = reinterpret_cast<T*>(a.K_S) + b * r * D;
+                for (int64_t e = (int64_t)rr * D + tid; e < (int64_t)r * D; e += NT) dst[e] = T(0.f);
+            }
         }
     }
     if constexpr (TCK) {
@@ -917,7 +993,7 @@ cudaError_t launch_select_t(const SelectArgs& a, size_t smem, cudaStream_t strea
         if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(a.BH * a.G));
+    cfg.gridDim = dim3((unsigned)(a.grid_ctas > 0 ? a.grid_ctas : a.BH * a.G));
     cfg.blockDim = dim3(NTH);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -1049,9 +1125,11 @@ int dispatch(const Variant& v, int dtype, int vec, int d, bool gs, const SelectA
 
 int g_cluster_override = 0;
 int g_kernel_override = 0;
+int g_phase_steps = 0;  // 0 automatic, > 0 fixed phase length, < 0 one launch
 thread_local int g_last_cluster = 0;
 thread_local int g_last_kernel = 0;
 thread_local int g_last_threads = 0;
+thread_local int g_last_phases = 0;
 
 }  // namespace
 
@@ -1103,16 +1181,35 @@ int choose_cluster_rows(int64_t n, int64_t BH, int (*fit)(int G, void* ctx), voi
     return best;
 }
 
-// Exchange buffers of the global-sync mode (G <= kGsMaxG CTAs per instance).
-constexpr int kGsMaxG = 32;
-size_t select_workspace_bytes(int64_t BH, int64_t n) {
-    Carve cv(nullptr, 0);
-    cv.take(sizeof(double) * BH * 2 * kGsMaxG * 33);
-    cv.take(sizeof(float) * BH * 2 * (n + (int64_t)kGsMaxG * 520));  // G Rpad <= n + G (4 + 511)
-    cv.take(sizeof(unsigned) * BH);
-    cv.take(sizeof(float) * BH * kGsMaxG);
-    return cv.used + 256;
+// Workspace of the global-sync mode (G <= kGsMaxCtas CTAs per instance) and
+// of phased launches.  ctl holds [count 0][barrier counter per instance][count 1]
+// so that one memset clears a launch's barriers and its output count.
+struct SelectWs {
+    double* inbox;
+    float* resid;
+    unsigned* ctl;
+    float* mk;
+    float* ph_resid;
+    float* ph_mk;
+    int* act;  // two lists of BH instance indices
+    size_t used;
+    bool fits;
+};
+static SelectWs carve_select_ws(void* ws, size_t bytes, int64_t BH, int64_t n) {
+    Carve cv(ws, bytes);
+    SelectWs w{};
+    w.inbox = static_cast<double*>(cv.take(sizeof(double) * BH * 2 * kGsMaxCtas * 33));
+    w.resid = static_cast<float*>(cv.take(sizeof(float) * BH * 2 * (n + (int64_t)kGsMaxCtas * 520)));  // G Rpad <= n + G (4 + 511)
+    w.ctl = static_cast<unsigned*>(cv.take(sizeof(unsigned) * (BH + 2)));
+    w.mk = static_cast<float*>(cv.take(sizeof(float) * BH * kGsMaxCtas));
+    w.ph_resid = static_cast<float*>(cv.take(sizeof(float) * BH * n));
+    w.ph_mk = static_cast<float*>(cv.take(sizeof(float) * BH));
+    w.act = static_cast<int*>(cv.take(sizeof(int) * 2 * BH));
+    w.used = cv.used;
+    w.fits = cv.fits();
+    return w;
 }
+size_t select_workspace_bytes(int64_t BH, int64_t n) { return carve_select_ws(nullptr, 0, BH, n).used + 256; }
 
 int read_select_gs_status(bool clear) {
     int v = 0;
@@ -1137,14 +1234,16 @@ int select_kernel_override(int k) {
 }
 int last_select_kernel() { return g_last_kernel; }
 int last_select_threads() { return g_last_threads; }
+int select_phase_steps_override(int k, bool set) {
+    if (set) g_phase_steps = k;
+    return g_phase_steps;
+}
+int last_select_phases() { return g_last_phases; }
 
 static void plan(int64_t n, int r, int d, int dtype, int G, int vec, bool gs, SelectArgs* a, size_t* smem,
                  Variant* v, int nt = 512) {
-    const int R = (int)round_up(ceil_div(n, G), 4);
-    int JG = 1;
-    while (JG * 2 <= 8 && (int64_t)(nt / (JG * 2)) * vec >= R) JG *= 2;
-    const int PL = (int)std::max<int64_t>(4, round_up(ceil_div(ceil_div(R, 32), 32), 4));
-    const int Rpad = (int)round_up(R, 32 * PL);
+    const SelectShape sh(n, G, nt, vec);
+    const int R = sh.R, JG = sh.JG, PL = sh.PL, Rpad = sh.Rpad;
     a->G = G;
     a->R = R;
     a->JG = JG;
@@ -1209,6 +1308,51 @@ static int cluster_fit(int g, void* p) {
 // share the SM's issue slots and bandwidth: their rows per CTA count 1.3x.
 constexpr double kHalfCtaCost = 1.3;
 
+// Phases: the factorisation of a long coreset runs as launches of `len`
+// steps.  The first is the ordinary launch; after it the instances still going
+// (the others truncated) continue in global-sync launches of the whole GPU,
+// each with about SMs / (instances left) CTAs, so that the longest factors no
+// longer run on the few CTAs the first launch gave them.
+constexpr int kPhaseMinRank = 512;
+constexpr int kPhaseCount = 8;
+struct PhasePlan {
+    int len = 0;
+    int Gmin = 0;
+    int P = 0;
+    Variant var{};
+    size_t smem = 0;
+    SelectArgs ra{};
+};
+static bool plan_phases(const SelectRequest& q, const SelectArgs& a, int vec, int sms, cudaStream_t st,
+                        PhasePlan* pp) {
+    int len = g_phase_steps;
+    if (len == 0) len = q.r >= kPhaseMinRank ? (int)ceil_div(q.r, kPhaseCount) : 0;
+    if (len <= 0 || len >= q.r || vec != 4 || q.BH > sms) return false;
+    const int Gmin = (int)std::min<int64_t>(kGsMaxCtas, sms / q.BH);
+    if (ceil_div(q.n, Gmin) > kMaxRowsPerCta) return false;
+    SelectArgs ra = a;
+    Variant var{};
+    size_t smem = 0;
+    plan(q.n, q.r, q.d, q.dtype, Gmin, vec, true, &ra, &smem, &var);
+    if (smem > kSmemCap) return false;
+    // the kernel may give an instance any G in [Gmin, kGsMaxCtas]: room for the largest layout
+    for (int G = Gmin; G <= kGsMaxCtas; ++G) {
+        const SelectShape sh(q.n, G, 512, vec);
+        smem = std::max(smem, SmemLayout(sh.Rpad, q.r, q.d, sh.JG, 512, vec, G, var.depth, 0, true).total);
+    }
+    if (smem > kSmemCap) return false;
+    int P = dispatch(var, q.dtype, vec, q.d, true, nullptr, smem, st, Gmin, nullptr);
+    P = std::min(P, sms);
+    if (P < q.BH * Gmin) return false;
+    pp->len = len;
+    pp->Gmin = Gmin;
+    pp->P = P;
+    pp->var = var;
+    pp->smem = smem;
+    pp->ra = ra;
+    return true;
+}
+
 Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     const int vec = (q.n % 4 == 0) ? 4 : 1;
     SelectArgs a{};
@@ -1227,6 +1371,9 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     a.F = q.F;
     a.rank = q.rank;
     a.K_S = q.K_S;
+    a.step0 = 0;
+    a.step_end = q.r;
+    g_last_phases = 1;
 
     if (g_kernel_override == 2) {
         // the bulk-copy kernel (select_bulk.cu) where its shape rules allow
@@ -1244,22 +1391,65 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     }
     size_t smem = 0;
     Variant var{};
-    int dev = 0;
+    int dev = 0, sms = 0;
     cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     ClusterCtx ctx{&q, &a, vec, stream};
+
+    const bool ws_ok = q.ws && q.ws_bytes >= select_workspace_bytes(q.BH, q.n) && vec == 4 &&
+                       (reinterpret_cast<uintptr_t>(q.ws) & 255u) == 0;
+    const SelectWs w = ws_ok ? carve_select_ws(q.ws, q.ws_bytes, q.BH, q.n) : SelectWs{};
+    PhasePlan pp;
+    const bool phased = ws_ok && w.fits && plan_phases(q, a, vec, sms, stream, &pp);
+    if (phased) {
+        a.step_end = pp.len;
+        a.ph_resid = w.ph_resid;
+        a.ph_mk = w.ph_mk;
+        a.act_out = w.act;
+        a.act_n_out = reinterpret_cast<int*>(w.ctl);
+        // count 0 and the barrier counters of the first launch
+        const cudaError_t err = cudaMemsetAsync(w.ctl, 0, sizeof(unsigned) * (q.BH + 1), stream);
+        if (err != cudaSuccess) return Status::cuda(err, "select: phase counters");
+    }
+    // the launches after the first one (global sync over the whole GPU)
+    auto resume = [&]() -> Status {
+        if (!phased) return Status::ok();
+        const int nph = (int)ceil_div(q.r, pp.len);
+        for (int p = 1; p < nph; ++p) {
+            SelectArgs ra = pp.ra;
+            ra.gs_inbox = w.inbox;
+            ra.gs_resid = w.resid;
+            ra.gs_mk = w.mk;
+            ra.gs_bar = w.ctl + 1;
+            ra.gs = 1;
+            ra.gs_force_ns = select_force_timeout_ns();
+            ra.step0 = p * pp.len;
+            ra.step_end = std::min(q.r, (p + 1) * pp.len);
+            ra.ph_resid = w.ph_resid;
+            ra.ph_mk = w.ph_mk;
+            ra.act_in = w.act + (size_t)((p - 1) & 1) * q.BH;
+            ra.act_n_in = reinterpret_cast<int*>(w.ctl + (((p - 1) & 1) ? q.BH + 1 : 0));
+            ra.act_out = w.act + (size_t)(p & 1) * q.BH;
+            ra.act_n_out = reinterpret_cast<int*>(w.ctl + ((p & 1) ? q.BH + 1 : 0));
+            ra.grid_ctas = pp.P;
+            // this launch's barrier counters and output count ([count 0][barriers][count 1])
+            cudaError_t err = cudaMemsetAsync(w.ctl + ((p & 1) ? 1 : 0), 0, sizeof(unsigned) * (q.BH + 1), stream);
+            if (err == cudaSuccess) dispatch(pp.var, q.dtype, vec, q.d, true, &ra, pp.smem, stream, pp.Gmin, &err);
+            if (err == cudaSuccess) err = cudaGetLastError();
+            if (err != cudaSuccess) return Status::cuda(err, "select (resumed phase) launch");
+        }
+        g_last_phases = nph;
+        return Status::ok();
+    };
 
     // Global-sync mode: given a workspace and few instances, more CTAs per
     // instance than clusters allow (all co-resident by a cooperative launch).
-    const bool ws_ok = q.ws && q.ws_bytes >= select_workspace_bytes(q.BH, q.n) && vec == 4 &&
-                       (reinterpret_cast<uintptr_t>(q.ws) & 255u) == 0;
     if (ws_ok && g_kernel_override != 1 && g_kernel_override != 4 && g_cluster_override <= 0) {
         const ClusterKey gkey{dev, g_kernel_override == 3 ? 4 : 3, q.n, q.BH, q.r, q.d, q.dtype};
         int Gg = cached_cluster_lookup(gkey);
         if (Gg == 0) {
             Gg = -1;
-            int sms = 0;
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-            const int cand = (int)std::min<int64_t>(kGsMaxG, sms / std::max<int64_t>(1, q.BH));
+            const int cand = (int)std::min<int64_t>(kGsMaxCtas, sms / std::max<int64_t>(1, q.BH));
             if (cand >= 2 && q.n / cand >= 512 && ceil_div(q.n, cand) <= kMaxRowsPerCta) {
                 SelectArgs t = a;
                 Variant v{};
@@ -1279,22 +1469,21 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
         }
         if (Gg > 0) {
             plan(q.n, q.r, q.d, q.dtype, Gg, vec, true, &a, &smem, &var);
-            Carve cv(q.ws, q.ws_bytes);
-            a.gs_inbox = static_cast<double*>(cv.take(sizeof(double) * q.BH * 2 * kGsMaxG * 33));
-            a.gs_resid = static_cast<float*>(cv.take(sizeof(float) * q.BH * 2 * (q.n + (int64_t)kGsMaxG * 520)));
-            a.gs_bar = static_cast<unsigned*>(cv.take(sizeof(unsigned) * q.BH));
-            a.gs_mk = static_cast<float*>(cv.take(sizeof(float) * q.BH * kGsMaxG));
-            if (!cv.fits()) return Status::fail(4, "select: workspace too small");
+            if (!w.fits) return Status::fail(4, "select: workspace too small");
+            a.gs_inbox = w.inbox;
+            a.gs_resid = w.resid;
+            a.gs_bar = w.ctl + 1;
+            a.gs_mk = w.mk;
             a.gs = 1;
             a.gs_force_ns = select_force_timeout_ns();
-            cudaError_t err = cudaMemsetAsync(a.gs_bar, 0, sizeof(unsigned) * q.BH, stream);
+            cudaError_t err = phased ? cudaSuccess : cudaMemsetAsync(w.ctl + 1, 0, sizeof(unsigned) * q.BH, stream);
             if (err == cudaSuccess) dispatch(var, q.dtype, vec, q.d, true, &a, smem, stream, Gg, &err);
             if (err == cudaSuccess) err = cudaGetLastError();
             if (err != cudaSuccess) return Status::cuda(err, "select (global sync) launch");
             g_last_cluster = Gg;
             g_last_kernel = 3;
             g_last_threads = 512;
-            return Status::ok();
+            return resume();
         }
     }
 
@@ -1337,7 +1526,7 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     g_last_cluster = G;
     g_last_kernel = var.km == 2 ? 4 : 1;
     g_last_threads = nt;
-    return Status::ok();
+    return resume();
 }
 
 Status launch_pivot_uniforms(uint64_t seed, int64_t BH, int steps, double* u, cudaStream_t stream) {

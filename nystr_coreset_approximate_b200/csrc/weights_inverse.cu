@@ -18,8 +18,8 @@
 //                    exp(beta (<k_Sa, k_l> - M_b)) (v_l, 1)
 //   inverse_kernel   one CTA per instance: the bordered inverse, pivot by
 //                    pivot (a matrix-vector product and a rank-one update per
-//                    pivot, the inverse in global memory), and the sum of Zpart
-//                    over splits
+//                    pivot; the inverse in shared memory when it fits, else in
+//                    global memory), and the sum of Zpart over splits
 //   xsolve_kernel    (V_S, w) = H_S^-1 Z, rounded to float32
 #include <algorithm>
 
@@ -178,12 +178,17 @@ __global__ void __launch_bounds__(kZThreads) z_kernel(const typename E::T* K, co
 
 // ---- the bordered inverse, one CTA per instance ----
 constexpr int kInvThreads = 512;
+constexpr size_t kInvSmemCap = 210 * 1024;
 
+template <bool A_SMEM>
 __global__ void __launch_bounds__(kInvThreads) inverse_kernel(const double* H, const int32_t* rank, int r, int D,
                                                               int nsplit, int64_t BH, double* Ainv, double* Zpart) {
     extern __shared__ __align__(16) unsigned char sm[];
     double* bvec = reinterpret_cast<double*>(sm);  // [r]
     double* y = bvec + r;                          // [r]
+    // with A_SMEM the inverse grows in shared memory ([r][r] after y) and is
+    // written to global memory once at the end
+    double* As = y + r;
     __shared__ double red[kInvThreads / 32];
     __shared__ double s_sc;
     const int64_t b = blockIdx.x;
@@ -191,7 +196,8 @@ __global__ void __launch_bounds__(kInvThreads) inverse_kernel(const double* H, c
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int NW = kInvThreads / 32;
     const double* Hb = H + b * (int64_t)r * r;
-    double* A = Ainv + b * (int64_t)r * r;
+    double* Ag = Ainv + b * (int64_t)r * r;
+    double* A = A_SMEM ? As : Ag;
     for (int a = 0; a < rr; ++a) {
         // b = h(K_S[:a], k_s): row a of H (symmetric)
         for (int j = tid; j < a; j += kInvThreads) bvec[j] = Hb[(int64_t)a * r + j];
@@ -229,6 +235,10 @@ __global__ void __launch_bounds__(kInvThreads) inverse_kernel(const double* H, c
         if (tid == 0) A[(int64_t)a * r + a] = 1.0 / sc;
         __syncthreads();
     }
+    if constexpr (A_SMEM)
+        for (int64_t e = tid; e < (int64_t)rr * r; e += kInvThreads) {
+            if (e % r < rr) Ag[e] = As[e];
+        }
     // Z = sum of the split partials, accumulated into split 0 in split order
     const int DP = D + 1;
     for (int64_t e = tid; e < (int64_t)rr * DP; e += kInvThreads) {
@@ -323,10 +333,14 @@ Status run_inverse(const WeightsInverseRequest& q, cudaStream_t st) {
     if (e != cudaSuccess) return Status::cuda(e, "weights_inverse: z smem attribute");
     z_kernel<E, D><<<dim3((unsigned)ceil_div(r, kZA), p.nsplit_z, (unsigned)q.BH), kZThreads, zsm, st>>>(
         K, V, q.S, q.rank, q.n, r, (double)q.beta, M, p.keys_per_split, q.BH, Zpart);
-    const size_t ism = sizeof(double) * 2 * (size_t)r;
-    e = cudaFuncSetAttribute(inverse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ism);
+    // the inverse in shared memory when it fits (r <= ~160): its r' sequential
+    // updates then never wait on L2
+    const bool a_sm = sizeof(double) * ((size_t)r * r + 2 * (size_t)r) <= kInvSmemCap;
+    const size_t ism = sizeof(double) * (2 * (size_t)r + (a_sm ? (size_t)r * r : 0));
+    auto kern = a_sm ? inverse_kernel<true> : inverse_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ism);
     if (e != cudaSuccess) return Status::cuda(e, "weights_inverse: inverse smem attribute");
-    inverse_kernel<<<(unsigned)q.BH, kInvThreads, ism, st>>>(H, q.rank, r, D, p.nsplit_z, q.BH, Ainv, Zpart);
+    kern<<<(unsigned)q.BH, kInvThreads, ism, st>>>(H, q.rank, r, D, p.nsplit_z, q.BH, Ainv, Zpart);
     xsolve_kernel<D><<<dim3((unsigned)ceil_div(r, kXA), (unsigned)q.BH), kXThreads, 0, st>>>(Ainv, Zpart, q.rank, r,
                                                                                              q.V_S, q.w);
     e = cudaGetLastError();
