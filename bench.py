@@ -123,16 +123,21 @@ def kernel_source_hash(kind=1):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload_name, kind=1):
-    """DRAM bytes per select launch from a committed ncu summary, if it was
-    taken on the current kernel source; else None."""
+def recorded_traffic(workload_name, kind=1, launches=1):
+    """DRAM bytes of one select call (the sum over its launches when it runs
+    in phases) from a committed ncu summary, if it was taken on the current
+    kernel source with the same number of launches; else None."""
     path = os.path.join(ROOT, "profiles", f"{SELECT_KERNELS[kind][1]}_{workload_name}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
-    m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_call = re.search(r"dram_bytes_per_call:\s*([0-9.eE+]+)", text)
+    m_tr = m_call or re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_n = re.search(r"select_launches:\s*([0-9]+)", text)
     if not m_hash or not m_tr or m_hash.group(1) != kernel_source_hash(kind):
+        return None
+    if (int(m_n.group(1)) if m_n else 1) != launches:
         return None
     return float(m_tr.group(1))
 
@@ -401,7 +406,7 @@ def main():
     peak, peak_kind = read_peaks()
     nbytes = select_bytes(w.scaled(n=w.n // nb), ranks)
     achieved = nbytes / (sel_ms / 1e3) / 1e9
-    traffic = recorded_traffic(w0.name if nb == 1 else f"{w0.name}_bins{nb}", sel_kind)
+    traffic = recorded_traffic(w0.name if nb == 1 else f"{w0.name}_bins{nb}", sel_kind, sel_launches)
     out = {
         "metric": METRIC, "value": value, "unit": "calls/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": total_ms / args.steps,
@@ -419,7 +424,8 @@ def main():
         "roofline": {"kernel": SELECT_KERNELS[sel_kind][0], "bound": "hbm", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": f"{peak_kind} hbm_gbs", "traffic": traffic,
-                     "algorithmic_bytes_per_launch": nbytes, "launch_ms": sel_ms},
+                     "algorithmic_bytes_per_launch": nbytes, "launch_ms": sel_ms,
+                     "launches_per_select": sel_launches},
         "gpu_launches": (launches_per_forward(w, sel_launches) + (1 if nb > 1 else 0)) * args.steps,
         "clocks": clk,
         "e2e": e2e,
