@@ -66,7 +66,7 @@ def parse():
     p.add_argument("--weights-inverse", action="store_true",
                    help="also time the inverse-maintenance weights route on the selected pivots")
     p.add_argument("--select-phase-steps", type=int, default=0,
-                   help="select steps per launch (0 = automatic: r / 8 for r >= 512; < 0 = one launch)")
+                   help="select steps per launch (0 = automatic: 64 for r >= 512; < 0 = one launch)")
     p.add_argument("--select-kernel", type=int, choices=[0, 1, 2, 3, 4], default=0,
                    help="0 = automatic (the cp.async kernel), 1 = cp.async, 2 = bulk-copy where it applies")
     return p.parse_args()

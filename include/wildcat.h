@@ -122,10 +122,11 @@ wildcat_status wildcat_select(const void* K, int dtype, int64_t BH, int64_t n, i
  * barrier wait is bounded (2 s, WILDCAT_ERR_TIMEOUT in the device status
  * word on expiry).  Results equal wildcat_select's to float32 rounding.
  * The workspace also enables phases for long coresets (r >= 512, BH at most
- * the SM count): the steps run as launches of about r / 8 steps; between
+ * the SM count): the steps run as launches of 64 steps; between
  * them each instance still going keeps its residual diagonal in the
  * workspace, and the next launch (global sync over the whole GPU) gives each
- * such instance about SMs / (instances still going) CTAs, up to 32.  The
+ * such instance about SMs / (instances still going) CTAs (at least 256 key
+ * rows each, up to 160 CTAs).  The
  * instances whose factor truncated early no longer leave the longest ones on
  * the few CTAs of the first launch.  workspace may be NULL (then exactly
  * wildcat_select).  wildcat_forward* carve this workspace from theirs.
@@ -442,7 +443,7 @@ int wildcat_last_select_threads(void);
 /*
  * wildcat_set_select_phase_steps -- steps per launch of a select call that
  * has a workspace (wildcat_select_ws and the forward calls): 0 (default)
- * automatic, ceil(r / 8) when r >= 512 and a single launch otherwise; > 0
+ * automatic, 64 when r >= 512 and a single launch otherwise; > 0
  * that many steps per launch for any r (the phases apply where the
  * workspace, BH <= SM count and n % 4 == 0 allow them); < 0 always one
  * launch.  Results do not depend on it beyond float32 rounding of the

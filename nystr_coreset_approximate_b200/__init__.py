@@ -517,7 +517,7 @@ def last_select_threads() -> int:
 
 def set_select_phase_steps(steps: int):
     """Steps per select launch when a workspace is given: 0 = automatic
-    (r / 8 for r >= 512), > 0 = that many, < 0 = one launch."""
+    (64 for r >= 512), > 0 = that many, < 0 = one launch."""
     _check(lib().wildcat_set_select_phase_steps(int(steps)))
 
 

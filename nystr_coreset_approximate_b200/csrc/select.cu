@@ -40,7 +40,7 @@ constexpr int kFsByWarp0 = 512;  // factor rows up to this length are gathered b
 constexpr unsigned kTckCols = 128;  // tensor memory columns of the key pass: 8 tiles x 16
 constexpr int kMaxPL = 16;  // R <= 16384 rows per CTA -> at most 16 values per lane
 constexpr size_t kSmemCap = 227 * 1024;
-constexpr int kGsMaxCtas = 32;  // global-sync CTAs per instance: one search lane each
+constexpr int kGsMaxCtas = 160;  // global-sync CTAs per instance (the search gives a lane ceil(G / 32))
 
 struct SelectArgs {
     const void* K;
@@ -253,7 +253,8 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
         if (A <= 0) return;
         int g = (int)(gridDim.x / (unsigned)A);
         g = g < kGsMaxCtas ? g : kGsMaxCtas;
-        const int64_t by_rows = a.n / 512;
+        // at least 256 rows per CTA (late steps stream 4 i bytes per row)
+        const int64_t by_rows = a.n / 256;
         g = (int64_t)g < by_rows ? g : (int)(by_rows > 1 ? by_rows : 1);
         G = g > a.G ? g : a.G;
         const SelectShape sh(a.n, G, NTH, VEC);
@@ -577,7 +578,7 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
         gsync();
         if (warp == 0) {
             float v = -INFINITY;
-            if (lane < G) v = __ldcg(a.gs_mk + b * G + lane);
+            for (int c = lane; c < G; c += 32) v = fmaxf(v, __ldcg(a.gs_mk + b * G + c));
             v = warp_max(v);
             if (lane == 0) misc[1] = v;
         }
@@ -627,7 +628,14 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
                 const int sf = a.S_fixed[b * r + i];
                 s = (sf >= 0 && (int64_t)sf < n) ? sf : -1;
             } else {
-                const double tc = lane < G ? (GS ? __ldcg(ginbox(cur, lane) + 32) : ib[lane * 33 + 32]) : 0.0;
+                // CTA totals, CPL consecutive CTAs per lane (one unless a global-sync
+                // launch has more than 32 CTAs per instance; clusters have at most 16)
+                const int CPL = GS ? (G + 31) >> 5 : 1;
+                auto cta_total = [&](int c) -> double {
+                    return c < G ? (GS ? __ldcg(ginbox(cur, c) + 32) : ib[c * 33 + 32]) : 0.0;
+                };
+                double tc = cta_total(lane * CPL);
+                for (int k = 1; k < CPL; ++k) tc += cta_total(lane * CPL + k);
                 const double incl = warp_scan_incl(tc, lane);
                 const double T = __shfl_sync(0xffffffffu, incl, 31);
                 const unsigned pos_cta = __ballot_sync(0xffffffffu, tc > 0.0);
@@ -635,8 +643,31 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
                     const double t = u_next * T;
                     // owner CTA: first with positive mass whose running total reaches t
                     unsigned m = __ballot_sync(0xffffffffu, tc > 0.0 && incl >= t);
-                    const int owner = m ? __ffs(m) - 1 : 31 - __clz(pos_cta);
-                    const double t1 = t - __shfl_sync(0xffffffffu, incl - tc, owner);
+                    const int ol = m ? __ffs(m) - 1 : 31 - __clz(pos_cta);
+                    double before = __shfl_sync(0xffffffffu, incl - tc, ol);
+                    int owner = ol;
+                    if (CPL > 1) {
+                        // the same running total through lane ol's CTAs (every lane alike)
+                        int hit = -1, last = -1;
+                        double c = before, hit_before = 0.0, last_before = 0.0;
+                        for (int k = 0; k < CPL; ++k) {
+                            const int cc = ol * CPL + k;
+                            const double v = cta_total(cc);
+                            const double prev = c;
+                            c += v;
+                            if (v > 0.0) {
+                                last = cc;
+                                last_before = prev;
+                                if (hit < 0 && c >= t) {
+                                    hit = cc;
+                                    hit_before = prev;
+                                }
+                            }
+                        }
+                        owner = hit >= 0 ? hit : last;
+                        before = hit >= 0 ? hit_before : last_before;
+                    }
+                    const double t1 = t - before;
                     // owner's chunk (its chunk sums are in the local inbox)
                     const double cv =
                         lane < nch ? (GS ? __ldcg(ginbox(cur, owner) + lane) : ib[owner * 33 + lane]) : 0.0;
@@ -1314,7 +1345,7 @@ constexpr double kHalfCtaCost = 1.3;
 // each with about SMs / (instances left) CTAs, so that the longest factors no
 // longer run on the few CTAs the first launch gave them.
 constexpr int kPhaseMinRank = 512;
-constexpr int kPhaseCount = 8;
+constexpr int kPhaseSteps = 64;  // c. 50 us per boundary against the rebalancing it allows
 struct PhasePlan {
     int len = 0;
     int Gmin = 0;
@@ -1326,9 +1357,10 @@ struct PhasePlan {
 static bool plan_phases(const SelectRequest& q, const SelectArgs& a, int vec, int sms, cudaStream_t st,
                         PhasePlan* pp) {
     int len = g_phase_steps;
-    if (len == 0) len = q.r >= kPhaseMinRank ? (int)ceil_div(q.r, kPhaseCount) : 0;
+    if (len == 0) len = q.r >= kPhaseMinRank ? kPhaseSteps : 0;
     if (len <= 0 || len >= q.r || vec != 4 || q.BH > sms) return false;
-    const int Gmin = (int)std::min<int64_t>(kGsMaxCtas, sms / q.BH);
+    // the least G a resumed launch gives an instance: all BH still going
+    const int Gmin = (int)std::min<int64_t>(std::min<int64_t>(32, sms / q.BH), std::max<int64_t>(1, q.n / 256));
     if (ceil_div(q.n, Gmin) > kMaxRowsPerCta) return false;
     SelectArgs ra = a;
     Variant var{};
@@ -1449,7 +1481,7 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
         int Gg = cached_cluster_lookup(gkey);
         if (Gg == 0) {
             Gg = -1;
-            const int cand = (int)std::min<int64_t>(kGsMaxCtas, sms / std::max<int64_t>(1, q.BH));
+            const int cand = (int)std::min<int64_t>(32, sms / std::max<int64_t>(1, q.BH));
             if (cand >= 2 && q.n / cand >= 512 && ceil_div(q.n, cand) <= kMaxRowsPerCta) {
                 SelectArgs t = a;
                 Variant v{};
