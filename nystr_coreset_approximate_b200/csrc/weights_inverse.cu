@@ -20,11 +20,18 @@
 //                    pivot (a matrix-vector product and a rank-one update per
 //                    pivot; the inverse in shared memory when it fits, else in
 //                    global memory), and the sum of Zpart over splits
+//   inverse_cluster_kernel  the same over a cluster of CS CTAs per instance,
+//                    each holding a block of the inverse's rows in shared
+//                    memory (r too large for one CTA, up to about 630)
 //   xsolve_kernel    (V_S, w) = H_S^-1 Z, rounded to float32
+#include <cooperative_groups.h>
+
 #include <algorithm>
 
 #include "common.cuh"
 #include "internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace wildcat {
 
@@ -98,9 +105,13 @@ __global__ void __launch_bounds__(kHT* kHT) hss_kernel(const typename E::T* K, c
     H[(b * r + a) * (int64_t)r + c] = v;
 }
 
-// ---- Z partials: 32 pivots x (D + 1) per CTA, keys of one split in chunks of 64 ----
+// ---- Z partials: 64 pivots x (D + 1) per CTA, keys of one split in chunks of 64 ----
+// Each thread forms a 4 x 4 block of (pivot, key) dot products (eight shared
+// memory loads per sixteen fp64 FMAs), then a 4 pivot x D/16 column block of
+// Z.  Every dot product and every Z entry is summed in key and dimension
+// order, one fma at a time.
 constexpr int kZThreads = 256;
-constexpr int kZA = 32;
+constexpr int kZA = 64;
 constexpr int kZL = 64;
 
 template <int D>
@@ -136,12 +147,17 @@ __global__ void __launch_bounds__(kZThreads) z_kernel(const typename E::T* K, co
         ks[i][c] = a < rr ? (double)E::to_float(K[(b * n + S[b * r + a]) * D + c]) : 0.0;
     }
     const int64_t l_begin = split * keys_per_split, l_end = std::min<int64_t>(n, l_begin + keys_per_split);
-    const int ia = tid / 8, q8 = tid % 8;  // pivot row of this thread; its key / column lane
-    constexpr int CJ = D / 8;
-    double acc[CJ];
+    // pivots tp * 4 + u of this thread; its keys tk + 16 v (dots) and columns tk + 16 j (Z)
+    const int tp = tid >> 4, tk = tid & 15;
+    constexpr int CJ = D / 16;
+    double acc[4][CJ];
+    double accw[4];
 #pragma unroll
-    for (int j = 0; j < CJ; ++j) acc[j] = 0.0;
-    double accw = 0.0;
+    for (int u = 0; u < 4; ++u) {
+        accw[u] = 0.0;
+#pragma unroll
+        for (int j = 0; j < CJ; ++j) acc[u][j] = 0.0;
+    }
     for (int64_t l0 = l_begin; l0 < l_end; l0 += kZL) {
         __syncthreads();  // the previous chunk is consumed (and the pivot keys are staged)
         for (int e = tid; e < kZL * D; e += kZThreads) {
@@ -152,27 +168,57 @@ __global__ void __launch_bounds__(kZThreads) z_kernel(const typename E::T* K, co
             vc[i][c] = ok ? E::to_float(V[(b * n + l) * D + c]) : 0.f;
         }
         __syncthreads();
+        {
+            double dot[4][4];
 #pragma unroll
-        for (int j = 0; j < kZL / 8; ++j) {
-            const int ll = q8 + 8 * j;
-            double dot = 0.0;
-            for (int t = 0; t < D; ++t) dot = fma(ks[ia][t], kc[ll][t], dot);
-            P[ia][ll] = (a0 + ia < rr && l0 + ll < l_end) ? exp(beta * (dot - Mb)) : 0.0;
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) dot[u][v] = 0.0;
+#pragma unroll 4
+            for (int t = 0; t < D; ++t) {
+                double x[4], y[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) x[u] = ks[tp * 4 + u][t];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) y[v] = kc[tk + 16 * v][t];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dot[u][v] = fma(x[u], y[v], dot[u][v]);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const int ia = tp * 4 + u, ll = tk + 16 * v;
+                    P[ia][ll] = (a0 + ia < rr && l0 + ll < l_end) ? exp(beta * (dot[u][v] - Mb)) : 0.0;
+                }
         }
         __syncthreads();
         for (int ll = 0; ll < kZL; ++ll) {
-            const double p = P[ia][ll];
+            double pv[4];
 #pragma unroll
-            for (int j = 0; j < CJ; ++j) acc[j] = fma(p, (double)vc[ll][q8 + 8 * j], acc[j]);
-            accw += p;
+            for (int u = 0; u < 4; ++u) pv[u] = P[tp * 4 + u][ll];
+#pragma unroll
+            for (int j = 0; j < CJ; ++j) {
+                const double v = (double)vc[ll][tk + 16 * j];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc[u][j] = fma(pv[u], v, acc[u][j]);
+            }
+            if (tk == 0)
+#pragma unroll
+                for (int u = 0; u < 4; ++u) accw[u] += pv[u];
         }
     }
-    const int a = a0 + ia;
-    if (a < rr) {
-        double* z = Zpart + (((int64_t)split * BH + b) * r + a) * (D + 1);
 #pragma unroll
-        for (int j = 0; j < CJ; ++j) z[q8 + 8 * j] = acc[j];
-        if (q8 == 0) z[D] = accw;
+    for (int u = 0; u < 4; ++u) {
+        const int a = a0 + tp * 4 + u;
+        if (a < rr) {
+            double* z = Zpart + (((int64_t)split * BH + b) * r + a) * (D + 1);
+#pragma unroll
+            for (int j = 0; j < CJ; ++j) z[tk + 16 * j] = acc[u][j];
+            if (tk == 0) z[D] = accw[u];
+        }
     }
 }
 
@@ -249,6 +295,109 @@ __global__ void __launch_bounds__(kInvThreads) inverse_kernel(const double* H, c
     }
 }
 
+// The bordered inverse over a cluster: CTA c keeps rows [c RB, c RB + RB) of
+// A = H_S^-1 in shared memory.  Step a applies pivot a's update to its rows
+// and, in the same pass over them, forms its rows of y' = A' b' for the next
+// pivot (b' = row a + 1 of H), together with its part of b'.y'.  The rows of
+// y' and the parts go to every CTA of the cluster (distributed shared
+// memory), so after the step's cluster barrier every CTA holds all of y' and
+// forms sc' = h(k_s', k_s') - b'.y' from the parts in CTA order.  y and the
+// parts are double-buffered: a peer writes step a + 1's values only after
+// the barrier that ends this CTA's reads of step a's.
+__global__ void __launch_bounds__(kInvThreads) inverse_cluster_kernel(const double* H, const int32_t* rank, int r,
+                                                                      int RB, int CS, int D, int nsplit, int64_t BH,
+                                                                      double* Ainv, double* Zpart) {
+    extern __shared__ __align__(16) unsigned char sm[];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int c = (int)cluster.block_rank();
+    const int64_t b = blockIdx.x / CS;
+    double* As = reinterpret_cast<double*>(sm);  // [RB][r]
+    double* yb = As + (size_t)RB * r;            // [2][r]
+    double* pd = yb + 2 * (size_t)r;             // [2][CS]
+    __shared__ double red[kInvThreads / 32];
+    constexpr int NW = kInvThreads / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int rr = b < BH ? rank[b] : 0;
+    const double* Hb = H + b * (int64_t)r * r;
+    const int j0 = c * RB;
+    double sc = rr > 0 ? Hb[0] : 1.0;  // pivot 0: y is empty
+    for (int a = 0; a < rr; ++a) {
+        const double* ycur = yb + (size_t)(a & 1) * r;  // y of pivot a (rows < a)
+        double* ynext = yb + (size_t)((a + 1) & 1) * r;
+        double* pnext = pd + (size_t)((a + 1) & 1) * CS;
+        const bool more = a + 1 < rr;
+        const double* bn = Hb + (int64_t)(a + 1) * r;  // read only when more
+        double wpart = 0.0;                             // lane 0: this warp's part of b'.y'
+        for (int jl = warp; jl < RB; jl += NW) {
+            const int j = j0 + jl;
+            if (j > a) break;  // rows past pivot a do not exist yet (warp-uniform)
+            double* Aj = As + (size_t)jl * r;
+            double s = 0.0;
+            if (j < a) {
+                // A <- A + y y^T / sc on row j, then column a = -y_j / sc
+                const double yj = ycur[j] / sc;
+                for (int k = lane; k < a; k += 32) {
+                    const double v = fma(yj, ycur[k], Aj[k]);
+                    Aj[k] = v;
+                    if (more) s = fma(v, bn[k], s);
+                }
+                if (lane == 0) {
+                    const double v = -ycur[j] / sc;
+                    Aj[a] = v;
+                    if (more) s = fma(v, bn[a], s);
+                }
+            } else {
+                // the new row: (-y^T / sc, 1 / sc)
+                for (int k = lane; k < a; k += 32) {
+                    const double v = -ycur[k] / sc;
+                    Aj[k] = v;
+                    if (more) s = fma(v, bn[k], s);
+                }
+                if (lane == 0) {
+                    const double v = 1.0 / sc;
+                    Aj[a] = v;
+                    if (more) s = fma(v, bn[a], s);
+                }
+            }
+            if (more) {
+                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                if (lane < CS) *cluster.map_shared_rank(ynext + j, lane) = s;
+                if (lane == 0) wpart = fma(bn[j], s, wpart);
+            }
+        }
+        if (more) {
+            if (lane == 0) red[warp] = wpart;
+            __syncthreads();
+            if (tid < CS) {
+                double t = 0.0;
+                for (int w = 0; w < NW; ++w) t += red[w];
+                *cluster.map_shared_rank(pnext + c, tid) = t;
+            }
+        }
+        cluster.sync();
+        if (more) {
+            double t = 0.0;
+            for (int q = 0; q < CS; ++q) t += pnext[q];
+            sc = bn[a + 1] - t;
+        }
+    }
+    if (b >= BH) return;
+    double* Ag = Ainv + b * (int64_t)r * r;
+    const int nown = std::max(0, std::min(RB, rr - j0));
+    for (int64_t e = tid; e < (int64_t)nown * r; e += kInvThreads) {
+        const int jl = (int)(e / r), k = (int)(e % r);
+        if (k < rr) Ag[(int64_t)(j0 + jl) * r + k] = As[e];
+    }
+    // Z = sum of the split partials, accumulated into split 0 in split order
+    const int DP = D + 1;
+    for (int64_t e = (int64_t)c * kInvThreads + tid; e < (int64_t)rr * DP; e += (int64_t)CS * kInvThreads) {
+        double* z0 = Zpart + (b * r) * (int64_t)DP + e;
+        double s = *z0;
+        for (int sp = 1; sp < nsplit; ++sp) s += Zpart[((int64_t)sp * BH + b) * r * DP + e];
+        *z0 = s;
+    }
+}
+
 // ---- (V_S, w) = A^-1 Z: 32 rows per CTA ----
 constexpr int kXThreads = 256;
 constexpr int kXA = 32;
@@ -281,6 +430,18 @@ __global__ void __launch_bounds__(kXThreads) xsolve_kernel(const double* Ainv, c
 #pragma unroll
     for (int j = 0; j < CJ; ++j) vs[q8 + 8 * j] = (float)acc[j];
     if (q8 == 0) w[b * r + a] = (float)accw;
+}
+
+// Cluster size for the shared-memory inverse: the least power of two (2..16)
+// whose row blocks fit; 0 when none does.
+size_t inverse_cluster_smem(int r, int CS) {
+    const size_t RB = (size_t)ceil_div(r, CS);
+    return sizeof(double) * (RB * r + 2 * (size_t)r + 2 * (size_t)CS);
+}
+int inverse_cluster_size(int r) {
+    for (int cs = 2; cs <= 16; cs *= 2)
+        if (inverse_cluster_smem(r, cs) <= kInvSmemCap) return cs;
+    return 0;
 }
 
 struct InvPlan {
@@ -333,14 +494,45 @@ Status run_inverse(const WeightsInverseRequest& q, cudaStream_t st) {
     if (e != cudaSuccess) return Status::cuda(e, "weights_inverse: z smem attribute");
     z_kernel<E, D><<<dim3((unsigned)ceil_div(r, kZA), p.nsplit_z, (unsigned)q.BH), kZThreads, zsm, st>>>(
         K, V, q.S, q.rank, q.n, r, (double)q.beta, M, p.keys_per_split, q.BH, Zpart);
-    // the inverse in shared memory when it fits (r <= ~160): its r' sequential
-    // updates then never wait on L2
+    // the inverse in shared memory: one CTA when it fits (r <= ~160), else
+    // spread over a cluster (r <= ~630) while the clusters need at most about
+    // two waves (then its r' sequential updates never wait on L2); else in
+    // global memory, one CTA per instance in one wave.
     const bool a_sm = sizeof(double) * ((size_t)r * r + 2 * (size_t)r) <= kInvSmemCap;
-    const size_t ism = sizeof(double) * (2 * (size_t)r + (a_sm ? (size_t)r * r : 0));
-    auto kern = a_sm ? inverse_kernel<true> : inverse_kernel<false>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ism);
-    if (e != cudaSuccess) return Status::cuda(e, "weights_inverse: inverse smem attribute");
-    kern<<<(unsigned)q.BH, kInvThreads, ism, st>>>(H, q.rank, r, D, p.nsplit_z, q.BH, Ainv, Zpart);
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int CS = a_sm ? 1 : inverse_cluster_size(r);
+    if (CS > 1 && q.BH * CS > 2 * (int64_t)sms) CS = 0;
+    if (CS > 1) {
+        const int RB = (int)ceil_div(r, CS);
+        const size_t csm = inverse_cluster_smem(r, CS);
+        e = cudaFuncSetAttribute(inverse_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csm);
+        if (e == cudaSuccess && CS > 8)
+            e = cudaFuncSetAttribute(inverse_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return Status::cuda(e, "weights_inverse: cluster inverse attributes");
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(q.BH * CS));
+        cfg.blockDim = dim3(kInvThreads);
+        cfg.dynamicSmemBytes = csm;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = CS;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, inverse_cluster_kernel, (const double*)H, q.rank, r, RB, CS, D, p.nsplit_z, q.BH,
+                               Ainv, Zpart);
+        if (e != cudaSuccess) return Status::cuda(e, "weights_inverse: cluster inverse launch");
+    } else {
+        const size_t ism = sizeof(double) * (2 * (size_t)r + (a_sm ? (size_t)r * r : 0));
+        auto kern = a_sm ? inverse_kernel<true> : inverse_kernel<false>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ism);
+        if (e != cudaSuccess) return Status::cuda(e, "weights_inverse: inverse smem attribute");
+        kern<<<(unsigned)q.BH, kInvThreads, ism, st>>>(H, q.rank, r, D, p.nsplit_z, q.BH, Ainv, Zpart);
+    }
     xsolve_kernel<D><<<dim3((unsigned)ceil_div(r, kXA), (unsigned)q.BH), kXThreads, 0, st>>>(Ainv, Zpart, q.rank, r,
                                                                                              q.V_S, q.w);
     e = cudaGetLastError();

@@ -8,6 +8,9 @@ instance (fp64 rounding amplified by the condition number of h(K_S, K_S),
 at most 1 / eps = 1e6 after truncation, then one rounding to float32).
 The value range is bit-exact.  The factor route (float32 on the device)
 must agree with the inverse route where h(K_S, K_S) is well conditioned.
+The cases cover the inverse held by one CTA (r up to about 160), spread over
+clusters of 2, 4 and 16 CTAs (ragged row blocks and truncation included),
+and held in global memory (r = 700).
 """
 import numpy as np
 import pytest
@@ -26,7 +29,11 @@ CASES = [
     gc.case("inv_bf16_mix", "mixture16", 2, 1568, 1568, 64, 96, "bf16"),
     gc.case("inv_bf16_d128", "iid", 2, 3000, 16, 128, 130, "bf16"),
     gc.case("inv_f32_d32_ragged", "iid", 2, 777, 16, 32, 33, "f32"),
-    gc.case("inv_walk_trunc", "walk", 2, 4096, 16, 128, 300, "bf16"),
+    gc.case("inv_walk_trunc", "walk", 2, 4096, 16, 128, 300, "bf16"),        # clusters of 4, truncated
+    gc.case("inv_cluster2", "iid", 2, 2048, 16, 64, 200, "bf16"),            # clusters of 2
+    gc.case("inv_cluster4_ragged", "iid", 3, 2500, 16, 64, 250, "f32"),      # 63 rows per CTA, last 61
+    gc.case("inv_cluster16", "iid", 2, 4096, 16, 128, 512, "bf16"),          # clusters of 16
+    gc.case("inv_global", "iid", 1, 2048, 16, 64, 700, "bf16"),              # inverse in global memory
 ]
 
 
