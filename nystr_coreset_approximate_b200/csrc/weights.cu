@@ -229,6 +229,7 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* Ypart, 
 // F_S[a, j] x_a from every y_j, j < a, reading row a contiguously.
 constexpr int kTrsmWarps = 16;
 constexpr int kTrsmWarpMaxR = 1024;
+constexpr int kTrsmRegs = kTrsmWarpMaxR / 32;  // y values per lane
 constexpr size_t kTrsmSmemCap = 200 * 1024;
 
 inline bool trsm_fs_in_smem(int r) {
@@ -253,16 +254,37 @@ __global__ void __launch_bounds__(kTrsmWarps * 32) trsm_warp_kernel(const float*
     if constexpr (FS_SMEM) {
         // the CTA sums its 16 columns' partials (coalesced over columns) and stages F_S
         float* Ls = ysm + (size_t)kTrsmWarps * r;
+#pragma unroll 4
         for (int e = threadIdx.x; e < rr * kTrsmWarps; e += kTrsmWarps * 32) {
             const int j = e / kTrsmWarps, c = e % kTrsmWarps;
             float s = 0.f;
-            if (cb0 + c < DP)
-                for (int sp = 0; sp < nsplit; ++sp) s += Ypart[(((int64_t)sp * BH + b) * r + j) * DP + cb0 + c];
+            if (cb0 + c < DP) {
+                const float* src = Ypart + ((int64_t)b * r + j) * DP + cb0 + c;
+                const int64_t stride = BH * (int64_t)r * DP;
+#pragma unroll 8
+                for (int sp = 0; sp < nsplit; ++sp) s += src[sp * stride];
+            }
             ysm[(size_t)c * r + j] = s;
         }
-        for (int e = threadIdx.x; e < rr * r; e += kTrsmWarps * 32) {
-            const int a = e / r, j = e % r;
-            Ls[e] = j <= a ? Lg[e] : 0.f;
+        // F_S rows: 16-byte loads, eight in flight per thread (r % 4 == 0), else scalar
+        if ((r & 3) == 0) {
+            const int q4 = r >> 2;
+#pragma unroll 8
+            for (int e = threadIdx.x; e < rr * q4; e += kTrsmWarps * 32) {
+                const int a = e / q4, j = (e % q4) * 4;
+                float4 v = __ldg(reinterpret_cast<const float4*>(Lg) + e);
+                if (j + 0 > a) v.x = 0.f;
+                if (j + 1 > a) v.y = 0.f;
+                if (j + 2 > a) v.z = 0.f;
+                if (j + 3 > a) v.w = 0.f;
+                reinterpret_cast<float4*>(Ls)[e] = v;
+            }
+        } else {
+#pragma unroll 8
+            for (int e = threadIdx.x; e < rr * r; e += kTrsmWarps * 32) {
+                const int a = e / r, j = e % r;
+                Ls[e] = j <= a ? Lg[e] : 0.f;
+            }
         }
         __syncthreads();
         Lb = Ls;
@@ -271,21 +293,44 @@ __global__ void __launch_bounds__(kTrsmWarps * 32) trsm_warp_kernel(const float*
         if (col >= DP) return;  // warps are independent from here on
         for (int j = lane; j < rr; j += 32) {
             float s = 0.f;
-            for (int sp = 0; sp < nsplit; ++sp) s += Ypart[(((int64_t)sp * BH + b) * r + j) * DP + col];
+            const float* src = Ypart + ((int64_t)b * r + j) * DP + col;
+            const int64_t stride = BH * (int64_t)r * DP;
+#pragma unroll 8
+            for (int sp = 0; sp < nsplit; ++sp) s += src[sp * stride];
             y[j] = s;
         }
         __syncwarp();
     }
-    for (int a = rr - 1; a >= 0; --a) {
-        const float* La = Lb + (int64_t)a * r;
-        const float xa = y[a] / La[a];
-        __syncwarp();
-        if (lane == 0) y[a] = xa;
-        for (int j = lane; j < a; j += 32) y[j] = fmaf(-La[j], xa, y[j]);
-        __syncwarp();
+    // y in registers: lane l holds y[32 m + l]; pivots bottom up in blocks of
+    // 32 (block mb compile-time, so every register index is static), y_a
+    // broadcast from its lane, the same divide and fmaf per element as a
+    // shared-memory sweep
+    float yr[kTrsmRegs];
+#pragma unroll
+    for (int m = 0; m < kTrsmRegs; ++m) {
+        const int j = 32 * m + lane;
+        yr[m] = j < rr ? y[j] : 0.f;
     }
-    for (int j = lane; j < r; j += 32) {
-        const float v = j < rr ? y[j] : 0.f;
+#pragma unroll
+    for (int mb = kTrsmRegs - 1; mb >= 0; --mb) {
+        if (32 * mb >= rr) continue;
+        const int top = min(31, rr - 1 - 32 * mb);
+        for (int la = top; la >= 0; --la) {
+            const int a = 32 * mb + la;
+            const float* La = Lb + (int64_t)a * r;
+            const float ya = __shfl_sync(0xffffffffu, yr[mb], la);
+            const float xa = ya / La[a];
+#pragma unroll
+            for (int m = 0; m < mb; ++m) yr[m] = fmaf(-La[32 * m + lane], xa, yr[m]);
+            if (lane < la) yr[mb] = fmaf(-La[32 * mb + lane], xa, yr[mb]);
+            if (lane == la) yr[mb] = xa;
+        }
+    }
+#pragma unroll
+    for (int m = 0; m < kTrsmRegs; ++m) {
+        const int j = 32 * m + lane;
+        if (j >= r) break;
+        const float v = j < rr ? yr[m] : 0.f;
         if (col < D)
             V_S[(b * r + j) * (int64_t)D + col] = v;
         else

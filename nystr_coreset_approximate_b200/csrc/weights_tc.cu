@@ -38,7 +38,8 @@ struct WtSmem {
     static constexpr size_t ahi = 0;                                   // 128 x 64 bf16
     static constexpr size_t alo = ahi + 128 * 128;
     static constexpr size_t b = alo + 128 * 128;                       // NB blocks of 64 keys x 128 B
-    static constexpr size_t bar = b + (size_t)NB * kWtKC * 128;
+    static constexpr size_t stage = b + (size_t)NB * kWtKC * 128;      // one pipeline stage
+    static constexpr size_t bar = 2 * stage;                           // two stages, then the barriers
     static constexpr size_t total = bar + 64 + 1024;
     static constexpr unsigned tmem_cols = 256;
 };
@@ -56,13 +57,13 @@ __global__ void __launch_bounds__(kWtThreads)
 
     extern __shared__ unsigned char sm_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
-    const unsigned sAhi = smem_u32(sm + L::ahi), sAlo = smem_u32(sm + L::alo), sB = smem_u32(sm + L::b);
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + L::bar);
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + L::bar);  // one per stage
     unsigned* tmem_slot = reinterpret_cast<unsigned*>(sm + L::bar + 16);
     const int tid = threadIdx.x, warp = tid >> 5;
 
     if (tid == 0) {
         mbar_init(&mbar[0], 1);
+        mbar_init(&mbar[1], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -79,49 +80,37 @@ __global__ void __launch_bounds__(kWtThreads)
 
     const int64_t l_begin = split * keys_per_split;
     const int64_t l_end = min(n, l_begin + keys_per_split);
+    const int nchunks = l_end > l_begin ? (int)ceil_div(l_end - l_begin, kWtKC) : 0;
     const float* Fb = F + b * (int64_t)r * n;
     const __nv_bfloat16* Vb = V + b * n * D;
-    bool ok = true;
-    int chunk = 0;
-    for (int64_t l0 = l_begin; l0 < l_end; l0 += kWtKC, ++chunk) {
-        // -- A: rows j0 + row of F, 32 keys per thread, split into bf16 hi / lo --
-        {
-            const int row = tid >> 1, half = tid & 1;
-            const int j = j0 + row;
-            float v[32];
-            const float* src = Fb + (int64_t)j * n + l0 + half * 32;
-            const bool full = j < r && l0 + half * 32 + 32 <= l_end;
-            if (full) {
+    const int row = tid >> 1, half = tid & 1;  // A: factor row j0 + row, 32 keys from half * 32
+    const int j = j0 + row;
+
+    // F rows of chunk c into registers (global loads left in flight)
+    auto load_a = [&](int c, float (&v)[32]) {
+        const int64_t l0 = l_begin + (int64_t)c * kWtKC;
+        const float* src = Fb + (int64_t)j * n + l0 + half * 32;
+        const bool full = j < r && l0 + half * 32 + 32 <= l_end;
+        if (full) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float4 x = __ldcs(reinterpret_cast<const float4*>(src) + k);
-                    v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const int64_t l = l0 + half * 32 + k;
-                    v[k] = (j < r && l < l_end) ? __ldcs(Fb + (int64_t)j * n + l) : 0.f;
-                }
+            for (int k = 0; k < 8; ++k) {
+                const float4 x = __ldcs(reinterpret_cast<const float4*>(src) + k);
+                v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
             }
+        } else {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float a0 = v[8 * c + 2 * e], a1 = v[8 * c + 2 * e + 1];
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
-                    const float2 hf = __bfloat1622float2(h);
-                    const __nv_bfloat162 g = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
-                    hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-                    lo[e] = *reinterpret_cast<const uint32_t*>(&g);
-                }
-                const unsigned off = swz(row, half * 4 + c);
-                *reinterpret_cast<uint4*>(sm + L::ahi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4*>(sm + L::alo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            for (int k = 0; k < 32; ++k) {
+                const int64_t l = l0 + half * 32 + k;
+                v[k] = (j < r && l < l_end) ? __ldcs(Fb + (int64_t)j * n + l) : 0.f;
             }
         }
-        // -- B: V rows (MN-major: key = row, 64 value columns per 128-byte row), ones, zeros --
+    };
+    // B of chunk c into stage st: V rows (MN-major: key = row, 64 value
+    // columns per 128-byte row) by cp.async, then the ones column and zeros
+    auto load_b = [&](int c, int st) {
+        const int64_t l0 = l_begin + (int64_t)c * kWtKC;
+        unsigned char* sb = sm + st * L::stage + L::b;
+        const unsigned sB = smem_u32(sb);
         for (int e = tid; e < kWtKC * (D / 8); e += kWtThreads) {
             const int kr = e / (D / 8), c8 = e % (D / 8);  // key row, 16-byte chunk along d
             const int64_t l = l0 + kr;
@@ -129,60 +118,120 @@ __global__ void __launch_bounds__(kWtThreads)
             const unsigned dst = (c8 >> 3) * (kWtKC * 128) + swz(kr, c8 & 7);
             cp_async16_zfill(sB + dst, Vb + (okl ? l : l0) * D + c8 * 8, okl);
         }
+        cp_async_commit();
         for (int kr = tid; kr < kWtKC; kr += kWtThreads) {
             const bool okl = l0 + kr < l_end;
             const int mb = D / 64;  // block holding columns D .. D + 15 (chunks 0 and 1)
             const __nv_bfloat16 one = __float2bfloat16_rn(okl ? 1.f : 0.f);
             uint4 c0 = make_uint4(0u, 0u, 0u, 0u);
             c0.x = (uint32_t)(*reinterpret_cast<const uint16_t*>(&one));
-            *reinterpret_cast<uint4*>(sm + L::b + mb * (kWtKC * 128) + swz(kr, 0)) = c0;
-            *reinterpret_cast<uint4*>(sm + L::b + mb * (kWtKC * 128) + swz(kr, 1)) = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(sb + mb * (kWtKC * 128) + swz(kr, 0)) = c0;
+            *reinterpret_cast<uint4*>(sb + mb * (kWtKC * 128) + swz(kr, 1)) = make_uint4(0u, 0u, 0u, 0u);
         }
-        cp_async_wait_all();
+    };
+
+    // Two stages: while the tensor cores work on chunk c, the V rows of chunk
+    // c + 1 land by cp.async and the F rows of chunks c + 1 and c + 2 are in
+    // flight into registers (two register sets, the loop unrolled by two).
+    // Stage s is rewritten only after the MMA that read it (chunk c - 1 for
+    // B, chunk c - 2 for A) has committed on mbar[s].
+    bool ok = true;
+    int issued = 0;  // MMA commits so far (commit k arrives on mbar[k & 1], phase k >> 1)
+    auto step = [&](int c, float (&v)[32]) -> bool {
+        const int st = c & 1;
+        if (c >= 1) {
+            // chunk c - 1's MMA has read stage st ^ 1: free it for chunk c + 1
+            const bool w = mbar_wait(&mbar[(c - 1) & 1], ((c - 1) >> 1) & 1);
+            if (__syncthreads_or(!w)) return false;
+            tc_fence_after();
+        }
+        if (c + 1 < nchunks) load_b(c + 1, st ^ 1);
+        // A of chunk c: bf16 hi / lo, K-major, 128-byte swizzle
+        unsigned char* sa = sm + st * L::stage;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float a0 = v[8 * q + 2 * e], a1 = v[8 * q + 2 * e + 1];
+                const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
+                const float2 hf = __bfloat1622float2(h);
+                const __nv_bfloat162 g = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
+                hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+                lo[e] = *reinterpret_cast<const uint32_t*>(&g);
+            }
+            const unsigned off = swz(row, half * 4 + q);
+            *reinterpret_cast<uint4*>(sa + L::ahi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(sa + L::alo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        if (c + 2 < nchunks) load_a(c + 2, v);
+        if (c + 1 < nchunks)
+            cp_async_wait_group<1>();  // chunk c's V rows (chunk c + 1's may still fly)
+        else
+            cp_async_wait_all();
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
         if (tid == 0) {
+            const unsigned sAhi = smem_u32(sa + L::ahi), sAlo = smem_u32(sa + L::alo), sB = smem_u32(sa + L::b);
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
-                const unsigned sa = part ? sAlo : sAhi;
+                const unsigned sap = part ? sAlo : sAhi;
 #pragma unroll
                 for (int kk = 0; kk < kWtKC / 16; ++kk)
-                    mma_bf16(tmem, umma_desc(sa + kk * 32), umma_desc_mn(sB + kk * 16 * 128, kWtKC * 128), idesc,
-                             (chunk > 0 || part > 0 || kk > 0) ? 1 : 0);
+                    mma_bf16(tmem, umma_desc(sap + kk * 32), umma_desc_mn(sB + kk * 16 * 128, kWtKC * 128), idesc,
+                             (c > 0 || part > 0 || kk > 0) ? 1 : 0);
             }
-            mma_commit(&mbar[0]);
+            mma_commit(&mbar[st]);
         }
-        const bool w = mbar_wait(&mbar[0], chunk & 1);
-        if (__syncthreads_or(!w)) { ok = false; break; }
+        ++issued;
+        return true;
+    };
+    float v0[32], v1[32];
+    if (nchunks > 0) {
+        load_b(0, 0);
+        load_a(0, v0);
+        if (nchunks > 1) load_a(1, v1);
+    }
+    for (int c = 0; c < nchunks; c += 2) {
+        if (!step(c, v0)) { ok = false; break; }
+        if (c + 1 < nchunks && !step(c + 1, v1)) { ok = false; break; }
+    }
+    // the last commit covers every MMA issued before it
+    if (issued > 0) {
+        const int k = issued - 1;
+        const bool w = mbar_wait(&mbar[k & 1], (k >> 1) & 1);
+        if (__syncthreads_or(!w)) ok = false;
         tc_fence_after();
     }
-    // -- epilogue: warps 0-3 read their 32 TMEM lanes (= factor columns j0 + row) --
-    if (ok && warp < 4 && chunk > 0) {
-        const int row = warp * 32 + (tid & 31);
-        const int j = j0 + row;
-        float* y = Ypart + (((int64_t)split * BH + b) * r + j) * (D + 1);
+    // -- epilogue: warps 0-3 read their 32 TMEM lanes (= factor columns j0 + lane row) --
+    if (ok && warp < 4 && issued > 0) {
+        const int rowe = warp * 32 + (tid & 31);
+        const int je = j0 + rowe;
+        float* y = Ypart + (((int64_t)split * BH + b) * r + je) * (D + 1);
 #pragma unroll 1
         for (int c0 = 0; c0 < D + 16; c0 += 16) {
-            float v[16];
-            tmem_ld16(tmem + ((unsigned)(warp * 32) << 16) + c0, v);
-            if (j < r) {
+            float vv[16];
+            tmem_ld16(tmem + ((unsigned)(warp * 32) << 16) + c0, vv);
+            if (je < r) {
 #pragma unroll
                 for (int k = 0; k < 16; ++k)
-                    if (c0 + k <= D) y[c0 + k] = v[k];
+                    if (c0 + k <= D) y[c0 + k] = vv[k];
             }
         }
-    } else if (ok && warp < 4 && chunk == 0) {
-        const int j = j0 + warp * 32 + (tid & 31);
-        if (j < r) {
-            float* y = Ypart + (((int64_t)split * BH + b) * r + j) * (D + 1);
+    } else if (ok && warp < 4 && issued == 0) {
+        const int je = j0 + warp * 32 + (tid & 31);
+        if (je < r) {
+            float* y = Ypart + (((int64_t)split * BH + b) * r + je) * (D + 1);
             for (int c = 0; c <= D; ++c) y[c] = 0.f;
         }
     }
     if (!ok) {
         if (tid == 0) atomicExch(&g_weights_status, 5);
-        mbar_wait(&mbar[0], chunk & 1);
+        // bounded wait for the last MMA still in flight before its memory is freed
+        if (issued > 0) mbar_wait(&mbar[(issued - 1) & 1], ((issued - 1) >> 1) & 1);
+        cp_async_wait_all();
     }
     tc_fence_before();
     __syncthreads();
