@@ -99,6 +99,36 @@ def test_cluster_knob_validation(L):
     assert L.wildcat_set_select_cluster(0) == 0
 
 
+def test_select_kernel_and_phase_knobs(L):
+    """The select knobs validate on the host; the per-thread records read 0
+    before any select call."""
+    try:
+        for bad in (-1, 5, 99):
+            assert L.wildcat_set_select_kernel(bad) == 1
+        for k in range(5):
+            assert L.wildcat_set_select_kernel(k) == 0
+        for steps in (-1, 0, 16, 64):
+            assert L.wildcat_set_select_phase_steps(steps) == 0
+        assert L.wildcat_last_select_kernel() == 0
+        assert L.wildcat_last_select_threads() == 0
+        assert L.wildcat_last_select_phases() == 0
+    finally:
+        L.wildcat_set_select_kernel(0)
+        L.wildcat_set_select_phase_steps(0)
+
+
+def test_select_workspace_holds_the_phase_state(L):
+    """The select workspace carries two residual copies per instance for the
+    global-sync exchange and one for a paused phase: at least 3 * 4 * BH * n
+    bytes, and it grows linearly with BH * n."""
+    for BH, n in ((32, 32768), (8, 131072), (1, 1024)):
+        ws = int(L.wildcat_select_workspace_size(BH, n))
+        assert ws >= 3 * 4 * BH * n
+    a = int(L.wildcat_select_workspace_size(8, 16384))
+    b = int(L.wildcat_select_workspace_size(8, 32768))
+    assert 3 * 4 * 8 * 16384 <= b - a <= 4 * 4 * 8 * 16384
+
+
 def test_binding_fails_loudly_without_cuda_tensors():
     import torch
 
