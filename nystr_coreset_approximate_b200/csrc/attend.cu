@@ -62,16 +62,30 @@ __global__ void shift_finalize(const float* part, int nsplit, const typename E::
     const int64_t b = blockIdx.x;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int rr = rank[b];
+    // one pivot row per thread, read as 16-byte pieces that are all in flight
+    // at once (the rows of an instance are contiguous: 16-byte aligned when
+    // D * sizeof(T) is a multiple of 16, which holds for every D here)
+    using T = typename E::T;
+    constexpr int EP = 16 / (int)sizeof(T);  // elements per 16-byte piece
     float kb = 0.f;
-    for (int l = warp; l < rr; l += nw) {
-        const typename E::T* k = K_S + (b * r + l) * D;
+    for (int l = threadIdx.x; l < rr; l += blockDim.x) {
+        const uint4* k4 = reinterpret_cast<const uint4*>(K_S + (b * r + l) * D);
+        uint4 pc[D / EP];
+#pragma unroll
+        for (int c = 0; c < D / EP; ++c) pc[c] = __ldg(k4 + c);
         float s = 0.f;
-        for (int c = lane; c < D; c += 32) {
-            const float v = E::to_float(k[c]);
-            s = fmaf(v, v, s);
+#pragma unroll
+        for (int c = 0; c < D / EP; ++c) {
+            const T* e = reinterpret_cast<const T*>(&pc[c]);
+#pragma unroll
+            for (int q = 0; q < EP; ++q) {
+                const float v = E::to_float(e[q]);
+                s = fmaf(v, v, s);
+            }
         }
-        kb = fmaxf(kb, sqrtf(warp_sum(s)));
+        kb = fmaxf(kb, sqrtf(s));
     }
+    kb = warp_max(kb);
     float qb = 0.f;
     for (int s = lane; s < nsplit; s += 32) qb = fmaxf(qb, part[b * nsplit + s]);
     qb = warp_max(qb);
