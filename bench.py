@@ -299,42 +299,34 @@ def main():
     # ---- timed forward: K steps, own events per step, L2 flushed in between ----
     clocks = ClockSampler(local)
     clocks.start()
+    # each timed forward also records stage markers on its own stream (after the
+    # select's launches, after the weights'), so the stage split and the select
+    # kernel's time come from the timed calls themselves
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    after_sel = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    after_wt = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for ev in after_sel + after_wt:
+        ev.record()  # creates the handle the library records into
+    torch.cuda.synchronize()
     barrier()
     for k in range(args.steps):
         flush.zero_()
+        wc.set_stage_events(after_sel[k], after_wt[k])
         starts[k].record()
         plan.run(Q, K, V, w.beta, w.pivot_seed, EPS)
         ends[k].record()
+    wc.set_stage_events(None, None)
     barrier()
     clk = clocks.stop()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = sharding.max_over_ranks(sum(step_ms), device="cuda")
 
-    # ---- per-stage breakdown through the staged C-ABI calls (same kernels;
-    #      binned: the same calls on the [BH * nbins, n / nbins] view) ----
-    Kv = K.view(w.BH * nb, w.n // nb, w.d)
-    Vv = V.view(w.BH * nb, w.n // nb, w.d)
-    rv = w.r // nb
-    stage_ms = {"select": [], "weights": [], "attend": []}
-    for k in range(args.steps + 2):
-        flush.zero_()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        ev[0].record()
-        S, F, rk, K_S = wc.select(Kv, w.beta, rv, w.pivot_seed, EPS)
-        ev[1].record()
-        V_S, wv, vmin, vmax = wc.weights(F, S, rk, Vv)
-        ev[2].record()
-        if nb == 1:
-            wc.attend(Q, K_S, rk, w.beta, V_S, wv, vmin, vmax)
-        ev[3].record()
-        torch.cuda.synchronize()
-        if k >= 2:
-            stage_ms["select"].append(ev[0].elapsed_time(ev[1]))
-            stage_ms["weights"].append(ev[1].elapsed_time(ev[2]))
-            if nb == 1:
-                stage_ms["attend"].append(ev[2].elapsed_time(ev[3]))
+    # ---- per-stage split of the timed forwards (binned: the attend stage also
+    #      holds the union of the bins' coresets) ----
+    stage_ms = {"select": [s.elapsed_time(e) for s, e in zip(starts, after_sel)],
+                "weights": [s.elapsed_time(e) for s, e in zip(after_sel, after_wt)],
+                "attend": [s.elapsed_time(e) for s, e in zip(after_wt, ends)]}
     inv = None
     if args.weights_inverse and nb == 1:
         # the inverse route (fp64) on the same pivots; ALU-bound by its Z contraction
@@ -343,12 +335,12 @@ def main():
             flush.zero_()
             a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a0.record()
-            wc.weights_inverse(K, S, rk, V, w.beta)
+            wc.weights_inverse(K, plan.S, plan.rank, V, w.beta)
             a1.record()
             torch.cuda.synchronize()
             if k >= 2:
                 inv_ms.append(a0.elapsed_time(a1))
-        rks = rk.cpu().tolist()
+        rks = plan.rank.cpu().tolist()
         zflops = sum(4.0 * rr * w.n * (w.d + 1) for rr in rks)       # dot products + accumulation, fp64
         invflops = sum(4.0 * rr ** 3 / 3.0 + 2.0 * rr * rr * (w.d + 1) for rr in rks)
         ms_inv = statistics.mean(inv_ms)
@@ -357,9 +349,6 @@ def main():
         inv = {"ms": ms_inv, "fp64_flops_per_call": zflops + invflops, "achieved_tflops": ach,
                "peak_tflops": peak64, "frac": ach / peak64, "bound": "alu",
                "peak_source": "fp64 unit count: 148 SMs x 64 FMA/clk x 2 x 1.965 GHz"}
-    del S, F, rk, K_S, V_S, wv, vmin, vmax
-    if not stage_ms["attend"]:
-        del stage_ms["attend"]
     sel_ms = statistics.mean(stage_ms["select"])
 
     # ---- end to end through wildcat_forward_host (host buffers) ----

@@ -456,6 +456,21 @@ wildcat_status wildcat_set_select_phase_steps(int steps);
 int wildcat_last_select_phases(void);
 
 /*
+ * wildcat_set_stage_events -- optional stage markers for timing the stages of
+ * a forward: every later wildcat_forward, wildcat_forward_ex,
+ * wildcat_forward_binned or wildcat_forward_host call on this thread records
+ * `after_select` on its stream right after the select's launches and
+ * `after_weights` right after the weights' launches, so that the caller can
+ * split one timed call into select, weights and attend with
+ * cudaEventElapsedTime.  Both are cudaEvent_t handles passed as void*,
+ * created and owned by the caller, and must stay valid while calls record
+ * them; NULL turns a marker off (the default).  Thread-local.  A failed
+ * record is reported as WILDCAT_ERR_CUDA by the forward call.  Always
+ * returns WILDCAT_OK.
+ */
+wildcat_status wildcat_set_stage_events(void* after_select, void* after_weights);
+
+/*
  * wildcat_set_select_cluster -- tuning knob for wildcat_select*: number of
  * CTAs (a thread-block cluster, 1..16, power of two) that share one
  * instance.  0 restores the automatic choice: the G with the least

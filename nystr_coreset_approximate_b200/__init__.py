@@ -27,6 +27,7 @@ __all__ = [
     "weights", "weights_inverse", "attend", "attend_noalloc", "decode_attend", "forward", "forward_ex", "Options", "forward_binned", "BinnedForwardPlan", "forward_host", "ForwardPlan", "pivot_uniforms",
     "set_select_cluster", "last_select_cluster", "set_select_kernel", "last_select_kernel",
     "force_select_timeout", "last_select_threads", "set_select_phase_steps", "last_select_phases",
+    "set_stage_events",
     "device_status", "DTYPES",
 ]
 
@@ -90,6 +91,7 @@ _SIGS = {
     "wildcat_last_select_threads": ([], _int),
     "wildcat_set_select_phase_steps": ([_int], _int),
     "wildcat_last_select_phases": ([], _int),
+    "wildcat_set_stage_events": ([_vp, _vp], _int),
 }
 
 
@@ -524,6 +526,21 @@ def set_select_phase_steps(steps: int):
 def last_select_phases() -> int:
     """Launches of the last select call (1 = no phases)."""
     return int(lib().wildcat_last_select_phases())
+
+
+def set_stage_events(after_select=None, after_weights=None):
+    """Stage markers for the forward calls on this thread: torch.cuda.Event
+    objects (each recorded once already, so that its handle exists) that a
+    forward records right after its select and right after its weights;
+    None turns a marker off."""
+    def handle(ev):
+        if ev is None:
+            return None
+        h = int(ev.cuda_event)
+        if h == 0:
+            raise ValueError("record the event once before passing it (its handle is created lazily)")
+        return h
+    _check(lib().wildcat_set_stage_events(handle(after_select), handle(after_weights)))
 
 
 def force_select_timeout(nanoseconds: int):

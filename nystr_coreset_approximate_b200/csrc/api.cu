@@ -113,6 +113,16 @@ ForwardLayout carve_forward(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, 
     return L;
 }
 
+// Stage markers (wildcat_set_stage_events): caller-owned events recorded on
+// a forward's stream right after its select and right after its weights.
+thread_local cudaEvent_t g_ev_after_select = nullptr;
+thread_local cudaEvent_t g_ev_after_weights = nullptr;
+static Status mark_stage(cudaEvent_t ev, cudaStream_t st, const char* what) {
+    if (!ev) return Status::ok();
+    const cudaError_t e = cudaEventRecord(ev, st);
+    return e == cudaSuccess ? Status::ok() : Status::cuda(e, what);
+}
+
 // wait_v / wait_q (optional): events the weights / attend stage waits for
 // (the host-buffer forward copies V and Q while the select runs).
 wildcat_status forward_impl(const void* Q, const void* K, const void* V, int dtype, int64_t BH, int64_t m, int64_t n,
@@ -125,10 +135,12 @@ wildcat_status forward_impl(const void* Q, const void* K, const void* V, int dty
     sq.ws = L.sws;
     sq.ws_bytes = L.sws_bytes;
     if ((s = wildcat::launch_select(sq, st)).code) return record(s);
+    if ((s = mark_stage(g_ev_after_select, st, "forward: stage event")).code) return record(s);
     if (wait_v && (ew = cudaStreamWaitEvent(st, wait_v, 0))) return record(Status::cuda(ew, "forward: wait for V"));
     wildcat::WeightsRequest wq{L.F, L.S, L.rank, V, dtype, BH, n, d, r, L.V_S, L.w, L.vmin, L.vmax, L.wws,
                                L.wws_bytes};
     if ((s = wildcat::launch_weights(wq, st)).code) return record(s);
+    if ((s = mark_stage(g_ev_after_weights, st, "forward: stage event")).code) return record(s);
     if (wait_q && (ew = cudaStreamWaitEvent(st, wait_q, 0))) return record(Status::cuda(ew, "forward: wait for Q"));
     if (m > 0) {
         wildcat::AttendRequest aq{Q,   L.K_S,  dtype, BH, m, d, r, L.rank, beta, L.V_S, L.w,
@@ -467,9 +479,11 @@ wildcat_status wildcat_forward_ex(const void* Q, const void* K, const void* V, i
     sq.ws = L.sws;
     sq.ws_bytes = L.sws_bytes;
     if ((z = wildcat::launch_select(sq, s)).code) return record(z);
+    if ((z = mark_stage(g_ev_after_select, s, "forward: stage event")).code) return record(z);
     wildcat::WeightsRequest wq{L.F, L.S, L.rank_b, V, dtype, BB, nb, d, rb, L.V_S, L.w, L.vmin_b, L.vmax_b, L.wws,
                                L.wws_bytes};
     if ((z = wildcat::launch_weights(wq, s)).code) return record(z);
+    if ((z = mark_stage(g_ev_after_weights, s, "forward: stage event")).code) return record(z);
     if ((z = wildcat::launch_binning_finish(L.vmin_b, L.vmax_b, L.S, L.rank_b, BH, nbins, nb, rb, d, L.vmin, L.vmax,
                                             L.rank_att, S_out, rank_out, s)).code)
         return record(z);
@@ -618,6 +632,12 @@ wildcat_status wildcat_set_select_phase_steps(int steps) {
 }
 
 int wildcat_last_select_phases(void) { return wildcat::last_select_phases(); }
+
+wildcat_status wildcat_set_stage_events(void* after_select, void* after_weights) {
+    g_ev_after_select = static_cast<cudaEvent_t>(after_select);
+    g_ev_after_weights = static_cast<cudaEvent_t>(after_weights);
+    return record(Status::ok());
+}
 
 wildcat_status wildcat_set_select_cluster(int ctas_per_instance) {
     const int G = ctas_per_instance;

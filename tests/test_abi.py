@@ -112,6 +112,7 @@ def test_select_kernel_and_phase_knobs(L):
         assert L.wildcat_last_select_kernel() == 0
         assert L.wildcat_last_select_threads() == 0
         assert L.wildcat_last_select_phases() == 0
+        assert L.wildcat_set_stage_events(None, None) == 0
     finally:
         L.wildcat_set_select_kernel(0)
         L.wildcat_set_select_phase_steps(0)
