@@ -48,11 +48,14 @@ constexpr int kTcThreads = 256;  // two threads per query row: each takes half o
 unsigned long long g_force_timeout_ns = 0;  // test hook, 0 = off
 constexpr int kTcRC = 64;  // coreset rows per chunk
 
-template <int D>
+// NS chunk stages: 3 in general; 2 when the coreset has at most two chunks
+// (r <= 128), which the prologue copies at once, so the third stage would
+// never be used and its 28-44 KB would keep a second CTA off the SM.
+template <int D, int NS = 3>
 struct TcSmem {
     static constexpr int NE = D + 16;                           // value columns + w + zero padding
     static constexpr int KB1 = D / 64;                          // 128-byte K blocks of Q / K_S rows
-    static constexpr int NSTAGE = 3;                            // K_S / [V_S|w] chunk stages
+    static constexpr int NSTAGE = NS;                           // K_S / [V_S|w] chunk stages
     static constexpr size_t a1 = 0;                             // Q tile 128 x D
     static constexpr size_t b1_bytes = (size_t)KB1 * kTcRC * 128;  // K_S chunk  RC x D
     static constexpr size_t b2_bytes = (size_t)NE * 128;           // [V_S|w]^T  NE x RC (one 128-byte K block)
@@ -65,14 +68,14 @@ struct TcSmem {
     static constexpr unsigned tmem_cols = (2 * kTcRC + NE) <= 256 ? 256u : 512u;
 };
 
-template <int D>
+template <int D, int NS>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attend_tc_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K_S,
                      const __nv_bfloat16* __restrict__ B2h, const __nv_bfloat16* __restrict__ B2l, int64_t m, int r,
                      int rpad, const int32_t* __restrict__ rank, float beta, const float* __restrict__ vmin,
                      const float* __restrict__ vmax, const float* __restrict__ MQ, float* __restrict__ O,
                      unsigned long long force_timeout_ns) {
-    using L = TcSmem<D>;
+    using L = TcSmem<D, NS>;
     constexpr int NE = L::NE;
     extern __shared__ unsigned char sm_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
@@ -310,6 +313,19 @@ __global__ void b2_prep_kernel(const float* __restrict__ V_S, const float* __res
     B2l[at] = lo;
 }
 
+template <int D, int NS>
+cudaError_t launch_tc_kernel(const AttendRequest& q, const float* MQ, const __nv_bfloat16* B2h,
+                             const __nv_bfloat16* B2l, int rpad, cudaStream_t st) {
+    using L = TcSmem<D, NS>;
+    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<D, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)L::total);
+    if (e != cudaSuccess) return e;
+    attend_tc_kernel<D, NS><<<dim3((unsigned)ceil_div(q.m, 128), (unsigned)q.BH), kTcThreads, L::total, st>>>(
+        static_cast<const __nv_bfloat16*>(q.Q), static_cast<const __nv_bfloat16*>(q.K_S), B2h, B2l, q.m, q.r, rpad,
+        q.rank, q.beta, q.vmin, q.vmax, MQ, q.O, g_force_timeout_ns);
+    return cudaGetLastError();
+}
+
 template <int D>
 Status run_tc(const AttendRequest& q, const float* MQ, void* b2ws, cudaStream_t st) {
     using L = TcSmem<D>;
@@ -318,11 +334,10 @@ Status run_tc(const AttendRequest& q, const float* MQ, void* b2ws, cudaStream_t 
     __nv_bfloat16* B2l = B2h + (size_t)q.BH * L::NE * rpad;
     b2_prep_kernel<D><<<dim3((unsigned)ceil_div(rpad, 128), L::NE, (unsigned)q.BH), 128, 0, st>>>(
         q.V_S, q.w, q.rank, q.r, rpad, B2h, B2l);
-    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::total);
-    if (e != cudaSuccess) return Status::cuda(e, "attend_tc: smem attribute");
-    attend_tc_kernel<D><<<dim3((unsigned)ceil_div(q.m, 128), (unsigned)q.BH), kTcThreads, L::total, st>>>(
-        static_cast<const __nv_bfloat16*>(q.Q), static_cast<const __nv_bfloat16*>(q.K_S), B2h, B2l, q.m, q.r, rpad,
-        q.rank, q.beta, q.vmin, q.vmax, MQ, q.O, g_force_timeout_ns);
+    // ranks never exceed r, so r <= 2 chunks bounds every instance's chunk count
+    cudaError_t e = q.r <= 2 * kTcRC ? launch_tc_kernel<D, 2>(q, MQ, B2h, B2l, rpad, st)
+                                     : launch_tc_kernel<D, 3>(q, MQ, B2h, B2l, rpad, st);
+    if (e != cudaSuccess) return Status::cuda(e, "attend_tc launch");
     e = cudaGetLastError();
     if (e != cudaSuccess) return Status::cuda(e, "attend_tc launch");
     return Status::ok();
