@@ -747,7 +747,11 @@ int oracle_decode_attend(const double* Qn, const double* Kn, const double* Vn, c
                     for (int c = 0; c < d; ++c) N[c] += u * VSb[(int64_t)l * d + c];
                     D += u * w[b * r + l];
                 }
+#if ORACLE_MUTANT == 7 /* planted: a new token does not see itself */
+                for (int64_t j = 0; j < i; ++j) {
+#else
                 for (int64_t j = 0; j <= i; ++j) {
+#endif
                     const double e = exp(beta * dot(q, Kb + j * d, d) - beta * M);
                     for (int c = 0; c < d; ++c) N[c] += e * Vb[j * d + c];
                     D += e;

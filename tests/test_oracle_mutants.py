@@ -1,6 +1,7 @@
 """Mutation check of the pins: each copy of the oracle with one planted
 mistake (dropped term, wrong sign, transposed operand, swapped clip bounds,
-greedy instead of random pivots, a wrong sign in the inverse update) must fail at least one pin.  The mistakes
+greedy instead of random pivots, a wrong sign in the inverse update, a
+decode step whose new token does not see itself) must fail at least one pin.  The mistakes
 are planted in the oracle's C source at compile time, on the CPU."""
 import os
 
@@ -16,6 +17,7 @@ MUTANTS = {
     4: "swaps the clip bounds",
     5: "takes the largest residual instead of a random pivot",
     6: "flips the sign of the rank-one inverse update",
+    7: "drops the diagonal of the causal mask in the decode step",
 }
 
 
