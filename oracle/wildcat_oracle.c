@@ -658,7 +658,12 @@ int oracle_wildcat_forward_binned(const double* Q, const double* K, const double
                         const int32_t sg = S_fixed[b * r + q * rb + a];
                         Sf[a] = (sg >= q * nb && sg < (q + 1) * nb) ? (int32_t)(sg - q * nb) : -1;
                     }
-                const int rr = rpc_one(Kcq, nb, d, beta_key, rb, seed, b * nbins + q, eps, 1,
+#if ORACLE_MUTANT == 8 /* planted: every bin of an instance draws the instance's stream */
+                const int64_t ctr = b;
+#else
+                const int64_t ctr = b * nbins + q;
+#endif
+                const int rr = rpc_one(Kcq, nb, d, beta_key, rb, seed, ctr, eps, 1,
                                        S_fixed ? Sf : NULL, Sb, F, NULL, NULL, dg, g);
                 if (rank_out) rank_out[b * nbins + q] = rr;
                 weights_one(F, Sb, rr, Vq, nb, d, rb, VS + (int64_t)q * rb * d, w + q * rb, Y);
@@ -669,7 +674,11 @@ int oracle_wildcat_forward_binned(const double* Q, const double* K, const double
                         KS[(int64_t)row * d + c] = a < rr ? Kq[(int64_t)Sb[a] * d + c] : 0.0;
                 }
             }
+#if ORACLE_MUTANT == 9 /* planted: the value range of the first bin only */
+            oracle_value_range(Vb, 1, nb, d, vmin, vmax);
+#else
             oracle_value_range(Vb, 1, n, d, vmin, vmax);
+#endif
             const double MQ = query_shift(Q + b * m * d, m, KS, r, d);
             for (int64_t ii = 0; ii < nr; ++ii) {
                 const int64_t i = rows ? rows[ii] : ii;

@@ -357,6 +357,38 @@ def pin_binning_closed_forms(o):
         assert len(set(valid.tolist())) == len(valid)
 
 
+def pin_binning_composes_unbinned_parts(o):
+    """Binning as a second derivation from the unbinned primitives (Sec. 2,
+    divide and conquer): select and weights on the [BH * nbins, n / nbins]
+    view of K and V (bin q of instance b is instance b * nbins + q, which is
+    also its Philox counter word), the union coreset puts the bins' pivot
+    rows and weights side by side (zero rows past a bin's rank), and the
+    attend over it clips to the value range of all n values.  The binned
+    forward gives the same pivots, ranks and output.  Bin q's values are
+    offset by 3 q, so the union's estimates mix bins and lie outside any one
+    bin's range (a clip to one bin's range would show)."""
+    Q, K, V = _rand(161, 2, 20, 48, 6)
+    beta, r, nb, seed = 0.4, 16, 4, 7
+    BH, n, d = K.shape
+    rb, nbk = r // nb, n // nb
+    V = V + 3.0 * (np.arange(n) // nbk)[None, :, None]
+    O, S, rank = o.wildcat_forward_binned(Q, K, V, beta, r, nb, seed=seed)
+    Kv, Vv = K.reshape(BH * nb, nbk, d), V.reshape(BH * nb, nbk, d)
+    res = o.rpcholesky(Kv, beta, rb, seed=seed)
+    np.testing.assert_array_equal(rank.reshape(-1), res["rank"])
+    for b in range(BH):
+        for q in range(nb):
+            rr = res["rank"][b * nb + q]
+            np.testing.assert_array_equal(S[b, q * rb:q * rb + rr], q * nbk + res["S"][b * nb + q, :rr])
+            assert np.all(S[b, q * rb + rr:(q + 1) * rb] == -1)
+    VS, w = o.weights(res["F"], res["S"], res["rank"], Vv)
+    KS = o.gather(Kv, res["S"], res["rank"])
+    lo, hi = o.value_range(V)
+    O2 = o.attend(Q, KS.reshape(BH, r, d), VS.reshape(BH, r, d), w.reshape(BH, r),
+                  np.full(BH, r, np.int32), lo, hi, beta)
+    np.testing.assert_allclose(O, O2, rtol=0, atol=1e-12)
+
+
 # --------------------------------------------------------------------------- decode
 def pin_decode_closed_form(o):
     """KV-cache decode: with the cache compressed at full rank (r = n, W a
@@ -464,6 +496,7 @@ ALL_PINS = [
     pin_single_pivot_closed_form,
     pin_hand_examples,
     pin_binning_closed_forms,
+    pin_binning_composes_unbinned_parts,
     pin_decode_closed_form,
     pin_recentring_and_temperature,
 ]

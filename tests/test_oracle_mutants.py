@@ -1,7 +1,8 @@
 """Mutation check of the pins: each copy of the oracle with one planted
 mistake (dropped term, wrong sign, transposed operand, swapped clip bounds,
 greedy instead of random pivots, a wrong sign in the inverse update, a
-decode step whose new token does not see itself) must fail at least one pin.  The mistakes
+decode step whose new token does not see itself, bins that share a pivot
+stream, a binned clip to one bin's range) must fail at least one pin.  The mistakes
 are planted in the oracle's C source at compile time, on the CPU."""
 import os
 
@@ -18,6 +19,8 @@ MUTANTS = {
     5: "takes the largest residual instead of a random pivot",
     6: "flips the sign of the rank-one inverse update",
     7: "drops the diagonal of the causal mask in the decode step",
+    8: "gives every bin of an instance the instance's pivot stream",
+    9: "clips the binned output to the first bin's value range",
 }
 
 
