@@ -615,7 +615,11 @@ int oracle_wildcat_forward_binned(const double* Q, const double* K, const double
      * key kernel exp(beta <x, y> / tau^2) (keys K / tau, queries tau Q); the
      * output step uses the original keys and beta, which differs only by a
      * per-query factor that cancels in N / D. */
+#if ORACLE_MUTANT == 10 /* planted: the temperature applied once instead of squared */
+    const double beta_key = beta / tau;
+#else
     const double beta_key = beta / (tau * tau);
+#endif
     const int64_t nb = n / nbins;
     const int rb = r / nbins;
     const int64_t nr = rows ? nrows : m;
@@ -644,8 +648,13 @@ int oracle_wildcat_forward_binned(const double* Q, const double* K, const double
             for (int c = 0; c < d; ++c) {
                 double mean = 0.0;
                 if (recenter) {
+#if ORACLE_MUTANT == 11 /* planted: the mean of the first bin's keys only */
+                    for (int64_t l = 0; l < nb; ++l) mean += Kb[l * d + c];
+                    mean /= (double)nb;
+#else
                     for (int64_t l = 0; l < n; ++l) mean += Kb[l * d + c];
                     mean /= (double)n;
+#endif
                 }
                 for (int64_t l = 0; l < n; ++l) Kc[l * d + c] = Kb[l * d + c] - mean;
             }

@@ -425,7 +425,9 @@ def pin_recentring_and_temperature(o):
     options change nothing; the pivots with temperature tau are those of the
     plain method on keys K / tau (key kernel exp(beta<x,y>/tau^2)); the
     pivots with recentring are those of the plain method on K - mean(K)
-    (numpy); full-rank bins stay exact attention with both options on."""
+    (numpy), also with several bins, whose keys share the mean of all n keys
+    of their instance; full-rank bins stay exact attention with both options
+    on."""
     Q, K, V = _rand(151, 2, 20, 48, 6, scale=1.2)
     beta = 0.4
     a = o.wildcat_forward_binned(Q, K, V, beta, 16, 2, seed=3)
@@ -439,6 +441,13 @@ def pin_recentring_and_temperature(o):
     _, S_r, _ = o.wildcat_forward_binned(Q, K, V, beta, 16, 1, seed=5, recenter=True)
     _, S_c, _ = o.wildcat_forward(Q, Kc, V, beta, 16, seed=5)
     np.testing.assert_array_equal(S_r, S_c)
+    # bins: the instance's mean, not a bin's (bins drift apart so the means differ)
+    Kd = K + 2.0 * (np.arange(K.shape[1]) // (K.shape[1] // 4))[None, :, None]
+    Kdc = Kd - Kd.mean(axis=1, keepdims=True)
+    _, S_rb, rk_rb = o.wildcat_forward_binned(Q, Kd, V, beta, 16, 4, seed=8, recenter=True)
+    _, S_cb, rk_cb = o.wildcat_forward_binned(Q, Kdc, V, beta, 16, 4, seed=8)
+    np.testing.assert_array_equal(S_rb, S_cb)
+    np.testing.assert_array_equal(rk_rb, rk_cb)
     O, _, rank = o.wildcat_forward_binned(Q, K, V, beta, 48, 4, seed=6, eps=1e-14, recenter=True,
                                           tau=1.3)
     assert np.all(rank == 12)

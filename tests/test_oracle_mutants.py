@@ -2,7 +2,8 @@
 mistake (dropped term, wrong sign, transposed operand, swapped clip bounds,
 greedy instead of random pivots, a wrong sign in the inverse update, a
 decode step whose new token does not see itself, bins that share a pivot
-stream, a binned clip to one bin's range) must fail at least one pin.  The mistakes
+stream, a binned clip to one bin's range, a temperature applied once, a
+recentring mean over one bin) must fail at least one pin.  The mistakes
 are planted in the oracle's C source at compile time, on the CPU."""
 import os
 
@@ -21,6 +22,8 @@ MUTANTS = {
     7: "drops the diagonal of the causal mask in the decode step",
     8: "gives every bin of an instance the instance's pivot stream",
     9: "clips the binned output to the first bin's value range",
+    10: "divides the key kernel's beta by tau instead of tau squared",
+    11: "recentres on the first bin's key mean instead of the instance's",
 }
 
 
