@@ -91,7 +91,11 @@ void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t
 /* Pivot uniform for (seed, step, instance), in (0, 1]. */
 double oracle_pivot_uniform(uint64_t seed, int64_t step, int64_t inst) {
     const uint32_t ctr[4] = {(uint32_t)step, (uint32_t)inst, 0u, 0u};
+#if ORACLE_MUTANT == 14 /* planted: the seed's words swapped in the key */
+    const uint32_t key[2] = {(uint32_t)(seed >> 32), (uint32_t)(seed & 0xffffffffu)};
+#else
     const uint32_t key[2] = {(uint32_t)(seed & 0xffffffffu), (uint32_t)(seed >> 32)};
+#endif
     uint32_t x[4];
     oracle_philox4x32_10(ctr, key, x);
     const uint64_t bits = (((uint64_t)x[1] << 32) | (uint64_t)x[0]) >> 11;
@@ -574,7 +578,19 @@ int oracle_wildcat_forward(const double* Q, const double* K, const double* V, in
             if (rank_out) rank_out[b] = rr;
             weights_one(F, S, rr, Vb, n, d, r, VS, w, Y);
             int32_t rk = rr;
+#if ORACLE_MUTANT == 12 /* planted: the value range of the pivots' rows only */
+            for (int c = 0; c < d; ++c) {
+                vmin[c] = INFINITY;
+                vmax[c] = -INFINITY;
+                for (int a = 0; a < rr; ++a) {
+                    const double v = Vb[(int64_t)S[a] * d + c];
+                    if (v < vmin[c]) vmin[c] = v;
+                    if (v > vmax[c]) vmax[c] = v;
+                }
+            }
+#else
             oracle_value_range(Vb, 1, n, d, vmin, vmax);
+#endif
             oracle_gather(Kb, S, &rk, 1, n, d, r, KS);
             const double MQ = query_shift(Q + b * m * d, m, KS, rr, d);
             for (int64_t ii = 0; ii < nr; ++ii) {
@@ -750,6 +766,9 @@ int oracle_decode_attend(const double* Qn, const double* Kn, const double* Vn, c
             for (int c = 0; c < d; ++c) {
                 lo[c] = vmin[b * d + c];
                 hi[c] = vmax[b * d + c];
+#if ORACLE_MUTANT == 13 /* planted: the range of the cache's values only */
+                continue;
+#endif
                 for (int64_t j = 0; j < m; ++j) {
                     const double v = Vb[j * d + c];
                     if (v < lo[c]) lo[c] = v;

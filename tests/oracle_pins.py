@@ -234,6 +234,20 @@ def pin_philox_matches_library(o):
     assert got == want, (got, want)
 
 
+def pin_uniform_mapping_matches_library(o):
+    """P7a': the pivot uniform of (seed, step, instance) is the triton
+    library's Philox4x32-10 run with that 64-bit seed (the library splits it
+    into the key words itself) on counter (step, instance, 0, 0), its first
+    two words joined high:low and cut to 53 bits, plus one, times 2^-53."""
+    cases = [(0x0123456789ABCDEF, 0, 0), (0x0123456789ABCDEF, 5, 3), (7, 127, 31),
+             (0xFEDCBA9876543210, 1, 2**31 - 1)]
+    ctrs = [(step, inst, 0, 0) for _, step, inst in cases]
+    keys = [(seed & 0xFFFFFFFF, seed >> 32) for seed, _, _ in cases]
+    for (seed, step, inst), x in zip(cases, _triton_philox(ctrs, keys)):
+        bits = ((x[1] << 32) | x[0]) >> 11
+        assert o.pivot_uniform(seed, step, inst) == (bits + 1) * 2.0 ** -53, (seed, step, inst)
+
+
 def pin_uniforms_uniform(o):
     """P7b: the pivot uniforms lie in (0, 1] and pass a Kolmogorov-Smirnov test."""
     u = np.array([o.pivot_uniform(9, i, b) for i in range(400) for b in range(50)])
@@ -497,6 +511,7 @@ ALL_PINS = [
     pin_partial_cholesky_interpolates,
     pin_residual_invariants,
     pin_philox_matches_library,
+    pin_uniform_mapping_matches_library,
     pin_uniforms_uniform,
     pin_first_pivot_law,
     pin_shift_invariance,

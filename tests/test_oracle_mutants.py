@@ -3,7 +3,8 @@ mistake (dropped term, wrong sign, transposed operand, swapped clip bounds,
 greedy instead of random pivots, a wrong sign in the inverse update, a
 decode step whose new token does not see itself, bins that share a pivot
 stream, a binned clip to one bin's range, a temperature applied once, a
-recentring mean over one bin) must fail at least one pin.  The mistakes
+recentring mean over one bin, clips to narrower value ranges, a swapped
+Philox key) must fail at least one pin.  The mistakes
 are planted in the oracle's C source at compile time, on the CPU."""
 import os
 
@@ -24,6 +25,9 @@ MUTANTS = {
     9: "clips the binned output to the first bin's value range",
     10: "divides the key kernel's beta by tau instead of tau squared",
     11: "recentres on the first bin's key mean instead of the instance's",
+    12: "clips to the value range of the pivots' rows instead of all n rows",
+    13: "clips a decode step to the cache's value range, without the new values",
+    14: "swaps the seed's two words in the Philox key",
 }
 
 
