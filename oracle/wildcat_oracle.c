@@ -454,7 +454,11 @@ void oracle_value_range(const double* V, int64_t BH, int64_t n, int d, double* v
     for (int64_t b = 0; b < BH; ++b)
         for (int c = 0; c < d; ++c) {
             double lo = INFINITY, hi = -INFINITY;
+#if ORACLE_MUTANT == 15 /* planted: the last row left out */
+            for (int64_t l = 0; l + 1 < n; ++l) {
+#else
             for (int64_t l = 0; l < n; ++l) {
+#endif
                 const double v = V[(b * n + l) * d + c];
                 if (v < lo) lo = v;
                 if (v > hi) hi = v;

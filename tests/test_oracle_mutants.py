@@ -28,6 +28,7 @@ MUTANTS = {
     12: "clips to the value range of the pivots' rows instead of all n rows",
     13: "clips a decode step to the cache's value range, without the new values",
     14: "swaps the seed's two words in the Philox key",
+    15: "leaves the last value row out of the value range",
 }
 
 
