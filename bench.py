@@ -5,27 +5,34 @@
     python bench.py --impl reference ...      # the fp64 CPU oracle, same metric
 
 One step = one wildcat_forward call over the whole workload (all instances)
-with inputs resident in device memory.  Each step is bracketed by its own
-CUDA events on the launching stream; a 256 MiB device write flushes the L2
-cache between steps, outside the events.  With N > 1 (torchrun, one rank per
-GPU) every rank runs its own copy of the workload (weak scaling; instances
-are independent, so there is no collective on the data path) and the
-reported time is the maximum over ranks.
+with inputs resident in device memory.  The default workload is the largest
+single-GPU one: the long-context sweep at n = m = 131072 (8 heads, d = 128,
+r = 512, bf16).  Each step is bracketed by its own CUDA events on the
+launching stream; a 256 MiB device write flushes the L2 cache between steps,
+outside the events.  With N > 1 (one rank per GPU, started by torchrun or,
+when --gpus N is given without it, by this script re-launching itself under
+torch.distributed.run) every rank runs its own copy of the workload (weak
+scaling; instances are independent, so there is no collective on the data
+path) and the reported time is the maximum over ranks.
 
 Printed (rank 0): one JSON line with the metric, the device-timed value,
 an end-to-end value through wildcat_forward_host (pinned host buffers,
-copies inside the timed region), a per-stage breakdown, the roofline of the
-dominant kernel (the RPCholesky select), sampled SM clocks, and the oracle
-timed on the host cores as a CPU baseline.
+copies inside the timed region), per-stage times with each stage's
+roofline fraction (select and weights against HBM bandwidth, attend against
+the bf16 tensor peak), the forward-level roofline (sum over stages of
+max(bytes / HBM, MMA flops / tensor peak, exps / MUFU rate) against the
+measured step time), the roofline of the dominant kernel, sampled SM clocks,
+and the oracle timed on the host cores as a CPU baseline.  Where the oracle
+cannot afford every query row (m > 4096) it runs select and weights in full
+and the attend on 256 seeded rows per head, and the per-call time is
+extrapolated per row (the line says so).
 """
 from __future__ import annotations
 
 import argparse
-import hashlib
 import json
-import math
 import os
-import re
+import socket
 import statistics
 import subprocess
 import sys
@@ -38,15 +45,10 @@ sys.path.insert(0, ROOT)
 METRIC = "WildCat fwd calls/s & effective m*n attention entries/s on 1 B200; % roofline"
 FLUSH_BYTES = 256 << 20
 EPS = 1e-6
-
-
-def launches_per_forward(w, select_launches=1):
-    """Kernels one wildcat_forward launches: select 1 (or one per phase of a
-    long coreset), weights 5 (range partial and finalize, F^T(V,1),
-    pivot-block gather, solve), attend 3 on CUDA cores (norm partials, shift,
-    attend) or 4 on the tensor-core path (plus the hi/lo split of [V_S|w])."""
-    tc = w.dtype == "bf16" and w.d in (64, 128)
-    return select_launches + 5 + (4 if tc else 3)
+ORACLE_FULL_ROWS_MAX = 4096   # above this m the oracle's attend runs on sampled rows
+ORACLE_SAMPLE_ROWS = 256
+MUFU_EX2_PER_CLK_SM = 16      # exponentials per clock per SM (SFU), nominal
+SM_COUNT = 148
 
 
 def parse():
@@ -55,10 +57,11 @@ def parse():
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["wildcat", "reference"], default="wildcat")
-    p.add_argument("--workload", default="c1_vit56")
+    p.add_argument("--workload", default="c4c_long128k")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline leg")
-    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
+                   help="minimum CPU time of the baseline leg when whole calls are cheap")
     p.add_argument("--nbins", type=int, default=1,
                    help="divide-and-conquer bins (1 = the unbinned method)")
     p.add_argument("--select-cluster", type=int, default=0,
@@ -72,21 +75,47 @@ def parse():
     return p.parse_args()
 
 
+def relaunch_if_needed(args):
+    """--gpus N > 1 outside torchrun: start N ranks under torch.distributed.run
+    (this script again, same arguments) and return their exit status.
+    Inside torchrun the world size must equal --gpus.  Returns None when this
+    process should run the benchmark itself."""
+    world = os.environ.get("WORLD_SIZE")
+    if world is None:
+        if args.gpus <= 1:
+            return None
+        with socket.socket() as s:
+            s.bind(("127.0.0.1", 0))
+            port = s.getsockname()[1]
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+               f"--nproc-per-node={args.gpus}", "--master-addr", "127.0.0.1",
+               "--master-port", str(port), os.path.abspath(__file__)] + sys.argv[1:]
+        return subprocess.call(cmd)
+    if int(world) != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+        return 2
+    return None
+
+
 def workload_config(w, extra=None):
     cfg = {"workload": f"{w.name}: BH={w.BH} (B={w.B}, H={w.H}), n={w.n}, m={w.m}, d={w.d}, "
                        f"r={w.r}, {w.dtype} inputs, {w.dist} keys",
            "BH": w.BH, "n": w.n, "m": w.m, "d": w.d, "r": w.r, "input_dtype": w.dtype,
-           "beta": w.beta, "distribution": w.dist}
+           "accumulate": "f32", "beta": w.beta, "distribution": w.dist}
     if extra:
         cfg.update(extra)
     return cfg
 
 
+def in_bytes(w):
+    return 2 if w.dtype == "bf16" else 4
+
+
 def select_bytes(w, ranks):
-    """Algorithmic bytes of one RPCholesky select launch: per step i the key
-    pass (n d b_K), the factor prefix read (4 n i), the new column write (4 n)
-    and the residual read + write (8 n)."""
-    bk = 2 if w.dtype == "bf16" else 4
+    """Algorithmic bytes of one RPCholesky select: per step i the key pass
+    (n d b_K), the factor prefix read (4 n i), the new column write (4 n) and
+    the residual read + write (8 n)."""
+    bk = in_bytes(w)
     total = 0
     for rr in ranks:
         rr = int(rr)
@@ -94,52 +123,44 @@ def select_bytes(w, ranks):
     return total
 
 
+def weights_bytes(w, ranks):
+    """Algorithmic bytes of the weights stage: the factor's r' rows read once
+    (4 r' n) and V read once (n d b_V)."""
+    return sum(4 * int(rr) * w.n + w.n * w.d * in_bytes(w) for rr in ranks)
+
+
+def attend_work(w, ranks):
+    """(MMA flops, exponentials, HBM bytes) of the attend: GEMM1 Q K_S^T and
+    GEMM2 P V_S at 2 m r' d flops each, m r' exponentials, Q read and the
+    float32 output written."""
+    flops = sum(4.0 * w.m * int(rr) * w.d for rr in ranks)
+    exps = sum(float(w.m) * int(rr) for rr in ranks)
+    nbytes = w.BH * w.m * w.d * (in_bytes(w) + 4)
+    return flops, exps, nbytes
+
+
 def read_peaks():
+    """HBM GB/s and bf16 TFLOP/s (burst, sustained) measured on this machine, else
+    the stated fallback."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "sm_max_mhz": float(p.get("sm_max_mhz", 1965.0)), "source": "measured"}
     except Exception:
-        return 6650.0, "fallback"
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "sm_max_mhz": 1965.0, "source": "fallback"}
 
 
 SELECT_KERNELS = {
-    # last_select_kernel() code -> (kernel name, profile prefix, source files)
-    1: ("rpc_select_kernel", "rpc_select", ("select.cu", "common.cuh", "philox.cuh")),
-    2: ("rpc_select_bulk_kernel", "rpc_select_bulk",
-        ("select_bulk.cu", "common.cuh", "philox.cuh", "tc_common.cuh")),
-    3: ("rpc_select_kernel (global sync)", "rpc_select_gs", ("select.cu", "common.cuh", "philox.cuh")),
-    4: ("rpc_select_kernel (tensor-core key pass)", "rpc_select",
-        ("select.cu", "common.cuh", "philox.cuh", "tc_common.cuh")),
+    # last_select_kernel() code -> kernel name
+    1: "rpc_select_kernel",
+    2: "rpc_select_bulk_kernel",
+    3: "rpc_select_kernel (global sync)",
+    4: "rpc_select_kernel (tensor-core key pass)",
 }
-
-
-def kernel_source_hash(kind=1):
-    h = hashlib.sha256()
-    for name in SELECT_KERNELS[kind][2]:
-        with open(os.path.join(ROOT, "nystr_coreset_approximate_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
-    return h.hexdigest()[:16]
-
-
-def recorded_traffic(workload_name, kind=1, launches=1):
-    """DRAM bytes of one select call (the sum over its launches when it runs
-    in phases) from a committed ncu summary, if it was taken on the current
-    kernel source with the same number of launches; else None."""
-    path = os.path.join(ROOT, "profiles", f"{SELECT_KERNELS[kind][1]}_{workload_name}.md")
-    if not os.path.exists(path):
-        return None
-    text = open(path).read()
-    m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
-    m_call = re.search(r"dram_bytes_per_call:\s*([0-9.eE+]+)", text)
-    m_tr = m_call or re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    m_n = re.search(r"select_launches:\s*([0-9]+)", text)
-    if not m_hash or not m_tr or m_hash.group(1) != kernel_source_hash(kind):
-        return None
-    if (int(m_n.group(1)) if m_n else 1) != launches:
-        return None
-    return float(m_tr.group(1))
 
 
 class ClockSampler:
@@ -193,11 +214,61 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+# ---------------------------------------------------------------------------
+# the fp64 CPU oracle, as it stands (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_rows(w):
+    """Query rows the oracle's attend covers: all of them, or 256 seeded rows
+    per head when m is large."""
+    import workloads
+
+    if w.m <= ORACLE_FULL_ROWS_MAX:
+        return None
+    return workloads.sample_rows(w, ORACLE_SAMPLE_ROWS)
+
+
+def oracle_call(orc, w, ex, rows):
+    """One oracle forward (select, weights, value range, gather, attend) on
+    the whole workload, the attend on `rows` (None = every row).  Returns
+    (seconds for a whole call, detail): select and weights are timed in
+    full; a sampled attend is scaled by m / len(rows) (rows cost the same)."""
+    t0 = time.perf_counter()
+    sel = orc.rpcholesky(ex["K"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
+    t1 = time.perf_counter()
+    VS, wv = orc.weights(sel["F"], sel["S"], sel["rank"], ex["V"])
+    vmin, vmax = orc.value_range(ex["V"])
+    t2 = time.perf_counter()
+    KS = orc.gather(ex["K"], sel["S"], sel["rank"])
+    orc.attend(ex["Q"], KS, VS, wv, sel["rank"], vmin, vmax, w.beta, rows=rows)
+    t3 = time.perf_counter()
+    scale = 1.0 if rows is None else w.m / len(rows)
+    est = (t1 - t0) + (t2 - t1) + (t3 - t2) * scale
+    return est, {"select_s": t1 - t0, "weights_s": t2 - t1, "attend_s": t3 - t2,
+                 "attend_rows": w.m if rows is None else len(rows), "attend_scale": scale}
+
+
+def oracle_sample_text(w, rows, reps=None):
+    if rows is None:
+        return (f"{reps} whole wildcat_forward calls of the workload ({w.BH} instances), fp64, "
+                "OpenMP over instances")
+    return (f"select and weights in full on all {w.BH} instances, attend on {len(rows)} seeded "
+            f"query rows per head scaled by m / {len(rows)} = {w.m / len(rows):g} (per-row "
+            "extrapolation); fp64, OpenMP over instances")
+
+
 def cpu_baseline(w, ex, seconds):
-    """The fp64 oracle, as it stands, on the host cores over the whole workload."""
+    """The fp64 oracle, as it stands, on the host cores: whole calls repeated
+    for `seconds`, or one call with a sampled attend when m is large."""
     import oracle
 
     orc = oracle.get()
+    rows = oracle_rows(w)
+    if rows is not None:
+        est, det = oracle_call(orc, w, ex, rows)
+        return {"value": 1.0 / est, "unit": "calls/s", "cores": orc.num_threads(), "kind": "oracle",
+                "partial": True, "sample": oracle_sample_text(w, rows), "seconds_per_call": est,
+                "detail": det}
     reps, t0 = 0, time.perf_counter()
     while True:
         orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
@@ -206,13 +277,14 @@ def cpu_baseline(w, ex, seconds):
         if el >= seconds:
             break
     return {"value": reps / el, "unit": "calls/s", "cores": orc.num_threads(), "kind": "oracle",
-            "sample": f"{reps} full wildcat_forward calls of the whole workload "
-                      f"({w.BH} instances) in {el:.1f} s, fp64, OpenMP over instances"}
+            "partial": False, "sample": oracle_sample_text(w, None, reps)}
 
 
 def run_reference(args):
-    """Reference arm: the fp64 CPU oracle on the same workload and metric."""
+    """Reference arm: the fp64 CPU oracle on the same workload and metric
+    (rank 0 only; other ranks exit at once)."""
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
     import oracle
@@ -221,32 +293,102 @@ def run_reference(args):
     w = workloads.CONFIGS[args.workload]
     _, ex = workloads.make(w)
     orc = oracle.get()
-    for _ in range(args.warmup):
-        orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
-    times = []
+    rows = oracle_rows(w)
+    for _ in range(max(args.warmup, 3)):
+        if rows is None:
+            orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
+        else:
+            oracle_call(orc, w, ex, rows)
+    secs, det = [], None
     for _ in range(args.steps):
-        t0 = time.perf_counter()
-        orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
-        times.append(time.perf_counter() - t0)
-    total = sum(times)
+        if rows is None:
+            t0 = time.perf_counter()
+            orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
+            secs.append(time.perf_counter() - t0)
+        else:
+            est, det = oracle_call(orc, w, ex, rows)
+            secs.append(est)
+    total = sum(secs)
     value = args.steps / total
+    cpu = {"value": value, "unit": "calls/s", "cores": orc.num_threads(), "kind": "oracle",
+           "partial": rows is not None,
+           "sample": (oracle_sample_text(w, rows) if rows is not None
+                      else f"one whole wildcat_forward call of the workload per step ({w.BH} instances), fp64")}
+    if det is not None:
+        cpu["detail_last_step"] = det
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "calls/s",
-           "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+           "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": workload_config(w, {"l2": "n/a (host)"}),
            "entries_per_s": value * w.BH * w.m * w.n,
-           "cpu_baseline": {"value": value, "unit": "calls/s", "cores": orc.num_threads(),
-                            "kind": "oracle",
-                            "sample": f"the whole workload per step ({w.BH} instances), fp64"},
+           "cpu_baseline": cpu,
            "e2e": {"value": value, "unit": "calls/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
     return 0
 
 
+# ---------------------------------------------------------------------------
+# rooflines
+# ---------------------------------------------------------------------------
+
+def count_library_launches(fn):
+    """Kernels that one call of fn launches (fn calls only this library, so
+    every kernel in the trace is one of its own), from the CUDA activity
+    trace of torch.profiler; copies and memsets are not counted.  None if the
+    profiler is unavailable.  Run outside the timed region."""
+    import torch
+
+    try:
+        from torch.autograd import DeviceType
+        from torch.profiler import ProfilerActivity, profile
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            fn()
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events() if e.device_type == DeviceType.CUDA
+                 and not e.name.startswith(("Memcpy", "Memset"))]
+        return len(names)
+    except Exception:
+        return None
+
+
+def stage_rooflines(w, ranks_sel, ranks_att, stage_ms, peaks, nbins=1):
+    """Per-stage achieved rates, their roofline fractions and the forward-level
+    roofline time.  ranks_sel: effective ranks of the select problems (per bin
+    when binned); ranks_att: coreset size per instance seen by the attend."""
+    wb = w.scaled(n=w.n // nbins) if nbins > 1 else w
+    bw = peaks["hbm_gbs"] * 1e9
+    tc = peaks["bf16_tflops_sustained"] * 1e12
+    mufu = MUFU_EX2_PER_CLK_SM * SM_COUNT * peaks["sm_max_mhz"] * 1e6
+    sb = select_bytes(wb, ranks_sel)
+    wtb = weights_bytes(wb, ranks_sel)
+    af, ae, ab = attend_work(w, ranks_att)
+    ms = {k: statistics.mean(v) for k, v in stage_ms.items()}
+    out = {
+        "select": {"ms": ms["select"], "bytes": sb, "achieved_gbs": sb / (ms["select"] / 1e3) / 1e9,
+                   "bound": "hbm", "frac": sb / (ms["select"] / 1e3) / bw,
+                   "roofline_ms": 1e3 * sb / bw},
+        "weights": {"ms": ms["weights"], "bytes": wtb,
+                    "achieved_gbs": wtb / (ms["weights"] / 1e3) / 1e9, "bound": "hbm",
+                    "frac": wtb / (ms["weights"] / 1e3) / bw, "roofline_ms": 1e3 * wtb / bw},
+        "attend": {"ms": ms["attend"], "mma_flops": af, "exps": ae, "bytes": ab,
+                   "achieved_tflops": af / (ms["attend"] / 1e3) / 1e12, "bound": "tensor",
+                   "frac": af / (ms["attend"] / 1e3) / tc,
+                   "roofline_ms": 1e3 * max(af / tc, ae / mufu, ab / bw),
+                   "limits_ms": {"tensor": 1e3 * af / tc, "mufu": 1e3 * ae / mufu, "hbm": 1e3 * ab / bw}},
+    }
+    total = sum(v["roofline_ms"] for v in out.values())
+    peaks_used = {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops_sustained": peaks["bf16_tflops_sustained"],
+                  "mufu_ex2_per_s": mufu, "source": peaks["source"] + " (MUFU: 16/clk/SM x 148 x max clock)"}
+    return out, total, peaks_used
+
+
 def main():
     args = parse()
+    rc = relaunch_if_needed(args)
+    if rc is not None:
+        return rc
     if args.impl == "reference":
         return run_reference(args)
 
@@ -291,10 +433,12 @@ def main():
         plan.run(Q, K, V, w.beta, w.pivot_seed, EPS)
     torch.cuda.synchronize()
     ranks = plan.rank.reshape(-1).cpu().tolist()  # per instance (per bin when binned)
+    ranks_att = plan.rank.reshape(w.BH, -1).sum(dim=1).cpu().tolist()
     sel_kind = wc.last_select_kernel()
     sel_cluster = wc.last_select_cluster()
     sel_threads = wc.last_select_threads()
     sel_launches = wc.last_select_phases()
+    launches = count_library_launches(lambda: plan.run(Q, K, V, w.beta, w.pivot_seed, EPS))
 
     # ---- timed forward: K steps, own events per step, L2 flushed in between ----
     clocks = ClockSampler(local)
@@ -344,12 +488,11 @@ def main():
         zflops = sum(4.0 * rr * w.n * (w.d + 1) for rr in rks)       # dot products + accumulation, fp64
         invflops = sum(4.0 * rr ** 3 / 3.0 + 2.0 * rr * rr * (w.d + 1) for rr in rks)
         ms_inv = statistics.mean(inv_ms)
-        peak64 = 148 * 64 * 2 * 1.965e9 / 1e12
+        peak64 = SM_COUNT * 64 * 2 * 1.965e9 / 1e12
         ach = (zflops + invflops) / (ms_inv / 1e3) / 1e12
         inv = {"ms": ms_inv, "fp64_flops_per_call": zflops + invflops, "achieved_tflops": ach,
                "peak_tflops": peak64, "frac": ach / peak64, "bound": "alu",
                "peak_source": "fp64 unit count: 148 SMs x 64 FMA/clk x 2 x 1.965 GHz"}
-    sel_ms = statistics.mean(stage_ms["select"])
 
     # ---- end to end through wildcat_forward_host (host buffers) ----
     e2e = None
@@ -374,7 +517,7 @@ def main():
             b.synchronize()
             e_ms.append(a.elapsed_time(b))
         e_tot = sharding.max_over_ranks(sum(e_ms), device="cuda")
-        eb = 2 if w.dtype == "bf16" else 4
+        eb = in_bytes(w)
         e2e = {"value": world * args.steps / (e_tot / 1e3), "unit": "calls/s",
                "h2d_bytes_per_step": eb * w.BH * (w.m + 2 * w.n) * w.d,
                "d2h_bytes_per_step": 4 * w.BH * w.m * w.d + 4 * w.BH * w.r + 4 * w.BH,
@@ -392,30 +535,36 @@ def main():
         return 0
 
     value = world * args.steps / (total_ms / 1e3)
-    peak, peak_kind = read_peaks()
-    nbytes = select_bytes(w.scaled(n=w.n // nb), ranks)
-    achieved = nbytes / (sel_ms / 1e3) / 1e9
-    traffic = recorded_traffic(w0.name if nb == 1 else f"{w0.name}_bins{nb}", sel_kind, sel_launches)
+    peaks = read_peaks()
+    stages, roof_ms, peaks_used = stage_rooflines(w, ranks, ranks_att, stage_ms, peaks, nb)
+    sel = stages["select"]
+    ms_per_step = total_ms / args.steps
     out = {
         "metric": METRIC, "value": value, "unit": "calls/s", "n_gpus": world,
-        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": total_ms / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic",
         "config": workload_config(w0, {"l2": "flushed between steps (256 MiB device write)",
                                        "parallelism": f"instances per rank x {world} ranks",
                                        "nbins": nb,
-                                       "select_kernel": SELECT_KERNELS[sel_kind][0],
+                                       "select_kernel": SELECT_KERNELS.get(sel_kind, str(sel_kind)),
                                        "select_cluster_ctas": sel_cluster,
                                        "select_cta_threads": sel_threads,
                                        "select_launches": sel_launches}),
         "entries_per_s": value * w.BH * w.m * w.n,
-        "stages_ms": {k: statistics.mean(v) for k, v in stage_ms.items()},
-        "roofline": {"kernel": SELECT_KERNELS[sel_kind][0], "bound": "hbm", "achieved": achieved,
-                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_source": f"{peak_kind} hbm_gbs", "traffic": traffic,
-                     "algorithmic_bytes_per_launch": nbytes, "launch_ms": sel_ms,
-                     "launches_per_select": sel_launches},
-        "gpu_launches": (launches_per_forward(w, sel_launches) + (1 if nb > 1 else 0)) * args.steps,
+        "stages_ms": {k: v["ms"] for k, v in stages.items()},
+        "stages": stages,
+        "forward_roofline": {"roofline_ms": roof_ms, "measured_ms": ms_per_step,
+                             "pct": 100.0 * roof_ms / ms_per_step,
+                             "rule": "sum over stages of max(bytes / HBM, MMA flops / bf16 sustained, "
+                                     "exps / MUFU)", "peaks": peaks_used},
+        "roofline": {"kernel": SELECT_KERNELS.get(sel_kind, str(sel_kind)), "bound": "hbm",
+                     "achieved": sel["achieved_gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": sel["frac"], "peak_source": f"{peaks['source']} hbm_gbs",
+                     "traffic": None,
+                     "algorithmic_bytes_per_call": sel["bytes"], "call_ms": sel["ms"],
+                     "launches_per_call": sel_launches},
+        "gpu_launches": None if launches is None else launches * args.steps,
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cpu,
