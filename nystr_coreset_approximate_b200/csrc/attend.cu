@@ -218,11 +218,12 @@ size_t attend_simt_workspace_bytes(int64_t BH, int64_t m) {
     return cv.used + 256;
 }
 
-// Scratch of wildcat_attend: the CUDA-core scratch, then (head dims served by
-// the tensor-core kernel) the bf16 hi/lo copies of [V_S | w]^T.
+// Scratch of wildcat_attend: the larger of the CUDA-core scratch and (head
+// dims served by the tensor-core kernel) the bf16 copy of V_S^T, the padded w
+// and the pivot-key norms.
 size_t attend_workspace_bytes(int64_t BH, int64_t m, int d, int r) {
     size_t bytes = attend_simt_workspace_bytes(BH, m);
-    if (attend_tc_supported(1, d)) bytes += attend_tc_scratch_bytes(BH, d, r) + 256;
+    if (attend_tc_supported(1, d)) bytes = std::max(bytes, attend_tc_scratch_bytes(BH, d, r) + 256);
     return bytes;
 }
 
@@ -236,30 +237,15 @@ Status launch_attend_simt(const AttendRequest& q, cudaStream_t st) {
     return Status::fail(2, "attend: unsupported head dim");
 }
 
-// bf16 inputs with d in {64, 128} run on the tensor cores (attend_tc.cu);
-// everything else on the CUDA-core kernel above.
+// bf16 inputs with d in {64, 128} run on the tensor cores (attend_tc.cu, which
+// shifts each query row by |q_i| * max_l |k_S,l| instead of one M_Q per
+// instance; both cancel in N / D); everything else on the CUDA-core kernel above.
 Status launch_attend(const AttendRequest& q, cudaStream_t st) {
     if (!attend_tc_supported(q.dtype, q.d)) return launch_attend_simt(q, st);
-    const int nsplit = (int)std::max<int64_t>(1, std::min<int64_t>(64, ceil_div(q.m, 1024)));
-    const int64_t rows_per_split = ceil_div(q.m, nsplit);
     Carve cv(q.ws, q.ws_bytes);
-    float* part = static_cast<float*>(cv.take(sizeof(float) * q.BH * nsplit));
-    float* MQ = static_cast<float*>(cv.take(sizeof(float) * q.BH));
-    cv.used = attend_simt_workspace_bytes(q.BH, q.m);
-    void* b2 = cv.take(attend_tc_scratch_bytes(q.BH, q.d, q.r));
+    void* scratch = cv.take(attend_tc_scratch_bytes(q.BH, q.d, q.r));
     if (!cv.fits()) return Status::fail(4, "attend: workspace too small");
-    const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(q.Q);
-    const __nv_bfloat16* KS = static_cast<const __nv_bfloat16*>(q.K_S);
-    if (q.d == 64) {
-        qnorm_partial<BF16, 64><<<dim3(nsplit, (unsigned)q.BH), kNormThreads, 0, st>>>(Q, q.m, rows_per_split, part);
-        shift_finalize<BF16, 64><<<(unsigned)q.BH, 256, 0, st>>>(part, nsplit, KS, q.rank, q.r, MQ);
-    } else {
-        qnorm_partial<BF16, 128><<<dim3(nsplit, (unsigned)q.BH), kNormThreads, 0, st>>>(Q, q.m, rows_per_split, part);
-        shift_finalize<BF16, 128><<<(unsigned)q.BH, 256, 0, st>>>(part, nsplit, KS, q.rank, q.r, MQ);
-    }
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return Status::cuda(e, "attend: shift launch");
-    return launch_attend_tc(q, MQ, b2, st);
+    return launch_attend_tc(q, scratch, st);
 }
 
 // ---------------------------------------------------------------------------

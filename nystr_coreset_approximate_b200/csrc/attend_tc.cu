@@ -2,30 +2,38 @@
 //
 // "WildCat: Near-Linear Attention in Theory and Practice", Sec. 2 plug-in
 // estimator and Alg. 3 WtdAttn, for bfloat16 inputs:
-//     P = exp(beta Q K_S^T - beta M_Q),  N = P V_S,  D = P w,  O = clip(N / D)
-// with one shift M_Q per instance (every exponent <= 0; it cancels in N / D).
+//     P = exp(beta Q K_S^T - beta m),  N = P V_S,  D = P w,  O = clip(N / D)
+// with a shift m_i = |q_i| max_l |k_S,l| per query row: every exponent is
+// <= 0, and the shift cancels in N / D like any per-row constant (the
+// CUDA-core kernel and the oracle use one shift per instance; the ratio is
+// the same).  The row's shift comes from the query tile already in shared
+// memory, so no separate pass over Q is needed.
 //
-// One CTA owns two tiles of 128 queries of one instance and walks the
-// coreset in chunks of 128 rows.  Warp roles (10 warps):
-//   warp 0     producer: TMA loads of the two Q tiles (once), of each K_S
-//              chunk and of each V_S^T chunk plus its slice of w, into
-//              128-byte-swizzled shared memory, ring of NS stages per operand
+// Persistent CTAs (one per SM) walk units of two 128-query tiles of one
+// instance; each unit walks the coreset in chunks of 128 rows.  Warp roles:
+//   warp 0     producer: TMA loads of each unit's two Q tiles (the next
+//              unit's tile as soon as the current one's last GEMM1 is done),
+//              of each K_S chunk and of each V_S^T chunk plus its slice of w,
+//              into 128-byte-swizzled shared memory, NS stages per operand
 //   warp 1     tensor cores (one thread issues):
 //                GEMM1  S_t = Q_t K_S,c^T   tcgen05.mma kind::f16, M = 128,
 //                       N = 128, both operands in shared memory, fp32 in TMEM
 //                GEMM2  O_t += P_t V_S,c    A operand P_t read from TMEM
 //                       (where the softmax threads left it), N = d
 //              in the order G2(c,0) G1(c+1,0) G2(c,1) G1(c+1,1): while one
-//              tile's scores are exponentiated the other tile's products run
+//              tile's scores are exponentiated the other tile's products run;
+//              the next unit's first GEMM1s run during this unit's epilogue
 //   warps 2-5  tile 0, warps 6-9 tile 1: thread i of the group owns query row
 //              i (= TMEM lane i).  Per chunk it reads its 128 scores with
-//              tcgen05.ld, forms P = 2^(s beta log2e - beta M_Q log2e) on the
+//              tcgen05.ld (the next 32 columns in flight while it works on
+//              these), forms P = 2^(s beta log2e - m_i beta log2e) on the
 //              special-function unit, rounds P once to bf16, writes the
 //              packed pairs back over the scores (tcgen05.st) for GEMM2 and
-//              accumulates D = sum_l P_l w_l in fp32 from the same rounded P.
-//              After the last chunk it reads its row of O from TMEM, forms
-//              clip(N / D, v_min, v_max), stages it in the freed Q tile and
-//              stores it with TMA.
+//              accumulates D = sum_l P_l w_l in fp32 (packed fp32x2 FMAs).
+//              After the unit's last chunk it reads its row of O from TMEM
+//              32 columns at a time, forms clip(N / D, v_min, v_max), stages
+//              the 128 x 32 box in its own shared-memory buffer and stores
+//              it with TMA.
 // Tensor memory (512 columns): O_0, O_1 (d columns each), S_0, S_1 (128 each).
 // V_S and w are prepared per call: V_S^T rounded to bf16 (its bf16 rounding
 // leaves the plug-in estimator within 6.1e-4 of the value range on every
@@ -79,16 +87,21 @@ using namespace tc;
 
 constexpr int kRows = 128;    // queries per tile = TMEM lanes
 constexpr int kChunk = 128;   // coreset rows per chunk = N of GEMM1
-constexpr int kWarps = 10;    // producer, tensor cores, two softmax warpgroups
+constexpr int kWarps = 16;    // producer / tensor cores, two softmax groups, one epilogue group
 constexpr int kThreads = kWarps * 32;
+// registers per thread after the split (launched with 65536 / 512 = 128 each):
+// warps 0-3 (producer, tensor cores, two idle) give up some to the softmax
+// and epilogue groups; per sub-partition 88 + 2 * 144 + 136 = 512 = 16384 / 32.
+constexpr int kRegsLow = 88, kRegsSoftmax = 144, kRegsEpilogue = 136;
+static_assert(kRegsLow + 2 * kRegsSoftmax + kRegsEpilogue == 512, "register split");
 constexpr unsigned long long kDrainNs = 100000000ull;  // 100 ms for work in flight after an abort
 unsigned long long g_force_timeout_ns = 0;             // test hook, 0 = off
 
 template <int NS>
 struct Bars {
-    uint64_t q_full[2];
+    uint64_t q_full[2], q_free[2];
     uint64_t k_full[NS], k_empty[NS], v_full[NS], v_empty[NS];
-    uint64_t s_full[2], p_full[2], o_full[2];
+    uint64_t s_full[2], p_full[2], o_full[2], o_free[2], den_full[2];
     uint64_t drain, never;
     unsigned tmem_base;
     int abort;
@@ -98,23 +111,387 @@ template <int D>
 struct Cfg {
     static constexpr int NS = D == 128 ? 2 : 4;          // stages per operand ring
     static constexpr int KB = D / 64;                    // 128-byte blocks per Q / K_S row
-    static constexpr uint32_t q_bytes = kRows * D * 2;   // one Q tile; also half of the fp32 O tile
+    static constexpr uint32_t q_bytes = kRows * D * 2;   // one Q tile
     static constexpr uint32_t k_bytes = kChunk * D * 2;  // one K_S chunk
     static constexpr uint32_t v_bytes = D * kChunk * 2;  // one V_S^T chunk
     static constexpr uint32_t w_bytes = kChunk * 4;      // one chunk of w
+    static constexpr uint32_t o_bytes = kRows * 128;     // one output box: 128 rows x 32 fp32
     static constexpr uint32_t off_q = 0;
     static constexpr uint32_t off_k = off_q + 2 * q_bytes;
     static constexpr uint32_t off_v = off_k + NS * k_bytes;
-    static constexpr uint32_t off_w = off_v + NS * v_bytes;
-    static constexpr uint32_t off_bar = off_w + NS * w_bytes;
-    static constexpr uint32_t total = off_bar + (uint32_t)sizeof(Bars<NS>) + 1024;  // + 1024-byte alignment slack
+    static constexpr uint32_t off_o = off_v + NS * v_bytes;  // the epilogue group's two output boxes
+    static constexpr uint32_t off_w = off_o + 2 * o_bytes;
+    static constexpr uint32_t off_den = off_w + NS * w_bytes;  // row denominators, [2][128]
+    static constexpr uint32_t off_bar = off_den + 2 * kRows * 4;
+    static constexpr uint32_t total = off_bar + (uint32_t)sizeof(Bars<NS>);
     static constexpr unsigned tmem_cols = 512;
     static constexpr unsigned col_O = 0;       // O_t at col_O + t * D
     static constexpr unsigned col_S = 2 * D;   // S_t at col_S + t * kChunk
     static_assert(2 * D + 2 * kChunk <= 512, "tensor memory");
-    static_assert(total <= 227 * 1024, "shared memory");
+    static_assert(total <= 232448, "shared memory");
 };
 
+// The work of one CTA is a sequence of units (two query tiles of one
+// instance): unit u covers queries [256 j, 256 j + 256) of instance u / upi,
+// j = u % upi.  Every role walks the same sequence.  A second tile that lies
+// past m loads zeros and has its stores dropped by the tensor map bounds, so
+// every unit has the same two-tile shape.
+struct Unit {
+    int b, nch;
+    int64_t i0;
+};
+__device__ __forceinline__ Unit unit_at(int64_t u, int64_t upi, int64_t m, const int32_t* rank) {
+    // the host keeps the unit count below 2^31, so 32-bit division suffices
+    Unit w;
+    const uint32_t uu = (uint32_t)u, up = (uint32_t)upi;
+    w.b = (int)(uu / up);
+    w.i0 = (int64_t)(uu - (uint32_t)w.b * up) * (2 * kRows);
+    w.nch = (rank[w.b] + kChunk - 1) / kChunk;
+    return w;
+}
+
+// State shared by the roles of one CTA.
+template <int D>
+struct Ctx {
+    unsigned char* sm;
+    unsigned sbase, tmem;
+    Bars<Cfg<D>::NS>* bars;
+    volatile int* abort_flag;
+    int64_t m, upi, units;
+    const int32_t* rank;
+    __device__ void give_up() const {
+        *abort_flag = 1;
+        atomicExch(&g_device_status, 5);
+    }
+};
+
+template <int D>
+__device__ __forceinline__ void role_producer(const Ctx<D>& x, const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                                              const CUtensorMap* tmV, const float* __restrict__ wpad, int rpad) {
+    using C = Cfg<D>;
+    constexpr int NS = C::NS;
+    auto* bars = x.bars;
+    prefetch_tmap(tmQ);
+    prefetch_tmap(tmK);
+    prefetch_tmap(tmV);
+    int64_t g = 0;       // chunks issued over this CTA's units
+    int qn0 = 0, qn1 = 0;  // Q tiles loaded into slot 0 / 1
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < x.units && ok; u += gridDim.x) {
+        const Unit w = unit_at(u, x.upi, x.m, x.rank);
+        if (w.nch == 0) continue;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            int& qn = t ? qn1 : qn0;
+            // the slot's previous tile: its last GEMM1 done and its row norms read
+            if (qn > 0 && !(ok = mbar_wait_suspend(&bars->q_free[t], (unsigned)(qn - 1) & 1u, x.abort_flag))) break;
+            mbar_expect_tx(&bars->q_full[t], C::q_bytes);
+#pragma unroll
+            for (int kb = 0; kb < C::KB; ++kb)
+                tma_load_3d(x.sbase + C::off_q + t * C::q_bytes + kb * (kRows * 128), tmQ, kb * 64,
+                            (int)(w.i0 + t * kRows), w.b, &bars->q_full[t]);
+            ++qn;
+        }
+        for (int c = 0; c < w.nch && ok; ++c, ++g) {
+            const int s = (int)(g % NS);
+            const unsigned ph = (unsigned)(g / NS) & 1u;
+            if (g >= NS && !(ok = mbar_wait_suspend(&bars->k_empty[s], ph ^ 1u, x.abort_flag))) break;
+            mbar_expect_tx(&bars->k_full[s], C::k_bytes);
+#pragma unroll
+            for (int kb = 0; kb < C::KB; ++kb)
+                tma_load_3d(x.sbase + C::off_k + s * C::k_bytes + kb * (kChunk * 128), tmK, kb * 64, c * kChunk, w.b,
+                            &bars->k_full[s]);
+            if (g >= NS && !(ok = mbar_wait_suspend(&bars->v_empty[s], ph ^ 1u, x.abort_flag))) {
+                ++g;  // this chunk's K copy is in flight
+                break;
+            }
+            mbar_expect_tx(&bars->v_full[s], C::v_bytes + C::w_bytes);
+#pragma unroll
+            for (int j = 0; j < kChunk / 64; ++j)
+                tma_load_3d(x.sbase + C::off_v + s * C::v_bytes + j * (D * 128), tmV, c * kChunk + j * 64, 0, w.b,
+                            &bars->v_full[s]);
+            bulk_load(x.sbase + C::off_w + s * C::w_bytes, wpad + (int64_t)w.b * rpad + (int64_t)c * kChunk,
+                      C::w_bytes, &bars->v_full[s]);
+        }
+    }
+    if (!ok) x.give_up();
+    if (*x.abort_flag) {
+        // copies still in flight land before the CTA's shared memory is released
+        if (qn0 > 0) mbar_wait(&bars->q_full[0], (unsigned)(qn0 - 1) & 1u, kDrainNs);
+        if (qn1 > 0) mbar_wait(&bars->q_full[1], (unsigned)(qn1 - 1) & 1u, kDrainNs);
+        for (int64_t c = g > NS ? g - NS : 0; c < g; ++c) {
+            mbar_wait(&bars->k_full[c % NS], (unsigned)(c / NS) & 1u, kDrainNs);
+            mbar_wait(&bars->v_full[c % NS], (unsigned)(c / NS) & 1u, kDrainNs);
+        }
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void gemm1(const Ctx<D>& x, int64_t g, int t) {  // S_t = Q_t K_g^T
+    using C = Cfg<D>;
+    const unsigned qa = x.sbase + C::off_q + t * C::q_bytes;
+    const unsigned kb = x.sbase + C::off_k + (unsigned)(g % C::NS) * C::k_bytes;
+    const uint64_t da = umma_desc(qa), db = umma_desc(kb);
+    const uint32_t hi = (uint32_t)(da >> 32);  // the same for both operands (layout and swizzle fields)
+    const uint32_t a_lo = (uint32_t)da, b_lo = (uint32_t)db;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        // descriptor start addresses advance in 16-byte units
+        const uint32_t oa = (uint32_t)(((kk >> 2) * (kRows * 128) + (kk & 3) * 32) >> 4);
+        const uint32_t ob = (uint32_t)(((kk >> 2) * (kChunk * 128) + (kk & 3) * 32) >> 4);
+        mma_bf16_w(x.tmem + C::col_S + t * kChunk, a_lo + oa, hi, b_lo + ob, hi, idesc_bf16(128, kChunk), kk > 0);
+    }
+}
+template <int D>
+__device__ __forceinline__ void gemm2(const Ctx<D>& x, int64_t g, int t, bool first) {  // O_t (+)= P_t V_g
+    using C = Cfg<D>;
+    const unsigned vb = x.sbase + C::off_v + (unsigned)(g % C::NS) * C::v_bytes;
+    const uint64_t db = umma_desc(vb);
+    const uint32_t hi = (uint32_t)(db >> 32), b_lo = (uint32_t)db;
+#pragma unroll
+    for (int kk = 0; kk < kChunk / 16; ++kk) {
+        const uint32_t ob = (uint32_t)(((kk >> 2) * (D * 128) + (kk & 3) * 32) >> 4);
+        mma_bf16_ts_w(x.tmem + C::col_O + t * D, x.tmem + C::col_S + t * kChunk + kk * 8, b_lo + ob, hi,
+                      idesc_bf16(128, D), (!first || kk > 0) ? 1 : 0);
+    }
+}
+
+// Position in the CTA's stream of chunks: unit u, its chunk c of nch, the
+// global chunk index g (over all of this CTA's units).
+struct Step {
+    int64_t u, g;
+    int c, nch;
+    Unit w;
+};
+// The chunk after `s`, skipping units of rank 0; false at the end.
+__device__ __forceinline__ bool next_step(Step& s, int64_t units, int64_t upi, int64_t m, const int32_t* rank) {
+    if (s.c + 1 < s.nch) {
+        ++s.c;
+        ++s.g;
+        return true;
+    }
+    for (int64_t u = s.u + gridDim.x; u < units; u += gridDim.x) {
+        const Unit w = unit_at(u, upi, m, rank);
+        if (w.nch == 0) continue;
+        s.u = u;
+        s.w = w;
+        s.c = 0;
+        s.nch = w.nch;
+        ++s.g;
+        return true;
+    }
+    return false;
+}
+
+// GEMM2 of chunk `cur` for tile slot T, then GEMM1 of the slot's next chunk
+// (the next unit's first chunk after a unit's last): each slot runs one
+// continuous stream, so the stagger between the two slots (one exponentiates
+// while the other's products run) carries over unit boundaries.  Returns
+// false when a wait gave up.
+template <int D, int T>
+__device__ __forceinline__ bool mma_slot_step(const Ctx<D>& x, const Step& cur, const Step& nxt, bool has_next,
+                                              int& ct, int& on, int& qn) {
+    using C = Cfg<D>;
+    auto* bars = x.bars;
+    if (!mbar_wait_suspend(&bars->p_full[T], (unsigned)ct & 1u, x.abort_flag)) return false;
+    ct ^= 1;
+    // the epilogue group has taken the slot's previous O out of tensor memory
+    if (cur.c == 0 && on > 0 && !mbar_wait_suspend(&bars->o_free[T], (unsigned)(on - 1) & 1u, x.abort_flag))
+        return false;
+    tc_fence_after();
+    gemm2<D>(x, cur.g, T, cur.c == 0);
+    if (cur.c + 1 == cur.nch) {
+        mma_commit(&bars->o_full[T]);
+        ++on;
+    }
+    if (has_next) {
+        if (T == 0 && !mbar_wait_suspend(&bars->k_full[nxt.g % C::NS], (unsigned)(nxt.g / C::NS) & 1u, x.abort_flag))
+            return false;
+        if (nxt.c == 0) {  // a new unit: its Q tile for this slot
+            if (!mbar_wait_suspend(&bars->q_full[T], (unsigned)qn & 1u, x.abort_flag)) return false;
+            qn ^= 1;
+        }
+        tc_fence_after();
+        // issued after GEMM2 of the same slot, which has read P_t out of these
+        // columns by the time this product writes them (tcgen05.mma executes in
+        // issue order)
+        gemm1<D>(x, nxt.g, T);
+        mma_commit(&bars->s_full[T]);
+        if (nxt.c + 1 == nxt.nch) mma_commit(&bars->q_free[T]);  // the slot's last GEMM1 of that unit
+    }
+    return true;
+}
+
+template <int D>
+__device__ __forceinline__ void role_mma(const Ctx<D>& x) {
+    using C = Cfg<D>;
+    constexpr int NS = C::NS;
+    auto* bars = x.bars;
+    int qn0 = 0, qn1 = 0;  // Q tiles consumed per slot (parity)
+    int ct0 = 0, ct1 = 0;  // chunks of each slot handed to the softmax (parity)
+    int on0 = 0, on1 = 0;  // accumulations of each slot's O
+    Step cur;
+    cur.u = (int64_t)blockIdx.x - gridDim.x;
+    cur.c = 0;
+    cur.nch = 0;
+    cur.g = -1;
+    bool ok = true;
+    if (next_step(cur, x.units, x.upi, x.m, x.rank)) {
+        // the first chunk's GEMM1 for both slots
+        ok = mbar_wait_suspend(&bars->k_full[0], 0, x.abort_flag) &&
+             mbar_wait_suspend(&bars->q_full[0], 0, x.abort_flag) &&
+             mbar_wait_suspend(&bars->q_full[1], 0, x.abort_flag);
+        if (ok) {
+            qn0 = qn1 = 1;
+            tc_fence_after();
+            gemm1<D>(x, 0, 0);
+            mma_commit(&bars->s_full[0]);
+            gemm1<D>(x, 0, 1);
+            mma_commit(&bars->s_full[1]);
+            if (cur.nch == 1) {
+                mma_commit(&bars->q_free[0]);
+                mma_commit(&bars->q_free[1]);
+            }
+            mma_commit(&bars->k_empty[0]);
+        }
+        while (ok) {
+            Step nxt = cur;
+            const bool has_next = next_step(nxt, x.units, x.upi, x.m, x.rank);
+            if (!(ok = mbar_wait_suspend(&bars->v_full[cur.g % NS], (unsigned)(cur.g / NS) & 1u, x.abort_flag)))
+                break;
+            ok = mma_slot_step<D, 0>(x, cur, nxt, has_next, ct0, on0, qn0) &&
+                 mma_slot_step<D, 1>(x, cur, nxt, has_next, ct1, on1, qn1);
+            if (!ok) break;
+            mma_commit(&bars->v_empty[cur.g % NS]);
+            if (!has_next) break;
+            mma_commit(&bars->k_empty[nxt.g % NS]);
+            cur = nxt;
+        }
+    }
+    if (!ok) x.give_up();
+    // every product issued has finished before tensor memory is released
+    mma_commit(&bars->drain);
+    mbar_wait(&bars->drain, 0, kDrainNs);
+}
+
+// Softmax group t (warps 4 + 4t .. 7 + 4t): thread `row` owns query row `row`
+// of tile slot t (TMEM lane `row`).
+template <int D>
+__device__ __forceinline__ void role_softmax(const Ctx<D>& x, int t, int quad, int lane, float beta,
+                                             const float* __restrict__ kmax) {
+    using C = Cfg<D>;
+    constexpr int NS = C::NS;
+    auto* bars = x.bars;
+    const int row = quad * 32 + lane;
+    const unsigned tS = x.tmem + C::col_S + t * kChunk + ((unsigned)(quad * 32) << 16);
+    const float a = beta * 1.4426950408889634f;
+    const unsigned char* qrow = x.sm + C::off_q + t * C::q_bytes + row * 128;
+    float* den_s = reinterpret_cast<float*>(x.sm + C::off_den);
+    int64_t g = 0;
+    int qn = 0, ct = 0, on = 0;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < x.units && ok; u += gridDim.x) {
+        const Unit w = unit_at(u, x.upi, x.m, x.rank);
+        if (w.nch == 0) {
+            g += w.nch;
+            continue;
+        }
+        const int rr = x.rank[w.b];
+        // per-row shift m_i = |q_i| * max_l |k_S,l| (>= <q_i, k_l>; it cancels in N / D)
+        ok = __all_sync(0xffffffffu, mbar_wait_suspend(&bars->q_full[t], (unsigned)qn & 1u, x.abort_flag));
+        if (!ok) break;
+        float qq = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < D / 8; ++cc) {
+            const uint4 q4 =
+                *reinterpret_cast<const uint4*>(qrow + (cc >> 3) * (kRows * 128) + (((cc & 7) ^ (row & 7)) << 4));
+            const uint32_t xs[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float lo = __uint_as_float(xs[e] << 16), hi = __uint_as_float(xs[e] & 0xffff0000u);
+                qq = fmaf(lo, lo, qq);
+                qq = fmaf(hi, hi, qq);
+            }
+        }
+        const float sh = a * sqrtf(qq) * kmax[w.b];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->q_free[t]);
+        qn ^= 1;
+        const float2 a2 = make_float2(a, a), nsh2 = make_float2(-sh, -sh);
+        float2 dacc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        for (int c = 0; c < w.nch && ok; ++c, ++g) {
+            const int s = (int)(g % NS);
+            const bool got = mbar_wait_suspend(&bars->s_full[t], (unsigned)ct & 1u, x.abort_flag) &&
+                             mbar_wait_suspend(&bars->v_full[s], (unsigned)(g / NS) & 1u, x.abort_flag);
+            ok = __all_sync(0xffffffffu, got);  // tcgen05.ld / st below are warp-collective
+            if (!ok) break;
+            ct ^= 1;
+            tc_fence_after();
+            const float4* w4 = reinterpret_cast<const float4*>(x.sm + C::off_w + s * C::w_bytes);
+            const int lim = rr - c * kChunk;  // keys of this chunk below the rank
+            uint32_t v[2][32];
+            tmem_ld32_nowait(tS, v[0]);
+#pragma unroll
+            for (int j = 0; j < kChunk / 32; ++j) {
+                tmem_wait_ld();
+                if (j + 1 < kChunk / 32) tmem_ld32_nowait(tS + 32 * (j + 1), v[(j + 1) & 1]);
+                uint32_t pk[16];
+#pragma unroll
+                for (int e2 = 0; e2 < 8; ++e2) {
+                    const float4 ww = w4[8 * j + e2];
+                    float p[4];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int e = 2 * e2 + h;
+                        const float2 x2 = ffma2(
+                            make_float2(__uint_as_float(v[j & 1][2 * e]), __uint_as_float(v[j & 1][2 * e + 1])), a2,
+                            nsh2);
+                        p[2 * h] = ex2_approx(x2.x);
+                        p[2 * h + 1] = ex2_approx(x2.y);
+                    }
+                    if (lim < kChunk) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) p[q] = 32 * j + 4 * e2 + q < lim ? p[q] : 0.f;
+                    }
+                    pk[2 * e2] = pack_bf16x2(p[0], p[1]);
+                    pk[2 * e2 + 1] = pack_bf16x2(p[2], p[3]);
+                    // denominator in fp32 from the unrounded P (its bf16 rounding in N is
+                    // unbiased, 2^-9 relative, far inside the 2e-2 bound)
+                    dacc[0] = ffma2(make_float2(p[0], p[1]), make_float2(ww.x, ww.y), dacc[0]);
+                    dacc[1] = ffma2(make_float2(p[2], p[3]), make_float2(ww.z, ww.w), dacc[1]);
+                }
+                tmem_st16(tS + 16 * j, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->p_full[t]);
+        }
+        if (!ok) break;
+        // the row's denominator for the epilogue group, once the epilogue has read
+        // the slot's previous one (with one chunk per unit this group can finish a
+        // unit before the epilogue has taken the previous unit's results)
+        if (on > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait_suspend(&bars->o_free[t], (unsigned)(on - 1) & 1u, x.abort_flag));
+            if (!ok) break;
+        }
+        ++on;
+        den_s[t * kRows + row] = (dacc[0].x + dacc[0].y) + (dacc[1].x + dacc[1].y);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->den_full[t]);
+    }
+    if (!ok && lane == 0) x.give_up();
+}
+
+// A read-only 16-byte load kept in program order (volatile), so the compiler
+// does not hoist a whole row's worth of bounds into registers.
+__device__ __forceinline__ float4 ld_nc_f4(const float* p) {
+    float4 r;
+    asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(p));
+    return r;
+}
+
+// AND of `v` over the 128 threads of the epilogue group (a group barrier).
 __device__ __forceinline__ bool group_all(int id, bool v) {
     uint32_t r;
     asm volatile(
@@ -128,34 +505,135 @@ __device__ __forceinline__ bool group_all(int id, bool v) {
     return r != 0;
 }
 
+// One 128 x 32 box of outputs O = clip(v * rcp, lo, hi) from 32 accumulator
+// values per thread, through box `buf` of the epilogue group's two
+// shared-memory boxes to TMA (the store of the other box may still be reading).
+template <int D>
+__device__ __forceinline__ void put_box(const Ctx<D>& x, int row, const uint32_t (&v)[32], int col0, float rcp,
+                                        const float* lo, const float* hi, int64_t y, int b, const CUtensorMap* tmO,
+                                        int buf) {
+    using C = Cfg<D>;
+    unsigned char* brow = x.sm + C::off_o + buf * C::o_bytes + row * 128;
+    if (row == 0) bulk_wait_read_1();  // this box's previous store has read it
+    named_barrier_sync(3, 128);
+    const float* lb = lo + col0;
+    const float* hb = hi + col0;
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+        const float4 l4 = ld_nc_f4(lb + 4 * cc);
+        const float4 h4 = ld_nc_f4(hb + 4 * cc);
+        float4 o;
+        o.x = fminf(fmaxf(__uint_as_float(v[4 * cc + 0]) * rcp, l4.x), h4.x);
+        o.y = fminf(fmaxf(__uint_as_float(v[4 * cc + 1]) * rcp, l4.y), h4.y);
+        o.z = fminf(fmaxf(__uint_as_float(v[4 * cc + 2]) * rcp, l4.z), h4.z);
+        o.w = fminf(fmaxf(__uint_as_float(v[4 * cc + 3]) * rcp, l4.w), h4.w);
+        // volatile like the loads above, so each 16-byte group of bounds is consumed
+        // before the next is fetched (few registers in flight)
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(brow + ((cc ^ (row & 7)) << 4))),
+                     "f"(o.x), "f"(o.y), "f"(o.z), "f"(o.w)
+                     : "memory");
+    }
+    fence_async_smem();
+    named_barrier_sync(3, 128);
+    if (row == 0) {
+        tma_store_3d(tmO, col0, (int)y, b, x.sbase + C::off_o + buf * C::o_bytes);
+        bulk_commit();
+    }
+}
+
+// The epilogue of tile slot T of one unit.  Returns false when a wait gave up.
+template <int D, int T>
+__device__ __forceinline__ bool epilogue_tile(const Ctx<D>& x, const Unit& w, int quad, int lane, int& on,
+                                              const CUtensorMap* tmO, const float* lo, const float* hi) {
+    using C = Cfg<D>;
+    const int row = quad * 32 + lane;
+    const int64_t y = w.i0 + T * kRows;
+    uint32_t v[D / 64][32];
+    if (w.nch == 0) {  // rank 0: 0 / 0 is NaN, which the clip turns into v_min
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[0][e] = 0u;
+#pragma unroll 1
+        for (int col0 = 0; col0 < D; col0 += 32)
+            put_box<D>(x, row, v[0], col0, __int_as_float(0x7f800000), lo, hi, y, w.b, tmO, (col0 >> 5) & 1);
+        return true;
+    }
+    const bool got = mbar_wait_suspend(&x.bars->o_full[T], (unsigned)on & 1u, x.abort_flag) &&
+                     mbar_wait_suspend(&x.bars->den_full[T], (unsigned)on & 1u, x.abort_flag);
+    // all four warps agree before the group barriers of put_box
+    if (!group_all(3, got)) return false;
+    ++on;
+    tc_fence_after();
+    const unsigned tO = x.tmem + C::col_O + T * D + ((unsigned)(quad * 32) << 16);
+    const float rcp = 1.0f / reinterpret_cast<const float*>(x.sm + C::off_den)[T * kRows + row];
+    constexpr int H = D / 2;  // columns per half
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int k = 0; k < H / 32; ++k) tmem_ld32_nowait(tO + h * H + 32 * k, v[k]);
+        tmem_wait_ld();
+        if (h == 1) {
+            // the slot's accumulator and denominator are read: release them (the
+            // slot's next GEMM2 comes after the next chunk's softmax, well later)
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&x.bars->o_free[T]);
+        }
+#pragma unroll
+        for (int k = 0; k < H / 32; ++k)
+            put_box<D>(x, row, v[k], h * H + 32 * k, rcp, lo, hi, y, w.b, tmO, (h * (H / 32) + k) & 1);
+    }
+    return true;
+}
+
+// Epilogue group (warps 12-15): O = clip(N / D) for every tile, in unit order.
+template <int D>
+__device__ __forceinline__ void role_epilogue(const Ctx<D>& x, int quad, int lane, const CUtensorMap* tmO,
+                                              const float* __restrict__ vmin, const float* __restrict__ vmax) {
+    int on0 = 0, on1 = 0;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < x.units && ok; u += gridDim.x) {
+        const Unit w = unit_at(u, x.upi, x.m, x.rank);
+        const float* lo = vmin + (int64_t)w.b * D;
+        const float* hi = vmax + (int64_t)w.b * D;
+        ok = epilogue_tile<D, 0>(x, w, quad, lane, on0, tmO, lo, hi) &&
+             epilogue_tile<D, 1>(x, w, quad, lane, on1, tmO, lo, hi);
+    }
+    if (!ok && lane == 0) x.give_up();
+    if (quad == 0 && lane == 0) bulk_wait_all();
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                     const float* __restrict__ wpad, int rpad, int64_t m, const int32_t* __restrict__ rank,
-                     float beta, const float* __restrict__ vmin, const float* __restrict__ vmax,
-                     const float* __restrict__ MQ, unsigned long long force_timeout_ns) {
+                     const float* __restrict__ wpad, int rpad, int64_t m, int64_t BH,
+                     const int32_t* __restrict__ rank, float beta, const float* __restrict__ vmin,
+                     const float* __restrict__ vmax, const float* __restrict__ kmax,
+                     unsigned long long force_timeout_ns) {
     using C = Cfg<D>;
     constexpr int NS = C::NS;
-    extern __shared__ unsigned char sm_raw[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
-    const unsigned sbase = smem_u32(sm);
-    Bars<NS>* bars = reinterpret_cast<Bars<NS>*>(sm + C::off_bar);
-    volatile int* abort_flag = &bars->abort;
-
+    extern __shared__ __align__(1024) unsigned char sm[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int b = blockIdx.y;
-    const int64_t i0 = (int64_t)blockIdx.x * (2 * kRows);
-    const int ntiles = (m - i0) > kRows ? 2 : 1;
-    const int rr = rank[b];
-    const int nch = (rr + kChunk - 1) / kChunk;
+    Ctx<D> x;
+    x.sm = sm;
+    x.sbase = smem_u32(sm);
+    x.bars = reinterpret_cast<Bars<NS>*>(sm + C::off_bar);
+    x.abort_flag = &x.bars->abort;
+    x.m = m;
+    x.upi = (m + 2 * kRows - 1) / (2 * kRows);  // units per instance
+    x.units = x.upi * BH;
+    x.rank = rank;
+    auto* bars = x.bars;
 
     if (tid == 0) {
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bars->q_full[t], 1);
+            mbar_init(&bars->q_free[t], 1 + 4);  // the tile's last GEMM1 + the softmax group's four warps
             mbar_init(&bars->s_full[t], 1);
-            mbar_init(&bars->p_full[t], 4);  // one arrival per warp of the softmax group
+            mbar_init(&bars->p_full[t], 4);      // one arrival per warp of the softmax group
             mbar_init(&bars->o_full[t], 1);
+            mbar_init(&bars->o_free[t], 4);      // one arrival per warp of the epilogue group
+            mbar_init(&bars->den_full[t], 4);    // one arrival per warp of the softmax group
         }
         for (int s = 0; s < NS; ++s) {
             mbar_init(&bars->k_full[s], 1);
@@ -165,7 +643,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&bars->drain, 1);
         mbar_init(&bars->never, 1);
-        bars->abort = 0;
+        // the operand layouts assume a 1024-byte aligned base (128-byte swizzle atoms)
+        bars->abort = (x.sbase & 1023u) ? 1 : 0;
+        if (x.sbase & 1023u) atomicExch(&g_device_status, 3);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -178,242 +658,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const unsigned tmem = bars->tmem_base;
+    x.tmem = bars->tmem_base;
     if (force_timeout_ns) {
         // test hook: a wait on a barrier phase that nothing completes
-        if (tid == 0 && !mbar_wait(&bars->never, 0, force_timeout_ns)) {
-            bars->abort = 1;
-            atomicExch(&g_device_status, 5);
-        }
+        if (tid == 0 && !mbar_wait(&bars->never, 0, force_timeout_ns)) x.give_up();
         __syncthreads();
     }
-    const bool go = *abort_flag == 0;
-    auto give_up = [&]() {
-        *abort_flag = 1;
-        atomicExch(&g_device_status, 5);
-    };
+    const bool go = *x.abort_flag == 0;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0 && go && nch > 0) {
-            prefetch_tmap(&tmQ);
-            prefetch_tmap(&tmK);
-            prefetch_tmap(&tmV);
-            for (int t = 0; t < ntiles; ++t) {
-                mbar_expect_tx(&bars->q_full[t], C::q_bytes);
-#pragma unroll
-                for (int kb = 0; kb < C::KB; ++kb)
-                    tma_load_3d(sbase + C::off_q + t * C::q_bytes + kb * (kRows * 128), &tmQ, kb * 64,
-                                (int)(i0 + t * kRows), b, &bars->q_full[t]);
-            }
-            int issued_k = 0, issued_v = 0;
-            bool ok = true;
-            for (int c = 0; c < nch; ++c) {
-                const int s = c % NS;
-                const unsigned ph = (unsigned)(c / NS) & 1u;
-                if (c >= NS && !(ok = mbar_wait_or_abort(&bars->k_empty[s], ph ^ 1u, abort_flag))) break;
-                mbar_expect_tx(&bars->k_full[s], C::k_bytes);
-#pragma unroll
-                for (int kb = 0; kb < C::KB; ++kb)
-                    tma_load_3d(sbase + C::off_k + s * C::k_bytes + kb * (kChunk * 128), &tmK, kb * 64, c * kChunk, b,
-                                &bars->k_full[s]);
-                ++issued_k;
-                if (c >= NS && !(ok = mbar_wait_or_abort(&bars->v_empty[s], ph ^ 1u, abort_flag))) break;
-                mbar_expect_tx(&bars->v_full[s], C::v_bytes + C::w_bytes);
-#pragma unroll
-                for (int j = 0; j < kChunk / 64; ++j)
-                    tma_load_3d(sbase + C::off_v + s * C::v_bytes + j * (D * 128), &tmV, c * kChunk + j * 64, 0, b,
-                                &bars->v_full[s]);
-                bulk_load(sbase + C::off_w + s * C::w_bytes, wpad + (int64_t)b * rpad + (int64_t)c * kChunk,
-                          C::w_bytes, &bars->v_full[s]);
-                ++issued_v;
-            }
-            if (!ok) give_up();
-            if (*abort_flag) {
-                // copies still in flight must land before the CTA's shared memory is released
-                for (int t = 0; t < ntiles; ++t) mbar_wait(&bars->q_full[t], 0, kDrainNs);
-                for (int c = std::max(0, issued_k - NS); c < issued_k; ++c)
-                    mbar_wait(&bars->k_full[c % NS], (unsigned)(c / NS) & 1u, kDrainNs);
-                for (int c = std::max(0, issued_v - NS); c < issued_v; ++c)
-                    mbar_wait(&bars->v_full[c % NS], (unsigned)(c / NS) & 1u, kDrainNs);
-            }
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+        if (go && lane == 0) {
+            if (warp == 0) role_producer<D>(x, &tmQ, &tmK, &tmV, wpad, rpad);
+            else if (warp == 1) role_mma<D>(x);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------- tensor cores
-        if (lane == 0 && go && nch > 0) {
-            constexpr uint32_t id1 = idesc_bf16(128, kChunk);
-            constexpr uint32_t id2 = idesc_bf16(128, D);
-            auto gemm1 = [&](int c, int t) {  // S_t = Q_t K_c^T
-                const unsigned qa = sbase + C::off_q + t * C::q_bytes;
-                const unsigned kb = sbase + C::off_k + (c % NS) * C::k_bytes;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    mma_bf16(tmem + C::col_S + t * kChunk,
-                             umma_desc(qa + (kk >> 2) * (kRows * 128) + (kk & 3) * 32),
-                             umma_desc(kb + (kk >> 2) * (kChunk * 128) + (kk & 3) * 32), id1, kk > 0);
-            };
-            auto gemm2 = [&](int c, int t) {  // O_t += P_t V_c (P_t in tensor memory)
-                const unsigned vb = sbase + C::off_v + (c % NS) * C::v_bytes;
-#pragma unroll
-                for (int kk = 0; kk < kChunk / 16; ++kk)
-                    mma_bf16_ts(tmem + C::col_O + t * D, tmem + C::col_S + t * kChunk + kk * 8,
-                                umma_desc(vb + (kk >> 2) * (D * 128) + (kk & 3) * 32), id2, (c > 0 || kk > 0) ? 1 : 0);
-            };
-            bool ok = mbar_wait_or_abort(&bars->k_full[0], 0, abort_flag);
-            for (int t = 0; t < ntiles && ok; ++t) {
-                if (!(ok = mbar_wait_or_abort(&bars->q_full[t], 0, abort_flag))) break;
-                tc_fence_after();
-                gemm1(0, t);
-                mma_commit(&bars->s_full[t]);
-            }
-            if (ok) mma_commit(&bars->k_empty[0]);
-            for (int c = 0; c < nch && ok; ++c) {
-                const int s = c % NS;
-                if (!(ok = mbar_wait_or_abort(&bars->v_full[s], (unsigned)(c / NS) & 1u, abort_flag))) break;
-                const bool more = c + 1 < nch;
-                const int s1 = (c + 1) % NS;
-                for (int t = 0; t < ntiles; ++t) {
-                    if (!(ok = mbar_wait_or_abort(&bars->p_full[t], (unsigned)c & 1u, abort_flag))) break;
-                    tc_fence_after();
-                    gemm2(c, t);
-                    if (more) {
-                        if (t == 0 &&
-                            !(ok = mbar_wait_or_abort(&bars->k_full[s1], (unsigned)((c + 1) / NS) & 1u, abort_flag)))
-                            break;
-                        tc_fence_after();
-                        // issued after GEMM2 of the same tile, which has read P_t out of these
-                        // columns by the time this product writes them (tcgen05.mma executes
-                        // in issue order)
-                        gemm1(c + 1, t);
-                        mma_commit(&bars->s_full[t]);
-                    } else {
-                        mma_commit(&bars->o_full[t]);
-                    }
-                }
-                if (!ok) break;
-                mma_commit(&bars->v_empty[s]);
-                if (more) mma_commit(&bars->k_empty[s1]);
-            }
-            if (!ok) give_up();
-            // every product issued has finished before tensor memory is released
-            mma_commit(&bars->drain);
-            mbar_wait(&bars->drain, 0, kDrainNs);
-        }
+    } else if (warp < 12) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+        if (go) role_softmax<D>(x, (warp - 4) >> 2, warp & 3, lane, beta, kmax);
     } else {
-        // ---------------------------------------------- softmax and epilogue
-        const int t = (warp - 2) >> 2;
-        const int quad = warp & 3;              // TMEM lane quadrant this warp may access
-        const int row = quad * 32 + lane;       // query row within the tile = TMEM lane
-        const unsigned lane_off = (unsigned)(quad * 32) << 16;
-        const unsigned tS = tmem + C::col_S + t * kChunk + lane_off;
-        const unsigned tO = tmem + C::col_O + t * D + lane_off;
-        const float a = beta * 1.4426950408889634f;
-        const float sh = beta * MQ[b] * 1.4426950408889634f;
-        float dsum[4] = {0.f, 0.f, 0.f, 0.f};
-        if (t < ntiles) {
-            bool ok = go;
-            for (int c = 0; c < nch && ok; ++c) {
-                const int s = c % NS;
-                bool w = mbar_wait_or_abort(&bars->s_full[t], (unsigned)c & 1u, abort_flag) &&
-                         mbar_wait_or_abort(&bars->v_full[s], (unsigned)(c / NS) & 1u, abort_flag);
-                ok = __all_sync(0xffffffffu, w);  // tcgen05.ld / st below are warp-collective
-                if (!ok) break;
-                tc_fence_after();
-                const float4* w4 = reinterpret_cast<const float4*>(sm + C::off_w + s * C::w_bytes);
-                const int lim = rr - c * kChunk;  // keys of this chunk below the rank
-#pragma unroll
-                for (int j = 0; j < kChunk / 32; ++j) {
-                    uint32_t v[32];
-                    tmem_ld32_nowait(tS + 32 * j, v);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        float p0 = ex2_approx(fmaf(__uint_as_float(v[2 * e]), a, -sh));
-                        float p1 = ex2_approx(fmaf(__uint_as_float(v[2 * e + 1]), a, -sh));
-                        if (lim < kChunk) {
-                            const int k0 = 32 * j + 2 * e;
-                            p0 = k0 < lim ? p0 : 0.f;
-                            p1 = k0 + 1 < lim ? p1 : 0.f;
-                        }
-                        pk[e] = pack_bf16x2(p0, p1);
-                    }
-#pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4) {
-                        const float4 ww = w4[8 * j + e4];
-                        const uint32_t x0 = pk[2 * e4], x1 = pk[2 * e4 + 1];
-                        dsum[0] = fmaf(__uint_as_float(x0 << 16), ww.x, dsum[0]);
-                        dsum[1] = fmaf(__uint_as_float(x0 & 0xffff0000u), ww.y, dsum[1]);
-                        dsum[2] = fmaf(__uint_as_float(x1 << 16), ww.z, dsum[2]);
-                        dsum[3] = fmaf(__uint_as_float(x1 & 0xffff0000u), ww.w, dsum[3]);
-                    }
-                    tmem_st16(tS + 16 * j, pk);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->p_full[t]);
-            }
-            if (ok && nch > 0) ok = __all_sync(0xffffffffu, mbar_wait_or_abort(&bars->o_full[t], 0, abort_flag));
-            if (!ok && lane == 0) give_up();
-            // the whole group agrees before the epilogue's group barriers
-            ok = group_all(1 + t, ok);
-            if (ok) {
-                tc_fence_after();
-                const float den = (dsum[0] + dsum[1]) + (dsum[2] + dsum[3]);
-                const float rcp = 1.0f / den;  // rank 0: 0 * inf = NaN, which the clip turns into v_min
-                const float* lo = vmin + (int64_t)b * D;
-                const float* hi = vmax + (int64_t)b * D;
-                unsigned char* stage = sm + C::off_q + t * C::q_bytes;  // this tile's Q is no longer read
-                const unsigned stage_s = sbase + C::off_q + t * C::q_bytes;
-#pragma unroll 1
-                for (int h = 0; h < 2; ++h) {
-#pragma unroll 1
-                    for (int g = 0; g < D / 64; ++g) {
-                        const int col0 = h * (D / 2) + g * 32;
-                        uint32_t v[32];
-                        if (nch > 0) {
-                            tmem_ld32_nowait(tO + col0, v);
-                            tmem_wait_ld();
-                        } else {
-#pragma unroll
-                            for (int k = 0; k < 32; ++k) v[k] = 0u;
-                        }
-                        unsigned char* box = stage + g * (kRows * 128) + row * 128;
-#pragma unroll
-                        for (int cc = 0; cc < 8; ++cc) {
-                            const float4 l4 = __ldg(reinterpret_cast<const float4*>(lo + col0) + cc);
-                            const float4 h4 = __ldg(reinterpret_cast<const float4*>(hi + col0) + cc);
-                            float4 o;
-                            o.x = fminf(fmaxf(__uint_as_float(v[4 * cc + 0]) * rcp, l4.x), h4.x);
-                            o.y = fminf(fmaxf(__uint_as_float(v[4 * cc + 1]) * rcp, l4.y), h4.y);
-                            o.z = fminf(fmaxf(__uint_as_float(v[4 * cc + 2]) * rcp, l4.z), h4.z);
-                            o.w = fminf(fmaxf(__uint_as_float(v[4 * cc + 3]) * rcp, l4.w), h4.w);
-                            *reinterpret_cast<float4*>(box + ((cc ^ (row & 7)) << 4)) = o;
-                        }
-                    }
-                    fence_async_smem();
-                    named_barrier_sync(1 + t, 128);
-                    if (row == 0) {
-#pragma unroll
-                        for (int g = 0; g < D / 64; ++g)
-                            tma_store_3d(&tmO, h * (D / 2) + g * 32, (int)(i0 + t * kRows), b,
-                                         stage_s + g * (kRows * 128));
-                        bulk_commit();
-                        bulk_wait_read_all();
-                    }
-                    named_barrier_sync(1 + t, 128);
-                }
-                if (row == 0) bulk_wait_all();
-            }
-        }
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpilogue));
+        if (go) role_epilogue<D>(x, warp & 3, lane, &tmO, vmin, vmax);
     }
 
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::tmem_cols) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(x.tmem), "r"(C::tmem_cols)
+                     : "memory");
     }
 }
 
@@ -440,15 +712,58 @@ __global__ void vt_prep_kernel(const float* __restrict__ V_S, const float* __res
     }
 }
 
+// kmax[b] = max_{l < rank} |K_S[b, l]| (the pivot-key half of the per-row shift)
 template <int D>
-Status run_tc(const AttendRequest& q, const float* MQ, void* scratch, cudaStream_t st) {
+__global__ void kmax_kernel(const __nv_bfloat16* __restrict__ K_S, const int32_t* __restrict__ rank, int r,
+                            float* __restrict__ kmax) {
+    const int64_t b = blockIdx.x;
+    const int rr = rank[b];
+    float best = 0.f;
+    for (int l = threadIdx.x; l < rr; l += blockDim.x) {
+        const uint4* k4 = reinterpret_cast<const uint4*>(K_S + (b * r + l) * D);
+        float s = 0.f;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+            float x[8];
+            load8(reinterpret_cast<const __nv_bfloat16*>(k4 + c), x);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s = fmaf(x[e], x[e], s);
+        }
+        best = fmaxf(best, sqrtf(s));
+    }
+    best = warp_max(best);
+    __shared__ float wb[32];
+    if ((threadIdx.x & 31) == 0) wb[threadIdx.x >> 5] = best;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float v = 0.f;
+        for (int k = 0; k < (int)(blockDim.x >> 5); ++k) v = fmaxf(v, wb[k]);
+        kmax[b] = v;
+    }
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 148;
+    }
+    return n;
+}
+
+template <int D>
+Status run_tc(const AttendRequest& q, void* scratch, cudaStream_t st) {
     using C = Cfg<D>;
     const int rpad = (int)round_up(q.r, kChunk);
-    __nv_bfloat16* VT = static_cast<__nv_bfloat16*>(scratch);
-    float* wpad = reinterpret_cast<float*>(static_cast<char*>(scratch) +
-                                           round_up((int64_t)sizeof(__nv_bfloat16) * q.BH * D * rpad, 256));
+    char* p = static_cast<char*>(scratch);
+    __nv_bfloat16* VT = reinterpret_cast<__nv_bfloat16*>(p);
+    p += round_up((int64_t)sizeof(__nv_bfloat16) * q.BH * D * rpad, 256);
+    float* wpad = reinterpret_cast<float*>(p);
+    p += round_up((int64_t)sizeof(float) * q.BH * rpad, 256);
+    float* kmax = reinterpret_cast<float*>(p);
     vt_prep_kernel<D><<<dim3((unsigned)(rpad / 32), D / 32, (unsigned)q.BH), dim3(32, 8), 0, st>>>(
         q.V_S, q.w, q.rank, q.r, rpad, VT, wpad);
+    kmax_kernel<D><<<(unsigned)q.BH, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q.K_S), q.rank, q.r, kmax);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return Status::cuda(e, "attend_tc: prep launch");
     if (q.m == 0) return Status::ok();
@@ -463,8 +778,11 @@ Status run_tc(const AttendRequest& q, const float* MQ, void* scratch, cudaStream
     if (!ok) return Status::fail(3, "attend_tc: tensor map encoding failed");
     e = cudaFuncSetAttribute(attend_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::total);
     if (e != cudaSuccess) return Status::cuda(e, "attend_tc: shared memory attribute");
-    attend_tc_kernel<D><<<dim3((unsigned)ceil_div(q.m, 2 * kRows), (unsigned)q.BH), kThreads, C::total, st>>>(
-        tmQ, tmK, tmV, tmO, wpad, rpad, q.m, q.rank, q.beta, q.vmin, q.vmax, MQ, g_force_timeout_ns);
+    const int64_t units = ceil_div(q.m, 2 * kRows) * q.BH;
+    if (units >= (int64_t(1) << 31)) return Status::fail(2, "attend_tc: more than 2^31 query-tile pairs");
+    const unsigned grid = (unsigned)std::min<int64_t>(units, sm_count());
+    attend_tc_kernel<D><<<grid, kThreads, C::total, st>>>(tmQ, tmK, tmV, tmO, wpad, rpad, q.m, q.BH, q.rank, q.beta,
+                                                         q.vmin, q.vmax, kmax, g_force_timeout_ns);
     e = cudaGetLastError();
     if (e != cudaSuccess) return Status::cuda(e, "attend_tc launch");
     return Status::ok();
@@ -476,17 +794,18 @@ bool attend_tc_supported(int dtype, int d) { return dtype == 1 && (d == 64 || d 
 
 size_t attend_tc_scratch_bytes(int64_t BH, int d, int r) {
     const int64_t rpad = round_up(r, kChunk);
-    return (size_t)round_up((int64_t)sizeof(__nv_bfloat16) * BH * d * rpad, 256) + sizeof(float) * (size_t)BH * rpad;
+    return (size_t)(round_up((int64_t)sizeof(__nv_bfloat16) * BH * d * rpad, 256) +
+                    round_up((int64_t)sizeof(float) * BH * rpad, 256) + (int64_t)sizeof(float) * BH);
 }
 
-Status launch_attend_tc(const AttendRequest& q, const float* MQ, void* scratch, cudaStream_t st) {
+Status launch_attend_tc(const AttendRequest& q, void* scratch, cudaStream_t st) {
     if ((reinterpret_cast<uintptr_t>(q.O) & 15u) || (reinterpret_cast<uintptr_t>(q.Q) & 15u) ||
         (reinterpret_cast<uintptr_t>(q.K_S) & 15u) || (reinterpret_cast<uintptr_t>(q.vmin) & 15u) ||
         (reinterpret_cast<uintptr_t>(q.vmax) & 15u))
         return Status::fail(1, "attend_tc: Q, K_S, O, vmin and vmax must be 16-byte aligned");
     switch (q.d) {
-        case 64: return run_tc<64>(q, MQ, scratch, st);
-        case 128: return run_tc<128>(q, MQ, scratch, st);
+        case 64: return run_tc<64>(q, scratch, st);
+        case 128: return run_tc<128>(q, scratch, st);
     }
     return Status::fail(2, "attend_tc: unsupported head dim");
 }

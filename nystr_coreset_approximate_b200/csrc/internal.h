@@ -139,7 +139,7 @@ Status launch_attend_simt(const AttendRequest& q, cudaStream_t stream);
 // tensor-core attend (attend_tc.cu)
 bool attend_tc_supported(int dtype, int d);
 size_t attend_tc_scratch_bytes(int64_t BH, int d, int r);
-Status launch_attend_tc(const AttendRequest& q, const float* MQ, void* b2_scratch, cudaStream_t stream);
+Status launch_attend_tc(const AttendRequest& q, void* scratch, cudaStream_t stream);
 // device status word set by bounded waits that expired (0 = none); -1 if unreadable
 int read_device_status(bool clear);  // first non-zero of the per-file status words below
 int read_attend_status(bool clear);

@@ -193,6 +193,8 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, int x, int y, int
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// all but the most recent bulk group have finished reading their source
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
@@ -202,6 +204,31 @@ __device__ __forceinline__ void bulk_load(unsigned dst, const void* src, unsigne
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "l"(src), "r"(bytes), "r"(smem_u32(mbar))
                  : "memory");
+}
+
+// The same products with each shared-memory descriptor given as its two
+// 32-bit words (the high word is the same for every K step of a tile, so the
+// caller keeps one register for it instead of one 64-bit value per step).
+__device__ __forceinline__ void mma_bf16_w(unsigned tmem_d, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo, uint32_t b_hi,
+                                           uint32_t idesc, int accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
+        "mov.b64 da, {%1, %2};\n\t"
+        "mov.b64 db, {%3, %4};\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}\n" ::"r"(tmem_d),
+        "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_bf16_ts_w(unsigned tmem_d, unsigned tmem_a, uint32_t b_lo, uint32_t b_hi,
+                                              uint32_t idesc, int accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
+        "mov.b64 db, {%2, %3};\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}\n" ::"r"(tmem_d),
+        "r"(tmem_a), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 // D (tmem) (+)= A (tmem, 128 lanes x K packed bf16 pairs) * B (smem descriptor)
@@ -237,6 +264,41 @@ __device__ __forceinline__ void tmem_st16(unsigned taddr, const uint32_t (&r)[16
         : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// {a.x * b.x + c.x, a.y * b.y + c.y} in one packed fp32x2 instruction.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long A = *reinterpret_cast<unsigned long long*>(&a);
+    unsigned long long B = *reinterpret_cast<unsigned long long*>(&b);
+    unsigned long long C = *reinterpret_cast<unsigned long long*>(&c);
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(C) : "l"(A), "l"(B));
+    return *reinterpret_cast<float2*>(&C);
+}
+
+// Bounded wait that also gives up as soon as *abort is set; the waiting
+// thread is suspended by the hardware (up to `hint_ns` per try) instead of
+// spinning, so it takes no issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_suspend(unsigned a, unsigned parity, unsigned hint_ns) {
+    unsigned done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(a), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return done != 0;
+}
+__device__ __forceinline__ bool mbar_wait_suspend(void* mbar, unsigned parity, const volatile int* abort,
+                                                  unsigned long long limit_ns = kWaitLimitNs) {
+    const unsigned a = smem_u32(mbar);
+    if (mbar_try_suspend(a, parity, 1000000u)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (;;) {
+        if (mbar_try_suspend(a, parity, 1000000u)) return true;
+        if (*abort) return false;
+        if (globaltimer() - t0 > limit_ns) return false;
+    }
+}
 
 // 2^x on the special-function unit (approximate, subnormal results flushed).
 __device__ __forceinline__ float ex2_approx(float x) {
