@@ -70,8 +70,8 @@ def parse():
                    help="also time the inverse-maintenance weights route on the selected pivots")
     p.add_argument("--select-phase-steps", type=int, default=0,
                    help="select steps per launch (0 = automatic: 64 for r >= 512; < 0 = one launch)")
-    p.add_argument("--select-kernel", type=int, choices=[0, 1, 2, 3, 4], default=0,
-                   help="0 = automatic (the cp.async kernel), 1 = cp.async, 2 = bulk-copy where it applies")
+    p.add_argument("--select-kernel", type=int, choices=[0, 1, 3], default=0,
+                   help="0 = automatic, 1 = clusters, 3 = global sync where it applies")
     return p.parse_args()
 
 
@@ -157,9 +157,7 @@ def read_peaks():
 SELECT_KERNELS = {
     # last_select_kernel() code -> kernel name
     1: "rpc_select_kernel",
-    2: "rpc_select_bulk_kernel",
     3: "rpc_select_kernel (global sync)",
-    4: "rpc_select_kernel (tensor-core key pass)",
 }
 
 

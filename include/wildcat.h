@@ -257,7 +257,12 @@ wildcat_status wildcat_decode_attend(const void* Q_new, const void* K_new, const
  *
  * The first call on each device looks up the array's device address (a
  * host-side runtime query, no allocation); make that first call before any
- * stream capture.  All calls share the one array, so calls whose work
+ * stream capture.  The address is remembered per device ordinal for the
+ * life of the process: it assumes the device's primary context is the one
+ * in use throughout, so after cudaDeviceReset (or with another context made
+ * current on that ordinal) the remembered address is stale and this entry
+ * point must not be called again in that process.  The call launches on the
+ * current device; every pointer must belong to it.  All calls share the one array, so calls whose work
  * overlaps on the GPU (e.g. on two streams) race and must be serialised by
  * the caller.  Each call writes every scratch word before reading it, so
  * the contents left by an earlier call do not matter.
@@ -376,7 +381,8 @@ wildcat_status wildcat_pivot_uniforms(uint64_t seed, int64_t BH, int steps, doub
 /*
  * wildcat_get_device_status -- waits for `stream`, then reports and clears
  * the device status words of the current device.  Kernels that wait on
- * mbarriers (the tensor-core weights and attend, the bulk-copy select) bound
+ * mbarriers (the tensor-core weights and attend) or on counters (the select's
+ * global-sync form) bound
  * every wait by a time limit; when one expires the kernel records
  * WILDCAT_ERR_TIMEOUT there, stops issuing work, waits (bounded) for its
  * copies in flight, releases its tensor memory and returns, leaving its
@@ -399,40 +405,28 @@ wildcat_status wildcat_test_force_wait_timeout(int64_t nanoseconds);
 
 /*
  * wildcat_test_force_select_timeout -- test hook for the bounded waits of
- * the select kernels that have them.  With nanoseconds > 0, every later
- * launch of the bulk-copy kernel waits that long, after step 1, on a barrier
- * phase that nothing completes (every instance then stops after two steps);
- * in the global-sync form, CTA 0 of every instance never arrives at the
- * third counter barrier and every wait there ends after `nanoseconds`
- * (every instance stops after one step).  Either expiry is handled like any
- * other: WILDCAT_ERR_TIMEOUT in the device status word.  0 turns the hook
- * off.  Process-wide; for tests only.  Returns WILDCAT_ERR_INVALID_ARG
- * outside [0, 1e9].
+ * the select's global-sync form.  With nanoseconds > 0, CTA 0 of every
+ * instance never arrives at the third counter barrier and every wait there
+ * ends after `nanoseconds` (every instance stops after one step).  The
+ * expiry is handled like any other: WILDCAT_ERR_TIMEOUT in the device status
+ * word.  0 turns the hook off.  Process-wide; for tests only.  Returns
+ * WILDCAT_ERR_INVALID_ARG outside [0, 1e9].
  */
 wildcat_status wildcat_test_force_select_timeout(int64_t nanoseconds);
 
 /*
- * wildcat_set_select_kernel -- which select kernel wildcat_select* launch:
- * 0 (default) the cp.async kernel (per-thread asynchronous copies): in its
- * global-sync form when a workspace is given and that form has less work per
- * CTA, else on clusters; 1 the cp.async kernel on clusters only;
- * 2 the bulk-copy kernel (copy-engine stages on mbarriers) wherever it
- * applies (n % 4 == 0, n / cluster size <= 8192, 16-byte aligned K and F,
- * d in {32, 64, 128}), else the cp.async kernel; 3 the global-sync form
- * wherever a workspace is given and all CTAs fit at once; 4 the cp.async
- * kernel on clusters with the key pass on the tensor cores where the keys
- * stay resident in shared memory and are bfloat16 with d in {64, 128}
- * (measured slower than the CUDA-core key pass; kept for comparison).  Both compute the same
- * factorisation (results agree to float32 rounding).  Process-wide; not
- * thread-safe against concurrent select calls.  Returns
- * WILDCAT_ERR_INVALID_ARG for other values.
+ * wildcat_set_select_kernel -- which form of the select kernel
+ * wildcat_select* launch: 0 (default) the global-sync form when a workspace
+ * is given and that form has less work per CTA, else clusters; 1 clusters
+ * only; 3 the global-sync form wherever a workspace is given and all CTAs
+ * fit at once.  Both forms compute the same factorisation (results agree to
+ * float32 rounding).  Process-wide; not thread-safe against concurrent
+ * select calls.  Returns WILDCAT_ERR_INVALID_ARG for other values.
  */
 wildcat_status wildcat_set_select_kernel(int kernel);
 
-/* The select kernel the last select launch on this thread used: 1 the
- * cp.async kernel on clusters (CUDA-core key pass), 2 the bulk-copy kernel,
- * 3 the cp.async kernel in global-sync form, 4 the cp.async kernel on
- * clusters with the tensor-core key pass, 0 if none. */
+/* The form of the select kernel the last select launch on this thread used:
+ * 1 clusters, 3 global sync, 0 if none. */
 int wildcat_last_select_kernel(void);
 
 /* Threads per CTA of the last select launch on this thread: 512, or 256 when

@@ -157,6 +157,12 @@ def _dtype_code(t) -> int:
 def _dev(t, name, dtype=None):
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    # the library launches on the current device (and keys per-device state on
+    # it): a tensor elsewhere would be read through the wrong GPU
+    cur = _torch().cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"{name} is on cuda:{t.device.index} but the current device is cuda:{cur}; "
+                         f"call under torch.cuda.device({t.device.index})")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
@@ -500,15 +506,13 @@ def last_select_cluster() -> int:
 
 
 def set_select_kernel(kernel: int):
-    """0 = automatic, 1 = the cp.async kernel on clusters (CUDA-core key pass),
-    2 = the bulk-copy kernel where it applies, 3 = the cp.async kernel in
-    global-sync form where it applies, 4 = the cp.async kernel on clusters with
-    the tensor-core key pass where it applies."""
+    """0 = automatic, 1 = the select kernel on clusters, 3 = its global-sync
+    form where it applies."""
     _check(lib().wildcat_set_select_kernel(int(kernel)))
 
 
 def last_select_kernel() -> int:
-    """1 = the cp.async kernel, 2 = the bulk-copy kernel (last select launch)."""
+    """1 = clusters, 3 = global sync (form of the last select launch)."""
     return int(lib().wildcat_last_select_kernel())
 
 
@@ -544,6 +548,6 @@ def set_stage_events(after_select=None, after_weights=None):
 
 
 def force_select_timeout(nanoseconds: int):
-    """Test hook: the bulk-copy select kernel waits this long on a barrier
-    nothing completes (0 = off)."""
+    """Test hook: the select's global-sync barrier waits this long on a
+    counter one CTA never bumps (0 = off)."""
     _check(lib().wildcat_test_force_select_timeout(int(nanoseconds)))

@@ -243,8 +243,7 @@ HostPipe* host_pipe(int dev) {
 
 namespace wildcat {
 int read_device_status(bool clear) {
-    const int parts[4] = {read_attend_status(clear), read_weights_status(clear), read_select_status(clear),
-                          read_select_gs_status(clear)};
+    const int parts[3] = {read_attend_status(clear), read_weights_status(clear), read_select_gs_status(clear)};
     for (const int v : parts)
         if (v < 0) return -1;
     for (const int v : parts)
@@ -615,9 +614,9 @@ wildcat_status wildcat_test_force_select_timeout(int64_t nanoseconds) {
 }
 
 wildcat_status wildcat_set_select_kernel(int kernel) {
-    if (kernel < 0 || kernel > 4)
-        return bad(1, "%s: kernel must be 0 (automatic), 1 (cp.async), 2 (bulk-copy), 3 (global sync) or 4 "
-                   "(cp.async with the tensor-core key pass)", "wildcat_set_select_kernel");
+    if (kernel != 0 && kernel != 1 && kernel != 3)
+        return bad(1, "%s: kernel must be 0 (automatic), 1 (clusters) or 3 (global sync)",
+                   "wildcat_set_select_kernel");
     wildcat::select_kernel_override(kernel);
     return record(Status::ok());
 }

@@ -266,7 +266,10 @@ Status launch_attend(const AttendRequest& q, cudaStream_t st) {
 // not pass the array's name to a kernel (on the host it is only a stand-in
 // symbol), so the device address is looked up with cudaGetSymbolAddress once
 // per device, with that device current, on the first no-alloc call made
-// there; make that first call before any stream capture.  All calls share
+// there; make that first call before any stream capture.  The address is
+// kept per device ordinal for the life of the process, which assumes the
+// device's primary context stays the one in use: after cudaDeviceReset, or
+// with another context current on that ordinal, it would be stale.  All calls share
 // the array: calls whose kernels overlap on the GPU (for example on two
 // streams at once) race on it and must be serialised by the caller.  Every
 // scratch word a call reads is written earlier in the same call, so nothing

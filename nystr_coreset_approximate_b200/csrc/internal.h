@@ -42,14 +42,13 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream);
 Status launch_pivot_uniforms(uint64_t seed, int64_t BH, int steps, double* u, cudaStream_t stream);
 int select_cluster_override(int G);  // G < 0: query only
 int last_select_cluster();
-int select_kernel_override(int k);  // k < 0: query only; 0 automatic, 1 cp.async (clusters, CUDA-core key
-                                    // pass), 2 bulk-copy, 3 cp.async with global sync where a workspace
-                                    // allows, 4 cp.async (clusters) with the tensor-core key pass where it applies
-int last_select_kernel();           // 1, 2, 3 as above; 4 clusters with the tensor-core key pass
+int select_kernel_override(int k);  // k < 0: query only; 0 automatic, 1 clusters, 3 global sync where a
+                                    // workspace allows
+int last_select_kernel();           // 1 clusters, 3 global sync
 int last_select_threads();          // threads per CTA of the last select launch (256 or 512)
 int select_phase_steps_override(int k, bool set);  // steps per launch: 0 automatic, < 0 one launch
 int last_select_phases();           // launches of the last select call (1 = no phases)
-// cluster-size choice shared by both select kernels (select.cu)
+// cluster-size choice of the select kernel (select.cu)
 struct ClusterKey {
     int dev, kernel;
     int64_t n, BH;
@@ -62,9 +61,8 @@ int choose_cluster_rows(int64_t n, int64_t BH, int (*fit)(int G, void* ctx), voi
                         int min_rows = 512);
 size_t select_workspace_bytes(int64_t BH, int64_t n);  // global-sync exchange buffers
 int read_select_gs_status(bool clear);
-// bulk-copy select kernel (select_bulk.cu); *used = false when the shape is not one it handles.
-// G_override > 0 fixes the cluster size.
-Status launch_select_bulk(const SelectRequest& q, int G_override, cudaStream_t stream, bool* used, int* G_used);
+// test hook: the global-sync barrier of the select waits on a counter that
+// one CTA never bumps for `ns` nanoseconds (0 = off)
 void set_select_force_timeout(unsigned long long ns);
 unsigned long long select_force_timeout_ns();
 
@@ -144,7 +142,6 @@ Status launch_attend_tc(const AttendRequest& q, void* scratch, cudaStream_t stre
 int read_device_status(bool clear);  // first non-zero of the per-file status words below
 int read_attend_status(bool clear);
 int read_weights_status(bool clear);
-int read_select_status(bool clear);
 // test hook: the tensor-core attend first waits `ns` nanoseconds on a barrier
 // that nothing completes, then reports a timeout (0 = off)
 void set_attend_force_timeout(unsigned long long ns);

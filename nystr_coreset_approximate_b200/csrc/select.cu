@@ -28,7 +28,6 @@
 #include "common.cuh"
 #include "internal.h"
 #include "philox.cuh"
-#include "tc_common.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -37,7 +36,6 @@ namespace wildcat {
 namespace {
 
 constexpr int kFsByWarp0 = 512;  // factor rows up to this length are gathered by warp 0 alone
-constexpr unsigned kTckCols = 128;  // tensor memory columns of the key pass: 8 tiles x 16
 constexpr int kMaxPL = 16;  // R <= 16384 rows per CTA -> at most 16 values per lane
 constexpr size_t kSmemCap = 227 * 1024;
 constexpr int kGsMaxCtas = 160;  // global-sync CTAs per instance (the search gives a lane ceil(G / 32))
@@ -95,19 +93,12 @@ struct SelectShape {
 };
 
 struct SmemLayout {
-    size_t ring, kres, inbox, csl, dbuf, dotb, ks, fs, red, misc, btile, mbar, total;
+    size_t ring, kres, inbox, csl, dbuf, dotb, ks, fs, red, misc, total;
     __host__ __device__ SmemLayout(int Rpad, int r, int D, int JG, int NT, int VEC, int G, int depth,
-                                   size_t kres_bytes, bool gs = false, bool tck = false) {
+                                   size_t kres_bytes, bool gs = false) {
         size_t o = 0;
-        if (tck) {
-            // key rows first, 1024-byte aligned tiles for the tensor cores; the
-            // last 128-row tile may read past them into the ring (rows ignored)
-            kres = o;  o += round_up(kres_bytes, 1024);
-            ring = o;  o += (size_t)depth * NT * 16;
-        } else {
-            ring = o;  o += (size_t)depth * NT * 16;               // per-thread cp.async ring, [slot][thread] x 16 B
-            kres = o;  o += round_up(kres_bytes, 16);              // the CTA's key rows, when resident
-        }
+        ring = o;  o += (size_t)depth * NT * 16;               // per-thread cp.async ring, [slot][thread] x 16 B
+        kres = o;  o += round_up(kres_bytes, 16);              // the CTA's key rows, when resident
         inbox = o; o += gs ? 0 : 2 * (size_t)G * 33 * sizeof(double);  // [parity][source CTA][32 chunk sums + total]
         csl = o;   o += 32 * sizeof(double);                   // own chunk sums
         dbuf = o;  o += 2 * (size_t)Rpad * sizeof(float);      // residual diagonal, double-buffered
@@ -117,14 +108,6 @@ struct SmemLayout {
         o = round_up(o, 16);
         red = o;   o += (size_t)(JG > 1 ? JG - 1 : 0) * (NT / JG) * VEC * sizeof(float);
         misc = o;  o += 16 * sizeof(float);
-        if (tck) {
-            o = round_up(o, 1024);
-            btile = o; o += (size_t)(D / 64) * 16 * 128;  // B: 16 columns x d, K-major, 128-byte swizzle
-            mbar = o;  o += 16;                           // MMA completion barrier, TMEM base address
-            o += 1024;                                    // slack: the base is rounded up to 1024 bytes
-        } else {
-            btile = mbar = 0;
-        }
         total = round_up(o, 16);
     }
 };
@@ -227,10 +210,8 @@ template <typename E, int D, int VEC, int DEPTH, int KM, bool GS, int NTH>
 __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const SelectArgs a) {
     // NTH threads per CTA: 512 (one CTA per SM), or 256 with twice the CTAs
     // per instance and two CTAs per SM, whose barriers and searches overlap.
-    // KM: 0 keys streamed each step, 1 keys resident in shared memory,
-    // 2 resident and multiplied by the tensor cores (bf16, d in {64, 128}).
+    // KM: 0 keys streamed each step, 1 keys resident in shared memory.
     constexpr bool KRES = KM >= 1;
-    constexpr bool TCK = KM == 2;
     // Launched with a cluster dimension of a.G (one cluster per instance), or,
     // with GS, as one cooperative grid whose a.G CTAs per instance exchange
     // chunk sums and residuals through global memory and meet at a counter
@@ -281,13 +262,8 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
     const int nch = (int)ceil_div(R, CH);
     const int Rpad = nch * CH;  // residual buffers cover whole search chunks
 
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    // the tensor-core key pass needs 1024-byte aligned tiles (the same offset in every CTA)
-    unsigned char* smem = TCK ? reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                                  ~uintptr_t(1023))
-                              : smem_raw;
-    const int Rk = (int)round_up(R, 8);  // resident key rows (whole 8-row swizzle atoms)
-    const SmemLayout L(Rpad, r, D, JG, NT, VEC, G, DEPTH, KRES ? (size_t)Rk * D * sizeof(T) : 0, GS, TCK);
+    extern __shared__ __align__(16) unsigned char smem[];
+    const SmemLayout L(Rpad, r, D, JG, NT, VEC, G, DEPTH, KRES ? (size_t)R * D * sizeof(T) : 0, GS);
     // Each thread streams through its own DEPTH slots of 16 bytes
     // (slot q of thread t at ring4[q * NT + t]); it only ever reads slots it
     // filled itself, so the pipeline needs no barrier.  A slot is refilled
@@ -345,16 +321,8 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
     // (x = ks) or |k_row|^2 (x = nullptr).  LPR lanes share one row, each
     // copying 16 contiguous bytes, so a warp reads RPW whole rows per item;
     // items stream through the thread's cp.async ring.
-    // 16-byte piece pc of resident key row `row`: row-major, or (tensor-core
-    // key pass) 64-element K blocks of 128-byte rows in 8-row atoms with the
-    // 128-byte swizzle (piece c of row r at c ^ (r % 8)), the UMMA K-major layout
-    auto kres_off = [&](int row, int pc) -> size_t {
-        if constexpr (TCK)
-            return (size_t)(pc >> 3) * Rk * 128 + (size_t)(row >> 3) * 1024 + (row & 7) * 128 +
-                   (((pc & 7) ^ (row & 7)) << 4);
-        else
-            return ((size_t)row * D + pc * EPL) * sizeof(T);
-    };
+    // 16-byte piece pc of resident key row `row` (row-major)
+    auto kres_off = [&](int row, int pc) -> size_t { return ((size_t)row * D + pc * EPL) * sizeof(T); };
     // Recentring: every key enters as k - kbar (kbar = 0 without recentring,
     // which leaves the arithmetic bit-identical).
     float kbr[EPL];
@@ -510,11 +478,6 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
     // (a resumed phase reads both back instead)
     const int step0 = a.step0;
     float MK;
-    // tensor-core key pass: B operand (zero outside its first three columns),
-    // the MMA completion barrier and the accumulator columns in tensor memory
-    unsigned tmem = 0;
-    uint64_t* tc_bar = reinterpret_cast<uint64_t*>(smem + L.mbar);
-    unsigned tc_phase = 0;
     if (resume) {
         if (tid == 0) misc[1] = a.ph_mk[b];
         const float* src = a.ph_resid + b * n + row0;
@@ -537,25 +500,6 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
         cp_async_commit();
         cp_async_wait<0>();
         __syncthreads();
-    }
-    if constexpr (TCK) {
-        for (int e = tid; e < (D / 64) * 16 * 128 / 16; e += NT)
-            reinterpret_cast<float4*>(smem + L.btile)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (tid == 0) {
-            tc::mbar_init(tc_bar, 1);
-            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        }
-        if (warp == 0) {
-            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                             tc::smem_u32(smem + L.mbar + 8)),
-                         "r"(kTckCols)
-                         : "memory");
-            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-        }
-        tc::tc_fence_before();
-        __syncthreads();
-        tc::tc_fence_after();
-        tmem = *reinterpret_cast<volatile unsigned*>(smem + L.mbar + 8);
     }
     {
         const float none[EPL] = {};
@@ -786,53 +730,7 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
             }
         }
         // -- <k_l - kbar, k_s - kbar> for the CTA's rows --
-        if constexpr (TCK) {
-            // B rows 0..2: x = k_s - kbar split into bf16 hi + mid + lo (x to ~2^-24)
-            for (int e = tid; e < D; e += NT) {
-                const float x = E::to_float(ksm[e]) - (has_kbar ? a.kbar[(b / a.kbar_div) * D + e] : 0.f);
-                const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-                const float r1 = x - __bfloat162float(hi);
-                const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-                const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-                const int kb = e >> 6, c8 = (e & 63) >> 3, w = e & 7;
-                __nv_bfloat16* bt = reinterpret_cast<__nv_bfloat16*>(smem + L.btile + kb * 2048);
-                bt[(0 * 128 + ((c8 ^ 0) << 4)) / 2 + w] = hi;
-                bt[(1 * 128 + ((c8 ^ 1) << 4)) / 2 + w] = mid;
-                bt[(2 * 128 + ((c8 ^ 2) << 4)) / 2 + w] = lo;
-            }
-            tc::fence_async_smem();
-            tc::tc_fence_before();
-            __syncthreads();
-            tc::tc_fence_after();
-            const int ntiles = (nrows + 127) / 128;
-            if (tid == 0 && ntiles > 0) {
-                const unsigned ka = tc::smem_u32(smem + L.kres), kbt = tc::smem_u32(smem + L.btile);
-                constexpr uint32_t idesc = tc::idesc_bf16(128, 16);
-                for (int t = 0; t < ntiles; ++t) {
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const unsigned oa = (unsigned)((kk >> 2) * Rk * 128 + t * 16384 + (kk & 3) * 32);
-                        const unsigned ob = (unsigned)((kk >> 2) * 2048 + (kk & 3) * 32);
-                        tc::mma_bf16(tmem + t * 16, tc::umma_desc(ka + oa), tc::umma_desc(kbt + ob), idesc, kk > 0);
-                    }
-                }
-                tc::mma_commit(tc_bar);
-            }
-            if (ntiles > 0) {
-                if (!tc::mbar_wait(tc_bar, tc_phase & 1u)) atomicExch(&g_select_gs_status, 5);
-                ++tc_phase;
-                tc::tc_fence_after();
-                for (int t = warp >> 2; t < ntiles; t += NW / 4) {
-                    float v[16];
-                    tc::tmem_ld16(tmem + ((unsigned)(32 * (warp & 3)) << 16) + t * 16, v);
-                    const int row = t * 128 + 32 * (warp & 3) + lane;
-                    if (row < nrows) dotb[row] = (v[0] + v[1]) + v[2];
-                }
-                tc::tc_fence_before();
-            }
-        } else {
-            key_pass(xr, false, dotb);
-        }
+        key_pass(xr, false, dotb);
         cp_async_wait<0>();
         __syncthreads();
         // -- pivot residual g_s (warp 0, the same on every CTA), read after the next barrier --
@@ -995,13 +893,6 @@ __global__ void __launch_bounds__(NTH, 512 / NTH) rpc_select_kernel(const Select
             }
         }
     }
-    if constexpr (TCK) {
-        tc::tc_fence_before();
-        __syncthreads();
-        tc::tc_fence_after();
-        if (warp == 0)
-            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTckCols) : "memory");
-    }
     // keep this CTA's shared memory alive until every peer is done reading it
     if constexpr (!GS) cluster.sync();
 }
@@ -1090,11 +981,8 @@ template <typename E, int VEC, int DEPTH, int KM, bool GS, int NTH = 512>
 int dispatch_d(int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int G_query, cudaError_t* err) {
     switch (d) {
         case 32:
-            if constexpr (KM != 2) {
-                if (a) { *err = launch_select_t<E, 32, VEC, DEPTH, KM, GS, NTH>(*a, smem, stream); return 0; }
-                return fit_t<E, 32, VEC, DEPTH, KM, GS, NTH>(G_query, smem);
-            }
-            break;
+            if (a) { *err = launch_select_t<E, 32, VEC, DEPTH, KM, GS, NTH>(*a, smem, stream); return 0; }
+            return fit_t<E, 32, VEC, DEPTH, KM, GS, NTH>(G_query, smem);
         case 64:
             if (a) { *err = launch_select_t<E, 64, VEC, DEPTH, KM, GS, NTH>(*a, smem, stream); return 0; }
             return fit_t<E, 64, VEC, DEPTH, KM, GS, NTH>(G_query, smem);
@@ -1111,7 +999,7 @@ int dispatch_d(int d, const SelectArgs* a, size_t smem, cudaStream_t stream, int
 // The global-sync mode exists for the vectorised streamed-key variants.
 struct Variant {
     int depth;
-    int km;        // key mode: 0 streamed, 1 resident, 2 resident with the tensor-core key pass
+    int km;        // key mode: 0 streamed, 1 resident
     int nt = 512;  // threads per CTA (256 only for resident keys on CUDA cores)
 };
 
@@ -1131,11 +1019,6 @@ int dispatch_e(const Variant& v, int vec, int d, bool gs, const SelectArgs* a, s
         return dispatch_d<E, 4, 6, 0, true>(d, a, smem, stream, G_query, err);
     }
     if (vec != 4) return dispatch_d<E, 1, 6, 0, false>(d, a, smem, stream, G_query, err);
-    if (v.km == 2) {
-        if constexpr (sizeof(typename E::T) == 2) return dispatch_d<E, 4, 12, 2, false>(d, a, smem, stream, G_query, err);
-        if (err) *err = cudaErrorInvalidValue;
-        return 0;
-    }
     if (v.km == 1) {
         if (v.nt == 256) return dispatch_d<E, 4, 12, 1, false, 256>(d, a, smem, stream, G_query, err);
         return dispatch_d<E, 4, 12, 1, false>(d, a, smem, stream, G_query, err);
@@ -1263,6 +1146,10 @@ int select_kernel_override(int k) {
     g_kernel_override = k;
     return k;
 }
+// test hook of the global-sync barrier (wildcat_test_force_select_timeout)
+static unsigned long long g_force_select_timeout_ns = 0;
+void set_select_force_timeout(unsigned long long ns) { g_force_select_timeout_ns = ns; }
+unsigned long long select_force_timeout_ns() { return g_force_select_timeout_ns; }
 int last_select_kernel() { return g_last_kernel; }
 int last_select_threads() { return g_last_threads; }
 int select_phase_steps_override(int k, bool set) {
@@ -1280,12 +1167,9 @@ static void plan(int64_t n, int r, int d, int dtype, int G, int vec, bool gs, Se
     a->JG = JG;
     a->PL = PL;
     auto bytes = [&](int depth, int km) {
-        const size_t kb = km ? (size_t)round_up(R, 8) * d * (dtype == 1 ? 2 : 4) : 0;
-        return SmemLayout(Rpad, r, d, JG, nt, vec, G, depth, kb, gs, km == 2).total;
+        const size_t kb = km ? (size_t)R * d * (dtype == 1 ? 2 : 4) : 0;
+        return SmemLayout(Rpad, r, d, JG, nt, vec, G, depth, kb, gs).total;
     };
-    // tensor-core key pass for resident bf16 keys: on request only (it measured
-    // slower than the CUDA-core pass on 784 resident rows: 1.33 vs 1.26 ms)
-    const bool tc_ok = g_kernel_override == 4 && dtype == 1 && (d == 64 || d == 128) && R <= 1024;
     if (gs) {
         *v = {6, 0};  // streamed keys only
         for (int depth : {24, 16, 12})
@@ -1295,8 +1179,6 @@ static void plan(int64_t n, int r, int d, int dtype, int G, int vec, bool gs, Se
             }
     } else if (vec != 4) {
         *v = {6, 0};
-    } else if (tc_ok && bytes(12, 2) <= kSmemCap) {
-        *v = {12, 2};  // resident keys, key pass on the tensor cores
     } else if (bytes(12, 1) <= kSmemCap) {
         *v = {12, 1};  // keys stay in shared memory: the per-step key pass reads no global memory
     } else {
@@ -1407,20 +1289,6 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     a.step_end = q.r;
     g_last_phases = 1;
 
-    if (g_kernel_override == 2) {
-        // the bulk-copy kernel (select_bulk.cu) where its shape rules allow
-        bool used = false;
-        int G_used = 0;
-        const Status st = launch_select_bulk(q, g_cluster_override, stream, &used, &G_used);
-        if (used) {
-            if (st.code == 0) {
-                g_last_cluster = G_used;
-                g_last_kernel = 2;
-                g_last_threads = 512;
-            }
-            return st;
-        }
-    }
     size_t smem = 0;
     Variant var{};
     int dev = 0, sms = 0;
@@ -1476,7 +1344,7 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
 
     // Global-sync mode: given a workspace and few instances, more CTAs per
     // instance than clusters allow (all co-resident by a cooperative launch).
-    if (ws_ok && g_kernel_override != 1 && g_kernel_override != 4 && g_cluster_override <= 0) {
+    if (ws_ok && g_kernel_override != 1 && g_cluster_override <= 0) {
         const ClusterKey gkey{dev, g_kernel_override == 3 ? 4 : 3, q.n, q.BH, q.r, q.d, q.dtype};
         int Gg = cached_cluster_lookup(gkey);
         if (Gg == 0) {
@@ -1523,7 +1391,7 @@ Status launch_select(const SelectRequest& q, cudaStream_t stream) {
     int nt = 512;
     if (G <= 0) {
         // the cluster size (and CTA width) with the least work per CTA times waves of clusters
-        const ClusterKey key{dev, g_kernel_override == 4 ? 5 : 1, q.n, q.BH, q.r, q.d, q.dtype};
+        const ClusterKey key{dev, 1, q.n, q.BH, q.r, q.d, q.dtype};
         const int memo = cached_cluster_lookup(key);
         if (memo > 0) {
             G = memo & 0xff;

@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* Ypart, 
 // warp sums its own column and reads the rows from global memory.  Then
 // pivot a (bottom up) gives x_a = y_a / F_S[a, a], and the lanes subtract
 // F_S[a, j] x_a from every y_j, j < a, reading row a contiguously.
-constexpr int kTrsmWarps = 16;
+constexpr int kTrsmWarps = 8;
 constexpr int kTrsmWarpMaxR = 1024;
 constexpr int kTrsmRegs = kTrsmWarpMaxR / 32;  // y values per lane
 constexpr size_t kTrsmSmemCap = 200 * 1024;
@@ -311,20 +311,54 @@ __global__ void __launch_bounds__(kTrsmWarps * 32) trsm_warp_kernel(const float*
         const int j = 32 * m + lane;
         yr[m] = j < rr ? y[j] : 0.f;
     }
+    if constexpr (FS_SMEM) {
+        // F_S in shared memory: the rows are read where they are used
+#pragma unroll
+        for (int mb = kTrsmRegs - 1; mb >= 0; --mb) {
+            if (32 * mb >= rr) continue;
+            const int top = min(31, rr - 1 - 32 * mb);
+            for (int la = top; la >= 0; --la) {
+                const int a = 32 * mb + la;
+                const float* La = Lb + (int64_t)a * r;
+                const float ya = __shfl_sync(0xffffffffu, yr[mb], la);
+                const float xa = ya / La[a];
+#pragma unroll
+                for (int m = 0; m < mb; ++m) yr[m] = fmaf(-La[32 * m + lane], xa, yr[m]);
+                if (lane < la) yr[mb] = fmaf(-La[32 * mb + lane], xa, yr[mb]);
+                if (lane == la) yr[mb] = xa;
+            }
+        }
+    } else {
+    // F_S in global memory: the row of pivot a - 1 is loaded while pivot a is
+    // applied (the loads do not depend on y), so the sweep is not a chain of
+    // dependent L2 reads; the diagonal F_S[a, a] comes from the loaded row by
+    // shuffle.
 #pragma unroll
     for (int mb = kTrsmRegs - 1; mb >= 0; --mb) {
         if (32 * mb >= rr) continue;
         const int top = min(31, rr - 1 - 32 * mb);
-        for (int la = top; la >= 0; --la) {
-            const int a = 32 * mb + la;
-            const float* La = Lb + (int64_t)a * r;
-            const float ya = __shfl_sync(0xffffffffu, yr[mb], la);
-            const float xa = ya / La[a];
+        float cur[kTrsmRegs], nxt[kTrsmRegs];
+        {
+            const float* La = Lb + (int64_t)(32 * mb + top) * r;
 #pragma unroll
-            for (int m = 0; m < mb; ++m) yr[m] = fmaf(-La[32 * m + lane], xa, yr[m]);
-            if (lane < la) yr[mb] = fmaf(-La[32 * mb + lane], xa, yr[mb]);
+            for (int m = 0; m <= mb; ++m) nxt[m] = La[32 * m + lane];
+        }
+        for (int la = top; la >= 0; --la) {
+#pragma unroll
+            for (int m = 0; m <= mb; ++m) cur[m] = nxt[m];
+            if (la > 0) {
+                const float* Ln = Lb + (int64_t)(32 * mb + la - 1) * r;
+#pragma unroll
+                for (int m = 0; m <= mb; ++m) nxt[m] = Ln[32 * m + lane];
+            }
+            const float ya = __shfl_sync(0xffffffffu, yr[mb], la);
+            const float xa = ya / __shfl_sync(0xffffffffu, cur[mb], la);
+#pragma unroll
+            for (int m = 0; m < mb; ++m) yr[m] = fmaf(-cur[m], xa, yr[m]);
+            if (lane < la) yr[mb] = fmaf(-cur[mb], xa, yr[mb]);
             if (lane == la) yr[mb] = xa;
         }
+    }
     }
 #pragma unroll
     for (int m = 0; m < kTrsmRegs; ++m) {

@@ -77,3 +77,27 @@ def column_rel_err(F_gpu, F_orc, rank):
             scale = max(np.abs(ref).max(), 1e-30)
             worst = max(worst, float(np.abs(F_gpu[b, i] - ref).max() / scale))
     return worst
+
+
+def binned_pivots_agree_until_tie(orc, K, beta, r, nbins, seed, eps, S_gpu, rank_gpu, recenter=False, tau=1.0):
+    """Free draws of the binned forward against the oracle's own draws, bin by
+    bin, with the near-tie rule of pivots_agree_until_tie.  Bin q of instance b
+    is the oracle's instance b * nbins + q of the [BH * nbins, n / nbins] view
+    of the keys (recentred by the instance's mean over all n keys when asked),
+    drawn with the key kernel exp(beta <x, y> / tau^2).  Returns the steps
+    compared per bin."""
+    BH, n, d = K.shape
+    nb, rb = n // nbins, r // nbins
+    Kx = K - K.mean(axis=1, keepdims=True) if recenter else K
+    Kv = np.ascontiguousarray(Kx.reshape(BH * nbins, nb, d))
+    beta_key = beta / (tau * tau)
+    own = orc.rpcholesky(Kv, beta_key, rb, seed=seed, eps=eps)
+    S_loc = np.asarray(S_gpu).reshape(BH, nbins, rb).copy()
+    for q in range(nbins):
+        valid = S_loc[:, q] >= 0
+        S_loc[:, q][valid] -= q * nb
+    S_loc = S_loc.reshape(BH * nbins, rb)
+    rank_loc = np.asarray(rank_gpu).reshape(BH * nbins)
+    # the factor on the device's pivots (for a stop at the truncation threshold)
+    fx = orc.rpcholesky(Kv, beta_key, rb, eps=0.0, S_fixed=S_loc)
+    return pivots_agree_until_tie(S_loc, own["S"], own["margin"], rank_loc, own["rank"], fx["F"], own["F"], eps)

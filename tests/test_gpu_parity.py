@@ -89,16 +89,20 @@ def test_stagewise_parity(orc, w):
 @pytest.mark.parametrize("w", [CASES[0], CASES[4], CASES[5]], ids=lambda w: w.name)
 def test_weights_kernel_alone(orc, w):
     """wildcat_weights on the oracle's own factor (rounded to float32) against
-    the oracle's weights on exactly that rounded factor."""
+    the oracle's weights on exactly that rounded factor.  Bounds, relative to
+    the largest entry: 1e-5 for float32 values (fp32 split-K sums and back
+    substitution; measured <= 1.3e-6), 5e-5 for bfloat16 values (the factor
+    split into bf16 hi + lo parts on the tensor cores, about 2^-17 relative
+    per entry; measured <= 1.1e-5)."""
     dev, ex = workloads.make(w)
     res = orc.rpcholesky(ex["K"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
     F32 = res["F"].astype(np.float32)
     VS_o, w_o = orc.weights(F32.astype(np.float64), res["S"], res["rank"], ex["V"])
     V_S, wv, _, _ = wc.weights(torch.from_numpy(F32).cuda(), torch.from_numpy(res["S"]).cuda(),
                                torch.from_numpy(res["rank"]).cuda(), dev["V"].cuda())
-    scale = np.abs(VS_o).max()
-    assert np.abs(V_S.cpu().numpy() - VS_o).max() <= 2e-3 * scale
-    assert np.abs(wv.cpu().numpy() - w_o).max() <= 2e-3 * np.abs(w_o).max()
+    tol = 1e-5 if w.dtype == "f32" else 5e-5
+    assert np.abs(V_S.cpu().numpy() - VS_o).max() <= tol * np.abs(VS_o).max()
+    assert np.abs(wv.cpu().numpy() - w_o).max() <= tol * np.abs(w_o).max()
 
 
 @pytest.mark.parametrize("w", [CASES[1], CASES[2], CASES[3], CASES[5], CASES[6]], ids=lambda w: w.name)

@@ -1,13 +1,12 @@
-"""The two select kernels -- the per-thread cp.async kernel (the default) and
-the bulk-copy kernel (where its shape rules allow) -- against the fp64 oracle
-and against each other, and the bulk kernel's bounded-wait path.
+"""The select kernel's two forms -- clusters (distributed shared memory, the
+hardware cluster barrier) and global sync (a cooperative grid meeting at a
+bounded counter barrier in the workspace) -- against the fp64 oracle and
+against each other, and the global-sync barrier's bounded-wait path.
 
-- Pivots drawn by either kernel agree with the oracle's own draws step by
+- Pivots drawn by either form agree with the oracle's own draws step by
   step until a near-tie; on the device's pivots (fixed-pivot mode, the oracle
   following the device's stopping step) every factor column is within 2e-4
   of the oracle's, relative to the column's largest entry.
-- On the same fixed pivots the two kernels' factors agree to 2e-4 and stop at
-  the same step.
 - A bounded wait that runs out (the test hook) is reported through the
   device status word, every instance stops at the same step, and the next
   call is clean.
@@ -57,16 +56,14 @@ def _run(K, w, kernel, S_fixed=None):
 
 
 @pytest.mark.parametrize("w,G", SHAPES, ids=[w.name for w, _ in SHAPES])
-def test_both_kernels_match_the_oracle(orc, w, G):
+def test_cluster_form_matches_the_oracle(orc, w, G):
     dev, ex = workloads.make(w)
     K = dev["K"].cuda()
     wc.set_select_cluster(G)
     own = orc.rpcholesky(ex["K"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
-    for kernel, expect in ((2, (2,)), (1, (1,)), (0, (1, 3, 4)), (4, (1, 4))):
+    for kernel, expect in ((1, (1,)), (0, (1, 3))):
         S, F, rank, K_S, used = _run(K, w, kernel)
         assert used in expect
-        if w.name == "kres_g4" and kernel == 4:
-            assert used == 4  # resident bf16 keys, d = 64: tensor-core key pass
         if w.name == "kres_g4" and kernel == 0 and G == 0:
             # automatic: two 256-thread CTAs per SM, 8 per instance
             assert wc.last_select_threads() == 256 and wc.last_select_cluster() == 8
@@ -83,85 +80,6 @@ def test_both_kernels_match_the_oracle(orc, w, G):
     assert wc.device_status() == 0
 
 
-def test_tensor_core_key_pass_recentred(orc):
-    """Resident bf16 keys with recentring: the tensor-core key pass splits
-    k_s - kbar into three bf16 parts; pivots follow the oracle's draws on
-    K - mean(K) and the factor matches the oracle on the device's pivots."""
-    w = gc.case("tck_recentre", "walk", 4, 3136, 64, 64, 96, "bf16")
-    dev, ex = workloads.make(w)
-    d = gc.cuda_inputs(dev)
-    wc.set_select_kernel(4)
-    O, S, rank = wc.forward_ex(d["Q"], d["K"], d["V"], w.beta, w.r, w.pivot_seed, EPS, recenter=True)
-    assert wc.last_select_kernel() == 4
-    S, rank = S.cpu().numpy(), rank.cpu().numpy().reshape(w.BH)
-    Kc = ex["K"] - ex["K"].mean(axis=1, keepdims=True)
-    res = orc.rpcholesky(Kc, w.beta, w.r, seed=w.pivot_seed, eps=EPS)
-    gc.pivots_agree_until_tie(S, res["S"], res["margin"], rank, res["rank"])
-    fx = orc.wildcat_forward_binned(ex["Q"], ex["K"], ex["V"], w.beta, w.r, 1, eps=0.0, S_fixed=S,
-                                    recenter=True)
-    lo, hi = orc.value_range(ex["V"])
-    assert gc.r12(O.cpu().numpy(), fx[0], lo, hi) <= gc.TOL_R12["bf16"]
-
-
-@pytest.mark.parametrize("w,G", SHAPES[:5], ids=[w.name for w, _ in SHAPES[:5]])
-def test_kernels_agree_on_fixed_pivots(orc, w, G):
-    dev, ex = workloads.make(w)
-    K = dev["K"].cuda()
-    wc.set_select_cluster(G)
-    own = orc.rpcholesky(ex["K"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
-    S_fixed = torch.from_numpy(own["S"]).cuda()
-    _, F_a, rank_a, _, used_a = _run(K, w, 2, S_fixed)
-    _, F_b, rank_b, _, used_b = _run(K, w, 1, S_fixed)
-    _, F_c, rank_c, _, used_c = _run(K, w, 4, S_fixed)
-    assert (used_a, used_b) == (2, 1) and used_c in (1, 4)
-    assert np.array_equal(rank_a, rank_b) and np.array_equal(rank_c, rank_b)
-    assert gc.column_rel_err(F_a, F_b.astype(np.float64), rank_a) < 2e-4
-    assert gc.column_rel_err(F_c, F_b.astype(np.float64), rank_c) < 2e-4
-
-
-def test_recentred_keys_bulk_kernel(orc):
-    """The bulk kernel's recentring hook: a forward with recenter on draws
-    the pivots the oracle draws on K - mean(K)."""
-    w = gc.case("recentre", "iid", 2, 2048, 64, 64, 48, "bf16")
-    dev, ex = workloads.make(w)
-    d = gc.cuda_inputs(dev)
-    wc.set_select_kernel(2)
-    O, S, rank = wc.forward_ex(d["Q"], d["K"], d["V"], w.beta, w.r, w.pivot_seed, EPS, recenter=True)
-    assert wc.last_select_kernel() == 2
-    S, rank = S.cpu().numpy(), rank.cpu().numpy().reshape(w.BH)
-    _, S_o, rank_o = orc.wildcat_forward_binned(ex["Q"], ex["K"], ex["V"], w.beta, w.r, 1,
-                                                seed=w.pivot_seed, eps=EPS, recenter=True)
-    res = orc.rpcholesky(ex["K"] - ex["K"].mean(axis=1, keepdims=True), w.beta, w.r,
-                         seed=w.pivot_seed, eps=EPS)
-    assert np.array_equal(S_o, res["S"])
-    gc.pivots_agree_until_tie(S, res["S"], res["margin"], rank, res["rank"])
-
-
-def test_bulk_select_bounded_wait_reports_timeout_and_recovers():
-    """The test hook makes every CTA's warp 0 wait 1 ms, after step 1, on a
-    barrier phase nothing completes.  The expiry is recorded in the device
-    status word, the abort reaches every CTA of the cluster with the chunk
-    sums, all stop after two steps, and the next call is clean."""
-    w = gc.case("sel_timeout", "iid", 3, 4096, 64, 64, 32, "bf16")
-    dev, _ = workloads.make(w)
-    K = dev["K"].cuda()
-    wc.set_select_cluster(4)
-    wc.set_select_kernel(2)
-    assert wc.device_status() == 0
-    wc.force_select_timeout(1_000_000)
-    try:
-        S, F, rank, _ = wc.select(K, w.beta, w.r, w.pivot_seed, EPS)
-        assert wc.last_select_kernel() == 2
-        assert wc.device_status() == 5
-        assert torch.all(rank == 2)
-        assert torch.all(S[:, 2:] == -1)
-    finally:
-        wc.force_select_timeout(0)
-    S, F, rank, _ = wc.select(K, w.beta, w.r, w.pivot_seed, EPS)
-    assert wc.device_status() == 0
-    assert torch.all(rank == w.r)
-
-
 GS_SHAPES = [
     gc.case("gs_bh2_d128", "iid", 2, 16384, 64, 128, 64, "bf16"),
     gc.case("gs_bh8_d128", "iid", 8, 16384, 64, 128, 48, "bf16"),
@@ -172,9 +90,9 @@ GS_SHAPES = [
 
 @pytest.mark.parametrize("w", GS_SHAPES, ids=lambda w: w.name)
 def test_global_sync_form_matches_the_oracle(orc, w):
-    """The cp.async kernel in global-sync form (CTAs of an instance meet at a
-    counter barrier in the workspace): same checks as above, and the same
-    factorisation as the cluster form on the same pivots."""
+    """The global-sync form (CTAs of an instance meet at a counter barrier in
+    the workspace): same checks as above, and the cluster form draws the same
+    pivots."""
     dev, ex = workloads.make(w)
     K = dev["K"].cuda()
     own = orc.rpcholesky(ex["K"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)

@@ -4,11 +4,14 @@ them, or cannot afford a cudaMalloc in their loop), so they cannot pass the
 workspace that wildcat_attend takes.  Its scratch is a static 1 MiB device
 array inside the library.
 
-Checked through the C ABI against wildcat_attend on the same inputs, on two
-calls in a row with different shapes and dtypes (the second call reuses the
-array the first one wrote), plus the host-side size limit.  This file is
-collected last so that a run stopping at the first failure has already run
-every other test; it also passes alone in a fresh process."""
+Checked through the C ABI on two calls in a row with different shapes and
+dtypes (the second call reuses the array the first one wrote): against the
+fp64 oracle's attend on the same coreset at 1e-4 of the value range for both
+dtypes (the no-alloc variant runs the float32 CUDA-core kernel), and against
+wildcat_attend on the same inputs at the parity tolerance of the tests.  Plus
+the host-side size limit.  This file is collected last so that a run stopping
+at the first failure has already run every other test; it also passes alone
+in a fresh process."""
 import ctypes
 import math
 
@@ -32,7 +35,14 @@ def _coreset(dist, BH, n, m, d, r, dtype, seed):
     return w, (Q, K_S, rank, w.beta, V_S, wv, vmin, vmax)
 
 
+def _np64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
 def test_noalloc_matches_attend_on_two_calls():
+    import oracle
+
+    orc = oracle.get()
     calls = [
         _coreset("mixture16", 4, 784, 784, 64, 64, "bf16", 21),
         _coreset("iid", 3, 1000, 2333, 32, 40, "f32", 22),
@@ -41,12 +51,16 @@ def test_noalloc_matches_attend_on_two_calls():
         O_ref = wc.attend(*args)
         O_na = wc.attend_noalloc(*args)
         torch.cuda.synchronize()
-        vmin, vmax = args[6].cpu().numpy(), args[7].cpu().numpy()
-        span = np.maximum(vmax - vmin, 1e-30)[:, None, :]
+        Q, K_S, rank, beta, V_S, wv, vmin, vmax = args
+        lo, hi = _np64(vmin), _np64(vmax)
+        span = np.maximum(hi - lo, 1e-30)[:, None, :]
+        # the oracle's attend on exactly the coreset the device holds
+        O_orc = orc.attend(_np64(Q), _np64(K_S), _np64(V_S), _np64(wv), rank.cpu().numpy(), lo, hi, beta)
+        err_orc = np.max(np.abs(O_na.cpu().numpy() - O_orc) / span)
+        assert err_orc <= 1e-4, (w.dtype, err_orc)
+        # and wildcat_attend at the parity tolerance of the tests: 1e-4 of the value
+        # range for float32 inputs, 2e-2 for bfloat16 (bf16 runs on the tensor cores)
         err = np.max(np.abs(O_na.cpu().numpy() - O_ref.cpu().numpy()) / span)
-        # the parity tolerance of the tests: 1e-4 of the value range for float32
-        # inputs, 2e-2 for bfloat16 (wildcat_attend runs bf16 on the tensor
-        # cores; the no-alloc variant runs the CUDA-core kernel)
         assert err <= (1e-4 if w.dtype == "f32" else 2e-2), (w.dtype, err)
 
 
