@@ -110,6 +110,7 @@ Status launch_weights_inverse(const WeightsInverseRequest& q, cudaStream_t strea
 constexpr int kInverseMaxRank = 2048;
 // tensor-core F^T (V, 1) partials (weights_tc.cu)
 bool weights_tc_supported(int dtype, int d, int64_t n);
+int64_t weights_tc_keys_per_split(int64_t BH, int64_t n, int d, int r, int sms);
 Status launch_weights_tc(const float* F, const void* V, const int32_t* rank, int64_t BH, int64_t n, int d, int r,
                          int nsplit, int64_t keys_per_split, float* Ypart, cudaStream_t stream);
 

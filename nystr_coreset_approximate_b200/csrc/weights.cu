@@ -382,7 +382,17 @@ struct WeightsPlan {
     int max_split() const { return nsplit_k > nsplit_tc ? nsplit_k : nsplit_tc; }
 };
 
-WeightsPlan make_plan(int64_t BH, int64_t n, int r) {
+int sm_count_or_default() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    return sms;
+}
+
+WeightsPlan make_plan(int64_t BH, int64_t n, int d, int r) {
     WeightsPlan p{};
     p.nsplit_range = (int)std::max<int64_t>(1, std::min<int64_t>(64, ceil_div(296, std::max<int64_t>(1, BH))));
     p.nsplit_range = (int)std::min<int64_t>(p.nsplit_range, std::max<int64_t>(1, n / 64));
@@ -393,19 +403,15 @@ WeightsPlan make_plan(int64_t BH, int64_t n, int r) {
     sk = std::min<int64_t>(sk, 64);
     p.keys_per_split = round_up(ceil_div(n, sk), kFtyNK);
     p.nsplit_k = (int)ceil_div(n, p.keys_per_split);
-    // tensor-core tiles cover 128 factor columns; aim at ~4 CTAs per SM
-    const int64_t tiles_tc = ceil_div(r, 128) * BH;
-    int64_t st = ceil_div(4 * 148, tiles_tc);
-    st = std::max<int64_t>(1, std::min<int64_t>(st, std::max<int64_t>(1, n / 512)));
-    st = std::min<int64_t>(st, 128);
-    p.keys_per_split_tc = round_up(ceil_div(n, st), 64);
+    // tensor-core tiles cover 128 factor columns (weights_tc.cu chooses the key splits)
+    p.keys_per_split_tc = weights_tc_keys_per_split(BH, n, d, r, sm_count_or_default());
     p.nsplit_tc = (int)ceil_div(n, p.keys_per_split_tc);
     return p;
 }
 
 template <typename E, int D>
 Status run_weights(const WeightsRequest& q, cudaStream_t st) {
-    const WeightsPlan p = make_plan(q.BH, q.n, q.r);
+    const WeightsPlan p = make_plan(q.BH, q.n, D, q.r);
     Carve cv(q.ws, q.ws_bytes);
     float* part = static_cast<float*>(cv.take(sizeof(float) * q.BH * p.nsplit_range * 2 * D));
     float* Ypart = static_cast<float*>(cv.take(sizeof(float) * p.max_split() * q.BH * (int64_t)q.r * (D + 1)));
@@ -453,7 +459,7 @@ Status run_weights(const WeightsRequest& q, cudaStream_t st) {
 }  // namespace
 
 size_t weights_workspace_bytes(int64_t BH, int64_t n, int d, int r) {
-    const WeightsPlan p = make_plan(BH, n, r);
+    const WeightsPlan p = make_plan(BH, n, d, r);
     Carve cv(nullptr, 0);
     cv.take(sizeof(float) * BH * p.nsplit_range * 2 * d);
     cv.take(sizeof(float) * p.max_split() * BH * (int64_t)r * (d + 1));
@@ -462,13 +468,13 @@ size_t weights_workspace_bytes(int64_t BH, int64_t n, int d, int r) {
 }
 
 size_t value_range_workspace_bytes(int64_t BH, int64_t n, int d) {
-    const WeightsPlan p = make_plan(BH, n, 1);
+    const WeightsPlan p = make_plan(BH, n, d, 1);
     return sizeof(float) * BH * p.nsplit_range * 2 * d + 256;
 }
 
 Status launch_value_range(const void* V, int dtype, int64_t BH, int64_t n, int d, float* vmin, float* vmax,
                           void* ws, size_t ws_bytes, cudaStream_t st) {
-    const WeightsPlan p = make_plan(BH, n, 1);
+    const WeightsPlan p = make_plan(BH, n, d, 1);
     Carve cv(ws, ws_bytes);
     float* part = static_cast<float*>(cv.take(sizeof(float) * BH * p.nsplit_range * 2 * d));
     if (!cv.fits()) return Status::fail(4, "value range: workspace too small");

@@ -5,21 +5,35 @@
 // W (V, 1) = F_S^-T Y and Y = F^T (V, 1).  This kernel forms split-K partials
 // of Y for bfloat16 values; the back substitution in weights.cu sums them.
 //
-// One CTA (256 threads) per (128 factor columns, key slice, instance).  Per
-// chunk of 64 keys:
-//   A = F[j0 .. j0+127, keys] (fp32 in HBM) split into bf16 hi + lo parts,
-//       written K-major with 128-byte swizzling;
-//   B = [V | 1 | 0] for the same keys (d + 16 columns, bf16), MN-major: V's
-//       rows are copied as they are, the ones column and the zero padding
-//       are written in shared memory;
-//   two tcgen05.mma (hi and lo) per 16 keys accumulate Y in tensor memory
-//   (M = 128, N = d + 16, fp32).
-// The epilogue writes the partial Y rows of the CTA's factor columns.
+// One CTA per (128 factor columns, key range, instance); the key range is
+// walked in chunks of 64 keys.  Warp roles:
+//   warp 0     TMA: the chunk's factor rows F[j0 .. j0+127, keys] (fp32, two
+//              128 x 32 boxes, 128-byte swizzle) into a ring of NF stages
+//   warp 2     TMA: the chunk's value rows V[keys, 0 .. d) (bf16, MN-major
+//              boxes of 64 keys x 64 columns) into stage s of the AB ring
+//   warps 4-7  split each factor row into bf16 hi + lo parts, written K-major
+//              with the 128-byte swizzle into stage s of the AB ring (thread
+//              i converts row i); the factor stage is then released
+//   warp 1     one thread issues per chunk two tcgen05.mma groups (hi and lo
+//              parts of A, the same B = [V | 1 | 0]) into the fp32
+//              accumulator Y (M = 128, N = d + 16) in tensor memory
+// The ones column (and zero padding to d + 16) is written once per AB stage.
+// Keys past n read as zeros through the tensor maps, so they add nothing.
+// The hi/lo split keeps Y accurate to ~2^-17 relative while the factor is
+// read from HBM once.  Afterwards warps 4-7 write the CTA's partial Y rows.
 // Tiles starting at or past the instance's effective rank do no work (those
 // rows of F are zero and the solve never reads them).
+//
+// Every mbarrier wait is bounded (2 s) and gives up when another role gave
+// up; an expiry records WILDCAT_ERR_TIMEOUT in the device status word, the
+// CTA drains what it issued (bounded), frees its tensor memory and returns.
+// No load uses cluster multicast.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
+#include "tmap.h"
 
 namespace wildcat {
 
@@ -30,225 +44,263 @@ namespace {
 using namespace tc;
 constexpr int kWtThreads = 256;
 constexpr int kWtKC = 64;  // keys per chunk
+constexpr int kWtNF = 3;   // factor staging stages (fp32)
+constexpr int kWtNAB = 2;  // converted-operand stages (A hi / lo, B)
+constexpr unsigned long long kDrainNs = 100000000ull;
 
-template <int D>
-struct WtSmem {
-    static constexpr int NE = D + 16;
-    static constexpr int NB = (NE + 63) / 64;                          // 64-column MN blocks of B
-    static constexpr size_t ahi = 0;                                   // 128 x 64 bf16
-    static constexpr size_t alo = ahi + 128 * 128;
-    static constexpr size_t b = alo + 128 * 128;                       // NB blocks of 64 keys x 128 B
-    static constexpr size_t stage = b + (size_t)NB * kWtKC * 128;      // one pipeline stage
-    static constexpr size_t bar = 2 * stage;                           // two stages, then the barriers
-    static constexpr size_t total = bar + 64 + 1024;
-    static constexpr unsigned tmem_cols = 256;
+struct WtBars {
+    uint64_t f_full[kWtNF], f_empty[kWtNF];
+    uint64_t a_full[kWtNAB], b_full[kWtNAB], ab_empty[kWtNAB];
+    uint64_t done;
+    unsigned tmem_base;
+    int abort;
 };
 
 template <int D>
-__global__ void __launch_bounds__(kWtThreads)
-    weights_tc_kernel(const float* __restrict__ F, const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ rank,
-                      int64_t n, int r, int64_t keys_per_split, float* __restrict__ Ypart, int64_t BH) {
-    using L = WtSmem<D>;
-    constexpr int NE = L::NE;
-    const int64_t b = blockIdx.z;
+struct WtCfg {
+    static constexpr int NE = D + 16;                          // value columns + ones column + zero padding
+    static constexpr int NBLK = D / 64 + 1;                    // 64-column MN blocks of B (the last holds the ones)
+    static constexpr uint32_t f_bytes = 2 * 128 * 128;         // 128 rows x 64 keys fp32: two 128-byte boxes
+    static constexpr uint32_t a_bytes = 128 * 128;             // one part: 128 rows x 64 keys bf16
+    static constexpr uint32_t b_bytes = NBLK * kWtKC * 128;    // 64 keys x NBLK * 64 columns bf16
+    static constexpr uint32_t v_bytes = (D / 64) * kWtKC * 128;  // the V part of B (what the TMA fills)
+    static constexpr uint32_t ab_bytes = 2 * a_bytes + b_bytes;
+    static constexpr uint32_t off_f = 0;
+    static constexpr uint32_t off_ab = off_f + kWtNF * f_bytes;
+    static constexpr uint32_t off_bar = off_ab + kWtNAB * ab_bytes;
+    static constexpr uint32_t total = off_bar + (uint32_t)sizeof(WtBars);
+    static constexpr unsigned tmem_cols = 256;
+    static_assert(NE <= 256, "accumulator columns");
+    static_assert(total <= 232448, "shared memory");
+};
+
+template <int D>
+__global__ void __launch_bounds__(kWtThreads, 1)
+    weights_tc_kernel(const __grid_constant__ CUtensorMap tmF, const __grid_constant__ CUtensorMap tmV,
+                      const int32_t* __restrict__ rank, int64_t n, int r, int64_t keys_per_split,
+                      float* __restrict__ Ypart, int64_t BH) {
+    using C = WtCfg<D>;
+    constexpr int NE = C::NE;
+    const int b = blockIdx.z;
     const int split = blockIdx.y;
     const int j0 = blockIdx.x * 128;
     if (j0 >= rank[b]) return;  // uniform: the whole CTA leaves before any allocation
 
-    extern __shared__ unsigned char sm_raw[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + L::bar);  // one per stage
-    unsigned* tmem_slot = reinterpret_cast<unsigned*>(sm + L::bar + 16);
-    const int tid = threadIdx.x, warp = tid >> 5;
+    extern __shared__ __align__(1024) unsigned char sm[];
+    const unsigned sbase = smem_u32(sm);
+    WtBars* bars = reinterpret_cast<WtBars*>(sm + C::off_bar);
+    volatile int* abort_flag = &bars->abort;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    const int64_t l_begin = split * keys_per_split;
+    const int64_t l_end = min(n, l_begin + keys_per_split);
+    const int nchunks = l_end > l_begin ? (int)ceil_div(l_end - l_begin, kWtKC) : 0;
 
     if (tid == 0) {
-        mbar_init(&mbar[0], 1);
-        mbar_init(&mbar[1], 1);
+        for (int s = 0; s < kWtNF; ++s) {
+            mbar_init(&bars->f_full[s], 1);
+            mbar_init(&bars->f_empty[s], 4);  // one arrival per converter warp
+        }
+        for (int s = 0; s < kWtNAB; ++s) {
+            mbar_init(&bars->a_full[s], 4);  // one arrival per converter warp
+            mbar_init(&bars->b_full[s], 1);
+            mbar_init(&bars->ab_empty[s], 1);
+        }
+        mbar_init(&bars->done, 1);
+        bars->abort = (sbase & 1023u) ? 1 : 0;  // the swizzled layouts need a 1024-byte aligned base
+        if (sbase & 1023u) atomicExch(&g_weights_status, 3);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(L::tmem_cols)
+    // the ones column (value column d) and the zero padding of every AB stage's B
+    for (int e = tid; e < kWtNAB * kWtKC; e += kWtThreads) {
+        const int s = e / kWtKC, kr = e % kWtKC;
+        unsigned char* blk = sm + C::off_ab + s * C::ab_bytes + 2 * C::a_bytes + (D / 64) * (kWtKC * 128);
+        const __nv_bfloat16 one = __float2bfloat16_rn(1.f);
+        uint4 c0 = make_uint4((uint32_t)(*reinterpret_cast<const uint16_t*>(&one)), 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(blk + swz(kr, 0)) = c0;
+        *reinterpret_cast<uint4*>(blk + swz(kr, 1)) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_async_smem();
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&bars->tmem_base)),
+                     "r"(C::tmem_cols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const unsigned tmem = *tmem_slot;
-    constexpr uint32_t idesc = idesc_bf16_bmn(128, NE);
-
-    const int64_t l_begin = split * keys_per_split;
-    const int64_t l_end = min(n, l_begin + keys_per_split);
-    const int nchunks = l_end > l_begin ? (int)ceil_div(l_end - l_begin, kWtKC) : 0;
-    const float* Fb = F + b * (int64_t)r * n;
-    const __nv_bfloat16* Vb = V + b * n * D;
-    const int row = tid >> 1, half = tid & 1;  // A: factor row j0 + row, 32 keys from half * 32
-    const int j = j0 + row;
-
-    // F rows of chunk c into registers (global loads left in flight)
-    auto load_a = [&](int c, float (&v)[32]) {
-        const int64_t l0 = l_begin + (int64_t)c * kWtKC;
-        const float* src = Fb + (int64_t)j * n + l0 + half * 32;
-        const bool full = j < r && l0 + half * 32 + 32 <= l_end;
-        if (full) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const float4 x = __ldcs(reinterpret_cast<const float4*>(src) + k);
-                v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
-            }
-        } else {
-#pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                const int64_t l = l0 + half * 32 + k;
-                v[k] = (j < r && l < l_end) ? __ldcs(Fb + (int64_t)j * n + l) : 0.f;
-            }
-        }
-    };
-    // B of chunk c into stage st: V rows (MN-major: key = row, 64 value
-    // columns per 128-byte row) by cp.async, then the ones column and zeros
-    auto load_b = [&](int c, int st) {
-        const int64_t l0 = l_begin + (int64_t)c * kWtKC;
-        unsigned char* sb = sm + st * L::stage + L::b;
-        const unsigned sB = smem_u32(sb);
-        for (int e = tid; e < kWtKC * (D / 8); e += kWtThreads) {
-            const int kr = e / (D / 8), c8 = e % (D / 8);  // key row, 16-byte chunk along d
-            const int64_t l = l0 + kr;
-            const bool okl = l < l_end;
-            const unsigned dst = (c8 >> 3) * (kWtKC * 128) + swz(kr, c8 & 7);
-            cp_async16_zfill(sB + dst, Vb + (okl ? l : l0) * D + c8 * 8, okl);
-        }
-        cp_async_commit();
-        for (int kr = tid; kr < kWtKC; kr += kWtThreads) {
-            const bool okl = l0 + kr < l_end;
-            const int mb = D / 64;  // block holding columns D .. D + 15 (chunks 0 and 1)
-            const __nv_bfloat16 one = __float2bfloat16_rn(okl ? 1.f : 0.f);
-            uint4 c0 = make_uint4(0u, 0u, 0u, 0u);
-            c0.x = (uint32_t)(*reinterpret_cast<const uint16_t*>(&one));
-            *reinterpret_cast<uint4*>(sb + mb * (kWtKC * 128) + swz(kr, 0)) = c0;
-            *reinterpret_cast<uint4*>(sb + mb * (kWtKC * 128) + swz(kr, 1)) = make_uint4(0u, 0u, 0u, 0u);
-        }
+    const unsigned tmem = bars->tmem_base;
+    const bool go = *abort_flag == 0;
+    auto give_up = [&]() {
+        *abort_flag = 1;
+        atomicExch(&g_weights_status, 5);
     };
 
-    // Two stages: while the tensor cores work on chunk c, the V rows of chunk
-    // c + 1 land by cp.async and the F rows of chunks c + 1 and c + 2 are in
-    // flight into registers (two register sets, the loop unrolled by two).
-    // Stage s is rewritten only after the MMA that read it (chunk c - 1 for
-    // B, chunk c - 2 for A) has committed on mbar[s].
-    bool ok = true;
-    int issued = 0;  // MMA commits so far (commit k arrives on mbar[k & 1], phase k >> 1)
-    auto step = [&](int c, float (&v)[32]) -> bool {
-        const int st = c & 1;
-        if (c >= 1) {
-            // chunk c - 1's MMA has read stage st ^ 1: free it for chunk c + 1
-            const bool w = mbar_wait(&mbar[(c - 1) & 1], ((c - 1) >> 1) & 1);
-            if (__syncthreads_or(!w)) return false;
+    if (warp == 0) {
+        // ---------------------------------------------------- factor rows (TMA)
+        if (lane == 0 && go) {
+            prefetch_tmap(&tmF);
+            int c = 0;
+            bool ok = true;
+            for (; c < nchunks; ++c) {
+                const int s = c % kWtNF;
+                if (c >= kWtNF &&
+                    !(ok = mbar_wait_suspend(&bars->f_empty[s], (unsigned)((c / kWtNF) - 1) & 1u, abort_flag)))
+                    break;
+                mbar_expect_tx(&bars->f_full[s], C::f_bytes);
+                const int x = (int)(l_begin + (int64_t)c * kWtKC);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    tma_load_3d(sbase + C::off_f + s * C::f_bytes + h * (128 * 128), &tmF, x + 32 * h, j0, b,
+                                &bars->f_full[s]);
+            }
+            if (!ok) give_up();
+            if (*abort_flag)
+                for (int k = std::max(0, c - kWtNF); k < c; ++k)
+                    mbar_wait(&bars->f_full[k % kWtNF], (unsigned)(k / kWtNF) & 1u, kDrainNs);
+        }
+    } else if (warp == 2) {
+        // ----------------------------------------------------- value rows (TMA)
+        if (lane == 0 && go) {
+            prefetch_tmap(&tmV);
+            int c = 0;
+            bool ok = true;
+            for (; c < nchunks; ++c) {
+                const int s = c % kWtNAB;
+                if (c >= kWtNAB &&
+                    !(ok = mbar_wait_suspend(&bars->ab_empty[s], (unsigned)((c / kWtNAB) - 1) & 1u, abort_flag)))
+                    break;
+                mbar_expect_tx(&bars->b_full[s], C::v_bytes);
+                const int y = (int)(l_begin + (int64_t)c * kWtKC);
+#pragma unroll
+                for (int blk = 0; blk < D / 64; ++blk)
+                    tma_load_3d(sbase + C::off_ab + s * C::ab_bytes + 2 * C::a_bytes + blk * (kWtKC * 128), &tmV,
+                                64 * blk, y, b, &bars->b_full[s]);
+            }
+            if (!ok) give_up();
+            if (*abort_flag)
+                for (int k = std::max(0, c - kWtNAB); k < c; ++k)
+                    mbar_wait(&bars->b_full[k % kWtNAB], (unsigned)(k / kWtNAB) & 1u, kDrainNs);
+        }
+    } else if (warp == 1) {
+        // -------------------------------------------------------- tensor cores
+        if (lane == 0 && go) {
+            constexpr uint32_t idesc = idesc_bf16_bmn(128, NE);
+            bool ok = true;
+            int c = 0;
+            for (; c < nchunks; ++c) {
+                const int s = c % kWtNAB;
+                const unsigned ph = (unsigned)(c / kWtNAB) & 1u;
+                if (!(ok = mbar_wait_suspend(&bars->a_full[s], ph, abort_flag) &&
+                           mbar_wait_suspend(&bars->b_full[s], ph, abort_flag)))
+                    break;
+                tc_fence_after();
+                const unsigned st = sbase + C::off_ab + s * C::ab_bytes;
+                const unsigned sB = st + 2 * C::a_bytes;
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+#pragma unroll
+                    for (int kk = 0; kk < kWtKC / 16; ++kk)
+                        mma_bf16(tmem, umma_desc(st + part * C::a_bytes + kk * 32),
+                                 umma_desc_mn(sB + kk * 16 * 128, kWtKC * 128), idesc, (c > 0 || part > 0 || kk > 0) ? 1 : 0);
+                }
+                mma_commit(&bars->ab_empty[s]);
+            }
+            if (!ok) give_up();
+            mma_commit(&bars->done);  // every product issued has finished when this arrives
+            mbar_wait(&bars->done, 0, ok ? kWaitLimitNs : kDrainNs);
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------- hi / lo split, then Y out
+        const int row = tid - 128;  // factor column j0 + row = TMEM lane
+        bool ok = go;
+        for (int c = 0; c < nchunks && ok; ++c) {
+            const int sf = c % kWtNF, sa = c % kWtNAB;
+            const bool got = mbar_wait_suspend(&bars->f_full[sf], (unsigned)(c / kWtNF) & 1u, abort_flag) &&
+                             (c < kWtNAB ||
+                              mbar_wait_suspend(&bars->ab_empty[sa], (unsigned)((c / kWtNAB) - 1) & 1u, abort_flag));
+            ok = __all_sync(0xffffffffu, got);
+            if (!ok) break;
+            const unsigned char* frow = sm + C::off_f + sf * C::f_bytes + row * 128;
+            unsigned char* ahi = sm + C::off_ab + sa * C::ab_bytes + row * 128;
+            unsigned char* alo = ahi + C::a_bytes;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {  // 8 keys per 16-byte piece of the bf16 row
+                const unsigned char* fb = frow + (k >> 2) * (128 * 128);
+                const int c0 = (2 * k) & 7;  // first fp32 piece (4 keys) of this group in its box
+                const float4 x0 = *reinterpret_cast<const float4*>(fb + ((c0 ^ (row & 7)) << 4));
+                const float4 x1 = *reinterpret_cast<const float4*>(fb + (((c0 + 1) ^ (row & 7)) << 4));
+                const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(xs[2 * e], xs[2 * e + 1]);
+                    const float2 hf = __bfloat1622float2(h);
+                    const __nv_bfloat162 g = __floats2bfloat162_rn(xs[2 * e] - hf.x, xs[2 * e + 1] - hf.y);
+                    hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+                    lo[e] = *reinterpret_cast<const uint32_t*>(&g);
+                }
+                const unsigned off = (unsigned)((k ^ (row & 7)) << 4);
+                *reinterpret_cast<uint4*>(ahi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(alo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            fence_async_smem();  // the generic-proxy writes become visible to the tensor cores
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars->f_empty[sf]);
+                mbar_arrive(&bars->a_full[sa]);
+            }
+        }
+        if (!ok && lane == 0) give_up();
+        // -- the CTA's partial Y rows (factor columns j0 + row) --
+        if (ok && nchunks > 0) ok = __all_sync(0xffffffffu, mbar_wait_suspend(&bars->done, 0, abort_flag));
+        const int je = j0 + row;
+        if (ok) {
             tc_fence_after();
-        }
-        if (c + 1 < nchunks) load_b(c + 1, st ^ 1);
-        // A of chunk c: bf16 hi / lo, K-major, 128-byte swizzle
-        unsigned char* sa = sm + st * L::stage;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float a0 = v[8 * q + 2 * e], a1 = v[8 * q + 2 * e + 1];
-                const __nv_bfloat162 h = __floats2bfloat162_rn(a0, a1);
-                const float2 hf = __bfloat1622float2(h);
-                const __nv_bfloat162 g = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
-                hi[e] = *reinterpret_cast<const uint32_t*>(&h);
-                lo[e] = *reinterpret_cast<const uint32_t*>(&g);
-            }
-            const unsigned off = swz(row, half * 4 + q);
-            *reinterpret_cast<uint4*>(sa + L::ahi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4*>(sa + L::alo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        }
-        if (c + 2 < nchunks) load_a(c + 2, v);
-        if (c + 1 < nchunks)
-            cp_async_wait_group<1>();  // chunk c's V rows (chunk c + 1's may still fly)
-        else
-            cp_async_wait_all();
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (tid == 0) {
-            const unsigned sAhi = smem_u32(sa + L::ahi), sAlo = smem_u32(sa + L::alo), sB = smem_u32(sa + L::b);
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const unsigned sap = part ? sAlo : sAhi;
-#pragma unroll
-                for (int kk = 0; kk < kWtKC / 16; ++kk)
-                    mma_bf16(tmem, umma_desc(sap + kk * 32), umma_desc_mn(sB + kk * 16 * 128, kWtKC * 128), idesc,
-                             (c > 0 || part > 0 || kk > 0) ? 1 : 0);
-            }
-            mma_commit(&mbar[st]);
-        }
-        ++issued;
-        return true;
-    };
-    float v0[32], v1[32];
-    if (nchunks > 0) {
-        load_b(0, 0);
-        load_a(0, v0);
-        if (nchunks > 1) load_a(1, v1);
-    }
-    for (int c = 0; c < nchunks; c += 2) {
-        if (!step(c, v0)) { ok = false; break; }
-        if (c + 1 < nchunks && !step(c + 1, v1)) { ok = false; break; }
-    }
-    // the last commit covers every MMA issued before it
-    if (issued > 0) {
-        const int k = issued - 1;
-        const bool w = mbar_wait(&mbar[k & 1], (k >> 1) & 1);
-        if (__syncthreads_or(!w)) ok = false;
-        tc_fence_after();
-    }
-    // -- epilogue: warps 0-3 read their 32 TMEM lanes (= factor columns j0 + lane row) --
-    if (ok && warp < 4 && issued > 0) {
-        const int rowe = warp * 32 + (tid & 31);
-        const int je = j0 + rowe;
-        float* y = Ypart + (((int64_t)split * BH + b) * r + je) * (D + 1);
-#pragma unroll 1
-        for (int c0 = 0; c0 < D + 16; c0 += 16) {
-            float vv[16];
-            tmem_ld16(tmem + ((unsigned)(warp * 32) << 16) + c0, vv);
-            if (je < r) {
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    if (c0 + k <= D) y[c0 + k] = vv[k];
-            }
-        }
-    } else if (ok && warp < 4 && issued == 0) {
-        const int je = j0 + warp * 32 + (tid & 31);
-        if (je < r) {
             float* y = Ypart + (((int64_t)split * BH + b) * r + je) * (D + 1);
-            for (int c = 0; c <= D; ++c) y[c] = 0.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < NE; c0 += 16) {
+                float vv[16];
+                if (nchunks > 0) {
+                    tmem_ld16(tmem + ((unsigned)(32 * (warp & 3)) << 16) + c0, vv);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) vv[k] = 0.f;
+                }
+                if (je < r) {
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        if (c0 + k <= D) y[c0 + k] = vv[k];
+                }
+            }
         }
     }
-    if (!ok) {
-        if (tid == 0) atomicExch(&g_weights_status, 5);
-        // bounded wait for the last MMA still in flight before its memory is freed
-        if (issued > 0) mbar_wait(&mbar[(issued - 1) & 1], ((issued - 1) >> 1) & 1);
-        cp_async_wait_all();
-    }
+
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(L::tmem_cols) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::tmem_cols) : "memory");
     }
 }
 
 template <int D>
 Status run_wt(const float* F, const void* V, const int32_t* rank, int64_t BH, int64_t n, int r, int nsplit,
               int64_t keys_per_split, float* Ypart, cudaStream_t st) {
-    using L = WtSmem<D>;
-    cudaError_t e = cudaFuncSetAttribute(weights_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::total);
+    using C = WtCfg<D>;
+    CUtensorMap tmF, tmV;
+    const bool ok =
+        make_tmap_3d(&tmF, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, F, (uint64_t)n, (uint64_t)r, (uint64_t)BH, n * 4ull,
+                     (uint64_t)r * n * 4ull, 32, 128) &&
+        make_tmap_3d(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, V, D, (uint64_t)n, (uint64_t)BH, D * 2ull,
+                     (uint64_t)n * D * 2ull, 64, kWtKC);
+    if (!ok) return Status::fail(3, "weights_tc: tensor map encoding failed");
+    cudaError_t e = cudaFuncSetAttribute(weights_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::total);
     if (e != cudaSuccess) return Status::cuda(e, "weights_tc: smem attribute");
-    weights_tc_kernel<D><<<dim3((unsigned)ceil_div(r, 128), nsplit, (unsigned)BH), kWtThreads, L::total, st>>>(
-        F, static_cast<const __nv_bfloat16*>(V), rank, n, r, keys_per_split, Ypart, BH);
+    weights_tc_kernel<D><<<dim3((unsigned)ceil_div(r, 128), nsplit, (unsigned)BH), kWtThreads, C::total, st>>>(
+        tmF, tmV, rank, n, r, keys_per_split, Ypart, BH);
     e = cudaGetLastError();
     if (e != cudaSuccess) return Status::cuda(e, "weights_tc launch");
     return Status::ok();
@@ -259,8 +311,34 @@ Status run_wt(const float* F, const void* V, const int32_t* rank, int64_t BH, in
 // bf16 values, d in {64, 128}, and n % 4 == 0 (16-byte aligned factor rows).
 bool weights_tc_supported(int dtype, int d, int64_t n) { return dtype == 1 && (d == 64 || d == 128) && n % 4 == 0; }
 
+// Key splits of the tensor-core kernel.  One CTA runs per SM at a time, so
+// the time is about (waves of CTAs) x (chunks per CTA); each split also
+// writes, and the solve reads back, one partial Y of every column tile.  The
+// split count minimising the sum (in units of one chunk's HBM traffic per SM)
+// is taken, keeping at least 8 chunks of 64 keys per CTA.
+int64_t weights_tc_keys_per_split(int64_t BH, int64_t n, int d, int r, int sms) {
+    const int64_t tiles = ceil_div(r, 128) * BH;
+    const int64_t chunks = ceil_div(n, kWtKC);
+    const double chunk_bytes = 128.0 * kWtKC * 4 + (double)kWtKC * d * 2;  // F and V per chunk
+    const double y_per_split = (double)tiles * 128 * (d + 1) * 4 * 2 / sms / chunk_bytes;
+    int64_t best_ns = 1;
+    double best = -1.0;
+    for (int64_t ns = 1; ns <= 512 && ns <= chunks; ++ns) {
+        const int64_t cpc = ceil_div(chunks, ns);
+        if (ns > 1 && cpc < 8) break;
+        const double t = (double)ceil_div(tiles * ns, sms) * cpc + ns * y_per_split;
+        if (best < 0 || t < best) {
+            best = t;
+            best_ns = ns;
+        }
+    }
+    return ceil_div(chunks, best_ns) * kWtKC;
+}
+
 Status launch_weights_tc(const float* F, const void* V, const int32_t* rank, int64_t BH, int64_t n, int d, int r,
                          int nsplit, int64_t keys_per_split, float* Ypart, cudaStream_t st) {
+    if ((reinterpret_cast<uintptr_t>(F) & 15u) || (reinterpret_cast<uintptr_t>(V) & 15u))
+        return Status::fail(1, "weights_tc: F and V must be 16-byte aligned");
     switch (d) {
         case 64: return run_wt<64>(F, V, rank, BH, n, r, nsplit, keys_per_split, Ypart, st);
         case 128: return run_wt<128>(F, V, rank, BH, n, r, nsplit, keys_per_split, Ypart, st);
