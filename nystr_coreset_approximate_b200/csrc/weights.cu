@@ -31,31 +31,61 @@ constexpr int kRangeThreads = 256;
 template <typename E, int D>
 __global__ void __launch_bounds__(kRangeThreads) colrange_partial(const typename E::T* V, int64_t n,
                                                                   int64_t rows_per_split, float* part) {
-    // part [BH, nsplit, 2, D]
+    // part [BH, nsplit, 2, D].  Each thread covers 8 consecutive columns
+    // (one 16-byte load per row for bf16, two for fp32) of every RS-th row,
+    // four rows in flight; the RS row slots are reduced in shared memory.
+    constexpr int CPT = 8;                      // columns per thread
+    constexpr int TPR = D / CPT;                // threads per row
+    constexpr int RS = kRangeThreads / TPR;     // row slots
     const int64_t b = blockIdx.y;
     const int split = blockIdx.x, nsplit = gridDim.x;
-    constexpr int RS = kRangeThreads / D;  // row slots
-    const int c = threadIdx.x % D, rs = threadIdx.x / D;
+    const int c0 = (threadIdx.x % TPR) * CPT, rs = threadIdx.x / TPR;
     const int64_t l0 = split * rows_per_split, l1 = min(n, l0 + rows_per_split);
-    float lo = INFINITY, hi = -INFINITY;
-    const typename E::T* Vb = V + b * n * D;
-    for (int64_t l = l0 + rs; l < l1; l += RS) {
-        const float v = E::to_float(Vb[l * D + c]);
-        lo = fminf(lo, v);
-        hi = fmaxf(hi, v);
+    float lo[CPT], hi[CPT];
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) {
+        lo[k] = INFINITY;
+        hi[k] = -INFINITY;
     }
-    __shared__ float slo[kRangeThreads], shi[kRangeThreads];
-    slo[threadIdx.x] = lo;
-    shi[threadIdx.x] = hi;
+    const typename E::T* Vb = V + b * n * D + c0;
+    int64_t l = l0 + rs;
+    for (; l + 3 * RS < l1; l += 4 * RS) {
+        float v[4][CPT];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) load8(Vb + (l + u * RS) * D, v[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int k = 0; k < CPT; ++k) {
+                lo[k] = fminf(lo[k], v[u][k]);
+                hi[k] = fmaxf(hi[k], v[u][k]);
+            }
+    }
+    for (; l < l1; l += RS) {
+        float v[CPT];
+        load8(Vb + l * D, v);
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) {
+            lo[k] = fminf(lo[k], v[k]);
+            hi[k] = fmaxf(hi[k], v[k]);
+        }
+    }
+    __shared__ float slo[RS][D], shi[RS][D];
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) {
+        slo[rs][c0 + k] = lo[k];
+        shi[rs][c0 + k] = hi[k];
+    }
     __syncthreads();
-    if (rs == 0) {
-        for (int k = 1; k < RS; ++k) {
-            lo = fminf(lo, slo[k * D + c]);
-            hi = fmaxf(hi, shi[k * D + c]);
+    for (int c = threadIdx.x; c < D; c += kRangeThreads) {
+        float a = INFINITY, z = -INFINITY;
+        for (int k = 0; k < RS; ++k) {
+            a = fminf(a, slo[k][c]);
+            z = fmaxf(z, shi[k][c]);
         }
         float* p = part + ((b * nsplit + split) * 2) * D;
-        p[c] = lo;
-        p[D + c] = hi;
+        p[c] = a;
+        p[D + c] = z;
     }
 }
 
