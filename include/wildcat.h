@@ -279,7 +279,9 @@ wildcat_status wildcat_attend_noalloc(const void* Q, const void* K_S, int dtype,
  * eps as in wildcat_select.
  *
  *   Q [BH, m, d], K and V [BH, n, d] (dtype `dtype`); O out [BH, m, d] float32
- *   S_out [BH, r] int32 and rank_out [BH] int32: optional copies (or NULL)
+ *   S_out [BH, r] int32 and rank_out [BH] int32: optional outputs (or NULL);
+ *     when given, the select writes them in place and the weights and attend
+ *     stages read them from there, so they must not overlap any other argument
  *   workspace >= wildcat_forward_workspace_size(BH, m, n, d, r, dtype) bytes
  */
 size_t wildcat_forward_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int dtype);

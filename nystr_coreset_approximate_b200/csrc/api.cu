@@ -425,10 +425,14 @@ wildcat_status wildcat_forward(const void* Q, const void* K, const void* V, int 
         return bad(1, "%s: Q, K and V must be 16-byte aligned", who);
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
     Carve cv(workspace, ws_bytes);
-    const ForwardLayout L = carve_forward(cv, BH, m, n, d, r, dtype);
+    ForwardLayout L = carve_forward(cv, BH, m, n, d, r, dtype);
     if (!cv.fits()) return bad(4, "%s: workspace too small", who);
     if (inst0 < 0 || inst0 + BH > 4294967296LL) return bad(1, "%s: inst0 must satisfy 0 <= inst0, inst0 + BH <= 2^32", who);
-    return forward_impl(Q, K, V, dtype, BH, m, n, d, beta, r, seed, inst0, eps, O, S_out, rank_out, L,
+    // the select writes the caller's pivot and rank arrays in place, and the
+    // later stages read them from there (no copy at the end)
+    if (S_out) L.S = S_out;
+    if (rank_out) L.rank = rank_out;
+    return forward_impl(Q, K, V, dtype, BH, m, n, d, beta, r, seed, inst0, eps, O, nullptr, nullptr, L,
                         static_cast<cudaStream_t>(stream));
 }
 

@@ -9,31 +9,42 @@
 // the same).  The row's shift comes from the query tile already in shared
 // memory, so no separate pass over Q is needed.
 //
-// Persistent CTAs (one per SM) walk units of two 128-query tiles of one
-// instance; each unit walks the coreset in chunks of 128 rows.  Warp roles:
-//   warp 0     producer: TMA loads of each unit's two Q tiles (the next
-//              unit's tile as soon as the current one's last GEMM1 is done),
-//              of each K_S chunk and of each V_S^T chunk plus its slice of w,
-//              into 128-byte-swizzled shared memory, NS stages per operand
+// Persistent CTAs (one per SM, 16 warps) walk units of two 128-query tiles
+// of one instance; each unit walks the coreset in chunks of 128 rows.  Warp
+// roles (setmaxnreg gives the softmax and epilogue groups the registers):
+//   warp 0     producer (one thread): TMA loads of each unit's two Q tiles
+//              (a slot's next tile as soon as its last GEMM1 and its row norms
+//              are done), of each K_S chunk and of each V_S^T chunk plus its
+//              slice of w, into 128-byte-swizzled shared memory, NS stages
 //   warp 1     tensor cores (one thread issues):
 //                GEMM1  S_t = Q_t K_S,c^T   tcgen05.mma kind::f16, M = 128,
 //                       N = 128, both operands in shared memory, fp32 in TMEM
 //                GEMM2  O_t += P_t V_S,c    A operand P_t read from TMEM
 //                       (where the softmax threads left it), N = d
-//              in the order G2(c,0) G1(c+1,0) G2(c,1) G1(c+1,1): while one
-//              tile's scores are exponentiated the other tile's products run;
-//              the next unit's first GEMM1s run during this unit's epilogue
-//   warps 2-5  tile 0, warps 6-9 tile 1: thread i of the group owns query row
-//              i (= TMEM lane i).  Per chunk it reads its 128 scores with
-//              tcgen05.ld (the next 32 columns in flight while it works on
-//              these), forms P = 2^(s beta log2e - m_i beta log2e) on the
-//              special-function unit, rounds P once to bf16, writes the
+//              as one stream per tile slot, G2(c, t) then G1(c + 1, t), the two
+//              slots alternating: while one slot's scores are exponentiated
+//              the other slot's products run, and a slot's next unit follows
+//              its last chunk without a break
+//   warps 2-3  idle (they keep the four groups below one warp per SM
+//              sub-partition each)
+//   warps 4-7  softmax of slot 0, warps 8-11 of slot 1: thread i of the group
+//              owns query row i (= TMEM lane i).  Per unit it forms its row's
+//              shift from the Q tile in shared memory; per chunk it reads its
+//              128 scores with tcgen05.ld (the next 32 columns in flight while
+//              it works on these), forms P = 2^(s beta log2e - m_i beta log2e)
+//              on the special-function unit, rounds P once to bf16, writes the
 //              packed pairs back over the scores (tcgen05.st) for GEMM2 and
-//              accumulates D = sum_l P_l w_l in fp32 (packed fp32x2 FMAs).
-//              After the unit's last chunk it reads its row of O from TMEM
-//              32 columns at a time, forms clip(N / D, v_min, v_max), stages
-//              the 128 x 32 box in its own shared-memory buffer and stores
-//              it with TMA.
+//              accumulates D = sum_l P_l w_l in fp32 (packed fp32x2 FMAs); at
+//              the unit's end it leaves D in shared memory
+//   warps 12-15 epilogue: per tile it reads the rows of O from TMEM (half the
+//              columns at a time, releasing the accumulator after the second
+//              half), forms clip(N / D, v_min, v_max), stages 128 x 32 boxes
+//              in two shared-memory buffers and stores them with TMA
+// The tensor pipe bounds the kernel: on this part one 128 x 128 x 16 MMA
+// takes about 124 cycles with both operands in shared memory and 136 with
+// A in tensor memory (a probe of back-to-back MMAs: 4.2 and 3.9 kflop per
+// clock per SM, against about 6.2 for a 128 x 256 x 16 MMA), so a unit's 16
+// products need about 16.6k cycles, and a unit takes about 20k.
 // Tensor memory (512 columns): O_0, O_1 (d columns each), S_0, S_1 (128 each).
 // V_S and w are prepared per call: V_S^T rounded to bf16 (its bf16 rounding
 // leaves the plug-in estimator within 6.1e-4 of the value range on every

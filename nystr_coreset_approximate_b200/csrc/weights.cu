@@ -14,9 +14,10 @@
 //                CUDA cores (float32 values, or n % 4 != 0); bf16 values use the
 //                tensor-core kernel of weights_tc.cu
 //   gather_fs    F_S[a, j] = F[j, S_a] for j <= a (pivot rows of the factor)
-//   trsm_warp_kernel / trsm_kernel  sum the split-K partials and
-//                back-substitute F_S^T X = Y (one warp per column for
-//                r <= 1024, else blocked by 32 pivots)
+//   trsm_warp_kernel / trsm_stream_kernel / trsm_kernel  sum the split-K
+//                partials and back-substitute F_S^T X = Y (one warp per column
+//                for r <= 1024, F_S read from shared memory; else blocked by 32
+//                pivots)
 #include <algorithm>
 
 #include "common.cuh"
@@ -250,13 +251,13 @@ __global__ void __launch_bounds__(kTrsmThreads) trsm_kernel(const float* Ypart, 
     }
 }
 
-// Back substitution with one warp per right-hand column (r <= kTrsmWarpMaxR).
-// When the pivot block fits in shared memory (r <= ~220) the CTA first sums
-// the split-K partials of its 16 columns (coalesced over the columns) and
-// copies F_S there, so the per-pivot row reads stay on chip; otherwise each
-// warp sums its own column and reads the rows from global memory.  Then
-// pivot a (bottom up) gives x_a = y_a / F_S[a, a], and the lanes subtract
-// F_S[a, j] x_a from every y_j, j < a, reading row a contiguously.
+// Back substitution with one warp per right-hand column (r <= kTrsmWarpMaxR),
+// kTrsmWarps columns per CTA.  The CTA sums the split-K partials of its
+// columns (coalesced over the columns); F_S is then read from shared memory,
+// copied whole when it fits (r <= ~220), else streamed a sub-block of pivots
+// at a time.  Pivot a (bottom up) gives x_a = y_a / F_S[a, a], and the lanes
+// subtract F_S[a, j] x_a from every y_j, j < a, reading row a contiguously;
+// lane l holds y[32 m + l] in registers.
 constexpr int kTrsmWarps = 8;
 constexpr int kTrsmWarpMaxR = 1024;
 constexpr int kTrsmRegs = kTrsmWarpMaxR / 32;  // y values per lane
@@ -266,130 +267,41 @@ inline bool trsm_fs_in_smem(int r) {
     return sizeof(float) * ((size_t)kTrsmWarps * r + (size_t)r * r) <= kTrsmSmemCap;
 }
 
-template <bool FS_SMEM>
-__global__ void __launch_bounds__(kTrsmWarps * 32) trsm_warp_kernel(const float* __restrict__ Ypart, int nsplit,
-                                                                    const float* __restrict__ FS,
-                                                                    const int32_t* rank, int64_t BH, int r, int D,
-                                                                    float* V_S, float* w) {
-    extern __shared__ float ysm[];  // [kTrsmWarps][r], then (FS_SMEM) F_S [r][r]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t b = blockIdx.y;
-    const int cb0 = blockIdx.x * kTrsmWarps;
-    const int DP = D + 1;
-    const int rr = rank[b];
-    const int col = cb0 + warp;
-    const float* __restrict__ Lg = FS + b * (int64_t)r * r;  // Lg[a * r + j] = F_S[a, j], j <= a
-    float* y = ysm + (size_t)warp * r;
-    const float* Lb = Lg;
-    if constexpr (FS_SMEM) {
-        // the CTA sums its 16 columns' partials (coalesced over columns) and stages F_S
-        float* Ls = ysm + (size_t)kTrsmWarps * r;
+// cp.async helpers (global -> shared, L2 only for 16 bytes)
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(static_cast<unsigned>(__cvta_generic_to_shared(smem_dst))),
+                 "l"(gmem_src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* smem_dst, const void* gmem_src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(static_cast<unsigned>(__cvta_generic_to_shared(smem_dst))),
+                 "l"(gmem_src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
+
+// Sum of the split-K partials of the CTA's kTrsmWarps columns, coalesced over
+// the columns: ysm[c][j] = sum_sp Ypart[sp][b][j][cb0 + c] for j < rr.
+__device__ __forceinline__ void trsm_sum_partials(const float* __restrict__ Ypart, int nsplit, int64_t BH, int64_t b,
+                                                  int r, int rr, int DP, int cb0, float* ysm) {
 #pragma unroll 4
-        for (int e = threadIdx.x; e < rr * kTrsmWarps; e += kTrsmWarps * 32) {
-            const int j = e / kTrsmWarps, c = e % kTrsmWarps;
-            float s = 0.f;
-            if (cb0 + c < DP) {
-                const float* src = Ypart + ((int64_t)b * r + j) * DP + cb0 + c;
-                const int64_t stride = BH * (int64_t)r * DP;
-#pragma unroll 8
-                for (int sp = 0; sp < nsplit; ++sp) s += src[sp * stride];
-            }
-            ysm[(size_t)c * r + j] = s;
-        }
-        // F_S rows: 16-byte loads, eight in flight per thread (r % 4 == 0), else scalar
-        if ((r & 3) == 0) {
-            const int q4 = r >> 2;
-#pragma unroll 8
-            for (int e = threadIdx.x; e < rr * q4; e += kTrsmWarps * 32) {
-                const int a = e / q4, j = (e % q4) * 4;
-                float4 v = __ldg(reinterpret_cast<const float4*>(Lg) + e);
-                if (j + 0 > a) v.x = 0.f;
-                if (j + 1 > a) v.y = 0.f;
-                if (j + 2 > a) v.z = 0.f;
-                if (j + 3 > a) v.w = 0.f;
-                reinterpret_cast<float4*>(Ls)[e] = v;
-            }
-        } else {
-#pragma unroll 8
-            for (int e = threadIdx.x; e < rr * r; e += kTrsmWarps * 32) {
-                const int a = e / r, j = e % r;
-                Ls[e] = j <= a ? Lg[e] : 0.f;
-            }
-        }
-        __syncthreads();
-        Lb = Ls;
-        if (col >= DP) return;  // no block-wide synchronisation below
-    } else {
-        if (col >= DP) return;  // warps are independent from here on
-        for (int j = lane; j < rr; j += 32) {
-            float s = 0.f;
-            const float* src = Ypart + ((int64_t)b * r + j) * DP + col;
+    for (int e = threadIdx.x; e < rr * kTrsmWarps; e += kTrsmWarps * 32) {
+        const int j = e / kTrsmWarps, c = e % kTrsmWarps;
+        float s = 0.f;
+        if (cb0 + c < DP) {
+            const float* src = Ypart + ((int64_t)b * r + j) * DP + cb0 + c;
             const int64_t stride = BH * (int64_t)r * DP;
 #pragma unroll 8
             for (int sp = 0; sp < nsplit; ++sp) s += src[sp * stride];
-            y[j] = s;
         }
-        __syncwarp();
+        ysm[(size_t)c * r + j] = s;
     }
-    // y in registers: lane l holds y[32 m + l]; pivots bottom up in blocks of
-    // 32 (block mb compile-time, so every register index is static), y_a
-    // broadcast from its lane, the same divide and fmaf per element as a
-    // shared-memory sweep
-    float yr[kTrsmRegs];
-#pragma unroll
-    for (int m = 0; m < kTrsmRegs; ++m) {
-        const int j = 32 * m + lane;
-        yr[m] = j < rr ? y[j] : 0.f;
-    }
-    if constexpr (FS_SMEM) {
-        // F_S in shared memory: the rows are read where they are used
-#pragma unroll
-        for (int mb = kTrsmRegs - 1; mb >= 0; --mb) {
-            if (32 * mb >= rr) continue;
-            const int top = min(31, rr - 1 - 32 * mb);
-            for (int la = top; la >= 0; --la) {
-                const int a = 32 * mb + la;
-                const float* La = Lb + (int64_t)a * r;
-                const float ya = __shfl_sync(0xffffffffu, yr[mb], la);
-                const float xa = ya / La[a];
-#pragma unroll
-                for (int m = 0; m < mb; ++m) yr[m] = fmaf(-La[32 * m + lane], xa, yr[m]);
-                if (lane < la) yr[mb] = fmaf(-La[32 * mb + lane], xa, yr[mb]);
-                if (lane == la) yr[mb] = xa;
-            }
-        }
-    } else {
-    // F_S in global memory: the row of pivot a - 1 is loaded while pivot a is
-    // applied (the loads do not depend on y), so the sweep is not a chain of
-    // dependent L2 reads; the diagonal F_S[a, a] comes from the loaded row by
-    // shuffle.
-#pragma unroll
-    for (int mb = kTrsmRegs - 1; mb >= 0; --mb) {
-        if (32 * mb >= rr) continue;
-        const int top = min(31, rr - 1 - 32 * mb);
-        float cur[kTrsmRegs], nxt[kTrsmRegs];
-        {
-            const float* La = Lb + (int64_t)(32 * mb + top) * r;
-#pragma unroll
-            for (int m = 0; m <= mb; ++m) nxt[m] = La[32 * m + lane];
-        }
-        for (int la = top; la >= 0; --la) {
-#pragma unroll
-            for (int m = 0; m <= mb; ++m) cur[m] = nxt[m];
-            if (la > 0) {
-                const float* Ln = Lb + (int64_t)(32 * mb + la - 1) * r;
-#pragma unroll
-                for (int m = 0; m <= mb; ++m) nxt[m] = Ln[32 * m + lane];
-            }
-            const float ya = __shfl_sync(0xffffffffu, yr[mb], la);
-            const float xa = ya / __shfl_sync(0xffffffffu, cur[mb], la);
-#pragma unroll
-            for (int m = 0; m < mb; ++m) yr[m] = fmaf(-cur[m], xa, yr[m]);
-            if (lane < la) yr[mb] = fmaf(-cur[mb], xa, yr[mb]);
-            if (lane == la) yr[mb] = xa;
-        }
-    }
-    }
+}
+
+// Writes column `col` of (V_S | w) from the registers of the warp's solve.
+__device__ __forceinline__ void trsm_store(const float (&yr)[kTrsmRegs], int lane, int64_t b, int r, int rr, int D,
+                                           int col, float* V_S, float* w) {
 #pragma unroll
     for (int m = 0; m < kTrsmRegs; ++m) {
         const int j = 32 * m + lane;
@@ -400,6 +312,167 @@ __global__ void __launch_bounds__(kTrsmWarps * 32) trsm_warp_kernel(const float*
         else
             w[b * r + j] = v;
     }
+}
+
+// Pivot a of the back substitution, from row a of F_S (La[j] = F_S[a, j]):
+// x_a = y_a / F_S[a, a] (y_a broadcast from its lane), then y_j -= F_S[a, j] x_a
+// for every j < a.  Called from loops over the register block MB = a / 32
+// that are unrolled, so every register index is static.
+__device__ __forceinline__ void trsm_pivot(float (&yr)[kTrsmRegs], const float* La, int a, int MB, int lane) {
+    const int la = a - 32 * MB;
+    const float ya = __shfl_sync(0xffffffffu, yr[MB], la);
+    const float xa = ya / La[a];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) yr[m] = fmaf(-La[32 * m + lane], xa, yr[m]);
+    if (lane < la) yr[MB] = fmaf(-La[32 * MB + lane], xa, yr[MB]);
+    if (lane == la) yr[MB] = xa;
+}
+
+// F_S in shared memory as a whole (small r): the CTA sums its columns'
+// partials and copies F_S (16-byte loads, eight in flight per thread), then
+// each warp solves its column with every row read on chip.
+__global__ void __launch_bounds__(kTrsmWarps * 32) trsm_warp_kernel(const float* __restrict__ Ypart, int nsplit,
+                                                                    const float* __restrict__ FS,
+                                                                    const int32_t* rank, int64_t BH, int r, int D,
+                                                                    float* V_S, float* w) {
+    extern __shared__ float ysm[];  // [kTrsmWarps][r], then F_S [r][r]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t b = blockIdx.y;
+    const int cb0 = blockIdx.x * kTrsmWarps;
+    const int DP = D + 1;
+    const int rr = rank[b];
+    const int col = cb0 + warp;
+    const float* __restrict__ Lg = FS + b * (int64_t)r * r;  // Lg[a * r + j] = F_S[a, j], j <= a
+    float* Ls = ysm + (size_t)kTrsmWarps * r;
+    trsm_sum_partials(Ypart, nsplit, BH, b, r, rr, DP, cb0, ysm);
+    if ((r & 3) == 0) {
+        const int q4 = r >> 2;
+#pragma unroll 8
+        for (int e = threadIdx.x; e < rr * q4; e += kTrsmWarps * 32) {
+            const int a = e / q4, j = (e % q4) * 4;
+            float4 v = __ldg(reinterpret_cast<const float4*>(Lg) + e);
+            if (j + 0 > a) v.x = 0.f;
+            if (j + 1 > a) v.y = 0.f;
+            if (j + 2 > a) v.z = 0.f;
+            if (j + 3 > a) v.w = 0.f;
+            reinterpret_cast<float4*>(Ls)[e] = v;
+        }
+    } else {
+#pragma unroll 8
+        for (int e = threadIdx.x; e < rr * r; e += kTrsmWarps * 32) {
+            const int a = e / r, j = e % r;
+            Ls[e] = j <= a ? Lg[e] : 0.f;
+        }
+    }
+    __syncthreads();
+    if (col >= DP) return;  // no block-wide synchronisation below
+    const float* y = ysm + (size_t)warp * r;
+    float yr[kTrsmRegs];
+#pragma unroll
+    for (int m = 0; m < kTrsmRegs; ++m) {
+        const int j = 32 * m + lane;
+        yr[m] = j < rr ? y[j] : 0.f;
+    }
+#pragma unroll
+    for (int mb = kTrsmRegs - 1; mb >= 0; --mb) {
+        if (32 * mb >= rr) continue;
+        const int top = min(31, rr - 1 - 32 * mb);
+        for (int la = top; la >= 0; --la) {
+            const int a = 32 * mb + la;
+            trsm_pivot(yr, Ls + (int64_t)a * r, a, mb, lane);
+        }
+    }
+    trsm_store(yr, lane, b, r, rr, D, col, V_S, w);
+}
+
+// F_S streamed through shared memory (larger r): rows are staged R at a time
+// (the R pivots of one sub-block, bottom up; only the columns j < 32 (a/32 + 1)
+// the sweep reads), double-buffered with cp.async, so every warp of the CTA
+// reads the rows on chip and the copy of the next sub-block runs while this
+// one is applied.  The same arithmetic per pivot as the kernel above.
+template <int R>
+__global__ void __launch_bounds__(kTrsmWarps * 32, 1) trsm_stream_kernel(const float* __restrict__ Ypart, int nsplit,
+                                                                      const float* __restrict__ FS,
+                                                                      const int32_t* rank, int64_t BH, int r, int D,
+                                                                      float* V_S, float* w) {
+    static_assert(R == 16 || R == 32, "sub-block of 16 or 32 pivots");
+    extern __shared__ float ysm[];  // [kTrsmWarps][r], then two buffers of R rows of r floats
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t b = blockIdx.y;
+    const int cb0 = blockIdx.x * kTrsmWarps;
+    const int DP = D + 1;
+    const int rr = rank[b];
+    const int col = cb0 + warp;
+    const bool active = col < DP;
+    const float* __restrict__ Lg = FS + b * (int64_t)r * r;
+    float* const buf0 = ysm + (size_t)kTrsmWarps * r;  // buffer k at buf0 + k * R * r
+    if (rr == 0) {
+        if (active) {
+            float yz[kTrsmRegs];
+#pragma unroll
+            for (int m = 0; m < kTrsmRegs; ++m) yz[m] = 0.f;
+            trsm_store(yz, lane, b, r, rr, D, col, V_S, w);
+        }
+        return;
+    }
+    const bool vec = (r & 3) == 0;
+    // copy of sub-block q: rows [qR, min(qR + R, rr)), columns [0, 32 (qR / 32 + 1))
+    auto issue = [&](int q) {
+        float* dst = buf0 + (size_t)(q & 1) * R * r;
+        const int a0 = q * R, a1 = min(a0 + R, rr);
+        const int cols = min(32 * (a0 / 32 + 1), r);
+        if (vec) {
+            const int c4 = cols >> 2;
+            for (int e = threadIdx.x; e < (a1 - a0) * c4; e += kTrsmWarps * 32) {
+                const int i = e / c4, j = (e % c4) * 4;
+                cp_async16(dst + (size_t)i * r + j, Lg + (int64_t)(a0 + i) * r + j);
+            }
+        } else {
+            for (int e = threadIdx.x; e < (a1 - a0) * cols; e += kTrsmWarps * 32) {
+                const int i = e / cols, j = e % cols;
+                cp_async4(dst + (size_t)i * r + j, Lg + (int64_t)(a0 + i) * r + j);
+            }
+        }
+    };
+    const int q_top = (rr - 1) / R;
+    issue(q_top);
+    cp_async_commit();
+    trsm_sum_partials(Ypart, nsplit, BH, b, r, rr, DP, cb0, ysm);
+    __syncthreads();
+    float yr[kTrsmRegs];
+    {
+        const float* y = ysm + (size_t)warp * r;
+#pragma unroll
+        for (int m = 0; m < kTrsmRegs; ++m) {
+            const int j = 32 * m + lane;
+            yr[m] = j < rr ? y[j] : 0.f;
+        }
+    }
+#pragma unroll
+    for (int mb = kTrsmRegs - 1; mb >= 0; --mb) {
+        if (32 * mb >= rr) continue;
+#pragma unroll
+        for (int h = 32 / R - 1; h >= 0; --h) {
+            const int q = mb * (32 / R) + h;
+            if (q > q_top) continue;
+            if (q >= 1) issue(q - 1);
+            cp_async_commit();
+            cp_async_wait1();  // this thread's copies of sub-block q have landed
+            __syncthreads();   // and everyone's
+            if (active) {
+                const float* B = buf0 + (size_t)(q & 1) * R * r;
+                for (int a = min(q * R + R - 1, rr - 1); a >= q * R; --a) trsm_pivot(yr, B + (size_t)(a - q * R) * r, a, mb, lane);
+            }
+            __syncthreads();  // the buffer is read before the copy two sub-blocks on refills it
+        }
+    }
+    if (active) trsm_store(yr, lane, b, r, rr, D, col, V_S, w);
+}
+
+// rows per staged sub-block: 32 while two buffers of 32 rows fit in 160 KB, else 16
+inline int trsm_stream_rows(int r) { return 2 * 32 * (size_t)r * sizeof(float) <= 160 * 1024 ? 32 : 16; }
+inline size_t trsm_stream_smem(int r) {
+    return sizeof(float) * ((size_t)kTrsmWarps * r + 2 * (size_t)trsm_stream_rows(r) * r);
 }
 
 struct WeightsPlan {
@@ -468,8 +541,10 @@ Status run_weights(const WeightsRequest& q, cudaStream_t st) {
     cudaError_t e;
     if (q.r <= kTrsmWarpMaxR) {
         const bool fs_sm = trsm_fs_in_smem(q.r);
-        const size_t smem = sizeof(float) * ((size_t)kTrsmWarps * q.r + (fs_sm ? (size_t)q.r * q.r : 0));
-        auto kern = fs_sm ? trsm_warp_kernel<true> : trsm_warp_kernel<false>;
+        const size_t smem = fs_sm ? sizeof(float) * ((size_t)kTrsmWarps * q.r + (size_t)q.r * q.r)
+                                  : trsm_stream_smem(q.r);
+        auto kern = fs_sm ? trsm_warp_kernel
+                          : (trsm_stream_rows(q.r) == 32 ? trsm_stream_kernel<32> : trsm_stream_kernel<16>);
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return Status::cuda(e, "weights: trsm smem attribute");
         kern<<<dim3((unsigned)ceil_div(D + 1, kTrsmWarps), (unsigned)q.BH), kTrsmWarps * 32, smem, st>>>(
