@@ -16,8 +16,8 @@ scaling; instances are independent, so there is no collective on the data
 path) and the reported time is the maximum over ranks.
 
 Printed (rank 0): one JSON line with the metric, the device-timed value,
-an end-to-end value through wildcat_forward_host (pinned host buffers,
-copies inside the timed region), per-stage times with each stage's
+an end-to-end value through wildcat_forward_host (with --nbins > 1,
+wildcat_forward_ex_host; pinned host buffers, copies inside the timed region), per-stage times with each stage's
 roofline fraction (select and weights against HBM bandwidth, attend against
 the bf16 tensor peak), the forward-level roofline (sum over stages of
 max(bytes / HBM, MMA flops / tensor peak, exps / MUFU rate) against the
@@ -492,14 +492,19 @@ def main():
                "peak_tflops": peak64, "frac": ach / peak64, "bound": "alu",
                "peak_source": "fp64 unit count: 148 SMs x 64 FMA/clk x 2 x 1.965 GHz"}
 
-    # ---- end to end through wildcat_forward_host (host buffers) ----
+    # ---- end to end through wildcat_forward_host / wildcat_forward_ex_host (host buffers) ----
     e2e = None
-    if not args.no_e2e and nb == 1:
-        hp = wc.HostForwardPlan(w.BH, w.m, w.n, w.d, w.r, w.dtype)
+    if not args.no_e2e:
+        if nb == 1:
+            hp = wc.HostForwardPlan(w.BH, w.m, w.n, w.d, w.r, w.dtype)
+            api = "wildcat_forward_host (pinned host buffers)"
+        else:
+            hp = wc.HostForwardExPlan(w.BH, w.m, w.n, w.d, w.r, w.dtype, nbins=nb)
+            api = f"wildcat_forward_ex_host with nbins = {nb} (pinned host buffers)"
         pinned = {k: v.pin_memory() for k, v in dev.items()}
         O_host = torch.empty((w.BH, w.m, w.d), dtype=torch.float32).pin_memory()
         S_host = torch.empty((w.BH, w.r), dtype=torch.int32).pin_memory()
-        r_host = torch.empty((w.BH,), dtype=torch.int32).pin_memory()
+        r_host = torch.empty((w.BH, nb) if nb > 1 else (w.BH,), dtype=torch.int32).pin_memory()
         for _ in range(2):
             hp.run(pinned["Q"], pinned["K"], pinned["V"], O_host, w.beta, w.pivot_seed, EPS,
                    S_host, r_host)
@@ -518,8 +523,8 @@ def main():
         eb = in_bytes(w)
         e2e = {"value": world * args.steps / (e_tot / 1e3), "unit": "calls/s",
                "h2d_bytes_per_step": eb * w.BH * (w.m + 2 * w.n) * w.d,
-               "d2h_bytes_per_step": 4 * w.BH * w.m * w.d + 4 * w.BH * w.r + 4 * w.BH,
-               "api": "wildcat_forward_host (pinned host buffers)"}
+               "d2h_bytes_per_step": 4 * w.BH * w.m * w.d + 4 * w.BH * w.r + 4 * w.BH * nb,
+               "api": api}
         del hp
 
     cpu = None

@@ -373,6 +373,29 @@ wildcat_status wildcat_forward_host(const void* Q_host, const void* K_host, cons
                                     void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * wildcat_forward_ex_host -- wildcat_forward_ex on HOST buffers, pipelined
+ * like wildcat_forward_host: K is copied first on the library's copy stream
+ * (the recentring mean and the select need only K), V and Q follow while the
+ * select runs, the weights stage waits for V and the attend for Q; then O
+ * (and optionally S, rank) are copied back and the stream is waited for.
+ * Options as in wildcat_forward_ex (NULL: the plain forward).
+ *
+ *   Q_host, K_host, V_host   host input arrays (layouts as wildcat_forward)
+ *   O_host                   host output [BH, m, d] float32
+ *   S_host [BH, r] int32, rank_host [BH, nbins] int32: optional host outputs
+ *                            as in wildcat_forward_ex (or NULL)
+ *   workspace >= wildcat_forward_ex_host_workspace_size(...) bytes (device)
+ */
+size_t wildcat_forward_ex_host_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r,
+                                              int dtype, const wildcat_options* opts);
+wildcat_status wildcat_forward_ex_host(const void* Q_host, const void* K_host,
+                                       const void* V_host, int dtype, int64_t BH, int64_t m,
+                                       int64_t n, int d, float beta, int r, uint64_t seed,
+                                       int64_t inst0, float eps, const wildcat_options* opts,
+                                       float* O_host, int32_t* S_host, int32_t* rank_host,
+                                       void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * wildcat_pivot_uniforms -- the pivot uniforms the select kernels draw
  * (test entry point): u[b, i] for b < BH, i < steps (instance offset 0), as
  * float64, written to the device array u [BH, steps].

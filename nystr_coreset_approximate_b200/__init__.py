@@ -80,6 +80,9 @@ _SIGS = {
     "wildcat_forward_host_workspace_size": ([_i64, _i64, _i64, _int, _int, _int], _sz),
     "wildcat_forward_host": ([_vp, _vp, _vp, _int, _i64, _i64, _i64, _int, _f32, _int, _u64, _i64, _f32,
                               _vp, _vp, _vp, _vp, _sz, _vp], _int),
+    "wildcat_forward_ex_host_workspace_size": ([_i64, _i64, _i64, _int, _int, _int, _vp], _sz),
+    "wildcat_forward_ex_host": ([_vp, _vp, _vp, _int, _i64, _i64, _i64, _int, _f32, _int, _u64, _i64, _f32,
+                                 _vp, _vp, _vp, _vp, _vp, _sz, _vp], _int),
     "wildcat_pivot_uniforms": ([_u64, _i64, _int, _vp, _vp], _int),
     "wildcat_get_device_status": ([_vp], _int),
     "wildcat_test_force_wait_timeout": ([_i64], _int),
@@ -477,6 +480,52 @@ def forward_host(Q_host, K_host, V_host, beta: float, r: int, seed: int = 0, eps
     O = torch.empty((BH, m, d), dtype=torch.float32).pin_memory()
     S = torch.empty((BH, r), dtype=torch.int32)
     rank = torch.empty((BH,), dtype=torch.int32)
+    plan.run(Q_host, K_host, V_host, O, beta, seed, eps, S, rank)
+    return O, S, rank
+
+
+class HostForwardExPlan:
+    """Device workspace for wildcat_forward_ex_host (the forward with the
+    options of Sec. 2; inputs and outputs in host memory)."""
+
+    def __init__(self, BH, m, n, d, r, dtype: str, nbins: int = 1, recenter: bool = False, tau: float = 1.0,
+                 device="cuda"):
+        torch = _torch()
+        self.BH, self.m, self.n, self.d, self.r = BH, m, n, d, r
+        self.code = DTYPES[dtype]
+        self.opts = Options(int(nbins), int(bool(recenter)), float(tau))
+        L = lib()
+        self.ws_bytes = int(L.wildcat_forward_ex_host_workspace_size(BH, m, n, d, r, self.code,
+                                                                      ctypes.byref(self.opts)))
+        if self.ws_bytes == 0:
+            raise ValueError("n and r must be multiples of nbins")
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=device)
+
+    def run(self, Q_host, K_host, V_host, O_host, beta, seed, eps=1e-6, S_host=None,
+            rank_host=None, stream=None, inst0=0):
+        for t, nm in ((Q_host, "Q"), (K_host, "K"), (V_host, "V"), (O_host, "O")):
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{nm} must be a contiguous host tensor")
+        _check(lib().wildcat_forward_ex_host(
+            _vp(Q_host.data_ptr()), _vp(K_host.data_ptr()), _vp(V_host.data_ptr()), self.code,
+            self.BH, self.m, self.n, self.d, float(beta), self.r, int(seed) & (2**64 - 1),
+            int(inst0), float(eps), ctypes.byref(self.opts), _vp(O_host.data_ptr()),
+            None if S_host is None else _vp(S_host.data_ptr()),
+            None if rank_host is None else _vp(rank_host.data_ptr()),
+            _dev(self.ws, "workspace"), self.ws_bytes, _stream(stream)))
+        return O_host
+
+
+def forward_ex_host(Q_host, K_host, V_host, beta: float, r: int, seed: int = 0, eps: float = 1e-6, *,
+                    nbins: int = 1, recenter: bool = False, tau: float = 1.0):
+    """wildcat_forward_ex on host tensors.  Returns (O_hat, S [BH, r], rank [BH, nbins]) on the host."""
+    torch = _torch()
+    BH, m, d = _shape3(Q_host, "Q")
+    n = K_host.shape[1]
+    plan = HostForwardExPlan(BH, m, n, d, r, "bf16" if _dtype_code(K_host) else "f32", nbins, recenter, tau)
+    O = torch.empty((BH, m, d), dtype=torch.float32).pin_memory()
+    S = torch.empty((BH, r), dtype=torch.int32)
+    rank = torch.empty((BH, nbins), dtype=torch.int32)
     plan.run(Q_host, K_host, V_host, O, beta, seed, eps, S, rank)
     return O, S, rank
 

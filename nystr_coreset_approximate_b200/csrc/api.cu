@@ -241,6 +241,27 @@ HostPipe* host_pipe(int dev) {
     return hp;
 }
 
+// Copies K, then V, then Q (host -> device) on the device's copy stream,
+// after the work already queued on `s`; `s` waits for K.  The caller holds
+// hp->mu and makes its weights and attend stages wait for hp->v_in / hp->q_in.
+Status stage_host_inputs(HostPipe* hp, cudaStream_t s, void* Kd, void* Vd, void* Qd, const void* K_host,
+                         const void* V_host, const void* Q_host, size_t kv_bytes, size_t q_bytes) {
+    cudaError_t e;
+    if ((e = cudaEventRecord(hp->ready, s))) return Status::cuda(e, "forward_host: record");
+    if ((e = cudaStreamWaitEvent(hp->cs, hp->ready, 0))) return Status::cuda(e, "forward_host: wait");
+    if ((e = cudaMemcpyAsync(Kd, K_host, kv_bytes, cudaMemcpyHostToDevice, hp->cs)))
+        return Status::cuda(e, "forward_host: copy K");
+    if ((e = cudaEventRecord(hp->k_in, hp->cs))) return Status::cuda(e, "forward_host: record");
+    if ((e = cudaMemcpyAsync(Vd, V_host, kv_bytes, cudaMemcpyHostToDevice, hp->cs)))
+        return Status::cuda(e, "forward_host: copy V");
+    if ((e = cudaEventRecord(hp->v_in, hp->cs))) return Status::cuda(e, "forward_host: record");
+    if (q_bytes && (e = cudaMemcpyAsync(Qd, Q_host, q_bytes, cudaMemcpyHostToDevice, hp->cs)))
+        return Status::cuda(e, "forward_host: copy Q");
+    if ((e = cudaEventRecord(hp->q_in, hp->cs))) return Status::cuda(e, "forward_host: record");
+    if ((e = cudaStreamWaitEvent(s, hp->k_in, 0))) return Status::cuda(e, "forward_host: wait for K");
+    return Status::ok();
+}
+
 namespace wildcat {
 int read_device_status(bool clear) {
     const int parts[3] = {read_attend_status(clear), read_weights_status(clear), read_select_gs_status(clear)};
@@ -445,13 +466,20 @@ size_t wildcat_forward_ex_workspace_size(int64_t BH, int64_t m, int64_t n, int d
     return cv.used + 256;
 }
 
-wildcat_status wildcat_forward_ex(const void* Q, const void* K, const void* V, int dtype, int64_t BH, int64_t m,
-                                  int64_t n, int d, float beta, int r, uint64_t seed, int64_t inst0, float eps,
-                                  const wildcat_options* opts, float* O, int32_t* S_out, int32_t* rank_out,
-                                  void* workspace, size_t ws_bytes, void* stream) {
-    const char* who = "wildcat_forward_ex";
+}  // extern "C"
+
+namespace {
+
+// Options of the extended forward, checked, with the key kernel's beta.
+struct ExOptions {
+    int nbins;
+    bool recenter;
+    float beta_key;  // beta / tau^2
+};
+
+wildcat_status check_ex(int dtype, int64_t BH, int64_t m, int64_t n, int d, float beta, int r, int64_t inst0, float eps,
+                        const wildcat_options* opts, const char* who, ExOptions* out) {
     const int nbins = opts ? opts->nbins : 1;
-    const bool recenter = opts && opts->recenter;
     const float tau = opts ? opts->tau : 1.f;
     wildcat_status st = check_common(dtype, BH, n, d, r, who);
     if (st != WILDCAT_OK) return st;
@@ -464,25 +492,30 @@ wildcat_status wildcat_forward_ex(const void* Q, const void* K, const void* V, i
     if (m < 0) return bad(1, "%s: m must be >= 0", who);
     if (inst0 < 0 || (inst0 + BH) * nbins > 4294967296LL)
         return bad(1, "%s: inst0 must satisfy 0 <= inst0, (inst0 + BH) * nbins <= 2^32", who);
-    if (BH == 0) return record(Status::ok());
-    if (!K || !V || !workspace || (m > 0 && (!Q || !O))) return bad(1, "%s: null pointer argument", who);
-    if (!aligned16(K) || !aligned16(V) || (Q && !aligned16(Q)))
-        return bad(1, "%s: Q, K and V must be 16-byte aligned", who);
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
-    Carve cv(workspace, ws_bytes);
-    const BinnedLayout L = carve_binned(cv, BH, m, n, d, r, nbins, dtype, recenter);
-    if (!cv.fits()) return bad(4, "%s: workspace too small", who);
+    *out = ExOptions{nbins, opts && opts->recenter, beta_key};
+    return WILDCAT_OK;
+}
+
+// The extended forward on device buffers: recentring mean, select and weights
+// on the [BH * nbins, n / nbins] view, the bins' union coreset, attend.
+// wait_v / wait_q (optional): events the weights / attend stage waits for.
+wildcat_status forward_ex_impl(const void* Q, const void* K, const void* V, int dtype, int64_t BH, int64_t m, int64_t n,
+                               int d, float beta, int r, uint64_t seed, int64_t inst0, float eps, const ExOptions& o,
+                               float* O, int32_t* S_out, int32_t* rank_out, const BinnedLayout& L, cudaStream_t s,
+                               cudaEvent_t wait_v = nullptr, cudaEvent_t wait_q = nullptr) {
+    const int nbins = o.nbins;
     const int64_t nb = n / nbins, BB = BH * nbins;
     const int rb = r / nbins;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     Status z;
-    if (recenter && (z = wildcat::launch_key_mean(K, dtype, BH, n, d, L.mws, L.kbar, s)).code) return record(z);
-    wildcat::SelectRequest sq{K, dtype, BB, nb, d, beta_key, rb, seed, inst0 * nbins, eps, nullptr, L.S, L.F, L.rank_b,
-                              L.K_S, L.kbar, nbins};
+    cudaError_t ew;
+    if (o.recenter && (z = wildcat::launch_key_mean(K, dtype, BH, n, d, L.mws, L.kbar, s)).code) return record(z);
+    wildcat::SelectRequest sq{K,      dtype, BB,      nb,  d,     o.beta_key, rb,      seed, inst0 * nbins,
+                              eps,    nullptr, L.S,   L.F, L.rank_b, L.K_S,   L.kbar,  nbins};
     sq.ws = L.sws;
     sq.ws_bytes = L.sws_bytes;
     if ((z = wildcat::launch_select(sq, s)).code) return record(z);
     if ((z = mark_stage(g_ev_after_select, s, "forward: stage event")).code) return record(z);
+    if (wait_v && (ew = cudaStreamWaitEvent(s, wait_v, 0))) return record(Status::cuda(ew, "forward: wait for V"));
     wildcat::WeightsRequest wq{L.F, L.S, L.rank_b, V, dtype, BB, nb, d, rb, L.V_S, L.w, L.vmin_b, L.vmax_b, L.wws,
                                L.wws_bytes};
     if ((z = wildcat::launch_weights(wq, s)).code) return record(z);
@@ -490,6 +523,7 @@ wildcat_status wildcat_forward_ex(const void* Q, const void* K, const void* V, i
     if ((z = wildcat::launch_binning_finish(L.vmin_b, L.vmax_b, L.S, L.rank_b, BH, nbins, nb, rb, d, L.vmin, L.vmax,
                                             L.rank_att, S_out, rank_out, s)).code)
         return record(z);
+    if (wait_q && (ew = cudaStreamWaitEvent(s, wait_q, 0))) return record(Status::cuda(ew, "forward: wait for Q"));
     if (m > 0) {
         // the attend is unchanged by recentring and temperature: it uses the
         // original pivot keys and beta (the shift and 1/tau cancel in N / D)
@@ -498,6 +532,30 @@ wildcat_status wildcat_forward_ex(const void* Q, const void* K, const void* V, i
         if ((z = wildcat::launch_attend(aq, s)).code) return record(z);
     }
     return record(Status::ok());
+}
+
+}  // namespace
+
+extern "C" {
+
+wildcat_status wildcat_forward_ex(const void* Q, const void* K, const void* V, int dtype, int64_t BH, int64_t m,
+                                  int64_t n, int d, float beta, int r, uint64_t seed, int64_t inst0, float eps,
+                                  const wildcat_options* opts, float* O, int32_t* S_out, int32_t* rank_out,
+                                  void* workspace, size_t ws_bytes, void* stream) {
+    const char* who = "wildcat_forward_ex";
+    ExOptions o{};
+    wildcat_status st = check_ex(dtype, BH, m, n, d, beta, r, inst0, eps, opts, who, &o);
+    if (st != WILDCAT_OK) return st;
+    if (BH == 0) return record(Status::ok());
+    if (!K || !V || !workspace || (m > 0 && (!Q || !O))) return bad(1, "%s: null pointer argument", who);
+    if (!aligned16(K) || !aligned16(V) || (Q && !aligned16(Q)))
+        return bad(1, "%s: Q, K and V must be 16-byte aligned", who);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
+    Carve cv(workspace, ws_bytes);
+    const BinnedLayout L = carve_binned(cv, BH, m, n, d, r, o.nbins, dtype, o.recenter);
+    if (!cv.fits()) return bad(4, "%s: workspace too small", who);
+    return forward_ex_impl(Q, K, V, dtype, BH, m, n, d, beta, r, seed, inst0, eps, o, O, S_out, rank_out, L,
+                           static_cast<cudaStream_t>(stream));
 }
 
 size_t wildcat_forward_binned_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int nbins, int dtype) {
@@ -560,18 +618,11 @@ wildcat_status wildcat_forward_host(const void* Q_host, const void* K_host, cons
     HostPipe* hp = host_pipe(dev);
     if (!hp) return record(Status::cuda(cudaErrorMemoryAllocation, "forward_host: copy stream"));
     std::lock_guard<std::mutex> lock(hp->mu);
-    if ((e = cudaEventRecord(hp->ready, s))) return record(Status::cuda(e, "forward_host: record"));
-    if ((e = cudaStreamWaitEvent(hp->cs, hp->ready, 0))) return record(Status::cuda(e, "forward_host: wait"));
-    if ((e = cudaMemcpyAsync(Kd, K_host, eb * BH * n * d, cudaMemcpyHostToDevice, hp->cs)))
-        return record(Status::cuda(e, "forward_host: copy K"));
-    if ((e = cudaEventRecord(hp->k_in, hp->cs))) return record(Status::cuda(e, "forward_host: record"));
-    if ((e = cudaMemcpyAsync(Vd, V_host, eb * BH * n * d, cudaMemcpyHostToDevice, hp->cs)))
-        return record(Status::cuda(e, "forward_host: copy V"));
-    if ((e = cudaEventRecord(hp->v_in, hp->cs))) return record(Status::cuda(e, "forward_host: record"));
-    if (m > 0 && (e = cudaMemcpyAsync(Qd, Q_host, eb * BH * m * d, cudaMemcpyHostToDevice, hp->cs)))
-        return record(Status::cuda(e, "forward_host: copy Q"));
-    if ((e = cudaEventRecord(hp->q_in, hp->cs))) return record(Status::cuda(e, "forward_host: record"));
-    if ((e = cudaStreamWaitEvent(s, hp->k_in, 0))) return record(Status::cuda(e, "forward_host: wait for K"));
+    Status z = stage_host_inputs(hp, s, Kd, Vd, Qd, K_host, V_host, Q_host, eb * BH * n * d, eb * BH * m * d);
+    if (z.code) {
+        cudaStreamSynchronize(hp->cs);
+        return record(z);
+    }
     st = forward_impl(m > 0 ? Qd : nullptr, Kd, Vd, dtype, BH, m, n, d, beta, r, seed, inst0, eps,
                       m > 0 ? Od : nullptr, nullptr, nullptr, L, s, hp->v_in, hp->q_in);
     if (st != WILDCAT_OK) {
@@ -583,6 +634,72 @@ wildcat_status wildcat_forward_host(const void* Q_host, const void* K_host, cons
     if (S_host && (e = cudaMemcpyAsync(S_host, L.S, sizeof(int32_t) * BH * r, cudaMemcpyDeviceToHost, s)))
         return record(Status::cuda(e, "forward_host: copy S"));
     if (rank_host && (e = cudaMemcpyAsync(rank_host, L.rank, sizeof(int32_t) * BH, cudaMemcpyDeviceToHost, s)))
+        return record(Status::cuda(e, "forward_host: copy rank"));
+    if ((e = cudaStreamSynchronize(s))) return record(Status::cuda(e, "forward_host: stream sync"));
+    return record(Status::ok());
+}
+
+size_t wildcat_forward_ex_host_workspace_size(int64_t BH, int64_t m, int64_t n, int d, int r, int dtype,
+                                              const wildcat_options* opts) {
+    const int nbins = opts ? opts->nbins : 1;
+    if (BH < 0 || m < 0 || n < 1 || r < 1 || d < 1 || nbins < 1 || n % nbins || r % nbins) return 0;
+    Carve cv(nullptr, 0);
+    cv.take(elem_bytes(dtype) * BH * m * d);
+    cv.take(elem_bytes(dtype) * BH * n * d);
+    cv.take(elem_bytes(dtype) * BH * n * d);
+    cv.take(sizeof(float) * BH * m * d);
+    cv.take(sizeof(int32_t) * BH * r);
+    cv.take(sizeof(int32_t) * BH * nbins);
+    carve_binned(cv, BH, m, n, d, r, nbins, dtype, opts && opts->recenter);
+    return cv.used + 256;
+}
+
+wildcat_status wildcat_forward_ex_host(const void* Q_host, const void* K_host, const void* V_host, int dtype,
+                                       int64_t BH, int64_t m, int64_t n, int d, float beta, int r, uint64_t seed,
+                                       int64_t inst0, float eps, const wildcat_options* opts, float* O_host,
+                                       int32_t* S_host, int32_t* rank_host, void* workspace, size_t ws_bytes,
+                                       void* stream) {
+    const char* who = "wildcat_forward_ex_host";
+    ExOptions o{};
+    wildcat_status st = check_ex(dtype, BH, m, n, d, beta, r, inst0, eps, opts, who, &o);
+    if (st != WILDCAT_OK) return st;
+    if (BH == 0) return record(Status::ok());
+    if (!K_host || !V_host || !workspace || (m > 0 && (!Q_host || !O_host)))
+        return bad(1, "%s: null pointer argument", who);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return bad(4, "%s: workspace must be 256-byte aligned", who);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t eb = elem_bytes(dtype);
+    Carve cv(workspace, ws_bytes);
+    void* Qd = cv.take(eb * BH * m * d);
+    void* Kd = cv.take(eb * BH * n * d);
+    void* Vd = cv.take(eb * BH * n * d);
+    float* Od = static_cast<float*>(cv.take(sizeof(float) * BH * m * d));
+    int32_t* Sd = static_cast<int32_t*>(cv.take(sizeof(int32_t) * BH * r));
+    int32_t* rankd = static_cast<int32_t*>(cv.take(sizeof(int32_t) * BH * o.nbins));
+    const BinnedLayout L = carve_binned(cv, BH, m, n, d, r, o.nbins, dtype, o.recenter);
+    if (!cv.fits()) return bad(4, "%s: workspace too small", who);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e) return record(Status::cuda(e, "forward_host: current device"));
+    HostPipe* hp = host_pipe(dev);
+    if (!hp) return record(Status::cuda(cudaErrorMemoryAllocation, "forward_host: copy stream"));
+    std::lock_guard<std::mutex> lock(hp->mu);
+    Status z = stage_host_inputs(hp, s, Kd, Vd, Qd, K_host, V_host, Q_host, eb * BH * n * d, eb * BH * m * d);
+    if (z.code) {
+        cudaStreamSynchronize(hp->cs);
+        return record(z);
+    }
+    st = forward_ex_impl(m > 0 ? Qd : nullptr, Kd, Vd, dtype, BH, m, n, d, beta, r, seed, inst0, eps, o,
+                         m > 0 ? Od : nullptr, Sd, rankd, L, s, hp->v_in, hp->q_in);
+    if (st != WILDCAT_OK) {
+        cudaStreamSynchronize(hp->cs);
+        return st;
+    }
+    if (m > 0 && (e = cudaMemcpyAsync(O_host, Od, sizeof(float) * BH * m * d, cudaMemcpyDeviceToHost, s)))
+        return record(Status::cuda(e, "forward_host: copy O"));
+    if (S_host && (e = cudaMemcpyAsync(S_host, Sd, sizeof(int32_t) * BH * r, cudaMemcpyDeviceToHost, s)))
+        return record(Status::cuda(e, "forward_host: copy S"));
+    if (rank_host && (e = cudaMemcpyAsync(rank_host, rankd, sizeof(int32_t) * BH * o.nbins, cudaMemcpyDeviceToHost, s)))
         return record(Status::cuda(e, "forward_host: copy rank"));
     if ((e = cudaStreamSynchronize(s))) return record(Status::cuda(e, "forward_host: stream sync"));
     return record(Status::ok());

@@ -92,6 +92,22 @@ def test_forward_workspace_accounts_for_the_factor(L):
                              None, ctypes.c_void_p(1 << 20), ws - 4096, None) == 4
 
 
+def test_forward_ex_host_workspace_and_checks(L):
+    BH, m, n, d, r = 8, 1024, 4096, 128, 64
+    opts = wc.Options(4, 1, 1.5)
+    we = int(L.wildcat_forward_ex_workspace_size(BH, m, n, d, r, 1, ctypes.byref(opts)))
+    wh = int(L.wildcat_forward_ex_host_workspace_size(BH, m, n, d, r, 1, ctypes.byref(opts)))
+    # the device forward's workspace plus staging for Q, K, V, O, S and the bins' ranks
+    assert wh >= we + 2 * BH * (m + 2 * n) * d + 4 * BH * m * d + 4 * BH * r + 4 * BH * 4
+    assert int(L.wildcat_forward_ex_host_workspace_size(BH, m, n, d, r, 1, ctypes.byref(wc.Options(3, 0, 1.0)))) == 0
+    # rejected before any copy: bins that do not divide n, a bad temperature, a null input
+    for o in (wc.Options(3, 0, 1.0), wc.Options(1, 0, 0.0)):
+        assert L.wildcat_forward_ex_host(FAKE, FAKE, FAKE, 1, BH, m, n, d, 0.125, r, 0, 0, 1e-6,
+                                         ctypes.byref(o), FAKE, None, None, FAKE, 1 << 30, None) == 1
+    assert L.wildcat_forward_ex_host(FAKE, None, FAKE, 1, BH, m, n, d, 0.125, r, 0, 0, 1e-6,
+                                     None, FAKE, None, None, FAKE, 1 << 30, None) == 1
+
+
 def test_cluster_knob_validation(L):
     assert L.wildcat_set_select_cluster(3) == 1
     assert L.wildcat_set_select_cluster(32) == 1

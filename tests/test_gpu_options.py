@@ -46,6 +46,21 @@ def test_options_parity(orc, w, nbins, recenter, tau):
                                      recenter=recenter, tau=tau)
 
 
+@pytest.mark.parametrize("nbins,recenter,tau", [(4, False, 1.0), (2, True, 1.6), (1, False, 1.0)])
+def test_forward_ex_host_matches_device(nbins, recenter, tau):
+    """The host-buffer extended forward (K copied first, V and Q while the
+    select runs) gives the device forward's outputs bit for bit."""
+    w = gc.case("ex_host", "walk", 3, 4096, 300, 128, 128, "bf16")
+    dev, _ = workloads.make(w)
+    d = gc.cuda_inputs(dev)
+    O_d, S_d, r_d = wc.forward_ex(d["Q"], d["K"], d["V"], w.beta, w.r, 11, EPS, nbins=nbins,
+                                  recenter=recenter, tau=tau)
+    pinned = {k: v.pin_memory() for k, v in dev.items()}
+    O_h, S_h, r_h = wc.forward_ex_host(pinned["Q"], pinned["K"], pinned["V"], w.beta, w.r, 11, EPS,
+                                       nbins=nbins, recenter=recenter, tau=tau)
+    assert torch.equal(S_h, S_d.cpu()) and torch.equal(r_h, r_d.cpu()) and torch.equal(O_h, O_d.cpu())
+
+
 def test_options_rejected_on_host():
     import ctypes
 
