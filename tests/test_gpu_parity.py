@@ -86,14 +86,26 @@ def test_stagewise_parity(orc, w):
     assert np.array_equal(O_f.cpu().numpy(), O)
 
 
-@pytest.mark.parametrize("w", [CASES[0], CASES[4], CASES[5]], ids=lambda w: w.name)
+# the triangular solve's shared-memory forms: the whole pivot block (r <= ~220),
+# streamed in sub-blocks of 32 pivots (r <= 640; 4-byte copies when r % 4 != 0)
+# and of 16 pivots (640 < r <= 1024)
+SOLVE_CASES = [
+    gc.case("solve_stream32_r250", "iid", 2, 1200, 16, 64, 250, "f32"),
+    gc.case("solve_stream32_bf16_r512", "iid", 1, 2048, 16, 128, 512, "bf16"),
+    gc.case("solve_stream16_r700", "walk", 1, 1500, 16, 64, 700, "bf16"),
+    gc.case("solve_stream16_r900_truncated", "walk", 1, 8000, 16, 128, 900, "bf16"),  # rank 466
+]
+
+
+@pytest.mark.parametrize("w", [CASES[0], CASES[4], CASES[5]] + SOLVE_CASES, ids=lambda w: w.name)
 def test_weights_kernel_alone(orc, w):
     """wildcat_weights on the oracle's own factor (rounded to float32) against
     the oracle's weights on exactly that rounded factor.  Bounds, relative to
     the largest entry: 1e-5 for float32 values (fp32 split-K sums and back
     substitution; measured <= 1.3e-6), 5e-5 for bfloat16 values (the factor
     split into bf16 hi + lo parts on the tensor cores, about 2^-17 relative
-    per entry; measured <= 1.1e-5)."""
+    per entry; measured <= 1.1e-5).  The SOLVE_CASES run the streamed forms
+    of the back substitution (including a rank below r on the walk keys)."""
     dev, ex = workloads.make(w)
     res = orc.rpcholesky(ex["K"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
     F32 = res["F"].astype(np.float32)
@@ -110,8 +122,8 @@ def test_attend_kernel_alone(orc, w):
     """wildcat_attend on the oracle's coreset (V_S, w rounded to float32)
     against the oracle's attend on the same rounded values.  float32 inputs
     run on CUDA cores in fp32; bfloat16 inputs with d in {64, 128} run on the
-    tensor cores, where P is rounded to bfloat16 once (the same rounded P in
-    numerator and denominator)."""
+    tensor cores, where V_S and P are rounded to bfloat16 for the numerator's
+    MMA and the denominator is summed in fp32 from the unrounded P."""
     dev, ex = workloads.make(w)
     res = orc.rpcholesky(ex["K"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
     VS_o, w_o = orc.weights(res["F"], res["S"], res["rank"], ex["V"])
