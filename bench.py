@@ -23,9 +23,12 @@ the bf16 tensor peak), the forward-level roofline (sum over stages of
 max(bytes / HBM, MMA flops / tensor peak, exps / MUFU rate) against the
 measured step time), the roofline of the dominant kernel, sampled SM clocks,
 and the oracle timed on the host cores as a CPU baseline.  Where the oracle
-cannot afford every query row (m > 4096) it runs select and weights in full
-and the attend on 256 seeded rows per head, and the per-call time is
-extrapolated per row (the line says so).
+cannot afford a whole call it runs a stated sample and extrapolates each
+part (the line says so): the attend on 256 seeded rows per head when m >
+4096, and, when one instance's select is large (the 65536- and 131072-token
+workloads), the first 64 pivot steps of every instance, scaled by the
+per-step cost n (d + i) to the rank, with the weights and attend on those 64
+pivots scaled by rank / 64.
 """
 from __future__ import annotations
 
@@ -216,56 +219,94 @@ class ClockSampler:
 # the fp64 CPU oracle, as it stands (cpu_baseline leg and the reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_rows(w):
-    """Query rows the oracle's attend covers: all of them, or 256 seeded rows
-    per head when m is large."""
+ORACLE_FULL_SELECT_WORK = 5e9   # per-instance select work n (r d + r^2 / 2) above which the oracle is sampled
+ORACLE_SAMPLE_STEPS = 64
+
+
+def oracle_plan(w):
+    """What the oracle runs per call: (rows, steps).  rows: every query row, or
+    256 seeded rows per head when m is large; steps: every pivot step, or the
+    first 64 of every instance when one instance's select is large (c4b, c4c:
+    tens of seconds of fp64 per instance)."""
     import workloads
 
-    if w.m <= ORACLE_FULL_ROWS_MAX:
-        return None
-    return workloads.sample_rows(w, ORACLE_SAMPLE_ROWS)
+    rows = None if w.m <= ORACLE_FULL_ROWS_MAX else workloads.sample_rows(w, ORACLE_SAMPLE_ROWS)
+    steps = None
+    if w.n * (w.r * w.d + w.r * w.r / 2) > ORACLE_FULL_SELECT_WORK:
+        steps = min(w.r, ORACLE_SAMPLE_STEPS)
+    return rows, steps
 
 
-def oracle_call(orc, w, ex, rows):
-    """One oracle forward (select, weights, value range, gather, attend) on
-    the whole workload, the attend on `rows` (None = every row).  Returns
-    (seconds for a whole call, detail): select and weights are timed in
-    full; a sampled attend is scaled by m / len(rows) (rows cost the same)."""
+def _select_work(w, k):
+    # the oracle's pivot step i costs n (d + i) multiply-adds (kernel column and factor prefix)
+    return w.n * (k * w.d + k * (k - 1) / 2.0)
+
+
+def oracle_call(orc, w, ex, rows, steps=None, ranks=None):
+    """One oracle forward (select, value range, weights, gather, attend),
+    timed per part.  rows: the attend's query rows (None = all); steps: pivot
+    steps run (None = all r).  Returns (seconds for a whole call, detail): a
+    sampled attend is scaled by m / len(rows); with sampled steps the select
+    is scaled by the per-step cost n (d + i) summed to each instance's rank
+    (`ranks`, default r) and the weights and attend by rank / steps (both
+    linear in the coreset size); the value range is timed in full."""
+    s = w.r if steps is None else steps
     t0 = time.perf_counter()
-    sel = orc.rpcholesky(ex["K"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
+    sel = orc.rpcholesky(ex["K"], w.beta, s, seed=w.pivot_seed, eps=EPS)
     t1 = time.perf_counter()
-    VS, wv = orc.weights(sel["F"], sel["S"], sel["rank"], ex["V"])
     vmin, vmax = orc.value_range(ex["V"])
     t2 = time.perf_counter()
+    VS, wv = orc.weights(sel["F"], sel["S"], sel["rank"], ex["V"])
+    t3 = time.perf_counter()
     KS = orc.gather(ex["K"], sel["S"], sel["rank"])
     orc.attend(ex["Q"], KS, VS, wv, sel["rank"], vmin, vmax, w.beta, rows=rows)
-    t3 = time.perf_counter()
-    scale = 1.0 if rows is None else w.m / len(rows)
-    est = (t1 - t0) + (t2 - t1) + (t3 - t2) * scale
-    return est, {"select_s": t1 - t0, "weights_s": t2 - t1, "attend_s": t3 - t2,
-                 "attend_rows": w.m if rows is None else len(rows), "attend_scale": scale}
+    t4 = time.perf_counter()
+    row_scale = 1.0 if rows is None else w.m / len(rows)
+    if steps is None:
+        sel_scale = lin_scale = 1.0
+    else:
+        rk = [w.r] * w.BH if ranks is None else [max(1, int(x)) for x in ranks]
+        sel_scale = statistics.mean(_select_work(w, k) for k in rk) / _select_work(w, s)
+        lin_scale = statistics.mean(rk) / s
+    est = (t1 - t0) * sel_scale + (t2 - t1) + (t3 - t2) * lin_scale + (t4 - t3) * row_scale * lin_scale
+    return est, {"select_s": t1 - t0, "select_steps": s, "select_scale": sel_scale,
+                 "value_range_s": t2 - t1, "weights_s": t3 - t2, "weights_scale": lin_scale,
+                 "attend_s": t4 - t3, "attend_rows": w.m if rows is None else len(rows),
+                 "attend_scale": row_scale * lin_scale}
 
 
-def oracle_sample_text(w, rows, reps=None):
-    if rows is None:
+def oracle_sample_text(w, rows, reps=None, steps=None):
+    if rows is None and steps is None:
         return (f"{reps} whole wildcat_forward calls of the workload ({w.BH} instances), fp64, "
                 "OpenMP over instances")
-    return (f"select and weights in full on all {w.BH} instances, attend on {len(rows)} seeded "
-            f"query rows per head scaled by m / {len(rows)} = {w.m / len(rows):g} (per-row "
-            "extrapolation); fp64, OpenMP over instances")
+    parts = []
+    if steps is None:
+        parts.append(f"select and weights in full on all {w.BH} instances")
+    else:
+        parts.append(f"select on the first {steps} of the r = {w.r} pivot steps of all {w.BH} instances, "
+                     f"scaled by the per-step cost n (d + i) summed to each instance's rank; weights on those "
+                     f"{steps} pivots scaled by rank / {steps}; value range in full")
+    if rows is None:
+        parts.append("attend on every query row")
+    else:
+        parts.append(f"attend on {len(rows)} seeded query rows per head scaled by m / {len(rows)} = "
+                     f"{w.m / len(rows):g}" + ("" if steps is None else f" and rank / {steps}"))
+    return "; ".join(parts) + " (per-part extrapolation); fp64, OpenMP over instances"
 
 
-def cpu_baseline(w, ex, seconds):
+def cpu_baseline(w, ex, seconds, ranks=None):
     """The fp64 oracle, as it stands, on the host cores: whole calls repeated
-    for `seconds`, or one call with a sampled attend when m is large."""
+    for `seconds`, or one sampled call (oracle_plan) when a call is large;
+    `ranks`: the effective rank of every instance from the device run, for
+    the extrapolation of sampled pivot steps."""
     import oracle
 
     orc = oracle.get()
-    rows = oracle_rows(w)
-    if rows is not None:
-        est, det = oracle_call(orc, w, ex, rows)
+    rows, steps = oracle_plan(w)
+    if rows is not None or steps is not None:
+        est, det = oracle_call(orc, w, ex, rows, steps, ranks)
         return {"value": 1.0 / est, "unit": "calls/s", "cores": orc.num_threads(), "kind": "oracle",
-                "partial": True, "sample": oracle_sample_text(w, rows), "seconds_per_call": est,
+                "partial": True, "sample": oracle_sample_text(w, rows, steps=steps), "seconds_per_call": est,
                 "detail": det}
     reps, t0 = 0, time.perf_counter()
     while True:
@@ -291,26 +332,27 @@ def run_reference(args):
     w = workloads.CONFIGS[args.workload]
     _, ex = workloads.make(w)
     orc = oracle.get()
-    rows = oracle_rows(w)
+    rows, steps = oracle_plan(w)
+    whole = rows is None and steps is None
     for _ in range(max(args.warmup, 3)):
-        if rows is None:
+        if whole:
             orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
         else:
-            oracle_call(orc, w, ex, rows)
+            oracle_call(orc, w, ex, rows, steps)
     secs, det = [], None
     for _ in range(args.steps):
-        if rows is None:
+        if whole:
             t0 = time.perf_counter()
             orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
             secs.append(time.perf_counter() - t0)
         else:
-            est, det = oracle_call(orc, w, ex, rows)
+            est, det = oracle_call(orc, w, ex, rows, steps)
             secs.append(est)
     total = sum(secs)
     value = args.steps / total
     cpu = {"value": value, "unit": "calls/s", "cores": orc.num_threads(), "kind": "oracle",
-           "partial": rows is not None,
-           "sample": (oracle_sample_text(w, rows) if rows is not None
+           "partial": not whole,
+           "sample": (oracle_sample_text(w, rows, steps=steps) if not whole
                       else f"one whole wildcat_forward call of the workload per step ({w.BH} instances), fp64")}
     if det is not None:
         cpu["detail_last_step"] = det
@@ -529,7 +571,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_baseline(w, ex, args.cpu_seconds)
+        cpu = cpu_baseline(w, ex, args.cpu_seconds, ranks=plan.rank.cpu().tolist() if nb == 1 else None)
 
     if world > 1:
         barrier()

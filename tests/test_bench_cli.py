@@ -77,6 +77,57 @@ def test_stage_rooflines_recompute():
 
 
 def test_oracle_sampling_rule():
-    assert bench.oracle_rows(workloads.CONFIGS["c1_vit56"]) is None
-    rows = bench.oracle_rows(workloads.CONFIGS["c4c_long128k"])
-    assert len(rows) == 256 and len(set(rows.tolist())) == 256
+    assert bench.oracle_plan(workloads.CONFIGS["c1_vit56"]) == (None, None)
+    assert bench.oracle_plan(workloads.CONFIGS["c4a_long16k"])[1] is None  # select in full
+    rows, steps = bench.oracle_plan(workloads.CONFIGS["c4c_long128k"])
+    assert len(rows) == 256 and len(set(rows.tolist())) == 256 and steps == 64
+
+
+class _FakeOracle:
+    """Stands in for the oracle with fixed part times (seconds)."""
+
+    def __init__(self, clock):
+        self.clock = clock
+
+    def _tick(self, dt):
+        self.clock[0] += dt
+
+    def rpcholesky(self, K, beta, r, seed, eps):
+        self._tick(2.0)
+        return {"F": None, "S": None, "rank": None}
+
+    def value_range(self, V):
+        self._tick(0.5)
+        return None, None
+
+    def weights(self, F, S, rank, V):
+        self._tick(1.0)
+        return None, None
+
+    def gather(self, K, S, rank):
+        return None
+
+    def attend(self, *a, rows=None):
+        self._tick(0.25)
+
+
+def test_oracle_extrapolation(monkeypatch):
+    """A sampled oracle call is scaled part by part: the select by the summed
+    per-step cost to the rank, weights and attend by rank / steps, the attend
+    rows by m / rows, the value range not at all."""
+    w = workloads.CONFIGS["c4c_long128k"]
+    clock = [0.0]
+    monkeypatch.setattr(bench.time, "perf_counter", lambda: clock[0])
+    rows, steps = bench.oracle_plan(w)
+    est, det = bench.oracle_call(_FakeOracle(clock), w, {"K": None, "V": None, "Q": None}, rows, steps)
+    s, r, n, d = 64, w.r, w.n, w.d
+    sel = (r * d + r * (r - 1) / 2) / (s * d + s * (s - 1) / 2)
+    assert det["select_scale"] == pytest.approx(sel)
+    assert est == pytest.approx(2.0 * sel + 0.5 + 1.0 * r / s + 0.25 * (w.m / 256) * (r / s))
+    # with the device's ranks (here half the instances stop at 256)
+    ranks = [512] * 4 + [256] * 4
+    clock[0] = 0.0
+    est2, det2 = bench.oracle_call(_FakeOracle(clock), w, {"K": None, "V": None, "Q": None}, rows, steps, ranks)
+    work = lambda k: k * d + k * (k - 1) / 2
+    assert det2["select_scale"] == pytest.approx((work(512) + work(256)) / 2 / work(64))
+    assert det2["weights_scale"] == pytest.approx(384 / 64)
