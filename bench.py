@@ -584,6 +584,8 @@ def main():
     stages, roof_ms, peaks_used = stage_rooflines(w, ranks, ranks_att, stage_ms, peaks, nb)
     sel = stages["select"]
     ms_per_step = total_ms / args.steps
+    # the select's factor of one rank's batch (bins: the largest instance group in flight is all of it)
+    factor_mb = 4.0 * w.BH * (w.r // nb) * (w.n // nb) * nb / 1e6
     out = {
         "metric": METRIC, "value": value, "unit": "calls/s", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step,
@@ -608,7 +610,12 @@ def main():
                      "frac": sel["frac"], "peak_source": f"{peaks['source']} hbm_gbs",
                      "traffic": None,
                      "algorithmic_bytes_per_call": sel["bytes"], "call_ms": sel["ms"],
-                     "launches_per_call": sel_launches},
+                     "launches_per_call": sel_launches,
+                     "bytes_model": ("streaming model: the factor prefix and keys re-read every step; "
+                                     + ("the factor (%.0f MB) fits in the 126 MB L2, so part of these bytes "
+                                        "are L2 hits and the kernel is bound by its per-step latency, not "
+                                        "DRAM" % (factor_mb,) if factor_mb < 126 else
+                                        "the factor (%.0f MB) exceeds the L2, so these are DRAM bytes" % (factor_mb,)))},
         "gpu_launches": None if launches is None else launches * args.steps,
         "clocks": clk,
         "e2e": e2e,

@@ -11,6 +11,6 @@ def test_profile_commands_leave_clocks_alone():
     files = glob.glob(os.path.join(ROOT, "profiles", "*.md")) + glob.glob(os.path.join(ROOT, "profiles", "*.txt"))
     assert files
     for path in files:
-        text = open(path).read()
+        text = open(path).read().replace("\\\n", " ")  # join continued lines
         for cmd in re.findall(r"ncu --[^\n]*", text):
             assert "--clock-control none" in cmd, f"{os.path.basename(path)}: {cmd}"
