@@ -92,6 +92,8 @@ struct ForwardLayout {
     size_t aws_bytes;
     void* sws;  // select workspace (global-sync mode)
     size_t sws_bytes;
+    void* rws;  // value-range partials (their own region: the range runs beside the select)
+    size_t rws_bytes;
 };
 
 ForwardLayout carve_forward(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, int r, int dtype) {
@@ -110,7 +112,73 @@ ForwardLayout carve_forward(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, 
     L.aws = cv.take(L.aws_bytes);
     L.sws_bytes = wildcat::select_workspace_bytes(BH, n);
     L.sws = cv.take(L.sws_bytes);
+    L.rws_bytes = wildcat::value_range_workspace_bytes(BH, n, d);
+    L.rws = cv.take(L.rws_bytes);
     return L;
+}
+
+// One auxiliary stream and two events per device, created on first use: a
+// forward runs the value range of V there, beside its select (only the
+// attend needs v_min / v_max).  A forward holds the device's mutex from the
+// fork to the join, so calls from several threads do not mix the events.
+struct AuxPipe {
+    std::mutex mu;
+    cudaStream_t s = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+AuxPipe* aux_pipe() {
+    static std::mutex pool_mu;
+    static std::map<int, AuxPipe*> pool;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(pool_mu);
+    auto it = pool.find(dev);
+    if (it != pool.end()) return it->second;
+    AuxPipe* ap = new AuxPipe();
+    bool ok = cudaStreamCreateWithFlags(&ap->s, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&ap->fork, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&ap->join, cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        delete ap;  // the handles that were created are left to the context's teardown
+        return nullptr;
+    }
+    pool[dev] = ap;
+    return ap;
+}
+
+// Starts the value range of V [BH, n, d] on the device's auxiliary stream
+// after the work queued on `st` (and after `wait_v` when given), so that it
+// runs beside the select.  Returns with `lock` holding the device's mutex and
+// *forked set; join_value_range makes `st` wait for the range.  Without an
+// auxiliary stream (*forked false) the caller forms the range on `st`.
+Status fork_value_range(const void* V, int dtype, int64_t BH, int64_t n, int d, float* vmin, float* vmax, void* ws,
+                        size_t ws_bytes, cudaStream_t st, cudaEvent_t wait_v, std::unique_lock<std::mutex>& lock,
+                        AuxPipe** ap_out, bool* forked) {
+    *forked = false;
+    AuxPipe* ap = aux_pipe();
+    *ap_out = ap;
+    if (!ap) return Status::ok();
+    lock = std::unique_lock<std::mutex>(ap->mu);
+    cudaError_t e;
+    if ((e = cudaEventRecord(ap->fork, st))) return Status::cuda(e, "forward: fork");
+    if ((e = cudaStreamWaitEvent(ap->s, ap->fork, 0))) return Status::cuda(e, "forward: fork");
+    if (wait_v && (e = cudaStreamWaitEvent(ap->s, wait_v, 0))) return Status::cuda(e, "forward: wait for V");
+    const Status z = wildcat::launch_value_range(V, dtype, BH, n, d, vmin, vmax, ws, ws_bytes, ap->s);
+    if (z.code) return z;
+    if ((e = cudaEventRecord(ap->join, ap->s))) return Status::cuda(e, "forward: join");
+    *forked = true;
+    return Status::ok();
+}
+
+Status join_value_range(AuxPipe* ap, cudaStream_t st, std::unique_lock<std::mutex>& lock) {
+    const cudaError_t e = cudaStreamWaitEvent(st, ap->join, 0);
+    lock.unlock();
+    return e ? Status::cuda(e, "forward: join") : Status::ok();
 }
 
 // Stage markers (wildcat_set_stage_events): caller-owned events recorded on
@@ -131,6 +199,12 @@ wildcat_status forward_impl(const void* Q, const void* K, const void* V, int dty
                             cudaEvent_t wait_v = nullptr, cudaEvent_t wait_q = nullptr) {
     Status s;
     cudaError_t ew;
+    std::unique_lock<std::mutex> aux_lock;
+    AuxPipe* ap = nullptr;
+    bool forked = false;
+    if ((s = fork_value_range(V, dtype, BH, n, d, L.vmin, L.vmax, L.rws, L.rws_bytes, st, wait_v, aux_lock, &ap,
+                              &forked)).code)
+        return record(s);
     wildcat::SelectRequest sq{K, dtype, BH, n, d, beta, r, seed, inst0, eps, nullptr, L.S, L.F, L.rank, L.K_S};
     sq.ws = L.sws;
     sq.ws_bytes = L.sws_bytes;
@@ -139,8 +213,10 @@ wildcat_status forward_impl(const void* Q, const void* K, const void* V, int dty
     if (wait_v && (ew = cudaStreamWaitEvent(st, wait_v, 0))) return record(Status::cuda(ew, "forward: wait for V"));
     wildcat::WeightsRequest wq{L.F, L.S, L.rank, V, dtype, BH, n, d, r, L.V_S, L.w, L.vmin, L.vmax, L.wws,
                                L.wws_bytes};
+    wq.skip_range = forked;
     if ((s = wildcat::launch_weights(wq, st)).code) return record(s);
     if ((s = mark_stage(g_ev_after_weights, st, "forward: stage event")).code) return record(s);
+    if (forked && (s = join_value_range(ap, st, aux_lock)).code) return record(s);
     if (wait_q && (ew = cudaStreamWaitEvent(st, wait_q, 0))) return record(Status::cuda(ew, "forward: wait for Q"));
     if (m > 0) {
         wildcat::AttendRequest aq{Q,   L.K_S,  dtype, BH, m, d, r, L.rank, beta, L.V_S, L.w,
@@ -175,6 +251,8 @@ struct BinnedLayout {
     void* mws;
     void* sws;     // select workspace (global-sync mode)
     size_t sws_bytes;
+    void* rws;     // value-range partials of the bins
+    size_t rws_bytes;
 };
 
 BinnedLayout carve_binned(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, int r, int nbins, int dtype,
@@ -202,6 +280,8 @@ BinnedLayout carve_binned(Carve& cv, int64_t BH, int64_t m, int64_t n, int d, in
     L.mws = recenter ? cv.take(wildcat::key_mean_workspace_bytes(BH, n, d)) : nullptr;
     L.sws_bytes = wildcat::select_workspace_bytes(BB, nb);
     L.sws = cv.take(L.sws_bytes);
+    L.rws_bytes = wildcat::value_range_workspace_bytes(BB, nb, d);
+    L.rws = cv.take(L.rws_bytes);
     return L;
 }
 
@@ -508,6 +588,12 @@ wildcat_status forward_ex_impl(const void* Q, const void* K, const void* V, int 
     const int rb = r / nbins;
     Status z;
     cudaError_t ew;
+    std::unique_lock<std::mutex> aux_lock;
+    AuxPipe* ap = nullptr;
+    bool forked = false;
+    if ((z = fork_value_range(V, dtype, BB, nb, d, L.vmin_b, L.vmax_b, L.rws, L.rws_bytes, s, wait_v, aux_lock, &ap,
+                              &forked)).code)
+        return record(z);
     if (o.recenter && (z = wildcat::launch_key_mean(K, dtype, BH, n, d, L.mws, L.kbar, s)).code) return record(z);
     wildcat::SelectRequest sq{K,      dtype, BB,      nb,  d,     o.beta_key, rb,      seed, inst0 * nbins,
                               eps,    nullptr, L.S,   L.F, L.rank_b, L.K_S,   L.kbar,  nbins};
@@ -518,8 +604,10 @@ wildcat_status forward_ex_impl(const void* Q, const void* K, const void* V, int 
     if (wait_v && (ew = cudaStreamWaitEvent(s, wait_v, 0))) return record(Status::cuda(ew, "forward: wait for V"));
     wildcat::WeightsRequest wq{L.F, L.S, L.rank_b, V, dtype, BB, nb, d, rb, L.V_S, L.w, L.vmin_b, L.vmax_b, L.wws,
                                L.wws_bytes};
+    wq.skip_range = forked;
     if ((z = wildcat::launch_weights(wq, s)).code) return record(z);
     if ((z = mark_stage(g_ev_after_weights, s, "forward: stage event")).code) return record(z);
+    if (forked && (z = join_value_range(ap, s, aux_lock)).code) return record(z);
     if ((z = wildcat::launch_binning_finish(L.vmin_b, L.vmax_b, L.S, L.rank_b, BH, nbins, nb, rb, d, L.vmin, L.vmax,
                                             L.rank_att, S_out, rank_out, s)).code)
         return record(z);

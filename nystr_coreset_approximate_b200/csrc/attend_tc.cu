@@ -676,6 +676,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
     }
     const bool go = *x.abort_flag == 0;
+    // the preparation grid (V_S^T, w, kmax) has finished and its writes are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
@@ -701,11 +703,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // V_S^T rounded to bf16 and w zero-padded to rpad rows, both zero at and past
-// the rank: VT[b, c, l] for c < D, l < rpad; wpad[b, l].
+// the rank: VT[b, c, l] for c < D, l < rpad; wpad[b, l].  The first block of
+// each instance also forms kmax[b] = max_{l < rank} |K_S[b, l]| (the
+// pivot-key half of the per-row shift).  The attend kernel that follows is
+// launched as a programmatic dependent: it may start its prologue now and
+// waits for this grid before it reads VT, wpad or kmax.
 template <int D>
 __global__ void vt_prep_kernel(const float* __restrict__ V_S, const float* __restrict__ w,
-                               const int32_t* __restrict__ rank, int r, int rpad, __nv_bfloat16* __restrict__ VT,
-                               float* __restrict__ wpad) {
+                               const __nv_bfloat16* __restrict__ K_S, const int32_t* __restrict__ rank, int r,
+                               int rpad, __nv_bfloat16* __restrict__ VT, float* __restrict__ wpad,
+                               float* __restrict__ kmax) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ float tile[32][33];
     const int64_t b = blockIdx.z;
     const int l0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
@@ -721,16 +729,10 @@ __global__ void vt_prep_kernel(const float* __restrict__ V_S, const float* __res
         const int l = l0 + threadIdx.x;
         wpad[b * rpad + l] = l < rr ? w[b * r + l] : 0.f;
     }
-}
-
-// kmax[b] = max_{l < rank} |K_S[b, l]| (the pivot-key half of the per-row shift)
-template <int D>
-__global__ void kmax_kernel(const __nv_bfloat16* __restrict__ K_S, const int32_t* __restrict__ rank, int r,
-                            float* __restrict__ kmax) {
-    const int64_t b = blockIdx.x;
-    const int rr = rank[b];
+    if (blockIdx.x != 0 || blockIdx.y != 0) return;  // uniform per block
+    const int tid = threadIdx.y * blockDim.x + threadIdx.x, nt = blockDim.x * blockDim.y;
     float best = 0.f;
-    for (int l = threadIdx.x; l < rr; l += blockDim.x) {
+    for (int l = tid; l < rr; l += nt) {
         const uint4* k4 = reinterpret_cast<const uint4*>(K_S + (b * r + l) * D);
         float s = 0.f;
 #pragma unroll
@@ -744,11 +746,11 @@ __global__ void kmax_kernel(const __nv_bfloat16* __restrict__ K_S, const int32_t
     }
     best = warp_max(best);
     __shared__ float wb[32];
-    if ((threadIdx.x & 31) == 0) wb[threadIdx.x >> 5] = best;
+    if ((tid & 31) == 0) wb[tid >> 5] = best;
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
         float v = 0.f;
-        for (int k = 0; k < (int)(blockDim.x >> 5); ++k) v = fmaxf(v, wb[k]);
+        for (int k = 0; k < nt / 32; ++k) v = fmaxf(v, wb[k]);
         kmax[b] = v;
     }
 }
@@ -773,8 +775,7 @@ Status run_tc(const AttendRequest& q, void* scratch, cudaStream_t st) {
     p += round_up((int64_t)sizeof(float) * q.BH * rpad, 256);
     float* kmax = reinterpret_cast<float*>(p);
     vt_prep_kernel<D><<<dim3((unsigned)(rpad / 32), D / 32, (unsigned)q.BH), dim3(32, 8), 0, st>>>(
-        q.V_S, q.w, q.rank, q.r, rpad, VT, wpad);
-    kmax_kernel<D><<<(unsigned)q.BH, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(q.K_S), q.rank, q.r, kmax);
+        q.V_S, q.w, static_cast<const __nv_bfloat16*>(q.K_S), q.rank, q.r, rpad, VT, wpad, kmax);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return Status::cuda(e, "attend_tc: prep launch");
     if (q.m == 0) return Status::ok();
@@ -792,9 +793,21 @@ Status run_tc(const AttendRequest& q, void* scratch, cudaStream_t st) {
     const int64_t units = ceil_div(q.m, 2 * kRows) * q.BH;
     if (units >= (int64_t(1) << 31)) return Status::fail(2, "attend_tc: more than 2^31 query-tile pairs");
     const unsigned grid = (unsigned)std::min<int64_t>(units, sm_count());
-    attend_tc_kernel<D><<<grid, kThreads, C::total, st>>>(tmQ, tmK, tmV, tmO, wpad, rpad, q.m, q.BH, q.rank, q.beta,
-                                                         q.vmin, q.vmax, kmax, g_force_timeout_ns);
-    e = cudaGetLastError();
+    // a programmatic dependent of vt_prep_kernel: its prologue overlaps the
+    // preparation, and it waits for that grid before the first read of VT, wpad, kmax
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::total;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, attend_tc_kernel<D>, tmQ, tmK, tmV, tmO, (const float*)wpad, rpad, (int64_t)q.m,
+                           (int64_t)q.BH, q.rank, q.beta, q.vmin, q.vmax, (const float*)kmax, g_force_timeout_ns);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return Status::cuda(e, "attend_tc launch");
     return Status::ok();
 }

@@ -81,6 +81,7 @@ struct WeightsRequest {
     float* vmax;
     void* ws;
     size_t ws_bytes;
+    bool skip_range = false;  // vmin / vmax are formed elsewhere (launch_value_range)
 };
 size_t weights_workspace_bytes(int64_t BH, int64_t n, int d, int r);
 Status launch_weights(const WeightsRequest& q, cudaStream_t stream);

@@ -523,10 +523,12 @@ Status run_weights(const WeightsRequest& q, cudaStream_t st) {
     using T = typename E::T;
     const T* V = static_cast<const T*>(q.V);
 
-    colrange_partial<E, D><<<dim3(p.nsplit_range, (unsigned)q.BH), kRangeThreads, 0, st>>>(V, q.n, p.rows_per_range,
-                                                                                           part);
-    colrange_finalize<<<(unsigned)ceil_div(q.BH * D, 256), 256, 0, st>>>(part, p.nsplit_range, D, q.BH, q.vmin,
-                                                                          q.vmax);
+    if (!q.skip_range) {
+        colrange_partial<E, D><<<dim3(p.nsplit_range, (unsigned)q.BH), kRangeThreads, 0, st>>>(V, q.n,
+                                                                                               p.rows_per_range, part);
+        colrange_finalize<<<(unsigned)ceil_div(q.BH * D, 256), 256, 0, st>>>(part, p.nsplit_range, D, q.BH, q.vmin,
+                                                                              q.vmax);
+    }
     int nsplit = p.nsplit_k;
     if (weights_tc_supported(q.dtype, D, q.n)) {
         nsplit = p.nsplit_tc;
