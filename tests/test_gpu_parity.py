@@ -309,3 +309,53 @@ def test_bounded_wait_reports_timeout_and_recovers():
     O = wc.attend(d["Q"], K_S, rank, w.beta, V_S, wv, vmin, vmax)
     assert wc.device_status() == 0
     assert torch.isfinite(O).all()
+
+
+def test_concurrent_forwards_on_two_streams():
+    """Two host threads run forwards at the same time, each on its own stream
+    (the forwards fork their value range onto the library's per-device
+    auxiliary stream under a per-device lock); every result equals the same
+    forward run alone, bit for bit."""
+    import threading
+
+    cases = [gc.case("conc_plain", "iid", 4, 3000, 1000, 64, 64, "bf16"),
+             gc.case("conc_binned", "normclip", 3, 4096, 700, 128, 96, "bf16", seed=9)]
+    inputs, refs = [], []
+    for k, w in enumerate(cases):
+        dev, _ = workloads.make(w)
+        d = gc.cuda_inputs(dev)
+        inputs.append(d)
+        if k == 0:
+            refs.append(wc.forward(d["Q"], d["K"], d["V"], w.beta, w.r, 5, EPS))
+        else:
+            refs.append(wc.forward_ex(d["Q"], d["K"], d["V"], w.beta, w.r, 5, EPS, nbins=2))
+    torch.cuda.synchronize()
+    out, errs = [None, None], []
+
+    def run(k):
+        try:
+            w, d = cases[k], inputs[k]
+            s = torch.cuda.Stream()
+            res = []
+            with torch.cuda.stream(s):
+                for _ in range(6):
+                    if k == 0:
+                        r = wc.forward(d["Q"], d["K"], d["V"], w.beta, w.r, 5, EPS, stream=s)
+                    else:
+                        r = wc.forward_ex(d["Q"], d["K"], d["V"], w.beta, w.r, 5, EPS, nbins=2, stream=s)
+                    res.append(r)
+            s.synchronize()
+            out[k] = res
+        except Exception as e:  # reported below
+            errs.append(e)
+
+    th = [threading.Thread(target=run, args=(k,)) for k in range(2)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    assert not errs, errs
+    assert wc.device_status() == 0
+    for k in range(2):
+        for O, S, rank in out[k]:
+            assert torch.equal(S, refs[k][1]) and torch.equal(rank, refs[k][2]) and torch.equal(O, refs[k][0])
