@@ -275,8 +275,13 @@ wildcat_status wildcat_attend_noalloc(const void* Q, const void* K_S, int dtype,
 
 /*
  * wildcat_forward -- the whole module (Alg. 4): select -> weights -> attend,
- * all on `stream`, with every intermediate in `workspace`.  seed, inst0 and
- * eps as in wildcat_select.
+ * on `stream`, with every intermediate in `workspace`.  seed, inst0 and eps
+ * as in wildcat_select.  The value range of V (needed only by the attend)
+ * runs on a library-owned stream of the current device, forked from `stream`
+ * before the select and joined back before the attend, so it overlaps the
+ * select; the same holds for wildcat_forward_ex / _binned / _host /
+ * _ex_host.  A per-device lock covers each call's fork-to-join section, so
+ * calls from several threads are correct (their value ranges serialize).
  *
  *   Q [BH, m, d], K and V [BH, n, d] (dtype `dtype`); O out [BH, m, d] float32
  *   S_out [BH, r] int32 and rank_out [BH] int32: optional outputs (or NULL);
