@@ -24,11 +24,11 @@ max(bytes / HBM, MMA flops / tensor peak, exps / MUFU rate) against the
 measured step time), the roofline of the dominant kernel, sampled SM clocks,
 and the oracle timed on the host cores as a CPU baseline.  Where the oracle
 cannot afford a whole call it runs a stated sample and extrapolates each
-part (the line says so): the attend on 256 seeded rows per head when m >
-4096, and, when one instance's select is large (the 65536- and 131072-token
-workloads), the first 64 pivot steps of every instance, scaled by the
-per-step cost n (d + i) to the rank, with the weights and attend on those 64
-pivots scaled by rank / 64.
+part from two sample sizes, a fixed cost plus a cost that grows with the
+size (the line says so): when m > 4096 the attend on 1024 and 4096 seeded
+rows per head, and, when one instance's select is large (the 65536- and
+131072-token workloads), the select and weights on the first 32 and 64
+pivot steps of every instance (step i of the select costs n (d + i)).
 """
 from __future__ import annotations
 
@@ -41,6 +41,8 @@ import subprocess
 import sys
 import tempfile
 import time
+
+import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
@@ -221,6 +223,7 @@ class ClockSampler:
 
 ORACLE_FULL_SELECT_WORK = 5e9   # per-instance select work n (r d + r^2 / 2) above which the oracle is sampled
 ORACLE_SAMPLE_STEPS = 64
+ORACLE_TIMING_ROWS = 4096       # rows of the larger sample that times a sampled attend
 
 
 def oracle_plan(w):
@@ -242,37 +245,81 @@ def _select_work(w, k):
     return w.n * (k * w.d + k * (k - 1) / 2.0)
 
 
+def _timed(fn):
+    t0 = time.perf_counter()
+    out = fn()
+    return out, time.perf_counter() - t0
+
+
 def oracle_call(orc, w, ex, rows, steps=None, ranks=None):
     """One oracle forward (select, value range, weights, gather, attend),
     timed per part.  rows: the attend's query rows (None = all); steps: pivot
-    steps run (None = all r).  Returns (seconds for a whole call, detail): a
-    sampled attend is scaled by m / len(rows); with sampled steps the select
-    is scaled by the per-step cost n (d + i) summed to each instance's rank
-    (`ranks`, default r) and the weights and attend by rank / steps (both
-    linear in the coreset size); the value range is timed in full."""
+    steps run (None = all r).  Returns (seconds for a whole call, detail).
+    With sampled steps the select and weights also run on half the steps, and
+    a fixed part plus a part growing with the steps (the select's step i
+    costs n (d + i); the weights grow with the coreset size) are fitted and
+    taken to each instance's rank (`ranks`, default r); the value range is
+    timed in full.  A sampled attend runs with a coreset of the full size r (the
+    first r keys when the steps were sampled: its cost depends on the sizes
+    only) on half of `rows` and on all of them, and is extrapolated to m rows
+    by the fitted cost: a fixed part (the query-norm pass over all m rows,
+    the setup) plus a per-row part."""
     s = w.r if steps is None else steps
-    t0 = time.perf_counter()
-    sel = orc.rpcholesky(ex["K"], w.beta, s, seed=w.pivot_seed, eps=EPS)
-    t1 = time.perf_counter()
-    vmin, vmax = orc.value_range(ex["V"])
-    t2 = time.perf_counter()
-    VS, wv = orc.weights(sel["F"], sel["S"], sel["rank"], ex["V"])
-    t3 = time.perf_counter()
-    KS = orc.gather(ex["K"], sel["S"], sel["rank"])
-    orc.attend(ex["Q"], KS, VS, wv, sel["rank"], vmin, vmax, w.beta, rows=rows)
-    t4 = time.perf_counter()
-    row_scale = 1.0 if rows is None else w.m / len(rows)
+    sel, t_sel = _timed(lambda: orc.rpcholesky(ex["K"], w.beta, s, seed=w.pivot_seed, eps=EPS))
+    (vmin, vmax), t_rng = _timed(lambda: orc.value_range(ex["V"]))
+    (VS, wv), t_wt = _timed(lambda: orc.weights(sel["F"], sel["S"], sel["rank"], ex["V"]))
+    if steps is not None:
+        # the same on half the steps: a fixed part (the prologue's pass over
+        # the keys, setup) and a part that grows with the steps are fitted
+        s2 = max(1, s // 2)
+        sel2, t_sel2 = _timed(lambda: orc.rpcholesky(ex["K"], w.beta, s2, seed=w.pivot_seed, eps=EPS))
+        _, t_wt2 = _timed(lambda: orc.weights(sel2["F"], sel2["S"], sel2["rank"], ex["V"]))
+    KS, rank_att = orc.gather(ex["K"], sel["S"], sel["rank"]), sel["rank"]
+    if steps is not None:
+        # a coreset of the full size for timing the attend (its values do not change its cost)
+        full = np.tile(np.arange(w.r, dtype=np.int32), (w.BH, 1))
+        rank_att = np.full(w.BH, w.r, dtype=np.int32)
+        KS = orc.gather(ex["K"], full, rank_att)
+        VS = np.zeros((w.BH, w.r, w.d))
+        wv = np.ones((w.BH, w.r))
+
+    def att(rs):
+        return _timed(lambda: orc.attend(ex["Q"], KS, VS, wv, rank_att, vmin, vmax, w.beta, rows=rs))[1]
+
+    if rows is None:
+        t_att = att(None)
+        att_det = {"attend_s": t_att, "attend_rows": w.m}
+    else:
+        import workloads
+
+        # two seeded row samples large enough that the per-row cost shows
+        # above the fixed part (rows cost the same)
+        na, nb = min(w.m, ORACLE_TIMING_ROWS // 4), min(w.m, ORACLE_TIMING_ROWS)
+        t1, t2 = att(workloads.sample_rows(w, na)), att(workloads.sample_rows(w, nb))
+        per_row = max(0.0, (t2 - t1) / (nb - na))
+        fixed = max(0.0, t1 - per_row * na)
+        t_att = fixed + per_row * w.m
+        att_det = {"attend_rows_timed": [na, nb], "attend_s_timed": [t1, t2], "attend_fixed_s": fixed,
+                   "attend_per_row_s": per_row, "attend_extrapolated_s": t_att}
     if steps is None:
-        sel_scale = lin_scale = 1.0
+        est_sel, est_wt = t_sel, t_wt
+        det = {"select_s": t_sel, "weights_s": t_wt}
     else:
         rk = [w.r] * w.BH if ranks is None else [max(1, int(x)) for x in ranks]
-        sel_scale = statistics.mean(_select_work(w, k) for k in rk) / _select_work(w, s)
-        lin_scale = statistics.mean(rk) / s
-    est = (t1 - t0) * sel_scale + (t2 - t1) + (t3 - t2) * lin_scale + (t4 - t3) * row_scale * lin_scale
-    return est, {"select_s": t1 - t0, "select_steps": s, "select_scale": sel_scale,
-                 "value_range_s": t2 - t1, "weights_s": t3 - t2, "weights_scale": lin_scale,
-                 "attend_s": t4 - t3, "attend_rows": w.m if rows is None else len(rows),
-                 "attend_scale": row_scale * lin_scale}
+        # select: fixed + b * work(steps), work = n (steps d + steps (steps - 1) / 2)
+        b_sel = max(0.0, (t_sel - t_sel2) / (_select_work(w, s) - _select_work(w, s2)))
+        a_sel = max(0.0, t_sel - b_sel * _select_work(w, s))
+        est_sel = a_sel + b_sel * statistics.mean(_select_work(w, k) for k in rk)
+        # weights: fixed + b * coreset size
+        b_wt = max(0.0, (t_wt - t_wt2) / (s - s2))
+        a_wt = max(0.0, t_wt - b_wt * s)
+        est_wt = a_wt + b_wt * statistics.mean(rk)
+        det = {"select_steps_timed": [s2, s], "select_s_timed": [t_sel2, t_sel], "select_extrapolated_s": est_sel,
+               "weights_s_timed": [t_wt2, t_wt], "weights_extrapolated_s": est_wt}
+    est = est_sel + t_rng + est_wt + t_att
+    det["value_range_s"] = t_rng
+    det.update(att_det)
+    return est, det
 
 
 def oracle_sample_text(w, rows, reps=None, steps=None):
@@ -283,15 +330,17 @@ def oracle_sample_text(w, rows, reps=None, steps=None):
     if steps is None:
         parts.append(f"select and weights in full on all {w.BH} instances")
     else:
-        parts.append(f"select on the first {steps} of the r = {w.r} pivot steps of all {w.BH} instances, "
-                     f"scaled by the per-step cost n (d + i) summed to each instance's rank; weights on those "
-                     f"{steps} pivots scaled by rank / {steps}; value range in full")
+        parts.append(f"select on the first {steps // 2} and {steps} of the r = {w.r} pivot steps of all {w.BH} "
+                     f"instances, extrapolated to each instance's rank by the fitted fixed + per-step cost "
+                     f"(step i costs n (d + i)); weights on those pivots, extrapolated linearly in the coreset "
+                     f"size; value range in full")
     if rows is None:
         parts.append("attend on every query row")
     else:
-        parts.append(f"attend on {len(rows)} seeded query rows per head scaled by m / {len(rows)} = "
-                     f"{w.m / len(rows):g}" + ("" if steps is None else f" and rank / {steps}"))
-    return "; ".join(parts) + " (per-part extrapolation); fp64, OpenMP over instances"
+        parts.append(f"attend with an r-row coreset on {ORACLE_TIMING_ROWS // 4} and {ORACLE_TIMING_ROWS} "
+                     f"seeded query rows per head, extrapolated to m = {w.m} rows by the fitted fixed + "
+                     "per-row cost")
+    return "; ".join(parts) + "; fp64, OpenMP over instances"
 
 
 def cpu_baseline(w, ex, seconds, ranks=None):

@@ -6,6 +6,7 @@ import os
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -84,50 +85,55 @@ def test_oracle_sampling_rule():
 
 
 class _FakeOracle:
-    """Stands in for the oracle with fixed part times (seconds)."""
+    """Stands in for the oracle: each part's time is a fixed cost plus a cost
+    that grows with its size, so the bench's extrapolation can be checked
+    against the exact time of a whole call."""
 
-    def __init__(self, clock):
-        self.clock = clock
+    def __init__(self, clock, w):
+        self.clock, self.w = clock, w
 
-    def _tick(self, dt):
-        self.clock[0] += dt
+    def sel_time(self, k):
+        return 0.3 + 2e-12 * self.w.n * (k * self.w.d + k * (k - 1) / 2)
+
+    def wt_time(self, k):
+        return 0.2 + 0.01 * k
+
+    def att_time(self, nrows):
+        return 0.05 + 1e-5 * nrows
 
     def rpcholesky(self, K, beta, r, seed, eps):
-        self._tick(2.0)
-        return {"F": None, "S": None, "rank": None}
+        self.clock[0] += self.sel_time(r)
+        return {"F": None, "S": np.zeros((self.w.BH, r), np.int32), "rank": np.full(self.w.BH, r, np.int32)}
 
     def value_range(self, V):
-        self._tick(0.5)
+        self.clock[0] += 0.5
         return None, None
 
     def weights(self, F, S, rank, V):
-        self._tick(1.0)
+        self.clock[0] += self.wt_time(S.shape[1])
         return None, None
 
     def gather(self, K, S, rank):
         return None
 
     def attend(self, *a, rows=None):
-        self._tick(0.25)
+        self.clock[0] += self.att_time(self.w.m if rows is None else len(rows))
 
 
 def test_oracle_extrapolation(monkeypatch):
-    """A sampled oracle call is scaled part by part: the select by the summed
-    per-step cost to the rank, weights and attend by rank / steps, the attend
-    rows by m / rows, the value range not at all."""
+    """A sampled oracle call is extrapolated part by part from two sample
+    sizes (fixed + growing cost): with part times that follow that model
+    exactly, the estimate equals the whole call's time."""
     w = workloads.CONFIGS["c4c_long128k"]
     clock = [0.0]
     monkeypatch.setattr(bench.time, "perf_counter", lambda: clock[0])
+    fake = _FakeOracle(clock, w)
     rows, steps = bench.oracle_plan(w)
-    est, det = bench.oracle_call(_FakeOracle(clock), w, {"K": None, "V": None, "Q": None}, rows, steps)
-    s, r, n, d = 64, w.r, w.n, w.d
-    sel = (r * d + r * (r - 1) / 2) / (s * d + s * (s - 1) / 2)
-    assert det["select_scale"] == pytest.approx(sel)
-    assert est == pytest.approx(2.0 * sel + 0.5 + 1.0 * r / s + 0.25 * (w.m / 256) * (r / s))
+    est, det = bench.oracle_call(fake, w, {"K": None, "V": None, "Q": None}, rows, steps)
+    whole = fake.sel_time(w.r) + 0.5 + fake.wt_time(w.r) + fake.att_time(w.m)
+    assert est == pytest.approx(whole, rel=1e-9)
     # with the device's ranks (here half the instances stop at 256)
     ranks = [512] * 4 + [256] * 4
-    clock[0] = 0.0
-    est2, det2 = bench.oracle_call(_FakeOracle(clock), w, {"K": None, "V": None, "Q": None}, rows, steps, ranks)
-    work = lambda k: k * d + k * (k - 1) / 2
-    assert det2["select_scale"] == pytest.approx((work(512) + work(256)) / 2 / work(64))
-    assert det2["weights_scale"] == pytest.approx(384 / 64)
+    est2, _ = bench.oracle_call(fake, w, {"K": None, "V": None, "Q": None}, rows, steps, ranks)
+    sel = 0.3 + 2e-12 * w.n * ((512 * w.d + 512 * 511 / 2) + (256 * w.d + 256 * 255 / 2)) / 2
+    assert est2 == pytest.approx(sel + 0.5 + (0.2 + 0.01 * 384) + fake.att_time(w.m), rel=1e-9)
