@@ -352,9 +352,11 @@ def cpu_baseline(w, ex, seconds, ranks=None):
 
     orc = oracle.get()
     rows, steps = oracle_plan(w)
+    T = orc.num_threads()
+    used = {"select_and_weights": min(w.BH, T), "attend": T}  # OpenMP over instances / over query rows
     if rows is not None or steps is not None:
         est, det = oracle_call(orc, w, ex, rows, steps, ranks)
-        return {"value": 1.0 / est, "unit": "calls/s", "cores": orc.num_threads(), "kind": "oracle",
+        return {"value": 1.0 / est, "unit": "calls/s", "cores": T, "threads_used": used, "kind": "oracle",
                 "partial": True, "sample": oracle_sample_text(w, rows, steps=steps), "seconds_per_call": est,
                 "detail": det}
     reps, t0 = 0, time.perf_counter()
@@ -364,7 +366,7 @@ def cpu_baseline(w, ex, seconds, ranks=None):
         el = time.perf_counter() - t0
         if el >= seconds:
             break
-    return {"value": reps / el, "unit": "calls/s", "cores": orc.num_threads(), "kind": "oracle",
+    return {"value": reps / el, "unit": "calls/s", "cores": T, "threads_used": used, "kind": "oracle",
             "partial": False, "sample": oracle_sample_text(w, None, reps)}
 
 
@@ -399,7 +401,9 @@ def run_reference(args):
             secs.append(est)
     total = sum(secs)
     value = args.steps / total
-    cpu = {"value": value, "unit": "calls/s", "cores": orc.num_threads(), "kind": "oracle",
+    T = orc.num_threads()
+    cpu = {"value": value, "unit": "calls/s", "cores": T, "kind": "oracle",
+           "threads_used": {"select_and_weights": min(w.BH, T), "attend": T},
            "partial": not whole,
            "sample": (oracle_sample_text(w, rows, steps=steps) if not whole
                       else f"one whole wildcat_forward call of the workload per step ({w.BH} instances), fp64")}
