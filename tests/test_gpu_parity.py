@@ -359,3 +359,19 @@ def test_concurrent_forwards_on_two_streams():
     for k in range(2):
         for O, S, rank in out[k]:
             assert torch.equal(S, refs[k][1]) and torch.equal(rank, refs[k][2]) and torch.equal(O, refs[k][0])
+
+
+def test_forward_without_queries():
+    """m = 0: the forward selects and forms the weights (pivots and ranks as
+    with queries) and launches no attend; the host-buffer forward agrees."""
+    w = gc.case("no_queries", "mixture16", 3, 1024, 64, 64, 48, "bf16")
+    dev, _ = workloads.make(w)
+    d = gc.cuda_inputs(dev)
+    O, S, rank = wc.forward(d["Q"], d["K"], d["V"], w.beta, w.r, 3, EPS)
+    Q0 = d["Q"][:, :0].contiguous()
+    O0, S0, rank0 = wc.forward(Q0, d["K"], d["V"], w.beta, w.r, 3, EPS)
+    assert O0.shape == (3, 0, 64)
+    assert torch.equal(S0, S) and torch.equal(rank0, rank)
+    Oe, Se, re_ = wc.forward_ex(Q0, d["K"], d["V"], w.beta, w.r, 3, EPS, nbins=2)
+    assert Oe.shape == (3, 0, 64) and torch.all(re_ >= 1)
+    assert wc.device_status() == 0
