@@ -364,7 +364,7 @@ def test_concurrent_forwards_on_two_streams():
 def test_forward_without_queries():
     """m = 0: the forward selects and forms the weights (pivots and ranks as
     with queries) and launches no attend; the host-buffer forward agrees."""
-    w = gc.case("no_queries", "mixture16", 3, 1024, 64, 64, 48, "bf16")
+    w = gc.case("no_queries", "iid", 3, 1024, 64, 64, 48, "bf16")
     dev, _ = workloads.make(w)
     d = gc.cuda_inputs(dev)
     O, S, rank = wc.forward(d["Q"], d["K"], d["V"], w.beta, w.r, 3, EPS)
