@@ -39,7 +39,6 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
 
 // Streaming loads that bypass L1 (data written by other SMs of the cluster,
 // or read once per step).
-__device__ __forceinline__ float4 ld_cg4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
 __device__ __forceinline__ float ld_cg1(const float* p) { return __ldcg(p); }
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -55,11 +54,6 @@ __device__ __forceinline__ double warp_sum(double v) {
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-__device__ __forceinline__ float warp_min(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
 }
 

@@ -105,19 +105,6 @@ __device__ __forceinline__ void tmem_ld16(unsigned taddr, float (&v)[16]) {
     for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
 }
 
-__device__ __forceinline__ void cp_async16_zfill(unsigned dst, const void* src, bool ok) {
-    const int n = ok ? 16 : 0;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// all but the N most recent committed groups have landed
-template <int N>
-__device__ __forceinline__ void cp_async_wait_group() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 
 }  // namespace tc
@@ -161,20 +148,6 @@ __device__ __forceinline__ void mbar_expect_tx(void* mbar, unsigned bytes) {
                  : "memory");
 }
 
-// Bounded wait that also gives up as soon as *abort is set (by another role
-// of the same CTA whose own wait expired).  Returns false on either.
-__device__ __forceinline__ bool mbar_wait_or_abort(void* mbar, unsigned parity, const volatile int* abort,
-                                                   unsigned long long limit_ns = kWaitLimitNs) {
-    const unsigned a = smem_u32(mbar);
-    if (mbar_try(a, parity)) return true;
-    const unsigned long long t0 = globaltimer();
-    for (;;) {
-        if (mbar_try(a, parity)) return true;
-        if (*abort) return false;
-        if (globaltimer() - t0 > limit_ns) return false;
-    }
-}
-
 // 3-D tiled TMA load (tensor map in kernel-parameter space) into shared
 // memory, completion counted in bytes on `mbar`.
 __device__ __forceinline__ void tma_load_3d(unsigned dst, const void* tmap, int x, int y, int z, void* mbar) {
@@ -192,7 +165,6 @@ __device__ __forceinline__ void tma_store_3d(const void* tmap, int x, int y, int
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // all but the most recent bulk group have finished reading their source
 __device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -228,17 +200,6 @@ __device__ __forceinline__ void mma_bf16_ts_w(unsigned tmem_d, unsigned tmem_a, 
         "setp.ne.b32 p, %5, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}\n" ::"r"(tmem_d),
         "r"(tmem_a), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// D (tmem) (+)= A (tmem, 128 lanes x K packed bf16 pairs) * B (smem descriptor)
-__device__ __forceinline__ void mma_bf16_ts(unsigned tmem_d, unsigned tmem_a, uint64_t b, uint32_t idesc,
-                                            int accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(tmem_d),
-        "r"(tmem_a), "l"(b), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
