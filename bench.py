@@ -343,31 +343,70 @@ def oracle_sample_text(w, rows, reps=None, steps=None):
     return "; ".join(parts) + "; fp64, OpenMP over instances"
 
 
-def cpu_baseline(w, ex, seconds, ranks=None):
+def oracle_binned_call(orc, w, ex, nb):
+    """One oracle binned forward (nb bins): whole when m <= 4096, else the
+    whole call on 1024 and on 4096 seeded query rows per head, extrapolated to
+    m rows by the fitted fixed (select, weights, query pass) + per-row cost."""
+    def call(rows):
+        t0 = time.perf_counter()
+        orc.wildcat_forward_binned(ex["Q"], ex["K"], ex["V"], w.beta, w.r, nb, seed=w.pivot_seed, eps=EPS,
+                                   rows=rows)
+        return time.perf_counter() - t0
+
+    if w.m <= ORACLE_FULL_ROWS_MAX:
+        t = call(None)
+        return t, {"binned_call_s": t}
+    import workloads
+
+    na, nbr = ORACLE_TIMING_ROWS // 4, ORACLE_TIMING_ROWS
+    t1, t2 = call(workloads.sample_rows(w, na)), call(workloads.sample_rows(w, nbr))
+    per_row = max(0.0, (t2 - t1) / (nbr - na))
+    fixed = max(0.0, t1 - per_row * na)
+    est = fixed + per_row * w.m
+    return est, {"rows_timed": [na, nbr], "s_timed": [t1, t2], "fixed_s": fixed, "per_row_s": per_row}
+
+
+def oracle_step(orc, w, ex, nb=1, ranks=None):
+    """The oracle's time for one call of the bench's workload: (seconds,
+    detail, whole, sample text).  whole: a whole call was timed as is."""
+    if nb > 1:
+        est, det = oracle_binned_call(orc, w, ex, nb)
+        whole = w.m <= ORACLE_FULL_ROWS_MAX
+        text = (f"one whole binned wildcat_forward ({nb} bins, {w.BH} instances)" if whole else
+                f"binned wildcat_forward ({nb} bins, {w.BH} instances) on {ORACLE_TIMING_ROWS // 4} and "
+                f"{ORACLE_TIMING_ROWS} seeded query rows per head, extrapolated to m = {w.m} rows by the fitted "
+                "fixed + per-row cost") + "; fp64, OpenMP over instances"
+        return est, det, whole, text
+    rows, steps = oracle_plan(w)
+    if rows is None and steps is None:
+        t0 = time.perf_counter()
+        orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
+        return time.perf_counter() - t0, None, True, (f"one whole wildcat_forward call of the workload "
+                                                      f"({w.BH} instances), fp64")
+    est, det = oracle_call(orc, w, ex, rows, steps, ranks)
+    return est, det, False, oracle_sample_text(w, rows, steps=steps)
+
+
+def cpu_baseline(w, ex, seconds, ranks=None, nb=1):
     """The fp64 oracle, as it stands, on the host cores: whole calls repeated
-    for `seconds`, or one sampled call (oracle_plan) when a call is large;
-    `ranks`: the effective rank of every instance from the device run, for
-    the extrapolation of sampled pivot steps."""
+    for `seconds`, or one sampled call (oracle_plan, oracle_binned_call) when a
+    call is large; `ranks`: the effective rank of every instance from the
+    device run, for the extrapolation of sampled pivot steps; nb: bins."""
     import oracle
 
     orc = oracle.get()
-    rows, steps = oracle_plan(w)
     T = orc.num_threads()
-    used = {"select_and_weights": min(w.BH, T), "attend": T}  # OpenMP over instances / over query rows
-    if rows is not None or steps is not None:
-        est, det = oracle_call(orc, w, ex, rows, steps, ranks)
+    used = {"select_and_weights": min(w.BH * nb, T), "attend": T}  # OpenMP over instances / over query rows
+    est, det, whole, text = oracle_step(orc, w, ex, nb, ranks)
+    if not whole:
         return {"value": 1.0 / est, "unit": "calls/s", "cores": T, "threads_used": used, "kind": "oracle",
-                "partial": True, "sample": oracle_sample_text(w, rows, steps=steps), "seconds_per_call": est,
-                "detail": det}
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
+                "partial": True, "sample": text, "seconds_per_call": est, "detail": det}
+    reps, el = 1, est
+    while el < seconds:
+        el += oracle_step(orc, w, ex, nb, ranks)[0]
         reps += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
     return {"value": reps / el, "unit": "calls/s", "cores": T, "threads_used": used, "kind": "oracle",
-            "partial": False, "sample": oracle_sample_text(w, None, reps)}
+            "partial": False, "sample": f"{reps} calls: {text}"}
 
 
 def run_reference(args):
@@ -383,37 +422,26 @@ def run_reference(args):
     w = workloads.CONFIGS[args.workload]
     _, ex = workloads.make(w)
     orc = oracle.get()
-    rows, steps = oracle_plan(w)
-    whole = rows is None and steps is None
+    nb = max(1, args.nbins)
     for _ in range(max(args.warmup, 3)):
-        if whole:
-            orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
-        else:
-            oracle_call(orc, w, ex, rows, steps)
-    secs, det = [], None
+        oracle_step(orc, w, ex, nb)
+    secs, det, whole, text = [], None, True, ""
     for _ in range(args.steps):
-        if whole:
-            t0 = time.perf_counter()
-            orc.wildcat_forward(ex["Q"], ex["K"], ex["V"], w.beta, w.r, seed=w.pivot_seed, eps=EPS)
-            secs.append(time.perf_counter() - t0)
-        else:
-            est, det = oracle_call(orc, w, ex, rows, steps)
-            secs.append(est)
+        est, det, whole, text = oracle_step(orc, w, ex, nb)
+        secs.append(est)
     total = sum(secs)
     value = args.steps / total
     T = orc.num_threads()
     cpu = {"value": value, "unit": "calls/s", "cores": T, "kind": "oracle",
-           "threads_used": {"select_and_weights": min(w.BH, T), "attend": T},
-           "partial": not whole,
-           "sample": (oracle_sample_text(w, rows, steps=steps) if not whole
-                      else f"one whole wildcat_forward call of the workload per step ({w.BH} instances), fp64")}
+           "threads_used": {"select_and_weights": min(w.BH * nb, T), "attend": T},
+           "partial": not whole, "sample": ("one step per call; " + text)}
     if det is not None:
         cpu["detail_last_step"] = det
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "calls/s",
            "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": workload_config(w, {"l2": "n/a (host)"}),
+           "config": workload_config(w, {"l2": "n/a (host)", "nbins": nb}),
            "entries_per_s": value * w.BH * w.m * w.n,
            "cpu_baseline": cpu,
            "e2e": {"value": value, "unit": "calls/s", "h2d_bytes_per_step": 0,
@@ -624,7 +652,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_baseline(w, ex, args.cpu_seconds, ranks=plan.rank.cpu().tolist() if nb == 1 else None)
+        cpu = cpu_baseline(w, ex, args.cpu_seconds, ranks=plan.rank.cpu().tolist() if nb == 1 else None, nb=nb)
 
     if world > 1:
         barrier()
