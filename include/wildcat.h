@@ -16,9 +16,9 @@
  *            clipped to the value range [v_min j, v_max j] of V
  *            (Sec. 2, value-range clip; Alg. 3 WtdAttn); bf16 inputs with
  *            d in {64, 128} run on the tensor cores (tcgen05, fp32
- *            accumulation in tensor memory, P rounded to bf16 once and used
- *            for both numerator and denominator, [V_S | w] split into bf16
- *            hi + lo parts); other inputs on CUDA cores in fp32
+ *            accumulation in tensor memory; P and V_S rounded to bf16 for
+ *            the numerator's products, the denominator sum_l P_l w_l in fp32
+ *            from the unrounded P); other inputs on CUDA cores in fp32
  *   forward  the three stages back to back (Alg. 4, the WildCat module)
  *
  * Conventions shared by every call
@@ -34,7 +34,8 @@
  *    the caller.  The library keeps no pointer after a call returns, and no
  *    call allocates device memory: scratch space is the caller's
  *    `workspace` (size from the matching *_workspace_size query, 256-byte
- *    aligned).
+ *    aligned).  (The forwards create, on first use per device, one library
+ *    stream and a few events; wildcat_attend_noalloc uses a static array.)
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
  *    enqueued asynchronously; a call returns once its kernels are launched.
  *  - Argument checks happen on the host before anything is launched and
@@ -199,7 +200,8 @@ wildcat_status wildcat_weights_inverse(const void* K, const void* V, int dtype, 
  *   u_il = exp(beta <q_i, k_S_l> - beta M_Q),  M_Q = max_i |q_i| * max_l |k_S_l|
  *   O_hat_ij = fminf(fmaxf(sum_l u_il V_S[l, j] / sum_l u_il w_l, vmin_j), vmax_j)
  * The shift M_Q (one per instance) keeps every u_il <= 1 and cancels in the
- * ratio.  A normaliser that is zero or negative (Nystrom weights have mixed
+ * ratio; the tensor-core path (bf16, d in {64, 128}) shifts each query row by
+ * beta |q_i| max_l |k_S_l| instead, which cancels in the same way.  A normaliser that is zero or negative (Nystrom weights have mixed
  * signs) is not special-cased: the ratio is clipped as is, and a NaN ratio
  * (0/0) becomes vmin_j.
  *
